@@ -1,0 +1,166 @@
+"""Layer-level pins of the CPU oracle.
+
+- one expert, top-1: the layer is a dense SwiGLU MLP, computed here with torch
+  fp64 matmuls and torch's SiLU on operands dequantised by torch's own fp8
+  conversion (and a literal E2M1 table), not by the oracle's decoder;
+- all logits equal: experts 0..k-1 with weight 1/k, so Y is the mean of those
+  experts' outputs;
+- sigmoid scores with zero router weights: the selection is the k largest
+  biases and the weights are sigmoid(b)/sum, a closed form;
+- permuting the tokens permutes routing and output.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_topk_b200 import synth, workloads as W
+
+E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def fp8_val(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def e2m1_val(packed):
+    p = np.ascontiguousarray(packed, np.uint8)
+    lo, hi = p & 15, p >> 4
+    nib = np.stack([lo, hi], axis=-1).reshape(*p.shape[:-1], p.shape[-1] * 2)
+    mag = E2M1_MAG[nib & 7]
+    return np.where(nib & 8, -mag, mag)
+
+
+def deq_weight(wl, d, p, e):
+    q = d[p + "_q"][e].numpy()
+    s = d[p + "_s"][e].numpy()
+    if wl.fmt == W.FMT_FP8_ROW:
+        return fp8_val(q) * s.astype(np.float64)[:, None]
+    if wl.fmt == W.FMT_FP8_BLOCK128:
+        return fp8_val(q) * np.kron(s.astype(np.float64), np.ones((128, 128)))
+    v = e2m1_val(q)
+    sb = np.repeat(fp8_val(s), 16, axis=1)
+    return v * sb * float(d[p + "_g"][e])
+
+
+def deq_act(wl, codes, scales, g=0.0):
+    if wl.fmt == W.FMT_FP8_ROW:
+        return fp8_val(codes) * scales.astype(np.float64)[:, None]
+    if wl.fmt == W.FMT_FP8_BLOCK128:
+        return fp8_val(codes) * np.repeat(scales.astype(np.float64), 128, axis=1)
+    return e2m1_val(codes) * np.repeat(fp8_val(scales), 16, axis=1) * g
+
+
+def bf16_bits(x):
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+FMTS = [W.FMT_FP8_ROW, W.FMT_FP8_BLOCK128, W.FMT_NVFP4]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_single_expert_is_dense_swiglu_mlp(fmt):
+    wl = W.custom(H=256, I=384, E=1, k=1, fmt=fmt)
+    d = synth.layer(wl, seed=5)
+    L = oracle.Layer(wl, d)
+    x = synth.tokens(wl, 6, seed=5)
+    xf = x.to(torch.float32).numpy()
+    g_x = oracle.nvfp4_global(xf) if fmt == W.FMT_NVFP4 else 0.0
+    codes, scales = oracle.quant_rows(fmt, xf, g_x)
+    h, hq, hs, o = L.expert_rows(0, codes, scales, g_x)
+
+    a = torch.from_numpy(deq_act(wl, codes, scales, g_x))
+    wg = torch.from_numpy(deq_weight(wl, d, "gate", 0))
+    wu = torch.from_numpy(deq_weight(wl, d, "up", 0))
+    wd = torch.from_numpy(deq_weight(wl, d, "down", 0))
+    h_ref = torch.nn.functional.silu(a @ wg.T) * (a @ wu.T)
+    np.testing.assert_allclose(h, h_ref.numpy(), rtol=1e-12, atol=1e-12)
+    # the requantised hidden is what the down projection sees
+    hq2, hs2 = oracle.quant_rows(fmt, h_ref.numpy().astype(np.float32), wl.hidden_global_scale)
+    assert (hq2 == hq).mean() > 0.999
+    o_ref = torch.from_numpy(deq_act(wl, hq, hs, wl.hidden_global_scale)) @ wd.T
+    np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-12, atol=1e-12)
+
+    # the whole layer with one expert and top-1 is the same MLP with weight 1
+    ids, w, y = L.forward(bf16_bits(x), d["wr"].numpy(), None)
+    assert (ids == 0).all() and (w == 1.0).all()
+    np.testing.assert_allclose(y, o_ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_equal_logits_average_the_first_k_experts(fmt):
+    wl = W.custom(H=256, I=256, E=5, k=3, fmt=fmt)
+    d = synth.layer(wl, seed=6)
+    L = oracle.Layer(wl, d)
+    x = synth.tokens(wl, 4, seed=6)
+    wr0 = np.zeros((wl.E, wl.H), np.float32)
+    ids, w, y = L.forward(bf16_bits(x), wr0, None)
+    assert (ids == np.arange(3)).all()
+    np.testing.assert_allclose(w, 1.0 / 3.0, rtol=1e-15)
+    xf = x.to(torch.float32).numpy()
+    g_x = oracle.nvfp4_global(xf) if fmt == W.FMT_NVFP4 else 0.0
+    codes, scales = oracle.quant_rows(fmt, xf, g_x)
+    outs = [L.expert_rows(e, codes, scales, g_x)[3] for e in range(3)]
+    np.testing.assert_allclose(y, sum(outs) / 3.0, rtol=1e-12, atol=1e-12)
+
+
+def test_sigmoid_scores_with_bias_only_closed_form():
+    wl = W.custom(H=256, I=128, E=6, k=2, score=W.SCORE_SIGMOID)
+    d = synth.layer(wl, seed=7)
+    L = oracle.Layer(wl, d)
+    x = synth.tokens(wl, 3, seed=7)
+    bias = np.float32([0.5, -1.0, 2.0, 2.0, 0.25, -3.0])
+    ids, w, _ = L.forward(bf16_bits(x), np.zeros((6, 256), np.float32), bias)
+    assert (ids == [2, 3]).all()          # tie at 2.0 -> lower id first
+    np.testing.assert_allclose(w, 0.5, rtol=1e-15)
+    bias[3] = 1.0
+    ids, w, _ = L.forward(bf16_bits(x), np.zeros((6, 256), np.float32), bias)
+    s2, s1 = 1 / (1 + math.exp(-2.0)), 1 / (1 + math.exp(-1.0))
+    assert (ids == [2, 3]).all()
+    np.testing.assert_allclose(w, np.broadcast_to([s2 / (s1 + s2), s1 / (s1 + s2)], w.shape), rtol=1e-14)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_token_permutation_equivariance(fmt):
+    wl = W.custom(H=256, I=128, E=8, k=2, fmt=fmt)
+    d = synth.layer(wl, seed=8)
+    L = oracle.Layer(wl, d)
+    x = synth.tokens(wl, 9, seed=8)
+    xb = bf16_bits(x)
+    ids, w, y = L.forward(xb, d["wr"].numpy(), None)
+    p = np.random.default_rng(8).permutation(9)
+    ids2, w2, y2 = L.forward(np.ascontiguousarray(xb[p]), d["wr"].numpy(), None)
+    assert (ids2 == ids[p]).all()
+    assert (w2 == w[p]).all()
+    assert (y2 == y[p]).all()
+
+
+def test_counts_sum_to_assignments_on_skewed_workload():
+    wl = W.custom(H=256, I=128, E=64, k=8, zipf_s=1.2)
+    d = synth.layer(wl, seed=9)
+    x = synth.tokens(wl, 200, seed=9)
+    lg = oracle.router_logits(bf16_bits(x), d["wr"].numpy(), d["bias"].numpy())
+    ids, _ = oracle.topk(lg, wl.k, wl.score)
+    counts, offsets, perm, inv = oracle.dispatch(ids, wl.E)
+    assert counts.sum() == 200 * 8 and offsets[-1] == 200 * 8
+    assert (counts == 0).sum() > 0          # the Zipf bias leaves experts empty
+    assert all(len(set(r)) == wl.k for r in ids)   # distinct experts per token
+
+
+def test_subset_forward_matches_full_forward():
+    wl = W.custom(H=256, I=128, E=8, k=2)
+    d = synth.layer(wl, seed=10)
+    x = synth.tokens(wl, 12, seed=10)
+    L = oracle.Layer(wl, d)
+    ids, w, y = L.forward(bf16_bits(x), d["wr"].numpy(), None)
+    sel = np.int32([11, 3, 4])
+    used = sorted(set(ids[sel].reshape(-1)))
+    slot = np.full(wl.E, -1, np.int32)
+    slot[used] = np.arange(len(used))
+    sub = {k_: (v[used] if k_.endswith(("_q", "_s", "_g")) else v) for k_, v in d.items()}
+    Ls = oracle.Layer(wl, sub, expert_slot=slot)
+    ids2, w2, y2 = Ls.forward(bf16_bits(x), d["wr"].numpy(), None, sel=sel)
+    assert (ids2 == ids).all()
+    assert (y2 == y[sel]).all()

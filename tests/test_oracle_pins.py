@@ -1,0 +1,230 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks one oracle function against a library routine (torch's fp8
+conversion, Python's stable sort, torch fp64 matmul + SiLU), brute force on
+tiny inputs, a hand-derived closed form, or an invariant of the layer.  The
+pages print no worked numeric example, so no value here comes from them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_topk_b200 import synth, workloads as W
+
+E2M1_MAG = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # OCP FP4 E2M1 magnitudes in code order
+
+
+def bf16_bits(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def torch_e4m3(x):
+    x = np.clip(np.asarray(x, np.float32), -448.0, 448.0)
+    return torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def torch_e4m3_value(codes):
+    return torch.from_numpy(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+# ------------------------------------------------------------------ codecs
+def test_e4m3_values_match_torch_for_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch_e4m3_value(codes)
+    ours = np.array([oracle.e4m3_value(c) for c in codes])
+    assert (np.isnan(ours) == np.isnan(ref)).all()
+    ok = ~np.isnan(ref)
+    assert (ours[ok] == ref[ok]).all()
+    assert ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_torch_on_bit_sweep_and_ties():
+    bits = np.arange(0, 2 ** 32, 509, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    x = x[np.isfinite(x)]
+    vals = torch_e4m3_value(np.arange(127, dtype=np.uint8))
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)            # exact ties
+    near = np.concatenate([mids, np.nextafter(mids, np.float32(np.inf)),
+                           np.nextafter(mids, np.float32(0)), vals.astype(np.float32),
+                           np.float32([448.0, 464.0, 480.0, 1e30, 3.4e38, 0.0])])
+    x = np.concatenate([x, near, -near])
+    assert (oracle.e4m3_encode(x) == torch_e4m3(x)).all()
+
+
+def _brute_e2m1(x):
+    a = min(abs(float(x)), 6.0)
+    c = min(range(8), key=lambda c: (abs(E2M1_MAG[c] - a), c & 1))   # nearest, tie -> even code
+    return c | (8 if math.copysign(1.0, float(x)) < 0 else 0)
+
+
+def test_e2m1_values_and_encode_by_brute_force():
+    for c in range(16):
+        v = E2M1_MAG[c & 7] * (-1.0 if c & 8 else 1.0)
+        assert oracle.e2m1_value(c) == v
+    grid = np.arange(-8.0, 8.0, 1.0 / 64, dtype=np.float32)
+    mids = np.float32([(a + b) / 2 for a, b in zip(E2M1_MAG[:-1], E2M1_MAG[1:])])
+    extra = np.concatenate([mids, np.nextafter(mids, np.float32(9)), np.nextafter(mids, np.float32(0)),
+                            np.float32([1e-30, 7.0, 1e9])])
+    rng = np.random.default_rng(0)
+    x = np.concatenate([grid, extra, -extra, rng.normal(0, 3, 5000).astype(np.float32)])
+    got = oracle.e2m1_encode(x)
+    want = np.array([_brute_e2m1(v) for v in x], np.uint8)
+    assert (got == want).all()
+    # hand-checked ties: 0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4
+    hand = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6}
+    for v, c in hand.items():
+        assert oracle.e2m1_encode(np.float32([v]))[0] == c
+
+
+# ------------------------------------------------------------------ router
+def test_router_canonical_order_within_fp64_bound():
+    rng = np.random.default_rng(1)
+    for H, E, T in [(256, 8, 5), (1024, 16, 7), (7168, 4, 3)]:
+        x = bf16_bits(rng.normal(size=(T, H)))
+        wr = rng.normal(0, 1 / math.sqrt(H), size=(E, H)).astype(np.float32)
+        bias = rng.normal(size=E).astype(np.float32)
+        l32 = oracle.router_logits(x, wr, bias).astype(np.float64)
+        l64 = oracle.router_logits_f64(x, wr, bias)
+        xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+        absdot = np.abs(xf) @ np.abs(wr.astype(np.float64)).T
+        bound = (H / 32 + 7) * 2.0 ** -24 * (absdot + np.abs(bias)[None, :])
+        assert (np.abs(l32 - l64) <= bound).all()
+
+
+def test_router_chain_and_lane_assignment_closed_form():
+    # lane 0's chain sees 2^24 first, so its later +1 terms round away (ties to
+    # even); lane 1 sums eight ones exactly; the tree adds 2^24 + 8 exactly.
+    H = 512
+    w = np.zeros((1, H), np.float32)
+    w[0, 0] = 2.0 ** 24
+    w[0, 1:8] = 1.0           # lane 0, i=0, j=1..7
+    w[0, 256] = 1.0           # lane 0, i=1, j=0
+    w[0, 8:16] = 1.0          # lane 1
+    x = bf16_bits(np.ones((1, H)))
+    assert oracle.router_logits(x, w)[0, 0] == np.float32(2.0 ** 24 + 8)
+
+
+def test_router_pairwise_tree_shape_closed_form():
+    # partials p0=2^24, p2=1, p3=1: ((p0+p1)+(p2+p3)) = 2^24+2 exactly, while a
+    # left-to-right sum or a tree that pairs lanes 16 apart gives 2^24.
+    H = 256
+    w = np.zeros((1, H), np.float32)
+    w[0, 0] = 2.0 ** 24
+    w[0, 16] = 1.0
+    w[0, 24] = 1.0
+    x = bf16_bits(np.ones((1, H)))
+    assert oracle.router_logits(x, w)[0, 0] == np.float32(2.0 ** 24 + 2)
+    # the bias is one fp32 add after the tree: 2^24+2 + 3 = 2^24+5 is a tie, rounded to even 2^24+4
+    got = oracle.router_logits(x, w, np.float32([3.0]))[0, 0]
+    assert got == np.float32(2.0 ** 24 + 4)
+
+
+def _brute_topk(l, k):
+    E = len(l)
+
+    def before(a, b):
+        return l[a] > l[b] or (l[a] == l[b] and a < b)
+
+    sets = [S for S in itertools.combinations(range(E), k)
+            if all(before(i, j) for i in S for j in range(E) if j not in S)]
+    assert len(sets) == 1
+    return sorted(sets[0], key=lambda i: (-l[i], i))
+
+
+@pytest.mark.parametrize("score", [W.SCORE_SOFTMAX, W.SCORE_SIGMOID])
+def test_topk_brute_force_with_ties(score):
+    rng = np.random.default_rng(2)
+    for E in range(3, 11):
+        for k in range(1, min(3, E - 1) + 1):
+            lg = rng.choice(np.float32([-1.0, 0.0, 0.5, 1.0, 2.0, -0.0]), size=(20, E)).astype(np.float32)
+            ids, w = oracle.topk(lg, k, score)
+            for t in range(lg.shape[0]):
+                want = _brute_topk(list(lg[t]), k)
+                assert list(ids[t]) == want
+                sel = [float(lg[t, i]) for i in want]
+                if score == W.SCORE_SOFTMAX:
+                    z = [math.exp(v) for v in sel]
+                else:
+                    z = [1.0 / (1.0 + math.exp(-v)) for v in sel]
+                np.testing.assert_allclose(w[t], np.array(z) / sum(z), rtol=1e-14)
+
+
+def test_topk_equal_logits_pick_lowest_ids_with_equal_weights():
+    ids, w = oracle.topk(np.zeros((3, 6), np.float32), 4, W.SCORE_SOFTMAX)
+    assert (ids == np.arange(4)).all()
+    assert np.allclose(w, 0.25, rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------------ dispatch
+def test_dispatch_matches_stable_sort():
+    rng = np.random.default_rng(3)
+    for T, k, E in [(1, 1, 1), (17, 2, 8), (300, 8, 64), (1000, 8, 256)]:
+        ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+        ids[ids == 3] = 0 if E > 3 and k == 1 else ids[ids == 3]      # leave some experts empty
+        counts, offsets, perm, inv = oracle.dispatch(ids, E)
+        flat = ids.reshape(-1)
+        assert counts.sum() == T * k
+        assert (counts == np.bincount(flat, minlength=E)).all()
+        assert (offsets == np.concatenate([[0], np.cumsum(counts)])).all()
+        want = sorted(range(T * k), key=lambda a: flat[a])        # Python's sort is stable
+        assert list(perm) == want
+        assert (inv[perm] == np.arange(T * k)).all()
+
+
+def test_schedule_tiles():
+    # counts 0, 1, 129 (ragged: two tiles), 0, 384 (exactly three tiles)
+    offsets = np.int32([0, 0, 1, 130, 130, 514])
+    te, tr = oracle.schedule(offsets)
+    assert list(te) == [1, 2, 2, 4, 4, 4]
+    assert list(tr) == [0, 1, 129, 130, 258, 386]
+
+
+# ------------------------------------------------------------------ quantisers
+def test_fp8_row_quant_hand_example():
+    x = np.zeros((2, 256), np.float32)
+    x[0, :5] = [448.0, 224.0, -112.0, 0.0, 1.0]          # amax 448 -> s = 1 exactly
+    codes, s = oracle.quant_rows(W.FMT_FP8_ROW, x)
+    assert s[0] == 1.0 and s[1] == 0.0
+    assert list(codes[0, :5]) == [0x7E, 0x76, 0xEE, 0x00, 0x38]
+    assert (codes[1] == 0).all()
+
+
+def test_fp8_block128_quant_hand_example():
+    x = np.zeros((1, 256), np.float32)
+    x[0, 0] = 448.0
+    x[0, 128] = 224.0
+    x[0, 129] = -56.0
+    codes, s = oracle.quant_rows(W.FMT_FP8_BLOCK128, x)
+    assert list(s[0]) == [1.0, 0.5]
+    assert codes[0, 0] == 0x7E and codes[0, 128] == 0x7E and codes[0, 129] == 0xEE
+
+
+def test_nvfp4_quant_hand_example():
+    x = np.zeros((1, 32), np.float32)
+    x[0, :4] = [6.0, 3.0, -1.5, 0.5]
+    codes, sb = oracle.quant_rows(W.FMT_NVFP4, x, g=2.0 ** -8)
+    assert sb[0, 0] == 0x78 and sb[0, 1] == 0x00     # 256 = 2^8 -> e=15, m=0
+    assert list(codes[0, :2]) == [0x57, 0x1B] and (codes[0, 2:] == 0).all()
+    assert oracle.nvfp4_global(np.float32([[-5376.0, 1.0]])) == 2.0
+
+
+@pytest.mark.parametrize("fmt", [W.FMT_FP8_ROW, W.FMT_FP8_BLOCK128])
+def test_fp8_quant_error_bound(fmt):
+    rng = np.random.default_rng(4)
+    x = (rng.normal(size=(8, 512)) * rng.uniform(0.01, 100, size=(8, 1))).astype(np.float32)
+    codes, s = oracle.quant_rows(fmt, x)
+    s_full = np.repeat(s.reshape(8, -1), 512 // s.reshape(8, -1).shape[1], axis=1)
+    deq = torch_e4m3_value(codes) * s_full
+    # half an e4m3 ulp: 2^-4 relative for normals, 2^-10 * s absolute in the subnormal range
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, s_full * 2.0 ** -10) * (1 + 1e-6)
+    assert (np.abs(deq - x) <= bound).all()
+    # the element holding the block maximum gets the +-448 code: x/s = amax/fl(amax/448)
+    nb = s.reshape(8, -1).shape[1]
+    xb = np.abs(x).reshape(8, nb, -1)
+    cb = codes.reshape(8, nb, -1)
+    at_max = np.take_along_axis(cb, xb.argmax(axis=2)[..., None], axis=2)[..., 0]
+    assert ((at_max & 0x7F) == 0x7E).all()
