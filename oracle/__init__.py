@@ -184,6 +184,11 @@ def scale_shape(fmt, rows, K):
     return (rows, K // 16), np.uint8
 
 
+def hidden_fmt(fmt):
+    """The hidden is requantised per (row, 128 columns) for both FP8 formats."""
+    return FMT_NVFP4 if fmt == FMT_NVFP4 else FMT_FP8_BLOCK128
+
+
 def quant_rows(fmt, x, g=0.0):
     """fp32 rows [R,K] -> (codes, scales) in the layer's activation format."""
     x = _c(x, np.float32)
@@ -242,7 +247,7 @@ class Layer:
         R = a_codes.shape[0]
         h = np.empty((R, wl.I), np.float64)
         hq = np.empty((R, code_bytes(wl.fmt, wl.I)), np.uint8)
-        shp, dt = scale_shape(wl.fmt, R, wl.I)
+        shp, dt = scale_shape(hidden_fmt(wl.fmt), R, wl.I)
         hs = np.empty(shp, dt)
         o = np.empty((R, wl.H), np.float64)
         lib().orc_expert_rows(self.ref(), e, R, _p(a_codes), _p(a_scales), float(x_global),

@@ -284,6 +284,12 @@ static int64_t act_scale_bytes(int fmt, int K)
 
 /* ------------------------------------------------------------ expert FFN */
 
+/* Format of the requantised hidden.  The gate/up epilogue of a tile sees 128
+ * hidden columns of a row, so the FP8 formats scale the hidden per (row,
+ * 128-column block) (the 1x128 activation rule); NVFP4 keeps its 16-blocks
+ * with the static global scale. */
+static int hidden_fmt(int fmt) { return fmt == ORC_FMT_NVFP4 ? ORC_FMT_NVFP4 : ORC_FMT_FP8_BLOCK128; }
+
 void orc_weight_row(const orc_layer* L, const orc_proj* P, int N, int K, int e, int n, double* out)
 {
     int slot = L->expert_slot ? L->expert_slot[e] : e;
@@ -330,13 +336,13 @@ static void down_dequantised(const orc_layer* L, int e, int rows, const double* 
     }
 }
 
-static void dequant_rows(const orc_layer* L, int rows, int K, const uint8_t* codes,
+static void dequant_rows(int fmt, int rows, int K, const uint8_t* codes,
                          const void* scales, float g, double* out)
 {
-    int64_t cb = row_code_bytes(L->fmt, K), sb = act_scale_bytes(L->fmt, K);
+    int64_t cb = row_code_bytes(fmt, K), sb = act_scale_bytes(fmt, K);
 #pragma omp parallel for schedule(static)
     for (int r = 0; r < rows; r++)
-        dequant_act_row(L->fmt, codes + r * cb, (const uint8_t*)scales + r * sb, g, K, out + (int64_t)r * K);
+        dequant_act_row(fmt, codes + r * cb, (const uint8_t*)scales + r * sb, g, K, out + (int64_t)r * K);
 }
 
 void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes,
@@ -346,7 +352,7 @@ void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes
     int H = L->H, I = L->I;
     double* a = (double*)malloc(sizeof(double) * (size_t)rows * H);
     double* hh = (double*)malloc(sizeof(double) * (size_t)rows * I);
-    dequant_rows(L, rows, H, a_codes, a_scales, x_global, a);
+    dequant_rows(L->fmt, rows, H, a_codes, a_scales, x_global, a);
 #pragma omp parallel
     {
         double* wg = (double*)malloc(sizeof(double) * (size_t)H);
@@ -365,14 +371,15 @@ void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes
         free(wu);
     }
     if (h) memcpy(h, hh, sizeof(double) * (size_t)rows * I);
-    /* requantise the hidden: round to fp32, then the layer's activation rule */
+    /* requantise the hidden: round to fp32, then the hidden's rule */
+    int hf_fmt = hidden_fmt(L->fmt);
     float* hf = (float*)malloc(sizeof(float) * (size_t)rows * I);
     for (int64_t i = 0; i < (int64_t)rows * I; i++) hf[i] = (float)hh[i];
-    uint8_t* qc = hq_codes ? hq_codes : (uint8_t*)malloc((size_t)(rows * row_code_bytes(L->fmt, I)));
-    void* qs = hq_scales ? hq_scales : malloc((size_t)(rows * act_scale_bytes(L->fmt, I)));
-    orc_quant_rows(L->fmt, hf, rows, I, L->hidden_global, qc, qs);
+    uint8_t* qc = hq_codes ? hq_codes : (uint8_t*)malloc((size_t)(rows * row_code_bytes(hf_fmt, I)));
+    void* qs = hq_scales ? hq_scales : malloc((size_t)(rows * act_scale_bytes(hf_fmt, I)));
+    orc_quant_rows(hf_fmt, hf, rows, I, L->hidden_global, qc, qs);
     double* hd = (double*)malloc(sizeof(double) * (size_t)rows * I);
-    dequant_rows(L, rows, I, qc, qs, L->hidden_global, hd);
+    dequant_rows(hf_fmt, rows, I, qc, qs, L->hidden_global, hd);
     down_dequantised(L, e, rows, hd, o);
     if (!hq_codes) free(qc);
     if (!hq_scales) free(qs);
@@ -386,7 +393,7 @@ void orc_down_rows(const orc_layer* L, int e, int rows, const uint8_t* h_codes,
                    const void* h_scales, double* o)
 {
     double* hd = (double*)malloc(sizeof(double) * (size_t)rows * L->I);
-    dequant_rows(L, rows, L->I, h_codes, h_scales, L->hidden_global, hd);
+    dequant_rows(hidden_fmt(L->fmt), rows, L->I, h_codes, h_scales, L->hidden_global, hd);
     down_dequantised(L, e, rows, hd, o);
     free(hd);
 }

@@ -104,14 +104,17 @@ void orc_weight_row(const orc_layer* L, const orc_proj* P, int N, int K, int e, 
 /* One expert on quantised input rows.
  *   a_codes/a_scales: rows of the quantised input in the layer's format (K = H)
  *   x_global: NVFP4 global scale of the input (ignored otherwise)
+ *   The hidden is requantised per (row, 128-column block) with fp32 scales for
+ *   both FP8 formats ([rows, I/128] scales), and with the NVFP4 rule and the
+ *   static hidden_global scale for NVFP4.
  *   outputs: h (fp64 SwiGLU output before requantisation, [rows, I]) may be NULL;
- *            hq codes/scales (requantised hidden, layer format) may be NULL;
+ *            hq codes/scales (requantised hidden) may be NULL;
  *            o [rows, H] fp64 down projection of the dequantised hidden. */
 void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes,
                      const void* a_scales, float x_global, double* h,
                      uint8_t* hq_codes, void* hq_scales, double* o);
 
-/* Down projection alone of quantised hidden rows (layer format) -> o [rows, H] fp64 */
+/* Down projection alone of quantised hidden rows (hidden format) -> o [rows, H] fp64 */
 void orc_down_rows(const orc_layer* L, int e, int rows, const uint8_t* h_codes,
                    const void* h_scales, double* o);
 

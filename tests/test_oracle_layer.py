@@ -78,9 +78,11 @@ def test_single_expert_is_dense_swiglu_mlp(fmt):
     h_ref = torch.nn.functional.silu(a @ wg.T) * (a @ wu.T)
     np.testing.assert_allclose(h, h_ref.numpy(), rtol=1e-12, atol=1e-12)
     # the requantised hidden is what the down projection sees
-    hq2, hs2 = oracle.quant_rows(fmt, h_ref.numpy().astype(np.float32), wl.hidden_global_scale)
+    hfmt = oracle.hidden_fmt(fmt)
+    hq2, hs2 = oracle.quant_rows(hfmt, h_ref.numpy().astype(np.float32), wl.hidden_global_scale)
     assert (hq2 == hq).mean() > 0.999
-    o_ref = torch.from_numpy(deq_act(wl, hq, hs, wl.hidden_global_scale)) @ wd.T
+    hwl = W.custom(H=wl.H, I=wl.I, E=1, k=1, fmt=hfmt)
+    o_ref = torch.from_numpy(deq_act(hwl, hq, hs, wl.hidden_global_scale)) @ wd.T
     np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-12, atol=1e-12)
 
     # the whole layer with one expert and top-1 is the same MLP with weight 1
