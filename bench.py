@@ -1,0 +1,335 @@
+"""Throughput of the routed MoE FFN forward pass on B200.
+
+One step = one whole layer call (router + top-k, dispatch with X quantisation,
+grouped gate/up GEMM with SwiGLU + requantisation, grouped down GEMM with the
+routing weight, combine) over one batch of T tokens of the workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--tokens T]
+                  [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own replica on its own
+batch: the tokens of a batch are independent, so the path shards by tokens
+with no data-path collective (weak scaling).  Timing: CUDA events on the
+launching stream, barrier + synchronize on both sides, max over ranks.
+The reference arm times the CPU oracle on a bounded sample of the same batch.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_topk_b200 import synth  # noqa: E402
+from mixture_experts_topk_b200.workloads import FMT_NVFP4, WORKLOADS  # noqa: E402
+
+METRIC = "fused MoE layer tokens/s & TFLOP/s on 1 B200; % of FP8/FP4 peak or HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm = [float(r[1]) for r in self.rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            if len(r) >= 9:
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def algorithmic_work(wl, T, counts):
+    """FLOPs and bytes of one layer call (intermediates excluded)."""
+    A = T * wl.k
+    flops_tensor = 2.0 * A * 3 * wl.H * wl.I
+    flops_router = 2.0 * T * wl.E * wl.H
+    touched = int((counts > 0).sum())
+    if wl.fmt == FMT_NVFP4:
+        per_expert = 3 * wl.H * wl.I * (0.5 + 1.0 / 16)
+    elif wl.fmt == 0:
+        per_expert = 3 * wl.H * wl.I + 4 * (2 * wl.I + wl.H)
+    else:
+        per_expert = 3 * wl.H * wl.I + 4 * 3 * (wl.H // 128) * (wl.I // 128)
+    byts = touched * per_expert + wl.E * wl.H * 4 + 2 * T * wl.H * 2
+    return flops_tensor, flops_router, byts, touched
+
+
+def run_ours(args, rank, world, local_rank):
+    from mixture_experts_topk_b200 import native
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    T = args.tokens
+    d = synth.layer(wl, seed=0, device=dev)
+    layer = native.Layer(wl, d, max_T=T, device=dev)
+    x = synth.tokens(wl, T, seed=rank, device=dev)
+    wr = d["wr"]
+    bias = d["bias"]
+    y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        native.moe_forward(layer.h, x, T, wr, bias, layer.packed, y, layer.ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, msg = layer.status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {msg}")
+    counts = layer.region("counts", torch.int32, wl.E).cpu().numpy()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- device-timed steps (inputs already resident)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    st, msg = layer.status()
+    if st != 0:
+        raise RuntimeError(f"device status after the timed steps: {msg}")
+
+    # ---- per-kernel durations of the same steps (events between the C-ABI calls)
+    v = layer.view
+    ids_t = layer.region("ids", torch.int32, T * wl.k)
+    w_t = layer.region("w", torch.float32, T * wl.k)
+    names = ["route", "dispatch", "gate_up", "down", "combine"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        e = evs[s]
+        e[0].record(stream)
+        native.moe_route(layer.h, x, T, wr, bias, ids_t, w_t, layer.ws)
+        e[1].record(stream)
+        native.moe_dispatch(layer.h, x, ids_t, T, layer.ws)
+        e[2].record(stream)
+        native.moe_gate_up(layer.h, layer.packed, T, layer.ws)
+        e[3].record(stream)
+        native.moe_down(layer.h, layer.packed, w_t, T, layer.ws)
+        e[4].record(stream)
+        native.moe_combine(layer.h, T, y, layer.ws)
+        e[5].record(stream)
+    torch.cuda.synchronize()
+    per = {n: sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps
+           for i, n in enumerate(names)}
+
+    # ---- end to end through the public call with host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(T, wl.H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        native.moe_forward(layer.h, x_dev, T, wr, bias, layer.packed, y, layer.ws)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        native.moe_forward(layer.h, x_dev, T, wr, bias, layer.packed, y, layer.ws)
+        y_host.copy_(y, non_blocking=True)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    fl_t, fl_r, byts, touched = algorithmic_work(wl, T, counts)
+    pk, pk_kind = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops_sustained"]          # fp8 dense = 2 x bf16 (nominal ratio)
+    gu_flops = 2.0 * T * wl.k * 2 * wl.H * wl.I
+    gu_ms = per["gate_up"]
+    achieved = gu_flops / (gu_ms * 1e-3) / 1e12
+    step_ms = ms_max / args.steps
+    t_roof_ms = max(fl_t / (fp8_peak * 1e12), byts / (pk["hbm_gbs"] * 1e9)) * 1e3
+    tokens_total = world * T * args.steps
+    out = {
+        "metric": METRIC,
+        "value": tokens_total / (ms_max * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8-e4m3 (fp32 accumulate)" if wl.fmt != FMT_NVFP4 else "nvfp4-e2m1 (fp32 accumulate)",
+        "data": "synthetic (seeded; X ~ N(0,1) bf16, weights ~ N(0,1/fan_in) quantised offline)",
+        "config": {"workload": f"{wl.name} T={T}", "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                   "T_per_gpu": T, "parallelism": f"replicas x{world} (token batches)",
+                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (byts / 1e9),
+                   "touched_experts": touched},
+        "tflops": (fl_t + fl_r) * world * args.steps / (ms_max * 1e-3) / 1e12,
+        "layer_roofline": {"t_roof_ms": t_roof_ms, "frac": t_roof_ms / step_ms,
+                           "peaks": f"{pk_kind}: fp8 = 2 x bf16_tflops_sustained, hbm_gbs"},
+        "roofline": {"kernel": "grouped_gemm gate/up (SwiGLU + requant epilogue)", "bound": "tensor",
+                     "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp8_peak, "traffic": None,
+                     "peak_source": f"{pk_kind} bf16_tflops_sustained x 2 (fp8:bf16 nominal ratio)"},
+        "kernel_ms": per,
+        "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clk.summary(),
+    }
+    layer.close()
+    return out
+
+
+def cpu_baseline(wl, T, n_sel, seed=0):
+    """The oracle as it stands on the host cores: full routing of the T-token
+    batch plus the expert MLP and combine of n_sel sampled tokens."""
+    import numpy as np
+    import oracle
+    x = synth.tokens(wl, T, seed=seed)
+    d_router = synth.router(wl, seed=0)
+    sel = np.linspace(0, T - 1, n_sel).astype(np.int32)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    lg = oracle.router_logits(xb, d_router[0].numpy(), None if d_router[1] is None else d_router[1].numpy())
+    ids, _ = oracle.topk(lg, wl.k, wl.score)
+    used = sorted(set(ids[sel].reshape(-1).tolist()))
+    d = synth.experts(wl, seed=0, experts_subset=used)
+    slot = np.full(wl.E, -1, np.int32)
+    slot[used] = np.arange(len(used))
+    sub = {k_: v[used] for k_, v in d.items()}
+    L = oracle.Layer(wl, sub, expert_slot=slot)
+    t0 = time.perf_counter()
+    L.forward(xb, d_router[0].numpy(), None if d_router[1] is None else d_router[1].numpy(), sel=sel)
+    dt = time.perf_counter() - t0
+    return {"value": n_sel / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_sel} of {T} tokens through the expert MLP and combine; router and top-k over all {T}",
+            "seconds": dt}
+
+
+def run_reference(args):
+    wl = WORKLOADS[args.workload]
+    T = args.tokens
+    for _ in range(args.warmup):
+        cpu_baseline(wl, T, 1)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        r = cpu_baseline(wl, T, args.ref_sample)
+        vals.append(r["value"])
+        secs += r["seconds"]
+    v = args.steps * args.ref_sample / secs
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 router)",
+            "data": "synthetic (seeded)", "config": {"workload": f"{wl.name} T={T}", "T_per_gpu": T},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral-8x7b")
+    ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-sample", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(WORKLOADS[args.workload], args.tokens, args.ref_sample)
+            cb.pop("seconds")
+            out["cpu_baseline"] = cb
+        print(json.dumps(out))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * moe_b200.h -- C ABI of the routed Mixture-of-Experts FFN forward pass on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (LightMoE README, "MoE inference"; Alpha-MoE article, "How the
+ * megakernel works"): given tokens X[T,H], router weights Wr[E,H] (+ optional
+ * per-expert bias), and per expert quantised W_gate, W_up [I,H] and W_down [H,I]
+ * with their scales, return
+ *     Y[t] = sum_{j<k} w[t,j] * W_down[e_j] q( SiLU(W_gate[e_j] q(x_t)) * (W_up[e_j] q(x_t)) )
+ * where e_j are the k experts with the largest router logits (ties -> lower
+ * expert id), w the softmax (or sigmoid) of those k logits normalised to sum 1,
+ * and q() the activation quantiser of the layer's format.
+ *
+ * Conventions for every entry point:
+ *   - All pointers named *device* are device addresses owned by the caller; the
+ *     library never allocates device memory.  A warmed call does not allocate
+ *     (LightMoE README, "Standalone GEMM": the caller owns the output).
+ *   - Device pointers must be 256-byte aligned (torch allocations are).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Argument errors return at once and launch nothing.  Errors seen
+ *     by a kernel (a bounded wait that ran out, an index out of range) go to a
+ *     status word inside the workspace; moe_get_status() reports them.
+ *   - One workspace per concurrent stream (LightMoE README, "MoE inference":
+ *     one plan per concurrent CUDA stream, its workspaces are reused).
+ *   - Shape limits (LightMoE README, "Limits": K aligned, at most 256 local
+ *     experts, at most 131,072 token-expert assignments): H a multiple of 256,
+ *     I a multiple of 128, 1 <= k <= 8, k <= E <= 256, max_T * k <= 131072.
+ *     Otherwise MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - moe_last_error() returns a thread-local message for the last failure.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_DEVICE_TIMEOUT = 5,
+    MOE_ERR_DEVICE_BOUNDS = 6
+} moe_status;
+
+/* score function of the router (LightMoE README, "MoE inference": top_k_weights) */
+enum { MOE_SCORE_SOFTMAX = 0,    /* softmax over the selected k logits */
+       MOE_SCORE_SIGMOID = 1 };  /* sigmoid of each selected logit, normalised to sum 1 */
+
+/* quantisation format of weights, activations and hidden (Alpha-MoE article:
+ * FP8 W8A8; LightMoE README, "Standalone GEMM": NVFP4 = E2M1 values, E4M3
+ * block scales, one fp32 per-tensor scale) */
+enum { MOE_FMT_FP8_ROW = 0,      /* e4m3; fp32 scale per weight row / per token; hidden per (token, 128 cols) */
+       MOE_FMT_FP8_BLOCK128 = 1, /* e4m3; fp32 scale per 128x128 weight block / per (token, 128 cols) */
+       MOE_FMT_NVFP4 = 2 };      /* e2m1; e4m3 scale per 16 along K; fp32 global per tensor */
+
+typedef struct {
+    int H, I, E, k;
+    int score;                    /* MOE_SCORE_* */
+    int fmt;                      /* MOE_FMT_* */
+    int has_bias;                 /* router logits get + bias[e] */
+    int max_T;                    /* largest T a workspace must hold */
+    float hidden_global_scale;    /* NVFP4 only: static fp32 scale of the hidden (a checkpoint
+                                     scale, LightMoE README "set_activation_scales") */
+} moe_config;
+
+typedef struct moe_handle moe_handle;
+
+/* Quantised expert weights in the plain layout (device pointers), per projection:
+ *   q: codes, [E, N, K] uint8 e4m3, or [E, N, K/2] uint8 e2m1 (element 2i in the low nibble)
+ *   s: FP8_ROW [E, N] fp32; FP8_BLOCK128 [E, N/128, K/128] fp32; NVFP4 [E, N, K/16] e4m3 codes
+ *   g: NVFP4 [E] fp32 global scales, else NULL
+ * gate and up have N = I, K = H; down has N = H, K = I. */
+typedef struct {
+    const void* gate_q; const void* gate_s; const float* gate_g;
+    const void* up_q;   const void* up_s;   const float* up_g;
+    const void* down_q; const void* down_s; const float* down_g;
+} moe_weights;
+
+/* Device addresses of the intermediates inside a workspace (for inspection and
+ * for feeding one step alone).  Row counts use A = max_T * k. */
+typedef struct {
+    int32_t* status;     /* [64] status[0] = first device error (moe_status), status[1] = where */
+    int32_t* ids;        /* [A] router top-k expert ids, token-major [T, k] */
+    float*   w;          /* [A] routing weights [T, k] */
+    int32_t* counts;     /* [E] assignments per expert */
+    int32_t* offsets;    /* [E+1] exclusive prefix sum of counts (m_indptr) */
+    int32_t* num_tiles;  /* [1] row tiles of 128 over all experts */
+    int32_t* tiles;      /* [A/128 + E + 1][2] (expert, first row) per row tile */
+    int32_t* perm;       /* [A] slot -> t*k + j */
+    int32_t* inv;        /* [A] t*k + j -> slot */
+    float*   x_global;   /* [1] NVFP4 global scale of X */
+    uint8_t* xq;         /* [A, H] e4m3 (NVFP4: [A, H/2]) quantised X rows in expert-major slot order */
+    void*    xs;         /* scales of xq: [A] fp32 | [A, H/128] fp32 | [A, H/16] e4m3 */
+    uint8_t* hq;         /* [A, I] (NVFP4: [A, I/2]) requantised hidden */
+    void*    hs;         /* scales of hq: [A, I/128] fp32 | [A, I/16] e4m3 */
+    float*   o;          /* [A, H] fp32 down projection times routing weight, slot order */
+} moe_workspace_view;
+
+const char* moe_last_error(void);
+
+/* Validate cfg and create a handle (host memory only; queries the current device). */
+moe_status moe_init(const moe_config* cfg, moe_handle** out);
+moe_status moe_destroy(moe_handle* h);
+
+/* Bytes of the packed expert weights / of one workspace (sized by cfg.max_T). */
+moe_status moe_weights_size(const moe_handle* h, size_t* bytes);
+moe_status moe_workspace_size(const moe_handle* h, size_t* bytes);
+/* Fill `view` with the addresses of the regions of workspace `ws` (no device work). */
+moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_workspace_view* view);
+
+/* Rearrange plain-layout weights into the packed device layout the GEMMs read
+ * (gate and up interleaved in 128-row blocks so one tile holds both).  Not on
+ * the timed path (LightMoE README, "Installation": packing outside latency). */
+moe_status moe_pack_weights(const moe_handle* h, const moe_weights* src, void* packed,
+                            moe_stream_t stream);
+
+/* Router + top-k (Alpha-MoE article: routing is one of the fused stages;
+ * LightMoE README "MoE inference": int32 ids, fp32 weights).
+ *   x [T, H] bf16, wr [E, H] fp32, bias [E] fp32 (NULL unless has_bias)
+ *   -> ids [T, k] int32 (larger logit first, ties -> lower id), w [T, k] fp32.
+ * Logits are fp32 in one fixed order: lane l of 32 owns h = 256 i + 8 l + j and
+ * runs one fused multiply-add chain over i then j; the 32 lane sums are added as
+ * a balanced pairwise tree; then + bias[e].  So ids are reproducible bit for bit. */
+moe_status moe_route(const moe_handle* h, const void* x, int T, const float* wr,
+                     const float* bias, int32_t* ids, float* w, void* ws, moe_stream_t stream);
+
+/* Deterministic expert-major dispatch (LightMoE README, "Grouped GEMM" m_indptr
+ * and "MoE training" MoEDispatch; pure-Triton article: block-id -> (expert,
+ * offset) map): counts, offsets, the row-tile schedule, the stable slot of each
+ * (t, j) in row-major order, and the quantised X rows written to their slots
+ * (LightMoE README: BF16 input quantisation).  ids may be caller-provided. */
+moe_status moe_dispatch(const moe_handle* h, const void* x, const int32_t* ids, int T,
+                        void* ws, moe_stream_t stream);
+
+/* Grouped gate+up GEMM over the dispatched rows with SiLU(gate)*up and the
+ * requantisation of the hidden fused into its epilogue (pure-Triton article:
+ * gate and up share one input tile, SiLU in registers; LightMoE README: gated
+ * activation + requantisation).  Reads xq/xs/tiles from ws, writes hq/hs. */
+moe_status moe_gate_up(const moe_handle* h, const void* packed, int T, void* ws,
+                       moe_stream_t stream);
+
+/* Grouped down GEMM over the hidden, times the routing weight of each row
+ * (LightMoE README: down projection, routing-weight application).
+ * w [T, k] fp32 (may be view.w).  Reads hq/hs, writes o. */
+moe_status moe_down(const moe_handle* h, const void* packed, const float* w, int T,
+                    void* ws, moe_stream_t stream);
+
+/* Deterministic combine (LightMoE README, "Highlights": deterministic
+ * combine): y[t] = bf16( sum_{j=0..k-1} o[inv[t k + j]] ) in fixed j order,
+ * fp32 rows and accumulation, one final rounding, no atomics.  y [T, H] bf16. */
+moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws, moe_stream_t stream);
+
+/* The whole layer: route -> dispatch -> gate/up -> down -> combine.  Routing
+ * results stay in the workspace (view.ids, view.w).  y [T, H] bf16. */
+moe_status moe_forward(const moe_handle* h, const void* x, int T, const float* wr,
+                       const float* bias, const void* packed, void* y, void* ws,
+                       moe_stream_t stream);
+
+/* The layer with routing given by the caller (LightMoE README, "MoE inference":
+ * __call__(x, top_k_ids, top_k_weights)).  ids [T, k] int32 distinct per token,
+ * w [T, k] fp32. */
+moe_status moe_forward_routed(const moe_handle* h, const void* x, int T, const int32_t* ids,
+                              const float* w, const void* packed, void* y, void* ws,
+                              moe_stream_t stream);
+
+/* Zero the status words of a freshly allocated workspace; call once before
+ * the workspace's first use. */
+moe_status moe_workspace_init(const moe_handle* h, void* ws, moe_stream_t stream);
+
+/* Synchronise `stream`, return the first device error recorded in ws since the
+ * last call (MOE_OK if none) and clear it. */
+moe_status moe_get_status(const moe_handle* h, void* ws, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

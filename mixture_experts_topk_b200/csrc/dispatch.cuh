@@ -1,0 +1,225 @@
+// dispatch.cuh -- deterministic expert-major dispatch and X quantisation.
+//
+// LightMoE README ("Grouped GEMM"): rows are contiguous per expert, m_indptr is
+// int32 of length E+1, zero-assignment experts are valid; ("MoE training"):
+// MoEDispatch returns gather indices, m_indptr and inverse slots.  Pure-Triton
+// article: a precomputed block-id -> (expert id, offset) map lets one launch
+// run variable-size groups without padding.
+//
+// Slot of assignment a = t*k + j (row-major order):
+//   offsets[e] + #{a' < a : ids[a'] == e}
+// computed without atomics on the result: the assignments are cut into chunks
+// of 1024; a per-chunk histogram, one scan over (expert, chunk), and inside a
+// chunk a per-warp match + per-expert scan over the 32 warps.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int DISPATCH_CHUNK = 1024;
+constexpr int TILE_M = 128;
+
+__global__ void __launch_bounds__(DISPATCH_CHUNK)
+    hist_kernel(const int32_t* ids, int A, int E, int32_t* chunk_counts, int32_t* status) {
+    __shared__ int h[256];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int a = blockIdx.x * DISPATCH_CHUNK + threadIdx.x;
+    if (a < A) {
+        const int e = ids[a];
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&h[e], 1);
+        else report(status, ST_BOUNDS, WHERE_DISPATCH);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[blockIdx.x * E + e] = h[e];
+}
+
+// One CTA: counts, offsets (exclusive scan), per-chunk bases (written over the
+// chunk counts), and the row-tile table (expert, first row) in expert order.
+__global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
+                                                   int32_t* offsets, int32_t* tiles, int32_t* num_tiles) {
+    __shared__ int s_cnt[256], s_off[257], s_tptr[257];
+    const int e = threadIdx.x;
+    int c = 0;
+    if (e < E)
+        for (int ch = 0; ch < nchunks; ch++) c += chunk_counts[ch * E + e];
+    s_cnt[e] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0, trun = 0;
+        for (int i = 0; i < E; i++) {
+            s_off[i] = run;
+            s_tptr[i] = trun;
+            run += s_cnt[i];
+            trun += (s_cnt[i] + TILE_M - 1) / TILE_M;
+        }
+        s_off[E] = run;
+        s_tptr[E] = trun;
+        offsets[E] = run;
+        *num_tiles = trun;
+    }
+    __syncthreads();
+    if (e < E) {
+        counts[e] = c;
+        offsets[e] = s_off[e];
+        int run = s_off[e];
+        for (int ch = 0; ch < nchunks; ch++) {
+            const int v = chunk_counts[ch * E + e];
+            chunk_counts[ch * E + e] = run;
+            run += v;
+        }
+        const int nt = s_tptr[e + 1] - s_tptr[e];
+        for (int i = 0; i < nt; i++) {
+            tiles[2 * (s_tptr[e] + i)] = e;
+            tiles[2 * (s_tptr[e] + i) + 1] = s_off[e] + TILE_M * i;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(DISPATCH_CHUNK)
+    rank_kernel(const int32_t* ids, int A, int E, const int32_t* chunk_base, int32_t* perm, int32_t* inv) {
+    __shared__ int wc[32][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) wc[i >> 8][i & 255] = 0;
+    __syncthreads();
+    const int a = blockIdx.x * DISPATCH_CHUNK + threadIdx.x;
+    int e = (a < A) ? ids[a] : -1;
+    const bool valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
+    if (!valid) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (valid && rank == 0) wc[warp][e] = __popc(peers);
+    __syncthreads();
+    if (threadIdx.x < E) {
+        int run = chunk_base[blockIdx.x * E + threadIdx.x];
+        for (int w = 0; w < 32; w++) {
+            const int v = wc[w][threadIdx.x];
+            wc[w][threadIdx.x] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    if (a < A) {
+        if (valid) {
+            const int slot = wc[warp][e] + rank;
+            perm[slot] = a;
+            inv[a] = slot;
+        } else {
+            inv[a] = -1;
+        }
+    }
+}
+
+// Quantise each token row of X once and write it to the k slots of its
+// assignments (LightMoE README: BF16 input quantisation inside the layer).
+// FP8_ROW: s = amax/448 over the row; BLOCK128: per 128 columns;
+// q = e4m3(x / s) with correctly rounded division, q = 0 when s == 0.
+// One warp per token; lane l handles columns 256 i + 8 l .. +8.
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_scatter_kernel(const __nv_bfloat16* x, int T, int H, int k,
+                                                            const int32_t* inv, uint8_t* xq, float* xs) {
+    const int lane = threadIdx.x & 31;
+    const int nI = H >> 8;
+    for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+        int slot[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
+        const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
+        float s_row = 0.0f;
+        if (FMT == 0) {
+            float amax = 0.0f;
+            for (int i = 0; i < nI; i++) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + 256 * i + 8 * lane));
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            s_row = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (j == lane && slot[j] >= 0) xs[slot[j]] = s_row;
+        }
+        for (int i = 0; i < nI; i++) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + 256 * i + 8 * lane));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            float s = s_row;
+            if (FMT == 1) {
+                float amax = 0.0f;
+#pragma unroll
+                for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                s = __fdiv_rn(amax, 448.0f);
+                if ((lane & 15) == 0) {
+#pragma unroll
+                    for (int j = 0; j < 8; j++)
+                        if (slot[j] >= 0) xs[static_cast<size_t>(slot[j]) * (H >> 7) + 2 * i + (lane >> 4)] = s;
+                }
+            }
+            uint32_t packed[2];
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const float a = bf16_lo(u[q]), b = bf16_hi(u[q]);
+                const uint16_t c = (s == 0.0f) ? static_cast<uint16_t>(0)
+                                               : f2_to_e4m3x2(__fdiv_rn(a, s), __fdiv_rn(b, s));
+                if (q & 1) packed[q >> 1] |= static_cast<uint32_t>(c) << 16;
+                else packed[q >> 1] = c;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (slot[j] >= 0)
+                    *reinterpret_cast<uint2*>(xq + static_cast<size_t>(slot[j]) * H + 256 * i + 8 * lane) =
+                        make_uint2(packed[0], packed[1]);
+        }
+    }
+}
+
+// y[t] = bf16(sum_j o[inv[t k + j]]) in fixed j order with fp32 accumulation;
+// o holds fp32 rows (weight already applied), so the only rounding to bf16 is
+// the final one.
+__global__ void __launch_bounds__(128) combine_kernel(const float* o, const int32_t* inv, int T, int H, int k,
+                                                      __nv_bfloat16* y) {
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        int slot[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
+        for (int c0 = 8 * threadIdx.x; c0 < H; c0 += 8 * blockDim.x) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (slot[j] < 0) continue;
+                const float4* src = reinterpret_cast<const float4*>(o + static_cast<size_t>(slot[j]) * H + c0);
+                const float4 a = src[0], b = src[1];
+                acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+                acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+            }
+            uint32_t r[4];
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+                r[q] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + c0) = make_uint4(r[0], r[1], r[2], r[3]);
+        }
+    }
+}
+
+// Interleave gate and up rows in groups of G: packed row R of expert e takes
+// gate row (R / 2G) G + R % 2G when R % 2G < G, else up row (R / 2G) G + R % 2G - G.
+// Rows are row_words 4-byte words long.
+__global__ void interleave_rows_kernel(const uint32_t* gate, const uint32_t* up, uint32_t* dst, int E,
+                                       int rows_per_proj, int G, int row_words) {
+    const long long total_rows = 2LL * E * rows_per_proj;
+    for (long long R = blockIdx.x; R < total_rows; R += gridDim.x) {
+        const int e = static_cast<int>(R / (2 * rows_per_proj));
+        const int r = static_cast<int>(R % (2 * rows_per_proj));
+        const int grp = r / (2 * G), within = r % (2 * G);
+        const uint32_t* src = (within < G) ? gate : up;
+        const long long sr = static_cast<long long>(e) * rows_per_proj + grp * G + (within < G ? within : within - G);
+        for (int c = threadIdx.x; c < row_words; c += blockDim.x) dst[R * row_words + c] = src[sr * row_words + c];
+    }
+}
+
+}  // namespace moe

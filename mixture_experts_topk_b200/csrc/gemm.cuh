@@ -1,0 +1,360 @@
+// gemm.cuh -- persistent grouped FP8 GEMM on the 5th-gen tensor cores (tcgen05)
+// with the two epilogues of the MoE expert MLP.
+//
+// Pure-Triton fused MoE article: gate and up projections share one input tile
+// load and SiLU runs in registers, so no intermediate buffers; a precomputed
+// block-id -> (expert id, offset) map runs variable-size expert groups in one
+// launch without padding.  LightMoE README ("MoE inference"): gated
+// activation, requantisation of the hidden, down projection and the routing
+// weight are part of the one layer call.
+//
+// Roles (320 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: A tile [128 rows x 128 K] + B tile [BN rows x 128 K]
+//               per stage into a STAGES-deep shared-memory ring (128-byte swizzle)
+//   warp 1      allocates TMEM, one thread issues tcgen05.mma (M=128, N=BN, K=32)
+//               into a double-buffered fp32 accumulator in TMEM
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator, scales, SwiGLU and
+//               requantisation (gate/up) or routing weight + fp32 store (down)
+// Tile t of the schedule: m-tile t % ntm (expert e, first row), n-block t / ntm.
+// A tile's rows past the expert's last row belong to the next expert or are
+// past the end (TMA zero-fills); the epilogue stores only the expert's rows.
+//
+// PROMOTE: the A operand (and for 128x128-block weights also B) carries one
+// fp32 scale per 128 columns of K, so each 128-deep K block is accumulated
+// alone in TMEM and the epilogue adds it into registers times its scales.
+// Without PROMOTE the whole K reduction stays in TMEM.
+//
+// Every wait is bounded (spin_limit clock cycles): on expiry the kernel records
+// MOE timeout in the status word and leaves its loops; nothing traps.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 128;                 // K bytes (= e4m3 elements) per stage
+constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK;
+
+enum { KIND_GATE_UP = 0, KIND_DOWN = 1 };
+enum { BSCALE_ROW = 0, BSCALE_BLOCK128 = 1 };
+
+struct GemmParams {
+    const int32_t* tiles;       // [ntiles][2] (expert, first row)
+    const int32_t* num_tiles;   // number of m-tiles (device scalar)
+    const int32_t* offsets;     // [E+1]
+    int n_blocks;               // N / BN
+    int num_kb;                 // K / 128
+    int b_rows;                 // rows of B per expert (2I for gate/up, H for down)
+    const float* a_scale;       // X or hidden scales, a_ld floats per row
+    int a_ld;
+    const float* b_scale;       // BSCALE_ROW: [E][b_rows]; BLOCK128: [E][b_rows/128][num_kb]
+    uint8_t* hq;                // gate/up: hidden codes [A][I], scales hs [A][I/128]
+    float* hs;
+    int I;
+    float* o;                   // down: [A][H] fp32
+    int H;
+    const int32_t* perm;        // down: slot -> t*k + j
+    const float* route_w;       // down: [T*k]
+    int32_t* status;
+    long long spin_limit;
+};
+
+template <int BN, int STAGES>
+struct GemmSmem {
+    static constexpr int B_BYTES = BN * GEMM_BK;
+    static constexpr int STAGE_BYTES = GEMM_A_BYTES + B_BYTES;
+    static constexpr int TILES_BYTES = STAGES * STAGE_BYTES;
+    // after the tiles: barriers, TMEM address, amax exchange
+    static constexpr int BAR_OFF = TILES_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 5;
+    static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * NUM_BARS;
+    static constexpr int XCHG_OFF = (TMEM_SLOT_OFF + 4 + 15) / 16 * 16;
+    static constexpr int XCHG_BYTES = 2 * 2 * 128 * 4 * 2;   // [parity][group][row] value + flag
+    static constexpr int TOTAL = XCHG_OFF + XCHG_BYTES + 1024; // + alignment slack
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit) {
+    const bool ok = mbar_wait(bar, parity, limit);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmParams p) {
+    using S = GemmSmem<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::TMEM_SLOT_OFF);
+    float* xval = reinterpret_cast<float*>(smem + S::XCHG_OFF);                 // [2][2][128]
+    int* xflag = reinterpret_cast<int*>(smem + S::XCHG_OFF + 2 * 2 * 128 * 4);  // [2][2][128]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t TMEM_COLS = 2 * BN;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);   // one arrival per epilogue warp
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    for (int i = threadIdx.x; i < 2 * 2 * 128; i += blockDim.x) xflag[i] = 0;
+    if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int ntm = *p.num_tiles;
+    const int total = ntm * p.n_blocks;
+    const long long limit = p.spin_limit;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const int mi = t % ntm, nb = t / ntm;
+                const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
+                const int brow = e * p.b_rows + nb * BN;
+                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, limit)) {
+                        report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + s * S::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
+                    tma_load_2d(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow);
+                }
+            }
+            // loads still in flight land before the CTA may exit
+            const uint32_t first = it > STAGES ? it - STAGES : 0;
+            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, limit);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_e4m3(GEMM_BM, BN);
+            uint32_t it = 0, u = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                uint32_t acc = 0;
+                if (!PROMOTE) {
+                    acc = u & 1;
+                    if (!mbar_wait(&tempty[acc], ((u >> 1) & 1) ^ 1, limit)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                    if (PROMOTE) {
+                        acc = u & 1;
+                        if (!mbar_wait(&tempty[acc], ((u >> 1) & 1) ^ 1, limit)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&full[s], (it / STAGES) & 1, limit)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * S::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + GEMM_A_BYTES;
+                    const uint32_t d = tmem_base + acc * BN;
+#pragma unroll
+                    for (int kk = 0; kk < GEMM_BK / 32; kk++)
+                        mma_f8(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
+                               PROMOTE ? (kk > 0) : (kb > 0 || kk > 0));
+                    mma_commit(&empty[s]);
+                    if (PROMOTE) {
+                        mma_commit(&tfull[acc]);
+                        u++;
+                    }
+                }
+                if (!ok) break;
+                if (!PROMOTE) {
+                    mma_commit(&tfull[acc]);
+                    u++;
+                }
+            }
+            if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
+            mma_commit(drain);                 // every issued MMA has completed ...
+            mbar_wait(drain, 0, limit);        // ... before TMEM can be released
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;
+        const int q = warp & 3;               // TMEM lane quadrant this warp may access
+        const int g = ew >> 2;                // column group
+        const int r = 32 * q + lane;          // row within the tile
+        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+        uint32_t u = 0, iter = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, iter++) {
+            const int mi = t % ntm, nb = t / ntm;
+            const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
+            const int row = row0 + r;
+            const bool valid = row < p.offsets[e + 1];
+
+            if (KIND == KIND_GATE_UP) {
+                float hv[64];
+                if (!PROMOTE) {
+                    const uint32_t acc = u & 1;
+                    if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
+                    tc_fence_after();
+                    const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld] : 0.0f;
+                    const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + nb * BN;
+#pragma unroll
+                    for (int half = 0; half < 2; half++) {
+                        float gv[32], uv[32];
+                        const int c0 = 64 * g + 32 * half;
+                        tmem_ld32(lane_addr + acc * BN + c0, gv);
+                        tmem_ld32(lane_addr + acc * BN + 128 + c0, uv);
+#pragma unroll
+                        for (int c = 0; c < 32; c++) {
+                            const float gg = gv[c] * (sa * __ldg(bs + c0 + c));
+                            const float uu = uv[c] * (sa * __ldg(bs + 128 + c0 + c));
+                            hv[32 * half + c] = gg / (1.0f + expf(-gg)) * uu;
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[acc]);
+                    u++;
+                } else {
+                    float ag[64], au[64];
+#pragma unroll
+                    for (int c = 0; c < 64; c++) ag[c] = au[c] = 0.0f;
+                    for (int kb = 0; kb < p.num_kb; kb++) {
+                        const uint32_t acc = u & 1;
+                        if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
+                        tc_fence_after();
+                        const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld + kb] : 0.0f;
+                        const float* bsb = p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + 2 * nb) * p.num_kb;
+                        const float sg = sa * __ldg(bsb + kb), su = sa * __ldg(bsb + p.num_kb + kb);
+#pragma unroll
+                        for (int half = 0; half < 2; half++) {
+                            float v[32];
+                            const int c0 = 64 * g + 32 * half;
+                            tmem_ld32(lane_addr + acc * BN + c0, v);
+#pragma unroll
+                            for (int c = 0; c < 32; c++) ag[32 * half + c] = fmaf(v[c], sg, ag[32 * half + c]);
+                            tmem_ld32(lane_addr + acc * BN + 128 + c0, v);
+#pragma unroll
+                            for (int c = 0; c < 32; c++) au[32 * half + c] = fmaf(v[c], su, au[32 * half + c]);
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[acc]);
+                        u++;
+                    }
+                    if (!ok) break;
+#pragma unroll
+                    for (int c = 0; c < 64; c++) hv[c] = ag[c] / (1.0f + expf(-ag[c])) * au[c];
+                }
+                // requantise the 128-column hidden block of this row: the two
+                // column groups exchange their partial amax through shared memory
+                float amax = 0.0f;
+#pragma unroll
+                for (int c = 0; c < 64; c++) amax = fmaxf(amax, fabsf(hv[c]));
+                const int par = iter & 1;
+                volatile float* xv = xval;
+                volatile int* xf = xflag;
+                xv[(par * 2 + g) * 128 + r] = amax;
+                __threadfence_block();
+                xf[(par * 2 + g) * 128 + r] = static_cast<int>(iter) + 1;
+                long long t0 = clock64();
+                while (xf[(par * 2 + (1 - g)) * 128 + r] < static_cast<int>(iter) + 1) {
+                    if (clock64() - t0 > limit) { ok = false; break; }
+                }
+                if (!ok) break;
+                __threadfence_block();
+                amax = fmaxf(amax, xv[(par * 2 + (1 - g)) * 128 + r]);
+                const float s = __fdiv_rn(amax, 448.0f);
+                if (valid) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4) {
+                        uint16_t lo = 0, hi = 0;
+                        if (s != 0.0f) {
+                            lo = f2_to_e4m3x2(__fdiv_rn(hv[c], s), __fdiv_rn(hv[c + 1], s));
+                            hi = f2_to_e4m3x2(__fdiv_rn(hv[c + 2], s), __fdiv_rn(hv[c + 3], s));
+                        }
+                        w[c / 4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(row) * p.I + nb * 128 + 64 * g);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                    if (g == 0) p.hs[static_cast<size_t>(row) * (p.I / 128) + nb] = s;
+                }
+            } else {
+                // ---------------------------------------------------- down
+                constexpr int NC = BN / 2;      // columns per thread
+                float acc_r[NC];
+#pragma unroll
+                for (int c = 0; c < NC; c++) acc_r[c] = 0.0f;
+                const int n0 = nb * BN + g * NC;
+                for (int kb = 0; kb < p.num_kb; kb++) {
+                    const uint32_t acc = u & 1;
+                    if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
+                    tc_fence_after();
+                    float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld + kb] : 0.0f;
+                    if (BSCALE == BSCALE_BLOCK128)
+                        sa *= __ldg(p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + n0 / 128) * p.num_kb + kb);
+#pragma unroll
+                    for (int ch = 0; ch < NC / 32; ch++) {
+                        float v[32];
+                        tmem_ld32(lane_addr + acc * BN + g * NC + 32 * ch, v);
+#pragma unroll
+                        for (int c = 0; c < 32; c++) acc_r[32 * ch + c] = fmaf(v[c], sa, acc_r[32 * ch + c]);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[acc]);
+                    u++;
+                }
+                if (!ok) break;
+                if (valid) {
+                    const float rw = p.route_w[p.perm[row]];
+                    const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + n0;
+                    float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(row) * p.H + n0);
+#pragma unroll
+                    for (int c = 0; c < NC; c += 4) {
+                        float v[4];
+#pragma unroll
+                        for (int i = 0; i < 4; i++) {
+                            v[i] = acc_r[c + i];
+                            if (BSCALE == BSCALE_ROW) v[i] *= __ldg(bs + c + i);
+                            v[i] *= rw;
+                        }
+                        dst[c / 4] = make_float4(v[0], v[1], v[2], v[3]);
+                    }
+                }
+            }
+        }
+        if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_EPILOGUE);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,507 @@
+// moe_api.cu -- the C ABI declared in include/moe_b200.h: argument checks,
+// workspace and packed-weight layouts, tensor maps, and the launch sequence
+// route -> dispatch -> gate/up GEMM -> down GEMM -> combine.
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "moe_b200.h"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "gemm.cuh"
+#include "router.cuh"
+
+using namespace moe;
+
+// ------------------------------------------------------------------ errors
+static thread_local char g_err[512] = "";
+
+static moe_status fail(moe_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+#define CUDA_TRY(expr)                                                                       \
+    do {                                                                                     \
+        cudaError_t err_ = (expr);                                                           \
+        if (err_ != cudaSuccess)                                                             \
+            return fail(MOE_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(err_));     \
+    } while (0)
+
+#define LAUNCH_CHECK(name)                                                                   \
+    do {                                                                                     \
+        cudaError_t err_ = cudaGetLastError();                                               \
+        if (err_ != cudaSuccess)                                                             \
+            return fail(MOE_ERR_CUDA, "launch of %s failed: %s", name, cudaGetErrorString(err_)); \
+    } while (0)
+
+extern "C" const char* moe_last_error(void) { return g_err; }
+
+// ------------------------------------------------------------------ layouts
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WsLayout {
+    size_t status, ids, w, counts, offsets, num_tiles, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
+};
+struct WLayout {
+    size_t gu_q, gu_s, d_q, d_s, gu_g, d_g, total;
+};
+
+struct moe_handle {
+    moe_config cfg;
+    int device;
+    int num_sms;
+    WsLayout ws;
+    WLayout wl;
+    long long spin_limit;
+};
+
+static size_t code_bytes(int fmt, int K) { return fmt == MOE_FMT_NVFP4 ? K / 2 : K; }
+static size_t act_scale_bytes(int fmt, int K) {
+    if (fmt == MOE_FMT_FP8_ROW) return 4;
+    if (fmt == MOE_FMT_FP8_BLOCK128) return 4 * (K / 128);
+    return K / 16;
+}
+static size_t hidden_scale_bytes(int fmt, int I) { return fmt == MOE_FMT_NVFP4 ? I / 16 : 4 * (I / 128); }
+
+static WsLayout make_ws_layout(const moe_config& c) {
+    const size_t A = static_cast<size_t>(c.max_T) * c.k;
+    const size_t nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
+    const size_t tiles_cap = A / TILE_M + c.E + 1;
+    WsLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    L.status = take(64 * 4);
+    L.ids = take(A * 4);
+    L.w = take(A * 4);
+    L.counts = take(c.E * 4);
+    L.offsets = take((c.E + 1) * 4);
+    L.num_tiles = take(4);
+    L.chunk = take(nchunks * c.E * 4);
+    L.tiles = take(tiles_cap * 8);
+    L.perm = take(A * 4);
+    L.inv = take(A * 4);
+    L.xglobal = take(16);
+    L.xq = take(A * code_bytes(c.fmt, c.H));
+    L.xs = take(A * act_scale_bytes(c.fmt, c.H));
+    L.hq = take(A * code_bytes(c.fmt, c.I));
+    L.hs = take(A * hidden_scale_bytes(c.fmt, c.I));
+    L.o = take(A * c.H * 4);
+    L.total = off;
+    return L;
+}
+
+static WLayout make_w_layout(const moe_config& c) {
+    const size_t E = c.E, H = c.H, I = c.I;
+    WLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    L.gu_q = take(E * 2 * I * code_bytes(c.fmt, c.H));
+    L.d_q = take(E * H * code_bytes(c.fmt, c.I));
+    if (c.fmt == MOE_FMT_FP8_ROW) {
+        L.gu_s = take(E * 2 * I * 4);
+        L.d_s = take(E * H * 4);
+    } else if (c.fmt == MOE_FMT_FP8_BLOCK128) {
+        L.gu_s = take(E * (2 * I / 128) * (H / 128) * 4);
+        L.d_s = take(E * (H / 128) * (I / 128) * 4);
+    } else {
+        L.gu_s = take(E * 2 * I * (H / 16));
+        L.d_s = take(E * H * (I / 16));
+    }
+    L.gu_g = take(E * 2 * 4);
+    L.d_g = take(E * 4);
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------------ init
+extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
+    if (!cfg || !out) return fail(MOE_ERR_INVALID_ARG, "moe_init: null argument");
+    const moe_config& c = *cfg;
+    if (c.H <= 0 || c.I <= 0 || c.E <= 0 || c.k <= 0 || c.max_T <= 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_init: sizes must be positive");
+    if (c.score != MOE_SCORE_SOFTMAX && c.score != MOE_SCORE_SIGMOID)
+        return fail(MOE_ERR_INVALID_ARG, "moe_init: unknown score function %d", c.score);
+    if (c.fmt != MOE_FMT_FP8_ROW && c.fmt != MOE_FMT_FP8_BLOCK128 && c.fmt != MOE_FMT_NVFP4)
+        return fail(MOE_ERR_INVALID_ARG, "moe_init: unknown format %d", c.fmt);
+    if (c.H % 256 != 0 || c.I % 128 != 0)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: H must be a multiple of 256 and I of 128 (H=%d I=%d)", c.H, c.I);
+    if (c.k > 8 || c.k > c.E || c.E > 256)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: need 1 <= k <= 8, k <= E <= 256 (E=%d k=%d)", c.E, c.k);
+    if (static_cast<long long>(c.max_T) * c.k > 131072)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: max_T * k must be <= 131072");
+    if (c.fmt == MOE_FMT_NVFP4)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: the NVFP4 format is not built in this library yet");
+    moe_handle* h = new (std::nothrow) moe_handle;
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_init: out of host memory");
+    h->cfg = c;
+    CUDA_TRY(cudaGetDevice(&h->device));
+    CUDA_TRY(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device));
+    h->ws = make_ws_layout(c);
+    h->wl = make_w_layout(c);
+    h->spin_limit = 2000000000LL;   // ~1 s of SM clock per wait
+    *out = h;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_destroy(moe_handle* h) {
+    delete h;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_weights_size(const moe_handle* h, size_t* bytes) {
+    if (!h || !bytes) return fail(MOE_ERR_INVALID_ARG, "moe_weights_size: null argument");
+    *bytes = h->wl.total;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_workspace_size(const moe_handle* h, size_t* bytes) {
+    if (!h || !bytes) return fail(MOE_ERR_INVALID_ARG, "moe_workspace_size: null argument");
+    *bytes = h->ws.total;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_workspace_view* v) {
+    if (!h || !ws || !v) return fail(MOE_ERR_INVALID_ARG, "moe_workspace_view_get: null argument");
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    const WsLayout& L = h->ws;
+    v->status = reinterpret_cast<int32_t*>(b + L.status);
+    v->ids = reinterpret_cast<int32_t*>(b + L.ids);
+    v->w = reinterpret_cast<float*>(b + L.w);
+    v->counts = reinterpret_cast<int32_t*>(b + L.counts);
+    v->offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+    v->num_tiles = reinterpret_cast<int32_t*>(b + L.num_tiles);
+    v->tiles = reinterpret_cast<int32_t*>(b + L.tiles);
+    v->perm = reinterpret_cast<int32_t*>(b + L.perm);
+    v->inv = reinterpret_cast<int32_t*>(b + L.inv);
+    v->x_global = reinterpret_cast<float*>(b + L.xglobal);
+    v->xq = b + L.xq;
+    v->xs = b + L.xs;
+    v->hq = b + L.hq;
+    v->hs = b + L.hs;
+    v->o = reinterpret_cast<float*>(b + L.o);
+    return MOE_OK;
+}
+
+static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+static moe_status check_T(const moe_handle* h, int T, const char* who) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "%s: null handle", who);
+    if (T < 0 || T > h->cfg.max_T) return fail(MOE_ERR_INVALID_ARG, "%s: T=%d outside [0, max_T=%d]", who, T, h->cfg.max_T);
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ pack
+extern "C" moe_status moe_pack_weights(const moe_handle* h, const moe_weights* src, void* packed, moe_stream_t stream) {
+    if (!h || !src || !packed) return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: null argument");
+    if (!src->gate_q || !src->up_q || !src->down_q || !src->gate_s || !src->up_s || !src->down_s)
+        return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: null weight pointer");
+    if (!aligned256(packed)) return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: packed must be 256-byte aligned");
+    const moe_config& c = h->cfg;
+    uint8_t* b = static_cast<uint8_t*>(packed);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int grid = 4 * h->num_sms;
+    interleave_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(src->gate_q),
+                                                 static_cast<const uint32_t*>(src->up_q),
+                                                 reinterpret_cast<uint32_t*>(b + h->wl.gu_q), c.E, c.I, 128,
+                                                 static_cast<int>(code_bytes(c.fmt, c.H) / 4));
+    LAUNCH_CHECK("interleave_rows_kernel(codes)");
+    if (c.fmt == MOE_FMT_FP8_ROW) {
+        interleave_rows_kernel<<<grid, 32, 0, st>>>(static_cast<const uint32_t*>(src->gate_s),
+                                                    static_cast<const uint32_t*>(src->up_s),
+                                                    reinterpret_cast<uint32_t*>(b + h->wl.gu_s), c.E, c.I, 128, 1);
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_s, src->down_s, static_cast<size_t>(c.E) * c.H * 4,
+                                 cudaMemcpyDeviceToDevice, st));
+    } else {
+        interleave_rows_kernel<<<grid, 32, 0, st>>>(static_cast<const uint32_t*>(src->gate_s),
+                                                    static_cast<const uint32_t*>(src->up_s),
+                                                    reinterpret_cast<uint32_t*>(b + h->wl.gu_s), c.E, c.I / 128, 1,
+                                                    c.H / 128);
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_s, src->down_s,
+                                 static_cast<size_t>(c.E) * (c.H / 128) * (c.I / 128) * 4, cudaMemcpyDeviceToDevice, st));
+    }
+    LAUNCH_CHECK("interleave_rows_kernel(scales)");
+    CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_q, src->down_q, static_cast<size_t>(c.E) * c.H * code_bytes(c.fmt, c.I),
+                             cudaMemcpyDeviceToDevice, st));
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ route
+extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const float* wr, const float* bias,
+                                int32_t* ids, float* w, void* ws, moe_stream_t stream) {
+    moe_status st0 = check_T(h, T, "moe_route");
+    if (st0 != MOE_OK) return st0;
+    if (T == 0) return MOE_OK;
+    if (!x || !wr || !ids || !w) return fail(MOE_ERR_INVALID_ARG, "moe_route: null argument");
+    if (h->cfg.has_bias && !bias) return fail(MOE_ERR_INVALID_ARG, "moe_route: config has a bias but bias is null");
+    if (!h->cfg.has_bias) bias = nullptr;
+    if (!aligned256(x) || !aligned256(wr)) return fail(MOE_ERR_INVALID_ARG, "moe_route: x and wr must be 256-byte aligned");
+    (void)ws;
+    RouterParams p;
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.wr = wr;
+    p.bias = bias;
+    p.ids = ids;
+    p.w = w;
+    p.T = T;
+    p.H = h->cfg.H;
+    p.E = h->cfg.E;
+    p.k = h->cfg.k;
+    p.score = h->cfg.score;
+    const int grid = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
+    router_topk_kernel<<<grid, ROUTER_WARPS * 32, ROUTER_TOKENS * h->cfg.E * sizeof(float),
+                         reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    LAUNCH_CHECK("router_topk_kernel");
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ dispatch
+extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int32_t* ids, int T, void* ws,
+                                   moe_stream_t stream) {
+    moe_status st0 = check_T(h, T, "moe_dispatch");
+    if (st0 != MOE_OK) return st0;
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "moe_dispatch: null workspace");
+    if (T > 0 && (!x || !ids)) return fail(MOE_ERR_INVALID_ARG, "moe_dispatch: null argument");
+    if (!aligned256(ws) || (T > 0 && !aligned256(x)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_dispatch: x and ws must be 256-byte aligned");
+    const moe_config& c = h->cfg;
+    moe_workspace_view v;
+    moe_workspace_view_get(h, ws, &v);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int A = T * c.k;
+    const int nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
+    int32_t* chunk = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + h->ws.chunk);
+    if (A > 0) {
+        hist_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.status);
+        LAUNCH_CHECK("hist_kernel");
+    }
+    scan_kernel<<<1, 256, 0, st>>>(chunk, nchunks, c.E, v.counts, v.offsets, v.tiles, v.num_tiles);
+    LAUNCH_CHECK("scan_kernel");
+    if (A == 0) return MOE_OK;
+    rank_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.perm, v.inv);
+    LAUNCH_CHECK("rank_kernel");
+    const int qgrid = std::min((T + 7) / 8, 8 * h->num_sms);
+    if (c.fmt == MOE_FMT_FP8_ROW)
+        quant_scatter_kernel<0><<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, v.inv, v.xq,
+                                                       static_cast<float*>(v.xs));
+    else
+        quant_scatter_kernel<1><<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, v.inv, v.xq,
+                                                       static_cast<float*>(v.xs));
+    LAUNCH_CHECK("quant_scatter_kernel");
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2D byte matrix [rows][inner] with row pitch `pitch`, 128-byte swizzled boxes
+// of box_inner bytes x box_rows rows; rows past the end read as zero.
+static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
+                            uint32_t box_inner, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {pitch};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return MOE_OK;
+}
+
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
+static moe_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
+                              cudaStream_t st) {
+    using S = GemmSmem<BN, STAGES>;
+    static_assert(S::TOTAL <= 232448, "shared memory of the GEMM exceeds 227 KB");
+    auto kern = grouped_gemm_kernel<KIND, BSCALE, PROMOTE, BN, STAGES>;
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL));
+    kern<<<grid, GEMM_THREADS, S::TOTAL, st>>>(ta, tb, p);
+    LAUNCH_CHECK("grouped_gemm_kernel");
+    return MOE_OK;
+}
+
+// upper bound of the m-tiles the schedule can hold for T tokens
+static int max_m_tiles(const moe_config& c, int T) {
+    const int A = T * c.k;
+    return A / TILE_M + std::min(c.E, A);
+}
+
+// ------------------------------------------------------------------ gate/up
+extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T, void* ws, moe_stream_t stream) {
+    moe_status st0 = check_T(h, T, "moe_gate_up");
+    if (st0 != MOE_OK) return st0;
+    if (T == 0) return MOE_OK;
+    if (!packed || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_gate_up: null argument");
+    if (!aligned256(packed) || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_gate_up: pointers must be 256-byte aligned");
+    if (T == 0) return MOE_OK;
+    const moe_config& c = h->cfg;
+    moe_workspace_view v;
+    moe_workspace_view_get(h, ws, &v);
+    const uint8_t* pw = static_cast<const uint8_t*>(packed);
+    const size_t A = static_cast<size_t>(c.max_T) * c.k;
+    CUtensorMap ta, tb;
+    moe_status r = make_tmap(&ta, v.xq, c.H, A, c.H, GEMM_BK, GEMM_BM);
+    if (r != MOE_OK) return r;
+    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * 2 * c.I, c.H, GEMM_BK, 256);
+    if (r != MOE_OK) return r;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.tiles = v.tiles;
+    p.num_tiles = v.num_tiles;
+    p.offsets = v.offsets;
+    p.n_blocks = 2 * c.I / 256;
+    p.num_kb = c.H / GEMM_BK;
+    p.b_rows = 2 * c.I;
+    p.a_scale = static_cast<const float*>(v.xs);
+    p.a_ld = (c.fmt == MOE_FMT_FP8_ROW) ? 1 : c.H / 128;
+    p.b_scale = reinterpret_cast<const float*>(pw + h->wl.gu_s);
+    p.hq = v.hq;
+    p.hs = static_cast<float*>(v.hs);
+    p.I = c.I;
+    p.H = c.H;
+    p.status = v.status;
+    p.spin_limit = h->spin_limit;
+    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4>(ta, tb, p, grid, st);
+    return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4>(ta, tb, p, grid, st);
+}
+
+// ------------------------------------------------------------------ down
+extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const float* w, int T, void* ws,
+                               moe_stream_t stream) {
+    moe_status st0 = check_T(h, T, "moe_down");
+    if (st0 != MOE_OK) return st0;
+    if (T == 0) return MOE_OK;
+    if (!packed || !ws || !w) return fail(MOE_ERR_INVALID_ARG, "moe_down: null argument");
+    if (!aligned256(packed) || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_down: pointers must be 256-byte aligned");
+    if (T == 0) return MOE_OK;
+    const moe_config& c = h->cfg;
+    moe_workspace_view v;
+    moe_workspace_view_get(h, ws, &v);
+    const uint8_t* pw = static_cast<const uint8_t*>(packed);
+    const size_t A = static_cast<size_t>(c.max_T) * c.k;
+    constexpr int BN = 256;
+    CUtensorMap ta, tb;
+    moe_status r = make_tmap(&ta, v.hq, c.I, A, c.I, GEMM_BK, GEMM_BM);
+    if (r != MOE_OK) return r;
+    r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, BN);
+    if (r != MOE_OK) return r;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.tiles = v.tiles;
+    p.num_tiles = v.num_tiles;
+    p.offsets = v.offsets;
+    p.n_blocks = c.H / BN;
+    p.num_kb = c.I / GEMM_BK;
+    p.b_rows = c.H;
+    p.a_scale = static_cast<const float*>(v.hs);
+    p.a_ld = c.I / 128;
+    p.b_scale = reinterpret_cast<const float*>(pw + h->wl.d_s);
+    p.o = static_cast<float*>(v.o);
+    p.H = c.H;
+    p.I = c.I;
+    p.perm = v.perm;
+    p.route_w = w;
+    p.status = v.status;
+    p.spin_limit = h->spin_limit;
+    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_DOWN, BSCALE_ROW, true, BN, 4>(ta, tb, p, grid, st);
+    return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, BN, 4>(ta, tb, p, grid, st);
+}
+
+// ------------------------------------------------------------------ combine
+extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws, moe_stream_t stream) {
+    moe_status st0 = check_T(h, T, "moe_combine");
+    if (st0 != MOE_OK) return st0;
+    if (T == 0) return MOE_OK;
+    if (!y || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_combine: null argument");
+    if (!aligned256(y) || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_combine: pointers must be 256-byte aligned");
+    if (T == 0) return MOE_OK;
+    moe_workspace_view v;
+    moe_workspace_view_get(h, ws, &v);
+    const int grid = std::min(T, 16 * h->num_sms);
+    combine_kernel<<<grid, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const float*>(v.o), v.inv, T, h->cfg.H, h->cfg.k, static_cast<__nv_bfloat16*>(y));
+    LAUNCH_CHECK("combine_kernel");
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ layer
+extern "C" moe_status moe_forward_routed(const moe_handle* h, const void* x, int T, const int32_t* ids, const float* w,
+                                         const void* packed, void* y, void* ws, moe_stream_t stream) {
+    moe_status r = moe_dispatch(h, x, ids, T, ws, stream);
+    if (r != MOE_OK) return r;
+    r = moe_gate_up(h, packed, T, ws, stream);
+    if (r != MOE_OK) return r;
+    r = moe_down(h, packed, w, T, ws, stream);
+    if (r != MOE_OK) return r;
+    return moe_combine(h, T, y, ws, stream);
+}
+
+extern "C" moe_status moe_forward(const moe_handle* h, const void* x, int T, const float* wr, const float* bias,
+                                  const void* packed, void* y, void* ws, moe_stream_t stream) {
+    moe_status st0 = check_T(h, T, "moe_forward");
+    if (st0 != MOE_OK) return st0;
+    if (!ws) return fail(MOE_ERR_INVALID_ARG, "moe_forward: null workspace");
+    moe_workspace_view v;
+    moe_workspace_view_get(h, ws, &v);
+    moe_status r = moe_route(h, x, T, wr, bias, v.ids, v.w, ws, stream);
+    if (r != MOE_OK) return r;
+    return moe_forward_routed(h, x, T, v.ids, v.w, packed, y, ws, stream);
+}
+
+// ------------------------------------------------------------------ status
+extern "C" moe_status moe_workspace_init(const moe_handle* h, void* ws, moe_stream_t stream) {
+    if (!h || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_workspace_init: null argument");
+    CUDA_TRY(cudaMemsetAsync(static_cast<uint8_t*>(ws) + h->ws.status, 0, 64 * 4,
+                             reinterpret_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_get_status(const moe_handle* h, void* ws, moe_stream_t stream) {
+    if (!h || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_get_status: null argument");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    CUDA_TRY(cudaStreamSynchronize(st));
+    int32_t s[2] = {0, 0};
+    int32_t* dev = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + h->ws.status);
+    CUDA_TRY(cudaMemcpy(s, dev, sizeof(s), cudaMemcpyDeviceToHost));
+    if (s[0] == 0) return MOE_OK;
+    CUDA_TRY(cudaMemset(dev, 0, sizeof(s)));
+    static const char* where[] = {"?", "GEMM producer", "GEMM MMA issuer", "GEMM epilogue", "dispatch",
+                                  "router", "combine", "GEMM schedule"};
+    const char* wn = (s[1] >= 0 && s[1] < 8) ? where[s[1]] : "?";
+    if (s[0] == MOE_ERR_DEVICE_TIMEOUT) return fail(MOE_ERR_DEVICE_TIMEOUT, "device wait ran out in %s", wn);
+    if (s[0] == MOE_ERR_DEVICE_BOUNDS) return fail(MOE_ERR_DEVICE_BOUNDS, "index out of range in %s", wn);
+    return fail(static_cast<moe_status>(s[0]), "device error %d in %s", s[0], wn);
+}

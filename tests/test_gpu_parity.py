@@ -1,0 +1,203 @@
+"""Parity of the CUDA path with the CPU oracle, step by step and end to end.
+
+Bit-exact: router ids, dispatch counts/offsets/perm/inv/tile table, quantised
+X codes and scales.  Floating point: routing weights within 2e-6 (fp32 vs
+fp64), the hidden codes within one code step on at most 1e-3 of the
+elements, the layer output within |gpu - ref| <= 2e-2 |ref| + 2e-3 rms(ref).
+All calls go through the C ABI (mixture_experts_topk_b200.native).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_topk_b200 import native, synth, workloads as W
+from helpers import bits, slot_order_reference, tolerance_violations
+
+pytestmark = pytest.mark.gpu
+
+# small shapes spanning several tiles and ragged tails, plus the named workloads at small T
+CASES = {
+    "tiny": (W.WORKLOADS["tiny"], 16),
+    "row-ragged": (W.custom(H=512, I=384, E=8, k=2), 300),
+    "row-skew-e64": (W.custom(H=256, I=256, E=64, k=8, zipf_s=1.2), 100),
+    "block128-ragged": (W.custom(H=512, I=384, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 300),
+    "t1": (W.custom(H=256, I=128, E=8, k=2), 1),
+}
+
+
+def build_case(name, seed=0):
+    wl, T = CASES[name]
+    d = synth.layer(wl, seed=seed)
+    x = synth.tokens(wl, T, seed=seed)
+    return wl, T, d, x
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    native.load()
+
+
+def run_route(layer, x, d):
+    T = x.shape[0]
+    wl = layer.wl
+    ids = torch.empty(T, wl.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, wl.k, dtype=torch.float32, device="cuda")
+    bias = d["bias"].cuda() if d["bias"] is not None else None
+    native.moe_route(layer.h, x.cuda(), T, d["wr"].cuda(), bias, ids, w, layer.ws)
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_router_ids_bit_exact(name):
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    ids, w = run_route(layer, x, d)
+    lg = oracle.router_logits(bits(x), d["wr"].numpy(), None if d["bias"] is None else d["bias"].numpy())
+    ids_ref, w_ref = oracle.topk(lg, wl.k, wl.score)
+    assert (ids == ids_ref).all()
+    np.testing.assert_allclose(w, w_ref, rtol=0, atol=2e-6)
+    assert layer.status()[0] == 0
+
+
+@pytest.mark.parametrize("H,E,k,score,T", [(7168, 256, 8, W.SCORE_SIGMOID, 20), (2048, 256, 8, W.SCORE_SOFTMAX, 64),
+                                           (4096, 8, 2, W.SCORE_SOFTMAX, 33)])
+def test_router_named_shapes_bit_exact(H, E, k, score, T):
+    wl = W.custom(H=H, I=128, E=E, k=k, score=score, router_init="uniform")
+    wr, _ = synth.router(wl, seed=3)
+    x = synth.tokens(wl, T, seed=3)
+    h = native.moe_init(wl, T)
+    ws = torch.empty(native.moe_workspace_size(h), dtype=torch.uint8, device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    native.moe_route(h, x.cuda(), T, wr.cuda(), None, ids, w, ws)
+    torch.cuda.synchronize()
+    ids_ref, w_ref = oracle.topk(oracle.router_logits(bits(x), wr.numpy()), k, score)
+    assert (ids.cpu().numpy() == ids_ref).all()
+    np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=0, atol=2e-6)
+    native.moe_destroy(h)
+
+
+def test_router_equal_logits_tie_break():
+    wl = W.custom(H=256, I=128, E=16, k=4)
+    h = native.moe_init(wl, 8)
+    ws = torch.empty(native.moe_workspace_size(h), dtype=torch.uint8, device="cuda")
+    x = synth.tokens(wl, 8, seed=1).cuda()
+    wr = torch.zeros(16, 256, device="cuda")
+    ids = torch.empty(8, 4, dtype=torch.int32, device="cuda")
+    w = torch.empty(8, 4, dtype=torch.float32, device="cuda")
+    native.moe_route(h, x, 8, wr, None, ids, w, ws)
+    torch.cuda.synchronize()
+    assert (ids.cpu().numpy() == np.arange(4)).all()
+    assert np.allclose(w.cpu().numpy(), 0.25, atol=0)
+    native.moe_destroy(h)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_dispatch_bit_exact(name):
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    L = oracle.Layer(wl, d)
+    ids, w, _ = L.forward(bits(x), d["wr"].numpy(), None if d["bias"] is None else d["bias"].numpy(),
+                          sel=np.zeros(0, np.int32))
+    ref = slot_order_reference(wl, L, x, ids, w, with_ffn=False)
+    native.moe_dispatch(layer.h, x.cuda(), torch.from_numpy(ids).cuda(), T, layer.ws)
+    torch.cuda.synchronize()
+    A = T * wl.k
+    E = wl.E
+    counts, offsets, perm, inv = oracle.dispatch(ids, E)
+    assert (layer.region("counts", torch.int32, E).cpu().numpy() == counts).all()
+    assert (layer.region("offsets", torch.int32, E + 1).cpu().numpy() == offsets).all()
+    assert (layer.region("perm", torch.int32, A).cpu().numpy() == perm).all()
+    assert (layer.region("inv", torch.int32, A).cpu().numpy() == inv).all()
+    te, tr = oracle.schedule(offsets)
+    nt = int(layer.region("num_tiles", torch.int32, 1).cpu().numpy()[0])
+    assert nt == te.size
+    tiles = layer.region("tiles", torch.int32, 2 * nt).cpu().numpy().reshape(nt, 2)
+    assert (tiles[:, 0] == te).all() and (tiles[:, 1] == tr).all()
+    xq = layer.region("xq", torch.uint8, A * wl.H).cpu().numpy().reshape(A, wl.H)
+    assert (xq == ref["xq"]).all()
+    if wl.fmt == W.FMT_FP8_ROW:
+        xs = layer.region("xs", torch.float32, A).cpu().numpy()
+    else:
+        xs = layer.region("xs", torch.float32, A * wl.H // 128).cpu().numpy().reshape(A, -1)
+    assert (xs == ref["xs"]).all()
+    assert layer.status()[0] == 0
+
+
+def _dispatch_and_reference(name):
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    L = oracle.Layer(wl, d)
+    bias = None if d["bias"] is None else d["bias"].numpy()
+    ids, w, _ = L.forward(bits(x), d["wr"].numpy(), bias, sel=np.zeros(0, np.int32))
+    ref = slot_order_reference(wl, L, x, ids, w)
+    native.moe_dispatch(layer.h, x.cuda(), torch.from_numpy(ids).cuda(), T, layer.ws)
+    return wl, T, d, x, layer, ids, w, ref
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_gate_up_hidden_matches_oracle(name):
+    wl, T, d, x, layer, ids, w, ref = _dispatch_and_reference(name)
+    native.moe_gate_up(layer.h, layer.packed, T, layer.ws)
+    torch.cuda.synchronize()
+    assert layer.status()[0] == 0
+    A = T * wl.k
+    hq = layer.region("hq", torch.uint8, A * wl.I).cpu().numpy().reshape(A, wl.I)
+    hs = layer.region("hs", torch.float32, A * wl.I // 128).cpu().numpy().reshape(A, -1)
+    np.testing.assert_allclose(hs, ref["hs"], rtol=1e-4, atol=0)
+    mism = hq != ref["hq"]
+    assert mism.mean() <= 1e-3, f"{mism.mean():.2e} of the hidden codes differ"
+    # a differing code is one step away (a rounding-boundary flip), never more
+    v_gpu = torch.from_numpy(hq).view(torch.float8_e4m3fn).float().numpy()
+    v_ref = torch.from_numpy(ref["hq"]).view(torch.float8_e4m3fn).float().numpy()
+    assert np.all(np.abs(v_gpu - v_ref) <= np.abs(v_ref) * 0.125 + 2.0 ** -9)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_down_matches_oracle_on_oracle_hidden(name):
+    wl, T, d, x, layer, ids, w, ref = _dispatch_and_reference(name)
+    A = T * wl.k
+    layer.region("hq", torch.uint8, A * wl.I).copy_(torch.from_numpy(ref["hq"].reshape(-1)).cuda())
+    layer.region("hs", torch.float32, A * wl.I // 128).copy_(torch.from_numpy(ref["hs"].reshape(-1)).cuda())
+    w_dev = torch.from_numpy(w.astype(np.float32)).cuda()
+    native.moe_down(layer.h, layer.packed, w_dev, T, layer.ws)
+    torch.cuda.synchronize()
+    assert layer.status()[0] == 0
+    o = layer.region("o", torch.float32, A * wl.H).cpu().numpy().reshape(A, wl.H)
+    assert tolerance_violations(o, ref["o_w"]) == 0
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_end_to_end(name):
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    bias = d["bias"].cuda() if d["bias"] is not None else None
+    y = layer.forward(x.cuda(), d["wr"].cuda(), bias)
+    torch.cuda.synchronize()
+    assert layer.status()[0] == 0
+    L = oracle.Layer(wl, d)
+    ids, w, y_ref = L.forward(bits(x), d["wr"].numpy(), None if d["bias"] is None else d["bias"].numpy())
+    assert (layer.region("ids", torch.int32, T * wl.k).cpu().numpy().reshape(T, wl.k) == ids).all()
+    assert tolerance_violations(y.float().cpu().numpy(), y_ref) == 0
+
+
+def test_forward_twice_same_bits():
+    wl, T, d, x = build_case("row-ragged")
+    layer = native.Layer(wl, d, max_T=T)
+    y1 = layer.forward(x.cuda(), d["wr"].cuda(), None).clone()
+    y2 = layer.forward(x.cuda(), d["wr"].cuda(), None)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_empty_batch():
+    wl, T, d, x = build_case("tiny")
+    layer = native.Layer(wl, d, max_T=T)
+    y = torch.empty(0, wl.H, dtype=torch.bfloat16, device="cuda")
+    native.moe_forward(layer.h, x[:0].cuda(), 0, d["wr"].cuda(), None, layer.packed, y, layer.ws)
+    torch.cuda.synchronize()
+    assert layer.status()[0] == 0
