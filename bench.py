@@ -57,7 +57,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -136,9 +136,20 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    # ---- device-timed steps (inputs already resident)
+    # ---- device-timed steps (inputs already resident).  The clock sampler
+    # starts first and ~0.5 s of untimed steps run before the timed ones, so
+    # samples land under load even when the timed region itself is short.
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(3):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    preroll = max(1, int(math.ceil(0.5 / max(ev0.elapsed_time(ev1) / 3e3, 1e-6))))
     with ClockSampler(local_rank) as clk:
+        time.sleep(0.2)
+        for _ in range(preroll):
+            step()
         barrier()
         torch.cuda.synchronize()
         ev0.record(stream)

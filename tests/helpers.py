@@ -55,3 +55,47 @@ def slot_order_reference(wl, L, x_bf16, ids, w, with_ffn=True):
     o_w = o * wflat[perm][:, None]
     return dict(counts=counts, offsets=offsets, perm=perm, inv=inv, xq=xq, xs=xs, h=h, hq=hq, hs=hs,
                 o=o, o_w=o_w, x_global=g)
+
+
+def fp8_values(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def hidden_deviation_bound(wl, L, ids, w, ref, hq_gpu, hs_gpu, tokens=None):
+    """Largest change of Y that differences between the GPU's and the oracle's
+    requantised hidden can cause, per output element:
+        sum_j |w_j| sum_n |h_gpu[slot(t,j), n] - h_ref[slot(t,j), n]| |W_down[e_j][m, n]|
+    h values are code value x block scale.  A hidden code that rounds the other
+    way at a rounding boundary (fp32 vs fp64 accumulation) moves its whole
+    output row by about one e4m3 step times the weights; this bound lets the
+    end-to-end check tell such moves from real errors.  (FP8 formats only.)"""
+    T = ids.shape[0]
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    nb = wl.I // 128
+    extra = np.zeros((len(tokens), wl.H))
+    wd_abs = {}
+    for i, t in enumerate(tokens):
+        for j in range(wl.k):
+            e = int(ids[t, j])
+            r = int(ref["inv"][t * wl.k + j])
+            v_gpu = fp8_values(hq_gpu[r]) * np.repeat(hs_gpu[r].reshape(nb).astype(np.float64), 128)
+            v_ref = fp8_values(ref["hq"][r]) * np.repeat(ref["hs"][r].reshape(nb).astype(np.float64), 128)
+            dv = np.abs(v_gpu - v_ref)
+            if not dv.any():
+                continue
+            if e not in wd_abs:
+                wd_abs[e] = np.abs(np.stack([L.weight_row("down", e, m) for m in range(wl.H)]))
+            extra[i] += abs(float(w[t, j])) * (wd_abs[e] @ dv)
+    return extra
+
+
+def tolerance_violations_with_bound(y_gpu, y_ref, extra):
+    """Elements outside 2e-2 |ref| + 2e-3 rms(ref) + extra, and outside the plain tolerance."""
+    y_gpu = np.asarray(y_gpu, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
+    tol = 2e-2 * np.abs(y_ref) + 2e-3 * rms
+    err = np.abs(y_gpu - y_ref)
+    # bf16 output: the bound gets the final rounding of the moved value too
+    slack = extra * (1 + 2.0 ** -8)
+    return int((err > tol + slack).sum()), int((err > tol).sum())
