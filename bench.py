@@ -115,9 +115,11 @@ def run_ours(args, rank, world, local_rank):
     T = args.tokens
     d = synth.layer(wl, seed=0, device=dev)
     layer = native.Layer(wl, d, max_T=T, device=dev)
-    x = synth.tokens(wl, T, seed=rank, device=dev)
     wr = d["wr"]
     bias = d["bias"]
+    del d                      # the packed copy is all the layer reads
+    torch.cuda.empty_cache()
+    x = synth.tokens(wl, T, seed=rank, device=dev)
     y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
