@@ -222,8 +222,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     for (int half = 0; half < 2; half++) {
                         float gv[32], uv[32];
                         const int c0 = 64 * g + 32 * half;
-                        tmem_ld32(lane_addr + acc * BN + c0, gv);
-                        tmem_ld32(lane_addr + acc * BN + 128 + c0, uv);
+                        tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, gv, uv);
 #pragma unroll
                         for (int c = 0; c < 32; c++) {
                             const float gg = gv[c] * (sa * __ldg(bs + c0 + c));
@@ -248,14 +247,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         const float sg = sa * __ldg(bsb + kb), su = sa * __ldg(bsb + p.num_kb + kb);
 #pragma unroll
                         for (int half = 0; half < 2; half++) {
-                            float v[32];
+                            float vg[32], vu[32];
                             const int c0 = 64 * g + 32 * half;
-                            tmem_ld32(lane_addr + acc * BN + c0, v);
+                            tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, vg, vu);
 #pragma unroll
-                            for (int c = 0; c < 32; c++) ag[32 * half + c] = fmaf(v[c], sg, ag[32 * half + c]);
-                            tmem_ld32(lane_addr + acc * BN + 128 + c0, v);
-#pragma unroll
-                            for (int c = 0; c < 32; c++) au[32 * half + c] = fmaf(v[c], su, au[32 * half + c]);
+                            for (int c = 0; c < 32; c++) {
+                                ag[32 * half + c] = fmaf(vg[c], sg, ag[32 * half + c]);
+                                au[32 * half + c] = fmaf(vu[c], su, au[32 * half + c]);
+                            }
                         }
                         tc_fence_before();
                         __syncwarp();
@@ -315,12 +314,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld + kb] : 0.0f;
                     if (BSCALE == BSCALE_BLOCK128)
                         sa *= __ldg(p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + n0 / 128) * p.num_kb + kb);
+                    if constexpr (NC >= 64) {
 #pragma unroll
-                    for (int ch = 0; ch < NC / 32; ch++) {
+                        for (int ch = 0; ch < NC / 64; ch++) {
+                            float v0[32], v1[32];
+                            const uint32_t a = lane_addr + acc * BN + g * NC + 64 * ch;
+                            tmem_ld32x2(a, a + 32, v0, v1);
+#pragma unroll
+                            for (int c = 0; c < 32; c++) {
+                                acc_r[64 * ch + c] = fmaf(v0[c], sa, acc_r[64 * ch + c]);
+                                acc_r[64 * ch + 32 + c] = fmaf(v1[c], sa, acc_r[64 * ch + 32 + c]);
+                            }
+                        }
+                    } else {
                         float v[32];
-                        tmem_ld32(lane_addr + acc * BN + g * NC + 32 * ch, v);
+                        tmem_ld32(lane_addr + acc * BN + g * NC, v);
 #pragma unroll
-                        for (int c = 0; c < 32; c++) acc_r[32 * ch + c] = fmaf(v[c], sa, acc_r[32 * ch + c]);
+                        for (int c = 0; c < 32; c++) acc_r[c] = fmaf(v[c], sa, acc_r[c]);
                     }
                     tc_fence_before();
                     __syncwarp();

@@ -263,8 +263,11 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
     p.E = h->cfg.E;
     p.k = h->cfg.k;
     p.score = h->cfg.score;
-    const int grid = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
-    router_topk_kernel<<<grid, ROUTER_WARPS * 32, ROUTER_TOKENS * h->cfg.E * sizeof(float),
+    const int ngroups = (h->cfg.E + 7) / 8;
+    p.token_groups = std::max(1, std::min(8, ROUTER_WARPS / ngroups));
+    const int tokens_per_cta = 8 * p.token_groups;
+    const int grid = (T + tokens_per_cta - 1) / tokens_per_cta;
+    router_topk_kernel<<<grid, ROUTER_WARPS * 32, tokens_per_cta * h->cfg.E * sizeof(float),
                          reinterpret_cast<cudaStream_t>(stream)>>>(p);
     LAUNCH_CHECK("router_topk_kernel");
     return MOE_OK;

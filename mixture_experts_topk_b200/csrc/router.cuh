@@ -16,7 +16,6 @@
 
 namespace moe {
 
-constexpr int ROUTER_TOKENS = 8;   // tokens per CTA (one per warp for the top-k)
 constexpr int ROUTER_WARPS = 8;
 
 struct RouterParams {
@@ -26,31 +25,44 @@ struct RouterParams {
     int32_t* ids;
     float* w;
     int T, H, E, k, score;
+    int token_groups;    // 8-token groups per CTA (more when E is small, so every warp has work)
 };
 
+__device__ __forceinline__ void router_load_x(const RouterParams& p, int t0, int h0, uint4* xv) {
+#pragma unroll
+    for (int tt = 0; tt < 8; tt++) {
+        const int t = t0 + tt;
+        xv[tt] = (t < p.T) ? __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * p.H + h0))
+                           : make_uint4(0, 0, 0, 0);
+    }
+}
+
 __global__ void __launch_bounds__(ROUTER_WARPS * 32) router_topk_kernel(RouterParams p) {
-    extern __shared__ float lg[];   // [ROUTER_TOKENS][E]
+    extern __shared__ float lg[];   // [8 * token_groups][E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * ROUTER_TOKENS;
+    const int tokens_per_cta = 8 * p.token_groups;
+    const int cta_t0 = blockIdx.x * tokens_per_cta;
     const int nI = p.H >> 8;
     const int ngroups = (p.E + 7) >> 3;
 
-    for (int grp = warp; grp < ngroups; grp += ROUTER_WARPS) {
-        float acc[ROUTER_TOKENS][8];
+    // work item = (8-token group, 8-expert group): an 8 x 8 micro-tile per warp
+    for (int item = warp; item < p.token_groups * ngroups; item += ROUTER_WARPS) {
+        const int tg = item / ngroups, grp = item % ngroups;
+        const int t0 = cta_t0 + 8 * tg;
+        float acc[8][8];
 #pragma unroll
-        for (int a = 0; a < ROUTER_TOKENS; a++)
+        for (int a = 0; a < 8; a++)
 #pragma unroll
             for (int b = 0; b < 8; b++) acc[a][b] = 0.0f;
 
+        uint4 xn[8];
+        router_load_x(p, t0, 8 * lane, xn);
         for (int i = 0; i < nI; i++) {
             const int h0 = 256 * i + 8 * lane;
-            uint4 xv[ROUTER_TOKENS];
+            uint4 xv[8];
 #pragma unroll
-            for (int tt = 0; tt < ROUTER_TOKENS; tt++) {
-                const int t = t0 + tt;
-                xv[tt] = (t < p.T) ? __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * p.H + h0))
-                                   : make_uint4(0, 0, 0, 0);
-            }
+            for (int tt = 0; tt < 8; tt++) xv[tt] = xn[tt];
+            if (i + 1 < nI) router_load_x(p, t0, h0 + 256, xn);   // next chunk in flight
 #pragma unroll
             for (int ee = 0; ee < 8; ee++) {
                 const int e = 8 * grp + ee;
@@ -59,7 +71,7 @@ __global__ void __launch_bounds__(ROUTER_WARPS * 32) router_topk_kernel(RouterPa
                 const float4 wa = __ldg(wp), wb = __ldg(wp + 1);
                 const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-                for (int tt = 0; tt < ROUTER_TOKENS; tt++) {
+                for (int tt = 0; tt < 8; tt++) {
                     const uint32_t u[4] = {xv[tt].x, xv[tt].y, xv[tt].z, xv[tt].w};
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
@@ -70,7 +82,7 @@ __global__ void __launch_bounds__(ROUTER_WARPS * 32) router_topk_kernel(RouterPa
             }
         }
 #pragma unroll
-        for (int tt = 0; tt < ROUTER_TOKENS; tt++)
+        for (int tt = 0; tt < 8; tt++)
 #pragma unroll
             for (int ee = 0; ee < 8; ee++)
 #pragma unroll
@@ -78,62 +90,64 @@ __global__ void __launch_bounds__(ROUTER_WARPS * 32) router_topk_kernel(RouterPa
                     acc[tt][ee] = __fadd_rn(acc[tt][ee], __shfl_xor_sync(0xffffffffu, acc[tt][ee], off));
         if (lane == 0) {
 #pragma unroll
-            for (int tt = 0; tt < ROUTER_TOKENS; tt++)
+            for (int tt = 0; tt < 8; tt++)
 #pragma unroll
                 for (int ee = 0; ee < 8; ee++) {
                     const int e = 8 * grp + ee;
                     if (e < p.E) {
                         float v = acc[tt][ee];
                         if (p.bias) v = __fadd_rn(v, p.bias[e]);
-                        lg[tt * p.E + e] = v;
+                        lg[(8 * tg + tt) * p.E + e] = v;
                     }
                 }
         }
     }
     __syncthreads();
 
-    // top-k of token t0 + warp: k rounds of a warp argmax, larger logit first,
-    // equal logits -> lower expert id.  Lane l owns experts l + 32 m.
-    const int t = t0 + warp;
-    if (t >= p.T) return;
-    const float* l = lg + warp * p.E;
-    uint32_t taken = 0;
-    float sel_v[8];
-    int sel_e[8];
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-        if (j >= p.k) break;
-        float bv = 0.0f;
-        int be = -1;
-        for (int m = 0; 32 * m + lane < p.E; m++) {
-            const int e = 32 * m + lane;
-            if ((taken >> m) & 1u) continue;
-            const float v = l[e];
-            if (be < 0 || v > bv) { bv = v; be = e; }   // e ascending: equal v keeps the lower id
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-        }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        sel_v[j] = bv;
-        sel_e[j] = be;
-    }
-    if (lane == 0) {
-        float z[8], sum = 0.0f;
+    // top-k per token: k rounds of a warp argmax, larger logit first, equal
+    // logits -> lower expert id.  Lane l owns experts l + 32 m.
+    for (int tl = warp; tl < tokens_per_cta; tl += ROUTER_WARPS) {
+        const int t = cta_t0 + tl;
+        if (t >= p.T) break;
+        const float* l = lg + tl * p.E;
+        uint32_t taken = 0;
+        float sel_v[8];
+        int sel_e[8];
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             if (j >= p.k) break;
-            z[j] = (p.score == 0) ? expf(sel_v[j] - sel_v[0]) : 1.0f / (1.0f + expf(-sel_v[j]));
-            sum += z[j];
-        }
+            float bv = 0.0f;
+            int be = -1;
+            for (int m = 0; 32 * m + lane < p.E; m++) {
+                const int e = 32 * m + lane;
+                if ((taken >> m) & 1u) continue;
+                const float v = l[e];
+                if (be < 0 || v > bv) { bv = v; be = e; }   // e ascending: equal v keeps the lower id
+            }
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            if (j >= p.k) break;
-            p.ids[static_cast<size_t>(t) * p.k + j] = sel_e[j];
-            p.w[static_cast<size_t>(t) * p.k + j] = z[j] / sum;
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+            }
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            sel_v[j] = bv;
+            sel_e[j] = be;
+        }
+        if (lane == 0) {
+            float z[8], sum = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (j >= p.k) break;
+                z[j] = (p.score == 0) ? expf(sel_v[j] - sel_v[0]) : 1.0f / (1.0f + expf(-sel_v[j]));
+                sum += z[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (j >= p.k) break;
+                p.ids[static_cast<size_t>(t) * p.k + j] = sel_e[j];
+                p.w[static_cast<size_t>(t) * p.k + j] = z[j] / sum;
+            }
         }
     }
 }
