@@ -140,6 +140,28 @@ moe_status moe_route(const moe_handle* h, const void* x, int T, const float* wr,
 moe_status moe_dispatch(const moe_handle* h, const void* x, const int32_t* ids, int T,
                         void* ws, moe_stream_t stream);
 
+/* moe_dispatch without a workspace.  The pages have no counterpart of this
+ * entry point; it exists for callers that cannot allocate device memory at
+ * all, e.g. a layer running inside a host framework that owns every device
+ * allocation and passes it only input and output buffers.  The dispatch's
+ * only scratch (per-chunk expert counts) lives in a 128 KB array inside this
+ * library that every GPU loading the library holds until the process exits.
+ *   Outputs, all device memory owned by the caller, with A = T*k:
+ *     counts [E], offsets [E+1], num_tiles [1], tiles [A/128 + E + 1][2],
+ *     perm [A], inv [A], xq [A, H] e4m3, xs [A] (FP8_ROW) or [A, H/128]
+ *     (FP8_BLOCK128) fp32, status [2] (zeroed by the call, then status[0] =
+ *     MOE_ERR_DEVICE_BOUNDS if an id was out of range).
+ *   Same results as moe_dispatch.  T*k may not exceed 131072 and the format
+ *   must be FP8 (else MOE_ERR_UNSUPPORTED_SHAPE).  The first call on a device
+ *   looks up the array's device address; make that first call before any
+ *   stream capture.  The array is shared by every call on the device and
+ *   keeps the last call's contents, so calls whose kernels overlap on the GPU
+ *   (other streams, other threads) race: serialise them.  No allocation. */
+moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, const int32_t* ids, int T,
+                                int32_t* counts, int32_t* offsets, int32_t* num_tiles, int32_t* tiles,
+                                int32_t* perm, int32_t* inv, uint8_t* xq, void* xs, int32_t* status,
+                                moe_stream_t stream);
+
 /* Grouped gate+up GEMM over the dispatched rows with SiLU(gate)*up and the
  * requantisation of the hidden fused into its epilogue (pure-Triton article:
  * gate and up share one input tile, SiLU in registers; LightMoE README: gated

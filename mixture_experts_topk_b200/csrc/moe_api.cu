@@ -508,3 +508,84 @@ extern "C" moe_status moe_get_status(const moe_handle* h, void* ws, moe_stream_t
     if (s[0] == MOE_ERR_DEVICE_BOUNDS) return fail(MOE_ERR_DEVICE_BOUNDS, "index out of range in %s", wn);
     return fail(static_cast<moe_status>(s[0]), "device error %d in %s", s[0], wn);
 }
+
+// ------------------------------------------------------------------ dispatch without a workspace
+// For callers that cannot allocate device memory at all: a service whose host
+// framework owns every device allocation and hands the layer only its input
+// and output buffers, so there is nowhere to put a caller-sized workspace.
+// The only scratch the dispatch needs, the per-chunk expert counts, lives in
+// this file-scope device array instead: at most 128 chunks of 1024
+// assignments x 256 experts = 128 KB.  Every GPU that loads this library holds
+// it until the process exits.
+constexpr int NOALLOC_MAX_CHUNKS = 131072 / DISPATCH_CHUNK;
+constexpr int NOALLOC_SCRATCH_INTS = NOALLOC_MAX_CHUNKS * 256;
+static __device__ __align__(256) int32_t g_dispatch_scratch[NOALLOC_SCRATCH_INTS];
+
+// Device address of g_dispatch_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+static moe_status dispatch_scratch(int32_t** out) {
+    static std::mutex mu;
+    static int32_t* addr[64] = {nullptr};
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(MOE_ERR_CUDA, "moe_dispatch_noalloc: device index %d out of range", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        CUDA_TRY(cudaGetSymbolAddress(&p, g_dispatch_scratch));
+        addr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = addr[dev];
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, const int32_t* ids, int T,
+                                           int32_t* counts, int32_t* offsets, int32_t* num_tiles, int32_t* tiles,
+                                           int32_t* perm, int32_t* inv, uint8_t* xq, void* xs, int32_t* status,
+                                           moe_stream_t stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: null handle");
+    const moe_config& c = h->cfg;
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: T=%d is negative", T);
+    const long long A = static_cast<long long>(T) * c.k;
+    const long long nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
+    if (nchunks * c.E > NOALLOC_SCRATCH_INTS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "moe_dispatch_noalloc: T*k=%lld assignments need %lld scratch counts, more than the %d "
+                    "this library holds (at most 131072 assignments with 256 experts)",
+                    A, nchunks * c.E, NOALLOC_SCRATCH_INTS);
+    if (c.fmt == MOE_FMT_NVFP4)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_dispatch_noalloc: NVFP4 is not supported");
+    if (!counts || !offsets || !num_tiles || !tiles || !status)
+        return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: null output");
+    if (A > 0 && (!x || !ids || !perm || !inv || !xq || !xs))
+        return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: null argument");
+    if (A > 0 && (!aligned256(x) || !aligned256(xq)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: x and xq must be 256-byte aligned");
+    int32_t* chunk = nullptr;
+    moe_status r = dispatch_scratch(&chunk);
+    if (r != MOE_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), st));
+    const int n = static_cast<int>(nchunks), a = static_cast<int>(A);
+    // the histogram writes every count of every chunk it covers, so the
+    // scratch left by an earlier call needs no clearing
+    if (a > 0) {
+        hist_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, status);
+        LAUNCH_CHECK("hist_kernel");
+    }
+    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles);
+    LAUNCH_CHECK("scan_kernel");
+    if (a == 0) return MOE_OK;
+    rank_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, perm, inv);
+    LAUNCH_CHECK("rank_kernel");
+    const int qgrid = std::min((T + 7) / 8, 8 * h->num_sms);
+    if (c.fmt == MOE_FMT_FP8_ROW)
+        quant_scatter_kernel<0><<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, inv, xq,
+                                                       static_cast<float*>(xs));
+    else
+        quant_scatter_kernel<1><<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, inv, xq,
+                                                       static_cast<float*>(xs));
+    LAUNCH_CHECK("quant_scatter_kernel");
+    return MOE_OK;
+}

@@ -22,7 +22,7 @@ EXPORTED = (
     "moe_last_error", "moe_init", "moe_destroy", "moe_weights_size", "moe_workspace_size",
     "moe_workspace_view_get", "moe_pack_weights", "moe_route", "moe_dispatch", "moe_gate_up",
     "moe_down", "moe_combine", "moe_forward", "moe_forward_routed", "moe_workspace_init",
-    "moe_get_status",
+    "moe_get_status", "moe_dispatch_noalloc",
 )
 
 
@@ -80,6 +80,7 @@ def load(path=LIB_PATH):
             "moe_forward_routed": (I, [P, P, I, P, P, P, P, P, P]),
             "moe_workspace_init": (I, [P, P, P]),
             "moe_get_status": (I, [P, P, P]),
+            "moe_dispatch_noalloc": (I, [P, P, P, I] + [P] * 10),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -170,6 +171,15 @@ def moe_forward(h, x, T, wr, bias, packed, y, ws, stream=None):
 def moe_forward_routed(h, x, T, ids, w, packed, y, ws, stream=None):
     _check(load().moe_forward_routed(h, _ptr(x), T, _ptr(ids), _ptr(w), _ptr(packed), _ptr(y), _ptr(ws),
                                      _stream(stream)))
+
+
+def moe_dispatch_noalloc(h, x, ids, T, counts, offsets, num_tiles, tiles, perm, inv, xq, xs, status,
+                         stream=None):
+    """moe_dispatch with caller-given outputs and no workspace (for callers that
+    cannot allocate device memory; the scratch is inside the library)."""
+    _check(load().moe_dispatch_noalloc(h, _ptr(x), _ptr(ids), T, _ptr(counts), _ptr(offsets), _ptr(num_tiles),
+                                       _ptr(tiles), _ptr(perm), _ptr(inv), _ptr(xq), _ptr(xs), _ptr(status),
+                                       _stream(stream)))
 
 
 def moe_workspace_init(h, ws, stream=None):
