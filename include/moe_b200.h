@@ -93,6 +93,7 @@ typedef struct {
     int32_t* counts;     /* [E] assignments per expert */
     int32_t* offsets;    /* [E+1] exclusive prefix sum of counts (m_indptr) */
     int32_t* num_tiles;  /* [1] row tiles of 128 over all experts */
+    int32_t* tile_ptr;   /* [E+1] index of each expert's first row tile */
     int32_t* tiles;      /* [A/128 + E + 1][2] (expert, first row) per row tile */
     int32_t* perm;       /* [A] slot -> t*k + j */
     int32_t* inv;        /* [A] t*k + j -> slot */

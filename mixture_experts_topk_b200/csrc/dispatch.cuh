@@ -35,9 +35,11 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
 }
 
 // One CTA: counts, offsets (exclusive scan), per-chunk bases (written over the
-// chunk counts), and the row-tile table (expert, first row) in expert order.
+// chunk counts), the row-tile table (expert, first row) in expert order, and
+// tile_ptr[e] = index of expert e's first row tile (may be null).
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
-                                                   int32_t* offsets, int32_t* tiles, int32_t* num_tiles) {
+                                                   int32_t* offsets, int32_t* tiles, int32_t* num_tiles,
+                                                   int32_t* tile_ptr) {
     __shared__ int s_cnt[256], s_off[257], s_tptr[257];
     const int e = threadIdx.x;
     int c = 0;
@@ -57,11 +59,13 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
         s_tptr[E] = trun;
         offsets[E] = run;
         *num_tiles = trun;
+        if (tile_ptr) tile_ptr[E] = trun;
     }
     __syncthreads();
     if (e < E) {
         counts[e] = c;
         offsets[e] = s_off[e];
+        if (tile_ptr) tile_ptr[e] = s_tptr[e];
         int run = s_off[e];
         for (int ch = 0; ch < nchunks; ch++) {
             const int v = chunk_counts[ch * E + e];

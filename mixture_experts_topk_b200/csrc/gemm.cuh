@@ -15,7 +15,9 @@
 //               into a double-buffered fp32 accumulator in TMEM
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator, scales, SwiGLU and
 //               requantisation (gate/up) or routing weight + fp32 store (down)
-// Tile t of the schedule: m-tile t % ntm (expert e, first row), n-block t / ntm.
+// Tiles are visited expert by expert; inside an expert, n-block-major with the
+// expert's m-tiles fastest, so all readers of one weight tile run at the same
+// time and an expert's rows stay in L2 while its n-blocks go by.
 // A tile's rows past the expert's last row belong to the next expert or are
 // past the end (TMA zero-fills); the epilogue stores only the expert's rows.
 //
@@ -42,6 +44,8 @@ enum { BSCALE_ROW = 0, BSCALE_BLOCK128 = 1 };
 struct GemmParams {
     const int32_t* tiles;       // [ntiles][2] (expert, first row)
     const int32_t* num_tiles;   // number of m-tiles (device scalar)
+    const int32_t* tile_ptr;    // [E+1] first m-tile of each expert
+    int E;
     const int32_t* offsets;     // [E+1]
     int n_blocks;               // N / BN
     int num_kb;                 // K / 128
@@ -73,6 +77,20 @@ struct GemmSmem {
     static constexpr int XCHG_BYTES = 2 * 2 * 128 * 4 * 2;   // [parity][group][row] value + flag
     static constexpr int TOTAL = XCHG_OFF + XCHG_BYTES + 1024; // + alignment slack
 };
+
+// Tile t -> (m-tile index, n-block): expert e owns tiles [tile_ptr[e] nb, tile_ptr[e+1] nb).
+__device__ __forceinline__ void decode_tile(int t, const int32_t* tile_ptr, int E, int n_blocks, int& mi, int& nb) {
+    int lo = 0, hi = E;   // tile_ptr[lo] * n_blocks <= t < tile_ptr[hi] * n_blocks
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(tile_ptr + mid) * n_blocks <= t) lo = mid; else hi = mid;
+    }
+    const int first = __ldg(tile_ptr + lo);
+    const int mt = __ldg(tile_ptr + lo + 1) - first;
+    const int local = t - first * n_blocks;
+    nb = local / mt;
+    mi = first + local % mt;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit) {
     const bool ok = mbar_wait(bar, parity, limit);
@@ -130,7 +148,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const int mi = t % ntm, nb = t / ntm;
+                int mi, nb;
+                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
                 const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
                 const int brow = e * p.b_rows + nb * BN;
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
@@ -205,7 +224,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t u = 0, iter = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, iter++) {
-            const int mi = t % ntm, nb = t / ntm;
+            int mi, nb;
+                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
             const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
             const int row = row0 + r;
             const bool valid = row < p.offsets[e + 1];
@@ -238,13 +258,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     float ag[64], au[64];
 #pragma unroll
                     for (int c = 0; c < 64; c++) ag[c] = au[c] = 0.0f;
+                    const float* arow = p.a_scale + static_cast<size_t>(valid ? row : 0) * p.a_ld;
+                    const float* bsb = p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + 2 * nb) * p.num_kb;
+                    // scales of the next K-block are loaded before waiting on this one
+                    float sa_n = valid ? arow[0] : 0.0f, wg_n = __ldg(bsb), wu_n = __ldg(bsb + p.num_kb);
                     for (int kb = 0; kb < p.num_kb; kb++) {
+                        const float sa = sa_n, sg = sa * wg_n, su = sa * wu_n;
+                        if (kb + 1 < p.num_kb) {
+                            sa_n = valid ? arow[kb + 1] : 0.0f;
+                            wg_n = __ldg(bsb + kb + 1);
+                            wu_n = __ldg(bsb + p.num_kb + kb + 1);
+                        }
                         const uint32_t acc = u & 1;
                         if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
                         tc_fence_after();
-                        const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld + kb] : 0.0f;
-                        const float* bsb = p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + 2 * nb) * p.num_kb;
-                        const float sg = sa * __ldg(bsb + kb), su = sa * __ldg(bsb + p.num_kb + kb);
 #pragma unroll
                         for (int half = 0; half < 2; half++) {
                             float vg[32], vu[32];
@@ -307,13 +334,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < NC; c++) acc_r[c] = 0.0f;
                 const int n0 = nb * BN + g * NC;
+                const float* arow = p.a_scale + static_cast<size_t>(valid ? row : 0) * p.a_ld;
+                const float* bsb = p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + n0 / 128) * p.num_kb;
+                // the scale of the next K-block is loaded before waiting on this one
+                float sa_n = valid ? arow[0] : 0.0f;
+                if (BSCALE == BSCALE_BLOCK128) sa_n *= __ldg(bsb);
                 for (int kb = 0; kb < p.num_kb; kb++) {
+                    const float sa = sa_n;
+                    if (kb + 1 < p.num_kb) {
+                        sa_n = valid ? arow[kb + 1] : 0.0f;
+                        if (BSCALE == BSCALE_BLOCK128) sa_n *= __ldg(bsb + kb + 1);
+                    }
                     const uint32_t acc = u & 1;
                     if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
-                    float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld + kb] : 0.0f;
-                    if (BSCALE == BSCALE_BLOCK128)
-                        sa *= __ldg(p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + n0 / 128) * p.num_kb + kb);
                     if constexpr (NC >= 64) {
 #pragma unroll
                         for (int ch = 0; ch < NC / 64; ch++) {

@@ -48,7 +48,7 @@ extern "C" const char* moe_last_error(void) { return g_err; }
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-    size_t status, ids, w, counts, offsets, num_tiles, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
+    size_t status, ids, w, counts, offsets, num_tiles, tile_ptr, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
 };
 struct WLayout {
     size_t gu_q, gu_s, d_q, d_s, gu_g, d_g, total;
@@ -88,6 +88,7 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.counts = take(c.E * 4);
     L.offsets = take((c.E + 1) * 4);
     L.num_tiles = take(4);
+    L.tile_ptr = take((c.E + 1) * 4);
     L.chunk = take(nchunks * c.E * 4);
     L.tiles = take(tiles_cap * 8);
     L.perm = take(A * 4);
@@ -186,6 +187,7 @@ extern "C" moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_
     v->counts = reinterpret_cast<int32_t*>(b + L.counts);
     v->offsets = reinterpret_cast<int32_t*>(b + L.offsets);
     v->num_tiles = reinterpret_cast<int32_t*>(b + L.num_tiles);
+    v->tile_ptr = reinterpret_cast<int32_t*>(b + L.tile_ptr);
     v->tiles = reinterpret_cast<int32_t*>(b + L.tiles);
     v->perm = reinterpret_cast<int32_t*>(b + L.perm);
     v->inv = reinterpret_cast<int32_t*>(b + L.inv);
@@ -293,7 +295,7 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
         hist_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.status);
         LAUNCH_CHECK("hist_kernel");
     }
-    scan_kernel<<<1, 256, 0, st>>>(chunk, nchunks, c.E, v.counts, v.offsets, v.tiles, v.num_tiles);
+    scan_kernel<<<1, 256, 0, st>>>(chunk, nchunks, c.E, v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr);
     LAUNCH_CHECK("scan_kernel");
     if (A == 0) return MOE_OK;
     rank_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.perm, v.inv);
@@ -380,6 +382,8 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     memset(&p, 0, sizeof(p));
     p.tiles = v.tiles;
     p.num_tiles = v.num_tiles;
+    p.tile_ptr = v.tile_ptr;
+    p.E = c.E;
     p.offsets = v.offsets;
     p.n_blocks = 2 * c.I / 256;
     p.num_kb = c.H / GEMM_BK;
@@ -423,6 +427,8 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     memset(&p, 0, sizeof(p));
     p.tiles = v.tiles;
     p.num_tiles = v.num_tiles;
+    p.tile_ptr = v.tile_ptr;
+    p.E = c.E;
     p.offsets = v.offsets;
     p.n_blocks = c.H / BN;
     p.num_kb = c.I / GEMM_BK;
@@ -574,7 +580,7 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, c
         hist_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, status);
         LAUNCH_CHECK("hist_kernel");
     }
-    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles);
+    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles, nullptr);
     LAUNCH_CHECK("scan_kernel");
     if (a == 0) return MOE_OK;
     rank_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, perm, inv);

@@ -43,7 +43,7 @@ class moe_weights(ctypes.Structure):
                 ("gate_q", "gate_s", "gate_g", "up_q", "up_s", "up_g", "down_q", "down_s", "down_g")]
 
 
-VIEW_FIELDS = ("status", "ids", "w", "counts", "offsets", "num_tiles", "tiles", "perm", "inv",
+VIEW_FIELDS = ("status", "ids", "w", "counts", "offsets", "num_tiles", "tile_ptr", "tiles", "perm", "inv",
                "x_global", "xq", "xs", "hq", "hs", "o")
 
 

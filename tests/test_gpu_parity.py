@@ -119,6 +119,8 @@ def test_dispatch_bit_exact(name):
     assert nt == te.size
     tiles = layer.region("tiles", torch.int32, 2 * nt).cpu().numpy().reshape(nt, 2)
     assert (tiles[:, 0] == te).all() and (tiles[:, 1] == tr).all()
+    tile_ptr = layer.region("tile_ptr", torch.int32, E + 1).cpu().numpy()
+    assert (tile_ptr == np.searchsorted(te, np.arange(E + 1), side="left")).all()
     xq = layer.region("xq", torch.uint8, A * wl.H).cpu().numpy().reshape(A, wl.H)
     assert (xq == ref["xq"]).all()
     if wl.fmt == W.FMT_FP8_ROW:
