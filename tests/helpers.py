@@ -61,6 +61,36 @@ def fp8_values(codes):
     return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
 
 
+def abs_down_weights(wl, weights, slot):
+    """|W_down| of the expert in weight slot `slot`, dequantised with torch's fp8 conversion ([H, I] fp64)."""
+    q = np.asarray(weights["down_q"][slot])
+    s = np.asarray(weights["down_s"][slot], np.float64)
+    v = np.abs(fp8_values(q))
+    if wl.fmt == W.FMT_FP8_ROW:
+        return v * s[:, None]
+    return v * np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)
+
+
+def deviation_bound_rows(wl, weights, slot_of, rows, n_out):
+    """sum over rows (out_index, expert, weight, h_gpu [I], h_ref [I]) of
+    |weight| * |W_down[e]| @ |h_gpu - h_ref|, per output row ([n_out, H])."""
+    extra = np.zeros((n_out, wl.H))
+    cache = {}
+    for i, e, wj, v_gpu, v_ref in rows:
+        dv = np.abs(np.asarray(v_gpu, np.float64) - np.asarray(v_ref, np.float64))
+        if not dv.any():
+            continue
+        if e not in cache:
+            cache[e] = abs_down_weights(wl, weights, slot_of(e))
+        extra[i] += abs(float(wj)) * (cache[e] @ dv)
+    return extra
+
+
+def hidden_values(codes, scales, I):
+    """FP8 hidden codes x their (row, 128-column) scales -> fp64 values."""
+    return fp8_values(codes) * np.repeat(np.asarray(scales, np.float64).reshape(-1), 128)[:I]
+
+
 def hidden_deviation_bound(wl, L, ids, w, ref, hq_gpu, hs_gpu, tokens=None):
     """Largest change of Y that differences between the GPU's and the oracle's
     requantised hidden can cause, per output element:
