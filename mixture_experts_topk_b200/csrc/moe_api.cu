@@ -48,7 +48,7 @@ extern "C" const char* moe_last_error(void) { return g_err; }
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-    size_t status, ids, w, counts, offsets, num_tiles, tile_ptr, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
+    size_t status, ids, w, logits, counts, offsets, num_tiles, tile_ptr, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
 };
 struct WLayout {
     size_t gu_q, gu_s, d_q, d_s, gu_g, d_g, total;
@@ -85,6 +85,7 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.status = take(64 * 4);
     L.ids = take(A * 4);
     L.w = take(A * 4);
+    L.logits = take(static_cast<size_t>(c.max_T) * c.E * 4);
     L.counts = take(c.E * 4);
     L.offsets = take((c.E + 1) * 4);
     L.num_tiles = take(4);
@@ -253,11 +254,12 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
     if (h->cfg.has_bias && !bias) return fail(MOE_ERR_INVALID_ARG, "moe_route: config has a bias but bias is null");
     if (!h->cfg.has_bias) bias = nullptr;
     if (!aligned256(x) || !aligned256(wr)) return fail(MOE_ERR_INVALID_ARG, "moe_route: x and wr must be 256-byte aligned");
-    (void)ws;
+    if (!ws || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_route: ws must be a 256-byte aligned workspace");
     RouterParams p;
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.wr = wr;
     p.bias = bias;
+    p.logits = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + h->ws.logits);
     p.ids = ids;
     p.w = w;
     p.T = T;
@@ -265,12 +267,18 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
     p.E = h->cfg.E;
     p.k = h->cfg.k;
     p.score = h->cfg.score;
-    const int ngroups = (h->cfg.E + 7) / 8;
-    p.token_groups = std::max(1, std::min(8, ROUTER_WARPS / ngroups));
-    const int tokens_per_cta = 8 * p.token_groups;
-    const int grid = (T + tokens_per_cta - 1) / tokens_per_cta;
-    router_topk_kernel<<<grid, ROUTER_WARPS * 32, tokens_per_cta * h->cfg.E * sizeof(float),
-                         reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (h->cfg.E <= 8) {
+        using RT = RouterTile<64, 8>;
+        CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<64, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, RT::SMEM));
+        router_logits_kernel<64, 8><<<dim3((T + 63) / 64, 1), RT_WARPS * 32, RT::SMEM, st>>>(p);
+    } else {
+        using RT = RouterTile<32, 16>;
+        CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<32, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, RT::SMEM));
+        router_logits_kernel<32, 16><<<dim3((T + 31) / 32, (h->cfg.E + 15) / 16), RT_WARPS * 32, RT::SMEM, st>>>(p);
+    }
+    LAUNCH_CHECK("router_logits_kernel");
+    router_topk_kernel<<<std::min((T + 7) / 8, 16 * h->num_sms), 256, 0, st>>>(p);
     LAUNCH_CHECK("router_topk_kernel");
     return MOE_OK;
 }
