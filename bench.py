@@ -132,6 +132,8 @@ def run_ours(args, rank, world, local_rank):
     T = args.tokens
     d = synth.layer(wl, seed=0, device=dev)
     layer = native.Layer(wl, d, max_T=T, device=dev)
+    if args.down_bn:
+        native.moe_set_tile_config(layer.h, args.down_bn)
     wr = d["wr"]
     bias = d["bias"]
     del d                      # the packed copy is all the layer reads
@@ -150,6 +152,8 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {msg}")
     counts = layer.region("counts", torch.int32, wl.E).cpu().numpy()
+    m_tiles = int(layer.region("num_tiles", torch.int32, 1).item())
+    pick = int(layer.region("pick", torch.int32, 1).item())
 
     def barrier():
         if world > 1:
@@ -260,7 +264,9 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"{wl.name} T={T}", "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
                    "T_per_gpu": T, "parallelism": f"replicas x{world} (token batches)",
                    "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (byts / 1e9),
-                   "touched_experts": touched},
+                   "touched_experts": touched, "m_tiles": m_tiles,
+                   "down_tile": args.down_bn or {0: 256, 1: 128, 2: 64}[pick],
+                   "down_tile_source": "fixed" if args.down_bn else "picked from the histogram"},
         "tflops": (fl_t + fl_r) * world * args.steps / (ms_max * 1e-3) / 1e12,
         "layer_roofline": {"t_roof_ms": t_roof_ms, "frac": t_roof_ms / step_ms,
                            "peaks": f"{pk_kind}: fp8 = 2 x bf16_tflops_sustained, hbm_gbs"},
@@ -334,6 +340,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-sample", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--down-bn", type=int, default=0, help="down GEMM tile width (0 = chosen per call)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

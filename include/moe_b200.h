@@ -94,6 +94,7 @@ typedef struct {
     int32_t* offsets;    /* [E+1] exclusive prefix sum of counts (m_indptr) */
     int32_t* num_tiles;  /* [1] row tiles of 128 over all experts */
     int32_t* tile_ptr;   /* [E+1] index of each expert's first row tile */
+    int32_t* pick;       /* [1] down GEMM tile chosen from the histogram: 0 -> 256, 1 -> 128, 2 -> 64 columns */
     int32_t* tiles;      /* [A/128 + E + 1][2] (expert, first row) per row tile */
     int32_t* perm;       /* [A] slot -> t*k + j */
     int32_t* inv;        /* [A] t*k + j -> slot */
@@ -175,6 +176,24 @@ moe_status moe_gate_up(const moe_handle* h, const void* packed, int T, void* ws,
  * w [T, k] fp32 (may be view.w).  Reads hq/hs, writes o. */
 moe_status moe_down(const moe_handle* h, const void* packed, const float* w, int T,
                     void* ws, moe_stream_t stream);
+
+/* Explicit tile choice of the down GEMM (LightMoE README, "Grouped GEMM": tile
+ * choices stay explicit because the fastest geometry depends on the shape and
+ * the expert assignment distribution).  down_bn: 0 = chosen per call, or 64,
+ * 128, 256 output columns per tile.  Host state only. */
+moe_status moe_set_tile_config(moe_handle* h, int down_bn);
+
+/* Parameters of the wave cost model that picks the down GEMM's tile width
+ * from the runtime expert histogram (RaMP abstract: four-parameter wave cost
+ * model fitted from a one-time profiling sweep).  The dispatch's scan kernel
+ * evaluates, for BN in {256, 128, 64}, with m_tiles = sum_e ceil(count_e/128):
+ *   t_mma  = ceil(m_tiles*(H/BN) / num_sms) * (I/128) * (alpha + beta*BN)
+ *   t_load = touched_experts*H*I*1e6 / (min(m_tiles*(H/BN), num_sms) * bw)
+ *   cost   = gamma + max(t_mma, t_load)     (integers: picoseconds, bytes/us)
+ * and writes the cheapest (the wider on ties) to view.pick.
+ * params = {alpha, beta, bw, gamma}; get also returns num_sms in params[4]. */
+moe_status moe_set_picker_params(moe_handle* h, const long long* params);
+moe_status moe_get_picker_params(const moe_handle* h, long long* params);
 
 /* Deterministic combine (LightMoE README, "Highlights": deterministic
  * combine): y[t] = bf16( sum_{j=0..k-1} o[inv[t k + j]] ) in fixed j order,

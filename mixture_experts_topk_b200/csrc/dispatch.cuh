@@ -19,6 +19,46 @@ namespace moe {
 constexpr int DISPATCH_CHUNK = 1024;
 constexpr int TILE_M = 128;
 
+// Wave cost model of the down GEMM's tile width (RaMP abstract: a
+// four-parameter wave cost model picks the configuration from the runtime
+// expert histogram and depends only on the CTA grid geometry).  Integer
+// picoseconds, so the choice is exact and reproducible.  For candidate c with
+// BN_c output columns per tile:
+//   tiles  = m_tiles * (H / BN_c)
+//   t_mma  = ceil(tiles / num_sms) * (I / 128) * (alpha + beta * BN_c)
+//   t_load = touched_experts * H * I / (min(tiles, num_sms) * bw_cta)   (weight bytes)
+//   cost   = gamma + max(t_mma, t_load)
+// The lowest cost wins; equal costs keep the wider tile.
+struct PickerParams {
+    long long alpha_ps;        // per K-block fixed cost of a tile
+    long long beta_ps;         // per K-block cost per output column
+    long long bw_cta;          // weight bytes per microsecond one CTA streams
+    long long gamma_ps;        // launch constant
+    int num_sms, H, I;
+};
+constexpr int PICK_NUM = 3;
+__host__ __device__ constexpr int pick_bn(int c) { return c == 0 ? 256 : (c == 1 ? 128 : 64); }
+
+__device__ __forceinline__ int pick_down_tile(const PickerParams& q, int m_tiles, int touched) {
+    int best = 0;
+    long long best_cost = 0;
+    for (int c = 0; c < PICK_NUM; c++) {
+        const long long bn = pick_bn(c);
+        const long long tiles = static_cast<long long>(m_tiles) * (q.H / bn);
+        const long long waves = (tiles + q.num_sms - 1) / q.num_sms;
+        const long long t_mma = waves * (q.I / 128) * (q.alpha_ps + q.beta_ps * bn);
+        const long long active = tiles < q.num_sms ? tiles : q.num_sms;
+        const long long bytes = static_cast<long long>(touched) * q.H * q.I;
+        const long long t_load = active > 0 ? bytes * 1000000LL / (active * q.bw_cta) : 0;
+        const long long cost = q.gamma_ps + (t_mma > t_load ? t_mma : t_load);
+        if (c == 0 || cost < best_cost) {
+            best = c;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
 __global__ void __launch_bounds__(DISPATCH_CHUNK)
     hist_kernel(const int32_t* ids, int A, int E, int32_t* chunk_counts, int32_t* status) {
     __shared__ int h[256];
@@ -36,10 +76,11 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
 
 // One CTA: counts, offsets (exclusive scan), per-chunk bases (written over the
 // chunk counts), the row-tile table (expert, first row) in expert order, and
-// tile_ptr[e] = index of expert e's first row tile (may be null).
+// tile_ptr[e] = index of expert e's first row tile (may be null), and the down
+// GEMM's tile choice from the histogram (pick_out, may be null).
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
                                                    int32_t* offsets, int32_t* tiles, int32_t* num_tiles,
-                                                   int32_t* tile_ptr) {
+                                                   int32_t* tile_ptr, int32_t* pick_out, PickerParams pq) {
     __shared__ int s_cnt[256], s_off[257], s_tptr[257];
     const int e = threadIdx.x;
     int c = 0;
@@ -60,6 +101,11 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
         offsets[E] = run;
         *num_tiles = trun;
         if (tile_ptr) tile_ptr[E] = trun;
+        if (pick_out) {
+            int touched = 0;
+            for (int i = 0; i < E; i++) touched += s_cnt[i] > 0;
+            pick_out[0] = pick_down_tile(pq, trun, touched);
+        }
     }
     __syncthreads();
     if (e < E) {

@@ -12,7 +12,8 @@
 //   warp 0      TMA producer: A tile [128 rows x 128 K] + B tile [BN rows x 128 K]
 //               per stage into a STAGES-deep shared-memory ring (128-byte swizzle)
 //   warp 1      allocates TMEM, one thread issues tcgen05.mma (M=128, N=BN, K=32)
-//               into a double-buffered fp32 accumulator in TMEM
+//               into a ring of NBUF fp32 accumulators in TMEM (2 for BN=256,
+//               4 for narrower tiles)
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator, scales, SwiGLU and
 //               requantisation (gate/up) or routing weight + fp32 store (down)
 // Tiles are visited expert by expert; inside an expert, n-block-major with the
@@ -66,12 +67,15 @@ struct GemmParams {
 
 template <int BN, int STAGES>
 struct GemmSmem {
+    // accumulator buffers in TMEM (512 columns): deeper for narrower tiles, so the
+    // MMA can run further ahead of a per-K-block epilogue
+    static constexpr int NBUF = (512 / BN) < 4 ? (512 / BN) : 4;
     static constexpr int B_BYTES = BN * GEMM_BK;
     static constexpr int STAGE_BYTES = GEMM_A_BYTES + B_BYTES;
     static constexpr int TILES_BYTES = STAGES * STAGE_BYTES;
     // after the tiles: barriers, TMEM address, amax exchange
     static constexpr int BAR_OFF = TILES_BYTES;
-    static constexpr int NUM_BARS = 2 * STAGES + 5;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
     static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int XCHG_OFF = (TMEM_SLOT_OFF + 4 + 15) / 16 * 16;
     static constexpr int XCHG_BYTES = 2 * 2 * 128 * 4 * 2;   // [parity][group][row] value + flag
@@ -98,31 +102,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
 }
 
 template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmParams p) {
+__device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
+                                          const int n_blocks, uint8_t* smem_raw) {
     using S = GemmSmem<BN, STAGES>;
-    extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
+    constexpr int NBUF = S::NBUF;
     uint64_t* tfull = bars + 2 * STAGES;
-    uint64_t* tempty = bars + 2 * STAGES + 2;
-    uint64_t* drain = bars + 2 * STAGES + 4;
+    uint64_t* tempty = bars + 2 * STAGES + NBUF;
+    uint64_t* drain = bars + 2 * STAGES + 2 * NBUF;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::TMEM_SLOT_OFF);
     float* xval = reinterpret_cast<float*>(smem + S::XCHG_OFF);                 // [2][2][128]
     int* xflag = reinterpret_cast<int*>(smem + S::XCHG_OFF + 2 * 2 * 128 * 4);  // [2][2][128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr uint32_t TMEM_COLS = 2 * BN;
+    constexpr uint32_t TMEM_COLS = NBUF * BN;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; b++) {
+        for (int b = 0; b < NBUF; b++) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 8);   // one arrival per epilogue warp
         }
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const int ntm = *p.num_tiles;
-    const int total = ntm * p.n_blocks;
+    const int total = ntm * n_blocks;
     const long long limit = p.spin_limit;
 
     if (warp == 0) {
@@ -149,7 +152,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 int mi, nb;
-                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
+                decode_tile(t, p.tile_ptr, p.E, n_blocks, mi, nb);
                 const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
                 const int brow = e * p.b_rows + nb * BN;
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
@@ -178,14 +181,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 uint32_t acc = 0;
                 if (!PROMOTE) {
-                    acc = u & 1;
-                    if (!mbar_wait(&tempty[acc], ((u >> 1) & 1) ^ 1, limit)) { ok = false; break; }
+                    acc = u % NBUF;
+                    if (!mbar_wait(&tempty[acc], ((u / NBUF) & 1) ^ 1, limit)) { ok = false; break; }
                     tc_fence_after();
                 }
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
                     if (PROMOTE) {
-                        acc = u & 1;
-                        if (!mbar_wait(&tempty[acc], ((u >> 1) & 1) ^ 1, limit)) { ok = false; break; }
+                        acc = u % NBUF;
+                        if (!mbar_wait(&tempty[acc], ((u / NBUF) & 1) ^ 1, limit)) { ok = false; break; }
                         tc_fence_after();
                     }
                     const int s = it % STAGES;
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, iter++) {
             int mi, nb;
-                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
+                decode_tile(t, p.tile_ptr, p.E, n_blocks, mi, nb);
             const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
             const int row = row0 + r;
             const bool valid = row < p.offsets[e + 1];
@@ -233,8 +236,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (KIND == KIND_GATE_UP) {
                 float hv[64];
                 if (!PROMOTE) {
-                    const uint32_t acc = u & 1;
-                    if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
+                    const uint32_t acc = u % NBUF;
+                    if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
                     const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld] : 0.0f;
                     const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + nb * BN;
@@ -269,8 +272,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                             wg_n = __ldg(bsb + kb + 1);
                             wu_n = __ldg(bsb + p.num_kb + kb + 1);
                         }
-                        const uint32_t acc = u & 1;
-                        if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
+                        const uint32_t acc = u % NBUF;
+                        if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int half = 0; half < 2; half++) {
@@ -345,8 +348,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         sa_n = valid ? arow[kb + 1] : 0.0f;
                         if (BSCALE == BSCALE_BLOCK128) sa_n *= __ldg(bsb + kb + 1);
                     }
-                    const uint32_t acc = u & 1;
-                    if (!warp_wait(&tfull[acc], (u >> 1) & 1, limit)) { ok = false; break; }
+                    const uint32_t acc = u % NBUF;
+                    if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
                     if constexpr (NC >= 64) {
 #pragma unroll
@@ -399,6 +402,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
+}
+
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    gemm_body<KIND, BSCALE, PROMOTE, BN, STAGES>(tmA, tmB, p, p.n_blocks, smem_raw);
+}
+
+// Down GEMM whose tile width is chosen on the device: the dispatch's scan
+// kernel evaluates the wave cost model on the expert histogram and writes the
+// choice (0: BN=256, 1: 128, 2: 64) to *cfg; every CTA reads it and runs that
+// tile body with the matching weight tensor map.  No host round trip.
+constexpr int POLY_SMEM = GemmSmem<256, 4>::TOTAL > GemmSmem<128, 6>::TOTAL
+                              ? (GemmSmem<256, 4>::TOTAL > GemmSmem<64, 8>::TOTAL ? GemmSmem<256, 4>::TOTAL
+                                                                                 : GemmSmem<64, 8>::TOTAL)
+                              : (GemmSmem<128, 6>::TOTAL > GemmSmem<64, 8>::TOTAL ? GemmSmem<128, 6>::TOTAL
+                                                                                 : GemmSmem<64, 8>::TOTAL);
+
+template <int BSCALE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    down_gemm_poly_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB256,
+                          const __grid_constant__ CUtensorMap tmB128, const __grid_constant__ CUtensorMap tmB64,
+                          const GemmParams p, const int32_t* cfg) {
+    extern __shared__ uint8_t smem_raw[];
+    const int c = *cfg;
+    if (c == 1)
+        gemm_body<KIND_DOWN, BSCALE, true, 128, 6>(tmA, tmB128, p, p.H / 128, smem_raw);
+    else if (c == 2)
+        gemm_body<KIND_DOWN, BSCALE, true, 64, 8>(tmA, tmB64, p, p.H / 64, smem_raw);
+    else
+        gemm_body<KIND_DOWN, BSCALE, true, 256, 4>(tmA, tmB256, p, p.H / 256, smem_raw);
 }
 
 }  // namespace moe

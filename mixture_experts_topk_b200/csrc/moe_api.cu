@@ -48,7 +48,7 @@ extern "C" const char* moe_last_error(void) { return g_err; }
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-    size_t status, ids, w, logits, counts, offsets, num_tiles, tile_ptr, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
+    size_t status, ids, w, logits, counts, offsets, num_tiles, tile_ptr, pick, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
 };
 struct WLayout {
     size_t gu_q, gu_s, d_q, d_s, gu_g, d_g, total;
@@ -61,6 +61,8 @@ struct moe_handle {
     WsLayout ws;
     WLayout wl;
     long long spin_limit;
+    int down_bn;          // 0 = picked per call, else 64 / 128 / 256
+    PickerParams picker;
 };
 
 static size_t code_bytes(int fmt, int K) { return fmt == MOE_FMT_NVFP4 ? K / 2 : K; }
@@ -90,6 +92,7 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.offsets = take((c.E + 1) * 4);
     L.num_tiles = take(4);
     L.tile_ptr = take((c.E + 1) * 4);
+    L.pick = take(4);
     L.chunk = take(nchunks * c.E * 4);
     L.tiles = take(tiles_cap * 8);
     L.perm = take(A * 4);
@@ -157,6 +160,14 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
     h->ws = make_ws_layout(c);
     h->wl = make_w_layout(c);
     h->spin_limit = 2000000000LL;   // ~1 s of SM clock per wait
+    h->down_bn = 0;
+    h->picker.alpha_ps = 334419;       // least-squares fit to a B200 tile sweep
+    h->picker.beta_ps = 2114;
+    h->picker.bw_cta = 38684;
+    h->picker.gamma_ps = 17030139;
+    h->picker.num_sms = h->num_sms;
+    h->picker.H = c.H;
+    h->picker.I = c.I;
     *out = h;
     return MOE_OK;
 }
@@ -189,6 +200,7 @@ extern "C" moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_
     v->offsets = reinterpret_cast<int32_t*>(b + L.offsets);
     v->num_tiles = reinterpret_cast<int32_t*>(b + L.num_tiles);
     v->tile_ptr = reinterpret_cast<int32_t*>(b + L.tile_ptr);
+    v->pick = reinterpret_cast<int32_t*>(b + L.pick);
     v->tiles = reinterpret_cast<int32_t*>(b + L.tiles);
     v->perm = reinterpret_cast<int32_t*>(b + L.perm);
     v->inv = reinterpret_cast<int32_t*>(b + L.inv);
@@ -303,7 +315,8 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
         hist_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.status);
         LAUNCH_CHECK("hist_kernel");
     }
-    scan_kernel<<<1, 256, 0, st>>>(chunk, nchunks, c.E, v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr);
+    scan_kernel<<<1, 256, 0, st>>>(chunk, nchunks, c.E, v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr,
+                                   v.pick, h->picker);
     LAUNCH_CHECK("scan_kernel");
     if (A == 0) return MOE_OK;
     rank_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.perm, v.inv);
@@ -425,8 +438,8 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     moe_workspace_view_get(h, ws, &v);
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
-    constexpr int BN = 256;
-    CUtensorMap ta, tb;
+    const int BN = h->down_bn ? h->down_bn : 256;
+    CUtensorMap ta, tb, tb128, tb64;
     moe_status r = make_tmap(&ta, v.hq, c.I, A, c.I, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
     r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, BN);
@@ -451,10 +464,65 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     p.route_w = w;
     p.status = v.status;
     p.spin_limit = h->spin_limit;
-    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_DOWN, BSCALE_ROW, true, BN, 4>(ta, tb, p, grid, st);
-    return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, BN, 4>(ta, tb, p, grid, st);
+    if (h->down_bn == 0) {
+        // tile width chosen on the device from the histogram (scan kernel)
+        r = make_tmap(&tb128, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, 128);
+        if (r != MOE_OK) return r;
+        r = make_tmap(&tb64, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, 64);
+        if (r != MOE_OK) return r;
+        const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * (c.H / 64)));
+        if (c.fmt == MOE_FMT_FP8_ROW) {
+            CUDA_TRY(cudaFuncSetAttribute(down_gemm_poly_kernel<BSCALE_ROW>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, POLY_SMEM));
+            down_gemm_poly_kernel<BSCALE_ROW><<<grid, GEMM_THREADS, POLY_SMEM, st>>>(ta, tb, tb128, tb64, p, v.pick);
+        } else {
+            CUDA_TRY(cudaFuncSetAttribute(down_gemm_poly_kernel<BSCALE_BLOCK128>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, POLY_SMEM));
+            down_gemm_poly_kernel<BSCALE_BLOCK128><<<grid, GEMM_THREADS, POLY_SMEM, st>>>(ta, tb, tb128, tb64, p,
+                                                                                         v.pick);
+        }
+        LAUNCH_CHECK("down_gemm_poly_kernel");
+        return MOE_OK;
+    }
+    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
+    if (c.fmt == MOE_FMT_FP8_ROW) {
+        if (BN == 256) return launch_gemm<KIND_DOWN, BSCALE_ROW, true, 256, 4>(ta, tb, p, grid, st);
+        if (BN == 128) return launch_gemm<KIND_DOWN, BSCALE_ROW, true, 128, 6>(ta, tb, p, grid, st);
+        return launch_gemm<KIND_DOWN, BSCALE_ROW, true, 64, 8>(ta, tb, p, grid, st);
+    }
+    if (BN == 256) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 256, 4>(ta, tb, p, grid, st);
+    if (BN == 128) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 128, 6>(ta, tb, p, grid, st);
+    return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 64, 8>(ta, tb, p, grid, st);
+}
+
+extern "C" moe_status moe_set_picker_params(moe_handle* h, const long long* params) {
+    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_set_picker_params: null argument");
+    if (params[0] < 0 || params[1] < 0 || params[2] <= 0 || params[3] < 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_picker_params: need alpha, beta, gamma >= 0 and bw > 0");
+    h->picker.alpha_ps = params[0];
+    h->picker.beta_ps = params[1];
+    h->picker.bw_cta = params[2];
+    h->picker.gamma_ps = params[3];
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_get_picker_params(const moe_handle* h, long long* params) {
+    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_get_picker_params: null argument");
+    params[0] = h->picker.alpha_ps;
+    params[1] = h->picker.beta_ps;
+    params[2] = h->picker.bw_cta;
+    params[3] = h->picker.gamma_ps;
+    params[4] = h->picker.num_sms;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_set_tile_config(moe_handle* h, int down_bn) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_tile_config: null handle");
+    if (down_bn != 0 && down_bn != 64 && down_bn != 128 && down_bn != 256)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_tile_config: down_bn must be 0, 64, 128 or 256 (got %d)", down_bn);
+    h->down_bn = down_bn;
+    return MOE_OK;
 }
 
 // ------------------------------------------------------------------ combine
@@ -588,7 +656,7 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, c
         hist_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, status);
         LAUNCH_CHECK("hist_kernel");
     }
-    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles, nullptr);
+    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles, nullptr, nullptr, h->picker);
     LAUNCH_CHECK("scan_kernel");
     if (a == 0) return MOE_OK;
     rank_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, perm, inv);

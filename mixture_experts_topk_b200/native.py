@@ -22,7 +22,8 @@ EXPORTED = (
     "moe_last_error", "moe_init", "moe_destroy", "moe_weights_size", "moe_workspace_size",
     "moe_workspace_view_get", "moe_pack_weights", "moe_route", "moe_dispatch", "moe_gate_up",
     "moe_down", "moe_combine", "moe_forward", "moe_forward_routed", "moe_workspace_init",
-    "moe_get_status", "moe_dispatch_noalloc",
+    "moe_get_status", "moe_dispatch_noalloc", "moe_set_tile_config", "moe_set_picker_params",
+    "moe_get_picker_params",
 )
 
 
@@ -43,7 +44,7 @@ class moe_weights(ctypes.Structure):
                 ("gate_q", "gate_s", "gate_g", "up_q", "up_s", "up_g", "down_q", "down_s", "down_g")]
 
 
-VIEW_FIELDS = ("status", "ids", "w", "counts", "offsets", "num_tiles", "tile_ptr", "tiles", "perm", "inv",
+VIEW_FIELDS = ("status", "ids", "w", "counts", "offsets", "num_tiles", "tile_ptr", "pick", "tiles", "perm", "inv",
                "x_global", "xq", "xs", "hq", "hs", "o")
 
 
@@ -81,6 +82,9 @@ def load(path=LIB_PATH):
             "moe_workspace_init": (I, [P, P, P]),
             "moe_get_status": (I, [P, P, P]),
             "moe_dispatch_noalloc": (I, [P, P, P, I] + [P] * 10),
+            "moe_set_tile_config": (I, [P, I]),
+            "moe_set_picker_params": (I, [P, P]),
+            "moe_get_picker_params": (I, [P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -180,6 +184,22 @@ def moe_dispatch_noalloc(h, x, ids, T, counts, offsets, num_tiles, tiles, perm, 
     _check(load().moe_dispatch_noalloc(h, _ptr(x), _ptr(ids), T, _ptr(counts), _ptr(offsets), _ptr(num_tiles),
                                        _ptr(tiles), _ptr(perm), _ptr(inv), _ptr(xq), _ptr(xs), _ptr(status),
                                        _stream(stream)))
+
+
+def moe_set_tile_config(h, down_bn):
+    _check(load().moe_set_tile_config(h, int(down_bn)))
+
+
+def moe_set_picker_params(h, alpha, beta, bw, gamma):
+    arr = (ctypes.c_longlong * 4)(alpha, beta, bw, gamma)
+    _check(load().moe_set_picker_params(h, arr))
+
+
+def moe_get_picker_params(h):
+    """-> (alpha, beta, bw, gamma, num_sms)"""
+    arr = (ctypes.c_longlong * 5)()
+    _check(load().moe_get_picker_params(h, arr))
+    return tuple(arr)
 
 
 def moe_workspace_init(h, ws, stream=None):

@@ -72,6 +72,7 @@ def lib():
             "orc_down_rows": (None, [P, I, I, P, P, P]),
             "orc_moe_forward": (I, [P, P, I, P, P, I, P, P, P, P]),
             "orc_num_threads": (I, []),
+            "orc_pick_down_tile": (I, [P, I, I, I, I, I64, I64, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -169,6 +170,15 @@ def schedule(offsets):
     tr = np.empty(cap, np.int32)
     n = lib().orc_schedule(_p(offsets), E, _p(te), _p(tr))
     return te[:n].copy(), tr[:n].copy()
+
+
+# ---------------------------------------------------------------- tile choice
+def pick_down_tile(counts, H, I, num_sms, alpha, beta, bw, gamma):
+    """Down GEMM tile choice from the expert histogram -> (candidate, [cost per candidate])."""
+    counts = _c(counts, np.int32)
+    costs = np.empty(3, np.int64)
+    c = lib().orc_pick_down_tile(_p(counts), counts.size, H, I, num_sms, alpha, beta, bw, gamma, _p(costs))
+    return c, costs
 
 
 # ---------------------------------------------------------------- quantisers

@@ -209,6 +209,31 @@ int orc_schedule(const int32_t* offsets, int E, int32_t* tile_expert, int32_t* t
     return n;
 }
 
+/* ------------------------------------------------------- down tile choice */
+
+int orc_pick_down_tile(const int32_t* counts, int E, int H, int I, int num_sms,
+                       int64_t alpha, int64_t beta, int64_t bw, int64_t gamma, int64_t* costs)
+{
+    int64_t m_tiles = 0, touched = 0;
+    for (int e = 0; e < E; e++) {
+        m_tiles += (counts[e] + ORC_TILE_M - 1) / ORC_TILE_M;
+        touched += counts[e] > 0;
+    }
+    const int64_t bn_of[3] = {256, 128, 64};
+    int best = 0;
+    for (int c = 0; c < 3; c++) {
+        int64_t bn = bn_of[c];
+        int64_t tiles = m_tiles * (H / bn);
+        int64_t waves = (tiles + num_sms - 1) / num_sms;
+        int64_t t_mma = waves * (I / 128) * (alpha + beta * bn);
+        int64_t active = tiles < num_sms ? tiles : num_sms;
+        int64_t t_load = active > 0 ? touched * H * I * 1000000LL / (active * bw) : 0;
+        costs[c] = gamma + (t_mma > t_load ? t_mma : t_load);
+        if (costs[c] < costs[best]) best = c;
+    }
+    return best;
+}
+
 /* ------------------------------------------------ activation quantisation */
 
 float orc_nvfp4_global(const float* x, int64_t n)

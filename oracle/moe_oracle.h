@@ -70,6 +70,19 @@ void orc_dispatch(const int32_t* ids, int T, int k, int E, int32_t* counts,
                   int32_t* offsets, int32_t* perm, int32_t* inv);
 int  orc_schedule(const int32_t* offsets, int E, int32_t* tile_expert, int32_t* tile_row);
 
+/* ---- down GEMM tile choice (wave cost model over the expert histogram) ----
+ * RaMP abstract: a four-parameter wave cost model selects the configuration
+ * from the runtime expert histogram and depends only on the CTA grid geometry.
+ * Candidates c = 0, 1, 2 have BN = 256, 128, 64 output columns per tile.  With
+ * m_tiles = sum_e ceil(counts[e]/128) and touched = #{e : counts[e] > 0}:
+ *   tiles  = m_tiles * (H / BN)
+ *   t_mma  = ceil(tiles / num_sms) * (I / 128) * (alpha + beta * BN)
+ *   t_load = touched * H * I * 1e6 / (min(tiles, num_sms) * bw)   (0 if no tiles)
+ *   cost   = gamma + max(t_mma, t_load)           (all integer; / truncates)
+ * Returns the c of the lowest cost, the lower c on equal costs. */
+int orc_pick_down_tile(const int32_t* counts, int E, int H, int I, int num_sms,
+                       int64_t alpha, int64_t beta, int64_t bw, int64_t gamma, int64_t* costs);
+
 /* ---- activation quantisation of token rows (X or the hidden) ----
  * FP8_ROW:      one fp32 scale per row: s = fp32(amax/448), q = e4m3(fp32(x/s)),
  *               q = 0 when s == 0.  scales: [rows]

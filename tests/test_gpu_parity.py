@@ -121,6 +121,9 @@ def test_dispatch_bit_exact(name):
     assert (tiles[:, 0] == te).all() and (tiles[:, 1] == tr).all()
     tile_ptr = layer.region("tile_ptr", torch.int32, E + 1).cpu().numpy()
     assert (tile_ptr == np.searchsorted(te, np.arange(E + 1), side="left")).all()
+    a, b, bw, g, sms = native.moe_get_picker_params(layer.h)
+    want, _ = oracle.pick_down_tile(counts, wl.H, wl.I, sms, a, b, bw, g)
+    assert int(layer.region("pick", torch.int32, 1).cpu().numpy()[0]) == want
     xq = layer.region("xq", torch.uint8, A * wl.H).cpu().numpy().reshape(A, wl.H)
     assert (xq == ref["xq"]).all()
     if wl.fmt == W.FMT_FP8_ROW:
@@ -160,9 +163,11 @@ def test_gate_up_hidden_matches_oracle(name):
     assert np.all(np.abs(v_gpu - v_ref) <= np.abs(v_ref) * 0.125 + 2.0 ** -9)
 
 
+@pytest.mark.parametrize("down_bn", [0, 64, 128, 256])
 @pytest.mark.parametrize("name", list(CASES))
-def test_down_matches_oracle_on_oracle_hidden(name):
+def test_down_matches_oracle_on_oracle_hidden(name, down_bn):
     wl, T, d, x, layer, ids, w, ref = _dispatch_and_reference(name)
+    native.moe_set_tile_config(layer.h, down_bn)
     A = T * wl.k
     layer.region("hq", torch.uint8, A * wl.I).copy_(torch.from_numpy(ref["hq"].reshape(-1)).cuda())
     layer.region("hs", torch.float32, A * wl.I // 128).copy_(torch.from_numpy(ref["hs"].reshape(-1)).cuda())

@@ -228,3 +228,31 @@ def test_fp8_quant_error_bound(fmt):
     cb = codes.reshape(8, nb, -1)
     at_max = np.take_along_axis(cb, xb.argmax(axis=2)[..., None], axis=2)[..., 0]
     assert ((at_max & 0x7F) == 0x7E).all()
+
+
+# ------------------------------------------------------------------ tile choice
+def test_pick_down_tile_hand_example():
+    # one token on one Mixtral-shaped expert: 1 m-tile, H/BN n-blocks, one wave
+    P = dict(H=4096, I=14336, num_sms=148, alpha=240000, beta=2200, bw=60000, gamma=5000)
+    c, costs = oracle.pick_down_tile(np.int32([1, 0]), **P)
+    # BN=256: 112 K-blocks x (240000 + 256*2200) = 89958400 > load 61166933
+    # BN=128: 112 x (240000 + 128*2200) = 58419200;  BN=64: 112 x 380800 = 42649600
+    assert list(costs) == [5000 + 89958400, 5000 + 58419200, 5000 + 42649600]
+    assert c == 2
+    # no assignments: every cost is gamma, the widest tile wins the tie
+    c, costs = oracle.pick_down_tile(np.zeros(8, np.int32), **P)
+    assert c == 0 and list(costs) == [5000, 5000, 5000]
+
+
+def test_pick_down_tile_load_term_and_waves():
+    P = dict(H=2048, I=512, num_sms=4, alpha=0, beta=0, bw=1000, gamma=0)
+    # beta = alpha = 0: only the load term counts; more active CTAs -> cheaper
+    c, costs = oracle.pick_down_tile(np.int32([5]), **P)
+    # m_tiles 1: tiles 8 / 16 / 32, all capped at 4 active CTAs -> equal -> widest
+    load = 1 * 2048 * 512 * 1000000 // (4 * 1000)
+    assert list(costs) == [load] * 3 and c == 0
+    P.update(alpha=100, num_sms=1000)
+    c, costs = oracle.pick_down_tile(np.int32([5]), **P)
+    # one wave each, t_mma = 4 x 100 everywhere; load shrinks with more tiles
+    loads = [1 * 2048 * 512 * 1000000 // (t * 1000) for t in (8, 16, 32)]
+    assert list(costs) == [max(400, l) for l in loads] and c == 2
