@@ -272,4 +272,118 @@ __global__ void interleave_rows_kernel(const uint32_t* gate, const uint32_t* up,
     }
 }
 
+
+// ------------------------------------------------------------------ NVFP4
+// LightMoE README ("Standalone GEMM", "MoE inference"): NVFP4 = packed E2M1
+// values, E4M3 scale factors per 16 elements, one fp32 scale per tensor; the
+// layer quantises its BF16 input itself.
+//
+// Global scale of X: g = amax(|X|) / (448 * 6).  amax as the bit pattern of a
+// non-negative float, so an integer max gives the float max (order-free).
+__global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* x, long long n8, int32_t* amax_bits) {
+    float m = 0.0f;
+    for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n8; i += 256LL * gridDim.x) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; q++) m = fmaxf(m, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_int(m));
+}
+
+// Byte offset of scale factor (row, column c = K index / 16) in the chunked
+// layout the tensor cores read: per 128-row tile, per 4 scale columns, 512
+// bytes with row r of the tile at (r % 32) * 16 + (r / 32) * 4 + c % 4.
+__host__ __device__ __forceinline__ size_t sf_offset(long long row, int c, int sf_cols) {
+    const long long tile = row >> 7;
+    const int r = static_cast<int>(row & 127);
+    return (static_cast<size_t>(tile) * (sf_cols >> 2) + (c >> 2)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (c & 3);
+}
+
+// NVFP4 quantisation of X rows, scattered to the rows of the assignments in the
+// 128-padded expert-major layout: assignment slot s of expert e goes to row
+// tile_ptr[e] * 128 + (s - offsets[e]).  Per 16-block: sb = e4m3((amax/6)/g),
+// d = value(sb) * g, q = e2m1(x / d) (all correctly rounded fp32; q = 0 when
+// d == 0).  One warp per token; lane l holds columns 256 i + 8 l .. +8, so a
+// 16-block is lanes (l, l^1).
+__global__ void __launch_bounds__(256) quant_scatter_nvfp4_kernel(
+    const __nv_bfloat16* x, int T, int H, int k, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
+    const int32_t* tile_ptr, const int32_t* amax_bits, uint8_t* xq, uint8_t* xsf) {
+    const int lane = threadIdx.x & 31;
+    const int nI = H >> 8;
+    const float g = __fdiv_rn(__int_as_float(*amax_bits), 2688.0f);
+    for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+        long long prow[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            prow[j] = -1;
+            if (j < k) {
+                const int s = inv[static_cast<size_t>(t) * k + j];
+                const int e = ids[static_cast<size_t>(t) * k + j];
+                if (s >= 0) prow[j] = static_cast<long long>(tile_ptr[e]) * 128 + (s - offsets[e]);
+            }
+        }
+        const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
+        for (int i = 0; i < nI; i++) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + 256 * i + 8 * lane));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            float f[8];
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                f[2 * q] = bf16_lo(u[q]);
+                f[2 * q + 1] = bf16_hi(u[q]);
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 8; q++) amax = fmaxf(amax, fabsf(f[q]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            uint8_t sb = 0;
+            float d = 0.0f;
+            if (g > 0.0f) {
+                sb = f_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+                d = __fmul_rn(e4m3_to_f(sb), g);
+            }
+            uint32_t packed = 0;
+            if (d != 0.0f) {
+#pragma unroll
+                for (int q = 0; q < 4; q++)
+                    packed |= static_cast<uint32_t>(f2_to_e2m1x2(__fdiv_rn(f[2 * q], d), __fdiv_rn(f[2 * q + 1], d)))
+                              << (8 * q);
+            }
+            const int c = 16 * i + (lane >> 1);   // scale column of this lane's block
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (prow[j] < 0) continue;
+                *reinterpret_cast<uint32_t*>(xq + prow[j] * (H / 2) + 128 * i + 4 * lane) = packed;
+                if ((lane & 1) == 0) xsf[sf_offset(prow[j], c, H / 16)] = sb;
+            }
+        }
+    }
+}
+
+// Scale factors of weights [E][rows][K/16] e4m3 -> the chunked layout per
+// expert (rows a multiple of 128).  With `interleave` the destination row R of
+// expert e takes source row (R / 2G) G + R % 2G of gate (R % 2G < G) or up.
+__global__ void pack_sf_kernel(const uint8_t* gate, const uint8_t* up, uint8_t* dst, int E, int rows_per_proj,
+                               int G, int sf_cols, int interleave) {
+    const int dst_rows = interleave ? 2 * rows_per_proj : rows_per_proj;
+    const long long total = static_cast<long long>(E) * dst_rows * sf_cols;
+    for (long long i = blockIdx.x * 256LL + threadIdx.x; i < total; i += 256LL * gridDim.x) {
+        const int c = static_cast<int>(i % sf_cols);
+        const long long er = i / sf_cols;
+        const int e = static_cast<int>(er / dst_rows), R = static_cast<int>(er % dst_rows);
+        const uint8_t* src = gate;
+        int sr = R;
+        if (interleave) {
+            const int grp = R / (2 * G), within = R % (2 * G);
+            src = within < G ? gate : up;
+            sr = grp * G + (within < G ? within : within - G);
+        }
+        const uint8_t v = src[(static_cast<long long>(e) * rows_per_proj + sr) * sf_cols + c];
+        dst[static_cast<size_t>(e) * dst_rows * sf_cols + sf_offset(R, c, sf_cols)] = v;
+    }
+}
+
 }  // namespace moe

@@ -1,0 +1,267 @@
+// gemm_fp4.cuh -- persistent grouped NVFP4 GEMM on the 5th-gen tensor cores
+// (tcgen05.mma kind::mxf4nvf4, E4M3 scale factor per 16 elements of K applied
+// by the hardware) with the two epilogues of the MoE expert MLP.
+//
+// LightMoE README ("Standalone GEMM", "MoE inference"): NVFP4 operands are
+// packed E2M1 values with blocked E4M3 scale factors and one fp32 per-tensor
+// scale; one layer call does gate/up, the gated activation, NVFP4
+// requantisation of the hidden, the down projection and the routing weight.
+// Pure-Triton fused MoE article: gate and up share one input tile.
+//
+// Tile 128 rows x 128 columns (gate/up: 64 gate + 64 up columns of one 64-wide
+// hidden block), K stage 256 values = 128 bytes per row, 6 stages.  Per stage
+// the producer brings, on one mbarrier: A and B tiles by TMA (128-byte swizzle)
+// and the 2 KB of A and 2 KB of B scale factors (4 chunks of 512 B, one per
+// MMA of K = 64) by plain bulk copies.  The MMA thread copies the chunks into a
+// TMEM ring (tcgen05.cp, 32 rows x 16 B repeated over the 4 lane quadrants),
+// then issues the 4 block-scaled MMAs, which read them in issue order.
+// TMEM: two 128-column accumulators at [0, 256), scale-factor ring at 256 +.
+//
+// Rows are in the 128-padded expert-major layout (m-tile i = rows 128 i ..),
+// so each tile's scale factors are whole chunks.  The epilogue maps a padded
+// row back to its assignment slot (offsets) for the outputs indexed by slot.
+#pragma once
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+
+constexpr int F4_BN = 128;
+constexpr int F4_STAGES = 6;
+constexpr int F4_A_BYTES = 128 * 128;
+constexpr int F4_B_BYTES = F4_BN * 128;
+constexpr int F4_SF_BYTES = 2048;                 // 4 chunks of 512 B
+constexpr int F4_STAGE_BYTES = F4_A_BYTES + F4_B_BYTES + 2 * F4_SF_BYTES;
+constexpr int F4_NBUF = 2;
+constexpr int F4_SF_TMEM = F4_NBUF * F4_BN;       // first column of the scale-factor ring
+constexpr int F4_BAR_OFF = F4_STAGES * F4_STAGE_BYTES;
+constexpr int F4_NUM_BARS = 2 * F4_STAGES + 2 * F4_NBUF + 1;
+constexpr int F4_TMEM_SLOT_OFF = F4_BAR_OFF + 8 * F4_NUM_BARS;
+constexpr int F4_SMEM = F4_TMEM_SLOT_OFF + 16 + 1024;
+static_assert(F4_SF_TMEM + 32 * F4_STAGES <= 512, "TMEM columns");
+
+struct Fp4Params {
+    const int32_t* tiles;
+    const int32_t* num_tiles;
+    const int32_t* tile_ptr;
+    const int32_t* offsets;
+    int E;
+    int n_blocks;             // N / 128
+    int num_kb;               // K / 256
+    int sf_cols;              // K / 16
+    int b_rows;               // rows of B per expert (2I for gate/up, H for down)
+    const uint8_t* sfa;       // activation scale factors, chunked by padded row tile
+    const uint8_t* sfb;       // weight scale factors, chunked per expert
+    const int32_t* x_amax;    // gate/up: amax bits of X (global scale = amax / 2688)
+    const float* w_global;    // gate/up: [E][2] (gate, up); down: [E]
+    float h_global;           // static hidden scale
+    uint8_t* hq;              // gate/up out: hidden codes [rows][I/2], scale factors hsf
+    uint8_t* hsf;
+    int I;
+    float* o;                 // down out: [A][H] fp32 rows in slot order
+    int H;
+    const int32_t* perm;
+    const float* route_w;
+    int32_t* status;
+    long long spin_limit;
+};
+
+template <int KIND>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    grouped_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                            const Fp4Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F4_BAR_OFF);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + F4_STAGES;
+    uint64_t* tfull = bars + 2 * F4_STAGES;
+    uint64_t* tempty = bars + 2 * F4_STAGES + F4_NBUF;
+    uint64_t* drain = bars + 2 * F4_STAGES + 2 * F4_NBUF;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F4_TMEM_SLOT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < F4_STAGES; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < F4_NBUF; b++) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int ntm = *p.num_tiles;
+    const int total = ntm * p.n_blocks;
+    const long long limit = p.spin_limit;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                int mi, nb;
+                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
+                const int e = p.tiles[2 * mi];
+                const int brow = e * p.b_rows + nb * F4_BN;
+                const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.sf_cols * 128;
+                const uint8_t* sfb = p.sfb + static_cast<size_t>(e) * p.b_rows * p.sf_cols +
+                                     static_cast<size_t>(nb) * p.sf_cols * 128;
+                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                    const int s = it % F4_STAGES;
+                    if (!mbar_wait(&empty[s], ((it / F4_STAGES) & 1) ^ 1, limit)) {
+                        report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + s * F4_STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], F4_STAGE_BYTES);
+                    tma_load_2d(st, &tmA, &full[s], kb * 128, mi * 128);
+                    tma_load_2d(st + F4_A_BYTES, &tmB, &full[s], kb * 128, brow);
+                    bulk_load(st + F4_A_BYTES + F4_B_BYTES, sfa + kb * F4_SF_BYTES, F4_SF_BYTES, &full[s]);
+                    bulk_load(st + F4_A_BYTES + F4_B_BYTES + F4_SF_BYTES, sfb + kb * F4_SF_BYTES, F4_SF_BYTES,
+                              &full[s]);
+                }
+            }
+            const uint32_t first = it > F4_STAGES ? it - F4_STAGES : 0;
+            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % F4_STAGES], (j / F4_STAGES) & 1, limit);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_nvf4(128, F4_BN);
+            uint32_t it = 0, u = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const uint32_t acc = u % F4_NBUF;
+                if (!mbar_wait(&tempty[acc], ((u / F4_NBUF) & 1) ^ 1, limit)) { ok = false; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                    const int s = it % F4_STAGES;
+                    if (!mbar_wait(&full[s], (it / F4_STAGES) & 1, limit)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * F4_STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + F4_A_BYTES;
+                    const uint32_t sfa_addr = b_addr + F4_B_BYTES;
+                    const uint32_t sfb_addr = sfa_addr + F4_SF_BYTES;
+                    const uint32_t sf_col = tmem_base + F4_SF_TMEM + 32 * s;
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        tmem_cp_32x128b_x4(sf_col + 4 * j, sdesc_sf_chunk(sfa_addr + 512 * j));
+                        tmem_cp_32x128b_x4(sf_col + 16 + 4 * j, sdesc_sf_chunk(sfb_addr + 512 * j));
+                    }
+                    const uint32_t d = tmem_base + acc * F4_BN;
+#pragma unroll
+                    for (int j = 0; j < 4; j++)
+                        mma_nvf4(d, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j), idesc, sf_col + 4 * j,
+                                 sf_col + 16 + 4 * j, (kb > 0 || j > 0));
+                    mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                u++;
+            }
+            if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
+            mma_commit(drain);
+            mbar_wait(drain, 0, limit);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int g = (warp - 2) >> 2;           // column group: 32 (gate/up) or 64 (down) columns
+        const int r = 32 * q + lane;
+        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+        uint32_t u = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int mi, nb;
+            decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
+            const int e = p.tiles[2 * mi];
+            const long long prow = static_cast<long long>(mi) * 128 + r;
+            const int local = static_cast<int>(prow - static_cast<long long>(p.tile_ptr[e]) * 128);
+            const bool valid = local < p.offsets[e + 1] - p.offsets[e];
+            const uint32_t acc = u % F4_NBUF;
+            if (!warp_wait(&tfull[acc], (u / F4_NBUF) & 1, limit)) { ok = false; break; }
+            tc_fence_after();
+            if (KIND == KIND_GATE_UP) {
+                float gv[32], uv[32];
+                tmem_ld32x2(lane_addr + acc * F4_BN + 32 * g, lane_addr + acc * F4_BN + 64 + 32 * g, gv, uv);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+                u++;
+                const float gx = __fdiv_rn(__int_as_float(*p.x_amax), 2688.0f);
+                const float sg = gx * __ldg(p.w_global + 2 * e), su = gx * __ldg(p.w_global + 2 * e + 1);
+                float hv[32];
+#pragma unroll
+                for (int c = 0; c < 32; c++) {
+                    const float gg = gv[c] * sg, uu = uv[c] * su;
+                    hv[c] = gg / (1.0f + expf(-gg)) * uu;
+                }
+                if (valid) {
+                    const int col0 = nb * 64 + 32 * g;      // first hidden column of this thread
+                    uint32_t w[4];
+#pragma unroll
+                    for (int b = 0; b < 2; b++) {           // two 16-blocks
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int c = 0; c < 16; c++) amax = fmaxf(amax, fabsf(hv[16 * b + c]));
+                        const uint8_t sb = f_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), p.h_global));
+                        const float d = __fmul_rn(e4m3_to_f(sb), p.h_global);
+#pragma unroll
+                        for (int c = 0; c < 16; c += 8) {
+                            uint32_t pk = 0;
+                            if (d != 0.0f) {
+#pragma unroll
+                                for (int i = 0; i < 4; i++)
+                                    pk |= static_cast<uint32_t>(f2_to_e2m1x2(__fdiv_rn(hv[16 * b + c + 2 * i], d),
+                                                                              __fdiv_rn(hv[16 * b + c + 2 * i + 1], d)))
+                                          << (8 * i);
+                            }
+                            w[2 * b + c / 8] = pk;
+                        }
+                        p.hsf[sf_offset(prow, col0 / 16 + b, p.I / 16)] = sb;
+                    }
+                    *reinterpret_cast<uint4*>(p.hq + prow * (p.I / 2) + col0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            } else {
+                float v0[32], v1[32];
+                tmem_ld32x2(lane_addr + acc * F4_BN + 64 * g, lane_addr + acc * F4_BN + 64 * g + 32, v0, v1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+                u++;
+                if (valid) {
+                    const int slot = p.offsets[e] + local;
+                    const float sc = p.h_global * __ldg(p.w_global + e) * p.route_w[p.perm[slot]];
+                    float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + 64 * g);
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        dst[c / 4] = make_float4(v0[c] * sc, v0[c + 1] * sc, v0[c + 2] * sc, v0[c + 3] * sc);
+                        dst[8 + c / 4] = make_float4(v1[c] * sc, v1[c + 1] * sc, v1[c + 2] * sc, v1[c + 3] * sc);
+                    }
+                }
+            }
+        }
+        if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_EPILOGUE);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace moe

@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "dispatch.cuh"
 #include "gemm.cuh"
+#include "gemm_fp4.cuh"
 #include "router.cuh"
 
 using namespace moe;
@@ -72,6 +73,10 @@ static size_t act_scale_bytes(int fmt, int K) {
     return K / 16;
 }
 static size_t hidden_scale_bytes(int fmt, int I) { return fmt == MOE_FMT_NVFP4 ? I / 16 : 4 * (I / 128); }
+static size_t padded_rows(const moe_config& c) {
+    const size_t A = static_cast<size_t>(c.max_T) * c.k;
+    return c.fmt == MOE_FMT_NVFP4 ? A + static_cast<size_t>(TILE_M) * c.E : A;
+}
 
 static WsLayout make_ws_layout(const moe_config& c) {
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
@@ -98,10 +103,13 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.perm = take(A * 4);
     L.inv = take(A * 4);
     L.xglobal = take(16);
-    L.xq = take(A * code_bytes(c.fmt, c.H));
-    L.xs = take(A * act_scale_bytes(c.fmt, c.H));
-    L.hq = take(A * code_bytes(c.fmt, c.I));
-    L.hs = take(A * hidden_scale_bytes(c.fmt, c.I));
+    // NVFP4 rows are padded to 128 per expert, so each row tile owns whole
+    // scale-factor chunks
+    const size_t R = (c.fmt == MOE_FMT_NVFP4) ? A + static_cast<size_t>(TILE_M) * c.E : A;
+    L.xq = take(R * code_bytes(c.fmt, c.H));
+    L.xs = take(R * act_scale_bytes(c.fmt, c.H));
+    L.hq = take(R * code_bytes(c.fmt, c.I));
+    L.hs = take(R * hidden_scale_bytes(c.fmt, c.I));
     L.o = take(A * c.H * 4);
     L.total = off;
     return L;
@@ -150,8 +158,10 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: need 1 <= k <= 8, k <= E <= 256 (E=%d k=%d)", c.E, c.k);
     if (static_cast<long long>(c.max_T) * c.k > 131072)
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: max_T * k must be <= 131072");
-    if (c.fmt == MOE_FMT_NVFP4)
-        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: the NVFP4 format is not built in this library yet");
+    if (c.fmt == MOE_FMT_NVFP4 && c.I % 256 != 0)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: NVFP4 needs I to be a multiple of 256 (I=%d)", c.I);
+    if (c.fmt == MOE_FMT_NVFP4 && !(c.hidden_global_scale > 0.0f))
+        return fail(MOE_ERR_INVALID_ARG, "moe_init: NVFP4 needs a positive hidden_global_scale");
     moe_handle* h = new (std::nothrow) moe_handle;
     if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_init: out of host memory");
     h->cfg = c;
@@ -231,6 +241,29 @@ extern "C" moe_status moe_pack_weights(const moe_handle* h, const moe_weights* s
     uint8_t* b = static_cast<uint8_t*>(packed);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int grid = 4 * h->num_sms;
+    if (c.fmt == MOE_FMT_NVFP4) {
+        if (!src->gate_g || !src->up_g || !src->down_g)
+            return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: NVFP4 needs the global scales");
+        // gate/up interleaved in 64-row groups (a 128-row tile = 64 gate + 64 up)
+        interleave_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(src->gate_q),
+                                                     static_cast<const uint32_t*>(src->up_q),
+                                                     reinterpret_cast<uint32_t*>(b + h->wl.gu_q), c.E, c.I, 64, c.H / 8);
+        LAUNCH_CHECK("interleave_rows_kernel(nvfp4 codes)");
+        pack_sf_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(src->gate_s),
+                                             static_cast<const uint8_t*>(src->up_s), b + h->wl.gu_s, c.E, c.I, 64,
+                                             c.H / 16, 1);
+        LAUNCH_CHECK("pack_sf_kernel(gate/up)");
+        pack_sf_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(src->down_s), nullptr, b + h->wl.d_s, c.E,
+                                             c.H, 0, c.I / 16, 0);
+        LAUNCH_CHECK("pack_sf_kernel(down)");
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_q, src->down_q, static_cast<size_t>(c.E) * c.H * (c.I / 2),
+                                 cudaMemcpyDeviceToDevice, st));
+        CUDA_TRY(cudaMemcpy2DAsync(b + h->wl.gu_g, 8, src->gate_g, 4, 4, c.E, cudaMemcpyDeviceToDevice, st));
+        CUDA_TRY(cudaMemcpy2DAsync(b + h->wl.gu_g + 4, 8, src->up_g, 4, 4, c.E, cudaMemcpyDeviceToDevice, st));
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_g, src->down_g, static_cast<size_t>(c.E) * 4, cudaMemcpyDeviceToDevice,
+                                 st));
+        return MOE_OK;
+    }
     interleave_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(src->gate_q),
                                                  static_cast<const uint32_t*>(src->up_q),
                                                  reinterpret_cast<uint32_t*>(b + h->wl.gu_q), c.E, c.I, 128,
@@ -322,6 +355,19 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
     rank_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.perm, v.inv);
     LAUNCH_CHECK("rank_kernel");
     const int qgrid = std::min((T + 7) / 8, 8 * h->num_sms);
+    if (c.fmt == MOE_FMT_NVFP4) {
+        int32_t* amax = reinterpret_cast<int32_t*>(v.x_global);
+        CUDA_TRY(cudaMemsetAsync(amax, 0, sizeof(int32_t), st));
+        const long long n8 = static_cast<long long>(T) * c.H / 8;
+        amax_kernel<<<static_cast<int>(std::min<long long>((n8 + 255) / 256, 4LL * h->num_sms)), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), n8, amax);
+        LAUNCH_CHECK("amax_kernel");
+        quant_scatter_nvfp4_kernel<<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, ids,
+                                                          v.inv, v.offsets, v.tile_ptr, amax, v.xq,
+                                                          static_cast<uint8_t*>(v.xs));
+        LAUNCH_CHECK("quant_scatter_nvfp4_kernel");
+        return MOE_OK;
+    }
     if (c.fmt == MOE_FMT_FP8_ROW)
         quant_scatter_kernel<0><<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, v.inv, v.xq,
                                                        static_cast<float*>(v.xs));
@@ -330,6 +376,66 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
                                                        static_cast<float*>(v.xs));
     LAUNCH_CHECK("quant_scatter_kernel");
     return MOE_OK;
+}
+
+// ------------------------------------------------------------------ NVFP4 GEMMs
+static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
+                            uint32_t box_inner, uint32_t box_rows);
+static int max_m_tiles(const moe_config& c, int T);
+
+template <int KIND>
+static moe_status launch_fp4(const CUtensorMap& ta, const CUtensorMap& tb, const Fp4Params& p, int grid,
+                             cudaStream_t st) {
+    auto kern = grouped_gemm_fp4_kernel<KIND>;
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F4_SMEM));
+    kern<<<grid, GEMM_THREADS, F4_SMEM, st>>>(ta, tb, p);
+    LAUNCH_CHECK("grouped_gemm_fp4_kernel");
+    return MOE_OK;
+}
+
+static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float* w, int T, void* ws,
+                           moe_stream_t stream, bool gate_up) {
+    const moe_config& c = h->cfg;
+    moe_workspace_view v;
+    moe_workspace_view_get(h, ws, &v);
+    const uint8_t* pw = static_cast<const uint8_t*>(packed);
+    const size_t R = padded_rows(c);
+    const int K = gate_up ? c.H : c.I;
+    const int N = gate_up ? 2 * c.I : c.H;
+    CUtensorMap ta, tb;
+    moe_status r = make_tmap(&ta, gate_up ? v.xq : v.hq, K / 2, R, K / 2, 128, 128);
+    if (r != MOE_OK) return r;
+    r = make_tmap(&tb, pw + (gate_up ? h->wl.gu_q : h->wl.d_q), K / 2, static_cast<uint64_t>(c.E) * N, K / 2, 128,
+                  F4_BN);
+    if (r != MOE_OK) return r;
+    Fp4Params p;
+    memset(&p, 0, sizeof(p));
+    p.tiles = v.tiles;
+    p.num_tiles = v.num_tiles;
+    p.tile_ptr = v.tile_ptr;
+    p.offsets = v.offsets;
+    p.E = c.E;
+    p.n_blocks = N / F4_BN;
+    p.num_kb = K / 256;
+    p.sf_cols = K / 16;
+    p.b_rows = N;
+    p.sfa = static_cast<const uint8_t*>(gate_up ? v.xs : v.hs);
+    p.sfb = pw + (gate_up ? h->wl.gu_s : h->wl.d_s);
+    p.x_amax = reinterpret_cast<const int32_t*>(v.x_global);
+    p.w_global = reinterpret_cast<const float*>(pw + (gate_up ? h->wl.gu_g : h->wl.d_g));
+    p.h_global = c.hidden_global_scale;
+    p.hq = v.hq;
+    p.hsf = static_cast<uint8_t*>(v.hs);
+    p.I = c.I;
+    p.o = v.o;
+    p.H = c.H;
+    p.perm = v.perm;
+    p.route_w = w;
+    p.status = v.status;
+    p.spin_limit = h->spin_limit;
+    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return gate_up ? launch_fp4<KIND_GATE_UP>(ta, tb, p, grid, st) : launch_fp4<KIND_DOWN>(ta, tb, p, grid, st);
 }
 
 // ------------------------------------------------------------------ tensor maps
@@ -388,7 +494,7 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     if (T == 0) return MOE_OK;
     if (!packed || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_gate_up: null argument");
     if (!aligned256(packed) || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_gate_up: pointers must be 256-byte aligned");
-    if (T == 0) return MOE_OK;
+    if (h->cfg.fmt == MOE_FMT_NVFP4) return fp4_gemm(h, packed, nullptr, T, ws, stream, true);
     const moe_config& c = h->cfg;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
@@ -432,7 +538,7 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     if (T == 0) return MOE_OK;
     if (!packed || !ws || !w) return fail(MOE_ERR_INVALID_ARG, "moe_down: null argument");
     if (!aligned256(packed) || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_down: pointers must be 256-byte aligned");
-    if (T == 0) return MOE_OK;
+    if (h->cfg.fmt == MOE_FMT_NVFP4) return fp4_gemm(h, packed, w, T, ws, stream, false);
     const moe_config& c = h->cfg;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);

@@ -91,7 +91,7 @@ def hidden_values(codes, scales, I):
     return fp8_values(codes) * np.repeat(np.asarray(scales, np.float64).reshape(-1), 128)[:I]
 
 
-def hidden_deviation_bound(wl, L, ids, w, ref, hq_gpu, hs_gpu, tokens=None):
+def hidden_deviation_bound(wl, L, ids, w, ref, hq_gpu, hs_gpu, tokens=None, values=None):
     """Largest change of Y that differences between the GPU's and the oracle's
     requantised hidden can cause, per output element:
         sum_j |w_j| sum_n |h_gpu[slot(t,j), n] - h_ref[slot(t,j), n]| |W_down[e_j][m, n]|
@@ -108,8 +108,11 @@ def hidden_deviation_bound(wl, L, ids, w, ref, hq_gpu, hs_gpu, tokens=None):
         for j in range(wl.k):
             e = int(ids[t, j])
             r = int(ref["inv"][t * wl.k + j])
-            v_gpu = fp8_values(hq_gpu[r]) * np.repeat(hs_gpu[r].reshape(nb).astype(np.float64), 128)
-            v_ref = fp8_values(ref["hq"][r]) * np.repeat(ref["hs"][r].reshape(nb).astype(np.float64), 128)
+            if values is not None:
+                v_gpu, v_ref = values[0][r], values[1][r]
+            else:
+                v_gpu = fp8_values(hq_gpu[r]) * np.repeat(hs_gpu[r].reshape(nb).astype(np.float64), 128)
+                v_ref = fp8_values(ref["hq"][r]) * np.repeat(ref["hs"][r].reshape(nb).astype(np.float64), 128)
             dv = np.abs(v_gpu - v_ref)
             if not dv.any():
                 continue
@@ -129,3 +132,47 @@ def tolerance_violations_with_bound(y_gpu, y_ref, extra):
     # bf16 output: the bound gets the final rounding of the moved value too
     slack = extra * (1 + 2.0 ** -8)
     return int((err > tol + slack).sum()), int((err > tol).sum())
+
+
+# ------------------------------------------------------------------ NVFP4 layout
+E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def sf_offset(row, c, sf_cols):
+    """Byte of scale factor (row, column c) in the chunked layout the tensor cores
+    read: per 128-row tile and 4 columns, 512 B, row r at (r%32)*16 + (r//32)*4 + c%4."""
+    row = np.asarray(row, np.int64)
+    c = np.asarray(c, np.int64)
+    r = row % 128
+    return ((row // 128) * (sf_cols // 4) + c // 4) * 512 + (r % 32) * 16 + (r // 32) * 4 + c % 4
+
+
+def padded_rows(slots, ids_flat, perm, offsets, tile_ptr):
+    """128-padded row of each assignment slot: tile_ptr[e]*128 + slot - offsets[e]."""
+    slots = np.asarray(slots, np.int64)
+    e = ids_flat[perm[slots]]
+    return tile_ptr[e].astype(np.int64) * 128 + slots - offsets[e]
+
+
+def gather_sf(buf, rows, sf_cols):
+    """Row-major [len(rows), sf_cols] scale factors out of the chunked layout."""
+    rows = np.asarray(rows, np.int64)
+    cols = np.arange(sf_cols)
+    return buf[sf_offset(rows[:, None], cols[None, :], sf_cols)]
+
+
+def scatter_sf(buf, rows, sf_rm, sf_cols):
+    rows = np.asarray(rows, np.int64)
+    cols = np.arange(sf_cols)
+    buf[sf_offset(rows[:, None], cols[None, :], sf_cols)] = sf_rm
+
+
+def e2m1_values(packed):
+    p = np.ascontiguousarray(packed, np.uint8)
+    nib = np.stack([p & 15, p >> 4], axis=-1).reshape(*p.shape[:-1], p.shape[-1] * 2)
+    mag = E2M1_MAG[nib & 7]
+    return np.where(nib & 8, -mag, mag)
+
+
+def nvfp4_hidden_values(codes, sf_rm, g):
+    return e2m1_values(codes) * np.repeat(fp8_values(sf_rm), 16, axis=-1) * float(g)

@@ -12,8 +12,8 @@ import torch
 
 import oracle
 from mixture_experts_topk_b200 import native, synth, workloads as W
-from helpers import (bits, hidden_deviation_bound, slot_order_reference, tolerance_violations,
-                     tolerance_violations_with_bound)
+from helpers import (bits, fp8_values, gather_sf, hidden_deviation_bound, nvfp4_hidden_values, padded_rows,
+                     scatter_sf, slot_order_reference, tolerance_violations, tolerance_violations_with_bound)
 
 pytestmark = pytest.mark.gpu
 
@@ -24,7 +24,29 @@ CASES = {
     "row-skew-e64": (W.custom(H=256, I=256, E=64, k=8, zipf_s=1.2), 100),
     "block128-ragged": (W.custom(H=512, I=384, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 300),
     "t1": (W.custom(H=256, I=128, E=8, k=2), 1),
+    "nvfp4-ragged": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4), 300),
+    "nvfp4-skew-e32": (W.custom(H=256, I=256, E=32, k=4, fmt=W.FMT_NVFP4, zipf_s=1.0), 50),
 }
+
+
+def nvfp4(wl):
+    return wl.fmt == W.FMT_NVFP4
+
+
+def gpu_slot_rows(layer, wl, ids, T):
+    """Row of each assignment slot in the GPU's X/hidden buffers (padded for NVFP4)."""
+    A = T * wl.k
+    if not nvfp4(wl):
+        return np.arange(A)
+    counts, offsets, perm, inv = oracle.dispatch(ids, wl.E)
+    tile_ptr = layer.region("tile_ptr", torch.int32, wl.E + 1).cpu().numpy()
+    return padded_rows(np.arange(A), ids.reshape(-1), perm, offsets, tile_ptr)
+
+
+def gpu_rows(layer, wl, name, nbytes_per_row):
+    v = layer.view[name] - layer.ws.data_ptr()
+    n = layer.max_T * wl.k + (128 * wl.E if nvfp4(wl) else 0)
+    return layer.ws[v:v + n * nbytes_per_row].cpu().numpy().reshape(n, nbytes_per_row)
 
 
 def build_case(name, seed=0):
@@ -124,12 +146,19 @@ def test_dispatch_bit_exact(name):
     a, b, bw, g, sms = native.moe_get_picker_params(layer.h)
     want, _ = oracle.pick_down_tile(counts, wl.H, wl.I, sms, a, b, bw, g)
     assert int(layer.region("pick", torch.int32, 1).cpu().numpy()[0]) == want
-    xq = layer.region("xq", torch.uint8, A * wl.H).cpu().numpy().reshape(A, wl.H)
-    assert (xq == ref["xq"]).all()
-    if wl.fmt == W.FMT_FP8_ROW:
-        xs = layer.region("xs", torch.float32, A).cpu().numpy()
+    rows = gpu_slot_rows(layer, wl, ids, T)
+    if nvfp4(wl):
+        xq = gpu_rows(layer, wl, "xq", wl.H // 2)[rows]
+        xs = gather_sf(gpu_rows(layer, wl, "xs", wl.H // 16).reshape(-1), rows, wl.H // 16)
+        amax = layer.region("x_global", torch.int32, 1).view(torch.float32).item()
+        assert amax == float(x.float().abs().max())
     else:
-        xs = layer.region("xs", torch.float32, A * wl.H // 128).cpu().numpy().reshape(A, -1)
+        xq = layer.region("xq", torch.uint8, A * wl.H).cpu().numpy().reshape(A, wl.H)
+        if wl.fmt == W.FMT_FP8_ROW:
+            xs = layer.region("xs", torch.float32, A).cpu().numpy()
+        else:
+            xs = layer.region("xs", torch.float32, A * wl.H // 128).cpu().numpy().reshape(A, -1)
+    assert (xq == ref["xq"]).all()
     assert (xs == ref["xs"]).all()
     assert layer.status()[0] == 0
 
@@ -152,6 +181,20 @@ def test_gate_up_hidden_matches_oracle(name):
     torch.cuda.synchronize()
     assert layer.status()[0] == 0
     A = T * wl.k
+    if nvfp4(wl):
+        rows = gpu_slot_rows(layer, wl, ids, T)
+        hq = gpu_rows(layer, wl, "hq", wl.I // 2)[rows]
+        sf = gpu_rows(layer, wl, "hs", wl.I // 16).reshape(-1)
+        hs = gather_sf(sf, rows, wl.I // 16)
+        assert (hs != ref["hs"]).mean() <= 1e-3
+        v_gpu = nvfp4_hidden_values(hq, hs, wl.hidden_global_scale)
+        v_ref = nvfp4_hidden_values(ref["hq"], ref["hs"], wl.hidden_global_scale)
+        mism = v_gpu != v_ref
+        assert mism.mean() <= 2e-3, f"{mism.mean():.2e} of the hidden values differ"
+        # a differing value is one rounding step away: at most a quarter of its 16-block's range
+        step = np.repeat(fp8_values(ref["hs"]), 16, axis=1) * wl.hidden_global_scale * 2.0
+        assert np.all(np.abs(v_gpu - v_ref) <= step * 1.0001)
+        return
     hq = layer.region("hq", torch.uint8, A * wl.I).cpu().numpy().reshape(A, wl.I)
     hs = layer.region("hs", torch.float32, A * wl.I // 128).cpu().numpy().reshape(A, -1)
     np.testing.assert_allclose(hs, ref["hs"], rtol=1e-4, atol=0)
@@ -169,8 +212,21 @@ def test_down_matches_oracle_on_oracle_hidden(name, down_bn):
     wl, T, d, x, layer, ids, w, ref = _dispatch_and_reference(name)
     native.moe_set_tile_config(layer.h, down_bn)
     A = T * wl.k
-    layer.region("hq", torch.uint8, A * wl.I).copy_(torch.from_numpy(ref["hq"].reshape(-1)).cuda())
-    layer.region("hs", torch.float32, A * wl.I // 128).copy_(torch.from_numpy(ref["hs"].reshape(-1)).cuda())
+    if nvfp4(wl):
+        if down_bn not in (0,):
+            pytest.skip("the NVFP4 down GEMM has one tile width")
+        torch.cuda.synchronize()
+        rows = gpu_slot_rows(layer, wl, ids, T)
+        n_rows = layer.max_T * wl.k + 128 * wl.E
+        hq_all = np.zeros((n_rows, wl.I // 2), np.uint8)
+        hq_all[rows] = ref["hq"]
+        sf_all = np.zeros(n_rows * wl.I // 16, np.uint8)
+        scatter_sf(sf_all, rows, ref["hs"], wl.I // 16)
+        layer.region("hq", torch.uint8, hq_all.size).copy_(torch.from_numpy(hq_all.reshape(-1)).cuda())
+        layer.region("hs", torch.uint8, sf_all.size).copy_(torch.from_numpy(sf_all).cuda())
+    else:
+        layer.region("hq", torch.uint8, A * wl.I).copy_(torch.from_numpy(ref["hq"].reshape(-1)).cuda())
+        layer.region("hs", torch.float32, A * wl.I // 128).copy_(torch.from_numpy(ref["hs"].reshape(-1)).cuda())
     w_dev = torch.from_numpy(w.astype(np.float32)).cuda()
     native.moe_down(layer.h, layer.packed, w_dev, T, layer.ws)
     torch.cuda.synchronize()
@@ -195,9 +251,17 @@ def test_forward_end_to_end(name):
     assert (layer.region("ids", torch.int32, T * wl.k).cpu().numpy().reshape(T, wl.k) == ids).all()
     A = T * wl.k
     ref = slot_order_reference(wl, L, x, ids, w)
-    hq = layer.region("hq", torch.uint8, A * wl.I).cpu().numpy().reshape(A, wl.I)
-    hs = layer.region("hs", torch.float32, A * wl.I // 128).cpu().numpy().reshape(A, -1)
-    extra = hidden_deviation_bound(wl, L, ids, w, ref, hq, hs)
+    if nvfp4(wl):
+        rows = gpu_slot_rows(layer, wl, ids, T)
+        hq = gpu_rows(layer, wl, "hq", wl.I // 2)[rows]
+        hs = gather_sf(gpu_rows(layer, wl, "hs", wl.I // 16).reshape(-1), rows, wl.I // 16)
+        v_gpu = nvfp4_hidden_values(hq, hs, wl.hidden_global_scale)
+        v_ref = nvfp4_hidden_values(ref["hq"], ref["hs"], wl.hidden_global_scale)
+        extra = hidden_deviation_bound(wl, L, ids, w, ref, None, None, values=(v_gpu, v_ref))
+    else:
+        hq = layer.region("hq", torch.uint8, A * wl.I).cpu().numpy().reshape(A, wl.I)
+        hs = layer.region("hs", torch.float32, A * wl.I // 128).cpu().numpy().reshape(A, -1)
+        extra = hidden_deviation_bound(wl, L, ids, w, ref, hq, hs)
     bad, plain = tolerance_violations_with_bound(y.float().cpu().numpy(), y_ref, extra)
     assert bad == 0
     assert plain <= 1e-3 * y_ref.size, f"{plain} elements outside the plain tolerance"
