@@ -64,6 +64,9 @@ def fp8_values(codes):
 def abs_down_weights(wl, weights, slot):
     """|W_down| of the expert in weight slot `slot`, dequantised with torch's fp8 conversion ([H, I] fp64)."""
     q = np.asarray(weights["down_q"][slot])
+    if wl.fmt == W.FMT_NVFP4:
+        sb = np.repeat(fp8_values(np.asarray(weights["down_s"][slot])), 16, axis=1)
+        return np.abs(e2m1_values(q)) * sb * float(np.asarray(weights["down_g"])[slot])
     s = np.asarray(weights["down_s"][slot], np.float64)
     v = np.abs(fp8_values(q))
     if wl.fmt == W.FMT_FP8_ROW:

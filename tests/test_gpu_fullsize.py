@@ -12,13 +12,14 @@ import torch
 
 import oracle
 from mixture_experts_topk_b200 import native, synth, workloads as W
-from helpers import bits, deviation_bound_rows, hidden_values, tolerance_violations_with_bound
+from helpers import (bits, deviation_bound_rows, gather_sf, hidden_values, nvfp4_hidden_values, padded_rows,
+                     tolerance_violations_with_bound)
 
 pytestmark = pytest.mark.gpu
 
 CASES = [("mixtral-8x7b", 1, None), ("mixtral-8x7b", 32, None), ("mixtral-8x7b", 4096, 6),
          ("qwen3.5-35b-a3b", 64, 16), ("qwen3.5-35b-a3b", 8192, 8),
-         ("deepseek-v3", 16, 6), ("deepseek-v3", 4096, 4)]
+         ("deepseek-v3", 16, 6), ("deepseek-v3", 4096, 4), ("glm-5.2", 8192, 4)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -66,17 +67,34 @@ def test_full_size_layer(name, T, n_sample):
     _, _, y_ref = L.forward(xb, wr, bias, sel=sel)
 
     # the hidden of every sampled (token, slot): oracle vs GPU, for the bound
-    xq_tok, xs_tok = oracle.quant_rows(wl.fmt, x[torch.from_numpy(sel).long().to(x.device)].float().cpu().numpy())
-    hq_gpu = layer.region("hq", torch.uint8, A * wl.I).view(A, wl.I)
-    hs_gpu = layer.region("hs", torch.float32, A * wl.I // 128).view(A, wl.I // 128)
+    fp4 = wl.fmt == W.FMT_NVFP4
+    x_sel = x[torch.from_numpy(sel).long().to(x.device)].float().cpu().numpy()
+    g_x = oracle.nvfp4_global(x.float().cpu().numpy()) if fp4 else 0.0
+    xq_tok, xs_tok = oracle.quant_rows(wl.fmt, x_sel, g_x)
+    if fp4:
+        tile_ptr = layer.region("tile_ptr", torch.int32, wl.E + 1).cpu().numpy()
+        n_rows = A + 128 * wl.E
+        off = layer.view["hq"] - layer.ws.data_ptr()
+        hq_all = layer.ws[off:off + n_rows * wl.I // 2].view(n_rows, wl.I // 2)
+        off = layer.view["hs"] - layer.ws.data_ptr()
+        hsf_all = layer.ws[off:off + n_rows * wl.I // 16].cpu().numpy()
+    else:
+        hq_gpu = layer.region("hq", torch.uint8, A * wl.I).view(A, wl.I)
+        hs_gpu = layer.region("hs", torch.float32, A * wl.I // 128).view(A, wl.I // 128)
     rows = []
     for i, t in enumerate(sel):
         for j in range(wl.k):
             e = int(ids[t, j])
-            _, hq_r, hs_r, _ = L.expert_rows(e, xq_tok[i:i + 1], xs_tok[i:i + 1])
+            _, hq_r, hs_r, _ = L.expert_rows(e, xq_tok[i:i + 1], xs_tok[i:i + 1], g_x)
             r = int(inv[t * wl.k + j])
-            v_gpu = hidden_values(hq_gpu[r].cpu().numpy(), hs_gpu[r].cpu().numpy(), wl.I)
-            v_ref = hidden_values(hq_r[0], hs_r[0], wl.I)
+            if fp4:
+                prow = int(padded_rows([r], ids.reshape(-1), perm, offsets, tile_ptr)[0])
+                v_gpu = nvfp4_hidden_values(hq_all[prow].cpu().numpy()[None], gather_sf(hsf_all, [prow], wl.I // 16),
+                                            wl.hidden_global_scale)[0]
+                v_ref = nvfp4_hidden_values(hq_r, hs_r, wl.hidden_global_scale)[0]
+            else:
+                v_gpu = hidden_values(hq_gpu[r].cpu().numpy(), hs_gpu[r].cpu().numpy(), wl.I)
+                v_ref = hidden_values(hq_r[0], hs_r[0], wl.I)
             rows.append((i, e, w[t, j], v_gpu, v_ref))
     extra = deviation_bound_rows(wl, sub, lambda e: int(slot[e]), rows, len(sel))
     y_gpu = y[torch.from_numpy(sel).long().cuda()].float().cpu().numpy()
