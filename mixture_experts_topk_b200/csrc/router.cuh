@@ -14,7 +14,7 @@
 //  router_logits_kernel  a 2-D grid of CTA tiles (TOK tokens x EXP experts; 32 x 16,
 //                        or 64 x 8 when E <= 8).
 //                        The 256-wide H chunks of X and Wr go through shared
-//                        memory with double-buffered cp.async; each of the 8
+//                        memory with a 4-stage cp.async pipeline; each of the 8
 //                        warps owns one 8-token x 8-expert micro-tile, so one
 //                        16-byte X read from shared memory feeds 64 fma.
 //  router_topk_kernel    one warp per token: k rounds of a warp argmax over
@@ -32,7 +32,8 @@ struct RouterTile {
     static constexpr int X_BYTES = TOK * 256 * 2;    // 256 bf16 of H per token
     static constexpr int W_BYTES = EXP * 256 * 4;    // 256 fp32 of H per expert
     static constexpr int STAGE = X_BYTES + W_BYTES;
-    static constexpr int SMEM = 2 * STAGE;           // 64 KB (32 x 16) or 80 KB (64 x 8)
+    static constexpr int NSTAGE = 4;                 // 3 chunks in flight hide L2 latency
+    static constexpr int SMEM = NSTAGE * STAGE;      // 128 KB (32 x 16) or 160 KB (64 x 8)
 };
 
 struct RouterParams {
@@ -53,29 +54,62 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool va
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// Load H-chunk i of the tile's X rows and Wr rows into stage buffer `st`.
-// Rows past T or E read nothing and are zero-filled.
-template <int TOK, int EXP>
-__device__ __forceinline__ void router_load_chunk(const RouterParams& p, uint8_t* st, int t0, int e0, int i) {
-    // X: TOK rows x 512 B = TOK * 32 pieces of 16 B
-    for (int q = threadIdx.x; q < TOK * 32; q += blockDim.x) {
-        const int r = q >> 5, c = q & 31;
-        const int t = t0 + r;
-        const bool ok = t < p.T;
-        const __nv_bfloat16* src = p.x + static_cast<size_t>(ok ? t : 0) * p.H + 256 * i + 8 * c;
-        cp_async16(st + r * 512 + c * 16, src, ok);
-    }
-    // Wr: EXP rows x 1024 B = EXP * 64 pieces of 16 B
-    for (int q = threadIdx.x; q < EXP * 64; q += blockDim.x) {
-        const int r = q >> 6, c = q & 63;
-        const int e = e0 + r;
-        const bool ok = e < p.E;
-        const float* src = p.wr + static_cast<size_t>(ok ? e : 0) * p.H + 256 * i + 4 * c;
-        cp_async16(st + RouterTile<TOK, EXP>::X_BYTES + r * 1024 + c * 16, src, ok);
-    }
-    cp_async_commit();
+__device__ __forceinline__ void cp_async_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
+// wait until at most n (0..3, clamped) of this thread's newest groups are pending
+__device__ __forceinline__ void cp_async_wait_le(int n) {
+    if (n >= 3) asm volatile("cp.async.wait_group 3;" ::: "memory");
+    else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
+    else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
+
+// The 16-byte pieces one thread copies for every H chunk: X piece m is row
+// (tid / 32) + 8 m, column 8 (tid % 32); Wr piece m is row (tid / 64) + 4 m,
+// column 4 (tid % 64).  Base pointers and validity are fixed per thread, so a
+// chunk costs one add and one cp.async per piece.  Rows past T or E read
+// nothing and are zero-filled.
+template <int TOK, int EXP>
+struct RouterLoader {
+    static constexpr int XP = TOK * 32 / (RT_WARPS * 32);   // X pieces per thread
+    static constexpr int WP = EXP * 64 / (RT_WARPS * 32);   // Wr pieces per thread
+    const __nv_bfloat16* xb;
+    const float* wb;
+    uint32_t xvalid, wvalid;   // bit m: piece m is inside the tensor
+    int H;
+    uint32_t xdst, wdst;       // shared-memory byte offsets of piece 0
+
+    __device__ __forceinline__ RouterLoader(const RouterParams& p, int t0, int e0) {
+        const int tid = threadIdx.x;
+        H = p.H;
+        xvalid = wvalid = 0;
+        const int xr = tid >> 5, xc = tid & 31;
+        const int wr = tid >> 6, wc = tid & 63;
+#pragma unroll
+        for (int m = 0; m < XP; m++) xvalid |= (t0 + xr + 8 * m < p.T ? 1u : 0u) << m;
+#pragma unroll
+        for (int m = 0; m < WP; m++) wvalid |= (e0 + wr + 4 * m < p.E ? 1u : 0u) << m;
+        xb = p.x + static_cast<size_t>(xvalid & 1u ? t0 + xr : 0) * p.H + 8 * xc;
+        wb = p.wr + static_cast<size_t>(wvalid & 1u ? e0 + wr : 0) * p.H + 4 * wc;
+        xdst = xr * 512 + xc * 16;
+        // Wr piece c holds h = 4c..4c+3, half (c & 1) of lane (c >> 1)'s eight values;
+        // stored at (c & 1) * 512 + (c >> 1) * 16 so each half-read of a warp is
+        // 512 contiguous bytes (no bank conflicts)
+        wdst = RouterTile<TOK, EXP>::X_BYTES + wr * 1024 + (wc & 1) * 512 + (wc >> 1) * 16;
+    }
+    __device__ __forceinline__ void load(uint8_t* st, int i) const {
+#pragma unroll
+        for (int m = 0; m < XP; m++) {
+            const bool ok = (xvalid >> m) & 1u;
+            cp_async16(st + xdst + m * 8 * 512, ok ? xb + static_cast<size_t>(8 * m) * H + 256 * i : xb, ok);
+        }
+#pragma unroll
+        for (int m = 0; m < WP; m++) {
+            const bool ok = (wvalid >> m) & 1u;
+            cp_async16(st + wdst + m * 4 * 1024, ok ? wb + static_cast<size_t>(4 * m) * H + 256 * i : wb, ok);
+        }
+        cp_async_commit();
+    }
+};
 
 template <int TOK, int EXP>
 __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterParams p) {
@@ -92,58 +126,106 @@ __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterPara
 #pragma unroll
         for (int b = 0; b < 8; b++) acc[a][b] = 0.0f;
 
-    router_load_chunk<TOK, EXP>(p, rsm, t0, e0, 0);
+    const RouterLoader<TOK, EXP> ld(p, t0, e0);
+    // prologue: chunks 0 .. NSTAGE-2 in flight
+    for (int c = 0; c < RT::NSTAGE - 1 && c < nI; c++) ld.load(rsm + c * RT::STAGE, c);
     for (int i = 0; i < nI; i++) {
-        uint8_t* st = rsm + (i & 1) * RT::STAGE;
-        if (i + 1 < nI) {
-            router_load_chunk<TOK, EXP>(p, rsm + ((i + 1) & 1) * RT::STAGE, t0, e0, i + 1);
-            cp_async_wait1();
-        } else {
-            cp_async_wait0();
-        }
+        uint8_t* st = rsm + (i % RT::NSTAGE) * RT::STAGE;
+        const int ahead = i + RT::NSTAGE - 1;
+        if (ahead < nI) ld.load(rsm + (ahead % RT::NSTAGE) * RT::STAGE, ahead);
+        // chunk i is complete once at most (issued after it) groups are pending
+        cp_async_wait_le(min(nI - 1 - i, RT::NSTAGE - 1));
         __syncthreads();
         const uint8_t* xs = st + (8 * tg) * 512 + lane * 16;
-        const uint8_t* ws = st + RT::X_BYTES + (8 * eg) * 1024 + lane * 32;
-        uint4 xv[8];
-#pragma unroll
-        for (int tt = 0; tt < 8; tt++) xv[tt] = *reinterpret_cast<const uint4*>(xs + tt * 512);
+        const uint8_t* ws = st + RT::X_BYTES + (8 * eg) * 1024 + lane * 16;
+        // The warp's 8 experts x 8 values and 8 tokens x 8 values of this chunk
+        // sit in registers; for each j the 64 accumulators take one fma each,
+        // so consecutive fma are independent.  Each (token, expert) chain
+        // still runs j = 0..7 in order.
+        float wv[8][8];
 #pragma unroll
         for (int ee = 0; ee < 8; ee++) {
             const float4 wa = *reinterpret_cast<const float4*>(ws + ee * 1024);
-            const float4 wb = *reinterpret_cast<const float4*>(ws + ee * 1024 + 16);
-            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-            for (int tt = 0; tt < 8; tt++) {
-                const uint32_t u[4] = {xv[tt].x, xv[tt].y, xv[tt].z, xv[tt].w};
-#pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    acc[tt][ee] = __fmaf_rn(bf16_lo(u[q]), wv[2 * q], acc[tt][ee]);
-                    acc[tt][ee] = __fmaf_rn(bf16_hi(u[q]), wv[2 * q + 1], acc[tt][ee]);
-                }
-            }
+            const float4 wb = *reinterpret_cast<const float4*>(ws + ee * 1024 + 512);
+            wv[ee][0] = wa.x; wv[ee][1] = wa.y; wv[ee][2] = wa.z; wv[ee][3] = wa.w;
+            wv[ee][4] = wb.x; wv[ee][5] = wb.y; wv[ee][6] = wb.z; wv[ee][7] = wb.w;
         }
-        __syncthreads();   // the stage is refilled two chunks later
+        uint32_t xw[8][4];
+#pragma unroll
+        for (int tt = 0; tt < 8; tt++) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(xs + tt * 512);
+            xw[tt][0] = xv.x; xw[tt][1] = xv.y; xw[tt][2] = xv.z; xw[tt][3] = xv.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            float xj[8];
+#pragma unroll
+            for (int tt = 0; tt < 8; tt++) xj[tt] = (j & 1) ? bf16_hi(xw[tt][j >> 1]) : bf16_lo(xw[tt][j >> 1]);
+#pragma unroll
+            for (int tt = 0; tt < 8; tt++)
+#pragma unroll
+                for (int ee = 0; ee < 8; ee++) acc[tt][ee] = __fmaf_rn(xj[tt], wv[ee][j], acc[tt][ee]);
+        }
+        __syncthreads();   // the stage is refilled NSTAGE-1 chunks later
     }
+    // Sum the 32 lane partials of all 64 (token, expert) pairs by recursive
+    // halving over lane offsets 1, 2, 4, 8, 16: at each step a lane keeps half
+    // of its values and adds the partner's copy of that half, so every sum is
+    // the pairwise tree ((p0+p1)+(p2+p3))+... of the fixed order.  Afterwards
+    // lane l holds pairs 2 r(l) and 2 r(l) + 1, r = 5-bit reversal of l.
+    float* a64 = &acc[0][0];
+    float a32[32], a16[16], a8[8], a4[4], a2[2];
+    {
+        const bool b = lane & 1;
 #pragma unroll
-    for (int tt = 0; tt < 8; tt++)
-#pragma unroll
-        for (int ee = 0; ee < 8; ee++)
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1)
-                acc[tt][ee] = __fadd_rn(acc[tt][ee], __shfl_xor_sync(0xffffffffu, acc[tt][ee], off));
-    // lane (tt * 8 + ee) % 32 writes one logit; each lane holds every sum
-#pragma unroll
-    for (int tt = 0; tt < 8; tt++)
-#pragma unroll
-        for (int ee = 0; ee < 8; ee++) {
-            if (((tt * 8 + ee) & 31) != lane) continue;
-            const int t = t0 + 8 * tg + tt, e = e0 + 8 * eg + ee;
-            if (t < p.T && e < p.E) {
-                float v = acc[tt][ee];
-                if (p.bias) v = __fadd_rn(v, p.bias[e]);
-                p.logits[static_cast<size_t>(t) * p.E + e] = v;
-            }
+        for (int v = 0; v < 32; v++) {
+            const float send = b ? a64[v] : a64[v + 32], keep = b ? a64[v + 32] : a64[v];
+            a32[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 1));
         }
+    }
+    {
+        const bool b = lane & 2;
+#pragma unroll
+        for (int v = 0; v < 16; v++) {
+            const float send = b ? a32[v] : a32[v + 16], keep = b ? a32[v + 16] : a32[v];
+            a16[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+        }
+    }
+    {
+        const bool b = lane & 4;
+#pragma unroll
+        for (int v = 0; v < 8; v++) {
+            const float send = b ? a16[v] : a16[v + 8], keep = b ? a16[v + 8] : a16[v];
+            a8[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+        }
+    }
+    {
+        const bool b = lane & 8;
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const float send = b ? a8[v] : a8[v + 4], keep = b ? a8[v + 4] : a8[v];
+            a4[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+        }
+    }
+    {
+        const bool b = lane & 16;
+#pragma unroll
+        for (int v = 0; v < 2; v++) {
+            const float send = b ? a4[v] : a4[v + 2], keep = b ? a4[v + 2] : a4[v];
+            a2[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+        }
+    }
+    const int rl = ((lane & 1) << 4) | ((lane & 2) << 2) | (lane & 4) | ((lane & 8) >> 2) | ((lane & 16) >> 4);
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+        const int idx = 2 * rl + u;
+        const int t = t0 + 8 * tg + (idx >> 3), e = e0 + 8 * eg + (idx & 7);
+        if (t < p.T && e < p.E) {
+            float val = a2[u];
+            if (p.bias) val = __fadd_rn(val, p.bias[e]);
+            p.logits[static_cast<size_t>(t) * p.E + e] = val;
+        }
+    }
 }
 
 // top-k per token: k rounds of a warp argmax, larger logit first, equal
