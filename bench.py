@@ -215,22 +215,48 @@ def run_ours(args, rank, world, local_rank):
     per = {n: sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps
            for i, n in enumerate(names)}
 
-    # ---- end to end through the public call with host buffers
+    # ---- end to end through the public call with host buffers: every step
+    # copies its X from pinned host memory and its Y back to pinned host
+    # memory.  Copies run on their own streams, double-buffered, so step i's
+    # copies overlap the layer of steps i-1 / i+1 (a serving loop's pipeline).
     x_host = x.cpu().pin_memory()
-    y_host = torch.empty(T, wl.H, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
-    for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        native.moe_forward(layer.h, x_dev, T, wr, bias, layer.packed, y, layer.ws)
-        y_host.copy_(y, non_blocking=True)
+    y_host = [torch.empty(T, wl.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    y_dev = [torch.empty_like(y) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def e2e_steps(n, ev_first=None, ev_last=None):
+        done_in = [torch.cuda.Event() for _ in range(n)]
+        done_fw = [torch.cuda.Event() for _ in range(n)]
+        done_out = [torch.cuda.Event() for _ in range(n)]
+        if ev_first is not None:
+            ev_first.record(s_in)
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done_fw[i - 2])          # x_dev[b] free again
+                x_dev[b].copy_(x_host, non_blocking=True)
+                done_in[i].record(s_in)
+            stream.wait_event(done_in[i])
+            if i >= 2:
+                stream.wait_event(done_out[i - 2])           # y_dev[b] read back already
+            native.moe_forward(layer.h, x_dev[b], T, wr, bias, layer.packed, y_dev[b], layer.ws)
+            done_fw[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done_fw[i])
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+                done_out[i].record(s_out)
+        if ev_last is not None:
+            s_out.wait_stream(s_in)
+            ev_last.record(s_out)
+
+    e2e_steps(2)
     torch.cuda.synchronize()
     barrier()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        native.moe_forward(layer.h, x_dev, T, wr, bias, layer.packed, y, layer.ws)
-        y_host.copy_(y, non_blocking=True)
-    ev1.record(stream)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps(args.steps, ev0, ev1)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = ev0.elapsed_time(ev1)
@@ -280,7 +306,8 @@ def run_ours(args, rank, world, local_rank):
         "kernel_ms": per,
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
-        "gpu_launches": 8 * args.steps,
+        # router 2 + dispatch 4 (+ amax for NVFP4) + gate/up + down + combine
+        "gpu_launches": (10 if wl.fmt == FMT_NVFP4 else 9) * args.steps,
         "clocks": clk.summary(),
     }
     layer.close()
