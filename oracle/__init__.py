@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "moe_oracle.c")
 LIB = os.path.join(HERE, "libmoe_oracle.so")
 
-FMT_FP8_ROW, FMT_FP8_BLOCK128, FMT_NVFP4 = 0, 1, 2
+FMT_FP8_ROW, FMT_FP8_BLOCK128, FMT_NVFP4, FMT_MX32 = 0, 1, 2, 3
 SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
 TILE_M = 128
 
@@ -191,12 +191,14 @@ def scale_shape(fmt, rows, K):
         return (rows,), np.float32
     if fmt == FMT_FP8_BLOCK128:
         return (rows, K // 128), np.float32
+    if fmt == FMT_MX32:
+        return (rows, K // 32), np.uint8
     return (rows, K // 16), np.uint8
 
 
 def hidden_fmt(fmt):
-    """The hidden is requantised per (row, 128 columns) for both FP8 formats."""
-    return FMT_NVFP4 if fmt == FMT_NVFP4 else FMT_FP8_BLOCK128
+    """Format of the requantised hidden: MX32 for FP8_ROW, otherwise the layer's own."""
+    return FMT_MX32 if fmt == FMT_FP8_ROW else fmt
 
 
 def quant_rows(fmt, x, g=0.0):

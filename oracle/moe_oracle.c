@@ -245,6 +245,17 @@ float orc_nvfp4_global(const float* x, int64_t n)
 
 static int64_t row_code_bytes(int fmt, int K) { return fmt == ORC_FMT_NVFP4 ? K / 2 : K; }
 
+/* smallest e with amax <= 448 * 2^e (amax > 0): amax = m 2^x, m in [0.5, 1),
+ * 448 = 0.875 2^9, so e = x - 9 when m <= 0.875, else x - 8 */
+static int mx_exponent(float amax)
+{
+    if (amax == 0.0f) return -127;
+    int x;
+    float m = frexpf(amax, &x);
+    int e = (m <= 0.875f) ? x - 9 : x - 8;
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
 void orc_quant_rows(int fmt, const float* x, int rows, int K, float g,
                     uint8_t* codes, void* scales)
 {
@@ -261,6 +272,15 @@ void orc_quant_rows(int fmt, const float* x, int rows, int K, float g,
                 ((float*)scales)[(int64_t)r * (K / bw) + b] = s;
                 for (int c = b * bw; c < (b + 1) * bw; c++)
                     qr[c] = (s == 0.0f) ? 0 : orc_e4m3_encode(xr[c] / s);
+            }
+        } else if (fmt == ORC_FMT_MX32) {
+            uint8_t* sr = (uint8_t*)scales + (int64_t)r * (K / 32);
+            for (int b = 0; b < K / 32; b++) {
+                float amax = 0.0f;
+                for (int c = 32 * b; c < 32 * b + 32; c++) amax = fmaxf(amax, fabsf(xr[c]));
+                int e = mx_exponent(amax);
+                sr[b] = (uint8_t)(e + 127);
+                for (int c = 32 * b; c < 32 * b + 32; c++) qr[c] = orc_e4m3_encode(ldexpf(xr[c], -e));
             }
         } else {
             uint8_t* sr = (uint8_t*)scales + (int64_t)r * (K / 16);
@@ -293,6 +313,8 @@ static void dequant_act_row(int fmt, const uint8_t* q, const void* s, float g, i
             out[c] = orc_e4m3_value(q[c]) * (double)((const float*)s)[0];
         else if (fmt == ORC_FMT_FP8_BLOCK128)
             out[c] = orc_e4m3_value(q[c]) * (double)((const float*)s)[c / 128];
+        else if (fmt == ORC_FMT_MX32)
+            out[c] = ldexp(orc_e4m3_value(q[c]), (int)((const uint8_t*)s)[c / 32] - 127);
         else {
             uint8_t nib = (c & 1) ? (q[c / 2] >> 4) : (q[c / 2] & 15);
             out[c] = orc_e2m1_value(nib) * orc_e4m3_value(((const uint8_t*)s)[c / 16]) * (double)g;
@@ -304,16 +326,23 @@ static int64_t act_scale_bytes(int fmt, int K)
 {
     if (fmt == ORC_FMT_FP8_ROW) return 4;
     if (fmt == ORC_FMT_FP8_BLOCK128) return 4 * (K / 128);
+    if (fmt == ORC_FMT_MX32) return K / 32;
     return K / 16;
 }
 
 /* ------------------------------------------------------------ expert FFN */
 
-/* Format of the requantised hidden.  The gate/up epilogue of a tile sees 128
- * hidden columns of a row, so the FP8 formats scale the hidden per (row,
- * 128-column block) (the 1x128 activation rule); NVFP4 keeps its 16-blocks
- * with the static global scale. */
-static int hidden_fmt(int fmt) { return fmt == ORC_FMT_NVFP4 ? ORC_FMT_NVFP4 : ORC_FMT_FP8_BLOCK128; }
+/* Format of the requantised hidden.  The gate/up epilogue of a tile sees a
+ * block of hidden columns of a row, never the whole row, so the hidden gets
+ * block scales: power-of-two scales per 32 columns (MX32, applied by the
+ * tensor cores in the down projection) for FP8_ROW, fp32 scales per 128
+ * columns (the 1x128 activation rule, like its X) for FP8_BLOCK128, and the
+ * NVFP4 16-blocks with the static global scale for NVFP4. */
+static int hidden_fmt(int fmt)
+{
+    if (fmt == ORC_FMT_FP8_ROW) return ORC_FMT_MX32;
+    return fmt;
+}
 
 void orc_weight_row(const orc_layer* L, const orc_proj* P, int N, int K, int e, int n, double* out)
 {

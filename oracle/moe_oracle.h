@@ -33,7 +33,7 @@ extern "C" {
 #endif
 
 enum { ORC_SCORE_SOFTMAX = 0, ORC_SCORE_SIGMOID = 1 };
-enum { ORC_FMT_FP8_ROW = 0, ORC_FMT_FP8_BLOCK128 = 1, ORC_FMT_NVFP4 = 2 };
+enum { ORC_FMT_FP8_ROW = 0, ORC_FMT_FP8_BLOCK128 = 1, ORC_FMT_NVFP4 = 2, ORC_FMT_MX32 = 3 };
 enum { ORC_TILE_M = 128 };
 
 /* ---- codecs (OCP FP8 E4M3 "fn" and FP4 E2M1, round to nearest even, saturating) ---- */
@@ -87,6 +87,10 @@ int orc_pick_down_tile(const int32_t* counts, int E, int H, int I, int num_sms,
  * FP8_ROW:      one fp32 scale per row: s = fp32(amax/448), q = e4m3(fp32(x/s)),
  *               q = 0 when s == 0.  scales: [rows]
  * FP8_BLOCK128: the same per 128-column block.  scales: [rows, K/128] fp32
+ * MX32:         e4m3 codes with a power-of-two scale 2^e per 32-column block (OCP MX
+ *               style, UE8M0 code e + 127): e is the smallest integer with
+ *               amax_b <= 448 * 2^e (e = -127 when amax_b == 0, clamped to [-127, 127]);
+ *               q = e4m3(x * 2^-e).  scales: [rows, K/32] uint8 codes.
  * NVFP4:        g given (fp32, > 0); per 16-column block b: sb = e4m3(fp32(fp32(amax_b/6)/g)),
  *               d = fp32(value(sb)*g), q = e2m1(fp32(x/d)) (q = 0 when d == 0).
  *               codes packed two per byte, element 2i in the low nibble;
@@ -117,9 +121,10 @@ void orc_weight_row(const orc_layer* L, const orc_proj* P, int N, int K, int e, 
 /* One expert on quantised input rows.
  *   a_codes/a_scales: rows of the quantised input in the layer's format (K = H)
  *   x_global: NVFP4 global scale of the input (ignored otherwise)
- *   The hidden is requantised per (row, 128-column block) with fp32 scales for
- *   both FP8 formats ([rows, I/128] scales), and with the NVFP4 rule and the
- *   static hidden_global scale for NVFP4.
+ *   The hidden is requantised with the MX32 rule (power-of-two scale per 32
+ *   columns) for FP8_ROW, per (row, 128-column block) with fp32 scales for
+ *   FP8_BLOCK128, and with the NVFP4 rule and the static hidden_global scale
+ *   for NVFP4.
  *   outputs: h (fp64 SwiGLU output before requantisation, [rows, I]) may be NULL;
  *            hq codes/scales (requantised hidden) may be NULL;
  *            o [rows, H] fp64 down projection of the dequantised hidden. */

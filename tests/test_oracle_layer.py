@@ -46,6 +46,8 @@ def deq_weight(wl, d, p, e):
 
 
 def deq_act(wl, codes, scales, g=0.0):
+    if wl.fmt == oracle.FMT_MX32:
+        return fp8_val(codes) * np.repeat(np.exp2(scales.astype(np.float64) - 127), 32, axis=1)
     if wl.fmt == W.FMT_FP8_ROW:
         return fp8_val(codes) * scales.astype(np.float64)[:, None]
     if wl.fmt == W.FMT_FP8_BLOCK128:

@@ -256,3 +256,29 @@ def test_pick_down_tile_load_term_and_waves():
     # one wave each, t_mma = 4 x 100 everywhere; load shrinks with more tiles
     loads = [1 * 2048 * 512 * 1000000 // (t * 1000) for t in (8, 16, 32)]
     assert list(costs) == [max(400, l) for l in loads] and c == 2
+
+
+# ------------------------------------------------------------------ MX32 hidden rule
+def test_mx32_quant_hand_example():
+    x = np.zeros((4, 64), np.float32)
+    x[0, 0] = 448.0            # 448 = 0.875 * 2^9 -> e = 0, code 127
+    x[0, 32] = 449.0           # just above: e = 1, code 128, 449/2 = 224.5 -> e4m3 224
+    x[1, 0] = 1.0              # 1 = 0.5 * 2^1 -> e = -8 (448 / 256 = 1.75 >= 1 > 0.875)
+    x[1, 1] = -0.5
+    codes, sc = oracle.quant_rows(oracle.FMT_MX32, x)
+    assert list(sc[0]) == [127, 128] and list(sc[1]) == [119, 0]
+    assert codes[0, 0] == 0x7E and codes[0, 32] == 0x76
+    assert codes[1, 0] == 0x78 and codes[1, 1] == 0xF0      # 256 and -128
+    assert (sc[2:] == 0).all() and (codes[2:] == 0).all()
+
+
+def test_mx32_exponent_is_the_smallest_that_fits():
+    rng = np.random.default_rng(11)
+    x = (rng.normal(size=(16, 256)) * np.exp(rng.uniform(-20, 20, size=(16, 1)))).astype(np.float32)
+    codes, sc = oracle.quant_rows(oracle.FMT_MX32, x)
+    amax = np.abs(x).reshape(16, 8, 32).max(axis=2).astype(np.float64)
+    scale = np.exp2(sc.astype(np.float64) - 127)
+    assert (amax <= 448.0 * scale).all() and (amax > 224.0 * scale).all()
+    deq = torch_e4m3_value(codes) * np.repeat(scale, 32, axis=1)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, np.repeat(scale, 32, axis=1) * 2.0 ** -10)
+    assert (np.abs(deq - x) <= bound).all()
