@@ -222,6 +222,31 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
     return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Byte offset of block scale factor (row, column c) in the chunked layout the
+// block-scaled tensor-core MMAs read: per 128-row tile, per 4 scale columns,
+// 512 bytes with row r of the tile at (r % 32) * 16 + (r / 32) * 4 + c % 4.
+// sf_cols = scale columns per row (K / 16 for NVFP4, K / 32 for MX).
+__host__ __device__ __forceinline__ size_t sf_offset(long long row, int c, int sf_cols) {
+    const long long tile = row >> 7;
+    const int r = static_cast<int>(row & 127);
+    return (static_cast<size_t>(tile) * (sf_cols >> 2) + (c >> 2)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (c & 3);
+}
+
+// MX (UE8M0) block exponent: the smallest e with amax <= 448 * 2^e; amax =
+// m 2^x with m in [0.5, 1) and 448 = 0.875 2^9 give e = x - 9 when m <= 0.875,
+// else x - 8.  amax == 0 -> -127.  Clamped to [-127, 127].
+__device__ __forceinline__ int mx_exponent(float amax) {
+    if (amax == 0.0f) return -127;
+    int x;
+    const float m = frexpf(amax, &x);
+    const int e = (m <= 0.875f) ? x - 9 : x - 8;
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+// 2^-e as a float for e in [-126, 127] (2^-127 is the subnormal 2^-127)
+__device__ __forceinline__ float mx_inv_scale(int e) {
+    return e >= 127 ? 5.877471754111438e-39f : __int_as_float((127 - e) << 23);
+}
+
 // ------------------------------------------------------------------ numerics
 // e4m3 of two floats, round to nearest even, saturating; .x -> low byte.
 __device__ __forceinline__ uint16_t f2_to_e4m3x2(float a, float b) {

@@ -293,15 +293,6 @@ __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* x, long 
     if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_int(m));
 }
 
-// Byte offset of scale factor (row, column c = K index / 16) in the chunked
-// layout the tensor cores read: per 128-row tile, per 4 scale columns, 512
-// bytes with row r of the tile at (r % 32) * 16 + (r / 32) * 4 + c % 4.
-__host__ __device__ __forceinline__ size_t sf_offset(long long row, int c, int sf_cols) {
-    const long long tile = row >> 7;
-    const int r = static_cast<int>(row & 127);
-    return (static_cast<size_t>(tile) * (sf_cols >> 2) + (c >> 2)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (c & 3);
-}
-
 // NVFP4 quantisation of X rows, scattered to the rows of the assignments in the
 // 128-padded expert-major layout: assignment slot s of expert e goes to row
 // tile_ptr[e] * 128 + (s - offsets[e]).  Per 16-block: sb = e4m3((amax/6)/g),

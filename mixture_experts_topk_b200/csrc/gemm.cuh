@@ -54,8 +54,9 @@ struct GemmParams {
     const float* a_scale;       // X or hidden scales, a_ld floats per row
     int a_ld;
     const float* b_scale;       // BSCALE_ROW: [E][b_rows]; BLOCK128: [E][b_rows/128][num_kb]
-    uint8_t* hq;                // gate/up: hidden codes [A][I], scales hs [A][I/128]
-    float* hs;
+    uint8_t* hq;                // gate/up: hidden codes; FP8_ROW: [padded rows][I] + MX scales in hsf,
+    float* hs;                  //   BLOCK128: [A][I] + fp32 scales hs [A][I/128]
+    uint8_t* hsf;
     int I;
     float* o;                   // down: [A][H] fp32
     int H;
@@ -295,8 +296,37 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 #pragma unroll
                     for (int c = 0; c < 64; c++) hv[c] = ag[c] / (1.0f + expf(-ag[c])) * au[c];
                 }
-                // requantise the 128-column hidden block of this row: the two
-                // column groups exchange their partial amax through shared memory
+                if (BSCALE == BSCALE_ROW) {
+                    // MX requantisation: power-of-two scale per 32 hidden columns (all
+                    // inside this thread), codes to the expert's 128-padded rows and
+                    // scales to the chunked layout the down GEMM's tensor cores read
+                    if (valid) {
+                        const long long prow = static_cast<long long>(mi) * 128 + r;
+                        const int col0 = nb * 128 + 64 * g;
+                        uint32_t w[16];
+#pragma unroll
+                        for (int b = 0; b < 2; b++) {
+                            float amax = 0.0f;
+#pragma unroll
+                            for (int c = 0; c < 32; c++) amax = fmaxf(amax, fabsf(hv[32 * b + c]));
+                            const int ex = mx_exponent(amax);
+                            const float inv = mx_inv_scale(ex);
+#pragma unroll
+                            for (int c = 0; c < 32; c += 4) {
+                                const uint16_t lo = f2_to_e4m3x2(__fmul_rn(hv[32 * b + c], inv), __fmul_rn(hv[32 * b + c + 1], inv));
+                                const uint16_t hi = f2_to_e4m3x2(__fmul_rn(hv[32 * b + c + 2], inv), __fmul_rn(hv[32 * b + c + 3], inv));
+                                w[8 * b + c / 4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+                            }
+                            p.hsf[sf_offset(prow, col0 / 32 + b, p.I / 32)] = static_cast<uint8_t>(ex + 127);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(p.hq + prow * p.I + col0);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                    }
+                    continue;
+                }
+                // BLOCK128: requantise the 128-column hidden block of this row; the
+                // two column groups exchange their partial amax through shared memory
                 float amax = 0.0f;
 #pragma unroll
                 for (int c = 0; c < 64; c++) amax = fmaxf(amax, fabsf(hv[c]));

@@ -1,0 +1,225 @@
+// gemm_mx.cuh -- persistent grouped down GEMM on MX-scaled FP8 (tcgen05.mma
+// kind::mxf8f6f4 with block32 UE8M0 scales applied by the tensor cores).
+//
+// LightMoE README ("MoE inference"): the requantised hidden feeds the down
+// projection and the routing weight is applied; Alpha-MoE article: FP8 W8A8.
+// The FP8_ROW hidden carries a power-of-two scale per 32 columns, so the whole
+// K reduction stays in TMEM (no per-K-block promotion).  The weights carry one
+// fp32 scale per output row, applied with the routing weight in the epilogue;
+// their MX scale is the constant 1 (UE8M0 127), copied into TMEM once.
+//
+// Tile 128 padded rows x 256 columns, K stage 128 (one 512-byte scale chunk of
+// A per stage: 4 scales of 32 per row), 4 stages.  MMA j of a stage (K = 32)
+// uses byte j of the chunk (scale-factor id j).  TMEM: one 256-column
+// accumulator, released as soon as the epilogue has it in registers, then the
+// A-scale ring and the constant B-scale chunks.
+#pragma once
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+
+constexpr int MX_BN = 256;
+constexpr int MX_STAGES = 4;
+constexpr int MX_A_BYTES = 128 * 128;
+constexpr int MX_B_BYTES = MX_BN * 128;
+constexpr int MX_SFA_BYTES = 512;
+constexpr int MX_STAGE_BYTES = MX_A_BYTES + MX_B_BYTES + 1024;   // + 512 B A scales, padded to 1 KB
+constexpr int MX_SFB_OFF = MX_STAGES * MX_STAGE_BYTES;            // 2 constant chunks (1 KB)
+constexpr int MX_BAR_OFF = MX_SFB_OFF + 1024;
+constexpr int MX_NUM_BARS = 2 * MX_STAGES + 3;
+constexpr int MX_TMEM_SLOT_OFF = MX_BAR_OFF + 8 * MX_NUM_BARS;
+constexpr int MX_SMEM = MX_TMEM_SLOT_OFF + 16 + 1024;
+constexpr int MX_SFA_TMEM = MX_BN;                    // 4 columns per stage
+constexpr int MX_SFB_TMEM = MX_BN + 4 * MX_STAGES;    // 8 columns (two 128-row chunks)
+
+// Instruction descriptor of kind::mxf8f6f4 block-scaled: A, B E4M3 (0), K-major,
+// N >> 3 at [17,23), UE8M0 scales ([23] = 1), M >> 4 at [24,29), A scale id at
+// [29,31), B scale id at [4,6), dense K = 32.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, int sf_id) {
+    return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
+}
+
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+struct MxDownParams {
+    const int32_t* tiles;
+    const int32_t* num_tiles;
+    const int32_t* tile_ptr;
+    const int32_t* offsets;
+    int E;
+    int n_blocks;              // H / 256
+    int num_kb;                // I / 128
+    int b_rows;                // H
+    const uint8_t* sfa;        // hidden MX scales, chunked by padded row tile (I / 32 per row)
+    const float* w_scale;      // [E][H] fp32 per output row of W_down
+    float* o;                  // [A][H] fp32 rows in slot order
+    int H;
+    const int32_t* perm;
+    const float* route_w;
+    int32_t* status;
+    long long spin_limit;
+};
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    grouped_gemm_mx_down_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                                const MxDownParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MX_BAR_OFF);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + MX_STAGES;
+    uint64_t* tfull = bars + 2 * MX_STAGES;
+    uint64_t* tempty = bars + 2 * MX_STAGES + 1;
+    uint64_t* drain = bars + 2 * MX_STAGES + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MX_TMEM_SLOT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // constant B scale chunks: 1.0 for every row and block
+    for (int i = threadIdx.x; i < 1024 / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(smem + MX_SFB_OFF)[i] = 0x7F7F7F7Fu;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < MX_STAGES; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(tempty, 8);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    // the generic-proxy writes of the constant chunks become visible to tcgen05.cp
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int ntm = *p.num_tiles;
+    const int total = ntm * p.n_blocks;
+    const long long limit = p.spin_limit;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                int mi, nb;
+                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
+                const int e = p.tiles[2 * mi];
+                const int brow = e * p.b_rows + nb * MX_BN;
+                const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.num_kb * 512;
+                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                    const int s = it % MX_STAGES;
+                    if (!mbar_wait(&empty[s], ((it / MX_STAGES) & 1) ^ 1, limit)) {
+                        report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + s * MX_STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], MX_A_BYTES + MX_B_BYTES + MX_SFA_BYTES);
+                    tma_load_2d(st, &tmA, &full[s], kb * 128, mi * 128);
+                    tma_load_2d(st + MX_A_BYTES, &tmB, &full[s], kb * 128, brow);
+                    bulk_load(st + MX_A_BYTES + MX_B_BYTES, sfa + kb * 512, MX_SFA_BYTES, &full[s]);
+                }
+            }
+            const uint32_t first = it > MX_STAGES ? it - MX_STAGES : 0;
+            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % MX_STAGES], (j / MX_STAGES) & 1, limit);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sfb = tmem_base + MX_SFB_TMEM;
+            tmem_cp_32x128b_x4(sfb, sdesc_sf_chunk(smem_u32(smem + MX_SFB_OFF)));
+            tmem_cp_32x128b_x4(sfb + 4, sdesc_sf_chunk(smem_u32(smem + MX_SFB_OFF + 512)));
+            uint32_t it = 0, u = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                if (!mbar_wait(tempty, (u & 1) ^ 1, limit)) { ok = false; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                    const int s = it % MX_STAGES;
+                    if (!mbar_wait(&full[s], (it / MX_STAGES) & 1, limit)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * MX_STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + MX_A_BYTES;
+                    const uint32_t sfa = tmem_base + MX_SFA_TMEM + 4 * s;
+                    tmem_cp_32x128b_x4(sfa, sdesc_sf_chunk(b_addr + MX_B_BYTES));
+#pragma unroll
+                    for (int j = 0; j < 4; j++)
+                        mma_mxf8(tmem_base, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
+                                 idesc_mxf8(128, MX_BN, j), sfa, sfb, (kb > 0 || j > 0));
+                    mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(tfull);
+                u++;
+            }
+            if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
+            mma_commit(drain);
+            mbar_wait(drain, 0, limit);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int g = (warp - 2) >> 2;             // 128 columns per column group
+        const int r = 32 * q + lane;
+        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+        uint32_t u = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            int mi, nb;
+            decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
+            const int e = p.tiles[2 * mi];
+            const int local = mi * 128 + r - p.tile_ptr[e] * 128;
+            const bool valid = local < p.offsets[e + 1] - p.offsets[e];
+            if (!warp_wait(tfull, u & 1, limit)) { ok = false; break; }
+            tc_fence_after();
+            float v[128];
+#pragma unroll
+            for (int ch = 0; ch < 2; ch++)
+                tmem_ld32x2(lane_addr + 128 * g + 64 * ch, lane_addr + 128 * g + 64 * ch + 32, v + 64 * ch,
+                            v + 64 * ch + 32);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty);   // the next tile's MMAs may start
+            u++;
+            if (valid) {
+                const int slot = p.offsets[e] + local;
+                const float rw = p.route_w[p.perm[slot]];
+                const int n0 = nb * MX_BN + 128 * g;
+                const float* ws = p.w_scale + static_cast<size_t>(e) * p.H + n0;
+                float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(slot) * p.H + n0);
+#pragma unroll
+                for (int c = 0; c < 128; c += 4) {
+                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(ws + c));
+                    dst[c / 4] = make_float4(v[c] * s4.x * rw, v[c + 1] * s4.y * rw, v[c + 2] * s4.z * rw,
+                                             v[c + 3] * s4.w * rw);
+                }
+            }
+        }
+        if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_EPILOGUE);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace moe

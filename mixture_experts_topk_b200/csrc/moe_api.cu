@@ -14,6 +14,7 @@
 #include "dispatch.cuh"
 #include "gemm.cuh"
 #include "gemm_fp4.cuh"
+#include "gemm_mx.cuh"
 #include "router.cuh"
 
 using namespace moe;
@@ -72,10 +73,21 @@ static size_t act_scale_bytes(int fmt, int K) {
     if (fmt == MOE_FMT_FP8_BLOCK128) return 4 * (K / 128);
     return K / 16;
 }
-static size_t hidden_scale_bytes(int fmt, int I) { return fmt == MOE_FMT_NVFP4 ? I / 16 : 4 * (I / 128); }
+// scale bytes per hidden row: MX (power of two per 32) for FP8_ROW, fp32 per 128
+// for FP8_BLOCK128, e4m3 per 16 for NVFP4
+static size_t hidden_scale_bytes(int fmt, int I) {
+    if (fmt == MOE_FMT_FP8_ROW) return I / 32;
+    return fmt == MOE_FMT_NVFP4 ? I / 16 : 4 * (I / 128);
+}
+// rows of the X / hidden buffers: 128-padded per expert where block-scaled
+// tensor-core MMAs read them (NVFP4 X and hidden, FP8_ROW hidden)
 static size_t padded_rows(const moe_config& c) {
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
     return c.fmt == MOE_FMT_NVFP4 ? A + static_cast<size_t>(TILE_M) * c.E : A;
+}
+static size_t hidden_rows(const moe_config& c) {
+    const size_t A = static_cast<size_t>(c.max_T) * c.k;
+    return c.fmt == MOE_FMT_FP8_BLOCK128 ? A : A + static_cast<size_t>(TILE_M) * c.E;
 }
 
 static WsLayout make_ws_layout(const moe_config& c) {
@@ -105,11 +117,11 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.xglobal = take(16);
     // NVFP4 rows are padded to 128 per expert, so each row tile owns whole
     // scale-factor chunks
-    const size_t R = (c.fmt == MOE_FMT_NVFP4) ? A + static_cast<size_t>(TILE_M) * c.E : A;
+    const size_t R = padded_rows(c), RH = hidden_rows(c);
     L.xq = take(R * code_bytes(c.fmt, c.H));
     L.xs = take(R * act_scale_bytes(c.fmt, c.H));
-    L.hq = take(R * code_bytes(c.fmt, c.I));
-    L.hs = take(R * hidden_scale_bytes(c.fmt, c.I));
+    L.hq = take(RH * code_bytes(c.fmt, c.I));
+    L.hs = take(RH * hidden_scale_bytes(c.fmt, c.I));
     L.o = take(A * c.H * 4);
     L.total = off;
     return L;
@@ -520,6 +532,7 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.b_scale = reinterpret_cast<const float*>(pw + h->wl.gu_s);
     p.hq = v.hq;
     p.hs = static_cast<float*>(v.hs);
+    p.hsf = static_cast<uint8_t*>(v.hs);
     p.I = c.I;
     p.H = c.H;
     p.status = v.status;
@@ -531,6 +544,44 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
 }
 
 // ------------------------------------------------------------------ down
+// FP8_ROW: MX-scaled hidden (tensor cores apply its scales), one tile width.
+static moe_status mx_down(const moe_handle* h, const void* packed, const float* w, int T, void* ws,
+                          moe_stream_t stream) {
+    const moe_config& c = h->cfg;
+    moe_workspace_view v;
+    moe_workspace_view_get(h, ws, &v);
+    const uint8_t* pw = static_cast<const uint8_t*>(packed);
+    CUtensorMap ta, tb;
+    moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
+    if (r != MOE_OK) return r;
+    r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, MX_BN);
+    if (r != MOE_OK) return r;
+    MxDownParams p;
+    memset(&p, 0, sizeof(p));
+    p.tiles = v.tiles;
+    p.num_tiles = v.num_tiles;
+    p.tile_ptr = v.tile_ptr;
+    p.offsets = v.offsets;
+    p.E = c.E;
+    p.n_blocks = c.H / MX_BN;
+    p.num_kb = c.I / 128;
+    p.b_rows = c.H;
+    p.sfa = static_cast<const uint8_t*>(v.hs);
+    p.w_scale = reinterpret_cast<const float*>(pw + h->wl.d_s);
+    p.o = v.o;
+    p.H = c.H;
+    p.perm = v.perm;
+    p.route_w = w;
+    p.status = v.status;
+    p.spin_limit = h->spin_limit;
+    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    CUDA_TRY(cudaFuncSetAttribute(grouped_gemm_mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MX_SMEM));
+    grouped_gemm_mx_down_kernel<<<grid, GEMM_THREADS, MX_SMEM, st>>>(ta, tb, p);
+    LAUNCH_CHECK("grouped_gemm_mx_down_kernel");
+    return MOE_OK;
+}
+
 extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const float* w, int T, void* ws,
                                moe_stream_t stream) {
     moe_status st0 = check_T(h, T, "moe_down");
@@ -539,6 +590,7 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     if (!packed || !ws || !w) return fail(MOE_ERR_INVALID_ARG, "moe_down: null argument");
     if (!aligned256(packed) || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_down: pointers must be 256-byte aligned");
     if (h->cfg.fmt == MOE_FMT_NVFP4) return fp4_gemm(h, packed, w, T, ws, stream, false);
+    if (h->cfg.fmt == MOE_FMT_FP8_ROW) return mx_down(h, packed, w, T, ws, stream);
     const moe_config& c = h->cfg;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
@@ -578,25 +630,14 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
         r = make_tmap(&tb64, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, 64);
         if (r != MOE_OK) return r;
         const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * (c.H / 64)));
-        if (c.fmt == MOE_FMT_FP8_ROW) {
-            CUDA_TRY(cudaFuncSetAttribute(down_gemm_poly_kernel<BSCALE_ROW>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, POLY_SMEM));
-            down_gemm_poly_kernel<BSCALE_ROW><<<grid, GEMM_THREADS, POLY_SMEM, st>>>(ta, tb, tb128, tb64, p, v.pick);
-        } else {
-            CUDA_TRY(cudaFuncSetAttribute(down_gemm_poly_kernel<BSCALE_BLOCK128>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, POLY_SMEM));
-            down_gemm_poly_kernel<BSCALE_BLOCK128><<<grid, GEMM_THREADS, POLY_SMEM, st>>>(ta, tb, tb128, tb64, p,
-                                                                                         v.pick);
-        }
+        CUDA_TRY(cudaFuncSetAttribute(down_gemm_poly_kernel<BSCALE_BLOCK128>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, POLY_SMEM));
+        down_gemm_poly_kernel<BSCALE_BLOCK128><<<grid, GEMM_THREADS, POLY_SMEM, st>>>(ta, tb, tb128, tb64, p,
+                                                                                     v.pick);
         LAUNCH_CHECK("down_gemm_poly_kernel");
         return MOE_OK;
     }
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
-    if (c.fmt == MOE_FMT_FP8_ROW) {
-        if (BN == 256) return launch_gemm<KIND_DOWN, BSCALE_ROW, true, 256, 4>(ta, tb, p, grid, st);
-        if (BN == 128) return launch_gemm<KIND_DOWN, BSCALE_ROW, true, 128, 6>(ta, tb, p, grid, st);
-        return launch_gemm<KIND_DOWN, BSCALE_ROW, true, 64, 8>(ta, tb, p, grid, st);
-    }
     if (BN == 256) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 256, 4>(ta, tb, p, grid, st);
     if (BN == 128) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 128, 6>(ta, tb, p, grid, st);
     return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 64, 8>(ta, tb, p, grid, st);

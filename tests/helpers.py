@@ -179,3 +179,31 @@ def e2m1_values(packed):
 
 def nvfp4_hidden_values(codes, sf_rm, g):
     return e2m1_values(codes) * np.repeat(fp8_values(sf_rm), 16, axis=-1) * float(g)
+
+
+def mx_hidden_values(codes, sf_rm):
+    """MX32 hidden: e4m3 code x 2^(scale code - 127) per 32 columns."""
+    return fp8_values(codes) * np.repeat(np.exp2(np.asarray(sf_rm, np.float64) - 127), 32, axis=-1)
+
+
+def hidden_padded(wl):
+    """The hidden sits in 128-padded rows with chunked block scales (FP8_ROW, NVFP4)."""
+    return wl.fmt != W.FMT_FP8_BLOCK128
+
+
+def hidden_sf_cols(wl):
+    return wl.I // 32 if wl.fmt == W.FMT_FP8_ROW else wl.I // 16
+
+
+def hidden_code_bytes(wl):
+    return wl.I // 2 if wl.fmt == W.FMT_NVFP4 else wl.I
+
+
+def hidden_values_of(wl, codes, scales):
+    """fp64 values of hidden rows given their codes and row-major scales, any format."""
+    if wl.fmt == W.FMT_FP8_ROW:
+        return mx_hidden_values(codes, scales)
+    if wl.fmt == W.FMT_NVFP4:
+        return nvfp4_hidden_values(codes, scales, wl.hidden_global_scale)
+    nb = wl.I // 128
+    return fp8_values(codes) * np.repeat(np.asarray(scales, np.float64).reshape(-1, nb), 128, axis=1)

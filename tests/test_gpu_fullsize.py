@@ -12,8 +12,8 @@ import torch
 
 import oracle
 from mixture_experts_topk_b200 import native, synth, workloads as W
-from helpers import (bits, deviation_bound_rows, gather_sf, hidden_values, nvfp4_hidden_values, padded_rows,
-                     tolerance_violations_with_bound)
+from helpers import (bits, deviation_bound_rows, gather_sf, hidden_code_bytes, hidden_padded, hidden_sf_cols,
+                     hidden_values_of, padded_rows, tolerance_violations_with_bound)
 
 pytestmark = pytest.mark.gpu
 
@@ -71,13 +71,14 @@ def test_full_size_layer(name, T, n_sample):
     x_sel = x[torch.from_numpy(sel).long().to(x.device)].float().cpu().numpy()
     g_x = oracle.nvfp4_global(x.float().cpu().numpy()) if fp4 else 0.0
     xq_tok, xs_tok = oracle.quant_rows(wl.fmt, x_sel, g_x)
-    if fp4:
+    padded = hidden_padded(wl)
+    if padded:
         tile_ptr = layer.region("tile_ptr", torch.int32, wl.E + 1).cpu().numpy()
         n_rows = A + 128 * wl.E
         off = layer.view["hq"] - layer.ws.data_ptr()
-        hq_all = layer.ws[off:off + n_rows * wl.I // 2].view(n_rows, wl.I // 2)
+        hq_all = layer.ws[off:off + n_rows * hidden_code_bytes(wl)].view(n_rows, hidden_code_bytes(wl))
         off = layer.view["hs"] - layer.ws.data_ptr()
-        hsf_all = layer.ws[off:off + n_rows * wl.I // 16].cpu().numpy()
+        hsf_all = layer.ws[off:off + n_rows * hidden_sf_cols(wl)].cpu().numpy()
     else:
         hq_gpu = layer.region("hq", torch.uint8, A * wl.I).view(A, wl.I)
         hs_gpu = layer.region("hs", torch.float32, A * wl.I // 128).view(A, wl.I // 128)
@@ -87,14 +88,13 @@ def test_full_size_layer(name, T, n_sample):
             e = int(ids[t, j])
             _, hq_r, hs_r, _ = L.expert_rows(e, xq_tok[i:i + 1], xs_tok[i:i + 1], g_x)
             r = int(inv[t * wl.k + j])
-            if fp4:
+            if padded:
                 prow = int(padded_rows([r], ids.reshape(-1), perm, offsets, tile_ptr)[0])
-                v_gpu = nvfp4_hidden_values(hq_all[prow].cpu().numpy()[None], gather_sf(hsf_all, [prow], wl.I // 16),
-                                            wl.hidden_global_scale)[0]
-                v_ref = nvfp4_hidden_values(hq_r, hs_r, wl.hidden_global_scale)[0]
+                v_gpu = hidden_values_of(wl, hq_all[prow].cpu().numpy()[None],
+                                         gather_sf(hsf_all, [prow], hidden_sf_cols(wl)))[0]
             else:
-                v_gpu = hidden_values(hq_gpu[r].cpu().numpy(), hs_gpu[r].cpu().numpy(), wl.I)
-                v_ref = hidden_values(hq_r[0], hs_r[0], wl.I)
+                v_gpu = hidden_values_of(wl, hq_gpu[r].cpu().numpy()[None], hs_gpu[r].cpu().numpy()[None])[0]
+            v_ref = hidden_values_of(wl, hq_r, hs_r)[0]
             rows.append((i, e, w[t, j], v_gpu, v_ref))
     extra = deviation_bound_rows(wl, sub, lambda e: int(slot[e]), rows, len(sel))
     y_gpu = y[torch.from_numpy(sel).long().cuda()].float().cpu().numpy()

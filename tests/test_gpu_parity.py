@@ -12,8 +12,9 @@ import torch
 
 import oracle
 from mixture_experts_topk_b200 import native, synth, workloads as W
-from helpers import (bits, fp8_values, gather_sf, hidden_deviation_bound, nvfp4_hidden_values, padded_rows,
-                     scatter_sf, slot_order_reference, tolerance_violations, tolerance_violations_with_bound)
+from helpers import (bits, fp8_values, gather_sf, hidden_code_bytes, hidden_deviation_bound, hidden_padded,
+                     hidden_sf_cols, hidden_values_of, nvfp4_hidden_values, padded_rows, scatter_sf,
+                     slot_order_reference, tolerance_violations, tolerance_violations_with_bound)
 
 pytestmark = pytest.mark.gpu
 
@@ -43,10 +44,50 @@ def gpu_slot_rows(layer, wl, ids, T):
     return padded_rows(np.arange(A), ids.reshape(-1), perm, offsets, tile_ptr)
 
 
-def gpu_rows(layer, wl, name, nbytes_per_row):
+def slot_rows(layer, wl, ids, T, padded):
+    A = T * wl.k
+    if not padded:
+        return np.arange(A)
+    counts, offsets, perm, inv = oracle.dispatch(ids, wl.E)
+    tile_ptr = layer.region("tile_ptr", torch.int32, wl.E + 1).cpu().numpy()
+    return padded_rows(np.arange(A), ids.reshape(-1), perm, offsets, tile_ptr)
+
+
+def gpu_rows(layer, wl, name, nbytes_per_row, padded=None):
+    padded = nvfp4(wl) if padded is None else padded
     v = layer.view[name] - layer.ws.data_ptr()
-    n = layer.max_T * wl.k + (128 * wl.E if nvfp4(wl) else 0)
+    n = layer.max_T * wl.k + (128 * wl.E if padded else 0)
     return layer.ws[v:v + n * nbytes_per_row].cpu().numpy().reshape(n, nbytes_per_row)
+
+
+def gpu_hidden(layer, wl, ids, T):
+    """(codes, row-major scales) of the GPU's hidden in slot order, any format."""
+    A = T * wl.k
+    if not hidden_padded(wl):
+        hq = layer.region("hq", torch.uint8, A * wl.I).cpu().numpy().reshape(A, wl.I)
+        hs = layer.region("hs", torch.float32, A * wl.I // 128).cpu().numpy().reshape(A, -1)
+        return hq, hs
+    rows = slot_rows(layer, wl, ids, T, True)
+    hq = gpu_rows(layer, wl, "hq", hidden_code_bytes(wl), True)[rows]
+    hs = gather_sf(gpu_rows(layer, wl, "hs", hidden_sf_cols(wl), True).reshape(-1), rows, hidden_sf_cols(wl))
+    return hq, hs
+
+
+def inject_hidden(layer, wl, ids, T, hq, hs):
+    """Write oracle hidden codes/scales (slot order) into the GPU's hidden buffers."""
+    A = T * wl.k
+    if not hidden_padded(wl):
+        layer.region("hq", torch.uint8, A * wl.I).copy_(torch.from_numpy(hq.reshape(-1)).cuda())
+        layer.region("hs", torch.float32, A * wl.I // 128).copy_(torch.from_numpy(hs.reshape(-1)).cuda())
+        return
+    rows = slot_rows(layer, wl, ids, T, True)
+    n_rows = layer.max_T * wl.k + 128 * wl.E
+    hq_all = np.zeros((n_rows, hidden_code_bytes(wl)), np.uint8)
+    hq_all[rows] = hq
+    sf_all = np.zeros(n_rows * hidden_sf_cols(wl), np.uint8)
+    scatter_sf(sf_all, rows, hs, hidden_sf_cols(wl))
+    layer.region("hq", torch.uint8, hq_all.size).copy_(torch.from_numpy(hq_all.reshape(-1)).cuda())
+    layer.region("hs", torch.uint8, sf_all.size).copy_(torch.from_numpy(sf_all).cuda())
 
 
 def build_case(name, seed=0):
@@ -180,30 +221,26 @@ def test_gate_up_hidden_matches_oracle(name):
     native.moe_gate_up(layer.h, layer.packed, T, layer.ws)
     torch.cuda.synchronize()
     assert layer.status()[0] == 0
-    A = T * wl.k
+    hq, hs = gpu_hidden(layer, wl, ids, T)
+    if wl.fmt == W.FMT_FP8_BLOCK128:
+        np.testing.assert_allclose(hs, ref["hs"], rtol=1e-4, atol=0)
+    else:
+        assert (hs != ref["hs"]).mean() <= 1e-3      # block scale codes
+    v_gpu = hidden_values_of(wl, hq, hs)
+    v_ref = hidden_values_of(wl, ref["hq"], ref["hs"])
+    # codes (and for the block-scaled formats the scale codes) decide the values;
+    # fp32 block scales (FP8_BLOCK128) differ in their last bits, so compare codes
+    mism = (hq != ref["hq"]) if wl.fmt == W.FMT_FP8_BLOCK128 else (v_gpu != v_ref)
+    assert mism.mean() <= 2e-3, f"{mism.mean():.2e} of the hidden codes differ"
+    # a differing value is one rounding step away (a flip at a rounding boundary):
+    # an e4m3 step is at most 1/8 of the value (+ the subnormal step), an e2m1
+    # step at most 2 x the block scale
     if nvfp4(wl):
-        rows = gpu_slot_rows(layer, wl, ids, T)
-        hq = gpu_rows(layer, wl, "hq", wl.I // 2)[rows]
-        sf = gpu_rows(layer, wl, "hs", wl.I // 16).reshape(-1)
-        hs = gather_sf(sf, rows, wl.I // 16)
-        assert (hs != ref["hs"]).mean() <= 1e-3
-        v_gpu = nvfp4_hidden_values(hq, hs, wl.hidden_global_scale)
-        v_ref = nvfp4_hidden_values(ref["hq"], ref["hs"], wl.hidden_global_scale)
-        mism = v_gpu != v_ref
-        assert mism.mean() <= 2e-3, f"{mism.mean():.2e} of the hidden values differ"
-        # a differing value is one rounding step away: at most a quarter of its 16-block's range
         step = np.repeat(fp8_values(ref["hs"]), 16, axis=1) * wl.hidden_global_scale * 2.0
         assert np.all(np.abs(v_gpu - v_ref) <= step * 1.0001)
-        return
-    hq = layer.region("hq", torch.uint8, A * wl.I).cpu().numpy().reshape(A, wl.I)
-    hs = layer.region("hs", torch.float32, A * wl.I // 128).cpu().numpy().reshape(A, -1)
-    np.testing.assert_allclose(hs, ref["hs"], rtol=1e-4, atol=0)
-    mism = hq != ref["hq"]
-    assert mism.mean() <= 1e-3, f"{mism.mean():.2e} of the hidden codes differ"
-    # a differing code is one step away (a rounding-boundary flip), never more
-    v_gpu = torch.from_numpy(hq).view(torch.float8_e4m3fn).float().numpy()
-    v_ref = torch.from_numpy(ref["hq"]).view(torch.float8_e4m3fn).float().numpy()
-    assert np.all(np.abs(v_gpu - v_ref) <= np.abs(v_ref) * 0.125 + 2.0 ** -9)
+    else:
+        unit = np.abs(hidden_values_of(wl, np.full_like(ref["hq"], 0x01), ref["hs"]))   # 2^-9 x scale
+        assert np.all(np.abs(v_gpu - v_ref) <= np.abs(v_ref) * 0.125 + unit * 1.0001 + 1e-30)
 
 
 @pytest.mark.parametrize("down_bn", [0, 64, 128, 256])
@@ -212,21 +249,10 @@ def test_down_matches_oracle_on_oracle_hidden(name, down_bn):
     wl, T, d, x, layer, ids, w, ref = _dispatch_and_reference(name)
     native.moe_set_tile_config(layer.h, down_bn)
     A = T * wl.k
-    if nvfp4(wl):
-        if down_bn not in (0,):
-            pytest.skip("the NVFP4 down GEMM has one tile width")
-        torch.cuda.synchronize()
-        rows = gpu_slot_rows(layer, wl, ids, T)
-        n_rows = layer.max_T * wl.k + 128 * wl.E
-        hq_all = np.zeros((n_rows, wl.I // 2), np.uint8)
-        hq_all[rows] = ref["hq"]
-        sf_all = np.zeros(n_rows * wl.I // 16, np.uint8)
-        scatter_sf(sf_all, rows, ref["hs"], wl.I // 16)
-        layer.region("hq", torch.uint8, hq_all.size).copy_(torch.from_numpy(hq_all.reshape(-1)).cuda())
-        layer.region("hs", torch.uint8, sf_all.size).copy_(torch.from_numpy(sf_all).cuda())
-    else:
-        layer.region("hq", torch.uint8, A * wl.I).copy_(torch.from_numpy(ref["hq"].reshape(-1)).cuda())
-        layer.region("hs", torch.float32, A * wl.I // 128).copy_(torch.from_numpy(ref["hs"].reshape(-1)).cuda())
+    if wl.fmt != W.FMT_FP8_BLOCK128 and down_bn != 0:
+        pytest.skip("this format's down GEMM has one tile width")
+    torch.cuda.synchronize()
+    inject_hidden(layer, wl, ids, T, ref["hq"], ref["hs"])
     w_dev = torch.from_numpy(w.astype(np.float32)).cuda()
     native.moe_down(layer.h, layer.packed, w_dev, T, layer.ws)
     torch.cuda.synchronize()
@@ -251,17 +277,10 @@ def test_forward_end_to_end(name):
     assert (layer.region("ids", torch.int32, T * wl.k).cpu().numpy().reshape(T, wl.k) == ids).all()
     A = T * wl.k
     ref = slot_order_reference(wl, L, x, ids, w)
-    if nvfp4(wl):
-        rows = gpu_slot_rows(layer, wl, ids, T)
-        hq = gpu_rows(layer, wl, "hq", wl.I // 2)[rows]
-        hs = gather_sf(gpu_rows(layer, wl, "hs", wl.I // 16).reshape(-1), rows, wl.I // 16)
-        v_gpu = nvfp4_hidden_values(hq, hs, wl.hidden_global_scale)
-        v_ref = nvfp4_hidden_values(ref["hq"], ref["hs"], wl.hidden_global_scale)
-        extra = hidden_deviation_bound(wl, L, ids, w, ref, None, None, values=(v_gpu, v_ref))
-    else:
-        hq = layer.region("hq", torch.uint8, A * wl.I).cpu().numpy().reshape(A, wl.I)
-        hs = layer.region("hs", torch.float32, A * wl.I // 128).cpu().numpy().reshape(A, -1)
-        extra = hidden_deviation_bound(wl, L, ids, w, ref, hq, hs)
+    hq, hs = gpu_hidden(layer, wl, ids, T)
+    v_gpu = hidden_values_of(wl, hq, hs)
+    v_ref = hidden_values_of(wl, ref["hq"], ref["hs"])
+    extra = hidden_deviation_bound(wl, L, ids, w, ref, None, None, values=(v_gpu, v_ref))
     bad, plain = tolerance_violations_with_bound(y.float().cpu().numpy(), y_ref, extra)
     assert bad == 0
     assert plain <= 1e-3 * y_ref.size, f"{plain} elements outside the plain tolerance"
