@@ -273,7 +273,9 @@ def run_ours(args, rank, world, local_rank):
     gu_ms = per["gate_up"]
     achieved = gu_flops / (gu_ms * 1e-3) / 1e12
     step_ms = ms_max / args.steps
-    t_roof_ms = max(fl_t / (fp8_peak * 1e12), byts / (pk["hbm_gbs"] * 1e9)) * 1e3
+    # fp32 SIMT peak of the router: 148 SMs x 128 FMA lanes x 2 FLOP x max SM clock
+    simt_peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6
+    t_roof_ms = max(fl_t / (fp8_peak * 1e12) + fl_r / simt_peak, byts / (pk["hbm_gbs"] * 1e9)) * 1e3
     tokens_total = world * T * args.steps
     out = {
         "metric": METRIC,
@@ -296,7 +298,9 @@ def run_ours(args, rank, world, local_rank):
                    "down_tile_source": "fixed" if args.down_bn else "picked from the histogram"},
         "tflops": (fl_t + fl_r) * world * args.steps / (ms_max * 1e-3) / 1e12,
         "layer_roofline": {"t_roof_ms": t_roof_ms, "frac": t_roof_ms / step_ms,
-                           "peaks": f"{pk_kind}: tensor = (2 fp8 | 4 fp4) x bf16_tflops_sustained, hbm_gbs"},
+                           "model": "max(tensor FLOPs / P_tensor + router FLOPs / P_fp32, algorithmic bytes / HBM)",
+                           "peaks": f"{pk_kind}: tensor = (2 fp8 | 4 fp4) x bf16_tflops_sustained, hbm_gbs; "
+                                    "P_fp32 = 148 SMs x 128 lanes x 2 x sm_max_mhz"},
         "roofline": {"kernel": "grouped_gemm gate/up (SwiGLU + requant epilogue)", "bound": "tensor",
                      "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp8_peak, "traffic": gemm_traffic(args.workload, T),
