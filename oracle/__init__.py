@@ -73,6 +73,7 @@ def lib():
             "orc_moe_forward": (I, [P, P, I, P, P, I, P, P, P, P]),
             "orc_num_threads": (I, []),
             "orc_pick_down_tile": (I, [P, I, I, I, I, I64, I64, I64, I64, P]),
+            "orc_pick_split": (I, [P, I, I, I, I64, I]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -179,6 +180,12 @@ def pick_down_tile(counts, H, I, num_sms, alpha, beta, bw, gamma):
     costs = np.empty(3, np.int64)
     c = lib().orc_pick_down_tile(_p(counts), counts.size, H, I, num_sms, alpha, beta, bw, gamma, _p(costs))
     return c, costs
+
+
+def pick_split(counts, split_nb, split_kb, o_rows, num_sms):
+    """K split S of the FP8_ROW down GEMM from the expert histogram (1 = none)."""
+    counts = _c(counts, np.int32)
+    return lib().orc_pick_split(_p(counts), counts.size, split_nb, split_kb, o_rows, num_sms)
 
 
 # ---------------------------------------------------------------- quantisers

@@ -234,6 +234,28 @@ int orc_pick_down_tile(const int32_t* counts, int E, int H, int I, int num_sms,
     return best;
 }
 
+/* K split of the down GEMM for small batches: S copies of the output rows, one
+ * per near-equal range of K-blocks.  units = m_tiles * split_nb; the split is
+ * bounded by 8, by the copies the output buffer holds (o_rows / A) and by at
+ * least four K-blocks per range; S is the largest admissible s with
+ * units * s <= num_sms, and 1 when split_nb is 0 or the batch is empty. */
+int orc_pick_split(const int32_t* counts, int E, int split_nb, int split_kb, int64_t o_rows, int num_sms)
+{
+    int64_t m_tiles = 0, A = 0;
+    for (int e = 0; e < E; e++) {
+        m_tiles += (counts[e] + ORC_TILE_M - 1) / ORC_TILE_M;
+        A += counts[e];
+    }
+    if (split_nb <= 0 || A == 0) return 1;
+    int64_t smax = 8;
+    if (o_rows / A < smax) smax = o_rows / A;
+    if (split_kb / 4 < smax) smax = split_kb / 4;
+    int best = 1;
+    for (int64_t s = 2; s <= smax; s++)
+        if (m_tiles * split_nb * s <= num_sms) best = (int)s;
+    return best;
+}
+
 /* ------------------------------------------------ activation quantisation */
 
 float orc_nvfp4_global(const float* x, int64_t n)

@@ -82,6 +82,8 @@ int  orc_schedule(const int32_t* offsets, int E, int32_t* tile_expert, int32_t* 
  * Returns the c of the lowest cost, the lower c on equal costs. */
 int orc_pick_down_tile(const int32_t* counts, int E, int H, int I, int num_sms,
                        int64_t alpha, int64_t beta, int64_t bw, int64_t gamma, int64_t* costs);
+/* K split of the FP8_ROW down GEMM (1 = none) from the expert histogram. */
+int orc_pick_split(const int32_t* counts, int E, int split_nb, int split_kb, int64_t o_rows, int num_sms);
 
 /* ---- activation quantisation of token rows (X or the hidden) ----
  * FP8_ROW:      one fp32 scale per row: s = fp32(amax/448), q = e4m3(fp32(x/s)),

@@ -258,6 +258,31 @@ def test_pick_down_tile_load_term_and_waves():
     assert list(costs) == [max(400, l) for l in loads] and c == 2
 
 
+def test_pick_split_hand_examples():
+    # Mixtral-shaped decode, one token on two experts: 2 m-tiles x 16 n-blocks =
+    # 32 units; 32 x 4 = 128 <= 148 < 160 = 32 x 5, and s_max = min(8, 16/2, 112/4) = 8
+    mix = dict(split_nb=16, split_kb=112, o_rows=2 + 7 * 2, num_sms=148)
+    counts = np.int32([1, 0, 0, 1, 0, 0, 0, 0])
+    assert oracle.pick_split(counts, **mix) == 4
+    # one expert only: 16 units -> 16 x 8 = 128 <= 148, capped by 8
+    assert oracle.pick_split(np.int32([2, 0, 0, 0, 0, 0, 0, 0]), **mix) == 8
+    # the output buffer bounds the copies: o_rows / A = 16 / 4 = 4 ... = 16 / 5 = 3
+    assert oracle.pick_split(np.int32([4, 0, 0, 0, 0, 0, 0, 0]), **mix) == 4
+    assert oracle.pick_split(np.int32([5, 0, 0, 0, 0, 0, 0, 0]), **mix) == 3
+    # at least four K-blocks per range: split_kb 8 -> s_max 2
+    assert oracle.pick_split(counts, **dict(mix, split_kb=8)) == 2
+    # units filling the SMs: 148 units -> no split; 75 units -> 150 > 148 -> no split; 74 -> 2
+    many = dict(split_nb=1, split_kb=112, o_rows=10 ** 6, num_sms=148)
+    assert oracle.pick_split(np.full(148, 1, np.int32), **many) == 1
+    assert oracle.pick_split(np.full(75, 1, np.int32), **many) == 1
+    assert oracle.pick_split(np.full(74, 1, np.int32), **many) == 2
+    # a 129-row expert is two m-tiles
+    assert oracle.pick_split(np.int32([129]), **dict(many, num_sms=4)) == 2
+    # no split for formats without one, nor for an empty batch
+    assert oracle.pick_split(counts, **dict(mix, split_nb=0)) == 1
+    assert oracle.pick_split(np.zeros(8, np.int32), **mix) == 1
+
+
 # ------------------------------------------------------------------ MX32 hidden rule
 def test_mx32_quant_hand_example():
     x = np.zeros((4, 64), np.float32)
