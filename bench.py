@@ -142,12 +142,25 @@ def run_ours(args, rank, world, local_rank):
     y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
+    def call():
         native.moe_forward(layer.h, x, T, wr, bias, layer.packed, y, layer.ws)
 
+    step = call
     for _ in range(args.warmup):
-        step()
+        call()
     torch.cuda.synchronize()
+    graph = None
+    if args.launch == "graph":
+        # the layer call, captured once and replayed: the same kernels with the
+        # same arguments, minus the host's per-launch cost
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        torch.cuda.synchronize()
+        step = graph.replay
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
     st, msg = layer.status()
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {msg}")
@@ -294,6 +307,8 @@ def run_ours(args, rank, world, local_rank):
                    "T_per_gpu": T, "parallelism": f"replicas x{world} (token batches)",
                    "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (byts / 1e9),
                    "touched_experts": touched, "m_tiles": m_tiles,
+                   "launch": "CUDA graph of one moe_forward call, replayed per step" if graph is not None
+                             else "moe_forward per step",
                    "down_tile": args.down_bn or {0: 256, 1: 128, 2: 64}[pick],
                    "down_tile_source": "fixed" if args.down_bn else "picked from the histogram"},
         "tflops": (fl_t + fl_r) * world * args.steps / (ms_max * 1e-3) / 1e12,
@@ -314,6 +329,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": (10 if wl.fmt == FMT_NVFP4 else 9) * args.steps,
         "clocks": clk.summary(),
     }
+    del graph
     layer.close()
     return out
 
@@ -374,6 +390,8 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--down-bn", type=int, default=0, help="down GEMM tile width (0 = chosen per call)")
+    ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
+                    help="timed steps replay a CUDA graph of the layer call, or call it directly")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

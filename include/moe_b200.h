@@ -94,7 +94,8 @@ typedef struct {
     int32_t* offsets;    /* [E+1] exclusive prefix sum of counts (m_indptr) */
     int32_t* num_tiles;  /* [1] row tiles of 128 over all experts */
     int32_t* tile_ptr;   /* [E+1] index of each expert's first row tile */
-    int32_t* pick;       /* [1] down GEMM tile chosen from the histogram: 0 -> 256, 1 -> 128, 2 -> 64 columns */
+    int32_t* pick;       /* [2] choices from the histogram: [0] down GEMM tile (0 -> 256, 1 -> 128, 2 -> 64
+                          * columns, FP8_BLOCK128); [1] S, the K split of the FP8_ROW down GEMM (1 = none) */
     int32_t* tiles;      /* [A/128 + E + 1][2] (expert, first row) per row tile */
     int32_t* perm;       /* [A] slot -> t*k + j */
     int32_t* inv;        /* [A] t*k + j -> slot */
@@ -103,7 +104,10 @@ typedef struct {
     void*    xs;         /* scales of xq: [A] fp32 | [A, H/128] fp32 | [A, H/16] e4m3 */
     uint8_t* hq;         /* [A, I] (NVFP4: [A, I/2]) requantised hidden */
     void*    hs;         /* scales of hq: [A, I/128] fp32 | [A, I/16] e4m3 */
-    float*   o;          /* [A, H] fp32 down projection times routing weight, slot order */
+    float*   o;          /* [S][T*k, H] fp32 down projection times routing weight, slot order; with a K
+                          * split (pick[1] = S > 1) copy s holds split s's partial sums.  FP8_ROW
+                          * workspaces hold A + 7 min(A, 256) rows so small batches can split. */
+    float*   logits;     /* [max_T, E] fp32 router logits (bias included) of the last moe_route */
 } moe_workspace_view;
 
 const char* moe_last_error(void);
@@ -183,6 +187,15 @@ moe_status moe_down(const moe_handle* h, const void* packed, const float* w, int
  * 128, 256 output columns per tile.  Host state only. */
 moe_status moe_set_tile_config(moe_handle* h, int down_bn);
 
+/* Launch option of every kernel the layer calls (no counterpart in the pages:
+ * a property of how the kernels are issued, not of what they compute).
+ * pdl = 1 (the default) launches each kernel with programmatic dependent
+ * launch allowed: it may be scheduled while the previous kernel in the stream
+ * finishes, and orders its memory accesses after that kernel's on the device,
+ * so results are identical with either setting.  pdl = 0 launches them in
+ * plain stream order.  Host state only; MOE_ERR_INVALID_ARG for other values. */
+moe_status moe_set_launch_options(moe_handle* h, int pdl);
+
 /* Parameters of the wave cost model that picks the down GEMM's tile width
  * from the runtime expert histogram (RaMP abstract: four-parameter wave cost
  * model fitted from a one-time profiling sweep).  The dispatch's scan kernel
@@ -190,7 +203,11 @@ moe_status moe_set_tile_config(moe_handle* h, int down_bn);
  *   t_mma  = ceil(m_tiles*(H/BN) / num_sms) * (I/128) * (alpha + beta*BN)
  *   t_load = touched_experts*H*I*1e6 / (min(m_tiles*(H/BN), num_sms) * bw)
  *   cost   = gamma + max(t_mma, t_load)     (integers: picoseconds, bytes/us)
- * and writes the cheapest (the wider on ties) to view.pick.
+ * and writes the cheapest (the wider on ties) to view.pick[0].
+ * For FP8_ROW it also writes view.pick[1] = S, the K split of the down GEMM
+ * (no parameters): with units = m_tiles * (H/256), A = T*k and
+ * s_max = min(8, o_rows / A, (I/128) / 4), S is the largest s <= s_max with
+ * units * s <= num_sms, else 1 (o_rows = A_max + 7 min(A_max, 256)).
  * params = {alpha, beta, bw, gamma}; get also returns num_sms in params[4]. */
 moe_status moe_set_picker_params(moe_handle* h, const long long* params);
 moe_status moe_get_picker_params(const moe_handle* h, long long* params);

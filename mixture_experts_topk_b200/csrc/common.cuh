@@ -22,6 +22,17 @@ __device__ __forceinline__ void report(int32_t* status, int code, int where) {
     if (atomicCAS(status, 0, code) == 0) status[1] = where;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the layer calls pdl_wait() before its first global-memory
+// access: it returns once the preceding kernel in the stream has completed and
+// its writes are visible (at once for a launch without the PDL attribute).
+// Since each kernel waits for its predecessor before it can complete, the
+// chain orders every kernel after all earlier ones.  pdl_trigger() lets the
+// next kernel be scheduled now, so its launch and prologue (barrier init, TMEM
+// allocation, tensor-map prefetch) overlap this kernel's tail.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -35,7 +35,31 @@ struct PickerParams {
     long long bw_cta;          // weight bytes per microsecond one CTA streams
     long long gamma_ps;        // launch constant
     int num_sms, H, I;
+    int split_nb;              // n-blocks of a K-splittable down GEMM (0: no split)
+    int split_kb;              // its K-blocks
+    int o_rows;                // rows of the fp32 down-output buffer
 };
+
+// Split of the down GEMM's K for small batches: when the (m-tile, n-block)
+// units leave SMs idle, each unit's K-blocks are cut into S near-equal ranges
+// run by different CTAs, whose fp32 partial rows go to S copies of the output
+// rows that the combine adds in fixed order.  Integer rule:
+//   units = m_tiles * split_nb,  s_max = min(8, o_rows / A, split_kb / 4)
+//   S = the largest s <= s_max with units * s <= num_sms, else 1.
+__host__ __device__ inline int split_limit(const PickerParams& q, int A) {
+    if (q.split_nb <= 0 || A <= 0) return 1;
+    int m = q.o_rows / A;
+    if (q.split_kb / 4 < m) m = q.split_kb / 4;
+    if (m > 8) m = 8;
+    return m < 1 ? 1 : m;
+}
+__host__ __device__ inline int pick_split(const PickerParams& q, int m_tiles, int A) {
+    const int smax = split_limit(q, A);
+    const long long units = static_cast<long long>(m_tiles) * q.split_nb;
+    int S = 1;
+    while (S < smax && units * (S + 1) <= q.num_sms) S++;
+    return S;
+}
 constexpr int PICK_NUM = 3;
 __host__ __device__ constexpr int pick_bn(int c) { return c == 0 ? 256 : (c == 1 ? 128 : 64); }
 
@@ -61,6 +85,8 @@ __device__ __forceinline__ int pick_down_tile(const PickerParams& q, int m_tiles
 
 __global__ void __launch_bounds__(DISPATCH_CHUNK)
     hist_kernel(const int32_t* ids, int A, int E, int32_t* chunk_counts, int32_t* status) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int h[256];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
@@ -77,57 +103,75 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
 // One CTA: counts, offsets (exclusive scan), per-chunk bases (written over the
 // chunk counts), the row-tile table (expert, first row) in expert order, and
 // tile_ptr[e] = index of expert e's first row tile (may be null), and the down
-// GEMM's tile choice from the histogram (pick_out, may be null).
+// GEMM's tile choice and K split from the histogram (pick_out[0], pick_out[1];
+// may be null).  One exclusive block scan over experts of the packed pair
+// (count, row tiles): count < 2^20, so count + (tiles << 20) cannot carry.
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
                                                    int32_t* offsets, int32_t* tiles, int32_t* num_tiles,
                                                    int32_t* tile_ptr, int32_t* pick_out, PickerParams pq) {
-    __shared__ int s_cnt[256], s_off[257], s_tptr[257];
-    const int e = threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
+    __shared__ int warp_tot[8];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     int c = 0;
-    if (e < E)
+    if (e < E) {
+#pragma unroll 8
         for (int ch = 0; ch < nchunks; ch++) c += chunk_counts[ch * E + e];
-    s_cnt[e] = c;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0, trun = 0;
-        for (int i = 0; i < E; i++) {
-            s_off[i] = run;
-            s_tptr[i] = trun;
-            run += s_cnt[i];
-            trun += (s_cnt[i] + TILE_M - 1) / TILE_M;
+    }
+    const int nt_e = (c + TILE_M - 1) / TILE_M;
+    const int packed = c + (nt_e << 20);
+    int inc = packed;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += n;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    const int touched = __syncthreads_count(e < E && c > 0);
+    if (warp == 0) {
+        int w = lane < 8 ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += n;
         }
-        s_off[E] = run;
-        s_tptr[E] = trun;
-        offsets[E] = run;
+        if (lane < 8) warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int excl = (warp ? warp_tot[warp - 1] : 0) + inc - packed;
+    const int total = warp_tot[7];
+    const int off_e = excl & 0xFFFFF, tptr_e = excl >> 20;
+    const int A = total & 0xFFFFF, trun = total >> 20;
+    if (e == 0) {
+        offsets[E] = A;
         *num_tiles = trun;
         if (tile_ptr) tile_ptr[E] = trun;
         if (pick_out) {
-            int touched = 0;
-            for (int i = 0; i < E; i++) touched += s_cnt[i] > 0;
             pick_out[0] = pick_down_tile(pq, trun, touched);
+            pick_out[1] = pick_split(pq, trun, A);
         }
     }
-    __syncthreads();
     if (e < E) {
         counts[e] = c;
-        offsets[e] = s_off[e];
-        if (tile_ptr) tile_ptr[e] = s_tptr[e];
-        int run = s_off[e];
+        offsets[e] = off_e;
+        if (tile_ptr) tile_ptr[e] = tptr_e;
+        int run = off_e;
         for (int ch = 0; ch < nchunks; ch++) {
             const int v = chunk_counts[ch * E + e];
             chunk_counts[ch * E + e] = run;
             run += v;
         }
-        const int nt = s_tptr[e + 1] - s_tptr[e];
-        for (int i = 0; i < nt; i++) {
-            tiles[2 * (s_tptr[e] + i)] = e;
-            tiles[2 * (s_tptr[e] + i) + 1] = s_off[e] + TILE_M * i;
+        for (int i = 0; i < nt_e; i++) {
+            tiles[2 * (tptr_e + i)] = e;
+            tiles[2 * (tptr_e + i) + 1] = off_e + TILE_M * i;
         }
     }
 }
 
 __global__ void __launch_bounds__(DISPATCH_CHUNK)
     rank_kernel(const int32_t* ids, int A, int E, const int32_t* chunk_base, int32_t* perm, int32_t* inv) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int wc[32][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) wc[i >> 8][i & 255] = 0;
@@ -168,6 +212,8 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
 template <int FMT>
 __global__ void __launch_bounds__(256) quant_scatter_kernel(const __nv_bfloat16* x, int T, int H, int k,
                                                             const int32_t* inv, uint8_t* xq, float* xs) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int nI = H >> 8;
     for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
@@ -226,11 +272,90 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(const __nv_bfloat16*
     }
 }
 
-// y[t] = bf16(sum_j o[inv[t k + j]]) in fixed j order with fp32 accumulation;
-// o holds fp32 rows (weight already applied), so the only rounding to bf16 is
-// the final one.
+// Small batches: the same quantisation with one 256-thread CTA per token, so a
+// row's loads are spread over 8 warps.  Thread i handles columns 8 (i + 256 m);
+// a 128-column block is 16 consecutive lanes, the row amax (FP8_ROW) is a
+// warp then CTA maximum.  Same operations per element as quant_scatter_kernel.
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_scatter_row_kernel(const __nv_bfloat16* x, int T, int H, int k,
+                                                                const int32_t* inv, uint8_t* xq, float* xs) {
+    pdl_wait();
+    pdl_trigger();
+    __shared__ float s_amax[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        int slot[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
+        const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
+        float s_row = 0.0f;
+        if (FMT == 0) {
+            float amax = 0.0f;
+            for (int m = 0; 8 * (tid + 256 * m) < H; m++) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + 8 * (tid + 256 * m)));
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            if (lane == 0) s_amax[warp] = amax;
+            __syncthreads();
+            amax = s_amax[0];
+#pragma unroll
+            for (int w = 1; w < 8; w++) amax = fmaxf(amax, s_amax[w]);
+            __syncthreads();   // s_amax is rewritten for the next token
+            s_row = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (j == tid && slot[j] >= 0) xs[slot[j]] = s_row;
+        }
+        for (int m = 0; 8 * (tid + 256 * m) < H; m++) {
+            const int c0 = 8 * (tid + 256 * m);
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + c0));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            float s = s_row;
+            if (FMT == 1) {
+                float amax = 0.0f;
+#pragma unroll
+                for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                s = __fdiv_rn(amax, 448.0f);
+                if ((lane & 15) == 0) {
+#pragma unroll
+                    for (int j = 0; j < 8; j++)
+                        if (slot[j] >= 0) xs[static_cast<size_t>(slot[j]) * (H >> 7) + (c0 >> 7)] = s;
+                }
+            }
+            uint32_t packed[2];
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const float a = bf16_lo(u[q]), b = bf16_hi(u[q]);
+                const uint16_t c = (s == 0.0f) ? static_cast<uint16_t>(0)
+                                               : f2_to_e4m3x2(__fdiv_rn(a, s), __fdiv_rn(b, s));
+                if (q & 1) packed[q >> 1] |= static_cast<uint32_t>(c) << 16;
+                else packed[q >> 1] = c;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (slot[j] >= 0)
+                    *reinterpret_cast<uint2*>(xq + static_cast<size_t>(slot[j]) * H + c0) =
+                        make_uint2(packed[0], packed[1]);
+        }
+    }
+}
+
+// y[t] = bf16(sum_j sum_s o[s][inv[t k + j]]) in fixed (j, s) order with fp32
+// accumulation; o holds fp32 rows (weight already applied) in S copies of A
+// rows when the down GEMM split its K (S from the dispatch's pick, clamped to
+// [1, s_max]), so the only rounding to bf16 is the final one.
 __global__ void __launch_bounds__(128) combine_kernel(const float* o, const int32_t* inv, int T, int H, int k,
-                                                      __nv_bfloat16* y) {
+                                                      const int32_t* split, int s_max, __nv_bfloat16* y) {
+    pdl_wait();
+    pdl_trigger();
+    const int S = split ? min(max(*split, 1), s_max) : 1;
+    const size_t copy = static_cast<size_t>(T) * k * H;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         int slot[8];
 #pragma unroll
@@ -240,10 +365,13 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* o, const int3
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 if (slot[j] < 0) continue;
-                const float4* src = reinterpret_cast<const float4*>(o + static_cast<size_t>(slot[j]) * H + c0);
-                const float4 a = src[0], b = src[1];
-                acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-                acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+                const float* row = o + static_cast<size_t>(slot[j]) * H + c0;
+                for (int sp = 0; sp < S; sp++) {
+                    const float4* src = reinterpret_cast<const float4*>(row + sp * copy);
+                    const float4 a = src[0], b = src[1];
+                    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+                    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+                }
             }
             uint32_t r[4];
 #pragma unroll
@@ -281,6 +409,8 @@ __global__ void interleave_rows_kernel(const uint32_t* gate, const uint32_t* up,
 // Global scale of X: g = amax(|X|) / (448 * 6).  amax as the bit pattern of a
 // non-negative float, so an integer max gives the float max (order-free).
 __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* x, long long n8, int32_t* amax_bits) {
+    pdl_wait();
+    pdl_trigger();
     float m = 0.0f;
     for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n8; i += 256LL * gridDim.x) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
@@ -302,6 +432,8 @@ __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* x, long 
 __global__ void __launch_bounds__(256) quant_scatter_nvfp4_kernel(
     const __nv_bfloat16* x, int T, int H, int k, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
     const int32_t* tile_ptr, const int32_t* amax_bits, uint8_t* xq, uint8_t* xsf) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int nI = H >> 8;
     const float g = __fdiv_rn(__int_as_float(*amax_bits), 2688.0f);

@@ -66,6 +66,9 @@ struct GemmParams {
     long long spin_limit;
 };
 
+constexpr int TMAP_STRIDE = 260;              // shared-memory tile map: 2 x (E + 1) ints, E <= 256
+constexpr int TMAP_BYTES = 2 * TMAP_STRIDE * 4;
+
 template <int BN, int STAGES>
 struct GemmSmem {
     // accumulator buffers in TMEM (512 columns): deeper for narrower tiles, so the
@@ -80,19 +83,34 @@ struct GemmSmem {
     static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int XCHG_OFF = (TMEM_SLOT_OFF + 4 + 15) / 16 * 16;
     static constexpr int XCHG_BYTES = 2 * 2 * 128 * 4 * 2;   // [parity][group][row] value + flag
-    static constexpr int TOTAL = XCHG_OFF + XCHG_BYTES + 1024; // + alignment slack
+    static constexpr int TMAP_OFF = XCHG_OFF + XCHG_BYTES;
+    static constexpr int TOTAL = TMAP_OFF + TMAP_BYTES + 1024; // + alignment slack
 };
 
-// Tile t -> (m-tile index, n-block): expert e owns tiles [tile_ptr[e] nb, tile_ptr[e+1] nb).
-__device__ __forceinline__ void decode_tile(int t, const int32_t* tile_ptr, int E, int n_blocks, int& mi, int& nb) {
+// The schedule's tile pointers and row offsets, copied into shared memory once
+// per CTA (after the dispatch wrote them), so decoding a tile is a few
+// shared-memory reads instead of a chain of dependent global loads.
+// Layout: tile_ptr[0..E] at s[0..], offsets[0..E] at s[TMAP_STRIDE..].
+__device__ __forceinline__ void stage_tile_map(int32_t* s, const int32_t* tile_ptr, const int32_t* offsets, int E) {
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+        s[i] = tile_ptr[i];
+        s[TMAP_STRIDE + i] = offsets[i];
+    }
+}
+
+// Tile t -> (expert, m-tile index, n-block): expert e owns tiles
+// [tile_ptr[e] nb, tile_ptr[e+1] nb), n-block-major with its m-tiles fastest.
+__device__ __forceinline__ void decode_tile(int t, const int32_t* s_tptr, int E, int n_blocks, int& e, int& mi,
+                                            int& nb) {
     int lo = 0, hi = E;   // tile_ptr[lo] * n_blocks <= t < tile_ptr[hi] * n_blocks
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (__ldg(tile_ptr + mid) * n_blocks <= t) lo = mid; else hi = mid;
+        if (s_tptr[mid] * n_blocks <= t) lo = mid; else hi = mid;
     }
-    const int first = __ldg(tile_ptr + lo);
-    const int mt = __ldg(tile_ptr + lo + 1) - first;
+    const int first = s_tptr[lo];
+    const int mt = s_tptr[lo + 1] - first;
     const int local = t - first * n_blocks;
+    e = lo;
     nb = local / mt;
     mi = first + local % mt;
 }
@@ -142,6 +160,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    pdl_wait();
+    pdl_trigger();
+    int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + S::TMAP_OFF);
+    const int32_t* s_off = s_tptr + TMAP_STRIDE;
+    stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
+    __syncthreads();
     const int ntm = *p.num_tiles;
     const int total = ntm * n_blocks;
     const long long limit = p.spin_limit;
@@ -152,9 +176,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                int mi, nb;
-                decode_tile(t, p.tile_ptr, p.E, n_blocks, mi, nb);
-                const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
+                int e, mi, nb;
+                decode_tile(t, s_tptr, p.E, n_blocks, e, mi, nb);
+                const int row0 = s_off[e] + GEMM_BM * (mi - s_tptr[e]);
                 const int brow = e * p.b_rows + nb * BN;
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
                     const int s = it % STAGES;
@@ -228,20 +252,29 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
         uint32_t u = 0, iter = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, iter++) {
-            int mi, nb;
-                decode_tile(t, p.tile_ptr, p.E, n_blocks, mi, nb);
-            const int e = p.tiles[2 * mi], row0 = p.tiles[2 * mi + 1];
+            int e, mi, nb;
+            decode_tile(t, s_tptr, p.E, n_blocks, e, mi, nb);
+            const int row0 = s_off[e] + GEMM_BM * (mi - s_tptr[e]);
             const int row = row0 + r;
-            const bool valid = row < p.offsets[e + 1];
+            const bool valid = row < s_off[e + 1];
 
             if (KIND == KIND_GATE_UP) {
                 float hv[64];
                 if (!PROMOTE) {
+                    // scales are loaded while the tile's MMAs run: the row's X scale,
+                    // and lane c holds the weight scale of column c of each 32-column
+                    // half (read back with a shuffle)
+                    const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld] : 0.0f;
+                    const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + nb * BN;
+                    float bsg[2], bsu[2];
+#pragma unroll
+                    for (int half = 0; half < 2; half++) {
+                        bsg[half] = __ldg(bs + 64 * g + 32 * half + lane);
+                        bsu[half] = __ldg(bs + 128 + 64 * g + 32 * half + lane);
+                    }
                     const uint32_t acc = u % NBUF;
                     if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
-                    const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld] : 0.0f;
-                    const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + nb * BN;
 #pragma unroll
                     for (int half = 0; half < 2; half++) {
                         float gv[32], uv[32];
@@ -249,8 +282,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, gv, uv);
 #pragma unroll
                         for (int c = 0; c < 32; c++) {
-                            const float gg = gv[c] * (sa * __ldg(bs + c0 + c));
-                            const float uu = uv[c] * (sa * __ldg(bs + 128 + c0 + c));
+                            const float gg = gv[c] * (sa * __shfl_sync(0xffffffffu, bsg[half], c));
+                            const float uu = uv[c] * (sa * __shfl_sync(0xffffffffu, bsu[half], c));
                             hv[32 * half + c] = gg / (1.0f + expf(-gg)) * uu;
                         }
                     }
@@ -367,6 +400,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 #pragma unroll
                 for (int c = 0; c < NC; c++) acc_r[c] = 0.0f;
                 const int n0 = nb * BN + g * NC;
+                const float rw = valid ? p.route_w[p.perm[row]] : 0.0f;   // loaded while the MMAs run
                 const float* arow = p.a_scale + static_cast<size_t>(valid ? row : 0) * p.a_ld;
                 const float* bsb = p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + n0 / 128) * p.num_kb;
                 // the scale of the next K-block is loaded before waiting on this one
@@ -406,7 +440,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                 }
                 if (!ok) break;
                 if (valid) {
-                    const float rw = p.route_w[p.perm[row]];
                     const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + n0;
                     float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(row) * p.H + n0);
 #pragma unroll
@@ -458,6 +491,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                           const __grid_constant__ CUtensorMap tmB128, const __grid_constant__ CUtensorMap tmB64,
                           const GemmParams p, const int32_t* cfg) {
     extern __shared__ uint8_t smem_raw[];
+    pdl_wait();   // the tile width was picked by the dispatch scan
     const int c = *cfg;
     if (c == 1)
         gemm_body<KIND_DOWN, BSCALE, true, 128, 6>(tmA, tmB128, p, p.H / 128, smem_raw);

@@ -37,7 +37,8 @@ constexpr int F4_SF_TMEM = F4_NBUF * F4_BN;       // first column of the scale-f
 constexpr int F4_BAR_OFF = F4_STAGES * F4_STAGE_BYTES;
 constexpr int F4_NUM_BARS = 2 * F4_STAGES + 2 * F4_NBUF + 1;
 constexpr int F4_TMEM_SLOT_OFF = F4_BAR_OFF + 8 * F4_NUM_BARS;
-constexpr int F4_SMEM = F4_TMEM_SLOT_OFF + 16 + 1024;
+constexpr int F4_TMAP_OFF = F4_TMEM_SLOT_OFF + 16;
+constexpr int F4_SMEM = F4_TMAP_OFF + TMAP_BYTES + 1024;
 static_assert(F4_SF_TMEM + 32 * F4_STAGES <= 512, "TMEM columns");
 
 struct Fp4Params {
@@ -100,6 +101,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+    int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + F4_TMAP_OFF);
+    const int32_t* s_off = s_tptr + TMAP_STRIDE;
+    stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
+    __syncthreads();
     const int ntm = *p.num_tiles;
     const int total = ntm * p.n_blocks;
     const long long limit = p.spin_limit;
@@ -110,9 +117,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                int mi, nb;
-                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
-                const int e = p.tiles[2 * mi];
+                int e, mi, nb;
+                decode_tile(t, s_tptr, p.E, p.n_blocks, e, mi, nb);
                 const int brow = e * p.b_rows + nb * F4_BN;
                 const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.sf_cols * 128;
                 const uint8_t* sfb = p.sfb + static_cast<size_t>(e) * p.b_rows * p.sf_cols +
@@ -184,12 +190,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t u = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            int mi, nb;
-            decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
-            const int e = p.tiles[2 * mi];
+            int e, mi, nb;
+            decode_tile(t, s_tptr, p.E, p.n_blocks, e, mi, nb);
             const long long prow = static_cast<long long>(mi) * 128 + r;
-            const int local = static_cast<int>(prow - static_cast<long long>(p.tile_ptr[e]) * 128);
-            const bool valid = local < p.offsets[e + 1] - p.offsets[e];
+            const int local = static_cast<int>(prow - static_cast<long long>(s_tptr[e]) * 128);
+            const bool valid = local < s_off[e + 1] - s_off[e];
+            // loaded while the tile's MMAs run
+            const int slot = s_off[e] + local;
+            const float gx = __fdiv_rn(__int_as_float(*p.x_amax), 2688.0f);
+            const float wg0 = __ldg(p.w_global + (KIND == KIND_GATE_UP ? 2 * e : e));
+            const float wg1 = KIND == KIND_GATE_UP ? __ldg(p.w_global + 2 * e + 1) : 0.0f;
+            const float rw = (KIND == KIND_DOWN && valid) ? p.route_w[p.perm[slot]] : 0.0f;
             const uint32_t acc = u % F4_NBUF;
             if (!warp_wait(&tfull[acc], (u / F4_NBUF) & 1, limit)) { ok = false; break; }
             tc_fence_after();
@@ -200,8 +211,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[acc]);
                 u++;
-                const float gx = __fdiv_rn(__int_as_float(*p.x_amax), 2688.0f);
-                const float sg = gx * __ldg(p.w_global + 2 * e), su = gx * __ldg(p.w_global + 2 * e + 1);
+                const float sg = gx * wg0, su = gx * wg1;
                 float hv[32];
 #pragma unroll
                 for (int c = 0; c < 32; c++) {
@@ -242,8 +252,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (lane == 0) mbar_arrive(&tempty[acc]);
                 u++;
                 if (valid) {
-                    const int slot = p.offsets[e] + local;
-                    const float sc = p.h_global * __ldg(p.w_global + e) * p.route_w[p.perm[slot]];
+                    const float sc = p.h_global * wg0 * rw;
                     float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + 64 * g);
 #pragma unroll
                     for (int c = 0; c < 32; c += 4) {

@@ -9,7 +9,10 @@
 // their MX scale is the constant 1 (UE8M0 127), copied into TMEM once.
 //
 // Tile 128 padded rows x 256 columns, K stage 128 (one 512-byte scale chunk of
-// A per stage: 4 scales of 32 per row), 4 stages.  MMA j of a stage (K = 32)
+// A per stage: 4 scales of 32 per row), 4 stages.  For small batches the K
+// range of each tile may be split S ways (S read from the dispatch's pick,
+// work unit = (split, tile)); split s writes its fp32 partial rows to copy s
+// of the output rows, o + s * A * H.  MMA j of a stage (K = 32)
 // uses byte j of the chunk (scale-factor id j).  TMEM: one 256-column
 // accumulator, released as soon as the epilogue has it in registers, then the
 // A-scale ring and the constant B-scale chunks.
@@ -29,7 +32,8 @@ constexpr int MX_SFB_OFF = MX_STAGES * MX_STAGE_BYTES;            // 2 constant 
 constexpr int MX_BAR_OFF = MX_SFB_OFF + 1024;
 constexpr int MX_NUM_BARS = 2 * MX_STAGES + 3;
 constexpr int MX_TMEM_SLOT_OFF = MX_BAR_OFF + 8 * MX_NUM_BARS;
-constexpr int MX_SMEM = MX_TMEM_SLOT_OFF + 16 + 1024;
+constexpr int MX_TMAP_OFF = MX_TMEM_SLOT_OFF + 16;
+constexpr int MX_SMEM = MX_TMAP_OFF + TMAP_BYTES + 1024;
 constexpr int MX_SFA_TMEM = MX_BN;                    // 4 columns per stage
 constexpr int MX_SFB_TMEM = MX_BN + 4 * MX_STAGES;    // 8 columns (two 128-row chunks)
 
@@ -63,8 +67,11 @@ struct MxDownParams {
     int b_rows;                // H
     const uint8_t* sfa;        // hidden MX scales, chunked by padded row tile (I / 32 per row)
     const float* w_scale;      // [E][H] fp32 per output row of W_down
-    float* o;                  // [A][H] fp32 rows in slot order
+    float* o;                  // [S][A][H] fp32 rows in slot order
     int H;
+    int A;                     // assignments T * k
+    const int32_t* split;      // S, the K split chosen by the dispatch's scan
+    int s_max;                 // S is clamped to [1, s_max] (s_max * A rows fit in o)
     const int32_t* perm;
     const float* route_w;
     int32_t* status;
@@ -107,8 +114,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+    int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + MX_TMAP_OFF);
+    const int32_t* s_off = s_tptr + TMAP_STRIDE;
+    stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
+    __syncthreads();
     const int ntm = *p.num_tiles;
-    const int total = ntm * p.n_blocks;
+    const int units = ntm * p.n_blocks;
+    const int S = min(max(*p.split, 1), p.s_max);
+    const int total = units * S;
     const long long limit = p.spin_limit;
 
     if (warp == 0) {
@@ -117,12 +132,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                int mi, nb;
-                decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
-                const int e = p.tiles[2 * mi];
+                const int sp = t / units;
+                int e, mi, nb;
+                decode_tile(t - sp * units, s_tptr, p.E, p.n_blocks, e, mi, nb);
                 const int brow = e * p.b_rows + nb * MX_BN;
                 const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.num_kb * 512;
-                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                const int kb1 = (sp + 1) * p.num_kb / S;
+                for (int kb = sp * p.num_kb / S; kb < kb1; kb++, it++) {
                     const int s = it % MX_STAGES;
                     if (!mbar_wait(&empty[s], ((it / MX_STAGES) & 1) ^ 1, limit)) {
                         report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
@@ -148,9 +164,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0, u = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const int sp = t / units;
+                const int kb0 = sp * p.num_kb / S, kb1 = (sp + 1) * p.num_kb / S;
                 if (!mbar_wait(tempty, (u & 1) ^ 1, limit)) { ok = false; break; }
                 tc_fence_after();
-                for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                for (int kb = kb0; kb < kb1; kb++, it++) {
                     const int s = it % MX_STAGES;
                     if (!mbar_wait(&full[s], (it / MX_STAGES) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
@@ -161,7 +179,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 4; j++)
                         mma_mxf8(tmem_base, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
-                                 idesc_mxf8(128, MX_BN, j), sfa, sfb, (kb > 0 || j > 0));
+                                 idesc_mxf8(128, MX_BN, j), sfa, sfb, (kb > kb0 || j > 0));
                     mma_commit(&empty[s]);
                 }
                 if (!ok) break;
@@ -181,11 +199,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t u = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            int mi, nb;
-            decode_tile(t, p.tile_ptr, p.E, p.n_blocks, mi, nb);
-            const int e = p.tiles[2 * mi];
-            const int local = mi * 128 + r - p.tile_ptr[e] * 128;
-            const bool valid = local < p.offsets[e + 1] - p.offsets[e];
+            const int sp = t / units;
+            int e, mi, nb;
+            decode_tile(t - sp * units, s_tptr, p.E, p.n_blocks, e, mi, nb);
+            const int local = mi * 128 + r - s_tptr[e] * 128;
+            const bool valid = local < s_off[e + 1] - s_off[e];
+            // loaded while the tile's MMAs run: the row's routing weight, and lane l
+            // holds the weight scales of columns 4l .. 4l+3 (read back by shuffle)
+            const int slot = s_off[e] + local;
+            const float rw = valid ? p.route_w[p.perm[slot]] : 0.0f;
+            const int n0 = nb * MX_BN + 128 * g;
+            const float4 ws4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + static_cast<size_t>(e) * p.H + n0) + lane);
             if (!warp_wait(tfull, u & 1, limit)) { ok = false; break; }
             tc_fence_after();
             float v[128];
@@ -197,18 +221,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty);   // the next tile's MMAs may start
             u++;
-            if (valid) {
-                const int slot = p.offsets[e] + local;
-                const float rw = p.route_w[p.perm[slot]];
-                const int n0 = nb * MX_BN + 128 * g;
-                const float* ws = p.w_scale + static_cast<size_t>(e) * p.H + n0;
-                float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(slot) * p.H + n0);
+            float4* dst = reinterpret_cast<float4*>(p.o + (static_cast<size_t>(sp) * p.A + slot) * p.H + n0);
 #pragma unroll
-                for (int c = 0; c < 128; c += 4) {
-                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(ws + c));
-                    dst[c / 4] = make_float4(v[c] * s4.x * rw, v[c + 1] * s4.y * rw, v[c + 2] * s4.z * rw,
-                                             v[c + 3] * s4.w * rw);
-                }
+            for (int c = 0; c < 128; c += 4) {
+                const float sx = __shfl_sync(0xffffffffu, ws4.x, c / 4), sy = __shfl_sync(0xffffffffu, ws4.y, c / 4);
+                const float sz = __shfl_sync(0xffffffffu, ws4.z, c / 4), sw = __shfl_sync(0xffffffffu, ws4.w, c / 4);
+                if (valid)
+                    dst[c / 4] = make_float4(v[c] * sx * rw, v[c + 1] * sy * rw, v[c + 2] * sz * rw, v[c + 3] * sw * rw);
             }
         }
         if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_EPILOGUE);

@@ -46,6 +46,34 @@ static moe_status fail(moe_status st, const char* fmt, ...) {
 
 extern "C" const char* moe_last_error(void) { return g_err; }
 
+// Launch a kernel of the layer.  With pdl set the launch carries the
+// programmatic-stream-serialization attribute: the kernel may be scheduled
+// while its predecessor finishes, and its own pdl_wait() orders its memory
+// accesses after that predecessor's.
+template <typename... KP, typename... Args>
+static cudaError_t launch_k(bool pdl, void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args&&... args) {
+    cudaLaunchConfig_t lc;
+    memset(&lc, 0, sizeof(lc));
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+}
+
+#define LAUNCH(pdl, name, kern, grid, block, smem, st, ...)                                  \
+    do {                                                                                     \
+        cudaError_t err_ = launch_k((pdl), kern, dim3(grid), dim3(block), (smem), (st), __VA_ARGS__); \
+        if (err_ != cudaSuccess)                                                             \
+            return fail(MOE_ERR_CUDA, "launch of %s failed: %s", name, cudaGetErrorString(err_)); \
+    } while (0)
+
 // ------------------------------------------------------------------ layouts
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -65,6 +93,7 @@ struct moe_handle {
     long long spin_limit;
     int down_bn;          // 0 = picked per call, else 64 / 128 / 256
     PickerParams picker;
+    int pdl;              // launch with programmatic dependent launch allowed
 };
 
 static size_t code_bytes(int fmt, int K) { return fmt == MOE_FMT_NVFP4 ? K / 2 : K; }
@@ -90,6 +119,13 @@ static size_t hidden_rows(const moe_config& c) {
     return c.fmt == MOE_FMT_FP8_BLOCK128 ? A : A + static_cast<size_t>(TILE_M) * c.E;
 }
 
+// rows of the fp32 down output: A, plus room for up to 8 K-split copies of
+// batches of at most 256 assignments where the down GEMM may split its K
+static size_t o_rows(const moe_config& c) {
+    const size_t A = static_cast<size_t>(c.max_T) * c.k;
+    return c.fmt == MOE_FMT_FP8_ROW ? A + 7 * std::min<size_t>(A, 256) : A;
+}
+
 static WsLayout make_ws_layout(const moe_config& c) {
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
     const size_t nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
@@ -109,7 +145,7 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.offsets = take((c.E + 1) * 4);
     L.num_tiles = take(4);
     L.tile_ptr = take((c.E + 1) * 4);
-    L.pick = take(4);
+    L.pick = take(8);
     L.chunk = take(nchunks * c.E * 4);
     L.tiles = take(tiles_cap * 8);
     L.perm = take(A * 4);
@@ -122,7 +158,7 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.xs = take(R * act_scale_bytes(c.fmt, c.H));
     L.hq = take(RH * code_bytes(c.fmt, c.I));
     L.hs = take(RH * hidden_scale_bytes(c.fmt, c.I));
-    L.o = take(A * c.H * 4);
+    L.o = take(o_rows(c) * c.H * 4);
     L.total = off;
     return L;
 }
@@ -188,8 +224,12 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
     h->picker.bw_cta = 38684;
     h->picker.gamma_ps = 17030139;
     h->picker.num_sms = h->num_sms;
+    h->pdl = 1;
     h->picker.H = c.H;
     h->picker.I = c.I;
+    h->picker.split_nb = c.fmt == MOE_FMT_FP8_ROW ? c.H / MX_BN : 0;
+    h->picker.split_kb = c.I / 128;
+    h->picker.o_rows = static_cast<int>(o_rows(c));
     *out = h;
     return MOE_OK;
 }
@@ -232,6 +272,7 @@ extern "C" moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_
     v->hq = b + L.hq;
     v->hs = b + L.hs;
     v->o = reinterpret_cast<float*>(b + L.o);
+    v->logits = reinterpret_cast<float*>(b + L.logits);
     return MOE_OK;
 }
 
@@ -325,18 +366,22 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
     p.k = h->cfg.k;
     p.score = h->cfg.score;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (h->cfg.E <= 8) {
+    if (T <= 128) {
+        LAUNCH(h->pdl, "router_logits_small_kernel", router_logits_small_kernel,
+               dim3((T + RS_TG - 1) / RS_TG, (h->cfg.E + RS_WARPS - 1) / RS_WARPS), RS_WARPS * 32, 0, st, p);
+    } else if (h->cfg.E <= 8) {
         using RT = RouterTile<64, 8>;
         CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<64, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, RT::SMEM));
-        router_logits_kernel<64, 8><<<dim3((T + 63) / 64, 1), RT_WARPS * 32, RT::SMEM, st>>>(p);
+        auto kern = router_logits_kernel<64, 8>;
+        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 63) / 64, 1), RT_WARPS * 32, RT::SMEM, st, p);
     } else {
         using RT = RouterTile<32, 16>;
         CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<32, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, RT::SMEM));
-        router_logits_kernel<32, 16><<<dim3((T + 31) / 32, (h->cfg.E + 15) / 16), RT_WARPS * 32, RT::SMEM, st>>>(p);
+        auto kern = router_logits_kernel<32, 16>;
+        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 31) / 32, (h->cfg.E + 15) / 16), RT_WARPS * 32,
+               RT::SMEM, st, p);
     }
-    LAUNCH_CHECK("router_logits_kernel");
-    router_topk_kernel<<<std::min((T + 7) / 8, 16 * h->num_sms), 256, 0, st>>>(p);
-    LAUNCH_CHECK("router_topk_kernel");
+    LAUNCH(h->pdl, "router_topk_kernel", router_topk_kernel, std::min((T + 7) / 8, 16 * h->num_sms), 256, 0, st, p);
     return MOE_OK;
 }
 
@@ -357,36 +402,37 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
     const int nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
     int32_t* chunk = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + h->ws.chunk);
     if (A > 0) {
-        hist_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.status);
-        LAUNCH_CHECK("hist_kernel");
+        LAUNCH(h->pdl, "hist_kernel", hist_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.status);
     }
-    scan_kernel<<<1, 256, 0, st>>>(chunk, nchunks, c.E, v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr,
-                                   v.pick, h->picker);
-    LAUNCH_CHECK("scan_kernel");
+    LAUNCH(h->pdl, "scan_kernel", scan_kernel, 1, 256, 0, st, chunk, nchunks, c.E, v.counts, v.offsets, v.tiles,
+           v.num_tiles, v.tile_ptr, v.pick, h->picker);
     if (A == 0) return MOE_OK;
-    rank_kernel<<<nchunks, DISPATCH_CHUNK, 0, st>>>(ids, A, c.E, chunk, v.perm, v.inv);
-    LAUNCH_CHECK("rank_kernel");
+    LAUNCH(h->pdl, "rank_kernel", rank_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.perm, v.inv);
     const int qgrid = std::min((T + 7) / 8, 8 * h->num_sms);
     if (c.fmt == MOE_FMT_NVFP4) {
         int32_t* amax = reinterpret_cast<int32_t*>(v.x_global);
         CUDA_TRY(cudaMemsetAsync(amax, 0, sizeof(int32_t), st));
         const long long n8 = static_cast<long long>(T) * c.H / 8;
-        amax_kernel<<<static_cast<int>(std::min<long long>((n8 + 255) / 256, 4LL * h->num_sms)), 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(x), n8, amax);
-        LAUNCH_CHECK("amax_kernel");
-        quant_scatter_nvfp4_kernel<<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, ids,
-                                                          v.inv, v.offsets, v.tile_ptr, amax, v.xq,
-                                                          static_cast<uint8_t*>(v.xs));
-        LAUNCH_CHECK("quant_scatter_nvfp4_kernel");
+        LAUNCH(h->pdl, "amax_kernel", amax_kernel,
+               static_cast<int>(std::min<long long>((n8 + 255) / 256, 4LL * h->num_sms)), 256, 0, st,
+               static_cast<const __nv_bfloat16*>(x), n8, amax);
+        LAUNCH(h->pdl, "quant_scatter_nvfp4_kernel", quant_scatter_nvfp4_kernel, qgrid, 256, 0, st,
+               static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, ids, v.inv, v.offsets, v.tile_ptr,
+               static_cast<const int32_t*>(amax), v.xq, static_cast<uint8_t*>(v.xs));
         return MOE_OK;
     }
-    if (c.fmt == MOE_FMT_FP8_ROW)
-        quant_scatter_kernel<0><<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, v.inv, v.xq,
-                                                       static_cast<float*>(v.xs));
-    else
-        quant_scatter_kernel<1><<<qgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, v.inv, v.xq,
-                                                       static_cast<float*>(v.xs));
-    LAUNCH_CHECK("quant_scatter_kernel");
+    if (T <= 4 * h->num_sms) {
+        // one CTA per token while the batch leaves SMs to spare
+        LAUNCH(h->pdl, "quant_scatter_row_kernel",
+               c.fmt == MOE_FMT_FP8_ROW ? quant_scatter_row_kernel<0> : quant_scatter_row_kernel<1>, T, 256, 0, st,
+               static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, static_cast<const int32_t*>(v.inv), v.xq,
+               static_cast<float*>(v.xs));
+        return MOE_OK;
+    }
+    LAUNCH(h->pdl, "quant_scatter_kernel",
+           c.fmt == MOE_FMT_FP8_ROW ? quant_scatter_kernel<0> : quant_scatter_kernel<1>, qgrid, 256, 0, st,
+           static_cast<const __nv_bfloat16*>(x), T, c.H, c.k, static_cast<const int32_t*>(v.inv), v.xq,
+           static_cast<float*>(v.xs));
     return MOE_OK;
 }
 
@@ -396,12 +442,11 @@ static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, u
 static int max_m_tiles(const moe_config& c, int T);
 
 template <int KIND>
-static moe_status launch_fp4(const CUtensorMap& ta, const CUtensorMap& tb, const Fp4Params& p, int grid,
+static moe_status launch_fp4(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const Fp4Params& p, int grid,
                              cudaStream_t st) {
     auto kern = grouped_gemm_fp4_kernel<KIND>;
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F4_SMEM));
-    kern<<<grid, GEMM_THREADS, F4_SMEM, st>>>(ta, tb, p);
-    LAUNCH_CHECK("grouped_gemm_fp4_kernel");
+    LAUNCH(pdl, "grouped_gemm_fp4_kernel", kern, grid, GEMM_THREADS, F4_SMEM, st, ta, tb, p);
     return MOE_OK;
 }
 
@@ -447,7 +492,8 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return gate_up ? launch_fp4<KIND_GATE_UP>(ta, tb, p, grid, st) : launch_fp4<KIND_DOWN>(ta, tb, p, grid, st);
+    return gate_up ? launch_fp4<KIND_GATE_UP>(h->pdl, ta, tb, p, grid, st)
+                   : launch_fp4<KIND_DOWN>(h->pdl, ta, tb, p, grid, st);
 }
 
 // ------------------------------------------------------------------ tensor maps
@@ -482,14 +528,13 @@ static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, u
 }
 
 template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
-static moe_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
+static moe_status launch_gemm(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
                               cudaStream_t st) {
     using S = GemmSmem<BN, STAGES>;
     static_assert(S::TOTAL <= 232448, "shared memory of the GEMM exceeds 227 KB");
     auto kern = grouped_gemm_kernel<KIND, BSCALE, PROMOTE, BN, STAGES>;
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL));
-    kern<<<grid, GEMM_THREADS, S::TOTAL, st>>>(ta, tb, p);
-    LAUNCH_CHECK("grouped_gemm_kernel");
+    LAUNCH(pdl, "grouped_gemm_kernel", kern, grid, GEMM_THREADS, S::TOTAL, st, ta, tb, p);
     return MOE_OK;
 }
 
@@ -539,8 +584,8 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4>(ta, tb, p, grid, st);
-    return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4>(ta, tb, p, grid, st);
+    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4>(h->pdl, ta, tb, p, grid, st);
+    return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4>(h->pdl, ta, tb, p, grid, st);
 }
 
 // ------------------------------------------------------------------ down
@@ -570,15 +615,18 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     p.w_scale = reinterpret_cast<const float*>(pw + h->wl.d_s);
     p.o = v.o;
     p.H = c.H;
+    p.A = T * c.k;
+    p.split = v.pick + 1;
+    p.s_max = split_limit(h->picker, p.A);
     p.perm = v.perm;
     p.route_w = w;
     p.status = v.status;
     p.spin_limit = h->spin_limit;
-    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
+    const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks * p.s_max));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     CUDA_TRY(cudaFuncSetAttribute(grouped_gemm_mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MX_SMEM));
-    grouped_gemm_mx_down_kernel<<<grid, GEMM_THREADS, MX_SMEM, st>>>(ta, tb, p);
-    LAUNCH_CHECK("grouped_gemm_mx_down_kernel");
+    LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", grouped_gemm_mx_down_kernel, grid, GEMM_THREADS, MX_SMEM, st, ta,
+           tb, p);
     return MOE_OK;
 }
 
@@ -632,15 +680,14 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
         const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * (c.H / 64)));
         CUDA_TRY(cudaFuncSetAttribute(down_gemm_poly_kernel<BSCALE_BLOCK128>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, POLY_SMEM));
-        down_gemm_poly_kernel<BSCALE_BLOCK128><<<grid, GEMM_THREADS, POLY_SMEM, st>>>(ta, tb, tb128, tb64, p,
-                                                                                     v.pick);
-        LAUNCH_CHECK("down_gemm_poly_kernel");
+        LAUNCH(h->pdl, "down_gemm_poly_kernel", down_gemm_poly_kernel<BSCALE_BLOCK128>, grid, GEMM_THREADS,
+               POLY_SMEM, st, ta, tb, tb128, tb64, p, static_cast<const int32_t*>(v.pick));
         return MOE_OK;
     }
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
-    if (BN == 256) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 256, 4>(ta, tb, p, grid, st);
-    if (BN == 128) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 128, 6>(ta, tb, p, grid, st);
-    return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 64, 8>(ta, tb, p, grid, st);
+    if (BN == 256) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 256, 4>(h->pdl, ta, tb, p, grid, st);
+    if (BN == 128) return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 128, 6>(h->pdl, ta, tb, p, grid, st);
+    return launch_gemm<KIND_DOWN, BSCALE_BLOCK128, true, 64, 8>(h->pdl, ta, tb, p, grid, st);
 }
 
 extern "C" moe_status moe_set_picker_params(moe_handle* h, const long long* params) {
@@ -672,6 +719,13 @@ extern "C" moe_status moe_set_tile_config(moe_handle* h, int down_bn) {
     return MOE_OK;
 }
 
+extern "C" moe_status moe_set_launch_options(moe_handle* h, int pdl) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_launch_options: null handle");
+    if (pdl != 0 && pdl != 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_launch_options: pdl must be 0 or 1 (got %d)", pdl);
+    h->pdl = pdl;
+    return MOE_OK;
+}
+
 // ------------------------------------------------------------------ combine
 extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws, moe_stream_t stream) {
     moe_status st0 = check_T(h, T, "moe_combine");
@@ -683,9 +737,10 @@ extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws,
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
     const int grid = std::min(T, 16 * h->num_sms);
-    combine_kernel<<<grid, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        static_cast<const float*>(v.o), v.inv, T, h->cfg.H, h->cfg.k, static_cast<__nv_bfloat16*>(y));
-    LAUNCH_CHECK("combine_kernel");
+    LAUNCH(h->pdl, "combine_kernel", combine_kernel, grid, 128, 0, reinterpret_cast<cudaStream_t>(stream),
+           static_cast<const float*>(v.o), static_cast<const int32_t*>(v.inv), T, h->cfg.H, h->cfg.k,
+           static_cast<const int32_t*>(h->cfg.fmt == MOE_FMT_FP8_ROW ? v.pick + 1 : nullptr),
+           split_limit(h->picker, T * h->cfg.k), static_cast<__nv_bfloat16*>(y));
     return MOE_OK;
 }
 

@@ -10,13 +10,15 @@
 // lane sums are combined by an xor butterfly over offsets 1, 2, 4, 8, 16, which
 // adds them as the balanced pairwise tree ((p0+p1)+(p2+p3))+...; then + bias[e].
 //
-// Two kernels:
+// Kernels:
 //  router_logits_kernel  a 2-D grid of CTA tiles (TOK tokens x EXP experts; 32 x 16,
 //                        or 64 x 8 when E <= 8).
 //                        The 256-wide H chunks of X and Wr go through shared
 //                        memory with a 4-stage cp.async pipeline; each of the 8
 //                        warps owns one 8-token x 8-expert micro-tile, so one
 //                        16-byte X read from shared memory feeds 64 fma.
+//  router_logits_small_kernel  batches of at most 128 tokens: one warp per
+//                        (expert, 4 tokens) reading global memory directly.
 //  router_topk_kernel    one warp per token: k rounds of a warp argmax over
 //                        the token's logits, then softmax or sigmoid weights.
 #pragma once
@@ -113,6 +115,8 @@ struct RouterLoader {
 
 template <int TOK, int EXP>
 __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterParams p) {
+    pdl_wait();
+    pdl_trigger();
     using RT = RouterTile<TOK, EXP>;
     extern __shared__ __align__(16) uint8_t rsm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -228,9 +232,64 @@ __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterPara
     }
 }
 
+// Small batches: one warp per (expert, group of RS_TG tokens), straight from
+// global memory (X rows stay in L1/L2, each Wr row is read once per token
+// group), 4 experts per CTA.  Same chains and tree as the tiled kernel: lane l
+// runs the fma chain over h = 256 i + 8 l + j, and the xor butterfly over
+// offsets 1, 2, 4, 8, 16 forms the same pairwise sums on every lane.
+constexpr int RS_TG = 4;
+constexpr int RS_WARPS = 4;
+__global__ void __launch_bounds__(RS_WARPS * 32) router_logits_small_kernel(RouterParams p) {
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.y * RS_WARPS + warp;
+    const int t0 = blockIdx.x * RS_TG;
+    if (e >= p.E) return;
+    const float* wrow = p.wr + static_cast<size_t>(e) * p.H + 8 * lane;
+    const __nv_bfloat16* xrow[RS_TG];
+#pragma unroll
+    for (int tt = 0; tt < RS_TG; tt++)
+        xrow[tt] = p.x + static_cast<size_t>(t0 + tt < p.T ? t0 + tt : t0) * p.H + 8 * lane;
+    float acc[RS_TG];
+#pragma unroll
+    for (int tt = 0; tt < RS_TG; tt++) acc[tt] = 0.0f;
+    const int nI = p.H >> 8;
+#pragma unroll 4
+    for (int i = 0; i < nI; i++) {
+        const float4 wa = __ldg(reinterpret_cast<const float4*>(wrow + 256 * i));
+        const float4 wb = __ldg(reinterpret_cast<const float4*>(wrow + 256 * i + 4));
+        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+        for (int tt = 0; tt < RS_TG; tt++) {
+            const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xrow[tt] + 256 * i));
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const float xj = (j & 1) ? bf16_hi(xw[j >> 1]) : bf16_lo(xw[j >> 1]);
+                acc[tt] = __fmaf_rn(xj, wv[j], acc[tt]);
+            }
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < RS_TG; tt++)
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) acc[tt] = __fadd_rn(acc[tt], __shfl_xor_sync(0xffffffffu, acc[tt], off));
+    if (lane < RS_TG && t0 + lane < p.T) {
+        float val = acc[0];
+#pragma unroll
+        for (int tt = 1; tt < RS_TG; tt++)
+            if (lane == tt) val = acc[tt];
+        if (p.bias) val = __fadd_rn(val, p.bias[e]);
+        p.logits[static_cast<size_t>(t0 + lane) * p.E + e] = val;
+    }
+}
+
 // top-k per token: k rounds of a warp argmax, larger logit first, equal
 // logits -> lower expert id.  Lane l owns experts l + 32 m.
 __global__ void __launch_bounds__(256) router_topk_kernel(RouterParams p) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < p.T; t += gridDim.x * 8) {
         const float* l = p.logits + static_cast<size_t>(t) * p.E;

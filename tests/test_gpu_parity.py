@@ -25,6 +25,10 @@ CASES = {
     "row-skew-e64": (W.custom(H=256, I=256, E=64, k=8, zipf_s=1.2), 100),
     "block128-ragged": (W.custom(H=512, I=384, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 300),
     "t1": (W.custom(H=256, I=128, E=8, k=2), 1),
+    "row-split-t3": (W.custom(H=512, I=2048, E=8, k=2), 3),
+    # above 4 x 148 tokens the quantisation runs one warp per token
+    "row-t700": (W.custom(H=256, I=128, E=8, k=2), 700),
+    "block128-t700": (W.custom(H=256, I=128, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 700),
     "nvfp4-ragged": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4), 300),
     "nvfp4-skew-e32": (W.custom(H=256, I=256, E=32, k=4, fmt=W.FMT_NVFP4, zipf_s=1.0), 50),
 }
@@ -90,6 +94,14 @@ def inject_hidden(layer, wl, ids, T, hq, hs):
     layer.region("hs", torch.uint8, sf_all.size).copy_(torch.from_numpy(sf_all).cuda())
 
 
+def expected_split(wl, max_T, counts, sms):
+    """The down GEMM's K split the oracle's rule gives for this workspace."""
+    if wl.fmt != W.FMT_FP8_ROW:
+        return 1
+    A_max = max_T * wl.k
+    return oracle.pick_split(counts, wl.H // 256, wl.I // 128, A_max + 7 * min(A_max, 256), sms)
+
+
 def build_case(name, seed=0):
     wl, T = CASES[name]
     d = synth.layer(wl, seed=seed)
@@ -128,18 +140,26 @@ def test_router_ids_bit_exact(name):
 
 
 @pytest.mark.parametrize("H,E,k,score,T", [(7168, 256, 8, W.SCORE_SIGMOID, 20), (2048, 256, 8, W.SCORE_SOFTMAX, 64),
-                                           (4096, 8, 2, W.SCORE_SOFTMAX, 33)])
+                                           (4096, 8, 2, W.SCORE_SOFTMAX, 33), (4096, 8, 2, W.SCORE_SOFTMAX, 1),
+                                           (2048, 250, 8, W.SCORE_SOFTMAX, 127),
+                                           (2048, 256, 8, W.SCORE_SOFTMAX, 129), (4096, 8, 2, W.SCORE_SOFTMAX, 150)])
 def test_router_named_shapes_bit_exact(H, E, k, score, T):
-    wl = W.custom(H=H, I=128, E=E, k=k, score=score, router_init="uniform")
-    wr, _ = synth.router(wl, seed=3)
+    """Both logits kernels (small batches, and the tiled one above 128 tokens)
+    give the oracle's fp32 logits bit for bit, and its ids."""
+    wl = W.custom(H=H, I=128, E=E, k=k, score=score, router_init="uniform", zipf_s=1.0)
+    wr, bias = synth.router(wl, seed=3)
     x = synth.tokens(wl, T, seed=3)
     h = native.moe_init(wl, T)
     ws = torch.empty(native.moe_workspace_size(h), dtype=torch.uint8, device="cuda")
     ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
     w = torch.empty(T, k, dtype=torch.float32, device="cuda")
-    native.moe_route(h, x.cuda(), T, wr.cuda(), None, ids, w, ws)
+    native.moe_route(h, x.cuda(), T, wr.cuda(), bias.cuda(), ids, w, ws)
     torch.cuda.synchronize()
-    ids_ref, w_ref = oracle.topk(oracle.router_logits(bits(x), wr.numpy()), k, score)
+    lg_ref = oracle.router_logits(bits(x), wr.numpy(), bias.numpy())
+    off = native.moe_workspace_view_get(h, ws)["logits"] - ws.data_ptr()
+    lg = ws[off:off + T * E * 4].view(torch.float32).cpu().numpy().reshape(T, E)
+    assert (lg.view(np.uint32) == lg_ref.astype(np.float32).view(np.uint32)).all()
+    ids_ref, w_ref = oracle.topk(lg_ref, k, score)
     assert (ids.cpu().numpy() == ids_ref).all()
     np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=0, atol=2e-6)
     native.moe_destroy(h)
@@ -186,7 +206,9 @@ def test_dispatch_bit_exact(name):
     assert (tile_ptr == np.searchsorted(te, np.arange(E + 1), side="left")).all()
     a, b, bw, g, sms = native.moe_get_picker_params(layer.h)
     want, _ = oracle.pick_down_tile(counts, wl.H, wl.I, sms, a, b, bw, g)
-    assert int(layer.region("pick", torch.int32, 1).cpu().numpy()[0]) == want
+    pick = layer.region("pick", torch.int32, 2).cpu().numpy()
+    assert int(pick[0]) == want
+    assert int(pick[1]) == expected_split(wl, T, counts, sms)
     rows = gpu_slot_rows(layer, wl, ids, T)
     if nvfp4(wl):
         xq = gpu_rows(layer, wl, "xq", wl.H // 2)[rows]
@@ -257,7 +279,10 @@ def test_down_matches_oracle_on_oracle_hidden(name, down_bn):
     native.moe_down(layer.h, layer.packed, w_dev, T, layer.ws)
     torch.cuda.synchronize()
     assert layer.status()[0] == 0
-    o = layer.region("o", torch.float32, A * wl.H).cpu().numpy().reshape(A, wl.H)
+    S = int(layer.region("pick", torch.int32, 2).cpu().numpy()[1])
+    if name == "row-split-t3":
+        assert S == 4                     # 10 units, s_max = 16 K-blocks / 4
+    o = layer.region("o", torch.float32, S * A * wl.H).cpu().numpy().reshape(S, A, wl.H).sum(axis=0)
     assert tolerance_violations(o, ref["o_w"]) == 0
 
 
@@ -293,6 +318,32 @@ def test_forward_twice_same_bits():
     y2 = layer.forward(x.cuda(), d["wr"].cuda(), None)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("name", ["row-skew-e64", "block128-ragged", "nvfp4-ragged"])
+def test_launch_modes_same_bits(name):
+    """Programmatic dependent launch on or off, direct calls or a replayed CUDA
+    graph of the call: the same kernels on the same data give the same bits."""
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    xc, wr = x.cuda(), d["wr"].cuda()
+    bias = d["bias"].cuda() if d["bias"] is not None else None
+    native.moe_set_launch_options(layer.h, 0)
+    y_plain = layer.forward(xc, wr, bias).clone()
+    native.moe_set_launch_options(layer.h, 1)
+    y_pdl = layer.forward(xc, wr, bias).clone()
+    y = torch.empty(T, wl.H, dtype=torch.bfloat16, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        native.moe_forward(layer.h, xc, T, wr, bias, layer.packed, y, layer.ws)
+    y.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert layer.status()[0] == 0
+    assert torch.equal(y_plain, y_pdl)
+    assert torch.equal(y_plain, y)
+    del g
 
 
 def test_empty_batch():
