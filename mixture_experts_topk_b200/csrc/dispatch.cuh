@@ -362,15 +362,27 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* o, const int3
         for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
         for (int c0 = 8 * threadIdx.x; c0 < H; c0 += 8 * blockDim.x) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (S == 1) {
+                // all k rows' loads in flight at once
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                if (slot[j] < 0) continue;
-                const float* row = o + static_cast<size_t>(slot[j]) * H + c0;
-                for (int sp = 0; sp < S; sp++) {
-                    const float4* src = reinterpret_cast<const float4*>(row + sp * copy);
+                for (int j = 0; j < 8; j++) {
+                    if (slot[j] < 0) continue;
+                    const float4* src = reinterpret_cast<const float4*>(o + static_cast<size_t>(slot[j]) * H + c0);
                     const float4 a = src[0], b = src[1];
                     acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
                     acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    if (slot[j] < 0) continue;
+                    const float* row = o + static_cast<size_t>(slot[j]) * H + c0;
+                    for (int sp = 0; sp < S; sp++) {
+                        const float4* src = reinterpret_cast<const float4*>(row + sp * copy);
+                        const float4 a = src[0], b = src[1];
+                        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+                        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+                    }
                 }
             }
             uint32_t r[4];

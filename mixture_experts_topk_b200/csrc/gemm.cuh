@@ -69,6 +69,12 @@ struct GemmParams {
 constexpr int TMAP_STRIDE = 260;              // shared-memory tile map: 2 x (E + 1) ints, E <= 256
 constexpr int TMAP_BYTES = 2 * TMAP_STRIDE * 4;
 
+// Sparse gate/up epilogue (a warp with few stored rows): per epilogue warp a
+// [8 rows][32 gate | 32 up] fp32 staging block and the 8 rows' X scales.
+constexpr int SPARSE_ROWS_MAX = 16;
+constexpr int SPARSE_WARP_FLOATS = 8 * 64 + 8;
+constexpr int SPARSE_BYTES = 8 * SPARSE_WARP_FLOATS * 4;
+
 template <int BN, int STAGES>
 struct GemmSmem {
     // accumulator buffers in TMEM (512 columns): deeper for narrower tiles, so the
@@ -84,7 +90,8 @@ struct GemmSmem {
     static constexpr int XCHG_OFF = (TMEM_SLOT_OFF + 4 + 15) / 16 * 16;
     static constexpr int XCHG_BYTES = 2 * 2 * 128 * 4 * 2;   // [parity][group][row] value + flag
     static constexpr int TMAP_OFF = XCHG_OFF + XCHG_BYTES;
-    static constexpr int TOTAL = TMAP_OFF + TMAP_BYTES + 1024; // + alignment slack
+    static constexpr int SPARSE_OFF = TMAP_OFF + TMAP_BYTES;
+    static constexpr int TOTAL = SPARSE_OFF + SPARSE_BYTES + 1024; // + alignment slack
 };
 
 // The schedule's tile pointers and row offsets, copied into shared memory once
@@ -275,6 +282,69 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     const uint32_t acc = u % NBUF;
                     if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
+                    if (!__any_sync(0xffffffffu, valid)) {
+                        // none of this warp's rows is stored: release the buffer only
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[acc]);
+                        u++;
+                        continue;
+                    }
+                    const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+                    const int nv = __popc(vmask);
+                    if (BSCALE == BSCALE_ROW && nv <= SPARSE_ROWS_MAX) {
+                        // Few stored rows (small batches): stage them in shared memory
+                        // 8 at a time and let lane c take column c of each, so the work
+                        // scales with the stored rows.  Same operations per element as
+                        // the row path below, so the same codes and scales.
+                        float* sb = reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * SPARSE_WARP_FLOATS;
+                        const int cidx = __popc(vmask & ((1u << lane) - 1u));
+#pragma unroll
+                        for (int half = 0; half < 2; half++) {
+                            float gv[32], uv[32];
+                            const int c0 = 64 * g + 32 * half;
+                            tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, gv, uv);
+                            if (half == 1) {
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(&tempty[acc]);
+                            }
+                            const int hcol = nb * 128 + c0;   // first hidden column of this 32-block
+                            uint32_t m = vmask;
+                            for (int r0 = 0; r0 < nv; r0 += 8) {
+                                if (valid && cidx >= r0 && cidx < r0 + 8) {
+                                    float4* d = reinterpret_cast<float4*>(sb + (cidx - r0) * 64);
+#pragma unroll
+                                    for (int q4 = 0; q4 < 8; q4++) {
+                                        d[q4] = make_float4(gv[4 * q4], gv[4 * q4 + 1], gv[4 * q4 + 2], gv[4 * q4 + 3]);
+                                        d[8 + q4] = make_float4(uv[4 * q4], uv[4 * q4 + 1], uv[4 * q4 + 2], uv[4 * q4 + 3]);
+                                    }
+                                    sb[512 + cidx - r0] = sa;
+                                }
+                                __syncwarp();
+                                const int nr = min(8, nv - r0);
+                                for (int i = 0; i < nr; i++) {
+                                    const int rl = __ffs(m) - 1;   // lane (tile row 32 q + rl) of stored row r0 + i
+                                    m &= m - 1;
+                                    const float sa_i = sb[512 + i];
+                                    const float gg = sb[i * 64 + lane] * (sa_i * bsg[half]);
+                                    const float uu = sb[i * 64 + 32 + lane] * (sa_i * bsu[half]);
+                                    const float hvv = gg / (1.0f + expf(-gg)) * uu;
+                                    float amax = fabsf(hvv);
+#pragma unroll
+                                    for (int off = 16; off > 0; off >>= 1)
+                                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                                    const int ex = mx_exponent(amax);
+                                    const long long prow = static_cast<long long>(mi) * 128 + 32 * q + rl;
+                                    p.hq[prow * p.I + hcol + lane] = f_to_e4m3(__fmul_rn(hvv, mx_inv_scale(ex)));
+                                    if (lane == 0) p.hsf[sf_offset(prow, hcol / 32, p.I / 32)] = static_cast<uint8_t>(ex + 127);
+                                }
+                                __syncwarp();
+                            }
+                        }
+                        u++;
+                        continue;
+                    }
 #pragma unroll
                     for (int half = 0; half < 2; half++) {
                         float gv[32], uv[32];
@@ -295,6 +365,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     float ag[64], au[64];
 #pragma unroll
                     for (int c = 0; c < 64; c++) ag[c] = au[c] = 0.0f;
+                    const bool any_valid = __any_sync(0xffffffffu, valid);
                     const float* arow = p.a_scale + static_cast<size_t>(valid ? row : 0) * p.a_ld;
                     const float* bsb = p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + 2 * nb) * p.num_kb;
                     // scales of the next K-block are loaded before waiting on this one
@@ -311,6 +382,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         tc_fence_after();
 #pragma unroll
                         for (int half = 0; half < 2; half++) {
+                            if (!any_valid) break;   // no stored row: skip the readback
                             float vg[32], vu[32];
                             const int c0 = 64 * g + 32 * half;
                             tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, vg, vu);
@@ -400,6 +472,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 #pragma unroll
                 for (int c = 0; c < NC; c++) acc_r[c] = 0.0f;
                 const int n0 = nb * BN + g * NC;
+                const bool any_valid = __any_sync(0xffffffffu, valid);
                 const float rw = valid ? p.route_w[p.perm[row]] : 0.0f;   // loaded while the MMAs run
                 const float* arow = p.a_scale + static_cast<size_t>(valid ? row : 0) * p.a_ld;
                 const float* bsb = p.b_scale + (static_cast<size_t>(e) * (p.b_rows / 128) + n0 / 128) * p.num_kb;
@@ -415,7 +488,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     const uint32_t acc = u % NBUF;
                     if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
-                    if constexpr (NC >= 64) {
+                    if (!any_valid) {
+                        // no stored row: skip the readback
+                    } else if constexpr (NC >= 64) {
 #pragma unroll
                         for (int ch = 0; ch < NC / 64; ch++) {
                             float v0[32], v1[32];

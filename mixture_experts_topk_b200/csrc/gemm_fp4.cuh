@@ -204,6 +204,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const uint32_t acc = u % F4_NBUF;
             if (!warp_wait(&tfull[acc], (u / F4_NBUF) & 1, limit)) { ok = false; break; }
             tc_fence_after();
+            if (!__any_sync(0xffffffffu, valid)) {
+                // none of this warp's rows is stored: release the accumulator only
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+                u++;
+                continue;
+            }
             if (KIND == KIND_GATE_UP) {
                 float gv[32], uv[32];
                 tmem_ld32x2(lane_addr + acc * F4_BN + 32 * g, lane_addr + acc * F4_BN + 64 + 32 * g, gv, uv);

@@ -212,6 +212,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const float4 ws4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + static_cast<size_t>(e) * p.H + n0) + lane);
             if (!warp_wait(tfull, u & 1, limit)) { ok = false; break; }
             tc_fence_after();
+            if (!__any_sync(0xffffffffu, valid)) {
+                // none of this warp's rows is stored: release the accumulator only
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty);
+                u++;
+                continue;
+            }
             float v[128];
 #pragma unroll
             for (int ch = 0; ch < 2; ch++)

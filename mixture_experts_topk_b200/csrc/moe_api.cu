@@ -110,13 +110,17 @@ static size_t hidden_scale_bytes(int fmt, int I) {
 }
 // rows of the X / hidden buffers: 128-padded per expert where block-scaled
 // tensor-core MMAs read them (NVFP4 X and hidden, FP8_ROW hidden)
+// Unpadded buffers (rows in slot order) get TILE_M rows of slack: a row tile
+// starting at any slot stays inside the tensor map, so the TMA box never
+// zero-fills past the end (which slows the copy); the slack rows feed only
+// accumulator rows the epilogue does not store.
 static size_t padded_rows(const moe_config& c) {
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
-    return c.fmt == MOE_FMT_NVFP4 ? A + static_cast<size_t>(TILE_M) * c.E : A;
+    return c.fmt == MOE_FMT_NVFP4 ? A + static_cast<size_t>(TILE_M) * c.E : A + TILE_M;
 }
 static size_t hidden_rows(const moe_config& c) {
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
-    return c.fmt == MOE_FMT_FP8_BLOCK128 ? A : A + static_cast<size_t>(TILE_M) * c.E;
+    return c.fmt == MOE_FMT_FP8_BLOCK128 ? A + TILE_M : A + static_cast<size_t>(TILE_M) * c.E;
 }
 
 // rows of the fp32 down output: A, plus room for up to 8 K-split copies of
@@ -558,7 +562,7 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
     CUtensorMap ta, tb;
-    moe_status r = make_tmap(&ta, v.xq, c.H, A, c.H, GEMM_BK, GEMM_BM);
+    moe_status r = make_tmap(&ta, v.xq, c.H, padded_rows(c), c.H, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
     r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * 2 * c.I, c.H, GEMM_BK, 256);
     if (r != MOE_OK) return r;
@@ -646,7 +650,7 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
     const int BN = h->down_bn ? h->down_bn : 256;
     CUtensorMap ta, tb, tb128, tb64;
-    moe_status r = make_tmap(&ta, v.hq, c.I, A, c.I, GEMM_BK, GEMM_BM);
+    moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
     r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, BN);
     if (r != MOE_OK) return r;
