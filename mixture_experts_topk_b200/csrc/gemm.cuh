@@ -73,7 +73,68 @@ constexpr int TMAP_BYTES = 2 * TMAP_STRIDE * 4;
 // [8 rows][32 gate | 32 up] fp32 staging block and the 8 rows' X scales.
 constexpr int SPARSE_ROWS_MAX = 16;
 constexpr int SPARSE_WARP_FLOATS = 8 * 64 + 8;
-constexpr int SPARSE_BYTES = 8 * SPARSE_WARP_FLOATS * 4;
+
+// Coalesced fp32 row stores of the down epilogues.  A warp holds 32 rows (one
+// per lane) x NC columns; 16-column chunks pass through a per-warp [32][20]
+// float block (rows padded to 80 B, so the row-wise float4 writes of 8 lanes
+// hit distinct banks), and every store instruction then writes 8 rows x 64
+// contiguous bytes (4 lanes per row) instead of 32 rows x 16 bytes.
+// dst: this lane's row at its first column, null when the row is not stored.
+// Stored value: (v[c] * cs[c]) * rs with column scales, else v[c] * rs.
+// Warps with at most 8 stored rows store them directly (fewer steps).
+constexpr int STG_STRIDE = 20;
+constexpr int STG_WARP_FLOATS = 32 * STG_STRIDE;
+template <int NC, bool HAS_CS>
+__device__ __forceinline__ void store_rows_coalesced(const float (&v)[NC], float* stg, float* dst, const float* cs,
+                                                     float rs, int lane) {
+    if (__popc(__ballot_sync(0xffffffffu, dst != nullptr)) <= 8) {
+        // few stored rows (small batches): each stores its own row directly
+        if (dst != nullptr) {
+#pragma unroll
+            for (int c = 0; c < NC; c += 4) {
+                float4 o;
+                if (HAS_CS) {
+                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(cs + c));
+                    o = make_float4(v[c] * s4.x * rs, v[c + 1] * s4.y * rs, v[c + 2] * s4.z * rs, v[c + 3] * s4.w * rs);
+                } else {
+                    o = make_float4(v[c] * rs, v[c + 1] * rs, v[c + 2] * rs, v[c + 3] * rs);
+                }
+                *reinterpret_cast<float4*>(dst + c) = o;
+            }
+        }
+        return;
+    }
+    const int rsub = lane >> 2, c4 = (lane & 3) * 4;
+#pragma unroll
+    for (int ch = 0; ch < NC / 16; ch++) {
+        float4* w = reinterpret_cast<float4*>(stg + lane * STG_STRIDE);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; q4++)
+            w[q4] = make_float4(v[16 * ch + 4 * q4], v[16 * ch + 4 * q4 + 1], v[16 * ch + 4 * q4 + 2],
+                                v[16 * ch + 4 * q4 + 3]);
+        __syncwarp();
+        float4 s4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        if (HAS_CS) s4 = __ldg(reinterpret_cast<const float4*>(cs + 16 * ch + c4));
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int row = 8 * i + rsub;
+            float* d = reinterpret_cast<float*>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), row));
+            const float r = __shfl_sync(0xffffffffu, rs, row);
+            const float4 x = *reinterpret_cast<const float4*>(stg + row * STG_STRIDE + c4);
+            if (d != nullptr) {
+                float4 o;
+                if (HAS_CS) o = make_float4(x.x * s4.x * r, x.y * s4.y * r, x.z * s4.z * r, x.w * s4.w * r);
+                else o = make_float4(x.x * r, x.y * r, x.z * r, x.w * r);
+                *reinterpret_cast<float4*>(d + 16 * ch + c4) = o;
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// per epilogue warp: the sparse gate/up staging or the down store staging
+constexpr int EPI_WARP_FLOATS = SPARSE_WARP_FLOATS > STG_WARP_FLOATS ? SPARSE_WARP_FLOATS : STG_WARP_FLOATS;
+constexpr int SPARSE_BYTES = 8 * EPI_WARP_FLOATS * 4;
 
 template <int BN, int STAGES>
 struct GemmSmem {
@@ -92,6 +153,7 @@ struct GemmSmem {
     static constexpr int TMAP_OFF = XCHG_OFF + XCHG_BYTES;
     static constexpr int SPARSE_OFF = TMAP_OFF + TMAP_BYTES;
     static constexpr int TOTAL = SPARSE_OFF + SPARSE_BYTES + 1024; // + alignment slack
+    static_assert(SPARSE_OFF % 16 == 0, "staging block must be 16-byte aligned");
 };
 
 // The schedule's tile pointers and row offsets, copied into shared memory once
@@ -297,7 +359,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         // 8 at a time and let lane c take column c of each, so the work
                         // scales with the stored rows.  Same operations per element as
                         // the row path below, so the same codes and scales.
-                        float* sb = reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * SPARSE_WARP_FLOATS;
+                        float* sb = reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * EPI_WARP_FLOATS;
                         const int cidx = __popc(vmask & ((1u << lane) - 1u));
 #pragma unroll
                         for (int half = 0; half < 2; half++) {
@@ -514,21 +576,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     u++;
                 }
                 if (!ok) break;
-                if (valid) {
-                    const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + n0;
-                    float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(row) * p.H + n0);
-#pragma unroll
-                    for (int c = 0; c < NC; c += 4) {
-                        float v[4];
-#pragma unroll
-                        for (int i = 0; i < 4; i++) {
-                            v[i] = acc_r[c + i];
-                            if (BSCALE == BSCALE_ROW) v[i] *= __ldg(bs + c + i);
-                            v[i] *= rw;
-                        }
-                        dst[c / 4] = make_float4(v[0], v[1], v[2], v[3]);
-                    }
-                }
+                store_rows_coalesced<NC, BSCALE == BSCALE_ROW>(
+                    acc_r, reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * EPI_WARP_FLOATS,
+                    valid ? p.o + static_cast<size_t>(row) * p.H + n0 : nullptr,
+                    p.b_scale + static_cast<size_t>(e) * p.b_rows + n0, rw, lane);
             }
         }
         if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_EPILOGUE);

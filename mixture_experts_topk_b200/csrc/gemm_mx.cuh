@@ -33,7 +33,9 @@ constexpr int MX_BAR_OFF = MX_SFB_OFF + 1024;
 constexpr int MX_NUM_BARS = 2 * MX_STAGES + 3;
 constexpr int MX_TMEM_SLOT_OFF = MX_BAR_OFF + 8 * MX_NUM_BARS;
 constexpr int MX_TMAP_OFF = MX_TMEM_SLOT_OFF + 16;
-constexpr int MX_SMEM = MX_TMAP_OFF + TMAP_BYTES + 1024;
+constexpr int MX_STG_OFF = (MX_TMAP_OFF + TMAP_BYTES + 15) / 16 * 16;   // float4 staging
+static_assert(MX_STG_OFF % 16 == 0, "staging block must be 16-byte aligned");
+constexpr int MX_SMEM = MX_STG_OFF + 8 * STG_WARP_FLOATS * 4 + 1024;
 constexpr int MX_SFA_TMEM = MX_BN;                    // 4 columns per stage
 constexpr int MX_SFB_TMEM = MX_BN + 4 * MX_STAGES;    // 8 columns (two 128-row chunks)
 
@@ -204,12 +206,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             decode_tile(t - sp * units, s_tptr, p.E, p.n_blocks, e, mi, nb);
             const int local = mi * 128 + r - s_tptr[e] * 128;
             const bool valid = local < s_off[e + 1] - s_off[e];
-            // loaded while the tile's MMAs run: the row's routing weight, and lane l
-            // holds the weight scales of columns 4l .. 4l+3 (read back by shuffle)
+            // the row's routing weight is loaded while the tile's MMAs run
             const int slot = s_off[e] + local;
             const float rw = valid ? p.route_w[p.perm[slot]] : 0.0f;
             const int n0 = nb * MX_BN + 128 * g;
-            const float4 ws4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + static_cast<size_t>(e) * p.H + n0) + lane);
             if (!warp_wait(tfull, u & 1, limit)) { ok = false; break; }
             tc_fence_after();
             if (!__any_sync(0xffffffffu, valid)) {
@@ -229,14 +229,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty);   // the next tile's MMAs may start
             u++;
-            float4* dst = reinterpret_cast<float4*>(p.o + (static_cast<size_t>(sp) * p.A + slot) * p.H + n0);
-#pragma unroll
-            for (int c = 0; c < 128; c += 4) {
-                const float sx = __shfl_sync(0xffffffffu, ws4.x, c / 4), sy = __shfl_sync(0xffffffffu, ws4.y, c / 4);
-                const float sz = __shfl_sync(0xffffffffu, ws4.z, c / 4), sw = __shfl_sync(0xffffffffu, ws4.w, c / 4);
-                if (valid)
-                    dst[c / 4] = make_float4(v[c] * sx * rw, v[c + 1] * sy * rw, v[c + 2] * sz * rw, v[c + 3] * sw * rw);
-            }
+            store_rows_coalesced<128, true>(
+                v, reinterpret_cast<float*>(smem + MX_STG_OFF) + (warp - 2) * STG_WARP_FLOATS,
+                valid ? p.o + (static_cast<size_t>(sp) * p.A + slot) * p.H + n0 : nullptr,
+                p.w_scale + static_cast<size_t>(e) * p.H + n0, rw, lane);
         }
         if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_EPILOGUE);
     }
