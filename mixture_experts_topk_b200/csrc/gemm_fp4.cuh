@@ -9,7 +9,7 @@
 // Pure-Triton fused MoE article: gate and up share one input tile.
 //
 // Tile 128 rows x 128 columns (gate/up: 64 gate + 64 up columns of one 64-wide
-// hidden block), K stage 256 values = 128 bytes per row, 6 stages.  Per stage
+// hidden block), K stage 256 values = 128 bytes per row, 5 stages.  Per stage
 // the producer brings, on one mbarrier: A and B tiles by TMA (128-byte swizzle)
 // and the 2 KB of A and 2 KB of B scale factors (4 chunks of 512 B, one per
 // MMA of K = 64) by plain bulk copies.  The MMA thread copies the chunks into a
@@ -27,7 +27,7 @@
 namespace moe {
 
 constexpr int F4_BN = 128;
-constexpr int F4_STAGES = 6;
+constexpr int F4_STAGES = 5;
 constexpr int F4_A_BYTES = 128 * 128;
 constexpr int F4_B_BYTES = F4_BN * 128;
 constexpr int F4_SF_BYTES = 2048;                 // 4 chunks of 512 B
@@ -38,7 +38,8 @@ constexpr int F4_BAR_OFF = F4_STAGES * F4_STAGE_BYTES;
 constexpr int F4_NUM_BARS = 2 * F4_STAGES + 2 * F4_NBUF + 1;
 constexpr int F4_TMEM_SLOT_OFF = F4_BAR_OFF + 8 * F4_NUM_BARS;
 constexpr int F4_TMAP_OFF = F4_TMEM_SLOT_OFF + 16;
-constexpr int F4_SMEM = F4_TMAP_OFF + TMAP_BYTES + 1024;
+constexpr int F4_STG_OFF = (F4_TMAP_OFF + TMAP_BYTES + 15) / 16 * 16;   // down-store staging
+constexpr int F4_SMEM = F4_STG_OFF + 8 * STG_WARP_FLOATS * 4 + 1024;
 static_assert(F4_SF_TMEM + 32 * F4_STAGES <= 512, "TMEM columns");
 
 struct Fp4Params {
@@ -259,15 +260,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[acc]);
                 u++;
-                if (valid) {
-                    const float sc = p.h_global * wg0 * rw;
-                    float4* dst = reinterpret_cast<float4*>(p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + 64 * g);
+                float v[64];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4) {
-                        dst[c / 4] = make_float4(v0[c] * sc, v0[c + 1] * sc, v0[c + 2] * sc, v0[c + 3] * sc);
-                        dst[8 + c / 4] = make_float4(v1[c] * sc, v1[c + 1] * sc, v1[c + 2] * sc, v1[c + 3] * sc);
-                    }
+                for (int c = 0; c < 32; c++) {
+                    v[c] = v0[c];
+                    v[32 + c] = v1[c];
                 }
+                store_rows_coalesced<64, false>(
+                    v, reinterpret_cast<float*>(smem + F4_STG_OFF) + (warp - 2) * STG_WARP_FLOATS,
+                    valid ? p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + 64 * g : nullptr, nullptr,
+                    p.h_global * wg0 * rw, lane);
             }
         }
         if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_EPILOGUE);
