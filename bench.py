@@ -101,7 +101,7 @@ def gemm_traffic(workload, T):
         return None
     d = json.load(open(p))
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "common.cuh"):
+    for f in ("gemm.cuh", "gemm_mx.cuh", "common.cuh"):
         h.update(open(os.path.join(ROOT, "mixture_experts_topk_b200", "csrc", f), "rb").read())
     if h.hexdigest()[:16] != d["kernel_sources_sha256_16"]:
         return None
