@@ -36,7 +36,7 @@ namespace moe {
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 128;                 // K bytes (= e4m3 elements) per stage
-constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_THREADS = 320;            // 8 epilogue warps
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK;
 
 enum { KIND_GATE_UP = 0, KIND_DOWN = 1 };
@@ -134,9 +134,19 @@ __device__ __forceinline__ void store_rows_coalesced(const float (&v)[NC], float
 
 // per epilogue warp: the sparse gate/up staging or the down store staging
 constexpr int EPI_WARP_FLOATS = SPARSE_WARP_FLOATS > STG_WARP_FLOATS ? SPARSE_WARP_FLOATS : STG_WARP_FLOATS;
-constexpr int SPARSE_BYTES = 8 * EPI_WARP_FLOATS * 4;
 
-template <int BN, int STAGES>
+// EPI epilogue warps (8 or 16): 4 TMEM lane quadrants x EPI/4 column groups.
+template <int EPI>
+__host__ __device__ constexpr int gemm_threads() { return 64 + 32 * EPI; }
+// sparse gate/up staging rows per round: 8 with 8 epilogue warps, 4 with 16
+template <int EPI>
+__host__ __device__ constexpr int sparse_round() { return EPI == 8 ? 8 : 4; }
+template <int EPI>
+__host__ __device__ constexpr int epi_warp_floats() {
+    return EPI == 8 ? EPI_WARP_FLOATS : sparse_round<EPI>() * 64 + sparse_round<EPI>();
+}
+
+template <int BN, int STAGES, int EPI = 8>
 struct GemmSmem {
     // accumulator buffers in TMEM (512 columns): deeper for narrower tiles, so the
     // MMA can run further ahead of a per-K-block epilogue
@@ -152,7 +162,7 @@ struct GemmSmem {
     static constexpr int XCHG_BYTES = 2 * 2 * 128 * 4 * 2;   // [parity][group][row] value + flag
     static constexpr int TMAP_OFF = XCHG_OFF + XCHG_BYTES;
     static constexpr int SPARSE_OFF = TMAP_OFF + TMAP_BYTES;
-    static constexpr int TOTAL = SPARSE_OFF + SPARSE_BYTES + 1024; // + alignment slack
+    static constexpr int TOTAL = SPARSE_OFF + EPI * epi_warp_floats<EPI>() * 4 + 1024; // + alignment slack
     static_assert(SPARSE_OFF % 16 == 0, "staging block must be 16-byte aligned");
 };
 
@@ -189,10 +199,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                                           const int n_blocks, uint8_t* smem_raw) {
-    using S = GemmSmem<BN, STAGES>;
+    static_assert(EPI == 8 || (EPI == 16 && KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW && !PROMOTE && BN == 256),
+                  "16 epilogue warps are built for the FP8_ROW gate/up GEMM only");
+    using S = GemmSmem<BN, STAGES, EPI>;
+    constexpr int CG = EPI / 4;          // column groups
+    constexpr int GC = 128 / CG;         // gate/up: hidden columns per thread (64 or 32)
+    constexpr int NH = GC / 32;          // 32-column blocks per thread
+    constexpr int SR = sparse_round<EPI>();
+    constexpr int EWF = epi_warp_floats<EPI>();
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
     uint64_t* full = bars;
@@ -215,7 +232,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
         }
         for (int b = 0; b < NBUF; b++) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 8);   // one arrival per epilogue warp
+            mbar_init(&tempty[b], EPI);   // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -335,11 +352,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     // half (read back with a shuffle)
                     const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld] : 0.0f;
                     const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + nb * BN;
-                    float bsg[2], bsu[2];
+                    float bsg[NH], bsu[NH];
 #pragma unroll
-                    for (int half = 0; half < 2; half++) {
-                        bsg[half] = __ldg(bs + 64 * g + 32 * half + lane);
-                        bsu[half] = __ldg(bs + 128 + 64 * g + 32 * half + lane);
+                    for (int half = 0; half < NH; half++) {
+                        bsg[half] = __ldg(bs + GC * g + 32 * half + lane);
+                        bsu[half] = __ldg(bs + 128 + GC * g + 32 * half + lane);
                     }
                     const uint32_t acc = u % NBUF;
                     if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
@@ -359,36 +376,36 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         // 8 at a time and let lane c take column c of each, so the work
                         // scales with the stored rows.  Same operations per element as
                         // the row path below, so the same codes and scales.
-                        float* sb = reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * EPI_WARP_FLOATS;
+                        float* sb = reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * EWF;
                         const int cidx = __popc(vmask & ((1u << lane) - 1u));
 #pragma unroll
-                        for (int half = 0; half < 2; half++) {
+                        for (int half = 0; half < NH; half++) {
                             float gv[32], uv[32];
-                            const int c0 = 64 * g + 32 * half;
+                            const int c0 = GC * g + 32 * half;
                             tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, gv, uv);
-                            if (half == 1) {
+                            if (half == NH - 1) {
                                 tc_fence_before();
                                 __syncwarp();
                                 if (lane == 0) mbar_arrive(&tempty[acc]);
                             }
                             const int hcol = nb * 128 + c0;   // first hidden column of this 32-block
                             uint32_t m = vmask;
-                            for (int r0 = 0; r0 < nv; r0 += 8) {
-                                if (valid && cidx >= r0 && cidx < r0 + 8) {
+                            for (int r0 = 0; r0 < nv; r0 += SR) {
+                                if (valid && cidx >= r0 && cidx < r0 + SR) {
                                     float4* d = reinterpret_cast<float4*>(sb + (cidx - r0) * 64);
 #pragma unroll
                                     for (int q4 = 0; q4 < 8; q4++) {
                                         d[q4] = make_float4(gv[4 * q4], gv[4 * q4 + 1], gv[4 * q4 + 2], gv[4 * q4 + 3]);
                                         d[8 + q4] = make_float4(uv[4 * q4], uv[4 * q4 + 1], uv[4 * q4 + 2], uv[4 * q4 + 3]);
                                     }
-                                    sb[512 + cidx - r0] = sa;
+                                    sb[SR * 64 + cidx - r0] = sa;
                                 }
                                 __syncwarp();
-                                const int nr = min(8, nv - r0);
+                                const int nr = min(SR, nv - r0);
                                 for (int i = 0; i < nr; i++) {
                                     const int rl = __ffs(m) - 1;   // lane (tile row 32 q + rl) of stored row r0 + i
                                     m &= m - 1;
-                                    const float sa_i = sb[512 + i];
+                                    const float sa_i = sb[SR * 64 + i];
                                     const float gg = sb[i * 64 + lane] * (sa_i * bsg[half]);
                                     const float uu = sb[i * 64 + 32 + lane] * (sa_i * bsu[half]);
                                     const float hvv = gg / (1.0f + expf(-gg)) * uu;
@@ -408,9 +425,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         continue;
                     }
 #pragma unroll
-                    for (int half = 0; half < 2; half++) {
+                    for (int half = 0; half < NH; half++) {
                         float gv[32], uv[32];
-                        const int c0 = 64 * g + 32 * half;
+                        const int c0 = GC * g + 32 * half;
                         tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, gv, uv);
 #pragma unroll
                         for (int c = 0; c < 32; c++) {
@@ -469,10 +486,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     // scales to the chunked layout the down GEMM's tensor cores read
                     if (valid) {
                         const long long prow = static_cast<long long>(mi) * 128 + r;
-                        const int col0 = nb * 128 + 64 * g;
-                        uint32_t w[16];
+                        const int col0 = nb * 128 + GC * g;
+                        uint32_t w[8 * NH];
 #pragma unroll
-                        for (int b = 0; b < 2; b++) {
+                        for (int b = 0; b < NH; b++) {
                             float amax = 0.0f;
 #pragma unroll
                             for (int c = 0; c < 32; c++) amax = fmaxf(amax, fabsf(hv[32 * b + c]));
@@ -488,7 +505,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         }
                         uint4* dst = reinterpret_cast<uint4*>(p.hq + prow * p.I + col0);
 #pragma unroll
-                        for (int v4 = 0; v4 < 4; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                        for (int v4 = 0; v4 < 2 * NH; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
                     }
                     continue;
                 }
@@ -577,7 +594,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                 }
                 if (!ok) break;
                 store_rows_coalesced<NC, BSCALE == BSCALE_ROW>(
-                    acc_r, reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * EPI_WARP_FLOATS,
+                    acc_r, reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * EWF,
                     valid ? p.o + static_cast<size_t>(row) * p.H + n0 : nullptr,
                     p.b_scale + static_cast<size_t>(e) * p.b_rows + n0, rw, lane);
             }
@@ -593,12 +610,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
     }
 }
 
-template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(gemm_threads<EPI>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
-    gemm_body<KIND, BSCALE, PROMOTE, BN, STAGES>(tmA, tmB, p, p.n_blocks, smem_raw);
+    gemm_body<KIND, BSCALE, PROMOTE, BN, STAGES, EPI>(tmA, tmB, p, p.n_blocks, smem_raw);
 }
 
 // Down GEMM whose tile width is chosen on the device: the dispatch's scan

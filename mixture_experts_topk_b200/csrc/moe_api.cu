@@ -531,14 +531,14 @@ static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, u
     return MOE_OK;
 }
 
-template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES>
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8>
 static moe_status launch_gemm(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
                               cudaStream_t st) {
-    using S = GemmSmem<BN, STAGES>;
+    using S = GemmSmem<BN, STAGES, EPI>;
     static_assert(S::TOTAL <= 232448, "shared memory of the GEMM exceeds 227 KB");
-    auto kern = grouped_gemm_kernel<KIND, BSCALE, PROMOTE, BN, STAGES>;
+    auto kern = grouped_gemm_kernel<KIND, BSCALE, PROMOTE, BN, STAGES, EPI>;
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL));
-    LAUNCH(pdl, "grouped_gemm_kernel", kern, grid, GEMM_THREADS, S::TOTAL, st, ta, tb, p);
+    LAUNCH(pdl, "grouped_gemm_kernel", kern, grid, gemm_threads<EPI>(), S::TOTAL, st, ta, tb, p);
     return MOE_OK;
 }
 
@@ -588,7 +588,7 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4>(h->pdl, ta, tb, p, grid, st);
+    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16>(h->pdl, ta, tb, p, grid, st);
     return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4>(h->pdl, ta, tb, p, grid, st);
 }
 
