@@ -325,8 +325,9 @@ def run_ours(args, rank, world, local_rank):
         "kernel_ms": per,
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
-        # router 2 + dispatch 4 (+ amax for NVFP4) + gate/up + down + combine
-        "gpu_launches": (10 if wl.fmt == FMT_NVFP4 else 9) * args.steps,
+        # router 2 + dispatch (hist, scan, rank, quantise; one fused kernel for the
+        # first three when T*k <= 1024; + amax for NVFP4) + gate/up + down + combine
+        "gpu_launches": (2 + (2 if T * wl.k <= 1024 else 4) + (1 if wl.fmt == FMT_NVFP4 else 0) + 3) * args.steps,
         "clocks": clk.summary(),
     }
     del graph

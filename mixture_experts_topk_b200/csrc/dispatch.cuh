@@ -204,6 +204,94 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
     }
 }
 
+// Small batches (A <= DISPATCH_CHUNK assignments, one chunk): histogram,
+// scan, tile table, tile choice and stable ranks in one 1024-thread CTA, with
+// the same results as hist_kernel + scan_kernel + rank_kernel on one chunk:
+// thread a takes assignment a; a warp match gives its rank among equal ids of
+// its warp; per-(warp, expert) counts are summed and scanned over experts
+// (count + (row tiles << 20), as in scan_kernel) and then over warps.
+__global__ void __launch_bounds__(DISPATCH_CHUNK) dispatch_small_kernel(
+    const int32_t* ids, int A, int E, int32_t* counts, int32_t* offsets, int32_t* tiles, int32_t* num_tiles,
+    int32_t* tile_ptr, int32_t* pick_out, PickerParams pq, int32_t* perm, int32_t* inv, int32_t* status) {
+    pdl_wait();
+    pdl_trigger();
+    __shared__ int wc[32][256];
+    __shared__ int warp_tot[8];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 32 * 256; i += blockDim.x) wc[i >> 8][i & 255] = 0;
+    __syncthreads();
+    int e = (tid < A) ? ids[tid] : -1;
+    const bool valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
+    if (tid < A && !valid) report(status, ST_BOUNDS, WHERE_DISPATCH);
+    if (!valid) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (valid && rank == 0) wc[warp][e] = __popc(peers);
+    __syncthreads();
+    // per-expert totals and the packed exclusive scan (threads 0..255 = warps 0..7)
+    int c = 0;
+    if (tid < E)
+        for (int w = 0; w < 32; w++) c += wc[w][tid];
+    const int nt_e = (c + TILE_M - 1) / TILE_M;
+    const int packed = c + (nt_e << 20);
+    int inc = packed;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += n;
+    }
+    if (warp < 8 && lane == 31) warp_tot[warp] = inc;
+    const int touched = __syncthreads_count(tid < E && c > 0);
+    if (warp == 0) {
+        int w = lane < 8 ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += n;
+        }
+        if (lane < 8) warp_tot[lane] = w;
+    }
+    __syncthreads();
+    if (tid < 256) {
+        const int excl = (warp ? warp_tot[warp - 1] : 0) + inc - packed;
+        const int total = warp_tot[7];
+        const int off_e = excl & 0xFFFFF, tptr_e = excl >> 20;
+        if (tid == 0) {
+            offsets[E] = total & 0xFFFFF;
+            *num_tiles = total >> 20;
+            tile_ptr[E] = total >> 20;
+            pick_out[0] = pick_down_tile(pq, total >> 20, touched);
+            pick_out[1] = pick_split(pq, total >> 20, total & 0xFFFFF);
+        }
+        if (tid < E) {
+            counts[tid] = c;
+            offsets[tid] = off_e;
+            tile_ptr[tid] = tptr_e;
+            for (int i = 0; i < nt_e; i++) {
+                tiles[2 * (tptr_e + i)] = tid;
+                tiles[2 * (tptr_e + i) + 1] = off_e + TILE_M * i;
+            }
+            // per-warp bases of this expert's slots, warps in order
+            int run = off_e;
+            for (int w = 0; w < 32; w++) {
+                const int v = wc[w][tid];
+                wc[w][tid] = run;
+                run += v;
+            }
+        }
+    }
+    __syncthreads();
+    if (tid < A) {
+        if (valid) {
+            const int slot = wc[warp][e] + rank;
+            perm[slot] = tid;
+            inv[tid] = slot;
+        } else {
+            inv[tid] = -1;
+        }
+    }
+}
+
 // Quantise each token row of X once and write it to the k slots of its
 // assignments (LightMoE README: BF16 input quantisation inside the layer).
 // FP8_ROW: s = amax/448 over the row; BLOCK128: per 128 columns;

@@ -405,13 +405,19 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
     const int A = T * c.k;
     const int nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
     int32_t* chunk = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + h->ws.chunk);
-    if (A > 0) {
-        LAUNCH(h->pdl, "hist_kernel", hist_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.status);
+    if (A > 0 && nchunks == 1) {
+        // one chunk: histogram, scan and ranks in one CTA
+        LAUNCH(h->pdl, "dispatch_small_kernel", dispatch_small_kernel, 1, DISPATCH_CHUNK, 0, st, ids, A, c.E,
+               v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr, v.pick, h->picker, v.perm, v.inv, v.status);
+    } else {
+        if (A > 0) {
+            LAUNCH(h->pdl, "hist_kernel", hist_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.status);
+        }
+        LAUNCH(h->pdl, "scan_kernel", scan_kernel, 1, 256, 0, st, chunk, nchunks, c.E, v.counts, v.offsets, v.tiles,
+               v.num_tiles, v.tile_ptr, v.pick, h->picker);
+        if (A == 0) return MOE_OK;
+        LAUNCH(h->pdl, "rank_kernel", rank_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.perm, v.inv);
     }
-    LAUNCH(h->pdl, "scan_kernel", scan_kernel, 1, 256, 0, st, chunk, nchunks, c.E, v.counts, v.offsets, v.tiles,
-           v.num_tiles, v.tile_ptr, v.pick, h->picker);
-    if (A == 0) return MOE_OK;
-    LAUNCH(h->pdl, "rank_kernel", rank_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.perm, v.inv);
     const int qgrid = std::min((T + 7) / 8, 8 * h->num_sms);
     if (c.fmt == MOE_FMT_NVFP4) {
         int32_t* amax = reinterpret_cast<int32_t*>(v.x_global);
