@@ -196,6 +196,17 @@ moe_status moe_set_tile_config(moe_handle* h, int down_bn);
  * plain stream order.  Host state only; MOE_ERR_INVALID_ARG for other values. */
 moe_status moe_set_launch_options(moe_handle* h, int pdl);
 
+/* Limit, in SM clock cycles, of every wait of the GEMM kernels on another
+ * role or CTA (stage, accumulator and exchange barriers); default 2e9 (about
+ * 1 s).  A wait that runs out records MOE_ERR_DEVICE_TIMEOUT and the role in
+ * the status word, and the kernel leaves its loops; it still waits (with a
+ * fixed limit) for its own copies and MMAs in flight and frees its TMEM, so
+ * the context stays usable (read the status with moe_get_status).  A small
+ * value makes the waits run out on purpose (failure-detection tests).  No
+ * counterpart in the pages.  Host state only; MOE_ERR_INVALID_ARG for
+ * cycles <= 0. */
+moe_status moe_set_wait_limit(moe_handle* h, long long cycles);
+
 /* Parameters of the wave cost model that picks the down GEMM's tile width
  * from the runtime expert histogram (RaMP abstract: four-parameter wave cost
  * model fitted from a one-time profiling sweep).  The dispatch's scan kernel

@@ -62,6 +62,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Limit of the waits for a CTA's own copies and MMAs in flight (the drain
+// before it exits or frees TMEM).  Those always finish, so this limit is fixed;
+// the configurable limit applies to the waits between roles and CTAs.
+constexpr long long DRAIN_LIMIT = 2000000000LL;
+
 // Wait until the phase with the given parity completed; give up after
 // `limit` clock cycles (returns false, the caller records ST_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {

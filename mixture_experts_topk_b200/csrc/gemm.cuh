@@ -281,7 +281,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
             }
             // loads still in flight land before the CTA may exit
             const uint32_t first = it > STAGES ? it - STAGES : 0;
-            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, limit);
+            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, DRAIN_LIMIT);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -326,7 +326,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
             }
             if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
             mma_commit(drain);                 // every issued MMA has completed ...
-            mbar_wait(drain, 0, limit);        // ... before TMEM can be released
+            mbar_wait(drain, 0, DRAIN_LIMIT);        // ... before TMEM can be released
         }
     } else {
         // ------------------------------------------------------------ epilogue

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
             }
             const uint32_t first = it > F4_STAGES ? it - F4_STAGES : 0;
-            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % F4_STAGES], (j / F4_STAGES) & 1, limit);
+            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % F4_STAGES], (j / F4_STAGES) & 1, DRAIN_LIMIT);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
             if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
             mma_commit(drain);
-            mbar_wait(drain, 0, limit);
+            mbar_wait(drain, 0, DRAIN_LIMIT);
         }
     } else {
         // ------------------------------------------------------------ epilogue

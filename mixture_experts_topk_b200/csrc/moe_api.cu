@@ -729,6 +729,13 @@ extern "C" moe_status moe_set_tile_config(moe_handle* h, int down_bn) {
     return MOE_OK;
 }
 
+extern "C" moe_status moe_set_wait_limit(moe_handle* h, long long cycles) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_wait_limit: null handle");
+    if (cycles <= 0) return fail(MOE_ERR_INVALID_ARG, "moe_set_wait_limit: cycles must be positive (got %lld)", cycles);
+    h->spin_limit = cycles;
+    return MOE_OK;
+}
+
 extern "C" moe_status moe_set_launch_options(moe_handle* h, int pdl) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_launch_options: null handle");
     if (pdl != 0 && pdl != 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_launch_options: pdl must be 0 or 1 (got %d)", pdl);
