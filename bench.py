@@ -124,6 +124,20 @@ def algorithmic_work(wl, T, counts):
     return flops_tensor, flops_router, byts, touched
 
 
+def max_over_ranks(ms, world, device):
+    """The largest of the ranks' times (every rank calls it, in the same order)."""
+    if world == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, steps, world, ms_max):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max * 1e-3)
+
+
 def run_ours(args, rank, world, local_rank):
     from mixture_experts_topk_b200 import native
     dev = torch.device("cuda", local_rank)
@@ -194,12 +208,7 @@ def run_ours(args, rank, world, local_rank):
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     st, msg = layer.status()
     if st != 0:
         raise RuntimeError(f"device status after the timed steps: {msg}")
@@ -272,11 +281,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_steps(args.steps, ev0, ev1)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
 
     fl_t, fl_r, byts, touched = algorithmic_work(wl, T, counts)
     pk, pk_kind = peaks()
@@ -289,10 +294,9 @@ def run_ours(args, rank, world, local_rank):
     # fp32 SIMT peak of the router: 148 SMs x 128 FMA lanes x 2 FLOP x max SM clock
     simt_peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6
     t_roof_ms = max(fl_t / (fp8_peak * 1e12) + fl_r / simt_peak, byts / (pk["hbm_gbs"] * 1e9)) * 1e3
-    tokens_total = world * T * args.steps
     out = {
         "metric": METRIC,
-        "value": tokens_total / (ms_max * 1e-3),
+        "value": job_throughput(T, args.steps, world, ms_max),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -323,7 +327,7 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"{pk_kind} bf16_tflops_sustained x {4 if wl.fmt == FMT_NVFP4 else 2} "
                                     "(nominal fp8:bf16 = 2, fp4:bf16 = 4)"},
         "kernel_ms": per,
-        "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(T, args.steps, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
         # router 2 + dispatch (hist, scan, rank, quantise; one fused kernel for the
         # first three when T*k <= 1024; + amax for NVFP4) + gate/up + down + combine
