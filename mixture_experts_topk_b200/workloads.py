@@ -19,6 +19,13 @@ FMT_NVFP4 = 2         # e2m1, e4m3 scale per 16-element block, fp32 global scale
 SCORE_SOFTMAX = 0     # softmax over the selected k logits
 SCORE_SIGMOID = 1     # sigmoid of the selected k logits, normalised to sum 1
 
+# gated activation of the expert MLP, h = act(gate, up)
+ACT_SWIGLU = 0          # silu(g) u
+ACT_SWIGLU_BOUNDED = 1  # silu(min(g, L)) clamp(u, -L, L)
+ACT_SWIGLU_OAI = 2      # g' sigmoid(alpha g') (u' + 1), g' = min(g, L), u' = clamp(u, -L, L)
+ACT_GEGLU = 3           # gelu(g) u (erf form)
+ACT_REGLU = 4           # relu(g) u
+
 
 @dataclass(frozen=True)
 class Workload:
@@ -33,6 +40,9 @@ class Workload:
     router_init: str            # "normal" (N(0,1/H)) or "uniform" (U(-sqrt(3/H), sqrt(3/H)))
     zipf_s: float = 0.0         # per-expert router bias exponent; 0 = no bias
     hidden_global_scale: float = 0.0   # static NVFP4 hidden scale (checkpoint-style input)
+    act: int = ACT_SWIGLU
+    act_alpha: float = 0.0
+    act_limit: float = 0.0
     notes: str = ""
 
     @property

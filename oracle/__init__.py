@@ -44,7 +44,8 @@ class _Layer(ctypes.Structure):
                 ("k", ctypes.c_int), ("score", ctypes.c_int), ("fmt", ctypes.c_int),
                 ("hidden_global", ctypes.c_float),
                 ("gate", _Proj), ("up", _Proj), ("down", _Proj),
-                ("expert_slot", ctypes.c_void_p)]
+                ("expert_slot", ctypes.c_void_p),
+                ("act", ctypes.c_int), ("act_alpha", ctypes.c_double), ("act_limit", ctypes.c_double)]
 
 
 def lib():
@@ -74,6 +75,7 @@ def lib():
             "orc_num_threads": (I, []),
             "orc_pick_down_tile": (I, [P, I, I, I, I, I64, I64, I64, I64, P]),
             "orc_pick_split": (I, [P, I, I, I, I64, I]),
+            "orc_glu": (ctypes.c_double, [I, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -182,6 +184,15 @@ def pick_down_tile(counts, H, I, num_sms, alpha, beta, bw, gamma):
     return c, costs
 
 
+ACT_SWIGLU, ACT_SWIGLU_BOUNDED, ACT_SWIGLU_OAI, ACT_GEGLU, ACT_REGLU = range(5)
+
+
+def glu(act, g, u, alpha=0.0, limit=0.0):
+    """Gated activation act(g, u) in fp64 (scalars or arrays)."""
+    f = np.vectorize(lambda a, b: lib().orc_glu(act, float(alpha), float(limit), float(a), float(b)))
+    return f(np.asarray(g, np.float64), np.asarray(u, np.float64))
+
+
 def pick_split(counts, split_nb, split_kb, o_rows, num_sms):
     """K split S of the FP8_ROW down GEMM from the expert histogram (1 = none)."""
     counts = _c(counts, np.int32)
@@ -235,6 +246,7 @@ class Layer:
         st.H, st.I, st.E, st.k = wl.H, wl.I, wl.E, wl.k
         st.score, st.fmt = wl.score, wl.fmt
         st.hidden_global = float(wl.hidden_global_scale)
+        st.act, st.act_alpha, st.act_limit = wl.act, float(wl.act_alpha), float(wl.act_limit)
         for p in ("gate", "up", "down"):
             q = _c(weights[p + "_q"], np.uint8)
             s = np.ascontiguousarray(weights[p + "_s"])

@@ -421,6 +421,28 @@ static void dequant_rows(int fmt, int rows, int K, const uint8_t* codes,
         dequant_act_row(fmt, codes + r * cb, (const uint8_t*)scales + r * sb, g, K, out + (int64_t)r * K);
 }
 
+double orc_glu(int act, double alpha, double limit, double g, double u)
+{
+    switch (act) {
+    case ORC_ACT_SWIGLU_BOUNDED: {
+        double gc = g < limit ? g : limit;
+        double uc = u < -limit ? -limit : (u > limit ? limit : u);
+        return gc / (1.0 + exp(-gc)) * uc;
+    }
+    case ORC_ACT_SWIGLU_OAI: {
+        double gc = g < limit ? g : limit;
+        double uc = u < -limit ? -limit : (u > limit ? limit : u);
+        return gc / (1.0 + exp(-alpha * gc)) * (uc + 1.0);
+    }
+    case ORC_ACT_GEGLU:
+        return 0.5 * g * (1.0 + erf(g / sqrt(2.0))) * u;
+    case ORC_ACT_REGLU:
+        return (g > 0.0 ? g : 0.0) * u;
+    default:
+        return g / (1.0 + exp(-g)) * u;
+    }
+}
+
 void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes,
                      const void* a_scales, float x_global, double* h,
                      uint8_t* hq_codes, void* hq_scales, double* o)
@@ -440,7 +462,7 @@ void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes
             for (int r = 0; r < rows; r++) {
                 double g = dot64(a + (int64_t)r * H, wg, H);
                 double u = dot64(a + (int64_t)r * H, wu, H);
-                hh[(int64_t)r * I + n] = g / (1.0 + exp(-g)) * u;     /* SiLU(gate) * up */
+                hh[(int64_t)r * I + n] = orc_glu(L->act, L->act_alpha, L->act_limit, g, u);
             }
         }
         free(wg);

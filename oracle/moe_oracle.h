@@ -115,7 +115,19 @@ typedef struct {
     float hidden_global;   /* NVFP4 static hidden scale */
     orc_proj gate, up, down;   /* gate/up: N=I, K=H.  down: N=H, K=I */
     const int32_t* expert_slot; /* [E] -> index into the weight arrays, -1 = not provided; NULL = identity */
+    int act;               /* gated activation, ORC_ACT_* */
+    double act_alpha, act_limit;
 } orc_layer;
+
+/* Gated activations h = act(g, u) of the expert MLP, in fp64 (LightMoE README,
+ * "Compatibility": SwiGLU, bounded SwiGLU, SwiGLU-OAI, GeGLU, ReGLU).
+ *   SWIGLU          silu(g) u,  silu(g) = g / (1 + exp(-g))
+ *   SWIGLU_BOUNDED  silu(min(g, L)) clamp(u, -L, L)
+ *   SWIGLU_OAI      g' / (1 + exp(-alpha g')) (u' + 1),  g' = min(g, L), u' = clamp(u, -L, L)
+ *   GEGLU           g Phi(g) u,  Phi(g) = (1 + erf(g / sqrt 2)) / 2
+ *   REGLU           max(g, 0) u */
+enum { ORC_ACT_SWIGLU = 0, ORC_ACT_SWIGLU_BOUNDED = 1, ORC_ACT_SWIGLU_OAI = 2, ORC_ACT_GEGLU = 3, ORC_ACT_REGLU = 4 };
+double orc_glu(int act, double alpha, double limit, double g, double u);
 
 /* dequantised weight row (fp64, exact) */
 void orc_weight_row(const orc_layer* L, const orc_proj* P, int N, int K, int e, int n, double* out);

@@ -93,6 +93,48 @@ def test_single_expert_is_dense_swiglu_mlp(fmt):
     np.testing.assert_allclose(y, o_ref.numpy(), rtol=1e-12, atol=1e-12)
 
 
+def _torch_glu(act, g, u, alpha, limit):
+    """The gated activations written with torch fp64 library routines."""
+    F = torch.nn.functional
+    if act == W.ACT_SWIGLU:
+        return F.silu(g) * u
+    if act == W.ACT_SWIGLU_BOUNDED:
+        return F.silu(torch.clamp(g, max=limit)) * torch.clamp(u, -limit, limit)
+    if act == W.ACT_SWIGLU_OAI:
+        gc = torch.clamp(g, max=limit)
+        return gc * torch.sigmoid(alpha * gc) * (torch.clamp(u, -limit, limit) + 1.0)
+    if act == W.ACT_GEGLU:
+        return F.gelu(g, approximate="none") * u
+    return F.relu(g) * u
+
+
+ACTS = [(W.ACT_SWIGLU, 0.0, 0.0), (W.ACT_SWIGLU_BOUNDED, 0.0, 0.25), (W.ACT_SWIGLU_OAI, 1.702, 0.3),
+        (W.ACT_GEGLU, 0.0, 0.0), (W.ACT_REGLU, 0.0, 0.0)]
+
+
+@pytest.mark.parametrize("act,alpha,limit", ACTS)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_single_expert_is_the_dense_gated_mlp_of_each_activation(fmt, act, alpha, limit):
+    """E = 1, top-1 with each gated activation: the hidden equals the dense MLP
+    written with torch fp64 routines (the limits are chosen inside the range of
+    the pre-activations, so the clamps bind on part of the elements)."""
+    wl = W.custom(H=256, I=256, E=1, k=1, fmt=fmt, act=act, act_alpha=alpha, act_limit=limit)
+    d = synth.layer(wl, seed=8)
+    L = oracle.Layer(wl, d)
+    x = synth.tokens(wl, 5, seed=8)
+    xf = x.to(torch.float32).numpy()
+    g_x = oracle.nvfp4_global(xf) if fmt == W.FMT_NVFP4 else 0.0
+    codes, scales = oracle.quant_rows(fmt, xf, g_x)
+    h, hq, hs, o = L.expert_rows(0, codes, scales, g_x)
+    a = torch.from_numpy(deq_act(wl, codes, scales, g_x))
+    g = a @ torch.from_numpy(deq_weight(wl, d, "gate", 0)).T
+    u = a @ torch.from_numpy(deq_weight(wl, d, "up", 0)).T
+    if limit > 0.0:
+        assert (g > limit).any() and (u.abs() > limit).any()
+    h_ref = _torch_glu(act, g, u, alpha, limit)
+    np.testing.assert_allclose(h, h_ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_equal_logits_average_the_first_k_experts(fmt):
     wl = W.custom(H=256, I=256, E=5, k=3, fmt=fmt)

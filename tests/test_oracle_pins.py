@@ -283,6 +283,47 @@ def test_pick_split_hand_examples():
     assert oracle.pick_split(np.zeros(8, np.int32), **mix) == 1
 
 
+# ------------------------------------------------------------------ gated activations
+def test_gated_activations_closed_forms():
+    # silu(1) = 1 / (1 + e^-1); Phi(1) = 0.8413447460685429 (normal CDF table value)
+    assert oracle.glu(oracle.ACT_SWIGLU, 1.0, 2.0) == pytest.approx(2.0 / (1.0 + np.exp(-1.0)), rel=1e-15)
+    assert oracle.glu(oracle.ACT_GEGLU, 1.0, 1.0) == pytest.approx(0.8413447460685429, rel=1e-15)
+    assert oracle.glu(oracle.ACT_GEGLU, -1.0, 1.0) == pytest.approx(-(1.0 - 0.8413447460685429), rel=1e-14)
+    # relu gate: exact
+    assert oracle.glu(oracle.ACT_REGLU, -3.0, 5.0) == 0.0
+    assert oracle.glu(oracle.ACT_REGLU, 3.0, 5.0) == 15.0
+    # bounded: the gate is capped from above only, the up projection on both sides
+    L = 10.0
+    assert oracle.glu(oracle.ACT_SWIGLU_BOUNDED, 50.0, 50.0, limit=L) == \
+        pytest.approx(10.0 / (1.0 + np.exp(-10.0)) * 10.0, rel=1e-15)
+    assert oracle.glu(oracle.ACT_SWIGLU_BOUNDED, -50.0, -50.0, limit=L) == \
+        pytest.approx(-50.0 / (1.0 + np.exp(50.0)) * -10.0, rel=1e-15)
+    # OAI: g sigmoid(alpha g) (u + 1) with the same clamps
+    assert oracle.glu(oracle.ACT_SWIGLU_OAI, 2.0, 3.0, alpha=1.702, limit=7.0) == \
+        pytest.approx(2.0 / (1.0 + np.exp(-3.404)) * 4.0, rel=1e-15)
+    assert oracle.glu(oracle.ACT_SWIGLU_OAI, 9.0, -9.0, alpha=1.702, limit=7.0) == \
+        pytest.approx(7.0 / (1.0 + np.exp(-1.702 * 7.0)) * -6.0, rel=1e-15)
+    # every variant is 0 at g = 0
+    for act in range(5):
+        assert oracle.glu(act, 0.0, 3.0, alpha=1.702, limit=7.0) == 0.0
+
+
+def test_gated_activations_match_torch_library_routines():
+    rng = np.random.default_rng(0)
+    g, u = rng.normal(0, 3, 2000), rng.normal(0, 3, 2000)
+    gt, ut = torch.from_numpy(g), torch.from_numpy(u)
+    F = torch.nn.functional
+    np.testing.assert_allclose(oracle.glu(oracle.ACT_SWIGLU, g, u), (F.silu(gt) * ut).numpy(), rtol=1e-14, atol=1e-300)
+    np.testing.assert_allclose(oracle.glu(oracle.ACT_GEGLU, g, u), (F.gelu(gt) * ut).numpy(), rtol=1e-13, atol=1e-300)
+    np.testing.assert_array_equal(oracle.glu(oracle.ACT_REGLU, g, u), (F.relu(gt) * ut).numpy())
+    ref = F.silu(torch.clamp(gt, max=2.0)) * torch.clamp(ut, -2.0, 2.0)
+    np.testing.assert_allclose(oracle.glu(oracle.ACT_SWIGLU_BOUNDED, g, u, limit=2.0), ref.numpy(), rtol=1e-14, atol=1e-300)
+    gc = torch.clamp(gt, max=2.0)
+    ref = gc * torch.sigmoid(1.702 * gc) * (torch.clamp(ut, -2.0, 2.0) + 1.0)
+    np.testing.assert_allclose(oracle.glu(oracle.ACT_SWIGLU_OAI, g, u, alpha=1.702, limit=2.0), ref.numpy(),
+                               rtol=1e-13, atol=1e-300)
+
+
 # ------------------------------------------------------------------ MX32 hidden rule
 def test_mx32_quant_hand_example():
     x = np.zeros((4, 64), np.float32)
