@@ -138,11 +138,24 @@ def job_throughput(tokens_per_rank, steps, world, ms_max):
     return world * tokens_per_rank * steps / (ms_max * 1e-3)
 
 
+# gated activations: (act id, alpha, limit); the clamp of 10 is the bounded-SwiGLU
+# setting the LightMoE README gives, alpha 1.702 / limit 7 the common SwiGLU-OAI one
+ACTS = {"swiglu": (0, 0.0, 0.0), "bounded": (1, 0.0, 10.0), "oai": (2, 1.702, 7.0), "geglu": (3, 0.0, 0.0),
+        "reglu": (4, 0.0, 0.0)}
+
+
+def workload_of(args):
+    import dataclasses
+    wl = WORKLOADS[args.workload]
+    act, alpha, limit = ACTS[args.act]
+    return dataclasses.replace(wl, act=act, act_alpha=alpha, act_limit=limit)
+
+
 def run_ours(args, rank, world, local_rank):
     from mixture_experts_topk_b200 import native
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     T = args.tokens
     d = synth.layer(wl, seed=0, device=dev)
     layer = native.Layer(wl, d, max_T=T, device=dev)
@@ -307,7 +320,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8-e4m3 (fp32 accumulate)" if wl.fmt != FMT_NVFP4 else "nvfp4-e2m1 (fp32 accumulate)",
         "data": "synthetic (seeded; X ~ N(0,1) bf16, weights ~ N(0,1/fan_in) quantised offline)",
-        "config": {"workload": f"{wl.name} T={T}", "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+        "config": {"workload": f"{wl.name} T={T}", "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "activation": args.act,
                    "T_per_gpu": T, "parallelism": f"replicas x{world} (token batches)",
                    "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (byts / 1e9),
                    "touched_experts": touched, "m_tiles": m_tiles,
@@ -365,7 +378,7 @@ def cpu_baseline(wl, T, n_sel, seed=0):
 
 
 def run_reference(args):
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     T = args.tokens
     for _ in range(args.warmup):
         cpu_baseline(wl, T, 1)
@@ -395,6 +408,8 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--down-bn", type=int, default=0, help="down GEMM tile width (0 = chosen per call)")
+    ap.add_argument("--act", default="swiglu", choices=sorted(ACTS),
+                    help="gated activation of the expert MLP (bounded: clamp 10; oai: alpha 1.702, limit 7)")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="timed steps replay a CUDA graph of the layer call, or call it directly")
     args = ap.parse_args()
@@ -417,7 +432,7 @@ def main():
     out = run_ours(args, rank, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_baseline(WORKLOADS[args.workload], args.tokens, args.ref_sample)
+            cb = cpu_baseline(workload_of(args), args.tokens, args.ref_sample)
             cb.pop("seconds")
             out["cpu_baseline"] = cb
         print(json.dumps(out))

@@ -69,7 +69,29 @@ typedef struct {
     int max_T;                    /* largest T a workspace must hold */
     float hidden_global_scale;    /* NVFP4 only: static fp32 scale of the hidden (a checkpoint
                                      scale, LightMoE README "set_activation_scales") */
+    int act;                      /* MOE_ACT_*, the gated activation h = act(gate, up) */
+    float act_alpha;              /* SWIGLU_OAI: sigmoid slope alpha */
+    float act_limit;              /* SWIGLU_BOUNDED, SWIGLU_OAI: clamp limit L > 0 */
 } moe_config;
+
+/* Gated activations of the expert MLP (LightMoE README, "Compatibility": complete
+ * inference supports bounded SwiGLU, SwiGLU-OAI, GeGLU and ReGLU besides SwiGLU;
+ * "MoE inference": activation_clamp for bounded SwiGLU).  The pages name them
+ * without formulas; the forms computed are, with silu(g) = g / (1 + e^-g):
+ *   SWIGLU          silu(g) * u
+ *   SWIGLU_BOUNDED  silu(min(g, L)) * clamp(u, -L, L)
+ *   SWIGLU_OAI      g' / (1 + e^(-alpha g')) * (u' + 1),  g' = min(g, L), u' = clamp(u, -L, L)
+ *   GEGLU           0.5 g (1 + erf(g / sqrt 2)) * u
+ *   REGLU           max(g, 0) * u
+ * moe_init returns MOE_ERR_INVALID_ARG for an unknown act, L <= 0 where a
+ * limit is used, or alpha <= 0 for SWIGLU_OAI. */
+enum {
+    MOE_ACT_SWIGLU = 0,
+    MOE_ACT_SWIGLU_BOUNDED = 1,
+    MOE_ACT_SWIGLU_OAI = 2,
+    MOE_ACT_GEGLU = 3,
+    MOE_ACT_REGLU = 4
+};
 
 typedef struct moe_handle moe_handle;
 

@@ -279,6 +279,27 @@ __device__ __forceinline__ float e4m3_to_f(uint8_t c) {
     const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
     return __half2float(__half(h));
 }
+// Gated activation h = act(g, u) of the expert MLP in fp32 (LightMoE README,
+// "Compatibility"): 0 SwiGLU silu(g) u; 1 bounded SwiGLU silu(min(g, L))
+// clamp(u, -L, L); 2 SwiGLU-OAI g' sigmoid(alpha g') (u' + 1) with the same
+// clamps; 3 GeGLU 0.5 g (1 + erf(g / sqrt 2)) u; 4 ReGLU max(g, 0) u.
+// The GEMM kernels are instantiated per activation (ACT is a compile-time
+// constant there), so each epilogue is straight-line code for its activation.
+template <int ACT>
+__device__ __forceinline__ float glu(float g, float u, float alpha, float limit) {
+    if constexpr (ACT == 0) {
+        return g / (1.0f + expf(-g)) * u;
+    } else if constexpr (ACT == 1 || ACT == 2) {
+        const float gc = fminf(g, limit), uc = fminf(fmaxf(u, -limit), limit);
+        if constexpr (ACT == 1) return gc / (1.0f + expf(-gc)) * uc;
+        else return gc / (1.0f + expf(-alpha * gc)) * (uc + 1.0f);
+    } else if constexpr (ACT == 3) {
+        return 0.5f * g * (1.0f + erff(g * 0.70710678118654752f)) * u;
+    } else {
+        return fmaxf(g, 0.0f) * u;
+    }
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 

@@ -58,6 +58,8 @@ struct GemmParams {
     float* hs;                  //   BLOCK128: [A][I] + fp32 scales hs [A][I/128]
     uint8_t* hsf;
     int I;
+    int act;                    // gate/up: gated activation (the kernel is instantiated for it)
+    float act_alpha, act_limit;
     float* o;                   // down: [A][H] fp32
     int H;
     const int32_t* perm;        // down: slot -> t*k + j
@@ -199,7 +201,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8>
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8, int ACT = 0>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                                           const int n_blocks, uint8_t* smem_raw) {
     static_assert(EPI == 8 || (EPI == 16 && KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW && !PROMOTE && BN == 256),
@@ -408,7 +410,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                                     const float sa_i = sb[SR * 64 + i];
                                     const float gg = sb[i * 64 + lane] * (sa_i * bsg[half]);
                                     const float uu = sb[i * 64 + 32 + lane] * (sa_i * bsu[half]);
-                                    const float hvv = gg / (1.0f + expf(-gg)) * uu;
+                                    const float hvv = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
                                     float amax = fabsf(hvv);
 #pragma unroll
                                     for (int off = 16; off > 0; off >>= 1)
@@ -433,7 +435,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         for (int c = 0; c < 32; c++) {
                             const float gg = gv[c] * (sa * __shfl_sync(0xffffffffu, bsg[half], c));
                             const float uu = uv[c] * (sa * __shfl_sync(0xffffffffu, bsu[half], c));
-                            hv[32 * half + c] = gg / (1.0f + expf(-gg)) * uu;
+                            hv[32 * half + c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
                         }
                     }
                     tc_fence_before();
@@ -478,7 +480,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     }
                     if (!ok) break;
 #pragma unroll
-                    for (int c = 0; c < 64; c++) hv[c] = ag[c] / (1.0f + expf(-ag[c])) * au[c];
+                    for (int c = 0; c < 64; c++) hv[c] = glu<ACT>(ag[c], au[c], p.act_alpha, p.act_limit);
                 }
                 if (BSCALE == BSCALE_ROW) {
                     // MX requantisation: power-of-two scale per 32 hidden columns (all
@@ -610,12 +612,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
     }
 }
 
-template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI>
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI, int ACT>
 __global__ void __launch_bounds__(gemm_threads<EPI>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
-    gemm_body<KIND, BSCALE, PROMOTE, BN, STAGES, EPI>(tmA, tmB, p, p.n_blocks, smem_raw);
+    gemm_body<KIND, BSCALE, PROMOTE, BN, STAGES, EPI, ACT>(tmA, tmB, p, p.n_blocks, smem_raw);
 }
 
 // Down GEMM whose tile width is chosen on the device: the dispatch's scan

@@ -57,6 +57,8 @@ struct Fp4Params {
     const int32_t* x_amax;    // gate/up: amax bits of X (global scale = amax / 2688)
     const float* w_global;    // gate/up: [E][2] (gate, up); down: [E]
     float h_global;           // static hidden scale
+    int act;                  // gate/up: gated activation (the kernel is instantiated for it)
+    float act_alpha, act_limit;
     uint8_t* hq;              // gate/up out: hidden codes [rows][I/2], scale factors hsf
     uint8_t* hsf;
     int I;
@@ -68,7 +70,7 @@ struct Fp4Params {
     long long spin_limit;
 };
 
-template <int KIND>
+template <int KIND, int ACT>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     grouped_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const Fp4Params p) {
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 32; c++) {
                     const float gg = gv[c] * sg, uu = uv[c] * su;
-                    hv[c] = gg / (1.0f + expf(-gg)) * uu;
+                    hv[c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
                 }
                 if (valid) {
                     const int col0 = nb * 64 + 32 * g;      // first hidden column of this thread

@@ -214,6 +214,12 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: NVFP4 needs I to be a multiple of 256 (I=%d)", c.I);
     if (c.fmt == MOE_FMT_NVFP4 && !(c.hidden_global_scale > 0.0f))
         return fail(MOE_ERR_INVALID_ARG, "moe_init: NVFP4 needs a positive hidden_global_scale");
+    if (c.act < MOE_ACT_SWIGLU || c.act > MOE_ACT_REGLU)
+        return fail(MOE_ERR_INVALID_ARG, "moe_init: unknown activation %d", c.act);
+    if ((c.act == MOE_ACT_SWIGLU_BOUNDED || c.act == MOE_ACT_SWIGLU_OAI) && !(c.act_limit > 0.0f))
+        return fail(MOE_ERR_INVALID_ARG, "moe_init: this activation needs a positive act_limit");
+    if (c.act == MOE_ACT_SWIGLU_OAI && !(c.act_alpha > 0.0f))
+        return fail(MOE_ERR_INVALID_ARG, "moe_init: SWIGLU_OAI needs a positive act_alpha");
     moe_handle* h = new (std::nothrow) moe_handle;
     if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_init: out of host memory");
     h->cfg = c;
@@ -451,10 +457,10 @@ static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, u
                             uint32_t box_inner, uint32_t box_rows);
 static int max_m_tiles(const moe_config& c, int T);
 
-template <int KIND>
+template <int KIND, int ACT = 0>
 static moe_status launch_fp4(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const Fp4Params& p, int grid,
                              cudaStream_t st) {
-    auto kern = grouped_gemm_fp4_kernel<KIND>;
+    auto kern = grouped_gemm_fp4_kernel<KIND, ACT>;
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F4_SMEM));
     LAUNCH(pdl, "grouped_gemm_fp4_kernel", kern, grid, GEMM_THREADS, F4_SMEM, st, ta, tb, p);
     return MOE_OK;
@@ -491,6 +497,9 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     p.x_amax = reinterpret_cast<const int32_t*>(v.x_global);
     p.w_global = reinterpret_cast<const float*>(pw + (gate_up ? h->wl.gu_g : h->wl.d_g));
     p.h_global = c.hidden_global_scale;
+    p.act = c.act;
+    p.act_alpha = c.act_alpha;
+    p.act_limit = c.act_limit;
     p.hq = v.hq;
     p.hsf = static_cast<uint8_t*>(v.hs);
     p.I = c.I;
@@ -502,8 +511,14 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return gate_up ? launch_fp4<KIND_GATE_UP>(h->pdl, ta, tb, p, grid, st)
-                   : launch_fp4<KIND_DOWN>(h->pdl, ta, tb, p, grid, st);
+    if (!gate_up) return launch_fp4<KIND_DOWN>(h->pdl, ta, tb, p, grid, st);
+    switch (c.act) {
+    case MOE_ACT_SWIGLU_BOUNDED: return launch_fp4<KIND_GATE_UP, MOE_ACT_SWIGLU_BOUNDED>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_SWIGLU_OAI: return launch_fp4<KIND_GATE_UP, MOE_ACT_SWIGLU_OAI>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_GEGLU: return launch_fp4<KIND_GATE_UP, MOE_ACT_GEGLU>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_REGLU: return launch_fp4<KIND_GATE_UP, MOE_ACT_REGLU>(h->pdl, ta, tb, p, grid, st);
+    default: return launch_fp4<KIND_GATE_UP, MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, grid, st);
+    }
 }
 
 // ------------------------------------------------------------------ tensor maps
@@ -537,12 +552,12 @@ static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, u
     return MOE_OK;
 }
 
-template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8>
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8, int ACT = 0>
 static moe_status launch_gemm(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
                               cudaStream_t st) {
     using S = GemmSmem<BN, STAGES, EPI>;
     static_assert(S::TOTAL <= 232448, "shared memory of the GEMM exceeds 227 KB");
-    auto kern = grouped_gemm_kernel<KIND, BSCALE, PROMOTE, BN, STAGES, EPI>;
+    auto kern = grouped_gemm_kernel<KIND, BSCALE, PROMOTE, BN, STAGES, EPI, ACT>;
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL));
     LAUNCH(pdl, "grouped_gemm_kernel", kern, grid, gemm_threads<EPI>(), S::TOTAL, st, ta, tb, p);
     return MOE_OK;
@@ -590,12 +605,39 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.hsf = static_cast<uint8_t*>(v.hs);
     p.I = c.I;
     p.H = c.H;
+    p.act = c.act;
+    p.act_alpha = c.act_alpha;
+    p.act_limit = c.act_limit;
     p.status = v.status;
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (c.fmt == MOE_FMT_FP8_ROW) return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16>(h->pdl, ta, tb, p, grid, st);
-    return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4>(h->pdl, ta, tb, p, grid, st);
+    if (c.fmt == MOE_FMT_FP8_ROW) {
+        switch (c.act) {
+        case MOE_ACT_SWIGLU_BOUNDED:
+            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_SWIGLU_BOUNDED>(h->pdl, ta, tb, p, grid, st);
+        case MOE_ACT_SWIGLU_OAI:
+            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_SWIGLU_OAI>(h->pdl, ta, tb, p, grid, st);
+        case MOE_ACT_GEGLU:
+            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_GEGLU>(h->pdl, ta, tb, p, grid, st);
+        case MOE_ACT_REGLU:
+            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_REGLU>(h->pdl, ta, tb, p, grid, st);
+        default:
+            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, grid, st);
+        }
+    }
+    switch (c.act) {
+    case MOE_ACT_SWIGLU_BOUNDED:
+        return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_SWIGLU_BOUNDED>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_SWIGLU_OAI:
+        return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_SWIGLU_OAI>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_GEGLU:
+        return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_GEGLU>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_REGLU:
+        return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_REGLU>(h->pdl, ta, tb, p, grid, st);
+    default:
+        return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, grid, st);
+    }
 }
 
 // ------------------------------------------------------------------ down

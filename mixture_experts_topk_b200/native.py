@@ -36,7 +36,8 @@ class MoeError(RuntimeError):
 class moe_config(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int), ("I", ctypes.c_int), ("E", ctypes.c_int), ("k", ctypes.c_int),
                 ("score", ctypes.c_int), ("fmt", ctypes.c_int), ("has_bias", ctypes.c_int),
-                ("max_T", ctypes.c_int), ("hidden_global_scale", ctypes.c_float)]
+                ("max_T", ctypes.c_int), ("hidden_global_scale", ctypes.c_float),
+                ("act", ctypes.c_int), ("act_alpha", ctypes.c_float), ("act_limit", ctypes.c_float)]
 
 
 class moe_weights(ctypes.Structure):
@@ -115,7 +116,7 @@ def _stream(stream=None):
 # ------------------------------------------------------------ same names as the C ABI
 def moe_init(wl, max_T):
     cfg = moe_config(wl.H, wl.I, wl.E, wl.k, wl.score, wl.fmt, int(wl.has_bias), int(max_T),
-                     float(wl.hidden_global_scale))
+                     float(wl.hidden_global_scale), int(wl.act), float(wl.act_alpha), float(wl.act_limit))
     h = ctypes.c_void_p()
     _check(load().moe_init(ctypes.byref(cfg), ctypes.byref(h)))
     return h

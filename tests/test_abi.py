@@ -52,6 +52,19 @@ def test_init_rejects_bad_shapes_without_a_gpu(lib):
     assert ei.value.status == 2
 
 
+def test_init_rejects_bad_activation_settings_without_a_gpu(lib):
+    from mixture_experts_topk_b200 import native, workloads as W
+    native.load()
+    bad = [W.custom(H=256, I=128, E=8, k=2, act=7),
+           W.custom(H=256, I=128, E=8, k=2, act=W.ACT_SWIGLU_BOUNDED, act_limit=0.0),
+           W.custom(H=256, I=128, E=8, k=2, act=W.ACT_SWIGLU_OAI, act_alpha=0.0, act_limit=7.0),
+           W.custom(H=256, I=128, E=8, k=2, act=W.ACT_SWIGLU_OAI, act_alpha=1.702, act_limit=-1.0)]
+    for wl in bad:
+        with pytest.raises(native.MoeError) as ei:
+            native.moe_init(wl, 16)
+        assert ei.value.status == 1
+
+
 def test_graft_build_compiles_everything():
     import __graft_entry__
     __graft_entry__.build()

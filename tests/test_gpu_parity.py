@@ -286,12 +286,42 @@ def test_down_matches_oracle_on_oracle_hidden(name, down_bn):
     assert tolerance_violations(o, ref["o_w"]) == 0
 
 
+# the gated activation variants, on each format; the limits bind on part of the
+# pre-activations, and T = 300 over 8 experts exercises the row and the sparse
+# gate/up epilogues
+ACT_CASES = {
+    "row-bounded": (W.custom(H=512, I=384, E=8, k=2, act=W.ACT_SWIGLU_BOUNDED, act_limit=0.25), 300),
+    "row-oai": (W.custom(H=512, I=384, E=8, k=2, act=W.ACT_SWIGLU_OAI, act_alpha=1.702, act_limit=0.3), 300),
+    "row-geglu": (W.custom(H=512, I=384, E=8, k=2, act=W.ACT_GEGLU), 300),
+    "row-reglu": (W.custom(H=512, I=384, E=8, k=2, act=W.ACT_REGLU), 300),
+    "block128-oai": (W.custom(H=512, I=384, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128,
+                              act=W.ACT_SWIGLU_OAI, act_alpha=1.702, act_limit=0.3), 300),
+    "block128-geglu": (W.custom(H=512, I=384, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128,
+                                act=W.ACT_GEGLU), 300),
+    "nvfp4-bounded": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4, act=W.ACT_SWIGLU_BOUNDED,
+                               act_limit=0.25), 300),
+    "nvfp4-reglu": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4, act=W.ACT_REGLU), 300),
+}
+
+
+@pytest.mark.parametrize("name", list(ACT_CASES))
+def test_forward_end_to_end_activation_variants(name):
+    wl, T = ACT_CASES[name]
+    d = synth.layer(wl, seed=0)
+    x = synth.tokens(wl, T, seed=0)
+    check_forward(wl, T, d, x)
+
+
 @pytest.mark.parametrize("name", list(CASES))
 def test_forward_end_to_end(name):
     """Y within 2e-2 |ref| + 2e-3 rms(ref), widened only by the bound on what
     hidden codes that rounded the other way can move (see helpers); the
     fraction of elements outside the plain tolerance is reported and small."""
     wl, T, d, x = build_case(name)
+    check_forward(wl, T, d, x)
+
+
+def check_forward(wl, T, d, x):
     layer = native.Layer(wl, d, max_T=T)
     bias = d["bias"].cuda() if d["bias"] is not None else None
     y = layer.forward(x.cuda(), d["wr"].cuda(), bias)
