@@ -342,9 +342,11 @@ def run_ours(args, rank, world, local_rank):
         "kernel_ms": per,
         "e2e": {"value": job_throughput(T, args.steps, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
-        # router 2 + dispatch (hist, scan, rank, quantise; one fused kernel for the
-        # first three when T*k <= 1024; + amax for NVFP4) + gate/up + down + combine
-        "gpu_launches": (2 + (2 if T * wl.k <= 1024 else 4) + (1 if wl.fmt == FMT_NVFP4 else 0) + 3) * args.steps,
+        # router (logits + top-k; one fused kernel for T <= 128 and E <= 32) + dispatch
+        # (hist, scan, rank, quantise; one fused kernel for the first three when
+        # T*k <= 1024; + amax for NVFP4) + gate/up + down + combine
+        "gpu_launches": ((1 if (T <= 128 and wl.E <= 32) else 2) + (2 if T * wl.k <= 1024 else 4)
+                         + (1 if wl.fmt == FMT_NVFP4 else 0) + 3) * args.steps,
         "clocks": clk.summary(),
     }
     del graph

@@ -376,6 +376,12 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
     p.k = h->cfg.k;
     p.score = h->cfg.score;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (T <= 128 && h->cfg.E <= RF_MAX_E) {
+        // logits and top-k in one launch
+        LAUNCH(h->pdl, "router_small_fused_kernel", router_small_fused_kernel, (T + RS_TG - 1) / RS_TG,
+               32 * std::max(h->cfg.E, RS_TG), 0, st, p);
+        return MOE_OK;
+    }
     if (T <= 128) {
         LAUNCH(h->pdl, "router_logits_small_kernel", router_logits_small_kernel,
                dim3((T + RS_TG - 1) / RS_TG, (h->cfg.E + RS_WARPS - 1) / RS_WARPS), RS_WARPS * 32, 0, st, p);

@@ -19,6 +19,8 @@
 //                        16-byte X read from shared memory feeds 64 fma.
 //  router_logits_small_kernel  batches of at most 128 tokens: one warp per
 //                        (expert, 4 tokens) reading global memory directly.
+//  router_small_fused_kernel   the same for at most 32 experts, with the top-k
+//                        of the CTA's 4 tokens in the same launch.
 //  router_topk_kernel    one warp per token: k rounds of a warp argmax over
 //                        the token's logits, then softmax or sigmoid weights.
 #pragma once
@@ -285,57 +287,116 @@ __global__ void __launch_bounds__(RS_WARPS * 32) router_logits_small_kernel(Rout
     }
 }
 
-// top-k per token: k rounds of a warp argmax, larger logit first, equal
-// logits -> lower expert id.  Lane l owns experts l + 32 m.
+// top-k of one token by one warp: k rounds of a warp argmax, larger logit
+// first, equal logits -> lower expert id; lane l owns experts l + 32 m.  `l` is
+// the token's E logits (global or shared memory).
+__device__ __forceinline__ void router_topk_token(const RouterParams& p, const float* l, int t, int lane) {
+    float lv[8];
+#pragma unroll
+    for (int m = 0; m < 8; m++) lv[m] = (32 * m + lane < p.E) ? l[32 * m + lane] : 0.0f;
+    uint32_t taken = 0;
+    float sel_v[8];
+    int sel_e[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        if (j >= p.k) break;
+        float bv = 0.0f;
+        int be = -1;
+#pragma unroll
+        for (int m = 0; m < 8; m++) {
+            const int e = 32 * m + lane;
+            if (e >= p.E || ((taken >> m) & 1u)) continue;
+            if (be < 0 || lv[m] > bv) { bv = lv[m]; be = e; }   // e ascending: ties keep the lower id
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        sel_v[j] = bv;
+        sel_e[j] = be;
+    }
+    if (lane == 0) {
+        float z[8], sum = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            if (j >= p.k) break;
+            z[j] = (p.score == 0) ? expf(sel_v[j] - sel_v[0]) : 1.0f / (1.0f + expf(-sel_v[j]));
+            sum += z[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            if (j >= p.k) break;
+            p.ids[static_cast<size_t>(t) * p.k + j] = sel_e[j];
+            p.w[static_cast<size_t>(t) * p.k + j] = z[j] / sum;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256) router_topk_kernel(RouterParams p) {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
-    for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < p.T; t += gridDim.x * 8) {
-        const float* l = p.logits + static_cast<size_t>(t) * p.E;
-        float lv[8];
+    for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < p.T; t += gridDim.x * 8)
+        router_topk_token(p, p.logits + static_cast<size_t>(t) * p.E, t, lane);
+}
+
+// Small batches with at most 32 experts: logits and top-k in one launch.  One
+// CTA per group of RS_TG tokens, warp e computes expert e's logits exactly as
+// router_logits_small_kernel does, they meet in shared memory, and warp tt
+// then selects token tt's experts with router_topk_token.
+constexpr int RF_MAX_E = 32;
+__global__ void __launch_bounds__(RF_MAX_E * 32) router_small_fused_kernel(RouterParams p) {
+    pdl_wait();
+    pdl_trigger();
+    __shared__ float s_l[RS_TG][RF_MAX_E];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = warp;
+    const int t0 = blockIdx.x * RS_TG;
+    if (e < p.E) {
+        const float* wrow = p.wr + static_cast<size_t>(e) * p.H + 8 * lane;
+        const __nv_bfloat16* xrow[RS_TG];
 #pragma unroll
-        for (int m = 0; m < 8; m++) lv[m] = (32 * m + lane < p.E) ? l[32 * m + lane] : 0.0f;
-        uint32_t taken = 0;
-        float sel_v[8];
-        int sel_e[8];
+        for (int tt = 0; tt < RS_TG; tt++)
+            xrow[tt] = p.x + static_cast<size_t>(t0 + tt < p.T ? t0 + tt : t0) * p.H + 8 * lane;
+        float acc[RS_TG];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            if (j >= p.k) break;
-            float bv = 0.0f;
-            int be = -1;
+        for (int tt = 0; tt < RS_TG; tt++) acc[tt] = 0.0f;
+        const int nI = p.H >> 8;
+#pragma unroll 4
+        for (int i = 0; i < nI; i++) {
+            const float4 wa = __ldg(reinterpret_cast<const float4*>(wrow + 256 * i));
+            const float4 wb = __ldg(reinterpret_cast<const float4*>(wrow + 256 * i + 4));
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-            for (int m = 0; m < 8; m++) {
-                const int e = 32 * m + lane;
-                if (e >= p.E || ((taken >> m) & 1u)) continue;
-                if (be < 0 || lv[m] > bv) { bv = lv[m]; be = e; }   // e ascending: ties keep the lower id
+            for (int tt = 0; tt < RS_TG; tt++) {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xrow[tt] + 256 * i));
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const float xj = (j & 1) ? bf16_hi(xw[j >> 1]) : bf16_lo(xw[j >> 1]);
+                    acc[tt] = __fmaf_rn(xj, wv[j], acc[tt]);
+                }
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            sel_v[j] = bv;
-            sel_e[j] = be;
         }
-        if (lane == 0) {
-            float z[8], sum = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                if (j >= p.k) break;
-                z[j] = (p.score == 0) ? expf(sel_v[j] - sel_v[0]) : 1.0f / (1.0f + expf(-sel_v[j]));
-                sum += z[j];
-            }
+        for (int tt = 0; tt < RS_TG; tt++)
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                if (j >= p.k) break;
-                p.ids[static_cast<size_t>(t) * p.k + j] = sel_e[j];
-                p.w[static_cast<size_t>(t) * p.k + j] = z[j] / sum;
-            }
+            for (int off = 1; off < 32; off <<= 1) acc[tt] = __fadd_rn(acc[tt], __shfl_xor_sync(0xffffffffu, acc[tt], off));
+        if (lane < RS_TG) {
+            float val = acc[0];
+#pragma unroll
+            for (int tt = 1; tt < RS_TG; tt++)
+                if (lane == tt) val = acc[tt];
+            if (p.bias) val = __fadd_rn(val, p.bias[e]);
+            s_l[lane][e] = val;
+            if (t0 + lane < p.T) p.logits[static_cast<size_t>(t0 + lane) * p.E + e] = val;
         }
     }
+    __syncthreads();
+    if (warp < RS_TG && t0 + warp < p.T) router_topk_token(p, s_l[warp], t0 + warp, lane);
 }
 
 }  // namespace moe
