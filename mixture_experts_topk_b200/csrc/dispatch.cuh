@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
 // (count, row tiles): count < 2^20, so count + (tiles << 20) cannot carry.
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
                                                    int32_t* offsets, int32_t* tiles, int32_t* num_tiles,
-                                                   int32_t* tile_ptr, int32_t* pick_out, PickerParams pq) {
+                                                   int32_t* tile_ptr, int32_t* pick_out, PickerParams pq,
+                                                   int32_t* gu_done) {
     pdl_wait();
     pdl_trigger();
     __shared__ int warp_tot[8];
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
     if (e < E) {
         counts[e] = c;
         offsets[e] = off_e;
+        if (gu_done) gu_done[e] = 0;
         if (tile_ptr) tile_ptr[e] = tptr_e;
         int run = off_e;
         for (int ch = 0; ch < nchunks; ch++) {
@@ -212,7 +214,8 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
 // (count + (row tiles << 20), as in scan_kernel) and then over warps.
 __global__ void __launch_bounds__(DISPATCH_CHUNK) dispatch_small_kernel(
     const int32_t* ids, int A, int E, int32_t* counts, int32_t* offsets, int32_t* tiles, int32_t* num_tiles,
-    int32_t* tile_ptr, int32_t* pick_out, PickerParams pq, int32_t* perm, int32_t* inv, int32_t* status) {
+    int32_t* tile_ptr, int32_t* pick_out, PickerParams pq, int32_t* perm, int32_t* inv, int32_t* status,
+    int32_t* gu_done) {
     pdl_wait();
     pdl_trigger();
     __shared__ int wc[32][256];
@@ -266,6 +269,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK) dispatch_small_kernel(
         if (tid < E) {
             counts[tid] = c;
             offsets[tid] = off_e;
+            gu_done[tid] = 0;
             tile_ptr[tid] = tptr_e;
             for (int i = 0; i < nt_e; i++) {
                 tiles[2 * (tptr_e + i)] = tid;

@@ -59,6 +59,8 @@ struct GemmParams {
     uint8_t* hsf;
     int I;
     int act;                    // gate/up: gated activation (the kernel is instantiated for it)
+    int32_t* gu_done;           // FP8_ROW gate/up: per-expert count of finished (tile, epilogue warp)
+                                //   parts, for a down GEMM that starts before this kernel ends
     float act_alpha, act_limit;
     float* o;                   // down: [A][H] fp32
     int H;
@@ -346,6 +348,18 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
             const int row = row0 + r;
             const bool valid = row < s_off[e + 1];
 
+            // FP8_ROW gate/up: this warp's part of the tile is stored; publish it
+            // (per-lane release, then one count per warp) for the chained down GEMM
+            auto publish = [&]() {
+                if constexpr (KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW) {
+                    if (p.gu_done != nullptr) {
+                        fence_proxy_async_global();
+                        __threadfence();
+                        __syncwarp();
+                        if (lane == 0) atomicAdd(p.gu_done + e, 1);
+                    }
+                }
+            };
             if (KIND == KIND_GATE_UP) {
                 float hv[64];
                 if (!PROMOTE) {
@@ -369,6 +383,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty[acc]);
                         u++;
+                        publish();
                         continue;
                     }
                     const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
@@ -424,6 +439,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                             }
                         }
                         u++;
+                        publish();
                         continue;
                     }
 #pragma unroll
@@ -509,6 +525,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 #pragma unroll
                         for (int v4 = 0; v4 < 2 * NH; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
                     }
+                    publish();
                     continue;
                 }
                 // BLOCK128: requantise the 128-column hidden block of this row; the

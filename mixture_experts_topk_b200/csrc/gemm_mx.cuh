@@ -11,7 +11,7 @@
 // Tile 128 padded rows x 256 columns, K stage 128 (one 512-byte scale chunk of
 // A per stage: 4 scales of 32 per row), 4 stages.  For small batches the K
 // range of each tile may be split S ways (S read from the dispatch's pick,
-// work unit = (split, tile)); split s writes its fp32 partial rows to copy s
+// work item t = (tile t / S, split t % S)); split s writes its fp32 partial rows to copy s
 // of the output rows, o + s * A * H.  MMA j of a stage (K = 32)
 // uses byte j of the chunk (scale-factor id j).  TMEM: one 256-column
 // accumulator, released as soon as the epilogue has it in registers, then the
@@ -74,6 +74,8 @@ struct MxDownParams {
     int A;                     // assignments T * k
     const int32_t* split;      // S, the K split chosen by the dispatch's scan
     int s_max;                 // S is clamped to [1, s_max] (s_max * A rows fit in o)
+    const int32_t* gu_done;    // chained after the gate/up GEMM: per-expert finished parts, else null
+    int gu_per_mtile;          //   parts per m-tile of an expert (gate/up n-blocks x epilogue warps)
     const int32_t* perm;
     const float* route_w;
     int32_t* status;
@@ -116,7 +118,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    pdl_wait();
+    // Chained after the gate/up GEMM, this kernel does not wait for that whole
+    // kernel: the schedule it reads was complete before the gate/up GEMM let it
+    // launch, and each expert's hidden is waited for below.  Otherwise wait for
+    // the preceding kernel.
+    if (p.gu_done == nullptr) pdl_wait();
     pdl_trigger();
     int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + MX_TMAP_OFF);
     const int32_t* s_off = s_tptr + TMAP_STRIDE;
@@ -133,10 +139,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
+            int ready_e = -1;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const int sp = t / units;
+                const int sp = t % S;   // unit-major: all splits of a unit together, experts in order
                 int e, mi, nb;
-                decode_tile(t - sp * units, s_tptr, p.E, p.n_blocks, e, mi, nb);
+                decode_tile(t / S, s_tptr, p.E, p.n_blocks, e, mi, nb);
+                if (p.gu_done != nullptr && e != ready_e) {
+                    // all gate/up parts of expert e are stored before its hidden is read
+                    const int target = (s_tptr[e + 1] - s_tptr[e]) * p.gu_per_mtile;
+                    const long long t0 = clock64();
+                    while (ld_acquire(p.gu_done + e) < target) {
+                        if (clock64() - t0 > limit) { ok = false; break; }
+                    }
+                    if (!ok) {
+                        report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
+                        break;
+                    }
+                    fence_proxy_async_global();
+                    ready_e = e;
+                }
                 const int brow = e * p.b_rows + nb * MX_BN;
                 const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.num_kb * 512;
                 const int kb1 = (sp + 1) * p.num_kb / S;
@@ -166,7 +187,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0, u = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const int sp = t / units;
+                const int sp = t % S;
                 const int kb0 = sp * p.num_kb / S, kb1 = (sp + 1) * p.num_kb / S;
                 if (!mbar_wait(tempty, (u & 1) ^ 1, limit)) { ok = false; break; }
                 tc_fence_after();
@@ -201,9 +222,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint32_t u = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const int sp = t / units;
+            const int sp = t % S;
             int e, mi, nb;
-            decode_tile(t - sp * units, s_tptr, p.E, p.n_blocks, e, mi, nb);
+            decode_tile(t / S, s_tptr, p.E, p.n_blocks, e, mi, nb);
             const int local = mi * 128 + r - s_tptr[e] * 128;
             const bool valid = local < s_off[e + 1] - s_off[e];
             // the row's routing weight is loaded while the tile's MMAs run

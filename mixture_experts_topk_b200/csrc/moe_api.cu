@@ -78,7 +78,7 @@ static cudaError_t launch_k(bool pdl, void (*kern)(KP...), dim3 grid, dim3 block
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-    size_t status, ids, w, logits, counts, offsets, num_tiles, tile_ptr, pick, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
+    size_t status, ids, w, logits, counts, offsets, num_tiles, tile_ptr, pick, gu_done, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
 };
 struct WLayout {
     size_t gu_q, gu_s, d_q, d_s, gu_g, d_g, total;
@@ -150,6 +150,7 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.num_tiles = take(4);
     L.tile_ptr = take((c.E + 1) * 4);
     L.pick = take(8);
+    L.gu_done = take(c.E * 4);
     L.chunk = take(nchunks * c.E * 4);
     L.tiles = take(tiles_cap * 8);
     L.perm = take(A * 4);
@@ -288,6 +289,11 @@ extern "C" moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_
 
 static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
 
+// per-expert count of finished gate/up parts (reset by the dispatch's scan)
+static int32_t* gu_done_of(const moe_handle* h, void* ws) {
+    return reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + h->ws.gu_done);
+}
+
 static moe_status check_T(const moe_handle* h, int T, const char* who) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "%s: null handle", who);
     if (T < 0 || T > h->cfg.max_T) return fail(MOE_ERR_INVALID_ARG, "%s: T=%d outside [0, max_T=%d]", who, T, h->cfg.max_T);
@@ -420,13 +426,14 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
     if (A > 0 && nchunks == 1) {
         // one chunk: histogram, scan and ranks in one CTA
         LAUNCH(h->pdl, "dispatch_small_kernel", dispatch_small_kernel, 1, DISPATCH_CHUNK, 0, st, ids, A, c.E,
-               v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr, v.pick, h->picker, v.perm, v.inv, v.status);
+               v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr, v.pick, h->picker, v.perm, v.inv, v.status,
+               gu_done_of(h, ws));
     } else {
         if (A > 0) {
             LAUNCH(h->pdl, "hist_kernel", hist_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.status);
         }
         LAUNCH(h->pdl, "scan_kernel", scan_kernel, 1, 256, 0, st, chunk, nchunks, c.E, v.counts, v.offsets, v.tiles,
-               v.num_tiles, v.tile_ptr, v.pick, h->picker);
+               v.num_tiles, v.tile_ptr, v.pick, h->picker, gu_done_of(h, ws));
         if (A == 0) return MOE_OK;
         LAUNCH(h->pdl, "rank_kernel", rank_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.perm, v.inv);
     }
@@ -587,7 +594,6 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
-    const size_t A = static_cast<size_t>(c.max_T) * c.k;
     CUtensorMap ta, tb;
     moe_status r = make_tmap(&ta, v.xq, c.H, padded_rows(c), c.H, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
@@ -614,6 +620,7 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.act = c.act;
     p.act_alpha = c.act_alpha;
     p.act_limit = c.act_limit;
+    p.gu_done = c.fmt == MOE_FMT_FP8_ROW ? gu_done_of(h, ws) : nullptr;
     p.status = v.status;
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
@@ -648,8 +655,11 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
 
 // ------------------------------------------------------------------ down
 // FP8_ROW: MX-scaled hidden (tensor cores apply its scales), one tile width.
+// chained: launched right after this call's gate/up GEMM (moe_forward_routed);
+// the kernel then waits per expert for the gate/up parts instead of for the
+// whole gate/up kernel, so down tiles of finished experts overlap its tail.
 static moe_status mx_down(const moe_handle* h, const void* packed, const float* w, int T, void* ws,
-                          moe_stream_t stream) {
+                          moe_stream_t stream, bool chained) {
     const moe_config& c = h->cfg;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
@@ -676,6 +686,8 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     p.A = T * c.k;
     p.split = v.pick + 1;
     p.s_max = split_limit(h->picker, p.A);
+    p.gu_done = chained ? gu_done_of(h, ws) : nullptr;
+    p.gu_per_mtile = (2 * c.I / 256) * 16;   // gate/up n-blocks x its 16 epilogue warps
     p.perm = v.perm;
     p.route_w = w;
     p.status = v.status;
@@ -696,7 +708,7 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     if (!packed || !ws || !w) return fail(MOE_ERR_INVALID_ARG, "moe_down: null argument");
     if (!aligned256(packed) || !aligned256(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_down: pointers must be 256-byte aligned");
     if (h->cfg.fmt == MOE_FMT_NVFP4) return fp4_gemm(h, packed, w, T, ws, stream, false);
-    if (h->cfg.fmt == MOE_FMT_FP8_ROW) return mx_down(h, packed, w, T, ws, stream);
+    if (h->cfg.fmt == MOE_FMT_FP8_ROW) return mx_down(h, packed, w, T, ws, stream, false);
     const moe_config& c = h->cfg;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
@@ -816,7 +828,12 @@ extern "C" moe_status moe_forward_routed(const moe_handle* h, const void* x, int
     if (r != MOE_OK) return r;
     r = moe_gate_up(h, packed, T, ws, stream);
     if (r != MOE_OK) return r;
-    r = moe_down(h, packed, w, T, ws, stream);
+    if (h->cfg.fmt == MOE_FMT_FP8_ROW && T > 0 && h->pdl) {
+        if (!w) return fail(MOE_ERR_INVALID_ARG, "moe_forward_routed: null argument");
+        r = mx_down(h, packed, w, T, ws, stream, true);
+    } else {
+        r = moe_down(h, packed, w, T, ws, stream);
+    }
     if (r != MOE_OK) return r;
     return moe_combine(h, T, y, ws, stream);
 }
@@ -923,7 +940,8 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, c
         hist_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, status);
         LAUNCH_CHECK("hist_kernel");
     }
-    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles, nullptr, nullptr, h->picker);
+    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles, nullptr, nullptr, h->picker,
+                                   nullptr);
     LAUNCH_CHECK("scan_kernel");
     if (a == 0) return MOE_OK;
     rank_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, perm, inv);
