@@ -448,11 +448,13 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* o, const int3
     pdl_trigger();
     const int S = split ? min(max(*split, 1), s_max) : 1;
     const size_t copy = static_cast<size_t>(T) * k * H;
+    // CTA (x, y): tokens x, x + gridDim.x, ..., columns [1024 y, 1024 y + 1024)
+    const int c_end = min(H, 1024 * (static_cast<int>(blockIdx.y) + 1));
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         int slot[8];
 #pragma unroll
         for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
-        for (int c0 = 8 * threadIdx.x; c0 < H; c0 += 8 * blockDim.x) {
+        for (int c0 = 1024 * blockIdx.y + 8 * threadIdx.x; c0 < c_end; c0 += 8 * blockDim.x) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (S == 1) {
                 // all k rows' loads in flight at once

@@ -713,7 +713,6 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
-    const size_t A = static_cast<size_t>(c.max_T) * c.k;
     const int BN = h->down_bn ? h->down_bn : 256;
     CUtensorMap ta, tb, tb128, tb64;
     moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
@@ -813,7 +812,9 @@ extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws,
     if (T == 0) return MOE_OK;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
-    const int grid = std::min(T, 16 * h->num_sms);
+    // one CTA per (token group, 1024-column slice): small batches still spread
+    const int ncb = (h->cfg.H + 1023) / 1024;
+    const dim3 grid(std::max(1, std::min(T, 16 * h->num_sms / ncb)), ncb);
     LAUNCH(h->pdl, "combine_kernel", combine_kernel, grid, 128, 0, reinterpret_cast<cudaStream_t>(stream),
            static_cast<const float*>(v.o), static_cast<const int32_t*>(v.inv), T, h->cfg.H, h->cfg.k,
            static_cast<const int32_t*>(h->cfg.fmt == MOE_FMT_FP8_ROW ? v.pick + 1 : nullptr),
