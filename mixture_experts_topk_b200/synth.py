@@ -22,7 +22,7 @@ import math
 
 import torch
 
-from .workloads import FMT_FP8_BLOCK128, FMT_FP8_ROW, FMT_NVFP4
+from .workloads import ACT_RELU2, FMT_FP8_BLOCK128, FMT_FP8_ROW, FMT_NVFP4
 
 E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 
@@ -120,9 +120,12 @@ def experts(wl, seed=0, device="cpu", experts_subset=None):
       p_g      [E] fp32 NVFP4 global scale (absent otherwise)
     gate/up: N = I, K = H; down: N = H, K = I.  experts_subset draws only those
     experts (the others are left zero), for sampled checks of huge layers.
+    ReLU^2 experts have no gate: gate_q / gate_s / gate_g are None.
     """
     E = wl.E
     shapes = {"gate": (wl.I, wl.H), "up": (wl.I, wl.H), "down": (wl.H, wl.I)}
+    if wl.act == ACT_RELU2:
+        del shapes["gate"]
     out = {}
     for p, (n, k) in shapes.items():
         kq = k // 2 if wl.fmt == FMT_NVFP4 else k
@@ -144,6 +147,8 @@ def experts(wl, seed=0, device="cpu", experts_subset=None):
             out[p + "_s"][e].copy_(s)
             if gg is not None:
                 out[p + "_g"][e] = gg[0]
+    if wl.act == ACT_RELU2:
+        out.update(gate_q=None, gate_s=None, gate_g=None)
     return out
 
 

@@ -25,6 +25,7 @@ ACT_SWIGLU_BOUNDED = 1  # silu(min(g, L)) clamp(u, -L, L)
 ACT_SWIGLU_OAI = 2      # g' sigmoid(alpha g') (u' + 1), g' = min(g, L), u' = clamp(u, -L, L)
 ACT_GEGLU = 3           # gelu(g) u (erf form)
 ACT_REGLU = 4           # relu(g) u
+ACT_RELU2 = 5           # relu(u)^2, experts without a gate projection
 
 
 @dataclass(frozen=True)

@@ -184,7 +184,7 @@ def pick_down_tile(counts, H, I, num_sms, alpha, beta, bw, gamma):
     return c, costs
 
 
-ACT_SWIGLU, ACT_SWIGLU_BOUNDED, ACT_SWIGLU_OAI, ACT_GEGLU, ACT_REGLU = range(5)
+ACT_SWIGLU, ACT_SWIGLU_BOUNDED, ACT_SWIGLU_OAI, ACT_GEGLU, ACT_REGLU, ACT_RELU2 = range(6)
 
 
 def glu(act, g, u, alpha=0.0, limit=0.0):
@@ -248,6 +248,9 @@ class Layer:
         st.hidden_global = float(wl.hidden_global_scale)
         st.act, st.act_alpha, st.act_limit = wl.act, float(wl.act_alpha), float(wl.act_limit)
         for p in ("gate", "up", "down"):
+            if weights.get(p + "_q") is None:      # ReLU^2 experts have no gate
+                setattr(st, p, _Proj(None, None, None))
+                continue
             q = _c(weights[p + "_q"], np.uint8)
             s = np.ascontiguousarray(weights[p + "_s"])
             g = None if wl.fmt != FMT_NVFP4 else _c(weights[p + "_g"], np.float32)

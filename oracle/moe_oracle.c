@@ -438,6 +438,8 @@ double orc_glu(int act, double alpha, double limit, double g, double u)
         return 0.5 * g * (1.0 + erf(g / sqrt(2.0))) * u;
     case ORC_ACT_REGLU:
         return (g > 0.0 ? g : 0.0) * u;
+    case ORC_ACT_RELU2:
+        return u > 0.0 ? u * u : 0.0;
     default:
         return g / (1.0 + exp(-g)) * u;
     }
@@ -455,12 +457,13 @@ void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes
     {
         double* wg = (double*)malloc(sizeof(double) * (size_t)H);
         double* wu = (double*)malloc(sizeof(double) * (size_t)H);
+        const int gated = L->act != ORC_ACT_RELU2;   /* ReLU^2 experts have no gate */
 #pragma omp for schedule(static)
         for (int n = 0; n < I; n++) {
-            orc_weight_row(L, &L->gate, I, H, e, n, wg);
+            if (gated) orc_weight_row(L, &L->gate, I, H, e, n, wg);
             orc_weight_row(L, &L->up, I, H, e, n, wu);
             for (int r = 0; r < rows; r++) {
-                double g = dot64(a + (int64_t)r * H, wg, H);
+                double g = gated ? dot64(a + (int64_t)r * H, wg, H) : 0.0;
                 double u = dot64(a + (int64_t)r * H, wu, H);
                 hh[(int64_t)r * I + n] = orc_glu(L->act, L->act_alpha, L->act_limit, g, u);
             }

@@ -125,8 +125,11 @@ typedef struct {
  *   SWIGLU_BOUNDED  silu(min(g, L)) clamp(u, -L, L)
  *   SWIGLU_OAI      g' / (1 + exp(-alpha g')) (u' + 1),  g' = min(g, L), u' = clamp(u, -L, L)
  *   GEGLU           g Phi(g) u,  Phi(g) = (1 + erf(g / sqrt 2)) / 2
- *   REGLU           max(g, 0) u */
-enum { ORC_ACT_SWIGLU = 0, ORC_ACT_SWIGLU_BOUNDED = 1, ORC_ACT_SWIGLU_OAI = 2, ORC_ACT_GEGLU = 3, ORC_ACT_REGLU = 4 };
+ *   REGLU           max(g, 0) u
+ *   RELU2           max(u, 0)^2; the expert has no gate projection (two weights,
+ *                   LightMoE README "MoE inference": ReLU^2 experts load up and down) */
+enum { ORC_ACT_SWIGLU = 0, ORC_ACT_SWIGLU_BOUNDED = 1, ORC_ACT_SWIGLU_OAI = 2, ORC_ACT_GEGLU = 3, ORC_ACT_REGLU = 4,
+       ORC_ACT_RELU2 = 5 };
 double orc_glu(int act, double alpha, double limit, double g, double u);
 
 /* dequantised weight row (fp64, exact) */

@@ -105,11 +105,13 @@ def _torch_glu(act, g, u, alpha, limit):
         return gc * torch.sigmoid(alpha * gc) * (torch.clamp(u, -limit, limit) + 1.0)
     if act == W.ACT_GEGLU:
         return F.gelu(g, approximate="none") * u
+    if act == W.ACT_RELU2:
+        return F.relu(u) ** 2
     return F.relu(g) * u
 
 
 ACTS = [(W.ACT_SWIGLU, 0.0, 0.0), (W.ACT_SWIGLU_BOUNDED, 0.0, 0.25), (W.ACT_SWIGLU_OAI, 1.702, 0.3),
-        (W.ACT_GEGLU, 0.0, 0.0), (W.ACT_REGLU, 0.0, 0.0)]
+        (W.ACT_GEGLU, 0.0, 0.0), (W.ACT_REGLU, 0.0, 0.0), (W.ACT_RELU2, 0.0, 0.0)]
 
 
 @pytest.mark.parametrize("act,alpha,limit", ACTS)
@@ -127,8 +129,10 @@ def test_single_expert_is_the_dense_gated_mlp_of_each_activation(fmt, act, alpha
     codes, scales = oracle.quant_rows(fmt, xf, g_x)
     h, hq, hs, o = L.expert_rows(0, codes, scales, g_x)
     a = torch.from_numpy(deq_act(wl, codes, scales, g_x))
-    g = a @ torch.from_numpy(deq_weight(wl, d, "gate", 0)).T
     u = a @ torch.from_numpy(deq_weight(wl, d, "up", 0)).T
+    g = u if act == W.ACT_RELU2 else a @ torch.from_numpy(deq_weight(wl, d, "gate", 0)).T
+    if act == W.ACT_RELU2:
+        assert d["gate_q"] is None
     if limit > 0.0:
         assert (g > limit).any() and (u.abs() > limit).any()
     h_ref = _torch_glu(act, g, u, alpha, limit)

@@ -303,7 +303,10 @@ def test_gated_activations_closed_forms():
         pytest.approx(2.0 / (1.0 + np.exp(-3.404)) * 4.0, rel=1e-15)
     assert oracle.glu(oracle.ACT_SWIGLU_OAI, 9.0, -9.0, alpha=1.702, limit=7.0) == \
         pytest.approx(7.0 / (1.0 + np.exp(-1.702 * 7.0)) * -6.0, rel=1e-15)
-    # every variant is 0 at g = 0
+    # ReLU^2 ignores the gate: max(u, 0)^2
+    assert oracle.glu(oracle.ACT_RELU2, 123.0, 3.0) == 9.0
+    assert oracle.glu(oracle.ACT_RELU2, 1.0, -3.0) == 0.0
+    # every gated variant is 0 at g = 0
     for act in range(5):
         assert oracle.glu(act, 0.0, 3.0, alpha=1.702, limit=7.0) == 0.0
 
@@ -316,6 +319,7 @@ def test_gated_activations_match_torch_library_routines():
     np.testing.assert_allclose(oracle.glu(oracle.ACT_SWIGLU, g, u), (F.silu(gt) * ut).numpy(), rtol=1e-14, atol=1e-300)
     np.testing.assert_allclose(oracle.glu(oracle.ACT_GEGLU, g, u), (F.gelu(gt) * ut).numpy(), rtol=1e-13, atol=1e-300)
     np.testing.assert_array_equal(oracle.glu(oracle.ACT_REGLU, g, u), (F.relu(gt) * ut).numpy())
+    np.testing.assert_array_equal(oracle.glu(oracle.ACT_RELU2, g, u), (F.relu(ut) ** 2).numpy())
     ref = F.silu(torch.clamp(gt, max=2.0)) * torch.clamp(ut, -2.0, 2.0)
     np.testing.assert_allclose(oracle.glu(oracle.ACT_SWIGLU_BOUNDED, g, u, limit=2.0), ref.numpy(), rtol=1e-14, atol=1e-300)
     gc = torch.clamp(gt, max=2.0)
