@@ -108,18 +108,24 @@ def gemm_traffic(workload, T):
     return d["gate_up"]["dram_read_bytes"] + d["gate_up"]["dram_write_bytes"]
 
 
+def n_proj(wl):
+    """Weight matrices per expert: gate, up, down; ReLU^2 experts have no gate."""
+    return 2 if wl.act == ACTS["relu2"][0] else 3
+
+
 def algorithmic_work(wl, T, counts):
     """FLOPs and bytes of one layer call (intermediates excluded)."""
     A = T * wl.k
-    flops_tensor = 2.0 * A * 3 * wl.H * wl.I
+    npj = n_proj(wl)
+    flops_tensor = 2.0 * A * npj * wl.H * wl.I
     flops_router = 2.0 * T * wl.E * wl.H
     touched = int((counts > 0).sum())
     if wl.fmt == FMT_NVFP4:
-        per_expert = 3 * wl.H * wl.I * (0.5 + 1.0 / 16)
+        per_expert = npj * wl.H * wl.I * (0.5 + 1.0 / 16)
     elif wl.fmt == 0:
-        per_expert = 3 * wl.H * wl.I + 4 * (2 * wl.I + wl.H)
+        per_expert = npj * wl.H * wl.I + 4 * ((npj - 1) * wl.I + wl.H)
     else:
-        per_expert = 3 * wl.H * wl.I + 4 * 3 * (wl.H // 128) * (wl.I // 128)
+        per_expert = npj * wl.H * wl.I + 4 * npj * (wl.H // 128) * (wl.I // 128)
     byts = touched * per_expert + wl.E * wl.H * 4 + 2 * T * wl.H * 2
     return flops_tensor, flops_router, byts, touched
 
@@ -141,7 +147,7 @@ def job_throughput(tokens_per_rank, steps, world, ms_max):
 # gated activations: (act id, alpha, limit); the clamp of 10 is the bounded-SwiGLU
 # setting the LightMoE README gives, alpha 1.702 / limit 7 the common SwiGLU-OAI one
 ACTS = {"swiglu": (0, 0.0, 0.0), "bounded": (1, 0.0, 10.0), "oai": (2, 1.702, 7.0), "geglu": (3, 0.0, 0.0),
-        "reglu": (4, 0.0, 0.0)}
+        "reglu": (4, 0.0, 0.0), "relu2": (5, 0.0, 0.0)}
 
 
 def workload_of(args):
@@ -300,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
     pk, pk_kind = peaks()
     # dense fp8 = 2 x bf16 and fp4 = 4 x bf16 (nominal ratios) of the measured bf16 figure
     fp8_peak = (4.0 if wl.fmt == FMT_NVFP4 else 2.0) * pk["bf16_tflops_sustained"]
-    gu_flops = 2.0 * T * wl.k * 2 * wl.H * wl.I
+    gu_flops = 2.0 * T * wl.k * (n_proj(wl) - 1) * wl.H * wl.I
     gu_ms = per["gate_up"]
     achieved = gu_flops / (gu_ms * 1e-3) / 1e12
     step_ms = ms_max / args.steps
@@ -336,7 +342,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"kernel": "grouped_gemm gate/up (SwiGLU + requant epilogue)", "bound": "tensor",
                      "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp8_peak, "traffic": gemm_traffic(args.workload, T),
-                     "algorithmic_bytes": int(T * wl.k * wl.H + 2 * wl.I * wl.H * touched + T * wl.k * wl.I),
+                     "algorithmic_bytes": int(T * wl.k * wl.H + (n_proj(wl) - 1) * wl.I * wl.H * touched + T * wl.k * wl.I),
                      "peak_source": f"{pk_kind} bf16_tflops_sustained x {4 if wl.fmt == FMT_NVFP4 else 2} "
                                     "(nominal fp8:bf16 = 2, fp4:bf16 = 4)"},
         "kernel_ms": per,

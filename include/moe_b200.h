@@ -83,14 +83,19 @@ typedef struct {
  *   SWIGLU_OAI      g' / (1 + e^(-alpha g')) * (u' + 1),  g' = min(g, L), u' = clamp(u, -L, L)
  *   GEGLU           0.5 g (1 + erf(g / sqrt 2)) * u
  *   REGLU           max(g, 0) * u
+ *   RELU2           max(u, 0)^2 with no gate projection: two weights per expert
+ *                   (README "MoE inference": ReLU^2 experts load up and down);
+ *                   moe_weights.gate_* may be NULL; needs I % 256 == 0
  * moe_init returns MOE_ERR_INVALID_ARG for an unknown act, L <= 0 where a
- * limit is used, or alpha <= 0 for SWIGLU_OAI. */
+ * limit is used, or alpha <= 0 for SWIGLU_OAI; MOE_ERR_UNSUPPORTED_SHAPE for
+ * RELU2 with I not a multiple of 256. */
 enum {
     MOE_ACT_SWIGLU = 0,
     MOE_ACT_SWIGLU_BOUNDED = 1,
     MOE_ACT_SWIGLU_OAI = 2,
     MOE_ACT_GEGLU = 3,
-    MOE_ACT_REGLU = 4
+    MOE_ACT_REGLU = 4,
+    MOE_ACT_RELU2 = 5
 };
 
 typedef struct moe_handle moe_handle;

@@ -312,6 +312,12 @@ __device__ __forceinline__ float glu(float g, float u, float alpha, float limit)
     }
 }
 
+// ReLU^2 experts (no gate): h = max(u, 0)^2
+__device__ __forceinline__ float relu_sq(float u) {
+    const float r = fmaxf(u, 0.0f);
+    return r * r;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 

@@ -362,7 +362,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
             };
             if (KIND == KIND_GATE_UP) {
                 float hv[64];
-                if (!PROMOTE) {
+                float hv2[64];                  // ReLU^2: the up-half columns' outputs (BLOCK128)
+                if constexpr (!PROMOTE) {
                     // scales are loaded while the tile's MMAs run: the row's X scale,
                     // and lane c holds the weight scale of column c of each 32-column
                     // half (read back with a shuffle)
@@ -405,7 +406,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                                 __syncwarp();
                                 if (lane == 0) mbar_arrive(&tempty[acc]);
                             }
-                            const int hcol = nb * 128 + c0;   // first hidden column of this 32-block
+                            // first hidden column of this 32-block (ReLU^2: the gate-half
+                            // columns are up rows 256 nb + c0, the up half 256 nb + 128 + c0)
+                            const int hcol = ACT == 5 ? nb * 256 + c0 : nb * 128 + c0;
                             uint32_t m = vmask;
                             for (int r0 = 0; r0 < nv; r0 += SR) {
                                 if (valid && cidx >= r0 && cidx < r0 + SR) {
@@ -425,15 +428,21 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                                     const float sa_i = sb[SR * 64 + i];
                                     const float gg = sb[i * 64 + lane] * (sa_i * bsg[half]);
                                     const float uu = sb[i * 64 + 32 + lane] * (sa_i * bsu[half]);
-                                    const float hvv = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
-                                    float amax = fabsf(hvv);
-#pragma unroll
-                                    for (int off = 16; off > 0; off >>= 1)
-                                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-                                    const int ex = mx_exponent(amax);
                                     const long long prow = static_cast<long long>(mi) * 128 + 32 * q + rl;
-                                    p.hq[prow * p.I + hcol + lane] = f_to_e4m3(__fmul_rn(hvv, mx_inv_scale(ex)));
-                                    if (lane == 0) p.hsf[sf_offset(prow, hcol / 32, p.I / 32)] = static_cast<uint8_t>(ex + 127);
+                                    // gated: one block act(gg, uu); ReLU^2: relu(gg)^2 and relu(uu)^2
+#pragma unroll
+                                    for (int ob = 0; ob < (ACT == 5 ? 2 : 1); ob++) {
+                                        const float hvv = ACT == 5 ? relu_sq(ob ? uu : gg)
+                                                                   : glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+                                        const int col = hcol + 128 * ob;
+                                        float amax = fabsf(hvv);
+#pragma unroll
+                                        for (int off = 16; off > 0; off >>= 1)
+                                            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                                        const int ex = mx_exponent(amax);
+                                        p.hq[prow * p.I + col + lane] = f_to_e4m3(__fmul_rn(hvv, mx_inv_scale(ex)));
+                                        if (lane == 0) p.hsf[sf_offset(prow, col / 32, p.I / 32)] = static_cast<uint8_t>(ex + 127);
+                                    }
                                 }
                                 __syncwarp();
                             }
@@ -451,7 +460,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         for (int c = 0; c < 32; c++) {
                             const float gg = gv[c] * (sa * __shfl_sync(0xffffffffu, bsg[half], c));
                             const float uu = uv[c] * (sa * __shfl_sync(0xffffffffu, bsu[half], c));
-                            hv[32 * half + c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+                            if constexpr (ACT == 5) {
+                                hv[32 * half + c] = relu_sq(gg);
+                                hv[32 * (NH + half) + c] = relu_sq(uu);
+                            } else {
+                                hv[32 * half + c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+                            }
                         }
                     }
                     tc_fence_before();
@@ -495,8 +509,16 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         u++;
                     }
                     if (!ok) break;
+                    if constexpr (ACT == 5) {
 #pragma unroll
-                    for (int c = 0; c < 64; c++) hv[c] = glu<ACT>(ag[c], au[c], p.act_alpha, p.act_limit);
+                        for (int c = 0; c < 64; c++) {
+                            hv[c] = relu_sq(ag[c]);
+                            hv2[c] = relu_sq(au[c]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 64; c++) hv[c] = glu<ACT>(ag[c], au[c], p.act_alpha, p.act_limit);
+                    }
                 }
                 if (BSCALE == BSCALE_ROW) {
                     // MX requantisation: power-of-two scale per 32 hidden columns (all
@@ -504,65 +526,81 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     // scales to the chunked layout the down GEMM's tensor cores read
                     if (valid) {
                         const long long prow = static_cast<long long>(mi) * 128 + r;
-                        const int col0 = nb * 128 + GC * g;
-                        uint32_t w[8 * NH];
+                        // 32-column blocks of this thread: gated NH blocks at hidden
+                        // 128 nb + GC g + 32 b; ReLU^2 2 NH blocks, the gate-half
+                        // columns at 256 nb + GC g + 32 b, the up half 128 further
+                        constexpr int NB = ACT == 5 ? 2 * NH : NH;
+                        static_assert(BSCALE != BSCALE_ROW || 32 * NB <= 64, "hidden values held per thread");
 #pragma unroll
-                        for (int b = 0; b < NH; b++) {
+                        for (int b = 0; b < NB; b++) {
+                            const int col = ACT == 5 ? nb * 256 + (b < NH ? GC * g + 32 * b : 128 + GC * g + 32 * (b - NH))
+                                                     : nb * 128 + GC * g + 32 * b;
                             float amax = 0.0f;
 #pragma unroll
                             for (int c = 0; c < 32; c++) amax = fmaxf(amax, fabsf(hv[32 * b + c]));
                             const int ex = mx_exponent(amax);
                             const float inv = mx_inv_scale(ex);
+                            uint32_t w[8];
 #pragma unroll
                             for (int c = 0; c < 32; c += 4) {
                                 const uint16_t lo = f2_to_e4m3x2(__fmul_rn(hv[32 * b + c], inv), __fmul_rn(hv[32 * b + c + 1], inv));
                                 const uint16_t hi = f2_to_e4m3x2(__fmul_rn(hv[32 * b + c + 2], inv), __fmul_rn(hv[32 * b + c + 3], inv));
-                                w[8 * b + c / 4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+                                w[c / 4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
                             }
-                            p.hsf[sf_offset(prow, col0 / 32 + b, p.I / 32)] = static_cast<uint8_t>(ex + 127);
+                            p.hsf[sf_offset(prow, col / 32, p.I / 32)] = static_cast<uint8_t>(ex + 127);
+                            uint4* dst = reinterpret_cast<uint4*>(p.hq + prow * p.I + col);
+                            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(p.hq + prow * p.I + col0);
-#pragma unroll
-                        for (int v4 = 0; v4 < 2 * NH; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
                     }
                     publish();
                     continue;
                 }
                 // BLOCK128: requantise the 128-column hidden block of this row; the
-                // two column groups exchange their partial amax through shared memory
-                float amax = 0.0f;
+                // two column groups exchange their partial amax through shared memory.
+                // ReLU^2 tiles hold two hidden blocks (the gate-half columns are up
+                // rows 256 nb .. +128, the up half the next 128); each is exchanged
+                // under its own tag.
 #pragma unroll
-                for (int c = 0; c < 64; c++) amax = fmaxf(amax, fabsf(hv[c]));
-                const int par = iter & 1;
-                volatile float* xv = xval;
-                volatile int* xf = xflag;
-                xv[(par * 2 + g) * 128 + r] = amax;
-                __threadfence_block();
-                xf[(par * 2 + g) * 128 + r] = static_cast<int>(iter) + 1;
-                long long t0 = clock64();
-                while (xf[(par * 2 + (1 - g)) * 128 + r] < static_cast<int>(iter) + 1) {
-                    if (clock64() - t0 > limit) { ok = false; break; }
+                for (int blk = 0; blk < (ACT == 5 ? 2 : 1); blk++) {
+                    const float (&hb)[64] = (blk == 1) ? hv2 : hv;
+                    const int tag = ACT == 5 ? 2 * static_cast<int>(iter) + blk : static_cast<int>(iter);
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int c = 0; c < 64; c++) amax = fmaxf(amax, fabsf(hb[c]));
+                    const int par = tag & 1;
+                    volatile float* xv = xval;
+                    volatile int* xf = xflag;
+                    xv[(par * 2 + g) * 128 + r] = amax;
+                    __threadfence_block();
+                    xf[(par * 2 + g) * 128 + r] = tag + 1;
+                    long long t0 = clock64();
+                    while (xf[(par * 2 + (1 - g)) * 128 + r] < tag + 1) {
+                        if (clock64() - t0 > limit) { ok = false; break; }
+                    }
+                    if (!ok) break;
+                    __threadfence_block();
+                    amax = fmaxf(amax, xv[(par * 2 + (1 - g)) * 128 + r]);
+                    const float s = __fdiv_rn(amax, 448.0f);
+                    if (valid) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4) {
+                            uint16_t lo = 0, hi = 0;
+                            if (s != 0.0f) {
+                                lo = f2_to_e4m3x2(__fdiv_rn(hb[c], s), __fdiv_rn(hb[c + 1], s));
+                                hi = f2_to_e4m3x2(__fdiv_rn(hb[c + 2], s), __fdiv_rn(hb[c + 3], s));
+                            }
+                            w[c / 4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+                        }
+                        const int hblock = ACT == 5 ? 2 * nb + blk : nb;   // 128-column hidden block
+                        uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(row) * p.I + hblock * 128 + 64 * g);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                        if (g == 0) p.hs[static_cast<size_t>(row) * (p.I / 128) + hblock] = s;
+                    }
                 }
                 if (!ok) break;
-                __threadfence_block();
-                amax = fmaxf(amax, xv[(par * 2 + (1 - g)) * 128 + r]);
-                const float s = __fdiv_rn(amax, 448.0f);
-                if (valid) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int c = 0; c < 64; c += 4) {
-                        uint16_t lo = 0, hi = 0;
-                        if (s != 0.0f) {
-                            lo = f2_to_e4m3x2(__fdiv_rn(hv[c], s), __fdiv_rn(hv[c + 1], s));
-                            hi = f2_to_e4m3x2(__fdiv_rn(hv[c + 2], s), __fdiv_rn(hv[c + 3], s));
-                        }
-                        w[c / 4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(row) * p.I + nb * 128 + 64 * g);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; v4++) dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
-                    if (g == 0) p.hs[static_cast<size_t>(row) * (p.I / 128) + nb] = s;
-                }
             } else {
                 // ---------------------------------------------------- down
                 constexpr int NC = BN / 2;      // columns per thread

@@ -223,37 +223,51 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (lane == 0) mbar_arrive(&tempty[acc]);
                 u++;
                 const float sg = gx * wg0, su = gx * wg1;
-                float hv[32];
+                // gated: one 32-column run act(g, u) at hidden 64 nb + 32 g; ReLU^2 (no
+                // gate, 128 up rows per tile): relu(v)^2 of both 32-column halves, at
+                // hidden 128 nb + 32 g and 128 nb + 64 + 32 g
+                constexpr int NR = ACT == 5 ? 2 : 1;
+                float hv[32 * NR];
 #pragma unroll
                 for (int c = 0; c < 32; c++) {
                     const float gg = gv[c] * sg, uu = uv[c] * su;
-                    hv[c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+                    if constexpr (ACT == 5) {
+                        hv[c] = relu_sq(gg);
+                        hv[32 + c] = relu_sq(uu);
+                    } else {
+                        hv[c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+                    }
                 }
                 if (valid) {
-                    const int col0 = nb * 64 + 32 * g;      // first hidden column of this thread
-                    uint32_t w[4];
 #pragma unroll
-                    for (int b = 0; b < 2; b++) {           // two 16-blocks
-                        float amax = 0.0f;
+                    for (int run = 0; run < NR; run++) {
+                        // first hidden column of this run
+                        const int col0 = ACT == 5 ? nb * 128 + 64 * run + 32 * g : nb * 64 + 32 * g;
+                        uint32_t w[4];
 #pragma unroll
-                        for (int c = 0; c < 16; c++) amax = fmaxf(amax, fabsf(hv[16 * b + c]));
-                        const uint8_t sb = f_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), p.h_global));
-                        const float d = __fmul_rn(e4m3_to_f(sb), p.h_global);
+                        for (int b = 0; b < 2; b++) {           // two 16-blocks
+                            float amax = 0.0f;
 #pragma unroll
-                        for (int c = 0; c < 16; c += 8) {
-                            uint32_t pk = 0;
-                            if (d != 0.0f) {
+                            for (int c = 0; c < 16; c++) amax = fmaxf(amax, fabsf(hv[32 * run + 16 * b + c]));
+                            const uint8_t sb = f_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), p.h_global));
+                            const float d = __fmul_rn(e4m3_to_f(sb), p.h_global);
 #pragma unroll
-                                for (int i = 0; i < 4; i++)
-                                    pk |= static_cast<uint32_t>(f2_to_e2m1x2(__fdiv_rn(hv[16 * b + c + 2 * i], d),
-                                                                              __fdiv_rn(hv[16 * b + c + 2 * i + 1], d)))
-                                          << (8 * i);
+                            for (int c = 0; c < 16; c += 8) {
+                                uint32_t pk = 0;
+                                if (d != 0.0f) {
+#pragma unroll
+                                    for (int i = 0; i < 4; i++)
+                                        pk |= static_cast<uint32_t>(f2_to_e2m1x2(
+                                                  __fdiv_rn(hv[32 * run + 16 * b + c + 2 * i], d),
+                                                  __fdiv_rn(hv[32 * run + 16 * b + c + 2 * i + 1], d)))
+                                              << (8 * i);
+                                }
+                                w[2 * b + c / 8] = pk;
                             }
-                            w[2 * b + c / 8] = pk;
+                            p.hsf[sf_offset(prow, col0 / 16 + b, p.I / 16)] = sb;
                         }
-                        p.hsf[sf_offset(prow, col0 / 16 + b, p.I / 16)] = sb;
+                        *reinterpret_cast<uint4*>(p.hq + prow * (p.I / 2) + col0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    *reinterpret_cast<uint4*>(p.hq + prow * (p.I / 2) + col0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             } else {
                 float v0[32], v1[32];

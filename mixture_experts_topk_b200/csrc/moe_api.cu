@@ -215,8 +215,10 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
         return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: NVFP4 needs I to be a multiple of 256 (I=%d)", c.I);
     if (c.fmt == MOE_FMT_NVFP4 && !(c.hidden_global_scale > 0.0f))
         return fail(MOE_ERR_INVALID_ARG, "moe_init: NVFP4 needs a positive hidden_global_scale");
-    if (c.act < MOE_ACT_SWIGLU || c.act > MOE_ACT_REGLU)
+    if (c.act < MOE_ACT_SWIGLU || c.act > MOE_ACT_RELU2)
         return fail(MOE_ERR_INVALID_ARG, "moe_init: unknown activation %d", c.act);
+    if (c.act == MOE_ACT_RELU2 && c.I % 256 != 0)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_init: ReLU^2 experts need I to be a multiple of 256 (I=%d)", c.I);
     if ((c.act == MOE_ACT_SWIGLU_BOUNDED || c.act == MOE_ACT_SWIGLU_OAI) && !(c.act_limit > 0.0f))
         return fail(MOE_ERR_INVALID_ARG, "moe_init: this activation needs a positive act_limit");
     if (c.act == MOE_ACT_SWIGLU_OAI && !(c.act_alpha > 0.0f))
@@ -303,13 +305,42 @@ static moe_status check_T(const moe_handle* h, int T, const char* who) {
 // ------------------------------------------------------------------ pack
 extern "C" moe_status moe_pack_weights(const moe_handle* h, const moe_weights* src, void* packed, moe_stream_t stream) {
     if (!h || !src || !packed) return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: null argument");
-    if (!src->gate_q || !src->up_q || !src->down_q || !src->gate_s || !src->up_s || !src->down_s)
+    const bool relu2 = h->cfg.act == MOE_ACT_RELU2;   // up and down only
+    if ((!relu2 && (!src->gate_q || !src->gate_s)) || !src->up_q || !src->down_q || !src->up_s || !src->down_s)
         return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: null weight pointer");
     if (!aligned256(packed)) return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: packed must be 256-byte aligned");
     const moe_config& c = h->cfg;
     uint8_t* b = static_cast<uint8_t*>(packed);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int grid = 4 * h->num_sms;
+    if (relu2) {
+        // the up projection alone, in row order: W_u [E, I, K-bytes] and its scales
+        const size_t E = c.E, I = c.I, H = c.H;
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.gu_q, src->up_q, E * I * code_bytes(c.fmt, c.H), cudaMemcpyDeviceToDevice,
+                                 st));
+        if (c.fmt == MOE_FMT_NVFP4) {
+            if (!src->up_g || !src->down_g)
+                return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: NVFP4 needs the global scales");
+            pack_sf_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(src->up_s), nullptr, b + h->wl.gu_s, c.E,
+                                                 c.I, 0, c.H / 16, 0);
+            LAUNCH_CHECK("pack_sf_kernel(up)");
+            pack_sf_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(src->down_s), nullptr, b + h->wl.d_s,
+                                                 c.E, c.H, 0, c.I / 16, 0);
+            LAUNCH_CHECK("pack_sf_kernel(down)");
+            CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_q, src->down_q, E * H * (I / 2), cudaMemcpyDeviceToDevice, st));
+            // [E][2] global scales as for gated experts, both entries the up scale
+            CUDA_TRY(cudaMemcpy2DAsync(b + h->wl.gu_g, 8, src->up_g, 4, 4, c.E, cudaMemcpyDeviceToDevice, st));
+            CUDA_TRY(cudaMemcpy2DAsync(b + h->wl.gu_g + 4, 8, src->up_g, 4, 4, c.E, cudaMemcpyDeviceToDevice, st));
+            CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_g, src->down_g, E * 4, cudaMemcpyDeviceToDevice, st));
+            return MOE_OK;
+        }
+        const size_t us = c.fmt == MOE_FMT_FP8_ROW ? E * I * 4 : E * (I / 128) * (H / 128) * 4;
+        const size_t ds = c.fmt == MOE_FMT_FP8_ROW ? E * H * 4 : E * (H / 128) * (I / 128) * 4;
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.gu_s, src->up_s, us, cudaMemcpyDeviceToDevice, st));
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_s, src->down_s, ds, cudaMemcpyDeviceToDevice, st));
+        CUDA_TRY(cudaMemcpyAsync(b + h->wl.d_q, src->down_q, E * H * I, cudaMemcpyDeviceToDevice, st));
+        return MOE_OK;
+    }
     if (c.fmt == MOE_FMT_NVFP4) {
         if (!src->gate_g || !src->up_g || !src->down_g)
             return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: NVFP4 needs the global scales");
@@ -487,7 +518,7 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
     const size_t R = padded_rows(c);
     const int K = gate_up ? c.H : c.I;
-    const int N = gate_up ? 2 * c.I : c.H;
+    const int N = gate_up ? (c.act == MOE_ACT_RELU2 ? c.I : 2 * c.I) : c.H;
     CUtensorMap ta, tb;
     moe_status r = make_tmap(&ta, gate_up ? v.xq : v.hq, K / 2, R, K / 2, 128, 128);
     if (r != MOE_OK) return r;
@@ -530,6 +561,7 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     case MOE_ACT_SWIGLU_OAI: return launch_fp4<KIND_GATE_UP, MOE_ACT_SWIGLU_OAI>(h->pdl, ta, tb, p, grid, st);
     case MOE_ACT_GEGLU: return launch_fp4<KIND_GATE_UP, MOE_ACT_GEGLU>(h->pdl, ta, tb, p, grid, st);
     case MOE_ACT_REGLU: return launch_fp4<KIND_GATE_UP, MOE_ACT_REGLU>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_RELU2: return launch_fp4<KIND_GATE_UP, MOE_ACT_RELU2>(h->pdl, ta, tb, p, grid, st);
     default: return launch_fp4<KIND_GATE_UP, MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, grid, st);
     }
 }
@@ -597,7 +629,8 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     CUtensorMap ta, tb;
     moe_status r = make_tmap(&ta, v.xq, c.H, padded_rows(c), c.H, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
-    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * 2 * c.I, c.H, GEMM_BK, 256);
+    const int n_gu = c.act == MOE_ACT_RELU2 ? c.I : 2 * c.I;   // rows of the packed gate/up weights
+    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, 256);
     if (r != MOE_OK) return r;
     GemmParams p;
     memset(&p, 0, sizeof(p));
@@ -606,9 +639,9 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.tile_ptr = v.tile_ptr;
     p.E = c.E;
     p.offsets = v.offsets;
-    p.n_blocks = 2 * c.I / 256;
+    p.n_blocks = n_gu / 256;
     p.num_kb = c.H / GEMM_BK;
-    p.b_rows = 2 * c.I;
+    p.b_rows = n_gu;
     p.a_scale = static_cast<const float*>(v.xs);
     p.a_ld = (c.fmt == MOE_FMT_FP8_ROW) ? 1 : c.H / 128;
     p.b_scale = reinterpret_cast<const float*>(pw + h->wl.gu_s);
@@ -635,6 +668,8 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
             return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_GEGLU>(h->pdl, ta, tb, p, grid, st);
         case MOE_ACT_REGLU:
             return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_REGLU>(h->pdl, ta, tb, p, grid, st);
+        case MOE_ACT_RELU2:
+            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_RELU2>(h->pdl, ta, tb, p, grid, st);
         default:
             return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, grid, st);
         }
@@ -648,6 +683,8 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
         return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_GEGLU>(h->pdl, ta, tb, p, grid, st);
     case MOE_ACT_REGLU:
         return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_REGLU>(h->pdl, ta, tb, p, grid, st);
+    case MOE_ACT_RELU2:
+        return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_RELU2>(h->pdl, ta, tb, p, grid, st);
     default:
         return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, grid, st);
     }
@@ -687,7 +724,7 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     p.split = v.pick + 1;
     p.s_max = split_limit(h->picker, p.A);
     p.gu_done = chained ? gu_done_of(h, ws) : nullptr;
-    p.gu_per_mtile = (2 * c.I / 256) * 16;   // gate/up n-blocks x its 16 epilogue warps
+    p.gu_per_mtile = ((c.act == MOE_ACT_RELU2 ? c.I : 2 * c.I) / 256) * 16;   // gate/up n-blocks x 16 epilogue warps
     p.perm = v.perm;
     p.route_w = w;
     p.status = v.status;

@@ -63,6 +63,10 @@ def test_init_rejects_bad_activation_settings_without_a_gpu(lib):
         with pytest.raises(native.MoeError) as ei:
             native.moe_init(wl, 16)
         assert ei.value.status == 1
+    # ReLU^2 experts tile the up projection alone, 256 rows at a time
+    with pytest.raises(native.MoeError) as ei:
+        native.moe_init(W.custom(H=256, I=384, E=8, k=2, act=W.ACT_RELU2), 16)
+    assert ei.value.status == 2
 
 
 def test_graft_build_compiles_everything():

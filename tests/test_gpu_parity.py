@@ -302,6 +302,12 @@ ACT_CASES = {
     "nvfp4-bounded": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4, act=W.ACT_SWIGLU_BOUNDED,
                                act_limit=0.25), 300),
     "nvfp4-reglu": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4, act=W.ACT_REGLU), 300),
+    # ReLU^2 experts: up and down only
+    "row-relu2": (W.custom(H=512, I=512, E=8, k=2, act=W.ACT_RELU2), 300),
+    "row-relu2-t3": (W.custom(H=512, I=512, E=8, k=2, act=W.ACT_RELU2), 3),
+    "block128-relu2": (W.custom(H=512, I=512, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128,
+                                act=W.ACT_RELU2), 300),
+    "nvfp4-relu2": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4, act=W.ACT_RELU2), 300),
 }
 
 
