@@ -33,6 +33,39 @@ __device__ __forceinline__ void report(int32_t* status, int code, int where) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ------------------------------------------------------------------ optional timeline trace
+// Built only with -DMOE_TRACE (off in the library): KTRACE(id) at the top of a
+// kernel body records the global timer of its first CTA's entry and of its
+// last warp's exit in slot id, for a per-kernel timeline of one layer step
+// as it runs in the stream (PDL overlap included).  moe_trace_clear() and
+// moe_trace_read() in the C API of such a build reset and fetch the slots.
+#ifdef MOE_TRACE
+constexpr int TRACE_SLOTS = 32;
+__device__ unsigned long long moe_trace_buf[2 * TRACE_SLOTS];
+__device__ __forceinline__ unsigned long long global_timer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+struct TraceScope {
+    int id;
+    __device__ explicit TraceScope(int i) : id(i) {
+        if (threadIdx.x == 0) atomicMin(&moe_trace_buf[2 * id], global_timer());
+    }
+    __device__ ~TraceScope() {
+        if ((threadIdx.x & 31) == 0) atomicMax(&moe_trace_buf[2 * id + 1], global_timer());
+    }
+};
+#define KTRACE(id) ::moe::TraceScope moe_trace_scope_(id)
+#else
+#define KTRACE(id) ((void)0)
+#endif
+enum : int {
+    TR_ROUTER = 0, TR_ROUTER_SMALL = 1, TR_TOPK = 2, TR_ROUTER_FUSED = 3, TR_HIST = 4, TR_SCAN = 5,
+    TR_RANK = 6, TR_DISPATCH_SMALL = 7, TR_QUANT = 8, TR_QUANT_ROW = 9, TR_COMBINE = 10, TR_AMAX = 11,
+    TR_QUANT_FP4 = 12, TR_GEMM = 13, TR_MX_DOWN = 14, TR_FP4 = 15
+};
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -104,6 +137,28 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, ui
         : "memory");
 }
 
+// L2 eviction priority of a load (createpolicy): expert weight tiles that one
+// m-tile alone reads go in as evict_first, so streaming them does not push the
+// layer's small buffers and kernels' code out of L2; tiles that several
+// m-tiles read keep the normal priority for their reuse.
+__device__ __forceinline__ uint64_t l2_policy(bool evict_first) {
+    uint64_t pol;
+    if (evict_first)
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    else
+        asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// tma_load_2d with an L2 cache policy
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* tm, uint64_t* bar, int x, int y,
+                                                 uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
+        : "memory");
+}
+
 // Plain (non-tensor) bulk copy global -> shared, completion counted in bytes
 // on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.  No multicast.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -111,6 +166,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                      smem_u32(dst)),
                  "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
+}
+
+// bulk_load with an L2 cache policy
+__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                               uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
     hist_kernel(const int32_t* ids, int A, int E, int32_t* chunk_counts, int32_t* status) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_HIST);
     __shared__ int h[256];
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
                                                    int32_t* gu_done) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_SCAN);
     __shared__ int warp_tot[8];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     int c = 0;
@@ -174,6 +176,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
     rank_kernel(const int32_t* ids, int A, int E, const int32_t* chunk_base, int32_t* perm, int32_t* inv) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_RANK);
     __shared__ int wc[32][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) wc[i >> 8][i & 255] = 0;
@@ -218,6 +221,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK) dispatch_small_kernel(
     int32_t* gu_done) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_DISPATCH_SMALL);
     __shared__ int wc[32][256];
     __shared__ int warp_tot[8];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -306,6 +310,7 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(const __nv_bfloat16*
                                                             const int32_t* inv, uint8_t* xq, float* xs) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_QUANT);
     const int lane = threadIdx.x & 31;
     const int nI = H >> 8;
     for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
@@ -373,6 +378,7 @@ __global__ void __launch_bounds__(256) quant_scatter_row_kernel(const __nv_bfloa
                                                                 const int32_t* inv, uint8_t* xq, float* xs) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_QUANT_ROW);
     __shared__ float s_amax[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
@@ -446,6 +452,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* o, const int3
                                                       const int32_t* split, int s_max, __nv_bfloat16* y) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_COMBINE);
     const int S = split ? min(max(*split, 1), s_max) : 1;
     const size_t copy = static_cast<size_t>(T) * k * H;
     // CTA (x, y): tokens x, x + gridDim.x, ..., columns [1024 y, 1024 y + 1024)
@@ -517,6 +524,7 @@ __global__ void interleave_rows_kernel(const uint32_t* gate, const uint32_t* up,
 __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* x, long long n8, int32_t* amax_bits) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_AMAX);
     float m = 0.0f;
     for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n8; i += 256LL * gridDim.x) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
@@ -540,6 +548,7 @@ __global__ void __launch_bounds__(256) quant_scatter_nvfp4_kernel(
     const int32_t* tile_ptr, const int32_t* amax_bits, uint8_t* xq, uint8_t* xsf) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_QUANT_FP4);
     const int lane = threadIdx.x & 31;
     const int nI = H >> 8;
     const float g = __fdiv_rn(__int_as_float(*amax_bits), 2688.0f);

@@ -252,6 +252,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 
     pdl_wait();
     pdl_trigger();
+    KTRACE(p.o != nullptr ? TR_GEMM + 3 : TR_GEMM);
     int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + S::TMAP_OFF);
     const int32_t* s_off = s_tptr + TMAP_STRIDE;
     stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
@@ -270,6 +271,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                 decode_tile(t, s_tptr, p.E, n_blocks, e, mi, nb);
                 const int row0 = s_off[e] + GEMM_BM * (mi - s_tptr[e]);
                 const int brow = e * p.b_rows + nb * BN;
+                const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
                     const int s = it % STAGES;
                     if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, limit)) {
@@ -280,7 +282,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     uint8_t* sa = smem + s * S::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
                     tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
-                    tma_load_2d(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow);
+                    tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
                 }
             }
             // loads still in flight land before the CTA may exit
@@ -520,7 +522,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         for (int c = 0; c < 64; c++) hv[c] = glu<ACT>(ag[c], au[c], p.act_alpha, p.act_limit);
                     }
                 }
-                if (BSCALE == BSCALE_ROW) {
+                if constexpr (BSCALE == BSCALE_ROW) {
                     // MX requantisation: power-of-two scale per 32 hidden columns (all
                     // inside this thread), codes to the expert's 128-padded rows and
                     // scales to the chunked layout the down GEMM's tensor cores read
@@ -554,8 +556,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         }
                     }
                     publish();
-                    continue;
-                }
+                } else {
                 // BLOCK128: requantise the 128-column hidden block of this row; the
                 // two column groups exchange their partial amax through shared memory.
                 // ReLU^2 tiles hold two hidden blocks (the gate-half columns are up
@@ -601,6 +602,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     }
                 }
                 if (!ok) break;
+                }
             } else {
                 // ---------------------------------------------------- down
                 constexpr int NC = BN / 2;      // columns per thread

@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     pdl_wait();
     pdl_trigger();
+    KTRACE(p.o != nullptr ? TR_FP4 + 1 : TR_FP4);
     int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + F4_TMAP_OFF);
     const int32_t* s_off = s_tptr + TMAP_STRIDE;
     stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 int e, mi, nb;
                 decode_tile(t, s_tptr, p.E, p.n_blocks, e, mi, nb);
                 const int brow = e * p.b_rows + nb * F4_BN;
+                const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
                 const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.sf_cols * 128;
                 const uint8_t* sfb = p.sfb + static_cast<size_t>(e) * p.b_rows * p.sf_cols +
                                      static_cast<size_t>(nb) * p.sf_cols * 128;
@@ -136,10 +138,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     uint8_t* st = smem + s * F4_STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], F4_STAGE_BYTES);
                     tma_load_2d(st, &tmA, &full[s], kb * 128, mi * 128);
-                    tma_load_2d(st + F4_A_BYTES, &tmB, &full[s], kb * 128, brow);
+                    tma_load_2d_hint(st + F4_A_BYTES, &tmB, &full[s], kb * 128, brow, pol);
                     bulk_load(st + F4_A_BYTES + F4_B_BYTES, sfa + kb * F4_SF_BYTES, F4_SF_BYTES, &full[s]);
-                    bulk_load(st + F4_A_BYTES + F4_B_BYTES + F4_SF_BYTES, sfb + kb * F4_SF_BYTES, F4_SF_BYTES,
-                              &full[s]);
+                    bulk_load_hint(st + F4_A_BYTES + F4_B_BYTES + F4_SF_BYTES, sfb + kb * F4_SF_BYTES, F4_SF_BYTES,
+                                   &full[s], pol);
                 }
             }
             const uint32_t first = it > F4_STAGES ? it - F4_STAGES : 0;

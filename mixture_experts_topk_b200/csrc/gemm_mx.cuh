@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // the preceding kernel.
     if (p.gu_done == nullptr) pdl_wait();
     pdl_trigger();
+    KTRACE(TR_MX_DOWN);
     int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + MX_TMAP_OFF);
     const int32_t* s_off = s_tptr + TMAP_STRIDE;
     stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     ready_e = e;
                 }
                 const int brow = e * p.b_rows + nb * MX_BN;
+                const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
                 const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.num_kb * 512;
                 const int kb1 = (sp + 1) * p.num_kb / S;
                 for (int kb = sp * p.num_kb / S; kb < kb1; kb++, it++) {
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     uint8_t* st = smem + s * MX_STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], MX_A_BYTES + MX_B_BYTES + MX_SFA_BYTES);
                     tma_load_2d(st, &tmA, &full[s], kb * 128, mi * 128);
-                    tma_load_2d(st + MX_A_BYTES, &tmB, &full[s], kb * 128, brow);
+                    tma_load_2d_hint(st + MX_A_BYTES, &tmB, &full[s], kb * 128, brow, pol);
                     bulk_load(st + MX_A_BYTES + MX_B_BYTES, sfa + kb * 512, MX_SFA_BYTES, &full[s]);
                 }
             }

@@ -994,3 +994,21 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, c
     LAUNCH_CHECK("quant_scatter_kernel");
     return MOE_OK;
 }
+
+#ifdef MOE_TRACE
+// Timeline trace of a build made with -DMOE_TRACE: slot 2i holds the earliest
+// entry of kernel i, slot 2i+1 its latest warp exit (global timer, ns).
+extern "C" int moe_trace_clear(void) {
+    unsigned long long init[2 * TRACE_SLOTS];
+    for (int i = 0; i < TRACE_SLOTS; i++) {
+        init[2 * i] = ~0ull;
+        init[2 * i + 1] = 0;
+    }
+    return cudaMemcpyToSymbol(moe_trace_buf, init, sizeof(init)) == cudaSuccess ? 0 : -1;
+}
+extern "C" int moe_trace_read(unsigned long long* out) {
+    return cudaMemcpyFromSymbol(out, moe_trace_buf, sizeof(unsigned long long) * 2 * TRACE_SLOTS) == cudaSuccess
+               ? 0
+               : -1;
+}
+#endif

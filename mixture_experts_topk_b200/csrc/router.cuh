@@ -119,6 +119,7 @@ template <int TOK, int EXP>
 __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterParams p) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_ROUTER);
     using RT = RouterTile<TOK, EXP>;
     extern __shared__ __align__(16) uint8_t rsm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -244,6 +245,7 @@ constexpr int RS_WARPS = 4;
 __global__ void __launch_bounds__(RS_WARPS * 32) router_logits_small_kernel(RouterParams p) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_ROUTER_SMALL);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.y * RS_WARPS + warp;
     const int t0 = blockIdx.x * RS_TG;
@@ -338,6 +340,7 @@ __device__ __forceinline__ void router_topk_token(const RouterParams& p, const f
 __global__ void __launch_bounds__(256) router_topk_kernel(RouterParams p) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_TOPK);
     const int lane = threadIdx.x & 31;
     for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < p.T; t += gridDim.x * 8)
         router_topk_token(p, p.logits + static_cast<size_t>(t) * p.E, t, lane);
@@ -351,6 +354,7 @@ constexpr int RF_MAX_E = 32;
 __global__ void __launch_bounds__(RF_MAX_E * 32) router_small_fused_kernel(RouterParams p) {
     pdl_wait();
     pdl_trigger();
+    KTRACE(TR_ROUTER_FUSED);
     __shared__ float s_l[RS_TG][RF_MAX_E];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = warp;
