@@ -57,8 +57,14 @@ struct TraceScope {
     }
 };
 #define KTRACE(id) ::moe::TraceScope moe_trace_scope_(id)
+// event k of accumulation unit i of CTA 0 (first TRACE_BLKS units)
+constexpr int TRACE_BLKS = 96;
+__device__ unsigned long long moe_trace_blk[TRACE_BLKS][8];
+#define KTRACE_BLK(i, k) \
+    do { if (blockIdx.x == 0 && (i) < ::moe::TRACE_BLKS) ::moe::moe_trace_blk[(i)][(k)] = ::moe::global_timer(); } while (0)
 #else
 #define KTRACE(id) ((void)0)
+#define KTRACE_BLK(i, k) ((void)0)
 #endif
 enum : int {
     TR_ROUTER = 0, TR_ROUTER_SMALL = 1, TR_TOPK = 2, TR_ROUTER_FUSED = 3, TR_HIST = 4, TR_SCAN = 5,

@@ -283,6 +283,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
                     tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
                     tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                    if (PROMOTE) KTRACE_BLK(it, 7);
                 }
             }
             // loads still in flight land before the CTA may exit
@@ -307,10 +308,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         acc = u % NBUF;
                         if (!mbar_wait(&tempty[acc], ((u / NBUF) & 1) ^ 1, limit)) { ok = false; break; }
                         tc_fence_after();
+                        KTRACE_BLK(u, 0);
                     }
                     const int s = it % STAGES;
                     if (!mbar_wait(&full[s], (it / STAGES) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
+                    if (PROMOTE) KTRACE_BLK(u, 1);
                     const uint32_t a_addr = smem_u32(smem + s * S::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + GEMM_A_BYTES;
                     const uint32_t d = tmem_base + acc * BN;
@@ -321,6 +324,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     mma_commit(&empty[s]);
                     if (PROMOTE) {
                         mma_commit(&tfull[acc]);
+                        KTRACE_BLK(u, 2);
                         u++;
                     }
                 }
@@ -493,6 +497,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         const uint32_t acc = u % NBUF;
                         if (!warp_wait(&tfull[acc], (u / NBUF) & 1, limit)) { ok = false; break; }
                         tc_fence_after();
+                        if (ew == 0 && lane == 0) KTRACE_BLK(u, 3);
 #pragma unroll
                         for (int half = 0; half < 2; half++) {
                             if (!any_valid) break;   // no stored row: skip the readback
@@ -505,9 +510,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                                 au[32 * half + c] = fmaf(vu[c], su, au[32 * half + c]);
                             }
                         }
+                        if (ew == 0 && lane == 0) KTRACE_BLK(u, 4);
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty[acc]);
+                        if (ew == 0 && lane == 0) KTRACE_BLK(u, 5);
+                        if (ew == EPI - 1 && lane == 0) KTRACE_BLK(u, 6);
                         u++;
                     }
                     if (!ok) break;

@@ -428,10 +428,11 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
         auto kern = router_logits_kernel<64, 8>;
         LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 63) / 64, 1), RT_WARPS * 32, RT::SMEM, st, p);
     } else {
-        using RT = RouterTile<32, 16>;
-        CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<32, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, RT::SMEM));
-        auto kern = router_logits_kernel<32, 16>;
-        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 31) / 32, (h->cfg.E + 15) / 16), RT_WARPS * 32,
+        using RT = RouterTile<64, 16, 16>;
+        CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<64, 16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      RT::SMEM));
+        auto kern = router_logits_kernel<64, 16, 16>;
+        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 63) / 64, (h->cfg.E + 15) / 16), RT_WARPS * 32,
                RT::SMEM, st, p);
     }
     LAUNCH(h->pdl, "router_topk_kernel", router_topk_kernel, std::min((T + 7) / 8, 16 * h->num_sms), 256, 0, st, p);
@@ -1005,6 +1006,11 @@ extern "C" int moe_trace_clear(void) {
         init[2 * i + 1] = 0;
     }
     return cudaMemcpyToSymbol(moe_trace_buf, init, sizeof(init)) == cudaSuccess ? 0 : -1;
+}
+extern "C" int moe_trace_blk_read(unsigned long long* out) {
+    return cudaMemcpyFromSymbol(out, moe::moe_trace_blk, sizeof(unsigned long long) * TRACE_BLKS * 8) == cudaSuccess
+               ? 0
+               : -1;
 }
 extern "C" int moe_trace_read(unsigned long long* out) {
     return cudaMemcpyFromSymbol(out, moe_trace_buf, sizeof(unsigned long long) * 2 * TRACE_SLOTS) == cudaSuccess

@@ -11,12 +11,13 @@
 // adds them as the balanced pairwise tree ((p0+p1)+(p2+p3))+...; then + bias[e].
 //
 // Kernels:
-//  router_logits_kernel  a 2-D grid of CTA tiles (TOK tokens x EXP experts; 32 x 16,
-//                        or 64 x 8 when E <= 8).
+//  router_logits_kernel  a 2-D grid of CTA tiles (TOK tokens x EXP experts; 64 x 16
+//                        with 16-token x 8-expert micro-tiles, or 64 x 8 with
+//                        8 x 8 micro-tiles when E <= 8).
 //                        The 256-wide H chunks of X and Wr go through shared
 //                        memory with a 4-stage cp.async pipeline; each of the 8
-//                        warps owns one 8-token x 8-expert micro-tile, so one
-//                        16-byte X read from shared memory feeds 64 fma.
+//                        warps owns one micro-tile: per 16 bytes read from
+//                        shared memory, 8 x 8 runs 43 fma and 16 x 8 64.
 //  router_logits_small_kernel  batches of at most 128 tokens: one warp per
 //                        (expert, 4 tokens) reading global memory directly.
 //  router_small_fused_kernel   the same for at most 32 experts, with the top-k
@@ -28,11 +29,11 @@
 
 namespace moe {
 
-constexpr int RT_WARPS = 8;   // (TOK / 8) x (EXP / 8) micro-tiles of 8 x 8
+constexpr int RT_WARPS = 8;   // (TOK / MT) x (EXP / 8) micro-tiles of MT tokens x 8 experts
 
-template <int TOK, int EXP>
+template <int TOK, int EXP, int MT = 8>
 struct RouterTile {
-    static_assert((TOK / 8) * (EXP / 8) == RT_WARPS, "one micro-tile per warp");
+    static_assert((TOK / MT) * (EXP / 8) == RT_WARPS, "one micro-tile per warp");
     static constexpr int X_BYTES = TOK * 256 * 2;    // 256 bf16 of H per token
     static constexpr int W_BYTES = EXP * 256 * 4;    // 256 fp32 of H per expert
     static constexpr int STAGE = X_BYTES + W_BYTES;
@@ -98,7 +99,7 @@ struct RouterLoader {
         // Wr piece c holds h = 4c..4c+3, half (c & 1) of lane (c >> 1)'s eight values;
         // stored at (c & 1) * 512 + (c >> 1) * 16 so each half-read of a warp is
         // 512 contiguous bytes (no bank conflicts)
-        wdst = RouterTile<TOK, EXP>::X_BYTES + wr * 1024 + (wc & 1) * 512 + (wc >> 1) * 16;
+        wdst = TOK * 512 + wr * 1024 + (wc & 1) * 512 + (wc >> 1) * 16;   // after the X rows
     }
     __device__ __forceinline__ void load(uint8_t* st, int i) const {
 #pragma unroll
@@ -115,21 +116,34 @@ struct RouterLoader {
     }
 };
 
-template <int TOK, int EXP>
+// One step of the lane butterfly: of the 2 HALF values in `in`, a lane keeps
+// the upper half if (lane & off), else the lower, and adds the partner lane's
+// copy of the kept half.
+template <int HALF>
+__device__ __forceinline__ void butterfly_halve(const float* in, float* out, int lane, int off) {
+    const bool b = lane & off;
+#pragma unroll
+    for (int v = 0; v < HALF; v++) {
+        const float send = b ? in[v] : in[v + HALF], keep = b ? in[v + HALF] : in[v];
+        out[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, off));
+    }
+}
+
+template <int TOK, int EXP, int MT = 8>
 __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterParams p) {
     pdl_wait();
     pdl_trigger();
     KTRACE(TR_ROUTER);
-    using RT = RouterTile<TOK, EXP>;
+    using RT = RouterTile<TOK, EXP, MT>;
     extern __shared__ __align__(16) uint8_t rsm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * TOK, e0 = blockIdx.y * EXP;
-    const int tg = warp % (TOK / 8), eg = warp / (TOK / 8);   // this warp's micro-tile
+    const int tg = warp % (TOK / MT), eg = warp / (TOK / MT);   // this warp's micro-tile
     const int nI = p.H >> 8;
 
-    float acc[8][8];
+    float acc[MT][8];
 #pragma unroll
-    for (int a = 0; a < 8; a++)
+    for (int a = 0; a < MT; a++)
 #pragma unroll
         for (int b = 0; b < 8; b++) acc[a][b] = 0.0f;
 
@@ -143,92 +157,89 @@ __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterPara
         // chunk i is complete once at most (issued after it) groups are pending
         cp_async_wait_le(min(nI - 1 - i, RT::NSTAGE - 1));
         __syncthreads();
-        const uint8_t* xs = st + (8 * tg) * 512 + lane * 16;
+        const uint8_t* xs = st + (MT * tg) * 512 + lane * 16;
         const uint8_t* ws = st + RT::X_BYTES + (8 * eg) * 1024 + lane * 16;
-        // The warp's 8 experts x 8 values and 8 tokens x 8 values of this chunk
-        // sit in registers; for each j the 64 accumulators take one fma each,
-        // so consecutive fma are independent.  Each (token, expert) chain
-        // still runs j = 0..7 in order.
-        float wv[8][8];
+        if constexpr (MT == 8) {
+            // The warp's 8 experts x 8 values and 8 tokens x 8 values of this chunk
+            // sit in registers; for each j the 64 accumulators take one fma each,
+            // so consecutive fma are independent.  Each (token, expert) chain
+            // still runs j = 0..7 in order.
+            float wv[8][8];
 #pragma unroll
-        for (int ee = 0; ee < 8; ee++) {
-            const float4 wa = *reinterpret_cast<const float4*>(ws + ee * 1024);
-            const float4 wb = *reinterpret_cast<const float4*>(ws + ee * 1024 + 512);
-            wv[ee][0] = wa.x; wv[ee][1] = wa.y; wv[ee][2] = wa.z; wv[ee][3] = wa.w;
-            wv[ee][4] = wb.x; wv[ee][5] = wb.y; wv[ee][6] = wb.z; wv[ee][7] = wb.w;
-        }
-        uint32_t xw[8][4];
+            for (int ee = 0; ee < 8; ee++) {
+                const float4 wa = *reinterpret_cast<const float4*>(ws + ee * 1024);
+                const float4 wb = *reinterpret_cast<const float4*>(ws + ee * 1024 + 512);
+                wv[ee][0] = wa.x; wv[ee][1] = wa.y; wv[ee][2] = wa.z; wv[ee][3] = wa.w;
+                wv[ee][4] = wb.x; wv[ee][5] = wb.y; wv[ee][6] = wb.z; wv[ee][7] = wb.w;
+            }
+            uint32_t xw[8][4];
 #pragma unroll
-        for (int tt = 0; tt < 8; tt++) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(xs + tt * 512);
-            xw[tt][0] = xv.x; xw[tt][1] = xv.y; xw[tt][2] = xv.z; xw[tt][3] = xv.w;
-        }
+            for (int tt = 0; tt < 8; tt++) {
+                const uint4 xv = *reinterpret_cast<const uint4*>(xs + tt * 512);
+                xw[tt][0] = xv.x; xw[tt][1] = xv.y; xw[tt][2] = xv.z; xw[tt][3] = xv.w;
+            }
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            float xj[8];
+            for (int j = 0; j < 8; j++) {
+                float xj[8];
 #pragma unroll
-            for (int tt = 0; tt < 8; tt++) xj[tt] = (j & 1) ? bf16_hi(xw[tt][j >> 1]) : bf16_lo(xw[tt][j >> 1]);
+                for (int tt = 0; tt < 8; tt++) xj[tt] = (j & 1) ? bf16_hi(xw[tt][j >> 1]) : bf16_lo(xw[tt][j >> 1]);
 #pragma unroll
-            for (int tt = 0; tt < 8; tt++)
+                for (int tt = 0; tt < 8; tt++)
 #pragma unroll
-                for (int ee = 0; ee < 8; ee++) acc[tt][ee] = __fmaf_rn(xj[tt], wv[ee][j], acc[tt][ee]);
+                    for (int ee = 0; ee < 8; ee++) acc[tt][ee] = __fmaf_rn(xj[tt], wv[ee][j], acc[tt][ee]);
+            }
+        } else {
+            // 16 tokens x 8 experts: each shared-memory value feeds twice the fma
+            // of the 8 x 8 tile.  The lane's 8 values per row go in two halves
+            // (j = 0..3, then 4..7), so each chain still runs j in order.
+#pragma unroll
+            for (int jh = 0; jh < 2; jh++) {
+                float wv[8][4];
+#pragma unroll
+                for (int ee = 0; ee < 8; ee++) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(ws + ee * 1024 + jh * 512);
+                    wv[ee][0] = w4.x; wv[ee][1] = w4.y; wv[ee][2] = w4.z; wv[ee][3] = w4.w;
+                }
+                uint32_t xw[MT][2];
+#pragma unroll
+                for (int tt = 0; tt < MT; tt++) {
+                    const uint2 x2 = *reinterpret_cast<const uint2*>(xs + tt * 512 + jh * 8);
+                    xw[tt][0] = x2.x; xw[tt][1] = x2.y;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    float xj[MT];
+#pragma unroll
+                    for (int tt = 0; tt < MT; tt++) xj[tt] = (j & 1) ? bf16_hi(xw[tt][j >> 1]) : bf16_lo(xw[tt][j >> 1]);
+#pragma unroll
+                    for (int tt = 0; tt < MT; tt++)
+#pragma unroll
+                        for (int ee = 0; ee < 8; ee++) acc[tt][ee] = __fmaf_rn(xj[tt], wv[ee][j], acc[tt][ee]);
+                }
+            }
         }
         __syncthreads();   // the stage is refilled NSTAGE-1 chunks later
     }
-    // Sum the 32 lane partials of all 64 (token, expert) pairs by recursive
-    // halving over lane offsets 1, 2, 4, 8, 16: at each step a lane keeps half
-    // of its values and adds the partner's copy of that half, so every sum is
-    // the pairwise tree ((p0+p1)+(p2+p3))+... of the fixed order.  Afterwards
-    // lane l holds pairs 2 r(l) and 2 r(l) + 1, r = 5-bit reversal of l.
-    float* a64 = &acc[0][0];
-    float a32[32], a16[16], a8[8], a4[4], a2[2];
-    {
-        const bool b = lane & 1;
-#pragma unroll
-        for (int v = 0; v < 32; v++) {
-            const float send = b ? a64[v] : a64[v + 32], keep = b ? a64[v + 32] : a64[v];
-            a32[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 1));
-        }
-    }
-    {
-        const bool b = lane & 2;
-#pragma unroll
-        for (int v = 0; v < 16; v++) {
-            const float send = b ? a32[v] : a32[v + 16], keep = b ? a32[v + 16] : a32[v];
-            a16[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-        }
-    }
-    {
-        const bool b = lane & 4;
-#pragma unroll
-        for (int v = 0; v < 8; v++) {
-            const float send = b ? a16[v] : a16[v + 8], keep = b ? a16[v + 8] : a16[v];
-            a8[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-        }
-    }
-    {
-        const bool b = lane & 8;
-#pragma unroll
-        for (int v = 0; v < 4; v++) {
-            const float send = b ? a8[v] : a8[v + 4], keep = b ? a8[v + 4] : a8[v];
-            a4[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 8));
-        }
-    }
-    {
-        const bool b = lane & 16;
-#pragma unroll
-        for (int v = 0; v < 2; v++) {
-            const float send = b ? a4[v] : a4[v + 2], keep = b ? a4[v + 2] : a4[v];
-            a2[v] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-        }
-    }
+    // Sum the 32 lane partials of all NV = 8 MT (token, expert) pairs by
+    // recursive halving over lane offsets 1, 2, 4, 8, 16: at each step a lane
+    // keeps half of its values and adds the partner's copy of that half, so every
+    // sum is the pairwise tree ((p0+p1)+(p2+p3))+... of the fixed order.
+    // Afterwards lane l holds pairs NV/32 r(l) .. NV/32 r(l) + NV/32 - 1,
+    // r = 5-bit reversal of l.
+    constexpr int NV = MT * 8;
+    float h1[NV / 2], h2[NV / 4], h3[NV / 8], h4[NV / 16], av[NV / 32];
+    butterfly_halve<NV / 2>(&acc[0][0], h1, lane, 1);
+    butterfly_halve<NV / 4>(h1, h2, lane, 2);
+    butterfly_halve<NV / 8>(h2, h3, lane, 4);
+    butterfly_halve<NV / 16>(h3, h4, lane, 8);
+    butterfly_halve<NV / 32>(h4, av, lane, 16);
     const int rl = ((lane & 1) << 4) | ((lane & 2) << 2) | (lane & 4) | ((lane & 8) >> 2) | ((lane & 16) >> 4);
 #pragma unroll
-    for (int u = 0; u < 2; u++) {
-        const int idx = 2 * rl + u;
-        const int t = t0 + 8 * tg + (idx >> 3), e = e0 + 8 * eg + (idx & 7);
+    for (int u = 0; u < NV / 32; u++) {
+        const int idx = (NV / 32) * rl + u;
+        const int t = t0 + MT * tg + (idx >> 3), e = e0 + 8 * eg + (idx & 7);
         if (t < p.T && e < p.E) {
-            float val = a2[u];
+            float val = av[u];
             if (p.bias) val = __fadd_rn(val, p.bias[e]);
             p.logits[static_cast<size_t>(t) * p.E + e] = val;
         }

@@ -143,7 +143,8 @@ def test_router_ids_bit_exact(name):
                                            (4096, 8, 2, W.SCORE_SOFTMAX, 33), (4096, 8, 2, W.SCORE_SOFTMAX, 1),
                                            (2048, 250, 8, W.SCORE_SOFTMAX, 127), (256, 32, 4, W.SCORE_SIGMOID, 5),
                                            (256, 3, 2, W.SCORE_SOFTMAX, 7),
-                                           (2048, 256, 8, W.SCORE_SOFTMAX, 129), (4096, 8, 2, W.SCORE_SOFTMAX, 150)])
+                                           (2048, 256, 8, W.SCORE_SOFTMAX, 129), (4096, 8, 2, W.SCORE_SOFTMAX, 150),
+                                           (512, 40, 4, W.SCORE_SIGMOID, 200), (6144, 256, 8, W.SCORE_SOFTMAX, 257)])
 def test_router_named_shapes_bit_exact(H, E, k, score, T):
     """Both logits kernels (small batches, and the tiled one above 128 tokens)
     give the oracle's fp32 logits bit for bit, and its ids."""
