@@ -153,6 +153,7 @@ def test_router_named_shapes_bit_exact(H, E, k, score, T):
     x = synth.tokens(wl, T, seed=3)
     h = native.moe_init(wl, T)
     ws = torch.empty(native.moe_workspace_size(h), dtype=torch.uint8, device="cuda")
+    native.moe_workspace_init(h, ws)
     ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
     w = torch.empty(T, k, dtype=torch.float32, device="cuda")
     native.moe_route(h, x.cuda(), T, wr.cuda(), bias.cuda(), ids, w, ws)
@@ -171,6 +172,7 @@ def test_router_equal_logits_tie_break():
     wl = W.custom(H=256, I=128, E=16, k=4)
     h = native.moe_init(wl, 8)
     ws = torch.empty(native.moe_workspace_size(h), dtype=torch.uint8, device="cuda")
+    native.moe_workspace_init(h, ws)
     x = synth.tokens(wl, 8, seed=1).cuda()
     wr = torch.zeros(16, 256, device="cuda")
     ids = torch.empty(8, 4, dtype=torch.int32, device="cuda")
