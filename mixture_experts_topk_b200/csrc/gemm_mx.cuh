@@ -149,8 +149,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     // all gate/up parts of expert e are stored before its hidden is read
                     const int target = (s_tptr[e + 1] - s_tptr[e]) * p.gu_per_mtile;
                     const long long t0 = clock64();
+                    // polled with a pause, so that a hundred CTAs waiting on the few
+                    // counters of the first experts do not keep those L2 lines busy
+                    // while the gate/up epilogues increment them
                     while (ld_acquire(p.gu_done + e) < target) {
                         if (clock64() - t0 > limit) { ok = false; break; }
+                        __nanosleep(500);
                     }
                     if (!ok) {
                         report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
