@@ -383,6 +383,26 @@ __device__ __forceinline__ float glu(float g, float u, float alpha, float limit)
     }
 }
 
+// The same activations for an e4m3 hidden: the sigmoid uses the hardware
+// exponential and reciprocal (__expf, __fdividef: a few ulp of fp32). The
+// result is rounded to an e4m3 code (a 2^-4 relative step) right after, so a
+// code changes only when the value sits within those ulp of a rounding
+// boundary; the parity tests bound the fraction of such codes.  (An e2m1
+// hidden keeps glu: one of its codes moves a value by up to half.)  For
+// g < -88 exp overflows and __fdividef(g, inf) is 0, the limit of silu.
+template <int ACT>
+__device__ __forceinline__ float glu_e4m3(float g, float u, float alpha, float limit) {
+    if constexpr (ACT == 0) {
+        return __fdividef(g, 1.0f + __expf(-g)) * u;
+    } else if constexpr (ACT == 1 || ACT == 2) {
+        const float gc = fminf(g, limit), uc = fminf(fmaxf(u, -limit), limit);
+        if constexpr (ACT == 1) return __fdividef(gc, 1.0f + __expf(-gc)) * uc;
+        else return __fdividef(gc, 1.0f + __expf(-alpha * gc)) * (uc + 1.0f);
+    } else {
+        return glu<ACT>(g, u, alpha, limit);
+    }
+}
+
 // ReLU^2 experts (no gate): h = max(u, 0)^2
 __device__ __forceinline__ float relu_sq(float u) {
     const float r = fmaxf(u, 0.0f);

@@ -439,7 +439,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 #pragma unroll
                                     for (int ob = 0; ob < (ACT == 5 ? 2 : 1); ob++) {
                                         const float hvv = ACT == 5 ? relu_sq(ob ? uu : gg)
-                                                                   : glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+                                                                   : glu_e4m3<ACT>(gg, uu, p.act_alpha, p.act_limit);
                                         const int col = hcol + 128 * ob;
                                         float amax = fabsf(hvv);
 #pragma unroll
@@ -470,7 +470,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                                 hv[32 * half + c] = relu_sq(gg);
                                 hv[32 * (NH + half) + c] = relu_sq(uu);
                             } else {
-                                hv[32 * half + c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+                                hv[32 * half + c] = glu_e4m3<ACT>(gg, uu, p.act_alpha, p.act_limit);
                             }
                         }
                     }
@@ -527,7 +527,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         }
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 64; c++) hv[c] = glu<ACT>(ag[c], au[c], p.act_alpha, p.act_limit);
+                        for (int c = 0; c < 64; c++) hv[c] = glu_e4m3<ACT>(ag[c], au[c], p.act_alpha, p.act_limit);
                     }
                 }
                 if constexpr (BSCALE == BSCALE_ROW) {
