@@ -145,29 +145,56 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const int sp = t % S;   // unit-major: all splits of a unit together, experts in order
                 int e, mi, nb;
                 decode_tile(t / S, s_tptr, p.E, p.n_blocks, e, mi, nb);
+                const int brow = e * p.b_rows + nb * MX_BN;
+                const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
+                const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.num_kb * 512;
+                const int kb0 = sp * p.num_kb / S, kb1 = (sp + 1) * p.num_kb / S;
+                int kb = kb0;
                 if (p.gu_done != nullptr && e != ready_e) {
-                    // all gate/up parts of expert e are stored before its hidden is read
-                    const int target = (s_tptr[e + 1] - s_tptr[e]) * p.gu_per_mtile;
-                    const long long t0 = clock64();
-                    // polled with a pause, so that a hundred CTAs waiting on the few
-                    // counters of the first experts do not keep those L2 lines busy
-                    // while the gate/up epilogues increment them
-                    while (ld_acquire(p.gu_done + e) < target) {
-                        if (clock64() - t0 > limit) { ok = false; break; }
-                        __nanosleep(500);
+                    // The weight tiles do not depend on the gate/up GEMM: the first
+                    // stages of the unit take their B tiles now, and their hidden
+                    // rows (A) and scales once all gate/up parts of expert e are
+                    // stored, so the weight stream overlaps the wait.
+                    const int npre = min(kb1 - kb0, MX_STAGES);
+                    int armed = 0;
+                    for (; armed < npre; armed++) {
+                        const uint32_t itj = it + armed;
+                        const int s = itj % MX_STAGES;
+                        if (!mbar_wait(&empty[s], ((itj / MX_STAGES) & 1) ^ 1, limit)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&full[s], MX_A_BYTES + MX_B_BYTES + MX_SFA_BYTES);
+                        tma_load_2d_hint(smem + s * MX_STAGE_BYTES + MX_A_BYTES, &tmB, &full[s], (kb0 + armed) * 128,
+                                         brow, pol);
                     }
+                    if (ok) {
+                        const int target = (s_tptr[e + 1] - s_tptr[e]) * p.gu_per_mtile;
+                        const long long t0 = clock64();
+                        // polled with a pause, so that a hundred CTAs waiting on the few
+                        // counters of the first experts do not keep those L2 lines busy
+                        // while the gate/up epilogues increment them
+                        while (ld_acquire(p.gu_done + e) < target) {
+                            if (clock64() - t0 > limit) { ok = false; break; }
+                            __nanosleep(500);
+                        }
+                    }
+                    fence_proxy_async_global();
+                    // the armed stages get their A and scales even after a timeout, so
+                    // that no copy into them is left incomplete
+                    for (int j = 0; j < armed; j++) {
+                        const uint32_t itj = it + j;
+                        uint8_t* st = smem + (itj % MX_STAGES) * MX_STAGE_BYTES;
+                        tma_load_2d(st, &tmA, &full[itj % MX_STAGES], (kb0 + j) * 128, mi * 128);
+                        bulk_load(st + MX_A_BYTES + MX_B_BYTES, sfa + (kb0 + j) * 512, MX_SFA_BYTES,
+                                  &full[itj % MX_STAGES]);
+                    }
+                    it += armed;
+                    kb += armed;
                     if (!ok) {
                         report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
                         break;
                     }
-                    fence_proxy_async_global();
                     ready_e = e;
                 }
-                const int brow = e * p.b_rows + nb * MX_BN;
-                const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
-                const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.num_kb * 512;
-                const int kb1 = (sp + 1) * p.num_kb / S;
-                for (int kb = sp * p.num_kb / S; kb < kb1; kb++, it++) {
+                for (; kb < kb1; kb++, it++) {
                     const int s = it % MX_STAGES;
                     if (!mbar_wait(&empty[s], ((it / MX_STAGES) & 1) ^ 1, limit)) {
                         report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
