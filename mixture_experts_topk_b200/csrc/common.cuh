@@ -57,7 +57,11 @@ struct TraceScope {
     }
 };
 #define KTRACE(id) ::moe::TraceScope moe_trace_scope_(id)
-// event k of accumulation unit i of CTA 0 (first TRACE_BLKS units)
+// Per-K-block events of CTA 0 in the promoted (FP8_BLOCK128) GEMMs, for the
+// first TRACE_BLKS accumulation units i: k = 0 MMA thread got a free
+// accumulator, 1 it got the filled stage, 2 it committed the MMAs, 3 epilogue
+// warp 0 saw the accumulator full, 4 it had read and added it, 5 it released
+// it, 6 the last epilogue warp released it, 7 the producer issued the stage.
 constexpr int TRACE_BLKS = 96;
 __device__ unsigned long long moe_trace_blk[TRACE_BLKS][8];
 #define KTRACE_BLK(i, k) \
