@@ -423,10 +423,13 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
         LAUNCH(h->pdl, "router_logits_small_kernel", router_logits_small_kernel,
                dim3((T + RS_TG - 1) / RS_TG, (h->cfg.E + RS_WARPS - 1) / RS_WARPS), RS_WARPS * 32, 0, st, p);
     } else if (h->cfg.E <= 8) {
-        using RT = RouterTile<64, 8>;
-        CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<64, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, RT::SMEM));
-        auto kern = router_logits_kernel<64, 8>;
-        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 63) / 64, 1), RT_WARPS * 32, RT::SMEM, st, p);
+        // 32-token tiles (4-token x 8-expert micro-tiles), so that T = 4096 keeps
+        // 128 SMs busy rather than 64
+        using RT = RouterTile<32, 8, 4>;
+        CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<32, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      RT::SMEM));
+        auto kern = router_logits_kernel<32, 8, 4>;
+        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 31) / 32, 1), RT_WARPS * 32, RT::SMEM, st, p);
     } else {
         using RT = RouterTile<64, 16, 16>;
         CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<64, 16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
