@@ -12,8 +12,8 @@
 //
 // Kernels:
 //  router_logits_kernel  a 2-D grid of CTA tiles (TOK tokens x EXP experts; 64 x 16
-//                        with 16-token x 8-expert micro-tiles, or 64 x 8 with
-//                        8 x 8 micro-tiles when E <= 8).
+//                        with 16-token x 8-expert micro-tiles, or 32 x 8 with
+//                        4 x 8 micro-tiles when E <= 8).
 //                        The 256-wide H chunks of X and Wr go through shared
 //                        memory with a 4-stage cp.async pipeline; each of the 8
 //                        warps owns one micro-tile: per 16 bytes read from
