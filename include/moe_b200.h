@@ -223,6 +223,18 @@ moe_status moe_set_tile_config(moe_handle* h, int down_bn);
  * plain stream order.  Host state only; MOE_ERR_INVALID_ARG for other values. */
 moe_status moe_set_launch_options(moe_handle* h, int pdl);
 
+/* GEMM options.  cta_pairs = 1 (the default): an FP8_ROW SwiGLU layer whose
+ * batch holds at least 4 row tiles of 128 per expert on average
+ * (T*k >= 512 E) runs the gate/up GEMM on CTA pairs: 2-CTA clusters whose
+ * tcgen05.mma.cta_group::2 covers two row tiles of one expert (M = 256), each
+ * CTA loading its own 128 rows of X and half of the 256 weight rows (no
+ * multicast), so a 32 KB stage feeds what a 48 KB stage feeds alone.  An
+ * expert with an odd row-tile count runs its last pair half empty.  The
+ * results are those of the single-CTA kernel up to the fp32 summation order
+ * inside the tensor core.  cta_pairs = 0 keeps single CTAs.  Errors:
+ * MOE_ERR_INVALID_ARG for a null handle or another value. */
+moe_status moe_set_gemm_options(moe_handle* h, int cta_pairs);
+
 /* Limit, in SM clock cycles, of every wait of the GEMM kernels on another
  * role or CTA (stage, accumulator and exchange barriers); default 2e9 (about
  * 1 s).  A wait that runs out records MOE_ERR_DEVICE_TIMEOUT and the role in

@@ -150,12 +150,12 @@ __host__ __device__ constexpr int epi_warp_floats() {
     return EPI == 8 ? EPI_WARP_FLOATS : sparse_round<EPI>() * 64 + sparse_round<EPI>();
 }
 
-template <int BN, int STAGES, int EPI = 8>
+template <int BN, int STAGES, int EPI = 8, bool PAIR = false>
 struct GemmSmem {
     // accumulator buffers in TMEM (512 columns): deeper for narrower tiles, so the
     // MMA can run further ahead of a per-K-block epilogue
     static constexpr int NBUF = (512 / BN) < 4 ? (512 / BN) : 4;
-    static constexpr int B_BYTES = BN * GEMM_BK;
+    static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * GEMM_BK;   // a CTA pair splits B by rows
     static constexpr int STAGE_BYTES = GEMM_A_BYTES + B_BYTES;
     static constexpr int TILES_BYTES = STAGES * STAGE_BYTES;
     // after the tiles: barriers, TMEM address, amax exchange
@@ -166,7 +166,8 @@ struct GemmSmem {
     static constexpr int XCHG_BYTES = 2 * 2 * 128 * 4 * 2;   // [parity][group][row] value + flag
     static constexpr int TMAP_OFF = XCHG_OFF + XCHG_BYTES;
     static constexpr int SPARSE_OFF = TMAP_OFF + TMAP_BYTES;
-    static constexpr int TOTAL = SPARSE_OFF + EPI * epi_warp_floats<EPI>() * 4 + 1024; // + alignment slack
+    static constexpr int PPTR_OFF = SPARSE_OFF + EPI * epi_warp_floats<EPI>() * 4;   // CTA pairs: m-pair map
+    static constexpr int TOTAL = PPTR_OFF + (PAIR ? TMAP_STRIDE * 4 : 0) + 1024;       // + alignment slack
     static_assert(SPARSE_OFF % 16 == 0, "staging block must be 16-byte aligned");
 };
 
@@ -198,17 +199,38 @@ __device__ __forceinline__ void decode_tile(int t, const int32_t* s_tptr, int E,
     mi = first + local % mt;
 }
 
+// CTA pairs: unit t -> (expert, m-pair, n-block).  Expert e owns m-pairs
+// [pptr[e], pptr[e+1]) (ceil(m-tiles / 2) of them), n-block-major with its
+// m-pairs fastest; m-pair j covers the expert's m-tiles 2j (rank 0) and 2j + 1
+// (rank 1, absent when the count is odd).
+__device__ __forceinline__ void decode_pair(int t, const int32_t* s_pptr, int E, int n_blocks, int& e, int& mp,
+                                            int& nb) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_pptr[mid] * n_blocks <= t) lo = mid; else hi = mid;
+    }
+    const int first = s_pptr[lo];
+    const int np = s_pptr[lo + 1] - first;
+    const int local = t - first * n_blocks;
+    e = lo;
+    nb = local / np;
+    mp = local % np;
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long long limit) {
     const bool ok = mbar_wait(bar, parity, limit);
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8, int ACT = 0>
+template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8, int ACT = 0, bool PAIR = false>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                                           const int n_blocks, uint8_t* smem_raw) {
     static_assert(EPI == 8 || (EPI == 16 && KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW && !PROMOTE && BN == 256),
                   "16 epilogue warps are built for the FP8_ROW gate/up GEMM only");
-    using S = GemmSmem<BN, STAGES, EPI>;
+    static_assert(!PAIR || (KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW && !PROMOTE && BN == 256),
+                  "CTA pairs are built for the FP8_ROW gate/up GEMM only");
+    using S = GemmSmem<BN, STAGES, EPI, PAIR>;
     constexpr int CG = EPI / 4;          // column groups
     constexpr int GC = 128 / CG;         // gate/up: hidden columns per thread (64 or 32)
     constexpr int NH = GC / 32;          // 32-column blocks per thread
@@ -228,15 +250,18 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t TMEM_COLS = NBUF * BN;
+    // CTA pairs: rank 0 issues the MMAs; its full and tempty barriers take the
+    // arrivals of both CTAs
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], PAIR ? 2 : 1);   // pairs: one expect_tx arrival per CTA
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < NBUF; b++) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], EPI);   // one arrival per epilogue warp
+            mbar_init(&tempty[b], PAIR ? 2 * EPI : EPI);   // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -244,9 +269,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
         tma_prefetch_desc(&tmB);
     }
     for (int i = threadIdx.x; i < 2 * 2 * 128; i += blockDim.x) xflag[i] = 0;
-    if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+    if (warp == 1) {
+        if constexpr (PAIR) tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        else tmem_alloc(tmem_slot, TMEM_COLS);
+    }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -256,21 +285,53 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
     int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + S::TMAP_OFF);
     const int32_t* s_off = s_tptr + TMAP_STRIDE;
     stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
+    int32_t* s_pptr = reinterpret_cast<int32_t*>(smem + S::PPTR_OFF);
+    if constexpr (PAIR) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // m-pairs per expert, prefix over experts (E <= 256 steps, once per CTA)
+            int acc_p = 0;
+            for (int i = 0; i < p.E; i++) {
+                s_pptr[i] = acc_p;
+                acc_p += (s_tptr[i + 1] - s_tptr[i] + 1) >> 1;
+            }
+            s_pptr[p.E] = acc_p;
+        }
+    }
     __syncthreads();
     const int ntm = *p.num_tiles;
-    const int total = ntm * n_blocks;
+    const int total = PAIR ? s_pptr[p.E] * n_blocks : ntm * n_blocks;
     const long long limit = p.spin_limit;
+    // CTA pairs walk the units by cluster; single CTAs by block
+    const int t_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int t_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    // this CTA's m-tile of unit t: (expert, global m-tile index, has rows)
+    auto unit_tile = [&](int t, int& e, int& mi, int& nb, bool& has_rows) {
+        if constexpr (PAIR) {
+            int mp;
+            decode_pair(t, s_pptr, p.E, n_blocks, e, mp, nb);
+            const int local = 2 * mp + static_cast<int>(rank);
+            has_rows = local < s_tptr[e + 1] - s_tptr[e];
+            mi = s_tptr[e] + local;
+        } else {
+            decode_tile(t, s_tptr, p.E, n_blocks, e, mi, nb);
+            has_rows = true;
+        }
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = t_first; t < total && ok; t += t_step) {
                 int e, mi, nb;
-                decode_tile(t, s_tptr, p.E, n_blocks, e, mi, nb);
-                const int row0 = s_off[e] + GEMM_BM * (mi - s_tptr[e]);
-                const int brow = e * p.b_rows + nb * BN;
+                bool has_rows;
+                unit_tile(t, e, mi, nb, has_rows);
+                // a pair's rank 1 without an m-tile (odd count) loads rank 0's rows,
+                // so its A stays inside the tensor; its accumulator rows are not stored
+                const int row0 = s_off[e] + GEMM_BM * (mi - (has_rows ? 0 : 1) - s_tptr[e]);
+                const int brow = e * p.b_rows + nb * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
                 const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
                     const int s = it % STAGES;
@@ -280,23 +341,36 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         break;
                     }
                     uint8_t* sa = smem + s * S::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
-                    tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                    if constexpr (PAIR) {
+                        // both CTAs' halves complete on rank 0's barrier
+                        const uint32_t fb = cluster_addr(&full[s], 0);
+                        mbar_arrive_expect_tx_cluster(fb, S::STAGE_BYTES);
+                        tma_load_2d_pair(sa, &tmA, fb, kb * GEMM_BK, row0, l2_policy(false));
+                        tma_load_2d_pair(sa + GEMM_A_BYTES, &tmB, fb, kb * GEMM_BK, brow, pol);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+                        tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
+                        tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                    }
                     if (PROMOTE) KTRACE_BLK(it, 7);
                 }
             }
-            // loads still in flight land before the CTA may exit
-            const uint32_t first = it > STAGES ? it - STAGES : 0;
-            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, DRAIN_LIMIT);
+            // loads still in flight land before the CTA may exit (for a pair, rank
+            // 0's barriers count both CTAs' loads, and the closing cluster barrier
+            // keeps rank 1 until rank 0 is past this)
+            if (!PAIR || rank == 0) {
+                const uint32_t first = it > STAGES ? it - STAGES : 0;
+                for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, DRAIN_LIMIT);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_e4m3(GEMM_BM, BN);
+        if (lane == 0 && (!PAIR || rank == 0)) {
+            // a pair's MMA covers both CTAs' 128 rows (M = 256)
+            constexpr uint32_t idesc = idesc_e4m3(PAIR ? 2 * GEMM_BM : GEMM_BM, BN);
             uint32_t it = 0, u = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = t_first; t < total && ok; t += t_step) {
                 uint32_t acc = 0;
                 if (!PROMOTE) {
                     acc = u % NBUF;
@@ -317,11 +391,19 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     const uint32_t a_addr = smem_u32(smem + s * S::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + GEMM_A_BYTES;
                     const uint32_t d = tmem_base + acc * BN;
+                    if constexpr (PAIR) {
 #pragma unroll
-                    for (int kk = 0; kk < GEMM_BK / 32; kk++)
-                        mma_f8(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
-                               PROMOTE ? (kk > 0) : (kb > 0 || kk > 0));
-                    mma_commit(&empty[s]);
+                        for (int kk = 0; kk < GEMM_BK / 32; kk++)
+                            mma_f8_pair(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
+                                        kb > 0 || kk > 0);
+                        mma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < GEMM_BK / 32; kk++)
+                            mma_f8(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
+                                   PROMOTE ? (kk > 0) : (kb > 0 || kk > 0));
+                        mma_commit(&empty[s]);
+                    }
                     if (PROMOTE) {
                         mma_commit(&tfull[acc]);
                         KTRACE_BLK(u, 2);
@@ -330,12 +412,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                 }
                 if (!ok) break;
                 if (!PROMOTE) {
-                    mma_commit(&tfull[acc]);
+                    if constexpr (PAIR) mma_commit_pair_both(&tfull[acc]);   // both CTAs' epilogues
+                    else mma_commit(&tfull[acc]);
                     u++;
                 }
             }
             if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
-            mma_commit(drain);                 // every issued MMA has completed ...
+            if constexpr (PAIR) mma_commit_pair(drain);   // every issued MMA has completed ...
+            else mma_commit(drain);
             mbar_wait(drain, 0, DRAIN_LIMIT);        // ... before TMEM can be released
         }
     } else {
@@ -347,18 +431,25 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
         const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
         uint32_t u = 0, iter = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, iter++) {
+        // the accumulator is free again: a pair's MMA thread (rank 0) counts both
+        // CTAs' epilogue warps
+        auto release_acc = [&](uint64_t* bar) {
+            if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(bar, 0));
+            else mbar_arrive(bar);
+        };
+        for (int t = t_first; t < total && ok; t += t_step, iter++) {
             int e, mi, nb;
-            decode_tile(t, s_tptr, p.E, n_blocks, e, mi, nb);
+            bool has_rows;
+            unit_tile(t, e, mi, nb, has_rows);
             const int row0 = s_off[e] + GEMM_BM * (mi - s_tptr[e]);
             const int row = row0 + r;
-            const bool valid = row < s_off[e + 1];
+            const bool valid = row < s_off[e + 1];   // none for a pair's absent m-tile
 
             // FP8_ROW gate/up: this warp's part of the tile is stored; publish it
             // (per-lane release, then one count per warp) for the chained down GEMM
             auto publish = [&]() {
                 if constexpr (KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW) {
-                    if (p.gu_done != nullptr) {
+                    if (p.gu_done != nullptr && has_rows) {
                         fence_proxy_async_global();
                         __threadfence();
                         __syncwarp();
@@ -388,7 +479,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         // none of this warp's rows is stored: release the buffer only
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty[acc]);
+                        if (lane == 0) release_acc(&tempty[acc]);
                         u++;
                         publish();
                         continue;
@@ -410,7 +501,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                             if (half == NH - 1) {
                                 tc_fence_before();
                                 __syncwarp();
-                                if (lane == 0) mbar_arrive(&tempty[acc]);
+                                if (lane == 0) release_acc(&tempty[acc]);
                             }
                             // first hidden column of this 32-block (ReLU^2: the gate-half
                             // columns are up rows 256 nb + c0, the up half 256 nb + 128 + c0)
@@ -476,7 +567,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[acc]);
+                    if (lane == 0) release_acc(&tempty[acc]);
                     u++;
                 } else {
                     float ag[64], au[64];
@@ -513,7 +604,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         if (ew == 0 && lane == 0) KTRACE_BLK(u, 4);
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty[acc]);
+                        if (lane == 0) release_acc(&tempty[acc]);
                         if (ew == 0 && lane == 0) KTRACE_BLK(u, 5);
                         if (ew == EPI - 1 && lane == 0) KTRACE_BLK(u, 6);
                         u++;
@@ -656,7 +747,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[acc]);
+                    if (lane == 0) release_acc(&tempty[acc]);
                     u++;
                 }
                 if (!ok) break;
@@ -671,9 +762,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 
     tc_fence_before();
     __syncthreads();
+    // a pair leaves together: no arrival or copy may target a CTA that has exited
+    if constexpr (PAIR) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
@@ -683,6 +777,17 @@ __global__ void __launch_bounds__(gemm_threads<EPI>(), 1)
                         const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     gemm_body<KIND, BSCALE, PROMOTE, BN, STAGES, EPI, ACT>(tmA, tmB, p, p.n_blocks, smem_raw);
+}
+
+// FP8_ROW gate/up on CTA pairs (launched as 2-CTA clusters)
+constexpr int GU_PAIR_STAGES = 6;
+template <int ACT>
+__global__ void __launch_bounds__(gemm_threads<16>(), 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 256, GU_PAIR_STAGES, 16, ACT, true>(tmA, tmB, p, p.n_blocks,
+                                                                                   smem_raw);
 }
 
 // Down GEMM whose tile width is chosen on the device: the dispatch's scan

@@ -67,6 +67,28 @@ static cudaError_t launch_k(bool pdl, void (*kern)(KP...), dim3 grid, dim3 block
     return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
 }
 
+// the same for a grid of 2-CTA clusters (CTA pairs)
+template <typename... KP, typename... Args>
+static cudaError_t launch_k_pairs(bool pdl, void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                  Args&&... args) {
+    cudaLaunchConfig_t lc;
+    memset(&lc, 0, sizeof(lc));
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 2;
+    return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+}
+
 #define LAUNCH(pdl, name, kern, grid, block, smem, st, ...)                                  \
     do {                                                                                     \
         cudaError_t err_ = launch_k((pdl), kern, dim3(grid), dim3(block), (smem), (st), __VA_ARGS__); \
@@ -92,6 +114,7 @@ struct moe_handle {
     WLayout wl;
     long long spin_limit;
     int down_bn;          // 0 = picked per call, else 64 / 128 / 256
+    int gemm_pairs;       // large FP8_ROW batches run the gate/up GEMM on CTA pairs
     PickerParams picker;
     int pdl;              // launch with programmatic dependent launch allowed
 };
@@ -238,6 +261,7 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
     h->picker.gamma_ps = 17030139;
     h->picker.num_sms = h->num_sms;
     h->pdl = 1;
+    h->gemm_pairs = 1;
     h->picker.H = c.H;
     h->picker.I = c.I;
     h->picker.split_nb = c.fmt == MOE_FMT_FP8_ROW ? c.H / MX_BN : 0;
@@ -612,6 +636,20 @@ static moe_status launch_gemm(bool pdl, const CUtensorMap& ta, const CUtensorMap
     return MOE_OK;
 }
 
+// FP8_ROW gate/up on CTA pairs: M = 256 MMAs over two m-tiles of one expert,
+// each CTA loading its 128 A rows and half of the B tile (32 KB stages, 6 deep)
+template <int ACT>
+static moe_status launch_gemm_pairs(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                                    int grid, cudaStream_t st) {
+    using S = GemmSmem<256, GU_PAIR_STAGES, 16, true>;
+    static_assert(S::TOTAL <= 232448, "shared memory of the GEMM exceeds 227 KB");
+    auto kern = grouped_gemm_pair_kernel<ACT>;
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL));
+    const cudaError_t err = launch_k_pairs(pdl, kern, dim3(grid), dim3(gemm_threads<16>()), S::TOTAL, st, ta, tb, p);
+    if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "launch of grouped_gemm_pair_kernel failed: %s", cudaGetErrorString(err));
+    return MOE_OK;
+}
+
 // upper bound of the m-tiles the schedule can hold for T tokens
 static int max_m_tiles(const moe_config& c, int T) {
     const int A = T * c.k;
@@ -634,7 +672,10 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     moe_status r = make_tmap(&ta, v.xq, c.H, padded_rows(c), c.H, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
     const int n_gu = c.act == MOE_ACT_RELU2 ? c.I : 2 * c.I;   // rows of the packed gate/up weights
-    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, 256);
+    // CTA pairs: each CTA loads half of a B tile's 256 rows
+    const bool pairs = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU && h->gemm_pairs &&
+                       static_cast<long long>(T) * c.k >= 4LL * TILE_M * c.E;
+    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, pairs ? 128 : 256);
     if (r != MOE_OK) return r;
     GemmParams p;
     memset(&p, 0, sizeof(p));
@@ -662,6 +703,12 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (pairs) {
+        // large batches (>= 4 m-tiles per expert on average): CTA pairs, so an odd
+        // m-tile count leaves at most one half-empty pair per expert
+        const int pairs = std::max(1, std::min(h->num_sms / 2, (max_m_tiles(c, T) + 1) / 2 * p.n_blocks));
+        return launch_gemm_pairs<MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, 2 * pairs, st);
+    }
     if (c.fmt == MOE_FMT_FP8_ROW) {
         switch (c.act) {
         case MOE_ACT_SWIGLU_BOUNDED:
@@ -840,6 +887,14 @@ extern "C" moe_status moe_set_launch_options(moe_handle* h, int pdl) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_launch_options: null handle");
     if (pdl != 0 && pdl != 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_launch_options: pdl must be 0 or 1 (got %d)", pdl);
     h->pdl = pdl;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_set_gemm_options(moe_handle* h, int cta_pairs) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: null handle");
+    if (cta_pairs != 0 && cta_pairs != 1)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: cta_pairs must be 0 or 1 (got %d)", cta_pairs);
+    h->gemm_pairs = cta_pairs;
     return MOE_OK;
 }
 

@@ -22,7 +22,7 @@ EXPORTED = (
     "moe_last_error", "moe_init", "moe_destroy", "moe_weights_size", "moe_workspace_size",
     "moe_workspace_view_get", "moe_pack_weights", "moe_route", "moe_dispatch", "moe_gate_up",
     "moe_down", "moe_combine", "moe_forward", "moe_forward_routed", "moe_workspace_init",
-    "moe_get_status", "moe_dispatch_noalloc", "moe_set_tile_config", "moe_set_launch_options", "moe_set_wait_limit", "moe_set_picker_params",
+    "moe_get_status", "moe_dispatch_noalloc", "moe_set_tile_config", "moe_set_launch_options", "moe_set_gemm_options", "moe_set_wait_limit", "moe_set_picker_params",
     "moe_get_picker_params",
 )
 
@@ -85,6 +85,7 @@ def load(path=LIB_PATH):
             "moe_dispatch_noalloc": (I, [P, P, P, I] + [P] * 10),
             "moe_set_tile_config": (I, [P, I]),
             "moe_set_launch_options": (I, [P, I]),
+            "moe_set_gemm_options": (I, [P, I]),
             "moe_set_wait_limit": (I, [P, ctypes.c_longlong]),
             "moe_set_picker_params": (I, [P, P]),
             "moe_get_picker_params": (I, [P, P]),
@@ -195,6 +196,10 @@ def moe_set_tile_config(h, down_bn):
 
 def moe_set_launch_options(h, pdl):
     _check(load().moe_set_launch_options(h, int(pdl)))
+
+
+def moe_set_gemm_options(h, cta_pairs):
+    _check(load().moe_set_gemm_options(h, int(cta_pairs)))
 
 
 def moe_set_wait_limit(h, cycles):

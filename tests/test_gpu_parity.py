@@ -26,6 +26,8 @@ CASES = {
     "block128-ragged": (W.custom(H=512, I=384, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 300),
     "t1": (W.custom(H=256, I=128, E=8, k=2), 1),
     "row-split-t3": (W.custom(H=512, I=2048, E=8, k=2), 3),
+    # T k >= 512 E: the gate/up GEMM runs on CTA pairs (odd row-tile counts included)
+    "row-pairs-t2100": (W.custom(H=512, I=256, E=8, k=2), 2100),
     # above 4 x 148 tokens the quantisation runs one warp per token
     "row-t700": (W.custom(H=256, I=128, E=8, k=2), 700),
     "block128-t700": (W.custom(H=256, I=128, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 700),
@@ -360,7 +362,7 @@ def test_forward_twice_same_bits():
     assert torch.equal(y1, y2)
 
 
-@pytest.mark.parametrize("name", ["row-skew-e64", "block128-ragged", "nvfp4-ragged"])
+@pytest.mark.parametrize("name", ["row-skew-e64", "row-pairs-t2100", "block128-ragged", "nvfp4-ragged"])
 def test_launch_modes_same_bits(name):
     """Programmatic dependent launch on or off, direct calls or a replayed CUDA
     graph of the call: the same kernels on the same data give the same bits."""
@@ -384,6 +386,27 @@ def test_launch_modes_same_bits(name):
     assert torch.equal(y_plain, y_pdl)
     assert torch.equal(y_plain, y)
     del g
+
+
+def test_cta_pairs_match_single_ctas():
+    """The gate/up GEMM on CTA pairs (M = 256 MMAs over two row tiles) gives the
+    hidden codes and the layer output of the single-CTA kernel, up to the fp32
+    summation order inside the tensor core."""
+    wl, T, d, x = build_case("row-pairs-t2100")
+    layer = native.Layer(wl, d, max_T=T)
+    xc, wr = x.cuda(), d["wr"].cuda()
+    native.moe_set_gemm_options(layer.h, 1)
+    y_pair = layer.forward(xc, wr, None).clone()
+    hq_pair = layer.region("hq", torch.uint8, (T * wl.k + 128 * wl.E) * wl.I).clone()
+    native.moe_set_gemm_options(layer.h, 0)
+    y_single = layer.forward(xc, wr, None).clone()
+    hq_single = layer.region("hq", torch.uint8, (T * wl.k + 128 * wl.E) * wl.I).clone()
+    torch.cuda.synchronize()
+    assert layer.status()[0] == 0
+    assert (hq_pair != hq_single).float().mean().item() <= 1e-3
+    assert tolerance_violations(y_pair.float().cpu().numpy(), y_single.float().cpu().numpy()) == 0
+    with pytest.raises(native.MoeError):
+        native.moe_set_gemm_options(layer.h, 2)
 
 
 def test_empty_batch():
