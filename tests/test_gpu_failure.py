@@ -18,6 +18,8 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 
 CASES = {
     "fp8-row": W.custom(H=512, I=256, E=8, k=2),
+    # T k >= 512 E: the gate/up GEMM on CTA pairs (waits on the other CTA's copies)
+    "fp8-row-pairs": W.custom(H=512, I=256, E=8, k=2),
     "fp8-block128": W.custom(H=512, I=256, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128),
     "nvfp4": W.custom(H=512, I=256, E=8, k=2, fmt=W.FMT_NVFP4),
 }
@@ -33,7 +35,7 @@ def _lib():
 @pytest.mark.parametrize("name", list(CASES))
 def test_wait_timeout_is_reported_and_the_context_stays_usable(name):
     wl = CASES[name]
-    T = 200
+    T = 2100 if name.endswith("pairs") else 200
     d = synth.layer(wl, seed=5)
     layer = native.Layer(wl, d, max_T=T)
     x, wr = synth.tokens(wl, T, seed=5).cuda(), d["wr"].cuda()
