@@ -256,8 +256,10 @@ moe_status moe_set_wait_limit(moe_handle* h, long long cycles);
  * and writes the cheapest (the wider on ties) to view.pick[0].
  * For FP8_ROW it also writes view.pick[1] = S, the K split of the down GEMM
  * (no parameters): with units = m_tiles * (H/256), A = T*k and
- * s_max = min(8, o_rows / A, (I/128) / 4), S is the largest s <= s_max with
- * units * s <= num_sms, else 1 (o_rows = A_max + 7 min(A_max, 256)).
+ * s_max = min(8, o_rows / A, (I/128) / 4) and
+ * cost(s) = ceil(units*s / num_sms) * 840/s, S is the s <= s_max of lowest
+ * cost (the smaller on ties) when that cost is at most 4/5 of cost(1), else 1
+ * (o_rows = A_max + 7 min(A_max, 256)).
  * params = {alpha, beta, bw, gamma}; get also returns num_sms in params[4]. */
 moe_status moe_set_picker_params(moe_handle* h, const long long* params);
 moe_status moe_get_picker_params(const moe_handle* h, long long* params);

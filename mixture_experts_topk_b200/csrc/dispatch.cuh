@@ -45,7 +45,9 @@ struct PickerParams {
 // run by different CTAs, whose fp32 partial rows go to S copies of the output
 // rows that the combine adds in fixed order.  Integer rule:
 //   units = m_tiles * split_nb,  s_max = min(8, o_rows / A, split_kb / 4)
-//   S = the largest s <= s_max with units * s <= num_sms, else 1.
+//   cost(s) = ceil(units s / num_sms) * 840 / s   (rounds of 1/s of a unit)
+//   S = the s <= s_max of lowest cost (the smaller on ties) if that cost is at
+//   most 4/5 of cost(1), else 1 (a split also costs copies of the output).
 __host__ __device__ inline int split_limit(const PickerParams& q, int A) {
     if (q.split_nb <= 0 || A <= 0) return 1;
     int m = q.o_rows / A;
@@ -56,8 +58,16 @@ __host__ __device__ inline int split_limit(const PickerParams& q, int A) {
 __host__ __device__ inline int pick_split(const PickerParams& q, int m_tiles, int A) {
     const int smax = split_limit(q, A);
     const long long units = static_cast<long long>(m_tiles) * q.split_nb;
+    const long long c1 = (units + q.num_sms - 1) / q.num_sms * 840;
     int S = 1;
-    while (S < smax && units * (S + 1) <= q.num_sms) S++;
+    long long best = c1;
+    for (int s = 2; s <= smax; s++) {
+        const long long c = (units * s + q.num_sms - 1) / q.num_sms * (840 / s);
+        if (c < best && 5 * c <= 4 * c1) {
+            S = s;
+            best = c;
+        }
+    }
     return S;
 }
 constexpr int PICK_NUM = 3;

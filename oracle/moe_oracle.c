@@ -250,9 +250,20 @@ int orc_pick_split(const int32_t* counts, int E, int split_nb, int split_kb, int
     int64_t smax = 8;
     if (o_rows / A < smax) smax = o_rows / A;
     if (split_kb / 4 < smax) smax = split_kb / 4;
+    /* cost(s) = ceil(units s / num_sms) 840 / s: rounds of 1/s of a unit, in
+       840ths (840 is a multiple of 1..8); the cheapest s wins (the smaller on
+       ties), if it is at least 20% cheaper than no split */
+    const int64_t units = m_tiles * split_nb;
+    const int64_t c1 = (units + num_sms - 1) / num_sms * 840;
     int best = 1;
-    for (int64_t s = 2; s <= smax; s++)
-        if (m_tiles * split_nb * s <= num_sms) best = (int)s;
+    int64_t best_cost = c1;
+    for (int64_t s = 2; s <= smax; s++) {
+        const int64_t c = (units * s + num_sms - 1) / num_sms * (840 / s);
+        if (c < best_cost && 5 * c <= 4 * c1) {
+            best = (int)s;
+            best_cost = c;
+        }
+    }
     return best;
 }
 

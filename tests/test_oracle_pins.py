@@ -271,11 +271,19 @@ def test_pick_split_hand_examples():
     assert oracle.pick_split(np.int32([5, 0, 0, 0, 0, 0, 0, 0]), **mix) == 3
     # at least four K-blocks per range: split_kb 8 -> s_max 2
     assert oracle.pick_split(counts, **dict(mix, split_kb=8)) == 2
-    # units filling the SMs: 148 units -> no split; 75 units -> 150 > 148 -> no split; 74 -> 2
+    # units filling the SMs: 148 units -> every s costs a full unit round (840),
+    # no split; 75 units -> rounds of 1/s for s = 2..8: 2, 2, 3, 3, 4, 4, 5, so
+    # costs 840, 560, 630, 504, 560, 480, 525 -> 7; 74 -> 2 (one round of halves)
     many = dict(split_nb=1, split_kb=112, o_rows=10 ** 6, num_sms=148)
     assert oracle.pick_split(np.full(148, 1, np.int32), **many) == 1
-    assert oracle.pick_split(np.full(75, 1, np.int32), **many) == 1
+    assert oracle.pick_split(np.full(75, 1, np.int32), **many) == 7
     assert oracle.pick_split(np.full(74, 1, np.int32), **many) == 2
+    # 208 units (Mixtral-8x7B T = 512: 13 m-tiles x 16) with s_max 2: 2 rounds
+    # (1680) against 3 rounds of halves (1260 <= 1344) -> 2; 128 units with
+    # s_max 8: the best, s = 8 at 7 rounds of eighths (735), saves under a
+    # fifth of one round (840) -> no split
+    assert oracle.pick_split(np.full(208, 1, np.int32), **dict(many, o_rows=416)) == 2
+    assert oracle.pick_split(np.full(128, 1, np.int32), **dict(many, o_rows=1024)) == 1
     # a 129-row expert is two m-tiles
     assert oracle.pick_split(np.int32([129]), **dict(many, num_sms=4)) == 2
     # no split for formats without one, nor for an empty batch
