@@ -453,13 +453,13 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
         CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<32, 8, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       RT::SMEM));
         auto kern = router_logits_kernel<32, 8, 4>;
-        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 31) / 32, 1), RT_WARPS * 32, RT::SMEM, st, p);
+        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 31) / 32, 1), RT::NT, RT::SMEM, st, p);
     } else {
         using RT = RouterTile<64, 16, 16>;
         CUDA_TRY(cudaFuncSetAttribute(router_logits_kernel<64, 16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       RT::SMEM));
         auto kern = router_logits_kernel<64, 16, 16>;
-        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 63) / 64, (h->cfg.E + 15) / 16), RT_WARPS * 32,
+        LAUNCH(h->pdl, "router_logits_kernel", kern, dim3((T + 63) / 64, (h->cfg.E + 15) / 16), RT::NT,
                RT::SMEM, st, p);
     }
     LAUNCH(h->pdl, "router_topk_kernel", router_topk_kernel, std::min((T + 7) / 8, 16 * h->num_sms), 256, 0, st, p);
@@ -752,10 +752,13 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, to;
     moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
     r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, MX_BN);
+    if (r != MOE_OK) return r;
+    // output rows (fp32 as bytes): boxes of 32 rows x 32 values for the epilogue's stores
+    r = make_tmap(&to, v.o, static_cast<uint64_t>(c.H) * 4, o_rows(c), static_cast<uint64_t>(c.H) * 4, 128, 32);
     if (r != MOE_OK) return r;
     MxDownParams p;
     memset(&p, 0, sizeof(p));
@@ -782,9 +785,17 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks * p.s_max));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    CUDA_TRY(cudaFuncSetAttribute(grouped_gemm_mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MX_SMEM));
-    LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", grouped_gemm_mx_down_kernel, grid, GEMM_THREADS, MX_SMEM, st, ta,
-           tb, p);
+    if (p.num_kb <= MX_BOX_MAX_KB) {
+        using Lb = MxSmem<3, true>;
+        auto kern = grouped_gemm_mx_down_kernel<3, true>;
+        CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lb::TOTAL));
+        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Lb::TOTAL, st, ta, tb, to, p);
+    } else {
+        using Lr = MxSmem<4, false>;
+        auto kern = grouped_gemm_mx_down_kernel<4, false>;
+        CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lr::TOTAL));
+        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Lr::TOTAL, st, ta, tb, to, p);
+    }
     return MOE_OK;
 }
 

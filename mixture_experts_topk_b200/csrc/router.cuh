@@ -15,9 +15,10 @@
 //                        with 16-token x 8-expert micro-tiles, or 32 x 8 with
 //                        4 x 8 micro-tiles when E <= 8).
 //                        The 256-wide H chunks of X and Wr go through shared
-//                        memory with a 4-stage cp.async pipeline; each of the 8
-//                        warps owns one micro-tile: per 16 bytes read from
-//                        shared memory, 8 x 8 runs 43 fma and 16 x 8 64.
+//                        memory with a 4-stage cp.async pipeline; each warp
+//                        owns one micro-tile: per 16 bytes read from
+//                        shared memory, 16 x 8 runs 64 fma; two tokens' chains
+//                        share each packed fp32 fma (fma.rn.f32x2).
 //  router_logits_small_kernel  batches of at most 128 tokens: one warp per
 //                        (expert, 4 tokens) reading global memory directly.
 //  router_small_fused_kernel   the same for at most 32 experts, with the top-k
@@ -29,11 +30,12 @@
 
 namespace moe {
 
-constexpr int RT_WARPS = 8;   // (TOK / MT) x (EXP / 8) micro-tiles of MT tokens x 8 experts
-
-template <int TOK, int EXP, int MT = 8>
+// A CTA tile of TOK tokens x EXP experts: one warp per micro-tile of MT
+// tokens x 8 experts.
+template <int TOK, int EXP, int MT>
 struct RouterTile {
-    static_assert((TOK / MT) * (EXP / 8) == RT_WARPS, "one micro-tile per warp");
+    static constexpr int NW = (TOK / MT) * (EXP / 8);
+    static constexpr int NT = 32 * NW;
     static constexpr int X_BYTES = TOK * 256 * 2;    // 256 bf16 of H per token
     static constexpr int W_BYTES = EXP * 256 * 4;    // 256 fp32 of H per expert
     static constexpr int STAGE = X_BYTES + W_BYTES;
@@ -68,15 +70,17 @@ __device__ __forceinline__ void cp_async_wait_le(int n) {
     else asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// The 16-byte pieces one thread copies for every H chunk: X piece m is row
-// (tid / 32) + 8 m, column 8 (tid % 32); Wr piece m is row (tid / 64) + 4 m,
-// column 4 (tid % 64).  Base pointers and validity are fixed per thread, so a
-// chunk costs one add and one cp.async per piece.  Rows past T or E read
-// nothing and are zero-filled.
-template <int TOK, int EXP>
+// The 16-byte pieces one of the NT threads copies for every H chunk: X piece
+// m is row (tid / 32) + (NT / 32) m, column 8 (tid % 32); Wr piece m is row
+// (tid / 64) + (NT / 64) m, column 4 (tid % 64).  Base pointers and validity
+// are fixed per thread, so a chunk costs one add and one cp.async per piece.
+// Rows past T or E read nothing and are zero-filled.
+template <int TOK, int EXP, int NT>
 struct RouterLoader {
-    static constexpr int XP = TOK * 32 / (RT_WARPS * 32);   // X pieces per thread
-    static constexpr int WP = EXP * 64 / (RT_WARPS * 32);   // Wr pieces per thread
+    static constexpr int XR = NT / 32, WR = NT / 64;   // rows per pass
+    static constexpr int XP = TOK / XR;                // X pieces per thread
+    static constexpr int WP = EXP / WR;                // Wr pieces per thread
+    static_assert(XP * XR == TOK && WP * WR == EXP, "whole passes");
     const __nv_bfloat16* xb;
     const float* wb;
     uint32_t xvalid, wvalid;   // bit m: piece m is inside the tensor
@@ -90,9 +94,9 @@ struct RouterLoader {
         const int xr = tid >> 5, xc = tid & 31;
         const int wr = tid >> 6, wc = tid & 63;
 #pragma unroll
-        for (int m = 0; m < XP; m++) xvalid |= (t0 + xr + 8 * m < p.T ? 1u : 0u) << m;
+        for (int m = 0; m < XP; m++) xvalid |= (t0 + xr + XR * m < p.T ? 1u : 0u) << m;
 #pragma unroll
-        for (int m = 0; m < WP; m++) wvalid |= (e0 + wr + 4 * m < p.E ? 1u : 0u) << m;
+        for (int m = 0; m < WP; m++) wvalid |= (e0 + wr + WR * m < p.E ? 1u : 0u) << m;
         xb = p.x + static_cast<size_t>(xvalid & 1u ? t0 + xr : 0) * p.H + 8 * xc;
         wb = p.wr + static_cast<size_t>(wvalid & 1u ? e0 + wr : 0) * p.H + 4 * wc;
         xdst = xr * 512 + xc * 16;
@@ -105,12 +109,12 @@ struct RouterLoader {
 #pragma unroll
         for (int m = 0; m < XP; m++) {
             const bool ok = (xvalid >> m) & 1u;
-            cp_async16(st + xdst + m * 8 * 512, ok ? xb + static_cast<size_t>(8 * m) * H + 256 * i : xb, ok);
+            cp_async16(st + xdst + m * XR * 512, ok ? xb + static_cast<size_t>(XR * m) * H + 256 * i : xb, ok);
         }
 #pragma unroll
         for (int m = 0; m < WP; m++) {
             const bool ok = (wvalid >> m) & 1u;
-            cp_async16(st + wdst + m * 4 * 1024, ok ? wb + static_cast<size_t>(4 * m) * H + 256 * i : wb, ok);
+            cp_async16(st + wdst + m * WR * 1024, ok ? wb + static_cast<size_t>(WR * m) * H + 256 * i : wb, ok);
         }
         cp_async_commit();
     }
@@ -129,8 +133,17 @@ __device__ __forceinline__ void butterfly_halve(const float* in, float* out, int
     }
 }
 
-template <int TOK, int EXP, int MT = 8>
-__global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterParams p) {
+// d0 = fma(a0, b, d0), d1 = fma(a1, b, d1), each rounded to nearest (one
+// packed sm_100 instruction for two independent chains).
+__device__ __forceinline__ void fma2_rn(float& d0, float& d1, float a0, float a1, float b) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rd, {%0, %1};\n\tfma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b));
+}
+
+template <int TOK, int EXP, int MT>
+__global__ void __launch_bounds__(RouterTile<TOK, EXP, MT>::NT, 1) router_logits_kernel(RouterParams p) {
     pdl_wait();
     pdl_trigger();
     KTRACE(TR_ROUTER);
@@ -147,7 +160,7 @@ __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterPara
 #pragma unroll
         for (int b = 0; b < 8; b++) acc[a][b] = 0.0f;
 
-    const RouterLoader<TOK, EXP> ld(p, t0, e0);
+    const RouterLoader<TOK, EXP, RT::NT> ld(p, t0, e0);
     // prologue: chunks 0 .. NSTAGE-2 in flight
     for (int c = 0; c < RT::NSTAGE - 1 && c < nI; c++) ld.load(rsm + c * RT::STAGE, c);
     for (int i = 0; i < nI; i++) {
@@ -159,63 +172,35 @@ __global__ void __launch_bounds__(RT_WARPS * 32) router_logits_kernel(RouterPara
         __syncthreads();
         const uint8_t* xs = st + (MT * tg) * 512 + lane * 16;
         const uint8_t* ws = st + RT::X_BYTES + (8 * eg) * 1024 + lane * 16;
-        if constexpr (MT == 8) {
-            // The warp's 8 experts x 8 values and 8 tokens x 8 values of this chunk
-            // sit in registers; for each j the 64 accumulators take one fma each,
-            // so consecutive fma are independent.  Each (token, expert) chain
-            // still runs j = 0..7 in order.
-            float wv[8][8];
+        // MT tokens x 8 experts: the lane's 8 values per row go in two halves
+        // (j = 0..3, then 4..7), so each chain still runs j in order.  Tokens
+        // 2 tp and 2 tp + 1 share one packed fma per (expert, j): two
+        // independent round-to-nearest fp32 fma, the same as two scalar ones.
+        static_assert(MT % 2 == 0, "token pairs");
+#pragma unroll
+        for (int jh = 0; jh < 2; jh++) {
+            float wv[8][4];
 #pragma unroll
             for (int ee = 0; ee < 8; ee++) {
-                const float4 wa = *reinterpret_cast<const float4*>(ws + ee * 1024);
-                const float4 wb = *reinterpret_cast<const float4*>(ws + ee * 1024 + 512);
-                wv[ee][0] = wa.x; wv[ee][1] = wa.y; wv[ee][2] = wa.z; wv[ee][3] = wa.w;
-                wv[ee][4] = wb.x; wv[ee][5] = wb.y; wv[ee][6] = wb.z; wv[ee][7] = wb.w;
+                const float4 w4 = *reinterpret_cast<const float4*>(ws + ee * 1024 + jh * 512);
+                wv[ee][0] = w4.x; wv[ee][1] = w4.y; wv[ee][2] = w4.z; wv[ee][3] = w4.w;
             }
-            uint32_t xw[8][4];
+            uint32_t xw[MT][2];
 #pragma unroll
-            for (int tt = 0; tt < 8; tt++) {
-                const uint4 xv = *reinterpret_cast<const uint4*>(xs + tt * 512);
-                xw[tt][0] = xv.x; xw[tt][1] = xv.y; xw[tt][2] = xv.z; xw[tt][3] = xv.w;
+            for (int tt = 0; tt < MT; tt++) {
+                const uint2 x2 = *reinterpret_cast<const uint2*>(xs + tt * 512 + jh * 8);
+                xw[tt][0] = x2.x; xw[tt][1] = x2.y;
             }
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                float xj[8];
+            for (int j = 0; j < 4; j++) {
+                float xj[MT];
 #pragma unroll
-                for (int tt = 0; tt < 8; tt++) xj[tt] = (j & 1) ? bf16_hi(xw[tt][j >> 1]) : bf16_lo(xw[tt][j >> 1]);
+                for (int tt = 0; tt < MT; tt++) xj[tt] = (j & 1) ? bf16_hi(xw[tt][j >> 1]) : bf16_lo(xw[tt][j >> 1]);
 #pragma unroll
-                for (int tt = 0; tt < 8; tt++)
+                for (int tp = 0; tp < MT / 2; tp++)
 #pragma unroll
-                    for (int ee = 0; ee < 8; ee++) acc[tt][ee] = __fmaf_rn(xj[tt], wv[ee][j], acc[tt][ee]);
-            }
-        } else {
-            // 16 tokens x 8 experts: each shared-memory value feeds twice the fma
-            // of the 8 x 8 tile.  The lane's 8 values per row go in two halves
-            // (j = 0..3, then 4..7), so each chain still runs j in order.
-#pragma unroll
-            for (int jh = 0; jh < 2; jh++) {
-                float wv[8][4];
-#pragma unroll
-                for (int ee = 0; ee < 8; ee++) {
-                    const float4 w4 = *reinterpret_cast<const float4*>(ws + ee * 1024 + jh * 512);
-                    wv[ee][0] = w4.x; wv[ee][1] = w4.y; wv[ee][2] = w4.z; wv[ee][3] = w4.w;
-                }
-                uint32_t xw[MT][2];
-#pragma unroll
-                for (int tt = 0; tt < MT; tt++) {
-                    const uint2 x2 = *reinterpret_cast<const uint2*>(xs + tt * 512 + jh * 8);
-                    xw[tt][0] = x2.x; xw[tt][1] = x2.y;
-                }
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    float xj[MT];
-#pragma unroll
-                    for (int tt = 0; tt < MT; tt++) xj[tt] = (j & 1) ? bf16_hi(xw[tt][j >> 1]) : bf16_lo(xw[tt][j >> 1]);
-#pragma unroll
-                    for (int tt = 0; tt < MT; tt++)
-#pragma unroll
-                        for (int ee = 0; ee < 8; ee++) acc[tt][ee] = __fmaf_rn(xj[tt], wv[ee][j], acc[tt][ee]);
-                }
+                    for (int ee = 0; ee < 8; ee++)
+                        fma2_rn(acc[2 * tp][ee], acc[2 * tp + 1][ee], xj[2 * tp], xj[2 * tp + 1], wv[ee][j]);
             }
         }
         __syncthreads();   // the stage is refilled NSTAGE-1 chunks later

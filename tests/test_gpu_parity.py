@@ -26,6 +26,9 @@ CASES = {
     "block128-ragged": (W.custom(H=512, I=384, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 300),
     "t1": (W.custom(H=256, I=128, E=8, k=2), 1),
     "row-split-t3": (W.custom(H=512, I=2048, E=8, k=2), 3),
+    # K = 2048: the down GEMM stores full 32-row groups as TMA boxes, here with a
+    # 4-way K split (rows per expert 52, 44, 48, 48: one full group and a ragged one)
+    "row-split-boxes-t96": (W.custom(H=512, I=2048, E=4, k=2), 96),
     # T k >= 512 E: the gate/up GEMM runs on CTA pairs (odd row-tile counts included)
     "row-pairs-t2100": (W.custom(H=512, I=256, E=8, k=2), 2100),
     # above 4 x 148 tokens the quantisation runs one warp per token
@@ -362,7 +365,7 @@ def test_forward_twice_same_bits():
     assert torch.equal(y1, y2)
 
 
-@pytest.mark.parametrize("name", ["row-skew-e64", "row-pairs-t2100", "block128-ragged", "nvfp4-ragged"])
+@pytest.mark.parametrize("name", ["row-skew-e64", "row-pairs-t2100", "row-split-boxes-t96", "block128-ragged", "nvfp4-ragged"])
 def test_launch_modes_same_bits(name):
     """Programmatic dependent launch on or off, direct calls or a replayed CUDA
     graph of the call: the same kernels on the same data give the same bits."""
