@@ -86,6 +86,20 @@ constexpr int SPARSE_WARP_FLOATS = 8 * 64 + 8;
 // dst: this lane's row at its first column, null when the row is not stored.
 // Stored value: (v[c] * cs[c]) * rs with column scales, else v[c] * rs.
 // Warps with at most 8 stored rows store them directly (fewer steps).
+// TMA tensor store of one box from shared memory, and the bulk-group waits.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one store group of this thread still reading shared memory
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// all store groups of this thread complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 constexpr int STG_STRIDE = 20;
 constexpr int STG_WARP_FLOATS = 32 * STG_STRIDE;
 template <int NC, bool HAS_CS>

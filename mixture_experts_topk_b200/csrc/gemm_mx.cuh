@@ -57,20 +57,6 @@ struct MxSmem {
     static_assert(4 * STAGES <= 16, "A-scale ring below the B-scale chunks");
 };
 
-// TMA tensor store of one box from shared memory, and the bulk-group waits.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* src, int x, int y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(tm)),
-                 "r"(smem_u32(src)), "r"(x), "r"(y)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// at most one store group of this thread still reading shared memory
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// all store groups of this thread complete
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
 // Instruction descriptor of kind::mxf8f6f4 block-scaled: A, B E4M3 (0), K-major,
 // N >> 3 at [17,23), UE8M0 scales ([23] = 1), M >> 4 at [24,29), A scale id at
 // [29,31), B scale id at [4,6), dense K = 32.
