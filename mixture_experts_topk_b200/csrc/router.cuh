@@ -165,11 +165,14 @@ __global__ void __launch_bounds__(RouterTile<TOK, EXP, MT>::NT, 1) router_logits
     for (int c = 0; c < RT::NSTAGE - 1 && c < nI; c++) ld.load(rsm + c * RT::STAGE, c);
     for (int i = 0; i < nI; i++) {
         uint8_t* st = rsm + (i % RT::NSTAGE) * RT::STAGE;
+        // chunk i is complete once at most the groups issued after it (chunks
+        // i + 1 .. i + NSTAGE - 2) are pending
+        cp_async_wait_le(min(nI - 1 - i, RT::NSTAGE - 2));
+        // one barrier per chunk: chunk i is visible to every warp, and every
+        // warp is done with chunk i - 1, whose stage the next load refills
+        __syncthreads();
         const int ahead = i + RT::NSTAGE - 1;
         if (ahead < nI) ld.load(rsm + (ahead % RT::NSTAGE) * RT::STAGE, ahead);
-        // chunk i is complete once at most (issued after it) groups are pending
-        cp_async_wait_le(min(nI - 1 - i, RT::NSTAGE - 1));
-        __syncthreads();
         const uint8_t* xs = st + (MT * tg) * 512 + lane * 16;
         const uint8_t* ws = st + RT::X_BYTES + (8 * eg) * 1024 + lane * 16;
         // MT tokens x 8 experts: the lane's 8 values per row go in two halves
@@ -203,7 +206,6 @@ __global__ void __launch_bounds__(RouterTile<TOK, EXP, MT>::NT, 1) router_logits
                         fma2_rn(acc[2 * tp][ee], acc[2 * tp + 1][ee], xj[2 * tp], xj[2 * tp + 1], wv[ee][j]);
             }
         }
-        __syncthreads();   // the stage is refilled NSTAGE-1 chunks later
     }
     // Sum the 32 lane partials of all NV = 8 MT (token, expert) pairs by
     // recursive halving over lane offsets 1, 2, 4, 8, 16: at each step a lane
