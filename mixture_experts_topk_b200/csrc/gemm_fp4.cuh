@@ -8,14 +8,22 @@
 // requantisation of the hidden, the down projection and the routing weight.
 // Pure-Triton fused MoE article: gate and up share one input tile.
 //
-// Tile 128 rows x 128 columns (gate/up: 64 gate + 64 up columns of one 64-wide
-// hidden block), K stage 256 values = 128 bytes per row, 5 stages.  Per stage
-// the producer brings, on one mbarrier: A and B tiles by TMA (128-byte swizzle)
-// and the 2 KB of A and 2 KB of B scale factors (4 chunks of 512 B, one per
-// MMA of K = 64) by plain bulk copies.  The MMA thread copies the chunks into a
-// TMEM ring (tcgen05.cp, 32 rows x 16 B repeated over the 4 lane quadrants),
-// then issues the 4 block-scaled MMAs, which read them in issue order.
-// TMEM: two 128-column accumulators at [0, 256), scale-factor ring at 256 +.
+// Tiles of 128 rows (widths below), K stage 256 values = 128 bytes per row.
+// The packed gate/up weights hold blocks of 64 gate + 64 up rows, one 64-wide
+// hidden block each.  Per stage the producer brings, on one mbarrier: A and B tiles by
+// TMA (128-byte swizzle) and the 2 KB of A scale factors and 2 KB per 128 rows
+// of B scale factors (4 chunks of 512 B, one per MMA of K = 64) by plain bulk
+// copies.  The MMA thread copies the chunks into a TMEM ring (tcgen05.cp, 32
+// rows x 16 B repeated over the 4 lane quadrants), then issues the 4
+// block-scaled MMAs, which read them in issue order.
+//  - Down GEMM and ReLU^2 gate/up: 128-column tiles, two 128-column
+//    accumulators at [0, 256), 5 stages.
+//  - Gated gate/up: 256-column tiles (two consecutive 64 gate + 64 up blocks of
+//    the packed weights, 128 hidden columns), so each 128 x 256 x 256 step
+//    needs 54 KB of operands and scales instead of 2 x 36 KB, and A is read
+//    half as often.  One 256-column accumulator, released as soon as the
+//    epilogue holds it in registers; 4 stages.
+// The scale-factor ring starts at TMEM column 256.
 //
 // Rows are in the 128-padded expert-major layout (m-tile i = rows 128 i ..),
 // so each tile's scale factors are whole chunks.  The epilogue maps a padded
@@ -26,21 +34,37 @@
 
 namespace moe {
 
-constexpr int F4_BN = 128;
-constexpr int F4_STAGES = 5;
 constexpr int F4_A_BYTES = 128 * 128;
-constexpr int F4_B_BYTES = F4_BN * 128;
-constexpr int F4_SF_BYTES = 2048;                 // 4 chunks of 512 B
-constexpr int F4_STAGE_BYTES = F4_A_BYTES + F4_B_BYTES + 2 * F4_SF_BYTES;
-constexpr int F4_NBUF = 2;
-constexpr int F4_SF_TMEM = F4_NBUF * F4_BN;       // first column of the scale-factor ring
-constexpr int F4_BAR_OFF = F4_STAGES * F4_STAGE_BYTES;
-constexpr int F4_NUM_BARS = 2 * F4_STAGES + 2 * F4_NBUF + 1;
-constexpr int F4_TMEM_SLOT_OFF = F4_BAR_OFF + 8 * F4_NUM_BARS;
-constexpr int F4_TMAP_OFF = F4_TMEM_SLOT_OFF + 16;
-constexpr int F4_STG_OFF = (F4_TMAP_OFF + TMAP_BYTES + 15) / 16 * 16;   // down-store staging
-constexpr int F4_SMEM = F4_STG_OFF + 8 * STG_WARP_FLOATS * 4 + 1024;
-static_assert(F4_SF_TMEM + 32 * F4_STAGES <= 512, "TMEM columns");
+constexpr int F4_SF_BYTES = 2048;                 // 4 chunks of 512 B per 128 rows
+constexpr int F4_SF_TMEM = 256;                   // first column of the scale-factor ring
+
+// Shared memory and TMEM of one instantiation.  Narrow (down, ReLU^2 gate/up):
+// 128-column tiles, two accumulators, 5 stages.  Wide (gated gate/up): 256
+// columns (two 64 gate + 64 up blocks), one accumulator released as soon as
+// the epilogue has it in registers, 4 stages.
+template <bool WIDE>
+struct Fp4Smem {
+    static constexpr int BN = WIDE ? 256 : 128;
+    static constexpr int NBUF = WIDE ? 1 : 2;
+    static constexpr int STAGES = WIDE ? 4 : 5;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int SFB_BYTES = (BN / 128) * F4_SF_BYTES;
+    static constexpr int STAGE_BYTES = F4_A_BYTES + B_BYTES + F4_SF_BYTES + SFB_BYTES;
+    static constexpr int SF_COLS = WIDE ? 64 : 32;      // TMEM columns per stage: A 16, B 16 per 128 rows
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
+    static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * NUM_BARS;
+    static constexpr int TMAP_OFF = TMEM_SLOT_OFF + 16;
+    static constexpr int STG_OFF = (TMAP_OFF + TMAP_BYTES + 15) / 16 * 16;   // down-store staging
+    static constexpr int TOTAL = STG_OFF + (WIDE ? 0 : 8 * STG_WARP_FLOATS * 4) + 1024;
+    static_assert(TOTAL <= 232448, "shared memory of the NVFP4 GEMM exceeds 227 KB");
+    static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 128-byte swizzle atoms aligned");
+    static_assert(NBUF * BN <= F4_SF_TMEM && F4_SF_TMEM + SF_COLS * STAGES <= 512, "TMEM columns");
+};
+template <int KIND, int ACT>
+__host__ __device__ constexpr bool fp4_wide() { return KIND == KIND_GATE_UP && ACT != 5; }
+template <int KIND, int ACT>
+using Fp4Layout = Fp4Smem<fp4_wide<KIND, ACT>()>;
 
 struct Fp4Params {
     const int32_t* tiles;
@@ -48,7 +72,7 @@ struct Fp4Params {
     const int32_t* tile_ptr;
     const int32_t* offsets;
     int E;
-    int n_blocks;             // N / 128
+    int n_blocks;             // N / tile width
     int num_kb;               // K / 256
     int sf_cols;              // K / 16
     int b_rows;               // rows of B per expert (2I for gate/up, H for down)
@@ -74,15 +98,19 @@ template <int KIND, int ACT>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     grouped_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const Fp4Params p) {
+    using L = Fp4Layout<KIND, ACT>;
+    constexpr bool WIDE = fp4_wide<KIND, ACT>();
+    constexpr int F4_BN = L::BN, F4_NBUF = L::NBUF, F4_STAGES = L::STAGES;
+    constexpr int F4_B_BYTES = L::B_BYTES, F4_STAGE_BYTES = L::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F4_BAR_OFF);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* full = bars;
     uint64_t* empty = bars + F4_STAGES;
     uint64_t* tfull = bars + 2 * F4_STAGES;
     uint64_t* tempty = bars + 2 * F4_STAGES + F4_NBUF;
     uint64_t* drain = bars + 2 * F4_STAGES + 2 * F4_NBUF;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F4_TMEM_SLOT_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -107,7 +135,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     pdl_wait();
     pdl_trigger();
     KTRACE(p.o != nullptr ? TR_FP4 + 1 : TR_FP4);
-    int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + F4_TMAP_OFF);
+    int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + L::TMAP_OFF);
     const int32_t* s_off = s_tptr + TMAP_STRIDE;
     stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
     __syncthreads();
@@ -126,8 +154,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const int brow = e * p.b_rows + nb * F4_BN;
                 const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
                 const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.sf_cols * 128;
+                // scale factors of the tile's 128-row blocks of B (BN / 128 of them)
                 const uint8_t* sfb = p.sfb + static_cast<size_t>(e) * p.b_rows * p.sf_cols +
-                                     static_cast<size_t>(nb) * p.sf_cols * 128;
+                                     static_cast<size_t>(nb) * (F4_BN / 128) * p.sf_cols * 128;
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
                     const int s = it % F4_STAGES;
                     if (!mbar_wait(&empty[s], ((it / F4_STAGES) & 1) ^ 1, limit)) {
@@ -140,8 +169,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     tma_load_2d(st, &tmA, &full[s], kb * 128, mi * 128);
                     tma_load_2d_hint(st + F4_A_BYTES, &tmB, &full[s], kb * 128, brow, pol);
                     bulk_load(st + F4_A_BYTES + F4_B_BYTES, sfa + kb * F4_SF_BYTES, F4_SF_BYTES, &full[s]);
-                    bulk_load_hint(st + F4_A_BYTES + F4_B_BYTES + F4_SF_BYTES, sfb + kb * F4_SF_BYTES, F4_SF_BYTES,
-                                   &full[s], pol);
+#pragma unroll
+                    for (int hb = 0; hb < F4_BN / 128; hb++)
+                        bulk_load_hint(st + F4_A_BYTES + F4_B_BYTES + F4_SF_BYTES * (1 + hb),
+                                       sfb + static_cast<size_t>(hb) * p.sf_cols * 128 + kb * F4_SF_BYTES, F4_SF_BYTES,
+                                       &full[s], pol);
                 }
             }
             const uint32_t first = it > F4_STAGES ? it - F4_STAGES : 0;
@@ -165,17 +197,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const uint32_t b_addr = a_addr + F4_A_BYTES;
                     const uint32_t sfa_addr = b_addr + F4_B_BYTES;
                     const uint32_t sfb_addr = sfa_addr + F4_SF_BYTES;
-                    const uint32_t sf_col = tmem_base + F4_SF_TMEM + 32 * s;
+                    // MMA j (K = 64) reads A-scale chunk j (4 columns) and, per
+                    // 128-row block hb of B, B-scale chunk j at 4 (BN / 128) j + 4 hb
+                    const uint32_t sf_col = tmem_base + F4_SF_TMEM + L::SF_COLS * s;
+                    constexpr int NHB = F4_BN / 128;
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
                         tmem_cp_32x128b_x4(sf_col + 4 * j, sdesc_sf_chunk(sfa_addr + 512 * j));
-                        tmem_cp_32x128b_x4(sf_col + 16 + 4 * j, sdesc_sf_chunk(sfb_addr + 512 * j));
+#pragma unroll
+                        for (int hb = 0; hb < NHB; hb++)
+                            tmem_cp_32x128b_x4(sf_col + 16 + 4 * NHB * j + 4 * hb,
+                                               sdesc_sf_chunk(sfb_addr + F4_SF_BYTES * hb + 512 * j));
                     }
                     const uint32_t d = tmem_base + acc * F4_BN;
 #pragma unroll
                     for (int j = 0; j < 4; j++)
                         mma_nvf4(d, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j), idesc, sf_col + 4 * j,
-                                 sf_col + 16 + 4 * j, (kb > 0 || j > 0));
+                                 sf_col + 16 + 4 * NHB * j, (kb > 0 || j > 0));
                     mma_commit(&empty[s]);
                 }
                 if (!ok) break;
@@ -218,33 +256,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 continue;
             }
             if (KIND == KIND_GATE_UP) {
-                float gv[32], uv[32];
-                tmem_ld32x2(lane_addr + acc * F4_BN + 32 * g, lane_addr + acc * F4_BN + 64 + 32 * g, gv, uv);
+                // TMEM columns of a 128-row block of B: gate [0, 64), up [64, 128).
+                // Narrow: one block, this warp's 32 columns at 32 g.  Wide: blocks
+                // g of the tile (columns 128 g ..), both 32-column runs.
+                constexpr int NL = WIDE ? 2 : 1;
+                float gv[NL][32], uv[NL][32];
+#pragma unroll
+                for (int ld = 0; ld < NL; ld++) {
+                    const int c0 = WIDE ? 128 * g + 32 * ld : 32 * g;
+                    tmem_ld32x2(lane_addr + acc * F4_BN + c0, lane_addr + acc * F4_BN + c0 + 64, gv[ld], uv[ld]);
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[acc]);
                 u++;
                 const float sg = gx * wg0, su = gx * wg1;
-                // gated: one 32-column run act(g, u) at hidden 64 nb + 32 g; ReLU^2 (no
-                // gate, 128 up rows per tile): relu(v)^2 of both 32-column halves, at
-                // hidden 128 nb + 32 g and 128 nb + 64 + 32 g
-                constexpr int NR = ACT == 5 ? 2 : 1;
+                // gated: run l = act(g, u) of load l, at hidden 64 nb + 32 g (narrow)
+                // or 128 nb + 64 g + 32 l (wide); ReLU^2 (no gate, 128 up rows per
+                // tile): relu(v)^2 of both 32-column halves, at hidden 128 nb + 32 g
+                // and 128 nb + 64 + 32 g
+                constexpr int NR = (ACT == 5 || WIDE) ? 2 : 1;
                 float hv[32 * NR];
 #pragma unroll
                 for (int c = 0; c < 32; c++) {
-                    const float gg = gv[c] * sg, uu = uv[c] * su;
                     if constexpr (ACT == 5) {
-                        hv[c] = relu_sq(gg);
-                        hv[32 + c] = relu_sq(uu);
+                        hv[c] = relu_sq(gv[0][c] * sg);
+                        hv[32 + c] = relu_sq(uv[0][c] * su);
                     } else {
-                        hv[c] = glu<ACT>(gg, uu, p.act_alpha, p.act_limit);
+#pragma unroll
+                        for (int ld = 0; ld < NL; ld++)
+                            hv[32 * ld + c] = glu<ACT>(gv[ld][c] * sg, uv[ld][c] * su, p.act_alpha, p.act_limit);
                     }
                 }
                 if (valid) {
 #pragma unroll
                     for (int run = 0; run < NR; run++) {
                         // first hidden column of this run
-                        const int col0 = ACT == 5 ? nb * 128 + 64 * run + 32 * g : nb * 64 + 32 * g;
+                        const int col0 = ACT == 5 ? nb * 128 + 64 * run + 32 * g
+                                                  : (WIDE ? nb * 128 + 64 * g + 32 * run : nb * 64 + 32 * g);
                         uint32_t w[4];
 #pragma unroll
                         for (int b = 0; b < 2; b++) {           // two 16-blocks
@@ -285,7 +334,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     v[32 + c] = v1[c];
                 }
                 store_rows_coalesced<64, false>(
-                    v, reinterpret_cast<float*>(smem + F4_STG_OFF) + (warp - 2) * STG_WARP_FLOATS,
+                    v, reinterpret_cast<float*>(smem + L::STG_OFF) + (warp - 2) * STG_WARP_FLOATS,
                     valid ? p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + 64 * g : nullptr, nullptr,
                     p.h_global * wg0 * rw, lane);
             }

@@ -533,8 +533,9 @@ template <int KIND, int ACT = 0>
 static moe_status launch_fp4(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const Fp4Params& p, int grid,
                              cudaStream_t st) {
     auto kern = grouped_gemm_fp4_kernel<KIND, ACT>;
-    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F4_SMEM));
-    LAUNCH(pdl, "grouped_gemm_fp4_kernel", kern, grid, GEMM_THREADS, F4_SMEM, st, ta, tb, p);
+    constexpr int smem = Fp4Layout<KIND, ACT>::TOTAL;
+    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    LAUNCH(pdl, "grouped_gemm_fp4_kernel", kern, grid, GEMM_THREADS, smem, st, ta, tb, p);
     return MOE_OK;
 }
 
@@ -550,8 +551,11 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     CUtensorMap ta, tb;
     moe_status r = make_tmap(&ta, gate_up ? v.xq : v.hq, K / 2, R, K / 2, 128, 128);
     if (r != MOE_OK) return r;
+    // gated gate/up: 256-row tiles of B (two packed 64 gate + 64 up blocks);
+    // down and ReLU^2 gate/up: 128-row tiles
+    const int bn = (gate_up && c.act != MOE_ACT_RELU2) ? 256 : 128;
     r = make_tmap(&tb, pw + (gate_up ? h->wl.gu_q : h->wl.d_q), K / 2, static_cast<uint64_t>(c.E) * N, K / 2, 128,
-                  F4_BN);
+                  bn);
     if (r != MOE_OK) return r;
     Fp4Params p;
     memset(&p, 0, sizeof(p));
@@ -560,7 +564,7 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     p.tile_ptr = v.tile_ptr;
     p.offsets = v.offsets;
     p.E = c.E;
-    p.n_blocks = N / F4_BN;
+    p.n_blocks = N / bn;
     p.num_kb = K / 256;
     p.sf_cols = K / 16;
     p.b_rows = N;
