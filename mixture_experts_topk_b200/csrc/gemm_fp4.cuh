@@ -16,19 +16,22 @@
 // copies.  The MMA thread copies the chunks into a TMEM ring (tcgen05.cp, 32
 // rows x 16 B repeated over the 4 lane quadrants), then issues the 4
 // block-scaled MMAs, which read them in issue order.
-//  - Down GEMM and ReLU^2 gate/up: 128-column tiles, two 128-column
-//    accumulators at [0, 256), 5 stages.
-//  - Gated gate/up: 256-column tiles (two consecutive 64 gate + 64 up blocks of
-//    the packed weights, 128 hidden columns), so each 128 x 256 x 256 step
-//    needs 54 KB of operands and scales instead of 2 x 36 KB, and A is read
-//    half as often.  One 256-column accumulator, released as soon as the
-//    epilogue holds it in registers; 4 stages.
+//  - Gated gate/up and down: 256-column tiles (gate/up: two consecutive 64
+//    gate + 64 up blocks of the packed weights, 128 hidden columns), so each
+//    128 x 256 x 256 step needs 54 KB of operands and scales instead of
+//    2 x 36 KB, and A is read half as often.  One 256-column accumulator,
+//    released as soon as the epilogue holds it in registers; 4 stages (down:
+//    3, beside the staging of its fp32 row stores).
+//  - ReLU^2 gate/up: 128-column tiles, two 128-column accumulators at
+//    [0, 256), 5 stages.
 // The scale-factor ring starts at TMEM column 256.
 //
 // Rows are in the 128-padded expert-major layout (m-tile i = rows 128 i ..),
 // so each tile's scale factors are whole chunks.  The epilogue maps a padded
 // row back to its assignment slot (offsets) for the outputs indexed by slot.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -38,33 +41,35 @@ constexpr int F4_A_BYTES = 128 * 128;
 constexpr int F4_SF_BYTES = 2048;                 // 4 chunks of 512 B per 128 rows
 constexpr int F4_SF_TMEM = 256;                   // first column of the scale-factor ring
 
-// Shared memory and TMEM of one instantiation.  Narrow (down, ReLU^2 gate/up):
-// 128-column tiles, two accumulators, 5 stages.  Wide (gated gate/up): 256
-// columns (two 64 gate + 64 up blocks), one accumulator released as soon as
-// the epilogue has it in registers, 4 stages.
-template <bool WIDE>
+// Shared memory and TMEM of one instantiation: BN-column tiles, NBUF
+// accumulators, STAGES smem stages, and the float4 row staging of the fp32
+// down stores (STG).
+template <int BN_, int NBUF_, int STAGES_, bool STG>
 struct Fp4Smem {
-    static constexpr int BN = WIDE ? 256 : 128;
-    static constexpr int NBUF = WIDE ? 1 : 2;
-    static constexpr int STAGES = WIDE ? 4 : 5;
+    static constexpr int BN = BN_;
+    static constexpr int NBUF = NBUF_;
+    static constexpr int STAGES = STAGES_;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int SFB_BYTES = (BN / 128) * F4_SF_BYTES;
     static constexpr int STAGE_BYTES = F4_A_BYTES + B_BYTES + F4_SF_BYTES + SFB_BYTES;
-    static constexpr int SF_COLS = WIDE ? 64 : 32;      // TMEM columns per stage: A 16, B 16 per 128 rows
+    static constexpr int SF_COLS = BN == 256 ? 64 : 32;   // TMEM columns per stage: A 16, B 16 per 128 rows
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
     static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int TMAP_OFF = TMEM_SLOT_OFF + 16;
-    static constexpr int STG_OFF = (TMAP_OFF + TMAP_BYTES + 15) / 16 * 16;   // down-store staging
-    static constexpr int TOTAL = STG_OFF + (WIDE ? 0 : 8 * STG_WARP_FLOATS * 4) + 1024;
+    static constexpr int STG_OFF = (TMAP_OFF + TMAP_BYTES + 15) / 16 * 16;
+    static constexpr int TOTAL = STG_OFF + (STG ? 8 * STG_WARP_FLOATS * 4 : 0) + 1024;
     static_assert(TOTAL <= 232448, "shared memory of the NVFP4 GEMM exceeds 227 KB");
     static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 128-byte swizzle atoms aligned");
     static_assert(NBUF * BN <= F4_SF_TMEM && F4_SF_TMEM + SF_COLS * STAGES <= 512, "TMEM columns");
 };
+// Gated gate/up: 256-column tiles (two 64 gate + 64 up blocks), one
+// accumulator released as soon as the epilogue holds it in registers, 4
+// stages.  Down: 256-column tiles, one accumulator, 3 stages and the row
+// staging.  ReLU^2 gate/up: 128-column tiles, two accumulators, 5 stages.
 template <int KIND, int ACT>
-__host__ __device__ constexpr bool fp4_wide() { return KIND == KIND_GATE_UP && ACT != 5; }
-template <int KIND, int ACT>
-using Fp4Layout = Fp4Smem<fp4_wide<KIND, ACT>()>;
+using Fp4Layout = std::conditional_t<KIND == KIND_DOWN, Fp4Smem<256, 1, 3, true>,
+                                     std::conditional_t<ACT == 5, Fp4Smem<128, 2, 5, false>, Fp4Smem<256, 1, 4, false>>>;
 
 struct Fp4Params {
     const int32_t* tiles;
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     grouped_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const Fp4Params p) {
     using L = Fp4Layout<KIND, ACT>;
-    constexpr bool WIDE = fp4_wide<KIND, ACT>();
+    constexpr bool WIDE = L::BN == 256;
     constexpr int F4_BN = L::BN, F4_NBUF = L::NBUF, F4_STAGES = L::STAGES;
     constexpr int F4_B_BYTES = L::B_BYTES, F4_STAGE_BYTES = L::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
@@ -227,7 +232,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
-        const int g = (warp - 2) >> 2;           // column group: 32 (gate/up) or 64 (down) columns
+        const int g = (warp - 2) >> 2;           // column group: half of the tile's columns
         const int r = 32 * q + lane;
         const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
         uint32_t u = 0;
@@ -321,21 +326,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     }
                 }
             } else {
-                float v0[32], v1[32];
-                tmem_ld32x2(lane_addr + acc * F4_BN + 64 * g, lane_addr + acc * F4_BN + 64 * g + 32, v0, v1);
+                // this warp's NC columns of the tile: 64 (narrow) or 128 (wide) at NC g
+                constexpr int NC = F4_BN / 2;
+                float v[NC];
+#pragma unroll
+                for (int ch = 0; ch < NC / 64; ch++)
+                    tmem_ld32x2(lane_addr + acc * F4_BN + NC * g + 64 * ch, lane_addr + acc * F4_BN + NC * g + 64 * ch + 32,
+                                v + 64 * ch, v + 64 * ch + 32);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[acc]);
                 u++;
-                float v[64];
-#pragma unroll
-                for (int c = 0; c < 32; c++) {
-                    v[c] = v0[c];
-                    v[32 + c] = v1[c];
-                }
-                store_rows_coalesced<64, false>(
+                store_rows_coalesced<NC, false>(
                     v, reinterpret_cast<float*>(smem + L::STG_OFF) + (warp - 2) * STG_WARP_FLOATS,
-                    valid ? p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + 64 * g : nullptr, nullptr,
+                    valid ? p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + NC * g : nullptr, nullptr,
                     p.h_global * wg0 * rw, lane);
             }
         }

@@ -551,9 +551,9 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     CUtensorMap ta, tb;
     moe_status r = make_tmap(&ta, gate_up ? v.xq : v.hq, K / 2, R, K / 2, 128, 128);
     if (r != MOE_OK) return r;
-    // gated gate/up: 256-row tiles of B (two packed 64 gate + 64 up blocks);
-    // down and ReLU^2 gate/up: 128-row tiles
-    const int bn = (gate_up && c.act != MOE_ACT_RELU2) ? 256 : 128;
+    // gated gate/up (two packed 64 gate + 64 up blocks) and down: 256-row
+    // tiles of B; ReLU^2 gate/up: 128-row tiles
+    const int bn = (gate_up && c.act == MOE_ACT_RELU2) ? 128 : 256;
     r = make_tmap(&tb, pw + (gate_up ? h->wl.gu_q : h->wl.d_q), K / 2, static_cast<uint64_t>(c.E) * N, K / 2, 128,
                   bn);
     if (r != MOE_OK) return r;
