@@ -150,7 +150,8 @@ moe_status moe_workspace_size(const moe_handle* h, size_t* bytes);
 moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_workspace_view* view);
 
 /* Rearrange plain-layout weights into the packed device layout the GEMMs read
- * (gate and up interleaved in 128-row blocks so one tile holds both).  Not on
+ * (gate and up interleaved in row blocks, 128 + 128 rows for the FP8 formats
+ * and 64 + 64 for NVFP4, so one tile holds both).  Not on
  * the timed path (LightMoE README, "Installation": packing outside latency). */
 moe_status moe_pack_weights(const moe_handle* h, const moe_weights* src, void* packed,
                             moe_stream_t stream);
