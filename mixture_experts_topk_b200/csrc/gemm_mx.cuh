@@ -17,6 +17,14 @@
 // accumulator, released as soon as the epilogue has it in registers, then the
 // A-scale ring and the constant B-scale chunks.
 //
+// Large batches with deep K run on CTA pairs (2-CTA clusters): one
+// tcgen05.mma.cta_group::2 with M = 256 covers two m-tiles of one expert; each
+// CTA loads its 128 hidden rows, its scale chunk and 128 of the 256 B rows,
+// completing them on rank 0's barrier (the scale chunk by TMA as two 256-byte
+// rows); rank 0 copies both CTAs' scale chunks into their TMEM and issues the
+// MMAs; commits reach both CTAs.  An expert with an odd m-tile count runs its
+// last pair with rank 1's rows unstored (it loads rank 0's rows).
+//
 // Output rows: a warp whose 32 rows are all stored (rows of one expert are
 // consecutive slots) writes them as four 32-row x 32-column fp32 boxes through
 // a 128-byte-swizzled shared buffer (two per warp, alternating) with TMA
@@ -30,19 +38,23 @@ namespace moe {
 
 constexpr int MX_BN = 256;
 constexpr int MX_A_BYTES = 128 * 128;
-constexpr int MX_B_BYTES = MX_BN * 128;
 constexpr int MX_SFA_BYTES = 512;
-constexpr int MX_STAGE_BYTES = MX_A_BYTES + MX_B_BYTES + 1024;   // + 512 B A scales, padded to 1 KB
 constexpr int MX_BOX_BYTES = 32 * 128;                           // 32 rows x 32 fp32
 constexpr int MX_SFA_TMEM = MX_BN;                               // 4 columns per stage
-constexpr int MX_SFB_TMEM = MX_BN + 16;                          // 8 columns (two 128-row chunks)
+constexpr int MX_SFB_TMEM = MX_BN + 32;                          // 8 columns (two 128-row chunks)
 // Deep K (many K stages per tile): 4 stages, rows stored from registers.
 // Shallow K, where a tile's stores outlast its MMAs: 3 stages and the box stores.
 constexpr int MX_BOX_MAX_KB = 16;
+// CTA pairs (deep K, large batches): 33 KB stages, 5 deep.
+constexpr int MX_PAIR_STAGES = 5;
 
-template <int STAGES, bool BOXES>
+// PAIR: a CTA pair (tcgen05 cta_group::2, M = 256) where each CTA loads its 128
+// A rows and 128 of the 256 B rows.
+template <int STAGES, bool BOXES, bool PAIR = false>
 struct MxSmem {
-    static constexpr int SFB_OFF = STAGES * MX_STAGE_BYTES;           // 2 constant chunks (1 KB)
+    static constexpr int B_BYTES = (PAIR ? MX_BN / 2 : MX_BN) * 128;
+    static constexpr int STAGE_BYTES = MX_A_BYTES + B_BYTES + 1024;   // + 512 B A scales, padded to 1 KB
+    static constexpr int SFB_OFF = STAGES * STAGE_BYTES;              // 2 constant chunks (1 KB)
     static constexpr int BAR_OFF = SFB_OFF + 1024;
     static constexpr int NUM_BARS = 2 * STAGES + 3;
     static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * NUM_BARS;
@@ -51,10 +63,12 @@ struct MxSmem {
     static constexpr int STG_OFF = BOXES ? (TMAP_OFF + TMAP_BYTES + 1023) / 1024 * 1024
                                          : (TMAP_OFF + TMAP_BYTES + 15) / 16 * 16;
     static constexpr int STG_WARP_BYTES = BOXES ? 2 * MX_BOX_BYTES : STG_WARP_FLOATS * 4;
-    static constexpr int TOTAL = STG_OFF + 8 * STG_WARP_BYTES + 1024;
+    static constexpr int PPTR_OFF = STG_OFF + 8 * STG_WARP_BYTES;     // pairs: m-pairs per expert
+    static constexpr int TOTAL = PPTR_OFF + (PAIR ? TMAP_STRIDE * 4 : 0) + 1024;
     static_assert(TOTAL <= 232448, "shared memory of the down GEMM exceeds 227 KB");
+    static_assert(!(PAIR && BOXES), "pairs store rows from registers");
     static_assert(STG_WARP_FLOATS * 4 <= STG_WARP_BYTES, "row staging fits");
-    static_assert(4 * STAGES <= 16, "A-scale ring below the B-scale chunks");
+    static_assert(4 * STAGES <= 32, "A-scale ring below the B-scale chunks");
 };
 
 // Instruction descriptor of kind::mxf8f6f4 block-scaled: A, B E4M3 (0), K-major,
@@ -74,6 +88,22 @@ __device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint6
             d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
+}
+
+// cta_group::2 forms: one thread of the pair's first CTA issues them for both
+// CTAs (each CTA's own shared memory to its own TMEM; its own A rows).
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 struct MxDownParams {
@@ -100,11 +130,12 @@ struct MxDownParams {
     long long spin_limit;
 };
 
-template <int STAGES, bool BOXES>
+template <int STAGES, bool BOXES, bool PAIR = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     grouped_gemm_mx_down_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                const __grid_constant__ CUtensorMap tmO, const MxDownParams p) {
-    using L = MxSmem<STAGES, BOXES>;
+                                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmS,
+                                const MxDownParams p) {
+    using L = MxSmem<STAGES, BOXES, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
@@ -115,28 +146,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     uint64_t* drain = bars + 2 * STAGES + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // CTA pairs: rank 0 issues the MMAs; its full and tempty barriers take the
+    // arrivals of both CTAs
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;
 
     // constant B scale chunks: 1.0 for every row and block
     for (int i = threadIdx.x; i < 1024 / 4; i += blockDim.x)
         reinterpret_cast<uint32_t*>(smem + L::SFB_OFF)[i] = 0x7F7F7F7Fu;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], PAIR ? 2 : 1);   // pairs: one expect_tx arrival per CTA
             mbar_init(&empty[s], 1);
         }
         mbar_init(tfull, 1);
-        mbar_init(tempty, 8);
+        mbar_init(tempty, PAIR ? 16 : 8);       // one arrival per epilogue warp
         mbar_init(drain, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmO);
+        if (PAIR) tma_prefetch_desc(&tmS);
     }
-    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    if (warp == 1) {
+        if constexpr (PAIR) tmem_alloc_pair(tmem_slot, 512);
+        else tmem_alloc(tmem_slot, 512);
+    }
     // the generic-proxy writes of the constant chunks become visible to tcgen05.cp
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // Chained after the gate/up GEMM, this kernel does not wait for that whole
@@ -149,12 +188,42 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int32_t* s_tptr = reinterpret_cast<int32_t*>(smem + L::TMAP_OFF);
     const int32_t* s_off = s_tptr + TMAP_STRIDE;
     stage_tile_map(s_tptr, p.tile_ptr, p.offsets, p.E);
+    int32_t* s_pptr = reinterpret_cast<int32_t*>(smem + L::PPTR_OFF);
+    if constexpr (PAIR) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // m-pairs per expert, prefix over experts (E <= 256 steps, once per CTA)
+            int acc_p = 0;
+            for (int i = 0; i < p.E; i++) {
+                s_pptr[i] = acc_p;
+                acc_p += (s_tptr[i + 1] - s_tptr[i] + 1) >> 1;
+            }
+            s_pptr[p.E] = acc_p;
+        }
+    }
     __syncthreads();
     const int ntm = *p.num_tiles;
-    const int units = ntm * p.n_blocks;
+    const int units = (PAIR ? s_pptr[p.E] : ntm) * p.n_blocks;
     const int S = min(max(*p.split, 1), p.s_max);
     const int total = units * S;
     const long long limit = p.spin_limit;
+    // CTA pairs walk the work items by cluster, single CTAs by block
+    const int t_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int t_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    // this CTA's m-tile of unit v: (expert, global m-tile, n-block, has rows);
+    // a pair's m-pair j holds the expert's m-tiles 2j (rank 0) and 2j + 1
+    auto unit_tile = [&](int v, int& e, int& mi, int& nb, bool& has_rows) {
+        if constexpr (PAIR) {
+            int mp;
+            decode_pair(v, s_pptr, p.E, p.n_blocks, e, mp, nb);
+            const int local = 2 * mp + static_cast<int>(rank);
+            has_rows = local < s_tptr[e + 1] - s_tptr[e];
+            mi = s_tptr[e] + local;
+        } else {
+            decode_tile(v, s_tptr, p.E, p.n_blocks, e, mi, nb);
+            has_rows = true;
+        }
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -162,13 +231,40 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             int ready_e = -1;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = t_first; t < total && ok; t += t_step) {
                 const int sp = t % S;   // unit-major: all splits of a unit together, experts in order
                 int e, mi, nb;
-                decode_tile(t / S, s_tptr, p.E, p.n_blocks, e, mi, nb);
-                const int brow = e * p.b_rows + nb * MX_BN;
+                bool has_rows;
+                unit_tile(t / S, e, mi, nb, has_rows);
+                // a pair's rank 1 without an m-tile (odd count) loads rank 0's rows and
+                // scales, so its reads stay inside the buffers; its rows are not stored
+                const int mi_ld = has_rows ? mi : mi - 1;
+                const int brow = e * p.b_rows + nb * MX_BN + (PAIR ? static_cast<int>(rank) * (MX_BN / 2) : 0);
                 const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
-                const uint8_t* sfa = p.sfa + static_cast<size_t>(mi) * p.num_kb * 512;
+                const uint8_t* sfa = p.sfa + static_cast<size_t>(mi_ld) * p.num_kb * 512;
+                // both CTAs of a pair complete their stage bytes on rank 0's barrier
+                auto stage_bar = [&](int s) -> uint32_t {
+                    return PAIR ? cluster_addr(&full[s], 0) : smem_u32(&full[s]);
+                };
+                auto expect = [&](int s) {
+                    if constexpr (PAIR) mbar_arrive_expect_tx_cluster(stage_bar(s), MX_A_BYTES + L::B_BYTES + MX_SFA_BYTES);
+                    else mbar_arrive_expect_tx(&full[s], MX_A_BYTES + L::B_BYTES + MX_SFA_BYTES);
+                };
+                auto load_b = [&](uint8_t* st, int s, int k) {
+                    if constexpr (PAIR) tma_load_2d_pair(st + MX_A_BYTES, &tmB, stage_bar(s), k * 128, brow, pol);
+                    else tma_load_2d_hint(st + MX_A_BYTES, &tmB, &full[s], k * 128, brow, pol);
+                };
+                auto load_a_sfa = [&](uint8_t* st, int s, int k) {
+                    if constexpr (PAIR) {
+                        tma_load_2d_pair(st, &tmA, stage_bar(s), k * 128, mi_ld * 128, l2_policy(false));
+                        // scale chunk (mi_ld, k) = rows 2 (mi_ld num_kb + k) .. + 1 of 256 bytes
+                        tma_load_2d_pair(st + MX_A_BYTES + L::B_BYTES, &tmS, stage_bar(s), 0, 2 * (mi_ld * p.num_kb + k),
+                                         l2_policy(false));
+                    } else {
+                        tma_load_2d(st, &tmA, &full[s], k * 128, mi * 128);
+                        bulk_load(st + MX_A_BYTES + L::B_BYTES, sfa + k * 512, MX_SFA_BYTES, &full[s]);
+                    }
+                };
                 const int kb0 = sp * p.num_kb / S, kb1 = (sp + 1) * p.num_kb / S;
                 int kb = kb0;
                 if (p.gu_done != nullptr && e != ready_e) {
@@ -182,9 +278,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         const uint32_t itj = it + armed;
                         const int s = itj % STAGES;
                         if (!mbar_wait(&empty[s], ((itj / STAGES) & 1) ^ 1, limit)) { ok = false; break; }
-                        mbar_arrive_expect_tx(&full[s], MX_A_BYTES + MX_B_BYTES + MX_SFA_BYTES);
-                        tma_load_2d_hint(smem + s * MX_STAGE_BYTES + MX_A_BYTES, &tmB, &full[s], (kb0 + armed) * 128,
-                                         brow, pol);
+                        expect(s);
+                        load_b(smem + s * L::STAGE_BYTES, s, kb0 + armed);
                     }
                     if (ok) {
                         const int target = (s_tptr[e + 1] - s_tptr[e]) * p.gu_per_mtile;
@@ -202,10 +297,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     // that no copy into them is left incomplete
                     for (int j = 0; j < armed; j++) {
                         const uint32_t itj = it + j;
-                        uint8_t* st = smem + (itj % STAGES) * MX_STAGE_BYTES;
-                        tma_load_2d(st, &tmA, &full[itj % STAGES], (kb0 + j) * 128, mi * 128);
-                        bulk_load(st + MX_A_BYTES + MX_B_BYTES, sfa + (kb0 + j) * 512, MX_SFA_BYTES,
-                                  &full[itj % STAGES]);
+                        load_a_sfa(smem + (itj % STAGES) * L::STAGE_BYTES, itj % STAGES, kb0 + j);
                     }
                     it += armed;
                     kb += armed;
@@ -222,25 +314,34 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    uint8_t* st = smem + s * MX_STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[s], MX_A_BYTES + MX_B_BYTES + MX_SFA_BYTES);
-                    tma_load_2d(st, &tmA, &full[s], kb * 128, mi * 128);
-                    tma_load_2d_hint(st + MX_A_BYTES, &tmB, &full[s], kb * 128, brow, pol);
-                    bulk_load(st + MX_A_BYTES + MX_B_BYTES, sfa + kb * 512, MX_SFA_BYTES, &full[s]);
+                    uint8_t* st = smem + s * L::STAGE_BYTES;
+                    expect(s);
+                    load_a_sfa(st, s, kb);
+                    load_b(st, s, kb);
                 }
             }
-            const uint32_t first = it > STAGES ? it - STAGES : 0;
-            for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, DRAIN_LIMIT);
+            // loads still in flight land before the CTA may exit (for a pair, rank
+            // 0's barriers count both CTAs' loads, and the closing cluster barrier
+            // keeps rank 1 until rank 0 is past this)
+            if (!PAIR || rank == 0) {
+                const uint32_t first = it > STAGES ? it - STAGES : 0;
+                for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, DRAIN_LIMIT);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && (!PAIR || rank == 0)) {
+            // a pair's copies and MMAs (issued here, by rank 0) cover both CTAs
+            auto cp_sf = [&](uint32_t taddr, uint64_t sdesc) {
+                if constexpr (PAIR) tmem_cp_32x128b_x4_pair(taddr, sdesc);
+                else tmem_cp_32x128b_x4(taddr, sdesc);
+            };
             const uint32_t sfb = tmem_base + MX_SFB_TMEM;
-            tmem_cp_32x128b_x4(sfb, sdesc_sf_chunk(smem_u32(smem + L::SFB_OFF)));
-            tmem_cp_32x128b_x4(sfb + 4, sdesc_sf_chunk(smem_u32(smem + L::SFB_OFF + 512)));
+            cp_sf(sfb, sdesc_sf_chunk(smem_u32(smem + L::SFB_OFF)));
+            cp_sf(sfb + 4, sdesc_sf_chunk(smem_u32(smem + L::SFB_OFF + 512)));
             uint32_t it = 0, u = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = t_first; t < total && ok; t += t_step) {
                 const int sp = t % S;
                 const int kb0 = sp * p.num_kb / S, kb1 = (sp + 1) * p.num_kb / S;
                 if (!mbar_wait(tempty, (u & 1) ^ 1, limit)) { ok = false; break; }
@@ -249,23 +350,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const int s = it % STAGES;
                     if (!mbar_wait(&full[s], (it / STAGES) & 1, limit)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + s * MX_STAGE_BYTES);
+                    const uint32_t a_addr = smem_u32(smem + s * L::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + MX_A_BYTES;
                     const uint32_t sfa = tmem_base + MX_SFA_TMEM + 4 * s;
-                    tmem_cp_32x128b_x4(sfa, sdesc_sf_chunk(b_addr + MX_B_BYTES));
+                    cp_sf(sfa, sdesc_sf_chunk(b_addr + L::B_BYTES));
 #pragma unroll
-                    for (int j = 0; j < 4; j++)
-                        mma_mxf8(tmem_base, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
-                                 idesc_mxf8(128, MX_BN, j), sfa, sfb, (kb > kb0 || j > 0));
-                    mma_commit(&empty[s]);
+                    for (int j = 0; j < 4; j++) {
+                        if constexpr (PAIR)
+                            mma_mxf8_pair(tmem_base, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
+                                          idesc_mxf8(256, MX_BN, j), sfa, sfb, (kb > kb0 || j > 0));
+                        else
+                            mma_mxf8(tmem_base, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
+                                     idesc_mxf8(128, MX_BN, j), sfa, sfb, (kb > kb0 || j > 0));
+                    }
+                    if constexpr (PAIR) mma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
+                    else mma_commit(&empty[s]);
                 }
                 if (!ok) break;
-                mma_commit(tfull);
+                if constexpr (PAIR) mma_commit_pair_both(tfull);   // both CTAs' epilogues
+                else mma_commit(tfull);
                 u++;
             }
             if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
-            mma_commit(drain);
-            mbar_wait(drain, 0, DRAIN_LIMIT);
+            if constexpr (PAIR) mma_commit_pair(drain);   // every issued MMA has completed ...
+            else mma_commit(drain);
+            mbar_wait(drain, 0, DRAIN_LIMIT);             // ... before TMEM can be released
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -276,10 +385,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         uint8_t* ostg = smem + L::STG_OFF + (warp - 2) * L::STG_WARP_BYTES;
         uint32_t u = 0, nbox = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        // the accumulator is free again: a pair's MMA thread (rank 0) counts both
+        // CTAs' epilogue warps
+        auto release_acc = [&]() {
+            if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(tempty, 0));
+            else mbar_arrive(tempty);
+        };
+        for (int t = t_first; t < total && ok; t += t_step) {
             const int sp = t % S;
             int e, mi, nb;
-            decode_tile(t / S, s_tptr, p.E, p.n_blocks, e, mi, nb);
+            bool has_rows;
+            unit_tile(t / S, e, mi, nb, has_rows);
+            // none for a pair's absent m-tile (its rows lie past the expert's count)
             const int local = mi * 128 + r - s_tptr[e] * 128;
             const bool valid = local < s_off[e + 1] - s_off[e];
             // the row's routing weight is loaded while the tile's MMAs run
@@ -293,7 +410,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 // none of this warp's rows is stored: release the accumulator only
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(tempty);
+                if (lane == 0) release_acc();
                 u++;
                 continue;
             }
@@ -304,7 +421,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                             v + 64 * ch + 32);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty);   // the next tile's MMAs may start
+            if (lane == 0) release_acc();   // the next tile's MMAs may start
             u++;
             if (BOXES && __all_sync(0xffffffffu, valid)) {
                 // rows sp A + slot(lane 0) + lane: four boxes of 32 columns
@@ -355,9 +472,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    // a pair leaves together: no arrival or copy may target a CTA that has exited
+    if constexpr (PAIR) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, 512);
+        else tmem_dealloc(tmem_base, 512);
     }
 }
 

@@ -526,7 +526,7 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
 
 // ------------------------------------------------------------------ NVFP4 GEMMs
 static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
-                            uint32_t box_inner, uint32_t box_rows);
+                            uint32_t box_inner, uint32_t box_rows, bool swizzle = true);
 static int max_m_tiles(const moe_config& c, int T);
 
 template <int KIND, int ACT = 0>
@@ -612,10 +612,11 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2D byte matrix [rows][inner] with row pitch `pitch`, 128-byte swizzled boxes
-// of box_inner bytes x box_rows rows; rows past the end read as zero.
+// 2D byte matrix [rows][inner] with row pitch `pitch`, boxes of box_inner
+// bytes x box_rows rows, 128-byte swizzled (else stored as they are in memory);
+// rows past the end read as zero.
 static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
-                            uint32_t box_inner, uint32_t box_rows) {
+                            uint32_t box_inner, uint32_t box_rows, bool swizzle) {
     auto fn = encode_fn();
     if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     cuuint64_t dims[2] = {inner, rows};
@@ -623,7 +624,8 @@ static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, u
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
     return MOE_OK;
@@ -756,10 +758,19 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
-    CUtensorMap ta, tb, to;
+    // Large batches with deep K: CTA pairs (M = 256), each CTA loading 128 of a
+    // tile's 256 B rows, when the experts average at least 4 row tiles (as for
+    // the gate/up GEMM); shallow K keeps single CTAs and the box stores.
+    const bool pairs = h->gemm_pairs && c.I / 128 > MX_BOX_MAX_KB && T * c.k >= 4 * TILE_M * c.E;
+    CUtensorMap ta, tb, to, ts;
     moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
-    r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, MX_BN);
+    r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, pairs ? MX_BN / 2 : MX_BN);
+    if (r != MOE_OK) return r;
+    // hidden scales as rows of 256 bytes (a 512-byte chunk per row tile and K
+    // stage is two rows), copied as they are: the pairs' scale loads
+    const uint64_t hs_bytes = hidden_rows(c) * hidden_scale_bytes(c.fmt, c.I);
+    r = make_tmap(&ts, v.hs, 256, hs_bytes / 256, 256, 256, 2, false);
     if (r != MOE_OK) return r;
     // output rows (fp32 as bytes): boxes of 32 rows x 32 values for the epilogue's stores
     r = make_tmap(&to, v.o, static_cast<uint64_t>(c.H) * 4, o_rows(c), static_cast<uint64_t>(c.H) * 4, 128, 32);
@@ -789,16 +800,27 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks * p.s_max));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (pairs) {
+        using Lp = MxSmem<MX_PAIR_STAGES, false, true>;
+        auto kern = grouped_gemm_mx_down_kernel<MX_PAIR_STAGES, false, true>;
+        const int npairs = std::max(1, std::min(h->num_sms / 2, (max_m_tiles(c, T) + 1) / 2 * p.n_blocks * p.s_max));
+        CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lp::TOTAL));
+        const cudaError_t err =
+            launch_k_pairs(h->pdl, kern, dim3(2 * npairs), dim3(GEMM_THREADS), Lp::TOTAL, st, ta, tb, to, ts, p);
+        if (err != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "launch of grouped_gemm_mx_down_kernel (pairs) failed: %s", cudaGetErrorString(err));
+        return MOE_OK;
+    }
     if (p.num_kb <= MX_BOX_MAX_KB) {
         using Lb = MxSmem<3, true>;
         auto kern = grouped_gemm_mx_down_kernel<3, true>;
         CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lb::TOTAL));
-        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Lb::TOTAL, st, ta, tb, to, p);
+        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Lb::TOTAL, st, ta, tb, to, ts, p);
     } else {
         using Lr = MxSmem<4, false>;
         auto kern = grouped_gemm_mx_down_kernel<4, false>;
         CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lr::TOTAL));
-        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Lr::TOTAL, st, ta, tb, to, p);
+        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Lr::TOTAL, st, ta, tb, to, ts, p);
     }
     return MOE_OK;
 }

@@ -20,6 +20,8 @@ CASES = {
     "fp8-row": W.custom(H=512, I=256, E=8, k=2),
     # K = I > 2048: the down GEMM's deep-K variant (4 stages, rows stored from registers)
     "fp8-row-deep-k": W.custom(H=512, I=2304, E=8, k=2),
+    # both GEMMs on CTA pairs (the down GEMM's pairs wait on each other's copies too)
+    "fp8-row-deep-k-pairs": W.custom(H=512, I=2304, E=8, k=2),
     # T k >= 512 E: the gate/up GEMM on CTA pairs (waits on the other CTA's copies)
     "fp8-row-pairs": W.custom(H=512, I=256, E=8, k=2),
     "fp8-block128": W.custom(H=512, I=256, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128),

@@ -31,6 +31,8 @@ CASES = {
     "row-split-boxes-t96": (W.custom(H=512, I=2048, E=4, k=2), 96),
     # T k >= 512 E: the gate/up GEMM runs on CTA pairs (odd row-tile counts included)
     "row-pairs-t2100": (W.custom(H=512, I=256, E=8, k=2), 2100),
+    # K = I = 2304 > 2048 as well: the down GEMM also runs on CTA pairs
+    "row-pairs-deepk-t2100": (W.custom(H=512, I=2304, E=8, k=2), 2100),
     # above 4 x 148 tokens the quantisation runs one warp per token
     "row-t700": (W.custom(H=256, I=128, E=8, k=2), 700),
     "block128-t700": (W.custom(H=256, I=128, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 700),
@@ -391,11 +393,13 @@ def test_launch_modes_same_bits(name):
     del g
 
 
-def test_cta_pairs_match_single_ctas():
-    """The gate/up GEMM on CTA pairs (M = 256 MMAs over two row tiles) gives the
-    hidden codes and the layer output of the single-CTA kernel, up to the fp32
-    summation order inside the tensor core."""
-    wl, T, d, x = build_case("row-pairs-t2100")
+@pytest.mark.parametrize("name", ["row-pairs-t2100", "row-pairs-deepk-t2100"])
+def test_cta_pairs_match_single_ctas(name):
+    """The GEMMs on CTA pairs (M = 256 MMAs over two row tiles; the gate/up GEMM,
+    and with K > 2048 the down GEMM too) give the hidden codes and the layer
+    output of the single-CTA kernels, up to the fp32 summation order inside
+    the tensor core."""
+    wl, T, d, x = build_case(name)
     layer = native.Layer(wl, d, max_T=T)
     xc, wr = x.cuda(), d["wr"].cuda()
     native.moe_set_gemm_options(layer.h, 1)
