@@ -9,7 +9,8 @@
 // their MX scale is the constant 1 (UE8M0 127), copied into TMEM once.
 //
 // Tile 128 padded rows x 256 columns, K stage 128 (one 512-byte scale chunk of
-// A per stage: 4 scales of 32 per row), 3 stages.  For small batches the K
+// A per stage: 4 scales of 32 per row), 3 to 5 stages (see the variants
+// below).  For small batches the K
 // range of each tile may be split S ways (S read from the dispatch's pick,
 // work item t = (tile t / S, split t % S)); split s writes its fp32 partial rows to copy s
 // of the output rows, o + s * A * H.  MMA j of a stage (K = 32)
