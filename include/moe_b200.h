@@ -230,7 +230,8 @@ moe_status moe_set_launch_options(moe_handle* h, int pdl);
  * tcgen05.mma.cta_group::2 covers two row tiles of one expert (M = 256), each
  * CTA loading its own 128 rows of X and half of the 256 weight rows (no
  * multicast), so a 32 KB stage feeds what a 48 KB stage feeds alone.  With
- * I > 2048 (FP8_ROW, any activation) the down GEMM runs on CTA pairs the same
+ * I > 2048 (FP8_ROW, any activation), and where the output rows leave no room
+ * for a K split of the down GEMM, the down GEMM runs on CTA pairs the same
  * way (each CTA loading its hidden rows, their scale chunk and 128 of the 256
  * rows of W_down).  An expert with an odd row-tile count runs its last pair
  * half empty.  The

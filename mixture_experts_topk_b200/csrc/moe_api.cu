@@ -760,8 +760,10 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     const uint8_t* pw = static_cast<const uint8_t*>(packed);
     // Large batches with deep K: CTA pairs (M = 256), each CTA loading 128 of a
     // tile's 256 B rows, when the experts average at least 4 row tiles (as for
-    // the gate/up GEMM); shallow K keeps single CTAs and the box stores.
-    const bool pairs = h->gemm_pairs && c.I / 128 > MX_BOX_MAX_KB && T * c.k >= 4 * TILE_M * c.E;
+    // the gate/up GEMM) and no K split can be chosen; shallow K keeps single
+    // CTAs and the box stores.
+    const bool pairs = h->gemm_pairs && c.I / 128 > MX_BOX_MAX_KB && T * c.k >= 4 * TILE_M * c.E &&
+                       split_limit(h->picker, T * c.k) == 1;
     CUtensorMap ta, tb, to, ts;
     moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
