@@ -22,8 +22,8 @@
  *     status word inside the workspace; moe_get_status() reports them.
  *   - One workspace per concurrent stream (LightMoE README, "MoE inference":
  *     one plan per concurrent CUDA stream, its workspaces are reused).
- *   - Shape limits (LightMoE README, "Limits": K aligned, at most 256 local
- *     experts, at most 131,072 token-expert assignments): H a multiple of 256,
+ *   - Shape limits (LightMoE README, "Limits", caps the experts of a layer at
+ *     256 and its token-expert pairs at 131,072, with K aligned): H a multiple of 256,
  *     I a multiple of 128, 1 <= k <= 8, k <= E <= 256, max_T * k <= 131072.
  *     Otherwise MOE_ERR_UNSUPPORTED_SHAPE.
  *   - moe_last_error() returns a thread-local message for the last failure.
