@@ -209,9 +209,9 @@ moe_status moe_gate_up(const moe_handle* h, const void* packed, int T, void* ws,
 moe_status moe_down(const moe_handle* h, const void* packed, const float* w, int T,
                     void* ws, moe_stream_t stream);
 
-/* Explicit tile choice of the down GEMM (LightMoE README, "Grouped GEMM": tile
- * choices stay explicit because the fastest geometry depends on the shape and
- * the expert assignment distribution).  down_bn: 0 = chosen per call, or 64,
+/* Explicit tile choice of the down GEMM (LightMoE README, "Grouped GEMM",
+ * leaves the tile configuration to the caller, since the best one varies with
+ * the matrix sizes and with how the assignments spread over experts).  down_bn: 0 = chosen per call, or 64,
  * 128, 256 output columns per tile.  Host state only. */
 moe_status moe_set_tile_config(moe_handle* h, int down_bn);
 

@@ -71,8 +71,9 @@ void orc_dispatch(const int32_t* ids, int T, int k, int E, int32_t* counts,
 int  orc_schedule(const int32_t* offsets, int E, int32_t* tile_expert, int32_t* tile_row);
 
 /* ---- down GEMM tile choice (wave cost model over the expert histogram) ----
- * RaMP abstract: a four-parameter wave cost model selects the configuration
- * from the runtime expert histogram and depends only on the CTA grid geometry.
+ * RaMP abstract: the configuration is picked from the expert histogram seen at
+ * run time by a cost model of CTA waves with four fitted parameters, which
+ * looks at nothing but the geometry of the CTA grid.
  * Candidates c = 0, 1, 2 have BN = 256, 128, 64 output columns per tile.  With
  * m_tiles = sum_e ceil(counts[e]/128) and touched = #{e : counts[e] > 0}:
  *   tiles  = m_tiles * (H / BN)
