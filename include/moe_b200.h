@@ -57,9 +57,12 @@ enum { MOE_SCORE_SOFTMAX = 0,    /* softmax over the selected k logits */
 /* quantisation format of weights, activations and hidden (Alpha-MoE article:
  * FP8 W8A8; LightMoE README, "Standalone GEMM": NVFP4 = E2M1 values, E4M3
  * block scales, one fp32 per-tensor scale) */
-enum { MOE_FMT_FP8_ROW = 0,      /* e4m3; fp32 scale per weight row / per token; hidden per (token, 128 cols) */
-       MOE_FMT_FP8_BLOCK128 = 1, /* e4m3; fp32 scale per 128x128 weight block / per (token, 128 cols) */
-       MOE_FMT_NVFP4 = 2 };      /* e2m1; e4m3 scale per 16 along K; fp32 global per tensor */
+enum { MOE_FMT_FP8_ROW = 0,      /* e4m3; fp32 scale per weight row and per token; the hidden with a
+                                    power-of-two (UE8M0) scale per 32 columns (MX) */
+       MOE_FMT_FP8_BLOCK128 = 1, /* e4m3; fp32 scale per 128x128 weight block, per (token, 128 cols) of X
+                                    and of the hidden */
+       MOE_FMT_NVFP4 = 2 };      /* e2m1; e4m3 scale per 16 along K; fp32 global per tensor (the hidden's
+                                    is the static hidden_global_scale) */
 
 typedef struct {
     int H, I, E, k;
@@ -112,7 +115,27 @@ typedef struct {
 } moe_weights;
 
 /* Device addresses of the intermediates inside a workspace (for inspection and
- * for feeding one step alone).  Row counts use A = max_T * k. */
+ * for feeding one step alone).  Row counts use A = max_T * k.
+ *
+ * Row layouts of xq/xs and hq/hs.  "Slot order": row = slot (the dispatch's
+ * expert-major position of an assignment), with 128 spare rows at the end.
+ * "Padded": every expert's rows start on a 128-row boundary, so that a row tile
+ * owns whole scale chunks: row = 128 * tile_ptr[e] + (slot - offsets[e]), with
+ * A + 128 E rows in all.  "Chunked" scale bytes: the scale of (row r, column
+ * block c) sits at byte ((r / 128) * (cols / 4) + c / 4) * 512
+ * + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4, cols = scale columns per row
+ * (the layout the block-scaled tensor-core MMAs read).
+ *   format        xq / xs                                hq / hs
+ *   FP8_ROW       slot order: [A+128, H] e4m3,            padded: [A+128E, I] e4m3,
+ *                 [A+128] fp32 per row                   chunked UE8M0 codes, I/32 per row
+ *                                                        (value = code * 2^(scale - 127))
+ *   FP8_BLOCK128  slot order: [A+128, H] e4m3,            slot order: [A+128, I] e4m3,
+ *                 [A+128, H/128] fp32                    [A+128, I/128] fp32
+ *   NVFP4         padded: [A+128E, H/2] e2m1 (2 per      padded: [A+128E, I/2] e2m1,
+ *                 byte, low nibble first), chunked e4m3  chunked e4m3 codes, I/16 per row
+ *                 codes, H/16 per row                    (x hidden_global_scale)
+ *                 (x the global scale amax|X| / 2688)
+ */
 typedef struct {
     int32_t* status;     /* [64] status[0] = first device error (moe_status), status[1] = where */
     int32_t* ids;        /* [A] router top-k expert ids, token-major [T, k] */
@@ -126,11 +149,11 @@ typedef struct {
     int32_t* tiles;      /* [A/128 + E + 1][2] (expert, first row) per row tile */
     int32_t* perm;       /* [A] slot -> t*k + j */
     int32_t* inv;        /* [A] t*k + j -> slot */
-    float*   x_global;   /* [1] NVFP4 global scale of X */
-    uint8_t* xq;         /* [A, H] e4m3 (NVFP4: [A, H/2]) quantised X rows in expert-major slot order */
-    void*    xs;         /* scales of xq: [A] fp32 | [A, H/128] fp32 | [A, H/16] e4m3 */
-    uint8_t* hq;         /* [A, I] (NVFP4: [A, I/2]) requantised hidden */
-    void*    hs;         /* scales of hq: [A, I/128] fp32 | [A, I/16] e4m3 */
+    float*   x_global;   /* [1] NVFP4: amax |X| over the batch (fp32); X's global scale is amax / 2688 */
+    uint8_t* xq;         /* quantised X rows, one per assignment (layout above) */
+    void*    xs;         /* scales of xq (layout above) */
+    uint8_t* hq;         /* requantised hidden, one row per assignment (layout above) */
+    void*    hs;         /* scales of hq (layout above) */
     float*   o;          /* [S][T*k, H] fp32 down projection times routing weight, slot order; with a K
                           * split (pick[1] = S > 1) copy s holds split s's partial sums.  FP8_ROW
                           * workspaces hold A + 7 min(A, 256) rows so small batches can split. */
@@ -185,10 +208,14 @@ moe_status moe_dispatch(const moe_handle* h, const void* x, const int32_t* ids, 
  *     perm [A], inv [A], xq [A, H] e4m3, xs [A] (FP8_ROW) or [A, H/128]
  *     (FP8_BLOCK128) fp32, status [2] (zeroed by the call, then status[0] =
  *     MOE_ERR_DEVICE_BOUNDS if an id was out of range).
- *   Same results as moe_dispatch.  T*k may not exceed 131072 and the format
- *   must be FP8 (else MOE_ERR_UNSUPPORTED_SHAPE).  The first call on a device
- *   looks up the array's device address; make that first call before any
- *   stream capture.  The array is shared by every call on the device and
+ *   Same results as moe_dispatch.  T*k may not exceed 131072, whatever E and
+ *   max_T are, and the format must be FP8 (else MOE_ERR_UNSUPPORTED_SHAPE).
+ *   Every call made outside stream capture looks up the array's device
+ *   address on the current device (so a cudaDeviceReset between calls is
+ *   harmless); a call under capture reuses the address of the last uncaptured
+ *   call on that device, so make the first call on a device before any stream
+ *   capture (a first call under capture returns MOE_ERR_INVALID_ARG).  The
+ *   array is shared by every call on the device and
  *   keeps the last call's contents, so calls whose kernels overlap on the GPU
  *   (other streams, other threads) race: serialise them.  No allocation. */
 moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, const int32_t* ids, int T,

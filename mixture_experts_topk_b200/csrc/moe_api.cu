@@ -1028,15 +1028,27 @@ static __device__ __align__(256) int32_t g_dispatch_scratch[NOALLOC_SCRATCH_INTS
 
 // Device address of g_dispatch_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
-static moe_status dispatch_scratch(int32_t** out) {
+// cudaGetSymbolAddress with that device current.  The lookup is repeated on
+// every call made outside stream capture (a host-side table lookup once the
+// module is loaded), so an address cached before a cudaDeviceReset, whose
+// context and module are then recreated, is never used afterwards.  Under
+// capture the address of the last uncaptured call on the device is used; the
+// first call on a device must therefore come before any capture.
+static moe_status dispatch_scratch(cudaStream_t st, int32_t** out) {
     static std::mutex mu;
     static int32_t* addr[64] = {nullptr};
     int dev = 0;
     CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return fail(MOE_ERR_CUDA, "moe_dispatch_noalloc: device index %d out of range", dev);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    CUDA_TRY(cudaStreamIsCapturing(st, &cap));
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone || !addr[dev]) {
+        if (cap != cudaStreamCaptureStatusNone)
+            return fail(MOE_ERR_INVALID_ARG,
+                        "moe_dispatch_noalloc: the first call on device %d is under stream capture; make one "
+                        "call before capturing",
+                        dev);
         void* p = nullptr;
         CUDA_TRY(cudaGetSymbolAddress(&p, g_dispatch_scratch));
         addr[dev] = static_cast<int32_t*>(p);
@@ -1054,6 +1066,11 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, c
     if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: T=%d is negative", T);
     const long long A = static_cast<long long>(T) * c.k;
     const long long nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
+    // the scan packs each count with its row-tile count into one int32, which
+    // holds for at most 131072 assignments whatever E is
+    if (A > 131072)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "moe_dispatch_noalloc: T*k=%lld assignments, more than the 131072 this entry point handles", A);
     if (nchunks * c.E > NOALLOC_SCRATCH_INTS)
         return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                     "moe_dispatch_noalloc: T*k=%lld assignments need %lld scratch counts, more than the %d "
@@ -1067,10 +1084,10 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, c
         return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: null argument");
     if (A > 0 && (!aligned256(x) || !aligned256(xq)))
         return fail(MOE_ERR_INVALID_ARG, "moe_dispatch_noalloc: x and xq must be 256-byte aligned");
-    int32_t* chunk = nullptr;
-    moe_status r = dispatch_scratch(&chunk);
-    if (r != MOE_OK) return r;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t* chunk = nullptr;
+    moe_status r = dispatch_scratch(st, &chunk);
+    if (r != MOE_OK) return r;
     CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int32_t), st));
     const int n = static_cast<int>(nchunks), a = static_cast<int>(A);
     // the histogram writes every count of every chunk it covers, so the

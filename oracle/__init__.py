@@ -45,7 +45,8 @@ class _Layer(ctypes.Structure):
                 ("hidden_global", ctypes.c_float),
                 ("gate", _Proj), ("up", _Proj), ("down", _Proj),
                 ("expert_slot", ctypes.c_void_p),
-                ("act", ctypes.c_int), ("act_alpha", ctypes.c_double), ("act_limit", ctypes.c_double)]
+                ("act", ctypes.c_int), ("act_alpha", ctypes.c_double), ("act_limit", ctypes.c_double),
+                ("hidden_rule", ctypes.c_int)]
 
 
 def lib():
@@ -214,8 +215,14 @@ def scale_shape(fmt, rows, K):
     return (rows, K // 16), np.uint8
 
 
-def hidden_fmt(fmt):
-    """Format of the requantised hidden: MX32 for FP8_ROW, otherwise the layer's own."""
+HIDDEN_LAYER, HIDDEN_PER_TOKEN = 0, 1
+
+
+def hidden_fmt(fmt, rule=HIDDEN_LAYER):
+    """Format of the requantised hidden: MX32 for FP8_ROW, otherwise the layer's
+    own; with the per-token reading (FP8 formats) one fp32 scale per row."""
+    if rule == HIDDEN_PER_TOKEN and fmt != FMT_NVFP4:
+        return FMT_FP8_ROW
     return FMT_MX32 if fmt == FMT_FP8_ROW else fmt
 
 
@@ -239,14 +246,16 @@ def nvfp4_global(x):
 class Layer:
     """Holds numpy copies of the quantised weights and the ctypes struct over them."""
 
-    def __init__(self, wl, weights, expert_slot=None):
+    def __init__(self, wl, weights, expert_slot=None, hidden_rule=HIDDEN_LAYER):
         self.wl = wl
+        self.hidden_rule = hidden_rule
         self._keep = {}
         st = _Layer()
         st.H, st.I, st.E, st.k = wl.H, wl.I, wl.E, wl.k
         st.score, st.fmt = wl.score, wl.fmt
         st.hidden_global = float(wl.hidden_global_scale)
         st.act, st.act_alpha, st.act_limit = wl.act, float(wl.act_alpha), float(wl.act_limit)
+        st.hidden_rule = hidden_rule
         for p in ("gate", "up", "down"):
             if weights.get(p + "_q") is None:      # ReLU^2 experts have no gate
                 setattr(st, p, _Proj(None, None, None))
@@ -281,7 +290,7 @@ class Layer:
         R = a_codes.shape[0]
         h = np.empty((R, wl.I), np.float64)
         hq = np.empty((R, code_bytes(wl.fmt, wl.I)), np.uint8)
-        shp, dt = scale_shape(hidden_fmt(wl.fmt), R, wl.I)
+        shp, dt = scale_shape(hidden_fmt(wl.fmt, self.hidden_rule), R, wl.I)
         hs = np.empty(shp, dt)
         o = np.empty((R, wl.H), np.float64)
         lib().orc_expert_rows(self.ref(), e, R, _p(a_codes), _p(a_scales), float(x_global),

@@ -236,9 +236,12 @@ int orc_pick_down_tile(const int32_t* counts, int E, int H, int I, int num_sms,
 
 /* K split of the down GEMM for small batches: S copies of the output rows, one
  * per near-equal range of K-blocks.  units = m_tiles * split_nb; the split is
- * bounded by 8, by the copies the output buffer holds (o_rows / A) and by at
- * least four K-blocks per range; S is the largest admissible s with
- * units * s <= num_sms, and 1 when split_nb is 0 or the batch is empty. */
+ * bounded by s_max = min(8, o_rows / A, split_kb / 4) (the copies the output
+ * buffer holds, at least four K-blocks per range).  With
+ * cost(s) = ceil(units * s / num_sms) * (840 / s), the time in rounds of 1/s
+ * of a unit, S is the s <= s_max of lowest cost (the smaller s on equal
+ * costs), taken only when that cost is at most 4/5 of cost(1); otherwise, and
+ * when split_nb is 0 or the batch is empty, S = 1. */
 int orc_pick_split(const int32_t* counts, int E, int split_nb, int split_kb, int64_t o_rows, int num_sms)
 {
     int64_t m_tiles = 0, A = 0;
@@ -370,11 +373,13 @@ static int64_t act_scale_bytes(int fmt, int K)
  * block scales: power-of-two scales per 32 columns (MX32, applied by the
  * tensor cores in the down projection) for FP8_ROW, fp32 scales per 128
  * columns (the 1x128 activation rule, like its X) for FP8_BLOCK128, and the
- * NVFP4 16-blocks with the static global scale for NVFP4. */
-static int hidden_fmt(int fmt)
+ * NVFP4 16-blocks with the static global scale for NVFP4.  The per-token
+ * reading (one fp32 scale per row, the FP8_ROW rule) is kept for comparison. */
+static int hidden_fmt(const orc_layer* L)
 {
-    if (fmt == ORC_FMT_FP8_ROW) return ORC_FMT_MX32;
-    return fmt;
+    if (L->hidden_rule == ORC_HIDDEN_PER_TOKEN && L->fmt != ORC_FMT_NVFP4) return ORC_FMT_FP8_ROW;
+    if (L->fmt == ORC_FMT_FP8_ROW) return ORC_FMT_MX32;
+    return L->fmt;
 }
 
 void orc_weight_row(const orc_layer* L, const orc_proj* P, int N, int K, int e, int n, double* out)
@@ -484,7 +489,7 @@ void orc_expert_rows(const orc_layer* L, int e, int rows, const uint8_t* a_codes
     }
     if (h) memcpy(h, hh, sizeof(double) * (size_t)rows * I);
     /* requantise the hidden: round to fp32, then the hidden's rule */
-    int hf_fmt = hidden_fmt(L->fmt);
+    int hf_fmt = hidden_fmt(L);
     float* hf = (float*)malloc(sizeof(float) * (size_t)rows * I);
     for (int64_t i = 0; i < (int64_t)rows * I; i++) hf[i] = (float)hh[i];
     uint8_t* qc = hq_codes ? hq_codes : (uint8_t*)malloc((size_t)(rows * row_code_bytes(hf_fmt, I)));
@@ -505,7 +510,7 @@ void orc_down_rows(const orc_layer* L, int e, int rows, const uint8_t* h_codes,
                    const void* h_scales, double* o)
 {
     double* hd = (double*)malloc(sizeof(double) * (size_t)rows * L->I);
-    dequant_rows(hidden_fmt(L->fmt), rows, L->I, h_codes, h_scales, L->hidden_global, hd);
+    dequant_rows(hidden_fmt(L), rows, L->I, h_codes, h_scales, L->hidden_global, hd);
     down_dequantised(L, e, rows, hd, o);
     free(hd);
 }

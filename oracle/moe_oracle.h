@@ -118,7 +118,17 @@ typedef struct {
     const int32_t* expert_slot; /* [E] -> index into the weight arrays, -1 = not provided; NULL = identity */
     int act;               /* gated activation, ORC_ACT_* */
     double act_alpha, act_limit;
+    int hidden_rule;       /* ORC_HIDDEN_*: how the hidden is requantised */
 } orc_layer;
+
+/* Requantisation rule of the hidden (the SwiGLU output).  The workloads ask
+ * for activations "dynamically quantised per token"; a GEMM epilogue that sees
+ * one block of hidden columns at a time cannot take a row's amax, so the layer
+ * uses block scales (ORC_HIDDEN_LAYER: MX32 for FP8_ROW, 1x128 fp32 for
+ * FP8_BLOCK128, NVFP4 16-blocks for NVFP4).  ORC_HIDDEN_PER_TOKEN is the
+ * literal reading, for comparison only (FP8 formats): one fp32 scale per
+ * hidden row, s = fp32(amax/448), q = e4m3(fp32(h/s)), the FP8_ROW rule of X. */
+enum { ORC_HIDDEN_LAYER = 0, ORC_HIDDEN_PER_TOKEN = 1 };
 
 /* Gated activations h = act(g, u) of the expert MLP, in fp64 (LightMoE README,
  * "Compatibility": SwiGLU, bounded SwiGLU, SwiGLU-OAI, GeGLU, ReGLU).
@@ -142,7 +152,8 @@ void orc_weight_row(const orc_layer* L, const orc_proj* P, int N, int K, int e, 
  *   The hidden is requantised with the MX32 rule (power-of-two scale per 32
  *   columns) for FP8_ROW, per (row, 128-column block) with fp32 scales for
  *   FP8_BLOCK128, and with the NVFP4 rule and the static hidden_global scale
- *   for NVFP4.
+ *   for NVFP4; with hidden_rule = ORC_HIDDEN_PER_TOKEN (FP8 formats) by the
+ *   FP8_ROW rule over the whole row (hq_scales then [rows] fp32).
  *   outputs: h (fp64 SwiGLU output before requantisation, [rows, I]) may be NULL;
  *            hq codes/scales (requantised hidden) may be NULL;
  *            o [rows, H] fp64 down projection of the dequantised hidden. */

@@ -214,3 +214,90 @@ def test_subset_forward_matches_full_forward():
     ids2, w2, y2 = Ls.forward(bf16_bits(x), d["wr"].numpy(), None, sel=sel)
     assert (ids2 == ids).all()
     assert (y2 == y[sel]).all()
+
+
+@pytest.mark.parametrize("fmt", [W.FMT_FP8_ROW, W.FMT_FP8_BLOCK128])
+def test_per_token_hidden_reading_is_the_row_rule_on_the_dense_mlp(fmt):
+    """The oracle-only per-token hidden (one fp32 scale per hidden row, the
+    FP8_ROW rule of X): with one expert and top-1, its codes and scales are
+    those of the row rule applied to the torch fp64 SwiGLU rounded to fp32,
+    and the output is their dequantised values through W_down."""
+    wl = W.custom(H=256, I=384, E=1, k=1, fmt=fmt)
+    d = synth.layer(wl, seed=15)
+    L = oracle.Layer(wl, d, hidden_rule=oracle.HIDDEN_PER_TOKEN)
+    x = synth.tokens(wl, 7, seed=15)
+    xf = x.to(torch.float32).numpy()
+    codes, scales = oracle.quant_rows(fmt, xf)
+    h, hq, hs, o = L.expert_rows(0, codes, scales)
+    assert hs.shape == (7,) and hs.dtype == np.float32
+    a = torch.from_numpy(deq_act(wl, codes, scales))
+    h_ref = torch.nn.functional.silu(a @ torch.from_numpy(deq_weight(wl, d, "gate", 0)).T) * \
+        (a @ torch.from_numpy(deq_weight(wl, d, "up", 0)).T)
+    np.testing.assert_allclose(h, h_ref.numpy(), rtol=1e-12, atol=1e-12)
+    hf = h_ref.numpy().astype(np.float32)
+    s_ref = np.abs(hf).max(axis=1) / np.float32(448.0)     # fp32 division, as the row rule
+    assert (hs == s_ref).all()
+    hq2, hs2 = oracle.quant_rows(W.FMT_FP8_ROW, hf)
+    assert (hs2 == hs).all()
+    assert (hq2 == hq).mean() > 0.999
+    o_ref = (fp8_val(hq) * hs.astype(np.float64)[:, None]) @ deq_weight(wl, d, "down", 0).T
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-12)
+
+
+# the FP8_ROW workloads at a few tokens each (only the experts those tokens use
+# are drawn)
+READING_CASES = [("tiny", 16), ("qwen3.5-35b-a3b", 6), ("mixtral-8x7b", 1)]
+
+
+@pytest.mark.parametrize("name,T", READING_CASES)
+def test_block_scaled_hidden_distance_from_per_token_reading(name, T):
+    """How far the layer's block-scaled hidden (MX32, a power-of-two scale per
+    32 columns) moves Y from the literal per-token reading of "activations
+    dynamically quantised per token".  Both round the same fp32 hidden to e4m3,
+    on different grids, so each hidden value moves by at most the sum of the
+    two half steps, and Y by at most sum_j |w_j| |W_down| |dh|; the measured
+    distance (elements outside the benchmark spec's tolerance when the per-token Y
+    is taken as the reference, the largest ratio to it, the relative rms) is
+    reported, and must stay inside that bound."""
+    wl = W.WORKLOADS[name]
+    x = synth.tokens(wl, T, seed=2)
+    wr, bias = synth.router(wl, seed=2)
+    lg = oracle.router_logits(bf16_bits(x), wr.numpy(), None if bias is None else bias.numpy())
+    ids, w = oracle.topk(lg, wl.k, wl.score)
+    used = sorted(set(ids.reshape(-1).tolist()))
+    slot = np.full(wl.E, -1, np.int32)
+    slot[used] = np.arange(len(used))
+    de = synth.experts(wl, seed=2, experts_subset=used)
+    sub = {k_: v[used] for k_, v in de.items() if v is not None}
+    b = None if bias is None else bias.numpy()
+    L_mx = oracle.Layer(wl, sub, expert_slot=slot)
+    L_pt = oracle.Layer(wl, sub, expert_slot=slot, hidden_rule=oracle.HIDDEN_PER_TOKEN)
+    _, _, y_mx = L_mx.forward(bf16_bits(x), wr.numpy(), b)
+    _, _, y_pt = L_pt.forward(bf16_bits(x), wr.numpy(), b)
+    rms = float(np.sqrt(np.mean(y_pt ** 2)))
+    tol = 2e-2 * np.abs(y_pt) + 2e-3 * rms
+    err = np.abs(y_mx - y_pt)
+    # the bound: per (t, j), |dh| <= half an e4m3 step of each grid at h
+    xq, xs = oracle.quant_rows(wl.fmt, x.to(torch.float32).numpy())
+    bound = np.zeros_like(y_pt)
+    for e in used:
+        rows = [(t, j) for t in range(T) for j in range(wl.k) if ids[t, j] == e]
+        tt = np.array([t for t, _ in rows])
+        h, hq_mx, hs_mx, _ = L_mx.expert_rows(e, xq[tt], xs[tt])
+        _, hq_pt, hs_pt, _ = L_pt.expert_rows(e, xq[tt], xs[tt])
+        v_mx = fp8_val(hq_mx) * np.repeat(np.exp2(hs_mx.astype(np.float64) - 127), 32, axis=1)
+        v_pt = fp8_val(hq_pt) * hs_pt.astype(np.float64)[:, None]
+        hf = h.astype(np.float32).astype(np.float64)
+        # half a step of e4m3 at |v| (2^-4 relative, or the subnormal step 2^-10 of the scale)
+        step_mx = np.maximum(np.abs(hf) * 2.0 ** -4, np.repeat(np.exp2(hs_mx.astype(np.float64) - 127), 32, axis=1)
+                             * 2.0 ** -10)
+        step_pt = np.maximum(np.abs(hf) * 2.0 ** -4, hs_pt.astype(np.float64)[:, None] * 2.0 ** -10)
+        assert np.all(np.abs(v_mx - v_pt) <= step_mx + step_pt + 1e-300)
+        wd = np.abs(deq_weight(wl, sub, "down", int(slot[e])))
+        dh = np.abs(v_mx - v_pt)
+        for r, (t, j) in enumerate(rows):
+            bound[t] += abs(w[t, j]) * (wd @ dh[r])
+    assert np.all(err <= bound * (1 + 1e-9) + 1e-300)
+    rec = {"case": f"{name} T={T}", "elements": int(y_pt.size), "outside_tolerance": int((err > tol).sum()),
+           "max_ratio": float(np.max(err / tol)), "rel_rms": float(np.sqrt(np.mean(err ** 2))) / rms}
+    print("HIDDEN_READING", rec)
