@@ -44,10 +44,13 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms for the whole
+    measurement; each sample keeps the host time it was read at, so that every
+    timed region gets the samples that fell inside it."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index):
         self.index = index
@@ -67,7 +70,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.rows.append([c.strip() for c in line.split(",")])
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -77,18 +80,37 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        sm = [float(r[1]) for r in self.rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+    def summary(self, t0=None, t1=None):
+        rows = [r for t, r in self.rows if (t0 is None or t >= t0) and (t1 is None or t <= t1) and len(r) >= 9]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in self.rows:
-            if len(r) >= 9:
-                for n, v in zip(names, r[5:9]):
-                    if v.strip().lower() == "active":
-                        reasons.add(n)
+        for r in rows:
+            for n, v in zip(self.REASONS, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class Regions:
+    """Host-time windows of the timed regions, for the clock samples."""
+
+    def __init__(self):
+        self.spans = {}
+
+    def __call__(self, name):
+        reg = self
+
+        class _Span:
+            def __enter__(self):
+                torch.cuda.synchronize()
+                self.t0 = time.time()
+
+            def __exit__(self, *a):
+                torch.cuda.synchronize()
+                reg.spans[name] = (self.t0, time.time())
+        return _Span()
 
 
 def gemm_traffic(workload, T):
@@ -157,23 +179,35 @@ def workload_of(args):
     return dataclasses.replace(wl, act=act, act_alpha=alpha, act_limit=limit)
 
 
-def run_ours(args, rank, world, local_rank):
-    from mixture_experts_topk_b200 import native
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    wl = workload_of(args)
-    T = args.tokens
-    d = synth.layer(wl, seed=0, device=dev)
-    layer = native.Layer(wl, d, max_T=T, device=dev)
-    if args.down_bn:
-        native.moe_set_tile_config(layer.h, args.down_bn)
-    wr = d["wr"]
-    bias = d["bias"]
-    del d                      # the packed copy is all the layer reads
-    torch.cuda.empty_cache()
-    x = synth.tokens(wl, T, seed=rank, device=dev)
+def tensor_peaks(wl, pk):
+    """Dense tensor peaks of the layer's format in TFLOP/s: (burst, sustained).
+    fp8 = 2 x and fp4 = 4 x the measured bf16 figures (nominal ratios)."""
+    r = 4.0 if wl.fmt == FMT_NVFP4 else 2.0
+    return r * pk["bf16_tflops"], r * pk["bf16_tflops_sustained"]
+
+
+def launches_per_step(wl, T):
+    """Kernels of one moe_forward call: router (logits + top-k; one fused kernel
+    for T <= 128 and E <= 32; above 128 tokens with more than 8 experts the
+    fixed-point rows, the integer tensor-core pass and the candidate select),
+    dispatch (hist, scan, rank, quantise; one fused kernel for the first three
+    when T*k <= 1024; + amax for NVFP4), gate/up, down, combine."""
+    if T <= 128:
+        route = 1 if wl.E <= 32 else 2
+    else:
+        route = 3 if wl.E > 8 else 2
+    return route + (2 if T * wl.k <= 1024 else 4) + (1 if wl.fmt == FMT_NVFP4 else 0) + 3
+
+
+def measure(native, layer, wl, T, x, wr, bias, args, world, dev, clk, e2e=True, min_region_s=0.5):
+    """One workload point: graph-replayed steps, per-kernel events and (when
+    e2e) the end-to-end steps fed from pinned host memory.  Every region runs
+    at least min_region_s of the same work (untimed pre-roll for the step and
+    e2e regions, more iterations for the per-kernel region), so that the
+    clock sampler sees it under load; each region reports its own clocks."""
     y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
+    regions = Regions()
 
     def call():
         native.moe_forward(layer.h, x, T, wr, bias, layer.packed, y, layer.ws)
@@ -199,25 +233,24 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status after warm-up: {msg}")
     counts = layer.region("counts", torch.int32, wl.E).cpu().numpy()
     m_tiles = int(layer.region("num_tiles", torch.int32, 1).item())
-    pick = int(layer.region("pick", torch.int32, 1).item())
+    pick = layer.region("pick", torch.int32, 2).cpu().tolist()
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    # ---- device-timed steps (inputs already resident).  The clock sampler
-    # starts first and ~0.5 s of untimed steps run before the timed ones, so
-    # samples land under load even when the timed region itself is short.
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(3):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    preroll = max(1, int(math.ceil(0.5 / max(ev0.elapsed_time(ev1) / 3e3, 1e-6))))
-    with ClockSampler(local_rank) as clk:
-        time.sleep(0.2)
-        for _ in range(preroll):
+    est_ms = max(ev0.elapsed_time(ev1) / 3, 1e-3)
+    fill = max(1, int(math.ceil(min_region_s * 1e3 / est_ms)))
+
+    # ---- device-timed steps (inputs already resident), after an untimed pre-roll
+    with regions("steps"):
+        for _ in range(fill):
             step()
         barrier()
         torch.cuda.synchronize()
@@ -232,87 +265,182 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status after the timed steps: {msg}")
 
-    # ---- per-kernel durations of the same steps (events between the C-ABI calls)
-    v = layer.view
+    # ---- per-kernel durations (events between the C-ABI calls), averaged over
+    # enough calls to fill the region
     ids_t = layer.region("ids", torch.int32, T * wl.k)
     w_t = layer.region("w", torch.float32, T * wl.k)
     names = ["route", "dispatch", "gate_up", "down", "combine"]
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for s in range(args.steps):
-        e = evs[s]
-        e[0].record(stream)
-        native.moe_route(layer.h, x, T, wr, bias, ids_t, w_t, layer.ws)
-        e[1].record(stream)
-        native.moe_dispatch(layer.h, x, ids_t, T, layer.ws)
-        e[2].record(stream)
-        native.moe_gate_up(layer.h, layer.packed, T, layer.ws)
-        e[3].record(stream)
-        native.moe_down(layer.h, layer.packed, w_t, T, layer.ws)
-        e[4].record(stream)
-        native.moe_combine(layer.h, T, y, layer.ws)
-        e[5].record(stream)
-    torch.cuda.synchronize()
-    per = {n: sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps
+    n_k = max(args.steps, fill)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(n_k)]
+    with regions("kernels"):
+        for s_ in range(n_k):
+            e = evs[s_]
+            e[0].record(stream)
+            native.moe_route(layer.h, x, T, wr, bias, ids_t, w_t, layer.ws)
+            e[1].record(stream)
+            native.moe_dispatch(layer.h, x, ids_t, T, layer.ws)
+            e[2].record(stream)
+            native.moe_gate_up(layer.h, layer.packed, T, layer.ws)
+            e[3].record(stream)
+            native.moe_down(layer.h, layer.packed, w_t, T, layer.ws)
+            e[4].record(stream)
+            native.moe_combine(layer.h, T, y, layer.ws)
+            e[5].record(stream)
+    per = {n: sum(evs[s_][i].elapsed_time(evs[s_][i + 1]) for s_ in range(n_k)) / n_k
            for i, n in enumerate(names)}
 
-    # ---- end to end through the public call with host buffers: every step
-    # copies its X from pinned host memory and its Y back to pinned host
-    # memory.  Copies run on their own streams, double-buffered, so step i's
-    # copies overlap the layer of steps i-1 / i+1 (a serving loop's pipeline).
-    x_host = x.cpu().pin_memory()
-    y_host = [torch.empty(T, wl.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    x_dev = [torch.empty_like(x) for _ in range(2)]
-    y_dev = [torch.empty_like(y) for _ in range(2)]
-    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    out = {"ms_max": ms_max, "counts": counts, "m_tiles": m_tiles, "pick": pick, "kernel_ms": per,
+           "graph": graph is not None, "regions": regions}
+    if e2e:
+        # end to end through the public call with host buffers: every step
+        # copies its X from pinned host memory and its Y back to pinned host
+        # memory.  Copies run on their own streams, double-buffered, so step i's
+        # copies overlap the layer of steps i-1 / i+1 (a serving loop's pipeline).
+        x_host = x.cpu().pin_memory()
+        y_host = [torch.empty(T, wl.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        x_dev = [torch.empty_like(x) for _ in range(2)]
+        y_dev = [torch.empty_like(y) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-    def e2e_steps(n, ev_first=None, ev_last=None):
-        done_in = [torch.cuda.Event() for _ in range(n)]
-        done_fw = [torch.cuda.Event() for _ in range(n)]
-        done_out = [torch.cuda.Event() for _ in range(n)]
-        if ev_first is not None:
-            ev_first.record(s_in)
-        for i in range(n):
-            b = i & 1
-            with torch.cuda.stream(s_in):
+        def e2e_steps(n, ev_first=None, ev_last=None):
+            done_in = [torch.cuda.Event() for _ in range(n)]
+            done_fw = [torch.cuda.Event() for _ in range(n)]
+            done_out = [torch.cuda.Event() for _ in range(n)]
+            if ev_first is not None:
+                ev_first.record(s_in)
+            for i in range(n):
+                b = i & 1
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(done_fw[i - 2])          # x_dev[b] free again
+                    x_dev[b].copy_(x_host, non_blocking=True)
+                    done_in[i].record(s_in)
+                stream.wait_event(done_in[i])
                 if i >= 2:
-                    s_in.wait_event(done_fw[i - 2])          # x_dev[b] free again
-                x_dev[b].copy_(x_host, non_blocking=True)
-                done_in[i].record(s_in)
-            stream.wait_event(done_in[i])
-            if i >= 2:
-                stream.wait_event(done_out[i - 2])           # y_dev[b] read back already
-            native.moe_forward(layer.h, x_dev[b], T, wr, bias, layer.packed, y_dev[b], layer.ws)
-            done_fw[i].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(done_fw[i])
-                y_host[b].copy_(y_dev[b], non_blocking=True)
-                done_out[i].record(s_out)
-        if ev_last is not None:
-            s_out.wait_stream(s_in)
-            ev_last.record(s_out)
+                    stream.wait_event(done_out[i - 2])           # y_dev[b] read back already
+                native.moe_forward(layer.h, x_dev[b], T, wr, bias, layer.packed, y_dev[b], layer.ws)
+                done_fw[i].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(done_fw[i])
+                    y_host[b].copy_(y_dev[b], non_blocking=True)
+                    done_out[i].record(s_out)
+            if ev_last is not None:
+                s_out.wait_stream(s_in)
+                ev_last.record(s_out)
 
-    e2e_steps(2)
-    torch.cuda.synchronize()
-    barrier()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    e2e_steps(args.steps, ev0, ev1)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        e2e_steps(2)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with regions("e2e"):
+            e2e_steps(fill)
+            torch.cuda.synchronize()
+            barrier()
+            e2e_steps(args.steps, e0, e1)
+            torch.cuda.synchronize()
+            barrier()
+        out["e2e_ms"] = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        out["h2d"] = int(x.numel() * 2)
+        out["d2h"] = int(y.numel() * 2)
+    del graph
+    return out
 
+
+def region_clocks(clk, regions, ms_of):
+    """Per timed region: its median SM clock and its time per step scaled to the
+    largest SM clock (ms x median MHz / max MHz), so regions that ran at
+    different power-capped clocks can be compared."""
+    res = {}
+    for name, (t0, t1) in regions.spans.items():
+        c = clk.summary(t0, t1)
+        ms = ms_of.get(name)
+        if ms is not None and c["sm_mhz"] and c["sm_max_mhz"]:
+            c["ms_per_step"] = ms
+            c["ms_at_max_clock"] = ms * c["sm_mhz"] / c["sm_max_mhz"]
+        res[name] = c
+    return res
+
+
+def roofline_numbers(wl, T, counts, step_ms, gu_ms, pk):
+    """Layer roofline and the gate/up GEMM's fraction of the tensor peak, both
+    against the burst and the sustained measured peaks."""
     fl_t, fl_r, byts, touched = algorithmic_work(wl, T, counts)
-    pk, pk_kind = peaks()
-    # dense fp8 = 2 x bf16 and fp4 = 4 x bf16 (nominal ratios) of the measured bf16 figure
-    fp8_peak = (4.0 if wl.fmt == FMT_NVFP4 else 2.0) * pk["bf16_tflops_sustained"]
+    burst, sustained = tensor_peaks(wl, pk)
+    simt_peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6   # fp32 FMA lanes x 2 x max clock
+
+    def t_roof(tp):
+        return max(fl_t / (tp * 1e12) + fl_r / simt_peak, byts / (pk["hbm_gbs"] * 1e9)) * 1e3
+
     gu_flops = 2.0 * T * wl.k * (n_proj(wl) - 1) * wl.H * wl.I
-    gu_ms = per["gate_up"]
     achieved = gu_flops / (gu_ms * 1e-3) / 1e12
+    return {"flops_tensor": fl_t, "flops_router": fl_r, "bytes": byts, "touched": touched,
+            "t_roof_ms": t_roof(burst), "frac": t_roof(burst) / step_ms,
+            "frac_sustained": t_roof(sustained) / step_ms,
+            "bound": "tensor" if fl_t / (burst * 1e12) > byts / (pk["hbm_gbs"] * 1e9) else "hbm",
+            "gu_achieved": achieved, "gu_frac": achieved / burst, "gu_frac_sustained": achieved / sustained,
+            "burst": burst, "sustained": sustained}
+
+
+# every (workload, T) point the layer is benchmarked on
+SWEEP = [(name, T) for name, wl in WORKLOADS.items() for T in wl.tokens]
+
+
+def per_workload_sweep(native, args, dev, clk, pk):
+    """All (workload, T) points in this invocation: ms/step, layer roofline
+    fraction, gate/up fraction and clocks for each."""
+    res = []
+    for name, wl in WORKLOADS.items():
+        d = synth.layer(wl, seed=0, device=dev)
+        for T in wl.tokens:
+            layer = native.Layer(wl, d, max_T=T, device=dev)
+            x = synth.tokens(wl, T, seed=0, device=dev)
+            m = measure(native, layer, wl, T, x, d["wr"], d["bias"], args, 1, dev, clk, e2e=False,
+                        min_region_s=0.25)
+            step_ms = m["ms_max"] / args.steps
+            rf = roofline_numbers(wl, T, m["counts"], step_ms, m["kernel_ms"]["gate_up"], pk)
+            rc = region_clocks(clk, m["regions"], {"steps": step_ms,
+                                                   "kernels": sum(m["kernel_ms"].values())})
+            res.append({"workload": f"{name} T={T}", "ms_per_step": step_ms, "tokens_per_s": T / (step_ms * 1e-3),
+                        "bound": rf["bound"], "layer_roofline_frac": rf["frac"],
+                        "layer_roofline_frac_sustained": rf["frac_sustained"],
+                        "gate_up_frac": rf["gu_frac"], "gate_up_frac_sustained": rf["gu_frac_sustained"],
+                        "kernel_ms": m["kernel_ms"], "touched_experts": rf["touched"],
+                        "clocks": rc.get("steps"), "kernel_clocks": rc.get("kernels")})
+            layer.close()
+            del x
+        del d
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args, rank, world, local_rank):
+    from mixture_experts_topk_b200 import native
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workload_of(args)
+    T = args.tokens
+    d = synth.layer(wl, seed=0, device=dev)
+    layer = native.Layer(wl, d, max_T=T, device=dev)
+    if args.down_bn:
+        native.moe_set_tile_config(layer.h, args.down_bn)
+    wr = d["wr"]
+    bias = d["bias"]
+    del d                      # the packed copy is all the layer reads
+    torch.cuda.empty_cache()
+    x = synth.tokens(wl, T, seed=rank, device=dev)
+    pk, pk_kind = peaks()
+    with ClockSampler(local_rank) as clk:
+        time.sleep(0.2)
+        m = measure(native, layer, wl, T, x, wr, bias, args, world, dev, clk)
+        layer.close()
+        sweep = None
+        if world == 1 and not args.no_per_workload:
+            sweep = per_workload_sweep(native, args, dev, clk, pk)
+    ms_max = m["ms_max"]
     step_ms = ms_max / args.steps
-    # fp32 SIMT peak of the router: 148 SMs x 128 FMA lanes x 2 FLOP x max SM clock
-    simt_peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6
-    t_roof_ms = max(fl_t / (fp8_peak * 1e12) + fl_r / simt_peak, byts / (pk["hbm_gbs"] * 1e9)) * 1e3
+    per = m["kernel_ms"]
+    rf = roofline_numbers(wl, T, m["counts"], step_ms, per["gate_up"], pk)
+    e2e_step_ms = m["e2e_ms"] / args.steps
+    clocks = region_clocks(clk, m["regions"], {"steps": step_ms, "kernels": sum(per.values()), "e2e": e2e_step_ms})
     out = {
         "metric": METRIC,
         "value": job_throughput(T, args.steps, world, ms_max),
@@ -328,35 +456,37 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded; X ~ N(0,1) bf16, weights ~ N(0,1/fan_in) quantised offline)",
         "config": {"workload": f"{wl.name} T={T}", "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "activation": args.act,
                    "T_per_gpu": T, "parallelism": f"replicas x{world} (token batches)",
-                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (byts / 1e9),
-                   "touched_experts": touched, "m_tiles": m_tiles,
-                   "launch": "CUDA graph of one moe_forward call, replayed per step" if graph is not None
+                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (rf["bytes"] / 1e9),
+                   "touched_experts": rf["touched"], "m_tiles": m["m_tiles"],
+                   "launch": "CUDA graph of one moe_forward call, replayed per step" if m["graph"]
                              else "moe_forward per step",
-                   "down_tile": args.down_bn or {0: 256, 1: 128, 2: 64}[pick],
-                   "down_tile_source": "fixed" if args.down_bn else "picked from the histogram"},
-        "tflops": (fl_t + fl_r) * world * args.steps / (ms_max * 1e-3) / 1e12,
-        "layer_roofline": {"t_roof_ms": t_roof_ms, "frac": t_roof_ms / step_ms,
+                   "down_tile": args.down_bn or {0: 256, 1: 128, 2: 64}[m["pick"][0]],
+                   "down_tile_source": "fixed" if args.down_bn else "picked from the histogram",
+                   "down_k_split": m["pick"][1]},
+        "tflops": (rf["flops_tensor"] + rf["flops_router"]) * world * args.steps / (ms_max * 1e-3) / 1e12,
+        "layer_roofline": {"t_roof_ms": rf["t_roof_ms"], "frac": rf["frac"], "frac_sustained": rf["frac_sustained"],
+                           "bound": rf["bound"],
                            "model": "max(tensor FLOPs / P_tensor + router FLOPs / P_fp32, algorithmic bytes / HBM)",
-                           "peaks": f"{pk_kind}: tensor = (2 fp8 | 4 fp4) x bf16_tflops_sustained, hbm_gbs; "
-                                    "P_fp32 = 148 SMs x 128 lanes x 2 x sm_max_mhz"},
+                           "peaks": f"{pk_kind}: P_tensor = (2 fp8 | 4 fp4) x bf16_tflops (burst; frac_sustained: "
+                                    "x bf16_tflops_sustained), hbm_gbs; P_fp32 = 148 SMs x 128 lanes x 2 x sm_max_mhz"},
         "roofline": {"kernel": "grouped_gemm gate/up (SwiGLU + requant epilogue)", "bound": "tensor",
-                     "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": achieved / fp8_peak, "traffic": gemm_traffic(args.workload, T),
-                     "algorithmic_bytes": int(T * wl.k * wl.H + (n_proj(wl) - 1) * wl.I * wl.H * touched + T * wl.k * wl.I),
-                     "peak_source": f"{pk_kind} bf16_tflops_sustained x {4 if wl.fmt == FMT_NVFP4 else 2} "
-                                    "(nominal fp8:bf16 = 2, fp4:bf16 = 4)"},
+                     "achieved": rf["gu_achieved"], "peak": rf["burst"], "unit": "TFLOP/s",
+                     "frac": rf["gu_frac"], "frac_sustained": rf["gu_frac_sustained"],
+                     "traffic": gemm_traffic(args.workload, T),
+                     "algorithmic_bytes": int(T * wl.k * wl.H + (n_proj(wl) - 1) * wl.I * wl.H * rf["touched"]
+                                              + T * wl.k * wl.I),
+                     "peak_source": f"{pk_kind} bf16_tflops (burst: the kernel is timed call by call) x "
+                                    f"{4 if wl.fmt == FMT_NVFP4 else 2} (nominal fp8:bf16 = 2, fp4:bf16 = 4); "
+                                    "frac_sustained uses bf16_tflops_sustained"},
         "kernel_ms": per,
-        "e2e": {"value": job_throughput(T, args.steps, world, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2)},
-        # router (logits + top-k; one fused kernel for T <= 128 and E <= 32) + dispatch
-        # (hist, scan, rank, quantise; one fused kernel for the first three when
-        # T*k <= 1024; + amax for NVFP4) + gate/up + down + combine
-        "gpu_launches": ((1 if (T <= 128 and wl.E <= 32) else 2) + (2 if T * wl.k <= 1024 else 4)
-                         + (1 if wl.fmt == FMT_NVFP4 else 0) + 3) * args.steps,
-        "clocks": clk.summary(),
+        "e2e": {"value": job_throughput(T, args.steps, world, m["e2e_ms"]), "unit": "tokens/s",
+                "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"], "ms_per_step": e2e_step_ms},
+        "gpu_launches": launches_per_step(wl, T) * args.steps,
+        "clocks": clocks.get("steps"),
+        "region_clocks": clocks,
     }
-    del graph
-    layer.close()
+    if sweep is not None:
+        out["per_workload"] = sweep
     return out
 
 
@@ -415,6 +545,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-sample", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the sweep over every (workload, T) point (done at N = 1 only)")
     ap.add_argument("--down-bn", type=int, default=0, help="down GEMM tile width (0 = chosen per call)")
     ap.add_argument("--act", default="swiglu", choices=sorted(ACTS),
                     help="gated activation of the expert MLP (bounded: clamp 10; oai: alpha 1.702, limit 7)")

@@ -154,10 +154,15 @@ typedef struct {
     void*    xs;         /* scales of xq (layout above) */
     uint8_t* hq;         /* requantised hidden, one row per assignment (layout above) */
     void*    hs;         /* scales of hq (layout above) */
-    float*   o;          /* [S][T*k, H] fp32 down projection times routing weight, slot order; with a K
-                          * split (pick[1] = S > 1) copy s holds split s's partial sums.  FP8_ROW
-                          * workspaces hold A + 7 min(A, 256) rows so small batches can split. */
-    float*   logits;     /* [max_T, E] fp32 router logits (bias included) of the last moe_route */
+    uint16_t* o;         /* [S][T*k, H] fp16 down projection times routing weight, slot order, each
+                          * 32-column block scaled by 2^(15 - o_exp): value = fp16 * 2^(o_exp - 15).
+                          * With a K split (pick[1] = S > 1) copy s holds split s's partial sums.
+                          * FP8_ROW workspaces hold A + 7 min(A, 256) rows so small batches can split. */
+    float*   logits;     /* [max_T, E] fp32 router logits (bias included) of the last moe_route: the
+                          * canonical logit for every expert that could be among a token's top k (all
+                          * experts up to 128 tokens or with at most 8 experts); above that, the
+                          * integer tensor-core approximation for the others (router_tc.cuh) */
+    int8_t*  o_exp;      /* [S][T*k, H/32] the block exponents of o */
 } moe_workspace_view;
 
 const char* moe_last_error(void);

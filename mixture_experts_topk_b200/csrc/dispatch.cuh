@@ -455,54 +455,67 @@ __global__ void __launch_bounds__(256) quant_scatter_row_kernel(const __nv_bfloa
 }
 
 // y[t] = bf16(sum_j sum_s o[s][inv[t k + j]]) in fixed (j, s) order with fp32
-// accumulation; o holds fp32 rows (weight already applied) in S copies of A
-// rows when the down GEMM split its K (S from the dispatch's pick, clamped to
-// [1, s_max]), so the only rounding to bf16 is the final one.
-__global__ void __launch_bounds__(128) combine_kernel(const float* o, const int32_t* inv, int T, int H, int k,
-                                                      const int32_t* split, int s_max, __nv_bfloat16* y) {
+// accumulation.  o holds the down GEMM's weighted rows in fp16 with a power-of-
+// two scale per 32 columns (value = fp16 * 2^(oe - 15), exact in fp32), in S
+// copies of A rows when the down GEMM split its K (S from the dispatch's pick,
+// clamped to [1, s_max]), so the only rounding to bf16 is the final one.
+// A thread takes 16 columns (32 bytes of each row, one exponent), so that the
+// k rows' loads in flight per thread are as many bytes as with fp32 rows.
+constexpr int COMBINE_COLS = 16;
+constexpr int COMBINE_THREADS = 128;
+__global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const uint16_t* o, const int8_t* oe,
+                                                                  const int32_t* inv, int T, int H, int k,
+                                                                  const int32_t* split, int s_max, __nv_bfloat16* y) {
     pdl_wait();
     pdl_trigger();
     KTRACE(TR_COMBINE);
     const int S = split ? min(max(*split, 1), s_max) : 1;
-    const size_t copy = static_cast<size_t>(T) * k * H;
-    // CTA (x, y): tokens x, x + gridDim.x, ..., columns [1024 y, 1024 y + 1024)
-    const int c_end = min(H, 1024 * (static_cast<int>(blockIdx.y) + 1));
+    const size_t copy = static_cast<size_t>(T) * k;   // rows per copy
+    const int HB = H >> 5;                            // exponent bytes per row
+    constexpr int SPAN = COMBINE_COLS * COMBINE_THREADS;
+    // CTA (x, y): tokens x, x + gridDim.x, ..., columns [SPAN y, SPAN y + SPAN)
+    const int c_end = min(H, SPAN * (static_cast<int>(blockIdx.y) + 1));
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         int slot[8];
 #pragma unroll
         for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
-        for (int c0 = 1024 * blockIdx.y + 8 * threadIdx.x; c0 < c_end; c0 += 8 * blockDim.x) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c0 = SPAN * blockIdx.y + COMBINE_COLS * threadIdx.x; c0 < c_end; c0 += SPAN) {
+            float acc[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) acc[i] = 0.0f;
+            auto add_row = [&](size_t row) {
+                const uint4* src = reinterpret_cast<const uint4*>(o + row * H + c0);
+                const uint4 q0 = src[0], q1 = src[1];
+                const float sc = __int_as_float((127 - 15 + oe[row * HB + (c0 >> 5)]) << 23);
+                const uint32_t wq[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wq[i]));
+                    acc[2 * i] += f.x * sc;
+                    acc[2 * i + 1] += f.y * sc;
+                }
+            };
             if (S == 1) {
                 // all k rows' loads in flight at once
 #pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    if (slot[j] < 0) continue;
-                    const float4* src = reinterpret_cast<const float4*>(o + static_cast<size_t>(slot[j]) * H + c0);
-                    const float4 a = src[0], b = src[1];
-                    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-                    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-                }
+                for (int j = 0; j < 8; j++)
+                    if (slot[j] >= 0) add_row(static_cast<size_t>(slot[j]));
             } else {
 #pragma unroll
                 for (int j = 0; j < 8; j++) {
                     if (slot[j] < 0) continue;
-                    const float* row = o + static_cast<size_t>(slot[j]) * H + c0;
-                    for (int sp = 0; sp < S; sp++) {
-                        const float4* src = reinterpret_cast<const float4*>(row + sp * copy);
-                        const float4 a = src[0], b = src[1];
-                        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-                        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-                    }
+                    for (int sp = 0; sp < S; sp++) add_row(static_cast<size_t>(sp) * copy + slot[j]);
                 }
             }
-            uint32_t r[4];
+            uint32_t r[8];
 #pragma unroll
-            for (int q = 0; q < 4; q++) {
+            for (int q = 0; q < 8; q++) {
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
                 r[q] = *reinterpret_cast<const uint32_t*>(&b2);
             }
-            *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + c0) = make_uint4(r[0], r[1], r[2], r[3]);
+            uint4* dst = reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + c0);
+            dst[0] = make_uint4(r[0], r[1], r[2], r[3]);
+            dst[1] = make_uint4(r[4], r[5], r[6], r[7]);
         }
     }
 }

@@ -62,7 +62,8 @@ struct GemmParams {
     int32_t* gu_done;           // FP8_ROW gate/up: per-expert count of finished (tile, epilogue warp)
                                 //   parts, for a down GEMM that starts before this kernel ends
     float act_alpha, act_limit;
-    float* o;                   // down: [A][H] fp32
+    uint16_t* o;                // down: [A][H] fp16 rows with block exponents oe
+    int8_t* oe;                 //   [A][H / 32]
     int H;
     const int32_t* perm;        // down: slot -> t*k + j
     const float* route_w;       // down: [T*k]
@@ -147,6 +148,101 @@ __device__ __forceinline__ void store_rows_coalesced(const float (&v)[NC], float
             }
         }
         __syncwarp();
+    }
+}
+
+// ------------------------------------------------------------------ fp16 output rows
+// The down GEMMs store each weighted output row (slot order) in fp16 with a
+// power-of-two scale per 32 columns: a block's values v are stored as
+// fp16(v 2^(15 - e)), e the binary exponent of the block's largest |v|
+// (amax < 2^e, clamped to [-110, 127]), and e in one signed byte.  The scaled
+// largest value is below 2^15, so nothing overflows, and every value keeps the
+// 11 significant bits of fp16 relative to its block's largest (a fifth of a
+// bf16 rounding).  The combine reads them back as fp16 2^(e - 15) and adds the
+// k rows (and K-split copies) in fixed order in fp32.
+__device__ __forceinline__ int o16_exponent(float amax) {
+    // amax = 1.m 2^(E - 127) < 2^(E - 126); 0 and subnormals clamp to -110
+    const int e = ((__float_as_int(amax) >> 23) & 0xFF) - 126;
+    return e < -110 ? -110 : (e > 127 ? 127 : e);
+}
+__device__ __forceinline__ float pow2f(int k) { return __int_as_float((127 + k) << 23); }   // k in [-126, 127]
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+// one 32-column block of this lane's row: (v * cs) * rs (or v * rs) rounded to
+// fp32 as before, its exponent, and the 16 words of fp16 pairs
+template <bool HAS_CS>
+__device__ __forceinline__ int o16_block(const float* v, const float* cs, float rs, uint32_t (&w)[16]) {
+    float val[32];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c4 = 0; c4 < 8; c4++) {
+        float4 s4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        if (HAS_CS) s4 = __ldg(reinterpret_cast<const float4*>(cs + 4 * c4));
+        const float sc[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int c = 4 * c4 + i;
+            val[c] = HAS_CS ? v[c] * sc[i] * rs : v[c] * rs;
+            amax = fmaxf(amax, fabsf(val[c]));
+        }
+    }
+    const int e = o16_exponent(amax);
+    const float up = pow2f(15 - e);
+#pragma unroll
+    for (int c = 0; c < 16; c++) w[c] = pack_h2(val[2 * c] * up, val[2 * c + 1] * up);
+    return e;
+}
+
+// Store this lane's NC output columns as fp16 rows with block exponents
+// (dst: the row's first fp16, dst_e: its first exponent byte; null when the
+// row is not stored).  32-column blocks pass through the per-warp [32][20]-word
+// staging so each store instruction writes 8 rows x 64 contiguous bytes; warps
+// with at most 8 stored rows store their rows directly.
+template <int NC, bool HAS_CS>
+__device__ __forceinline__ void store_rows16(const float (&v)[NC], uint32_t* stg, uint16_t* dst, int8_t* dst_e,
+                                             const float* cs, float rs, int lane) {
+    static_assert(NC % 32 == 0 && NC <= 128, "whole 32-column blocks, at most 4 exponent bytes");
+    uint32_t ebytes = 0;
+    if (__popc(__ballot_sync(0xffffffffu, dst != nullptr)) <= 8) {
+        if (dst != nullptr) {
+#pragma unroll
+            for (int b = 0; b < NC / 32; b++) {
+                uint32_t w[16];
+                const int e = o16_block<HAS_CS>(v + 32 * b, HAS_CS ? cs + 32 * b : nullptr, rs, w);
+                ebytes |= (static_cast<uint32_t>(e) & 0xFFu) << (8 * b);
+                uint4* d = reinterpret_cast<uint4*>(dst + 32 * b);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; q4++) d[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+            }
+        }
+    } else {
+        const int rsub = lane >> 2, c4 = (lane & 3) * 4;
+#pragma unroll
+        for (int b = 0; b < NC / 32; b++) {
+            uint32_t w[16];
+            const int e = o16_block<HAS_CS>(v + 32 * b, HAS_CS ? cs + 32 * b : nullptr, rs, w);
+            ebytes |= (static_cast<uint32_t>(e) & 0xFFu) << (8 * b);
+            uint4* sw = reinterpret_cast<uint4*>(stg + lane * STG_STRIDE);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; q4++) sw[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const int row = 8 * i + rsub;
+                uint16_t* d = reinterpret_cast<uint16_t*>(
+                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), row));
+                const uint4 x = *reinterpret_cast<const uint4*>(stg + row * STG_STRIDE + c4);
+                if (d != nullptr) *reinterpret_cast<uint4*>(d + 32 * b + 2 * c4) = x;
+            }
+            __syncwarp();
+        }
+    }
+    if (dst != nullptr) {
+        if constexpr (NC == 128) *reinterpret_cast<uint32_t*>(dst_e) = ebytes;
+        else if constexpr (NC == 64) *reinterpret_cast<uint16_t*>(dst_e) = static_cast<uint16_t>(ebytes);
+        else *dst_e = static_cast<int8_t>(ebytes & 0xFFu);
     }
 }
 
@@ -765,9 +861,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     u++;
                 }
                 if (!ok) break;
-                store_rows_coalesced<NC, BSCALE == BSCALE_ROW>(
-                    acc_r, reinterpret_cast<float*>(smem + S::SPARSE_OFF) + ew * EWF,
+                store_rows16<NC, BSCALE == BSCALE_ROW>(
+                    acc_r, reinterpret_cast<uint32_t*>(smem + S::SPARSE_OFF) + ew * EWF,
                     valid ? p.o + static_cast<size_t>(row) * p.H + n0 : nullptr,
+                    p.oe + static_cast<size_t>(row) * (p.H / 32) + n0 / 32,
                     p.b_scale + static_cast<size_t>(e) * p.b_rows + n0, rw, lane);
             }
         }

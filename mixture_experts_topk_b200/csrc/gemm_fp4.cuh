@@ -91,7 +91,8 @@ struct Fp4Params {
     uint8_t* hq;              // gate/up out: hidden codes [rows][I/2], scale factors hsf
     uint8_t* hsf;
     int I;
-    float* o;                 // down out: [A][H] fp32 rows in slot order
+    uint16_t* o;              // down out: [A][H] fp16 rows in slot order, block exponents in oe
+    int8_t* oe;               //   [A][H / 32]
     int H;
     const int32_t* perm;
     const float* route_w;
@@ -337,9 +338,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[acc]);
                 u++;
-                store_rows_coalesced<NC, false>(
-                    v, reinterpret_cast<float*>(smem + L::STG_OFF) + (warp - 2) * STG_WARP_FLOATS,
-                    valid ? p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + NC * g : nullptr, nullptr,
+                store_rows16<NC, false>(
+                    v, reinterpret_cast<uint32_t*>(smem + L::STG_OFF) + (warp - 2) * STG_WARP_FLOATS,
+                    valid ? p.o + static_cast<size_t>(slot) * p.H + nb * F4_BN + NC * g : nullptr,
+                    p.oe + static_cast<size_t>(slot) * (p.H / 32) + (nb * F4_BN + NC * g) / 32, nullptr,
                     p.h_global * wg0 * rw, lane);
             }
         }

@@ -12,7 +12,7 @@
 // A per stage: 4 scales of 32 per row), 3 to 5 stages (see the variants
 // below).  For small batches the K
 // range of each tile may be split S ways (S read from the dispatch's pick,
-// work item t = (tile t / S, split t % S)); split s writes its fp32 partial rows to copy s
+// work item t = (tile t / S, split t % S)); split s writes its partial rows to copy s
 // of the output rows, o + s * A * H.  MMA j of a stage (K = 32)
 // uses byte j of the chunk (scale-factor id j).  TMEM: one 256-column
 // accumulator, released as soon as the epilogue has it in registers, then the
@@ -26,8 +26,9 @@
 // MMAs; commits reach both CTAs.  An expert with an odd m-tile count runs its
 // last pair with rank 1's rows unstored (it loads rank 0's rows).
 //
-// Output rows: a warp whose 32 rows are all stored (rows of one expert are
-// consecutive slots) writes them as four 32-row x 32-column fp32 boxes through
+// Output rows (fp16 with a power-of-two scale per 32 columns, see
+// store_rows16): a warp whose 32 rows are all stored (rows of one expert are
+// consecutive slots) writes them as two 32-row x 64-column fp16 boxes through
 // a 128-byte-swizzled shared buffer (two per warp, alternating) with TMA
 // tensor stores, so the store runs asynchronously beside the next tile's
 // accumulator read; a warp with fewer rows stores its rows directly.
@@ -40,7 +41,7 @@ namespace moe {
 constexpr int MX_BN = 256;
 constexpr int MX_A_BYTES = 128 * 128;
 constexpr int MX_SFA_BYTES = 512;
-constexpr int MX_BOX_BYTES = 32 * 128;                           // 32 rows x 32 fp32
+constexpr int MX_BOX_BYTES = 32 * 128;                           // 32 rows x 64 fp16
 constexpr int MX_SFA_TMEM = MX_BN;                               // 4 columns per stage
 constexpr int MX_SFB_TMEM = MX_BN + 32;                          // 8 columns (two 128-row chunks)
 // Deep K (many K stages per tile): 4 stages, rows stored from registers.
@@ -118,7 +119,8 @@ struct MxDownParams {
     int b_rows;                // H
     const uint8_t* sfa;        // hidden MX scales, chunked by padded row tile (I / 32 per row)
     const float* w_scale;      // [E][H] fp32 per output row of W_down
-    float* o;                  // [S][A][H] fp32 rows in slot order
+    uint16_t* o;               // [S][A][H] fp16 rows in slot order (block exponents in oe)
+    int8_t* oe;                // [S][A][H / 32]
     int H;
     int A;                     // assignments T * k
     const int32_t* split;      // S, the K split chosen by the dispatch's scan
@@ -424,42 +426,45 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             __syncwarp();
             if (lane == 0) release_acc();   // the next tile's MMAs may start
             u++;
+            const size_t orow = static_cast<size_t>(sp) * p.A + slot;
             if (BOXES && __all_sync(0xffffffffu, valid)) {
-                // rows sp A + slot(lane 0) + lane: four boxes of 32 columns
-                const int y0 = __shfl_sync(0xffffffffu, sp * p.A + slot, 0);
+                // rows sp A + slot(lane 0) + lane: two boxes of 64 fp16 columns
+                const int y0 = __shfl_sync(0xffffffffu, static_cast<int>(orow), 0);
+                uint32_t ebytes = 0;
 #pragma unroll
-                for (int b = 0; b < 4; b++, nbox++) {
+                for (int b = 0; b < 2; b++, nbox++) {
                     uint8_t* buf = ostg + (nbox & 1) * MX_BOX_BYTES;
-                    float4 s4[8];
-#pragma unroll
-                    for (int c = 0; c < 8; c++) s4[c] = __ldg(reinterpret_cast<const float4*>(cs + 32 * b + 4 * c));
+                    uint32_t w0[16], w1[16];
+                    const int e0 = o16_block<true>(v + 64 * b, cs + 64 * b, rw, w0);
+                    const int e1 = o16_block<true>(v + 64 * b + 32, cs + 64 * b + 32, rw, w1);
+                    ebytes |= ((static_cast<uint32_t>(e0) & 0xFFu) | ((static_cast<uint32_t>(e1) & 0xFFu) << 8))
+                              << (16 * b);
                     // the store issued from this buffer two boxes ago has read it
                     if (lane == 0) bulk_wait_read1();
                     __syncwarp();
 #pragma unroll
                     for (int c = 0; c < 8; c++) {
-                        const float* x = v + 32 * b + 4 * c;
                         // 16-byte chunk c of row `lane` sits at chunk c ^ (lane % 8) (128-byte swizzle)
-                        *reinterpret_cast<float4*>(buf + lane * 128 + 16 * (c ^ (lane & 7))) =
-                            make_float4(x[0] * s4[c].x * rw, x[1] * s4[c].y * rw, x[2] * s4[c].z * rw,
-                                        x[3] * s4[c].w * rw);
+                        const uint32_t* w = c < 4 ? w0 + 4 * c : w1 + 4 * (c - 4);
+                        *reinterpret_cast<uint4*>(buf + lane * 128 + 16 * (c ^ (lane & 7))) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmO, buf, (n0 + 32 * b) * 4, y0);
+                        tma_store_2d(&tmO, buf, (n0 + 64 * b) * 2, y0);
                         bulk_commit();
                     }
                 }
+                *reinterpret_cast<uint32_t*>(p.oe + orow * (p.H / 32) + n0 / 32) = ebytes;
             } else {
                 if constexpr (BOXES) {
                     // the box buffers serve as the row staging once their stores have read them
                     if (lane == 0) bulk_wait_read0();
                     __syncwarp();
                 }
-                store_rows_coalesced<128, true>(
-                    v, reinterpret_cast<float*>(ostg), valid ? p.o + (static_cast<size_t>(sp) * p.A + slot) * p.H + n0 : nullptr,
-                    cs, rw, lane);
+                store_rows16<128, true>(v, reinterpret_cast<uint32_t*>(ostg), valid ? p.o + orow * p.H + n0 : nullptr,
+                                        p.oe + orow * (p.H / 32) + n0 / 32, cs, rw, lane);
                 __syncwarp();
             }
         }

@@ -16,6 +16,7 @@
 #include "gemm_fp4.cuh"
 #include "gemm_mx.cuh"
 #include "router.cuh"
+#include "router_tc.cuh"
 
 using namespace moe;
 
@@ -100,7 +101,10 @@ static cudaError_t launch_k_pairs(bool pdl, void (*kern)(KP...), dim3 grid, dim3
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
-    size_t status, ids, w, logits, counts, offsets, num_tiles, tile_ptr, pick, gu_done, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, total;
+    size_t status, ids, w, logits, counts, offsets, num_tiles, tile_ptr, pick, gu_done, chunk, tiles, perm, inv, xglobal, xq, xs, hq, hs, o, oe;
+    // fixed-point rows of the tensor-core router (0 when the workspace has none)
+    size_t rxh, rxl, rwh, rwl, rx_exp, rx_sum, rx_max, rw_exp, rw_sum, rw_sumq, rw_max;
+    size_t total;
 };
 struct WLayout {
     size_t gu_q, gu_s, d_q, d_s, gu_g, d_g, total;
@@ -153,6 +157,22 @@ static size_t o_rows(const moe_config& c) {
     return c.fmt == MOE_FMT_FP8_ROW ? A + 7 * std::min<size_t>(A, 256) : A;
 }
 
+// The large-batch router (router_tc.cuh): batches above 128 tokens with more
+// than 8 experts.  Expert tiles of 128, or of E rounded up to 16.
+static bool router_tc_sized(const moe_config& c) { return c.max_T > 128 && c.E > 8 && c.H <= RTC_MAX_H; }
+// experts per tile: 128, or 64 when 128-wide tiles would leave over half of
+// the SMs idle; E rounded up to 16 when E <= 128
+static int router_tc_nt(int E, int T, int num_sms) {
+    if (E <= RTC_NT_MAX) return (E + 15) / 16 * 16;
+    const int tiles = (T + RTC_BM - 1) / RTC_BM * ((E + RTC_NT_MAX - 1) / RTC_NT_MAX);
+    return 2 * tiles < num_sms ? RTC_NT_MAX / 2 : RTC_NT_MAX;
+}
+// Wr rows padded to whole tiles (the workspace holds the widest padding)
+static int router_tc_epad(int E, int nt) { return (E + nt - 1) / nt * nt; }
+static int router_tc_epad_max(int E) {
+    return E <= RTC_NT_MAX ? (E + 15) / 16 * 16 : (E + RTC_NT_MAX - 1) / RTC_NT_MAX * RTC_NT_MAX;
+}
+
 static WsLayout make_ws_layout(const moe_config& c) {
     const size_t A = static_cast<size_t>(c.max_T) * c.k;
     const size_t nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
@@ -186,7 +206,23 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.xs = take(R * act_scale_bytes(c.fmt, c.H));
     L.hq = take(RH * code_bytes(c.fmt, c.I));
     L.hs = take(RH * hidden_scale_bytes(c.fmt, c.I));
-    L.o = take(o_rows(c) * c.H * 4);
+    L.o = take(o_rows(c) * c.H * 2);        // fp16 rows
+    L.oe = take(o_rows(c) * (c.H / 32));    // their block exponents
+    L.rxh = L.rxl = L.rwh = L.rwl = L.rx_exp = L.rx_sum = L.rx_max = L.rw_exp = L.rw_sum = L.rw_sumq = L.rw_max = 0;
+    if (router_tc_sized(c)) {
+        const size_t T = c.max_T, H = c.H, Ep = router_tc_epad_max(c.E);
+        L.rxh = take(T * H);
+        L.rxl = take(T * H);
+        L.rwh = take(Ep * H);
+        L.rwl = take(Ep * H);
+        L.rx_exp = take(T * 4);
+        L.rx_sum = take(T * 8);
+        L.rx_max = take(T * 4);
+        L.rw_exp = take(Ep * 4);
+        L.rw_sum = take(Ep * 8);
+        L.rw_sumq = take(Ep * 8);
+        L.rw_max = take(Ep * 4);
+    }
     L.total = off;
     return L;
 }
@@ -308,7 +344,8 @@ extern "C" moe_status moe_workspace_view_get(const moe_handle* h, void* ws, moe_
     v->xs = b + L.xs;
     v->hq = b + L.hq;
     v->hs = b + L.hs;
-    v->o = reinterpret_cast<float*>(b + L.o);
+    v->o = reinterpret_cast<uint16_t*>(b + L.o);
+    v->o_exp = reinterpret_cast<int8_t*>(b + L.oe);
     v->logits = reinterpret_cast<float*>(b + L.logits);
     return MOE_OK;
 }
@@ -414,6 +451,61 @@ extern "C" moe_status moe_pack_weights(const moe_handle* h, const moe_weights* s
 }
 
 // ------------------------------------------------------------------ route
+static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
+                            uint32_t box_inner, uint32_t box_rows, bool swizzle = true);
+
+// Large batches: fixed-point rows, exact int8 tensor-core products, and the
+// certified candidate filter with canonical logits for the candidates
+// (router_tc.cuh).  Same ids and weights as the SIMT kernels.
+static moe_status route_tc(const moe_handle* h, const void* x, int T, const float* wr, const RouterParams& p, void* ws,
+                           cudaStream_t st) {
+    const moe_config& c = h->cfg;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    const WsLayout& L = h->ws;
+    RouterFix f;
+    f.xh = reinterpret_cast<int8_t*>(b + L.rxh);
+    f.xl = reinterpret_cast<int8_t*>(b + L.rxl);
+    f.wh = reinterpret_cast<int8_t*>(b + L.rwh);
+    f.wl = reinterpret_cast<int8_t*>(b + L.rwl);
+    f.x_exp = reinterpret_cast<int32_t*>(b + L.rx_exp);
+    f.x_sum = reinterpret_cast<double*>(b + L.rx_sum);
+    f.x_max = reinterpret_cast<float*>(b + L.rx_max);
+    f.w_exp = reinterpret_cast<int32_t*>(b + L.rw_exp);
+    f.w_sum = reinterpret_cast<double*>(b + L.rw_sum);
+    f.w_sumq = reinterpret_cast<double*>(b + L.rw_sumq);
+    f.w_max = reinterpret_cast<float*>(b + L.rw_max);
+    const int NT = router_tc_nt(c.E, T, h->num_sms), Ep = router_tc_epad(c.E, NT);
+    const int nbx = (T + 7) / 8, nbw = (Ep + 7) / 8;
+    LAUNCH(h->pdl, "router_fixpoint_kernel", router_fixpoint_kernel, nbx + nbw, 256, 0, st,
+           static_cast<const __nv_bfloat16*>(x), wr, T, c.H, c.E, Ep, nbx, f);
+    CUtensorMap txh, txl, twh, twl;
+    moe_status r = make_tmap(&txh, f.xh, c.H, T, c.H, RTC_BK, RTC_BM);
+    if (r != MOE_OK) return r;
+    r = make_tmap(&txl, f.xl, c.H, T, c.H, RTC_BK, RTC_BM);
+    if (r != MOE_OK) return r;
+    r = make_tmap(&twh, f.wh, c.H, Ep, c.H, RTC_BK, NT);
+    if (r != MOE_OK) return r;
+    r = make_tmap(&twl, f.wl, c.H, Ep, c.H, RTC_BK, NT);
+    if (r != MOE_OK) return r;
+    RouterI8Params q;
+    q.T = T;
+    q.H = c.H;
+    q.E = c.E;
+    q.NT = NT;
+    q.x_exp = f.x_exp;
+    q.w_exp = f.w_exp;
+    q.bias = p.bias;
+    q.logits = p.logits;
+    q.status = reinterpret_cast<int32_t*>(b + L.status);
+    q.spin_limit = h->spin_limit;
+    CUDA_TRY(cudaFuncSetAttribute(router_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RTC_SMEM));
+    LAUNCH(h->pdl, "router_i8_kernel", router_i8_kernel, dim3((T + RTC_BM - 1) / RTC_BM, Ep / NT), RTC_THREADS,
+           RTC_SMEM, st, txh, txl, twh, twl, q);
+    LAUNCH(h->pdl, "router_select_kernel", router_select_kernel, std::min((T + 7) / 8, 16 * h->num_sms), 256, 0, st,
+           p, f);
+    return MOE_OK;
+}
+
 extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const float* wr, const float* bias,
                                 int32_t* ids, float* w, void* ws, moe_stream_t stream) {
     moe_status st0 = check_T(h, T, "moe_route");
@@ -437,6 +529,7 @@ extern "C" moe_status moe_route(const moe_handle* h, const void* x, int T, const
     p.k = h->cfg.k;
     p.score = h->cfg.score;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (T > 128 && router_tc_sized(h->cfg)) return route_tc(h, x, T, wr, p, ws, st);
     if (T <= 128 && h->cfg.E <= RF_MAX_E) {
         // logits and top-k in one launch
         LAUNCH(h->pdl, "router_small_fused_kernel", router_small_fused_kernel, (T + RS_TG - 1) / RS_TG,
@@ -525,8 +618,6 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
 }
 
 // ------------------------------------------------------------------ NVFP4 GEMMs
-static moe_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
-                            uint32_t box_inner, uint32_t box_rows, bool swizzle = true);
 static int max_m_tiles(const moe_config& c, int T);
 
 template <int KIND, int ACT = 0>
@@ -580,6 +671,7 @@ static moe_status fp4_gemm(const moe_handle* h, const void* packed, const float*
     p.hsf = static_cast<uint8_t*>(v.hs);
     p.I = c.I;
     p.o = v.o;
+    p.oe = v.o_exp;
     p.H = c.H;
     p.perm = v.perm;
     p.route_w = w;
@@ -774,8 +866,8 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     const uint64_t hs_bytes = hidden_rows(c) * hidden_scale_bytes(c.fmt, c.I);
     r = make_tmap(&ts, v.hs, 256, hs_bytes / 256, 256, 256, 2, false);
     if (r != MOE_OK) return r;
-    // output rows (fp32 as bytes): boxes of 32 rows x 32 values for the epilogue's stores
-    r = make_tmap(&to, v.o, static_cast<uint64_t>(c.H) * 4, o_rows(c), static_cast<uint64_t>(c.H) * 4, 128, 32);
+    // output rows (fp16 as bytes): boxes of 32 rows x 64 values for the epilogue's stores
+    r = make_tmap(&to, v.o, static_cast<uint64_t>(c.H) * 2, o_rows(c), static_cast<uint64_t>(c.H) * 2, 128, 32);
     if (r != MOE_OK) return r;
     MxDownParams p;
     memset(&p, 0, sizeof(p));
@@ -790,6 +882,7 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     p.sfa = static_cast<const uint8_t*>(v.hs);
     p.w_scale = reinterpret_cast<const float*>(pw + h->wl.d_s);
     p.o = v.o;
+    p.oe = v.o_exp;
     p.H = c.H;
     p.A = T * c.k;
     p.split = v.pick + 1;
@@ -859,7 +952,8 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
     p.a_scale = static_cast<const float*>(v.hs);
     p.a_ld = c.I / 128;
     p.b_scale = reinterpret_cast<const float*>(pw + h->wl.d_s);
-    p.o = static_cast<float*>(v.o);
+    p.o = v.o;
+    p.oe = v.o_exp;
     p.H = c.H;
     p.I = c.I;
     p.perm = v.perm;
@@ -947,14 +1041,16 @@ extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws,
     if (T == 0) return MOE_OK;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
-    // one CTA per (token group, 1024-column slice): small batches still spread.
+    // one CTA per (token group, 2048-column slice): small batches still spread.
     // Launched without the PDL attribute: launched early, its CTAs would be
     // placed on the few SMs the down GEMM leaves room on and run ~2x slower
     // (Qwen3.5 T=64: 5.4 vs 2.6 us) than when placed after the GEMM ends.
-    const int ncb = (h->cfg.H + 1023) / 1024;
+    constexpr int span = COMBINE_COLS * COMBINE_THREADS;
+    const int ncb = (h->cfg.H + span - 1) / span;
     const dim3 grid(std::max(1, std::min(T, 16 * h->num_sms / ncb)), ncb);
-    LAUNCH(false, "combine_kernel", combine_kernel, grid, 128, 0, reinterpret_cast<cudaStream_t>(stream),
-           static_cast<const float*>(v.o), static_cast<const int32_t*>(v.inv), T, h->cfg.H, h->cfg.k,
+    LAUNCH(false, "combine_kernel", combine_kernel, grid, COMBINE_THREADS, 0, reinterpret_cast<cudaStream_t>(stream),
+           static_cast<const uint16_t*>(v.o), static_cast<const int8_t*>(v.o_exp), static_cast<const int32_t*>(v.inv),
+           T, h->cfg.H, h->cfg.k,
            static_cast<const int32_t*>(h->cfg.fmt == MOE_FMT_FP8_ROW ? v.pick + 1 : nullptr),
            split_limit(h->picker, T * h->cfg.k), static_cast<__nv_bfloat16*>(y));
     return MOE_OK;

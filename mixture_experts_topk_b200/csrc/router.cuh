@@ -288,12 +288,11 @@ __global__ void __launch_bounds__(RS_WARPS * 32) router_logits_small_kernel(Rout
 }
 
 // top-k of one token by one warp: k rounds of a warp argmax, larger logit
-// first, equal logits -> lower expert id; lane l owns experts l + 32 m.  `l` is
-// the token's E logits (global or shared memory).
-__device__ __forceinline__ void router_topk_token(const RouterParams& p, const float* l, int t, int lane) {
-    float lv[8];
-#pragma unroll
-    for (int m = 0; m < 8; m++) lv[m] = (32 * m + lane < p.E) ? l[32 * m + lane] : 0.0f;
+// first, equal logits -> lower expert id; lane l owns experts l + 32 m, with
+// logit lv[m], taking part only where bit m of `allowed` is set; then the
+// softmax or sigmoid weights of the k selected logits.
+__device__ __forceinline__ void router_topk_select(const RouterParams& p, const float* lv, uint32_t allowed, int t,
+                                                   int lane) {
     uint32_t taken = 0;
     float sel_v[8];
     int sel_e[8];
@@ -305,7 +304,7 @@ __device__ __forceinline__ void router_topk_token(const RouterParams& p, const f
 #pragma unroll
         for (int m = 0; m < 8; m++) {
             const int e = 32 * m + lane;
-            if (e >= p.E || ((taken >> m) & 1u)) continue;
+            if (e >= p.E || !((allowed >> m) & 1u) || ((taken >> m) & 1u)) continue;
             if (be < 0 || lv[m] > bv) { bv = lv[m]; be = e; }   // e ascending: ties keep the lower id
         }
 #pragma unroll
@@ -333,6 +332,26 @@ __device__ __forceinline__ void router_topk_token(const RouterParams& p, const f
             p.w[static_cast<size_t>(t) * p.k + j] = z[j] / sum;
         }
     }
+}
+
+// top-k of one token over all its E logits `l` (global or shared memory)
+__device__ __forceinline__ void router_topk_token(const RouterParams& p, const float* l, int t, int lane) {
+    float lv[8];
+    uint32_t allowed = 0;
+#pragma unroll
+    for (int m = 0; m < 8; m++) {
+        const bool in = 32 * m + lane < p.E;
+        lv[m] = in ? l[32 * m + lane] : 0.0f;
+        allowed |= (in ? 1u : 0u) << m;
+    }
+    router_topk_select(p, lv, allowed, t, lane);
+}
+
+// top-k of one token among its candidate experts (bit m of `cand`: expert
+// 32 m + lane), whose canonical logits are in cv
+__device__ __forceinline__ void router_topk_candidates(const RouterParams& p, const float* cv, uint32_t cand, int t,
+                                                       int lane) {
+    router_topk_select(p, cv, cand, t, lane);
 }
 
 __global__ void __launch_bounds__(256) router_topk_kernel(RouterParams p) {

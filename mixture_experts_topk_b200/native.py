@@ -46,7 +46,7 @@ class moe_weights(ctypes.Structure):
 
 
 VIEW_FIELDS = ("status", "ids", "w", "counts", "offsets", "num_tiles", "tile_ptr", "pick", "tiles", "perm", "inv",
-               "x_global", "xq", "xs", "hq", "hs", "o", "logits")
+               "x_global", "xq", "xs", "hq", "hs", "o", "logits", "o_exp")
 
 
 class moe_workspace_view(ctypes.Structure):

@@ -38,6 +38,9 @@ CASES = {
     "block128-t700": (W.custom(H=256, I=128, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 700),
     "nvfp4-ragged": (W.custom(H=512, I=512, E=8, k=2, fmt=W.FMT_NVFP4), 300),
     "nvfp4-skew-e32": (W.custom(H=256, I=256, E=32, k=4, fmt=W.FMT_NVFP4, zipf_s=1.0), 50),
+    # above 128 tokens with more than 8 experts the router runs on the tensor cores
+    "row-skew-e64-t300": (W.custom(H=512, I=256, E=64, k=8, zipf_s=1.2), 300),
+    "block128-e48-t260": (W.custom(H=512, I=256, E=48, k=6, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 260),
 }
 
 
@@ -151,7 +154,9 @@ def test_router_ids_bit_exact(name):
                                            (2048, 250, 8, W.SCORE_SOFTMAX, 127), (256, 32, 4, W.SCORE_SIGMOID, 5),
                                            (256, 3, 2, W.SCORE_SOFTMAX, 7),
                                            (2048, 256, 8, W.SCORE_SOFTMAX, 129), (4096, 8, 2, W.SCORE_SOFTMAX, 150),
-                                           (512, 40, 4, W.SCORE_SIGMOID, 200), (6144, 256, 8, W.SCORE_SOFTMAX, 257)])
+                                           (512, 40, 4, W.SCORE_SIGMOID, 200), (6144, 256, 8, W.SCORE_SOFTMAX, 257),
+                                           # enough 128-token tiles for 128-expert tensor-core tiles
+                                           (256, 256, 8, W.SCORE_SOFTMAX, 4864), (512, 200, 6, W.SCORE_SIGMOID, 9600)])
 def test_router_named_shapes_bit_exact(H, E, k, score, T):
     """Both logits kernels (small batches, and the tiled one above 128 tokens)
     give the oracle's fp32 logits bit for bit, and its ids."""
@@ -168,8 +173,88 @@ def test_router_named_shapes_bit_exact(H, E, k, score, T):
     lg_ref = oracle.router_logits(bits(x), wr.numpy(), bias.numpy())
     off = native.moe_workspace_view_get(h, ws)["logits"] - ws.data_ptr()
     lg = ws[off:off + T * E * 4].view(torch.float32).cpu().numpy().reshape(T, E)
-    assert (lg.view(np.uint32) == lg_ref.astype(np.float32).view(np.uint32)).all()
     ids_ref, w_ref = oracle.topk(lg_ref, k, score)
+    assert (ids.cpu().numpy() == ids_ref).all()
+    np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=0, atol=2e-6)
+    same = lg.view(np.uint32) == lg_ref.astype(np.float32).view(np.uint32)
+    if not router_uses_filter(T, E):
+        assert same.all()
+    else:
+        # the selected experts' logits are canonical; every other logit is
+        # canonical or within the certified distance of it
+        assert same[np.arange(T)[:, None], ids_ref].all()
+        D = router_filter_bound(x, wr.numpy(), bias.numpy(), lg)
+        assert np.all(same | (np.abs(lg.astype(np.float64) - lg_ref.astype(np.float64)) <= D))
+    native.moe_destroy(h)
+
+
+def router_uses_filter(T, E):
+    """Batches above 128 tokens with more than 8 experts route through the
+    integer tensor-core pass and the certified candidate filter."""
+    return T > 128 and E > 8
+
+
+def router_filter_bound(x_bf16, wr, bias, l_stored):
+    """The distance the filter certifies between a stored approximate logit
+    and the canonical one, restated from its definition: fixed-point rows
+    rounded at half of 2^(e - 14) (e the smallest integer with max|row| <=
+    2^e), the canonical chain's gamma(H/32 + 6) (sum|x w| + |b|) with
+    sum|x w| <= min(sum|x| max|w|, max|x| sum|w|), and the fp32 storage of
+    the approximation."""
+    x = x_bf16.float().numpy().astype(np.float64)
+    w = np.asarray(wr, np.float64)
+    H = x.shape[1]
+
+    def expo(a):
+        m = np.abs(a).max(axis=1)
+        return np.where(m > 0, np.frexp(m)[1], 0)
+
+    ex, ew = expo(x), expo(w)
+    qw = np.rint(w * np.exp2(14.0 - ew)[:, None])
+    sx, mx = np.abs(x).sum(1), np.abs(x).max(1)
+    sw, mw = np.abs(w).sum(1), np.abs(w).max(1)
+    swq = np.abs(qw).sum(1) * np.exp2(ew - 14.0)
+    n = H // 32 + 6
+    gamma = n * 2.0 ** -24 / (1 - n * 2.0 ** -24)
+    dfix = np.exp2(ew - 15.0)[None, :] * sx[:, None] + np.exp2(ex - 15.0)[:, None] * swq[None, :]
+    sxw = np.minimum(sx[:, None] * mw[None, :], mx[:, None] * sw[None, :])
+    b = np.zeros(w.shape[0]) if bias is None else np.abs(np.asarray(bias, np.float64))
+    return (dfix + gamma * (sxw + b[None, :]) + np.abs(l_stored.astype(np.float64)) * 2.0 ** -23) * (1 + 2.0 ** -20)
+
+
+@pytest.mark.parametrize("T", [129, 300])
+def test_router_filter_keeps_exact_and_near_ties(T):
+    """Batches on the tensor-core router with experts whose canonical logits
+    tie exactly (duplicated router rows: the lower id must come first) or
+    differ in their last bits (a row with one element nudged by one ulp): the
+    ids are the oracle's, bit for bit."""
+    wl = W.custom(H=2048, I=128, E=64, k=8, router_init="uniform")
+    wr, _ = synth.router(wl, seed=4)
+    wr = wr.clone()
+    x = synth.tokens(wl, T, seed=4)
+    # nine experts made strong for every token (the batch's mean direction adds
+    # about sqrt(H / T) to their logits), so the top 8 is cut inside them and
+    # the tie groups below land on both sides of the cut
+    boost = x.float().mean(0)
+    for e in (3, 5, 9, 10, 11, 12, 17, 40, 41):
+        wr[e] += boost / boost.norm()
+    wr[5] = wr[3]                                    # exact tie with expert 3
+    wr[17] = wr[9]                                   # exact tie with expert 9
+    wr[10] = wr[9]
+    wr[10, 100] = torch.nextafter(wr[10, 100], torch.tensor(1.0))   # a near tie
+    wr[41] = wr[40]
+    wr[41, 7] = torch.nextafter(wr[41, 7], torch.tensor(-1.0))
+    h = native.moe_init(wl, T)
+    ws = torch.empty(native.moe_workspace_size(h), dtype=torch.uint8, device="cuda")
+    native.moe_workspace_init(h, ws)
+    ids = torch.empty(T, 8, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, 8, dtype=torch.float32, device="cuda")
+    native.moe_route(h, x.cuda(), T, wr.cuda(), None, ids, w, ws)
+    torch.cuda.synchronize()
+    lg_ref = oracle.router_logits(bits(x), wr.numpy(), None)
+    ids_ref, w_ref = oracle.topk(lg_ref, 8, wl.score)
+    assert ((ids_ref == 3).any(1) & (ids_ref == 5).any(1)).any(), "the exact tie reaches the top k"
+    assert ((ids_ref == 9).any(1) & ~(ids_ref == 17).any(1)).any(), "an exact tie is cut by k"
     assert (ids.cpu().numpy() == ids_ref).all()
     np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=0, atol=2e-6)
     native.moe_destroy(h)
@@ -295,8 +380,16 @@ def test_down_matches_oracle_on_oracle_hidden(name, down_bn):
     S = int(layer.region("pick", torch.int32, 2).cpu().numpy()[1])
     if name == "row-split-t3":
         assert S == 4                     # 10 units, s_max = 16 K-blocks / 4
-    o = layer.region("o", torch.float32, S * A * wl.H).cpu().numpy().reshape(S, A, wl.H).sum(axis=0)
+    o = decode_o(layer, wl, S, A).sum(axis=0)
     assert tolerance_violations(o, ref["o_w"]) == 0
+
+
+def decode_o(layer, wl, S, A):
+    """The down GEMM's weighted rows [S, A, H]: fp16 values times 2^(e - 15),
+    one exponent e per 32 columns (the layout moe_b200.h documents)."""
+    q = layer.region("o", torch.float16, S * A * wl.H).float().cpu().numpy().reshape(S, A, wl.H // 32, 32)
+    e = layer.region("o_exp", torch.int8, S * A * wl.H // 32).cpu().numpy().reshape(S, A, wl.H // 32, 1)
+    return (q.astype(np.float64) * np.exp2(e.astype(np.float64) - 15)).reshape(S, A, wl.H)
 
 
 # the gated activation variants, on each format; the limits bind on part of the
@@ -517,5 +610,6 @@ def test_workspace_regions_hold_the_documented_layouts(fmt):
     assert v["hq"] - v["xs"] >= xs
     assert v["hs"] - v["hq"] >= hq
     assert v["o"] - v["hs"] >= hs
-    assert ws.data_ptr() + size - v["o"] >= A * H * 4
+    assert v["o_exp"] - v["o"] >= A * H * 2                 # fp16 rows
+    assert ws.data_ptr() + size - v["o_exp"] >= A * H // 32  # one exponent byte per 32 columns
     native.moe_destroy(h)
