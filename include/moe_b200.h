@@ -268,8 +268,10 @@ moe_status moe_set_launch_options(moe_handle* h, int pdl);
  * rows of W_down).  An expert with an odd row-tile count runs its last pair
  * half empty.  The
  * results are those of the single-CTA kernel up to the fp32 summation order
- * inside the tensor core.  cta_pairs = 0 keeps single CTAs.  Errors:
- * MOE_ERR_INVALID_ARG for a null handle or another value. */
+ * inside the tensor core.  cta_pairs = 0 keeps single CTAs; cta_pairs = 2
+ * runs these GEMMs on CTA pairs at every batch size (the down GEMM still only
+ * where K > 2048 and no K split is chosen).  Errors: MOE_ERR_INVALID_ARG for a
+ * null handle or another value. */
 moe_status moe_set_gemm_options(moe_handle* h, int cta_pairs);
 
 /* Limit, in SM clock cycles, of every wait of the GEMM kernels on another

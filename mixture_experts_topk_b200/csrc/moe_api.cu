@@ -771,8 +771,8 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     if (r != MOE_OK) return r;
     const int n_gu = c.act == MOE_ACT_RELU2 ? c.I : 2 * c.I;   // rows of the packed gate/up weights
     // CTA pairs: each CTA loads half of a B tile's 256 rows
-    const bool pairs = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU && h->gemm_pairs &&
-                       static_cast<long long>(T) * c.k >= 4LL * TILE_M * c.E;
+    const bool pairs = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU &&
+                       (h->gemm_pairs == 2 || (h->gemm_pairs == 1 && static_cast<long long>(T) * c.k >= 4LL * TILE_M * c.E));
     r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, pairs ? 128 : 256);
     if (r != MOE_OK) return r;
     GemmParams p;
@@ -854,8 +854,8 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     // tile's 256 B rows, when the experts average at least 4 row tiles (as for
     // the gate/up GEMM) and no K split can be chosen; shallow K keeps single
     // CTAs and the box stores.
-    const bool pairs = h->gemm_pairs && c.I / 128 > MX_BOX_MAX_KB && T * c.k >= 4 * TILE_M * c.E &&
-                       split_limit(h->picker, T * c.k) == 1;
+    const bool pairs = c.I / 128 > MX_BOX_MAX_KB && split_limit(h->picker, T * c.k) == 1 &&
+                       (h->gemm_pairs == 2 || (h->gemm_pairs == 1 && T * c.k >= 4 * TILE_M * c.E));
     CUtensorMap ta, tb, to, ts;
     moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
@@ -1025,8 +1025,8 @@ extern "C" moe_status moe_set_launch_options(moe_handle* h, int pdl) {
 
 extern "C" moe_status moe_set_gemm_options(moe_handle* h, int cta_pairs) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: null handle");
-    if (cta_pairs != 0 && cta_pairs != 1)
-        return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: cta_pairs must be 0 or 1 (got %d)", cta_pairs);
+    if (cta_pairs < 0 || cta_pairs > 2)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: cta_pairs must be 0, 1 or 2 (got %d)", cta_pairs);
     h->gemm_pairs = cta_pairs;
     return MOE_OK;
 }

@@ -17,8 +17,9 @@
 //    -> int32, exact) gives, per (token, expert), S_hh = sum hi_x hi_w,
 //    S_x = sum (hi_x lo_w + lo_x hi_w) and S_ll = sum lo_x lo_w, so
 //        L~ = 2^(e_x + e_w - 28) (65536 S_hh + 256 S_x + S_ll) + bias[e]
-//    is the exact dot product of the rounded rows (+ bias), evaluated in fp64
-//    without rounding and stored as fp32.  |int32 sums| <= 2^14 * 2 H * 64, so
+//    is the exact dot product of the rounded rows (+ bias).  The integer sum
+//    is exact in 64 bits; it is rounded once to fp32, scaled by an exact power
+//    of two and rounded once more by the bias add, and stored.  |int32 sums| <= 2^14 * 2 H * 64, so
 //    H <= 65536 cannot overflow.
 // 3. Certified filter (router_select_kernel).  With eps = 2^(e - 15) the
 //    rounding of one value (half a unit), the exact logit L* = sum x w + b and
@@ -26,10 +27,10 @@
 //    5-level tree, one bias add: at most n + 6 roundings on any path),
 //        |L~ - L*| <= eps_w sum|x| + eps_x sum|w~|              (fixed point)
 //        |C  - L*| <= gamma(n + 6) (sum|x w| + |b|),             gamma(m) = m u / (1 - m u), u = 2^-24
-//        |fp32(L~) - L~| <= 2^-24 |L~|,
+//        |l - L~| <= 2^-23 (|l| + |b|) + 2^-126     (l: L~ evaluated in fp32, stored),
 //    with sum|x w| <= min(sum|x| max|w|, max|x| sum|w|).  So C lies in
-//    [l - D, l + D] around the stored l = fp32(L~), D their sum (x (1 + 2^-20)
-//    for the fp64 evaluation of D itself).  Let LB_k be the k-th largest
+//    [l - D, l + D] around the stored l, D their sum (x (1 + 2^-20) for the
+//    fp64 evaluation of D itself).  Let LB_k be the k-th largest
 //    l - D of the token.  An expert with l + D < LB_k has k experts whose C
 //    is strictly larger, so it is not among the canonical top k whatever the
 //    tie rule; every other expert is a candidate.  The candidates get the
@@ -37,7 +38,7 @@
 //    candidates by C (ties to the lower id) is the canonical top k, and the
 //    weights are computed from those C exactly as on the SIMT path.
 // The logits buffer then holds C for the candidates (a superset of the
-// selected experts) and fp32(L~) for the others.
+// selected experts) and l for the others.
 #pragma once
 #include "common.cuh"
 #include "router.cuh"
@@ -197,6 +198,12 @@ __global__ void __launch_bounds__(256) router_fixpoint_kernel(const __nv_bfloat1
     }
 }
 
+// 2^k as a float; outside the normal range the value is tiny or huge and the
+// product is formed by ldexpf (exact scaling either way, up to the final rounding)
+__device__ __forceinline__ float pow2_or_ldexp(int k) {
+    return (k >= -126 && k <= 127) ? __int_as_float((127 + k) << 23) : ldexpf(1.0f, k);
+}
+
 // Instruction descriptor of kind::i8: s32 accumulate [4,6) = 2, A and B signed
 // 8-bit [7,10) = [10,13) = 1, both K-major, N >> 3 at [17,23), M >> 4 at [24,29).
 __host__ __device__ constexpr uint32_t idesc_s8(int M, int N) {
@@ -270,6 +277,15 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     pdl_wait();
     pdl_trigger();
     const long long limit = p.spin_limit;
+    // the tile's expert exponents and biases, once per CTA
+    __shared__ int s_wexp[RTC_NT_MAX];
+    __shared__ float s_bias[RTC_NT_MAX];
+    for (int c = threadIdx.x; c < NT; c += blockDim.x) {
+        const int e = n0 + c;
+        s_wexp[c] = e < p.E ? p.w_exp[e] : 0;
+        s_bias[c] = (e < p.E && p.bias) ? p.bias[e] : 0.0f;
+    }
+    __syncthreads();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -334,22 +350,32 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         } else if (mma_ok) {
             tc_fence_after();
             const int ex = t < p.T ? p.x_exp[t] : 0;
+            const bool vec = (p.E & 3) == 0;
             for (int c0 = 0; c0 < NT; c0 += 32) {
                 float vh[32], vx[32], vl[32];
                 tmem_ld32x2(lane_addr + c0, lane_addr + NT + c0, vh, vx);
                 tmem_ld32(lane_addr + 2 * NT + c0, vl);
                 if (t < p.T) {
-                    float* dst = p.logits + static_cast<size_t>(t) * p.E;
+                    float* dst = p.logits + static_cast<size_t>(t) * p.E + n0 + c0;
+                    float out[32];
 #pragma unroll
                     for (int c = 0; c < 32; c++) {
-                        const int e = n0 + c0 + c;
-                        if (e >= p.E) continue;
-                        const double s = static_cast<double>(__float_as_int(vh[c])) * 65536.0 +
-                                         static_cast<double>(__float_as_int(vx[c])) * 256.0 +
-                                         static_cast<double>(__float_as_int(vl[c]));
-                        double l = ldexp(s, ex + __ldg(p.w_exp + e) - 28);
-                        if (p.bias) l += static_cast<double>(__ldg(p.bias + e));
-                        dst[e] = static_cast<float>(l);
+                        // 65536 S_hh + 256 S_x + S_ll is exact in 64 bits; one rounding to
+                        // fp32, an exact power-of-two scale, one rounding of the bias add
+                        const long long si = (static_cast<long long>(__float_as_int(vh[c])) << 16) +
+                                             (static_cast<long long>(__float_as_int(vx[c])) << 8) +
+                                             static_cast<long long>(__float_as_int(vl[c]));
+                        const float l = __fmul_rn(__ll2float_rn(si), pow2_or_ldexp(ex + s_wexp[c0 + c] - 28));
+                        out[c] = __fadd_rn(l, s_bias[c0 + c]);
+                    }
+                    if (vec && n0 + c0 + 32 <= p.E) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4)
+                            *reinterpret_cast<float4*>(dst + c) = make_float4(out[c], out[c + 1], out[c + 2], out[c + 3]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; c++)
+                            if (n0 + c0 + c < p.E) dst[c] = out[c];
                     }
                 }
             }
@@ -363,70 +389,80 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     }
 }
 
-// Bound D of |C - fp32(L~)| for token t and expert e (see the file comment).
-__device__ __forceinline__ double router_bound(int ex, double sx, float mx, int ew, double sw, double swq, float mw,
-                                               float bias_abs, float l, double gamma) {
-    const double eps_x = ldexp(1.0, ex - 15), eps_w = ldexp(1.0, ew - 15);
+// 2^k as a double (k inside the normal range, as every exponent here is)
+__device__ __forceinline__ double pow2d(int k) { return __longlong_as_double(static_cast<long long>(1023 + k) << 52); }
+
+// Bound D of |C - l| for token t and expert e, l the stored approximation (see
+// the file comment): the fixed-point term, the canonical chain's term, and
+// the fp32 evaluation of l (one rounding of the integer sum, one of the bias
+// add: within 2^-23 (|l| + |b|), plus 2^-126 for scales outside the normal
+// range).
+__device__ __forceinline__ double router_bound(double eps_x, double sx, float mx, double eps_w, double sw, double swq,
+                                               float mw, float babs, float l, double gamma) {
     const double dfix = eps_w * sx + eps_x * swq;
     const double sxw = fmin(sx * static_cast<double>(mw), static_cast<double>(mx) * sw);
-    const double dcan = gamma * (sxw + static_cast<double>(bias_abs));
-    const double dst = ldexp(fabs(static_cast<double>(l)), -23);
+    const double dcan = gamma * (sxw + static_cast<double>(babs));
+    const double dst = (fabs(static_cast<double>(l)) + static_cast<double>(babs)) * 0x1p-23 + 0x1p-126;
     return (dfix + dcan + dst) * (1.0 + 0x1p-20);
 }
 
-// The canonical fp32 logits of token t for up to RS_BATCH experts es[0..n),
-// computed by one warp: lane l runs each expert's chain over h = 256 i + 8 l + j
-// (i, then j = 0..7), the chains advancing together so that their loads
-// overlap; the xor butterfly over offsets 1..16 forms the pairwise tree on
-// every lane, then + bias.  Per expert the same operations as
-// router_logits_small_kernel, so the same bits.
-constexpr int RS_BATCH = 8;
-__device__ __forceinline__ void canonical_logits(const RouterParams& p, int t, const int* es, int n, int lane,
-                                                 float* out) {
+// The canonical fp32 logits of (token t, experts e0 and e1) computed by one
+// warp: lane l runs each expert's chain over h = 256 i + 8 l + j (i, then
+// j = 0..7); the two chains share each packed fma (fma.rn.f32x2: two
+// independent round-to-nearest fma, the same as two scalar ones).  The xor
+// butterfly over offsets 1..16 forms the pairwise tree on every lane, then
+// + bias.  Per expert the same operations as router_logits_small_kernel, so
+// the same bits.  With two == false only e0 is computed.
+__device__ __forceinline__ void canonical_logit2(const RouterParams& p, int t, int e0, int e1, bool two, int lane,
+                                                 float& c0, float& c1) {
+    const float* w0 = p.wr + static_cast<size_t>(e0) * p.H + 8 * lane;
+    const float* w1 = p.wr + static_cast<size_t>(two ? e1 : e0) * p.H + 8 * lane;
     const __nv_bfloat16* xrow = p.x + static_cast<size_t>(t) * p.H + 8 * lane;
-    float acc[RS_BATCH];
-#pragma unroll
-    for (int c = 0; c < RS_BATCH; c++) acc[c] = 0.0f;
+    float a0 = 0.0f, a1 = 0.0f;
     const int nI = p.H >> 8;
+#pragma unroll 4
     for (int i = 0; i < nI; i++) {
+        const float4 pa = __ldg(reinterpret_cast<const float4*>(w0 + 256 * i));
+        const float4 pb = __ldg(reinterpret_cast<const float4*>(w0 + 256 * i + 4));
+        const float4 qa = __ldg(reinterpret_cast<const float4*>(w1 + 256 * i));
+        const float4 qb = __ldg(reinterpret_cast<const float4*>(w1 + 256 * i + 4));
         const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xrow + 256 * i));
-        float4 wa[RS_BATCH], wb[RS_BATCH];
-#pragma unroll
-        for (int c = 0; c < RS_BATCH; c++) {
-            if (c < n) {
-                const float* w = p.wr + static_cast<size_t>(es[c]) * p.H + 8 * lane + 256 * i;
-                wa[c] = __ldg(reinterpret_cast<const float4*>(w));
-                wb[c] = __ldg(reinterpret_cast<const float4*>(w + 4));
-            }
-        }
+        const float wp[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+        const float wq[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-        for (int c = 0; c < RS_BATCH; c++) {
-            if (c < n) {
-                const float wv[8] = {wa[c].x, wa[c].y, wa[c].z, wa[c].w, wb[c].x, wb[c].y, wb[c].z, wb[c].w};
-#pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    const float xj = (j & 1) ? bf16_hi(xw[j >> 1]) : bf16_lo(xw[j >> 1]);
-                    acc[c] = __fmaf_rn(xj, wv[j], acc[c]);
-                }
-            }
+        for (int j = 0; j < 8; j++) {
+            const float xj = (j & 1) ? bf16_hi(xw[j >> 1]) : bf16_lo(xw[j >> 1]);
+            // chain 0 += xj * wp[j], chain 1 += xj * wq[j]
+            asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+                "mov.b64 rd, {%0, %1};\n\tfma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+                : "+f"(a0), "+f"(a1)
+                : "f"(xj), "f"(wp[j]), "f"(wq[j]));
         }
     }
 #pragma unroll
-    for (int c = 0; c < RS_BATCH; c++) {
-        if (c < n) {
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) acc[c] = __fadd_rn(acc[c], __shfl_xor_sync(0xffffffffu, acc[c], off));
-            if (p.bias) acc[c] = __fadd_rn(acc[c], p.bias[es[c]]);
-            out[c] = acc[c];
-        }
+    for (int off = 1; off < 32; off <<= 1) {
+        a0 = __fadd_rn(a0, __shfl_xor_sync(0xffffffffu, a0, off));
+        a1 = __fadd_rn(a1, __shfl_xor_sync(0xffffffffu, a1, off));
     }
+    if (p.bias) {
+        a0 = __fadd_rn(a0, p.bias[e0]);
+        if (two) a1 = __fadd_rn(a1, p.bias[e1]);
+    }
+    c0 = a0;
+    c1 = a1;
+}
+
+// (v, id) ranks before (v', id') when v > v', or v == v' and id < id' (the
+// selection order: larger logit first, ties to the lower id)
+__device__ __forceinline__ bool rank_before(float v, int id, float v2, int id2) {
+    return v > v2 || (v == v2 && id < id2);
 }
 
 // One warp per token: bounds, the k-th largest lower bound, candidates, their
 // canonical logits (written over the approximations), then the top k of the
-// candidates and the weights exactly as router_topk_token computes them.
-__global__ void __launch_bounds__(256) router_select_kernel(RouterParams p, RouterFix f) {
+// candidates and the weights, computed as router_topk_select computes them.
+__global__ void __launch_bounds__(256, 3) router_select_kernel(RouterParams p, RouterFix f) {
     __shared__ int s_list[8][256];
     pdl_wait();
     pdl_trigger();
@@ -434,90 +470,141 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouterParams p, Rout
     const int nm = (p.E + 31) >> 5;
     const double nr = static_cast<double>((p.H >> 5) + 6) * 0x1p-24;
     const double gamma = nr / (1.0 - nr);
+    int* list = s_list[threadIdx.x >> 5];
     for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < p.T; t += gridDim.x * 8) {
         float* lrow = p.logits + static_cast<size_t>(t) * p.E;
-        const int ex = f.x_exp[t];
+        const double eps_x = pow2d(f.x_exp[t] - 15);
         const double sx = f.x_sum[t];
         const float mx = f.x_max[t];
-        float lv[8];
-        double dv[8];
+        // bounds of the canonical logits, rounded outward to fp32 (only looser)
+        float lb[8], ub[8];
 #pragma unroll
         for (int m = 0; m < 8; m++) {
             const int e = 32 * m + lane;
-            lv[m] = 0.0f;
-            dv[m] = 0.0;
+            lb[m] = -INFINITY;
+            ub[m] = -INFINITY;
             if (m < nm && e < p.E) {
-                lv[m] = lrow[e];
-                dv[m] = router_bound(ex, sx, mx, f.w_exp[e], f.w_sum[e], f.w_sumq[e], f.w_max[e],
-                                     p.bias ? fabsf(p.bias[e]) : 0.0f, lv[m], gamma);
+                const float l = lrow[e];
+                const double d = router_bound(eps_x, sx, mx, pow2d(f.w_exp[e] - 15), f.w_sum[e], f.w_sumq[e],
+                                              f.w_max[e], p.bias ? fabsf(p.bias[e]) : 0.0f, l, gamma);
+                lb[m] = __double2float_rd(static_cast<double>(l) - d);
+                ub[m] = __double2float_ru(static_cast<double>(l) + d);
             }
         }
-        // LB_k: the k-th largest lower bound (k rounds of a warp maximum)
-        uint32_t taken = 0;
-        double lbk = 0.0;
-        for (int j = 0; j < p.k; j++) {
-            double bv = -INFINITY;
-            int bm = -1;
+        // LB_k, the k-th largest lower bound: each lane sorts its eight lower
+        // bounds (descending), then k rounds take the warp maximum of the
+        // lanes' current heads and advance the winning lane's head
+        float srt[8];
 #pragma unroll
-            for (int m = 0; m < 8; m++) {
-                if (m >= nm || 32 * m + lane >= p.E || ((taken >> m) & 1u)) continue;
-                const double lb = static_cast<double>(lv[m]) - dv[m];
-                if (bm < 0 || lb > bv) { bv = lb; bm = m; }
-            }
-            int owner = bm >= 0 ? lane : 32;
-            double wv = bv;
+        for (int m = 0; m < 8; m++) srt[m] = lb[m];
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+#pragma unroll
+            for (int j = 7; j > i; j--)
+                if (srt[j] > srt[j - 1]) {
+                    const float tmp = srt[j];
+                    srt[j] = srt[j - 1];
+                    srt[j - 1] = tmp;
+                }
+        float lbk = -INFINITY;
+        for (int j = 0; j < p.k; j++) {
+            const float head = srt[0];
+            float wv = head;
+            int owner = lane;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
-                const double ov = __shfl_xor_sync(0xffffffffu, wv, off);
+                const float ov = __shfl_xor_sync(0xffffffffu, wv, off);
                 const int oo = __shfl_xor_sync(0xffffffffu, owner, off);
-                if (oo < 32 && (owner == 32 || ov > wv || (ov == wv && oo < owner))) { wv = ov; owner = oo; }
+                if (ov > wv || (ov == wv && oo < owner)) { wv = ov; owner = oo; }
             }
-            // the winning lane marks its best slot as taken
-            if (owner == lane) taken |= 1u << bm;
             lbk = wv;
-        }
-        // candidates: upper bound reaches LB_k; their canonical logits
-        uint32_t cand = 0;
+            if (owner == lane) {
 #pragma unroll
-        for (int m = 0; m < 8; m++) {
-            const int e = 32 * m + lane;
-            if (m < nm && e < p.E && static_cast<double>(lv[m]) + dv[m] >= lbk) cand |= 1u << m;
+                for (int m = 0; m < 7; m++) srt[m] = srt[m + 1];
+                srt[7] = -INFINITY;
+            }
         }
-        // the candidates in expert order (a per-warp list in shared memory),
-        // RS_BATCH at a time; lane e % 32 keeps expert e's canonical logit
-        int* list = s_list[threadIdx.x >> 5];
+        // candidates: upper bound reaches LB_k; a per-warp list in expert order
+        uint32_t cand = 0;
         int ncand = 0;
 #pragma unroll
         for (int m = 0; m < 8; m++) {
-            const bool c = m < nm && ((cand >> m) & 1u);
+            const bool c = m < nm && 32 * m + lane < p.E && ub[m] >= lbk;
+            cand |= (c ? 1u : 0u) << m;
             const uint32_t bal = __ballot_sync(0xffffffffu, c);
             if (c) list[ncand + __popc(bal & ((1u << lane) - 1u))] = 32 * m + lane;
             ncand += __popc(bal);
         }
         __syncwarp();
+        // their canonical logits, two at a time; lane e % 32 keeps expert e's,
+        // and lane i < 32 also holds candidate i's (for the sort below)
         float cv[8];
 #pragma unroll
         for (int m = 0; m < 8; m++) cv[m] = 0.0f;
-        for (int b0 = 0; b0 < ncand; b0 += RS_BATCH) {
-            const int n = min(RS_BATCH, ncand - b0);
-            int es[RS_BATCH];
+        float my_v = -INFINITY;
+        int my_e = 0x7FFFFFFF;
+        for (int i = 0; i < ncand; i += 2) {
+            const bool two = i + 1 < ncand;
+            const int e0 = list[i], e1 = two ? list[i + 1] : e0;
+            float c0, c1;
+            canonical_logit2(p, t, e0, e1, two, lane, c0, c1);
 #pragma unroll
-            for (int q = 0; q < RS_BATCH; q++) es[q] = q < n ? list[b0 + q] : 0;
-            float c[RS_BATCH];
-            canonical_logits(p, t, es, n, lane, c);
-#pragma unroll
-            for (int q = 0; q < RS_BATCH; q++) {
-                if (q < n && (es[q] & 31) == lane) {
-                    const int mq = es[q] >> 5;
+            for (int h = 0; h < 2; h++) {
+                if (h == 1 && !two) break;
+                const int e = h ? e1 : e0;
+                const float c = h ? c1 : c0;
+                if ((e & 31) == lane) {
 #pragma unroll
                     for (int m = 0; m < 8; m++)
-                        if (m == mq) cv[m] = c[q];
-                    lrow[es[q]] = c[q];
+                        if (m == (e >> 5)) cv[m] = c;
+                    lrow[e] = c;
+                }
+                if (lane == i + h) {
+                    my_v = c;
+                    my_e = e;
                 }
             }
         }
         __syncwarp();   // the list is rewritten for the warp's next token
-        router_topk_candidates(p, cv, cand, t, lane);
+        if (ncand > 32) {
+            router_topk_candidates(p, cv, cand, t, lane);
+            continue;
+        }
+        // at most 32 candidates: a bitonic sort over the lanes in selection order
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, my_v, stride);
+                const int oe = __shfl_xor_sync(0xffffffffu, my_e, stride);
+                const bool lower = (lane & stride) == 0;           // this lane keeps the earlier rank ...
+                const bool up = (lane & size) == 0;                // ... in an ascending-rank block
+                const bool other_first = rank_before(ov, oe, my_v, my_e);
+                if (lower == up ? other_first : !other_first) {
+                    my_v = ov;
+                    my_e = oe;
+                }
+            }
+        }
+        // lanes 0..k-1 hold the top k in order; weights as router_topk_select
+        float sel_v[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) sel_v[j] = __shfl_sync(0xffffffffu, my_v, j);
+        if (lane == 0) {
+            float z[8], sum = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (j >= p.k) break;
+                z[j] = (p.score == 0) ? expf(sel_v[j] - sel_v[0]) : 1.0f / (1.0f + expf(-sel_v[j]));
+                sum += z[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (j >= p.k) break;
+                p.w[static_cast<size_t>(t) * p.k + j] = z[j] / sum;
+            }
+        }
+        if (lane < p.k) p.ids[static_cast<size_t>(t) * p.k + lane] = my_e;
     }
 }
 

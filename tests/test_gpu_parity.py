@@ -199,8 +199,8 @@ def router_filter_bound(x_bf16, wr, bias, l_stored):
     and the canonical one, restated from its definition: fixed-point rows
     rounded at half of 2^(e - 14) (e the smallest integer with max|row| <=
     2^e), the canonical chain's gamma(H/32 + 6) (sum|x w| + |b|) with
-    sum|x w| <= min(sum|x| max|w|, max|x| sum|w|), and the fp32 storage of
-    the approximation."""
+    sum|x w| <= min(sum|x| max|w|, max|x| sum|w|), and the fp32 evaluation
+    of the approximation (2^-23 (|l| + |b|) + 2^-126)."""
     x = x_bf16.float().numpy().astype(np.float64)
     w = np.asarray(wr, np.float64)
     H = x.shape[1]
@@ -219,7 +219,8 @@ def router_filter_bound(x_bf16, wr, bias, l_stored):
     dfix = np.exp2(ew - 15.0)[None, :] * sx[:, None] + np.exp2(ex - 15.0)[:, None] * swq[None, :]
     sxw = np.minimum(sx[:, None] * mw[None, :], mx[:, None] * sw[None, :])
     b = np.zeros(w.shape[0]) if bias is None else np.abs(np.asarray(bias, np.float64))
-    return (dfix + gamma * (sxw + b[None, :]) + np.abs(l_stored.astype(np.float64)) * 2.0 ** -23) * (1 + 2.0 ** -20)
+    dst = (np.abs(l_stored.astype(np.float64)) + b[None, :]) * 2.0 ** -23 + 2.0 ** -126
+    return (dfix + gamma * (sxw + b[None, :]) + dst) * (1 + 2.0 ** -20)
 
 
 @pytest.mark.parametrize("T", [129, 300])
@@ -569,7 +570,7 @@ def test_cta_pairs_match_single_ctas(name):
     assert (hq_pair != hq_single).float().mean().item() <= 1e-3
     assert tolerance_violations(y_pair.float().cpu().numpy(), y_single.float().cpu().numpy()) == 0
     with pytest.raises(native.MoeError):
-        native.moe_set_gemm_options(layer.h, 2)
+        native.moe_set_gemm_options(layer.h, 3)
 
 
 def test_empty_batch():
