@@ -190,13 +190,18 @@ def launches_per_step(wl, T):
     """Kernels of one moe_forward call: router (logits + top-k; one fused kernel
     for T <= 128 and E <= 32; above 128 tokens with more than 8 experts the
     fixed-point rows, the integer tensor-core pass and the candidate select),
-    dispatch (hist, scan, rank, quantise; one fused kernel for the first three
-    when T*k <= 1024; + amax for NVFP4), gate/up, down, combine."""
+    dispatch (hist, scan, rank, quantise; for T*k <= 1024 one kernel for all
+    four with FP8, one for the first three with NVFP4; + amax for NVFP4),
+    gate/up, down, combine."""
     if T <= 128:
         route = 1 if wl.E <= 32 else 2
     else:
         route = 3 if wl.E > 8 else 2
-    return route + (2 if T * wl.k <= 1024 else 4) + (1 if wl.fmt == FMT_NVFP4 else 0) + 3
+    if T * wl.k <= 1024:
+        dispatch = 3 if wl.fmt == FMT_NVFP4 else 1     # fused dispatch + quantisation for FP8
+    else:
+        dispatch = 5 if wl.fmt == FMT_NVFP4 else 4
+    return route + dispatch + 3
 
 
 def measure(native, layer, wl, T, x, wr, bias, args, world, dev, clk, e2e=True, min_region_s=0.5):

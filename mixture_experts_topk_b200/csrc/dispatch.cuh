@@ -379,10 +379,74 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(const __nv_bfloat16*
     }
 }
 
-// Small batches: the same quantisation with one 256-thread CTA per token, so a
-// row's loads are spread over 8 warps.  Thread i handles columns 8 (i + 256 m);
-// a 128-column block is 16 consecutive lanes, the row amax (FP8_ROW) is a
-// warp then CTA maximum.  Same operations per element as quant_scatter_kernel.
+// Quantise token row t with one 256-thread CTA and write it to the slots
+// slot[0..k) (-1: none).  Thread i handles columns 8 (i + 256 m); a 128-column
+// block is 16 consecutive lanes, the row amax (FP8_ROW) is a warp then CTA
+// maximum.  Same operations per element as quant_scatter_kernel.  s_amax: 8
+// floats of shared memory.
+template <int FMT>
+__device__ __forceinline__ void quant_row_to_slots(const __nv_bfloat16* x, int t, int H, int k, const int* slot,
+                                                   uint8_t* xq, float* xs, float* s_amax) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
+    float s_row = 0.0f;
+    if (FMT == 0) {
+        float amax = 0.0f;
+        for (int m = 0; 8 * (tid + 256 * m) < H; m++) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + 8 * (tid + 256 * m)));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) s_amax[warp] = amax;
+        __syncthreads();
+        amax = s_amax[0];
+#pragma unroll
+        for (int w = 1; w < 8; w++) amax = fmaxf(amax, s_amax[w]);
+        __syncthreads();   // s_amax is rewritten for the next token
+        s_row = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+        for (int j = 0; j < 8; j++)
+            if (j < k && j == tid && slot[j] >= 0) xs[slot[j]] = s_row;
+    }
+    for (int m = 0; 8 * (tid + 256 * m) < H; m++) {
+        const int c0 = 8 * (tid + 256 * m);
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + c0));
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        float s = s_row;
+        if (FMT == 1) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            s = __fdiv_rn(amax, 448.0f);
+            if ((lane & 15) == 0) {
+#pragma unroll
+                for (int j = 0; j < 8; j++)
+                    if (j < k && slot[j] >= 0) xs[static_cast<size_t>(slot[j]) * (H >> 7) + (c0 >> 7)] = s;
+            }
+        }
+        uint32_t packed[2];
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const float a = bf16_lo(u[q]), b = bf16_hi(u[q]);
+            const uint16_t c = (s == 0.0f) ? static_cast<uint16_t>(0)
+                                           : f2_to_e4m3x2(__fdiv_rn(a, s), __fdiv_rn(b, s));
+            if (q & 1) packed[q >> 1] |= static_cast<uint32_t>(c) << 16;
+            else packed[q >> 1] = c;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++)
+            if (j < k && slot[j] >= 0)
+                *reinterpret_cast<uint2*>(xq + static_cast<size_t>(slot[j]) * H + c0) = make_uint2(packed[0], packed[1]);
+    }
+}
+
+// Small batches: the quantisation with one 256-thread CTA per token, so a
+// row's loads are spread over 8 warps.
 template <int FMT>
 __global__ void __launch_bounds__(256) quant_scatter_row_kernel(const __nv_bfloat16* x, int T, int H, int k,
                                                                 const int32_t* inv, uint8_t* xq, float* xs) {
@@ -390,67 +454,119 @@ __global__ void __launch_bounds__(256) quant_scatter_row_kernel(const __nv_bfloa
     pdl_trigger();
     KTRACE(TR_QUANT_ROW);
     __shared__ float s_amax[8];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         int slot[8];
 #pragma unroll
         for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
-        const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
-        float s_row = 0.0f;
-        if (FMT == 0) {
-            float amax = 0.0f;
-            for (int m = 0; 8 * (tid + 256 * m) < H; m++) {
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + 8 * (tid + 256 * m)));
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        quant_row_to_slots<FMT>(x, t, H, k, slot, xq, xs, s_amax);
+    }
+}
+
+// Small batches (A <= DISPATCH_CHUNK assignments): the dispatch and the X
+// quantisation in one launch, one 256-thread CTA per token.  Every CTA reads
+// all A ids and derives the histogram, the offsets and the slots of its own
+// token's k assignments itself -- slot of a = offsets[e] + #{a' < a : ids[a'] ==
+// e}, the stable order of rank_kernel -- so the CTAs need nothing from one
+// another.  CTA 0 also writes the counts, offsets, row-tile table, tile
+// pointers and picks (the packed (count, tiles) scan of scan_kernel) and resets
+// the per-expert gate/up counters.  Then the CTA quantises its token's row as
+// quant_scatter_row_kernel does.  Same results as dispatch_small_kernel +
+// quant_scatter_row_kernel.
+template <int FMT>
+__global__ void __launch_bounds__(256) dispatch_quant_small_kernel(
+    const int32_t* ids, int A, int E, int T, int H, int k, const __nv_bfloat16* x, int32_t* counts, int32_t* offsets,
+    int32_t* tiles, int32_t* num_tiles, int32_t* tile_ptr, int32_t* pick_out, PickerParams pq, int32_t* perm,
+    int32_t* inv, int32_t* status, int32_t* gu_done, uint8_t* xq, float* xs) {
+    pdl_wait();
+    pdl_trigger();
+    KTRACE(TR_DISPATCH_SMALL);
+    __shared__ int s_ids[DISPATCH_CHUNK];
+    __shared__ int s_cnt[256];
+    __shared__ int s_off[256];
+    __shared__ int warp_tot[8];
+    __shared__ int s_slot[8];
+    __shared__ float s_amax[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int a = tid; a < A; a += 256) s_ids[a] = ids[a];
+    s_cnt[tid] = 0;
+    __syncthreads();
+    for (int a = tid; a < A; a += 256) {
+        const int e = s_ids[a];
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&s_cnt[e], 1);
+        else if (blockIdx.x == 0) report(status, ST_BOUNDS, WHERE_DISPATCH);
+    }
+    __syncthreads();
+    // exclusive scan over experts of the packed (count, row tiles), as scan_kernel
+    const int c = tid < E ? s_cnt[tid] : 0;
+    const int nt_e = (c + TILE_M - 1) / TILE_M;
+    const int packed = c + (nt_e << 20);
+    int inc = packed;
 #pragma unroll
-                for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
-            }
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += n;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    const int touched = __syncthreads_count(tid < E && c > 0);
+    if (warp == 0) {
+        int w = lane < 8 ? warp_tot[lane] : 0;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            if (lane == 0) s_amax[warp] = amax;
-            __syncthreads();
-            amax = s_amax[0];
-#pragma unroll
-            for (int w = 1; w < 8; w++) amax = fmaxf(amax, s_amax[w]);
-            __syncthreads();   // s_amax is rewritten for the next token
-            s_row = __fdiv_rn(amax, 448.0f);
-#pragma unroll
-            for (int j = 0; j < 8; j++)
-                if (j == tid && slot[j] >= 0) xs[slot[j]] = s_row;
+        for (int off = 1; off < 8; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += n;
         }
-        for (int m = 0; 8 * (tid + 256 * m) < H; m++) {
-            const int c0 = 8 * (tid + 256 * m);
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + c0));
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-            float s = s_row;
-            if (FMT == 1) {
-                float amax = 0.0f;
-#pragma unroll
-                for (int q = 0; q < 4; q++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[q])), fabsf(bf16_hi(u[q]))));
-#pragma unroll
-                for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-                s = __fdiv_rn(amax, 448.0f);
-                if ((lane & 15) == 0) {
-#pragma unroll
-                    for (int j = 0; j < 8; j++)
-                        if (slot[j] >= 0) xs[static_cast<size_t>(slot[j]) * (H >> 7) + (c0 >> 7)] = s;
-                }
-            }
-            uint32_t packed[2];
-#pragma unroll
-            for (int q = 0; q < 4; q++) {
-                const float a = bf16_lo(u[q]), b = bf16_hi(u[q]);
-                const uint16_t c = (s == 0.0f) ? static_cast<uint16_t>(0)
-                                               : f2_to_e4m3x2(__fdiv_rn(a, s), __fdiv_rn(b, s));
-                if (q & 1) packed[q >> 1] |= static_cast<uint32_t>(c) << 16;
-                else packed[q >> 1] = c;
-            }
-#pragma unroll
-            for (int j = 0; j < 8; j++)
-                if (slot[j] >= 0)
-                    *reinterpret_cast<uint2*>(xq + static_cast<size_t>(slot[j]) * H + c0) =
-                        make_uint2(packed[0], packed[1]);
+        if (lane < 8) warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int excl = (warp ? warp_tot[warp - 1] : 0) + inc - packed;
+    const int total = warp_tot[7];
+    const int off_e = excl & 0xFFFFF, tptr_e = excl >> 20;
+    s_off[tid] = off_e;
+    if (blockIdx.x == 0) {
+        if (tid == 0) {
+            offsets[E] = total & 0xFFFFF;
+            *num_tiles = total >> 20;
+            tile_ptr[E] = total >> 20;
+            pick_out[0] = pick_down_tile(pq, total >> 20, touched);
+            pick_out[1] = pick_split(pq, total >> 20, total & 0xFFFFF);
         }
+        if (tid < E) {
+            counts[tid] = c;
+            offsets[tid] = off_e;
+            gu_done[tid] = 0;
+            tile_ptr[tid] = tptr_e;
+            for (int i = 0; i < nt_e; i++) {
+                tiles[2 * (tptr_e + i)] = tid;
+                tiles[2 * (tptr_e + i) + 1] = off_e + TILE_M * i;
+            }
+        }
+    }
+    __syncthreads();
+    // the slots of this CTA's token: warp j ranks assignment t k + j among the
+    // earlier ones with the same expert
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        if (warp < k) {
+            const int a = t * k + warp;
+            const int e = s_ids[a];
+            const bool valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
+            int cnt = 0;
+            if (valid)
+                for (int a2 = lane; a2 < a; a2 += 32) cnt += s_ids[a2] == e;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+            if (lane == 0) {
+                const int slot = valid ? s_off[e] + cnt : -1;
+                s_slot[warp] = slot;
+                inv[a] = slot;
+                if (valid) perm[slot] = a;
+            }
+        }
+        __syncthreads();
+        int slot[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) slot[j] = j < k ? s_slot[j] : -1;
+        __syncthreads();   // s_slot is rewritten for the next token
+        quant_row_to_slots<FMT>(x, t, H, k, slot, xq, xs, s_amax);
     }
 }
 

@@ -575,6 +575,15 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
     const int A = T * c.k;
     const int nchunks = (A + DISPATCH_CHUNK - 1) / DISPATCH_CHUNK;
     int32_t* chunk = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + h->ws.chunk);
+    if (A > 0 && nchunks == 1 && c.fmt != MOE_FMT_NVFP4) {
+        // one chunk: the dispatch and the quantisation in one launch, a CTA per token
+        LAUNCH(h->pdl, "dispatch_quant_small_kernel",
+               c.fmt == MOE_FMT_FP8_ROW ? dispatch_quant_small_kernel<0> : dispatch_quant_small_kernel<1>,
+               std::min(T, 8 * h->num_sms), 256, 0, st, ids, A, c.E, T, c.H, c.k,
+               static_cast<const __nv_bfloat16*>(x), v.counts, v.offsets, v.tiles, v.num_tiles, v.tile_ptr, v.pick,
+               h->picker, v.perm, v.inv, v.status, gu_done_of(h, ws), v.xq, static_cast<float*>(v.xs));
+        return MOE_OK;
+    }
     if (A > 0 && nchunks == 1) {
         // one chunk: histogram, scan and ranks in one CTA
         LAUNCH(h->pdl, "dispatch_small_kernel", dispatch_small_kernel, 1, DISPATCH_CHUNK, 0, st, ids, A, c.E,
@@ -755,7 +764,18 @@ static int max_m_tiles(const moe_config& c, int T) {
 }
 
 // ------------------------------------------------------------------ gate/up
+// publish: the FP8_ROW gate/up epilogue counts each finished part of a tile
+// per expert (a fence and an atomic per warp and tile) for a down GEMM chained
+// behind it (mx_down with chained = true); without such a consumer it does not.
+static moe_status gate_up_impl(const moe_handle* h, const void* packed, int T, void* ws, moe_stream_t stream,
+                               bool publish);
+
 extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T, void* ws, moe_stream_t stream) {
+    return gate_up_impl(h, packed, T, ws, stream, false);
+}
+
+static moe_status gate_up_impl(const moe_handle* h, const void* packed, int T, void* ws, moe_stream_t stream,
+                               bool publish) {
     moe_status st0 = check_T(h, T, "moe_gate_up");
     if (st0 != MOE_OK) return st0;
     if (T == 0) return MOE_OK;
@@ -796,7 +816,7 @@ extern "C" moe_status moe_gate_up(const moe_handle* h, const void* packed, int T
     p.act = c.act;
     p.act_alpha = c.act_alpha;
     p.act_limit = c.act_limit;
-    p.gu_done = c.fmt == MOE_FMT_FP8_ROW ? gu_done_of(h, ws) : nullptr;
+    p.gu_done = (c.fmt == MOE_FMT_FP8_ROW && publish) ? gu_done_of(h, ws) : nullptr;
     p.status = v.status;
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
@@ -1057,13 +1077,21 @@ extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws,
 }
 
 // ------------------------------------------------------------------ layer
+constexpr long long CHAIN_MAX_A = 4096;
+
 extern "C" moe_status moe_forward_routed(const moe_handle* h, const void* x, int T, const int32_t* ids, const float* w,
                                          const void* packed, void* y, void* ws, moe_stream_t stream) {
     moe_status r = moe_dispatch(h, x, ids, T, ws, stream);
     if (r != MOE_OK) return r;
-    r = moe_gate_up(h, packed, T, ws, stream);
+    // FP8_ROW batches of at most CHAIN_MAX_A assignments chain the down GEMM
+    // behind the gate/up GEMM (per-expert waits, so it starts on the SMs the
+    // gate/up GEMM's last wave leaves idle); larger batches fill every SM with
+    // gate/up tiles to the end, where the per-tile counting only costs time
+    const bool chained = h->cfg.fmt == MOE_FMT_FP8_ROW && T > 0 && h->pdl &&
+                         static_cast<long long>(T) * h->cfg.k <= CHAIN_MAX_A;
+    r = gate_up_impl(h, packed, T, ws, stream, chained);
     if (r != MOE_OK) return r;
-    if (h->cfg.fmt == MOE_FMT_FP8_ROW && T > 0 && h->pdl) {
+    if (chained) {
         if (!w) return fail(MOE_ERR_INVALID_ARG, "moe_forward_routed: null argument");
         r = mx_down(h, packed, w, T, ws, stream, true);
     } else {
