@@ -434,6 +434,19 @@ def run_ours(args, rank, world, local_rank):
     del d                      # the packed copy is all the layer reads
     torch.cuda.empty_cache()
     x = synth.tokens(wl, T, seed=rank, device=dev)
+    if args.profile:
+        # plain layer calls for a profiler's launch list: --warmup calls, then
+        # --steps more, nothing else launched and nothing timed
+        y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.warmup + args.steps):
+            native.moe_forward(layer.h, x, T, wr, bias, layer.packed, y, layer.ws)
+        torch.cuda.synchronize()
+        st, msg = layer.status()
+        layer.close()
+        if st != 0:
+            raise RuntimeError(f"device status: {msg}")
+        return {"profile": f"{wl.name} T={T}", "calls": args.warmup + args.steps,
+                "launches_per_call": launches_per_step(wl, T)}
     pk, pk_kind = peaks()
     with ClockSampler(local_rank) as clk:
         time.sleep(0.2)
@@ -559,6 +572,8 @@ def main():
                     help="FP8_ROW GEMMs on CTA pairs: 0 never, 1 by the library's rule (default), 2 always")
     ap.add_argument("--act", default="swiglu", choices=sorted(ACTS),
                     help="gated activation of the expert MLP (bounded: clamp 10; oai: alpha 1.702, limit 7)")
+    ap.add_argument("--profile", action="store_true",
+                    help="only run --warmup + --steps plain layer calls (for a profiler's launch list)")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="timed steps replay a CUDA graph of the layer call, or call it directly")
     args = ap.parse_args()
@@ -580,7 +595,7 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     out = run_ours(args, rank, world, local_rank)
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not args.profile:
             cb = cpu_baseline(workload_of(args), args.tokens, args.ref_sample)
             cb.pop("seconds")
             out["cpu_baseline"] = cb

@@ -144,8 +144,9 @@ typedef struct {
     int32_t* offsets;    /* [E+1] exclusive prefix sum of counts (m_indptr) */
     int32_t* num_tiles;  /* [1] row tiles of 128 over all experts */
     int32_t* tile_ptr;   /* [E+1] index of each expert's first row tile */
-    int32_t* pick;       /* [2] choices from the histogram: [0] down GEMM tile (0 -> 256, 1 -> 128, 2 -> 64
-                          * columns, FP8_BLOCK128); [1] S, the K split of the FP8_ROW down GEMM (1 = none) */
+    int32_t* pick;       /* [3] choices from the histogram: [0] down GEMM tile (0 -> 256, 1 -> 128, 2 -> 64
+                          * columns, FP8_BLOCK128); [1] S, the K split of the FP8_ROW down GEMM (1 = none);
+                          * [2] the FP8_ROW SwiGLU gate/up GEMM on CTA pairs (1) or single CTAs (0) */
     int32_t* tiles;      /* [A/128 + E + 1][2] (expert, first row) per row tile */
     int32_t* perm;       /* [A] slot -> t*k + j */
     int32_t* inv;        /* [A] t*k + j -> slot */
@@ -256,17 +257,18 @@ moe_status moe_set_tile_config(moe_handle* h, int down_bn);
  * plain stream order.  Host state only; MOE_ERR_INVALID_ARG for other values. */
 moe_status moe_set_launch_options(moe_handle* h, int pdl);
 
-/* GEMM options.  cta_pairs = 1 (the default): an FP8_ROW SwiGLU layer whose
- * batch holds at least 4 row tiles of 128 per expert on average
- * (T*k >= 512 E) runs the gate/up GEMM on CTA pairs: 2-CTA clusters whose
+/* GEMM options.  cta_pairs = 1 (the default): an FP8_ROW SwiGLU layer runs
+ * the gate/up GEMM on CTA pairs where the dispatch's cost model picks them
+ * from the expert histogram (moe_set_pair_params): 2-CTA clusters whose
  * tcgen05.mma.cta_group::2 covers two row tiles of one expert (M = 256), each
  * CTA loading its own 128 rows of X and half of the 256 weight rows (no
  * multicast), so a 32 KB stage feeds what a 48 KB stage feeds alone.  With
- * I > 2048 (FP8_ROW, any activation), and where the output rows leave no room
- * for a K split of the down GEMM, the down GEMM runs on CTA pairs the same
- * way (each CTA loading its hidden rows, their scale chunk and 128 of the 256
- * rows of W_down).  An expert with an odd row-tile count runs its last pair
- * half empty.  The
+ * I > 2048 (FP8_ROW, any activation), where the output rows leave no room for
+ * a K split of the down GEMM and the batch holds at least 4 row tiles per
+ * expert on average (T*k >= 512 E, a host-side rule), the down GEMM runs on
+ * CTA pairs the same way (each CTA loading its hidden rows, their scale chunk
+ * and 128 of the 256 rows of W_down).  An expert with an odd row-tile count
+ * runs its last pair half empty.  The
  * results are those of the single-CTA kernel up to the fp32 summation order
  * inside the tensor core.  cta_pairs = 0 keeps single CTAs; cta_pairs = 2
  * runs these GEMMs on CTA pairs at every batch size (the down GEMM still only
@@ -302,6 +304,22 @@ moe_status moe_set_wait_limit(moe_handle* h, long long cycles);
  * params = {alpha, beta, bw, gamma}; get also returns num_sms in params[4]. */
 moe_status moe_set_picker_params(moe_handle* h, const long long* params);
 moe_status moe_get_picker_params(const moe_handle* h, long long* params);
+
+/* Parameters of the model that picks, from the runtime expert histogram, whether
+ * the FP8_ROW SwiGLU gate/up GEMM runs on single CTAs or on CTA pairs (RaMP
+ * abstract: a cost model of CTA waves, fitted once to a profiling sweep).  The
+ * dispatch evaluates, with mt_e = ceil(count_e / 128), m_tiles = sum_e mt_e,
+ * n_odd = #{e : mt_e odd}, nb = 2I / 256 n-blocks and kb = H / 128 K-blocks:
+ *   single = ceil(m_tiles nb / num_sms) (kb a_s + b_s)
+ *   pair   = ceil((m_tiles + n_odd) / 2 nb / (num_sms / 2)) (kb a_p + b_p)
+ * (integers, picoseconds) and writes view.pick[2] = 1 (pairs) when pair <
+ * single, else 0; the gate/up kernel, launched as 2-CTA clusters, reads it.
+ * params = {a_s, b_s, a_p, b_p}; get also returns nb, kb and num_sms in
+ * params[4..6] (nb = 0: the layer has no choice, single CTAs).  Host state only;
+ * MOE_ERR_INVALID_ARG for a negative cost.  moe_set_gemm_options overrides
+ * the pick. */
+moe_status moe_set_pair_params(moe_handle* h, const long long* params);
+moe_status moe_get_pair_params(const moe_handle* h, long long* params);
 
 /* Deterministic combine (LightMoE README, "Highlights": deterministic
  * combine): y[t] = bf16( sum_{j=0..k-1} o[inv[t k + j]] ) in fixed j order,

@@ -38,7 +38,30 @@ struct PickerParams {
     int split_nb;              // n-blocks of a K-splittable down GEMM (0: no split)
     int split_kb;              // its K-blocks
     int o_rows;                // rows of the fp32 down-output buffer
+    // gate/up GEMM on single CTAs or on CTA pairs (pick_gu_pairs)
+    int gu_nb;                 // its n-blocks (0: no choice, single CTAs)
+    int gu_kb;                 // its K-blocks
+    long long gu_ps[4];        // per-unit cost kb * a + b: single (a, b), pair (a, b), picoseconds
 };
+
+// Gate/up GEMM on single CTAs or on 2-CTA pairs (M = 256 over two m-tiles of
+// one expert), chosen from the expert histogram.  A single unit is an
+// (m-tile, n-block), num_sms run at once; a pair unit is an (m-pair, n-block)
+// whose m-tiles are an expert's 2j and 2j + 1 (the second absent for the last
+// of an odd count), num_sms / 2 run at once.  With m_tiles = sum_e mt_e and
+// n_odd = #{e : mt_e odd}:
+//   single = ceil(m_tiles nb / num_sms) (kb a_s + b_s)
+//   pair   = ceil((m_tiles + n_odd) / 2 nb / (num_sms / 2)) (kb a_p + b_p)
+// Pairs when strictly cheaper (1), else single CTAs (0).
+__host__ __device__ inline int pick_gu_pairs(const PickerParams& q, int m_tiles, int n_odd) {
+    if (q.gu_nb <= 0 || m_tiles <= 0) return 0;
+    const long long su = static_cast<long long>(m_tiles) * q.gu_nb;
+    const long long pu = static_cast<long long>((m_tiles + n_odd) / 2) * q.gu_nb;
+    const long long ns = q.num_sms, np = q.num_sms / 2;
+    const long long c_s = (su + ns - 1) / ns * (q.gu_kb * q.gu_ps[0] + q.gu_ps[1]);
+    const long long c_p = (pu + np - 1) / np * (q.gu_kb * q.gu_ps[2] + q.gu_ps[3]);
+    return c_p < c_s ? 1 : 0;
+}
 
 // Split of the down GEMM's K for small batches: when the (m-tile, n-block)
 // units leave SMs idle, each unit's K-blocks are cut into S near-equal ranges
@@ -141,6 +164,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
     }
     if (lane == 31) warp_tot[warp] = inc;
     const int touched = __syncthreads_count(e < E && c > 0);
+    const int n_odd = __syncthreads_count(e < E && (nt_e & 1));
     if (warp == 0) {
         int w = lane < 8 ? warp_tot[lane] : 0;
 #pragma unroll
@@ -162,6 +186,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
         if (pick_out) {
             pick_out[0] = pick_down_tile(pq, trun, touched);
             pick_out[1] = pick_split(pq, trun, A);
+            pick_out[2] = pick_gu_pairs(pq, trun, n_odd);
         }
     }
     if (e < E) {
@@ -259,6 +284,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK) dispatch_small_kernel(
     }
     if (warp < 8 && lane == 31) warp_tot[warp] = inc;
     const int touched = __syncthreads_count(tid < E && c > 0);
+    const int n_odd = __syncthreads_count(tid < E && (nt_e & 1));
     if (warp == 0) {
         int w = lane < 8 ? warp_tot[lane] : 0;
 #pragma unroll
@@ -279,6 +305,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK) dispatch_small_kernel(
             tile_ptr[E] = total >> 20;
             pick_out[0] = pick_down_tile(pq, total >> 20, touched);
             pick_out[1] = pick_split(pq, total >> 20, total & 0xFFFFF);
+            pick_out[2] = pick_gu_pairs(pq, total >> 20, n_odd);
         }
         if (tid < E) {
             counts[tid] = c;
@@ -508,6 +535,7 @@ __global__ void __launch_bounds__(256) dispatch_quant_small_kernel(
     }
     if (lane == 31) warp_tot[warp] = inc;
     const int touched = __syncthreads_count(tid < E && c > 0);
+    const int n_odd = __syncthreads_count(tid < E && (nt_e & 1));
     if (warp == 0) {
         int w = lane < 8 ? warp_tot[lane] : 0;
 #pragma unroll
@@ -529,6 +557,7 @@ __global__ void __launch_bounds__(256) dispatch_quant_small_kernel(
             tile_ptr[E] = total >> 20;
             pick_out[0] = pick_down_tile(pq, total >> 20, touched);
             pick_out[1] = pick_split(pq, total >> 20, total & 0xFFFFF);
+            pick_out[2] = pick_gu_pairs(pq, total >> 20, n_odd);
         }
         if (tid < E) {
             counts[tid] = c;
@@ -575,10 +604,13 @@ __global__ void __launch_bounds__(256) dispatch_quant_small_kernel(
 // two scale per 32 columns (value = fp16 * 2^(oe - 15), exact in fp32), in S
 // copies of A rows when the down GEMM split its K (S from the dispatch's pick,
 // clamped to [1, s_max]), so the only rounding to bf16 is the final one.
-// A thread takes 16 columns (32 bytes of each row, one exponent), so that the
-// k rows' loads in flight per thread are as many bytes as with fp32 rows.
+// A thread takes 16 columns (32 bytes of each row, one exponent) of a group of
+// G = max(1, 8 / k) consecutive tokens, so that up to 8 rows' loads are in
+// flight per thread whatever k is: all loads of the group are issued before
+// the first is used (a load followed by its use would keep one row in flight).
 constexpr int COMBINE_COLS = 16;
 constexpr int COMBINE_THREADS = 128;
+__host__ __device__ constexpr int combine_group(int k) { return k >= 8 ? 1 : 8 / k; }
 __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const uint16_t* o, const int8_t* oe,
                                                                   const int32_t* inv, int T, int H, int k,
                                                                   const int32_t* split, int s_max, __nv_bfloat16* y) {
@@ -588,21 +620,35 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const uint16_t
     const int S = split ? min(max(*split, 1), s_max) : 1;
     const size_t copy = static_cast<size_t>(T) * k;   // rows per copy
     const int HB = H >> 5;                            // exponent bytes per row
+    const int G = combine_group(k);
     constexpr int SPAN = COMBINE_COLS * COMBINE_THREADS;
-    // CTA (x, y): tokens x, x + gridDim.x, ..., columns [SPAN y, SPAN y + SPAN)
+    // CTA (x, y): token groups x, x + gridDim.x, ..., columns [SPAN y, SPAN y + SPAN)
     const int c_end = min(H, SPAN * (static_cast<int>(blockIdx.y) + 1));
-    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    for (int t0 = blockIdx.x * G; t0 < T; t0 += gridDim.x * G) {
+        // row r of the group: token t0 + r / k, its j = r % k
         int slot[8];
 #pragma unroll
-        for (int j = 0; j < 8; j++) slot[j] = (j < k) ? inv[static_cast<size_t>(t) * k + j] : -1;
+        for (int r = 0; r < 8; r++) {
+            const int g = r / k, j = r - g * k;
+            slot[r] = (g < G && t0 + g < T) ? inv[static_cast<size_t>(t0 + g) * k + j] : -1;
+        }
         for (int c0 = SPAN * blockIdx.y + COMBINE_COLS * threadIdx.x; c0 < c_end; c0 += SPAN) {
-            float acc[16];
+            uint4 q[8][2];
+            int8_t ex[8];
+            if (S == 1) {
 #pragma unroll
-            for (int i = 0; i < 16; i++) acc[i] = 0.0f;
-            auto add_row = [&](size_t row) {
-                const uint4* src = reinterpret_cast<const uint4*>(o + row * H + c0);
-                const uint4 q0 = src[0], q1 = src[1];
-                const float sc = __int_as_float((127 - 15 + oe[row * HB + (c0 >> 5)]) << 23);
+                for (int r = 0; r < 8; r++) {
+                    if (slot[r] < 0) continue;
+                    const size_t row = static_cast<size_t>(slot[r]);
+                    const uint4* src = reinterpret_cast<const uint4*>(o + row * H + c0);
+                    q[r][0] = src[0];
+                    q[r][1] = src[1];
+                    ex[r] = oe[row * HB + (c0 >> 5)];
+                }
+            }
+            float acc[16];
+            auto add = [&](const uint4& q0, const uint4& q1, int8_t e8) {
+                const float sc = __int_as_float((127 - 15 + e8) << 23);
                 const uint32_t wq[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
                 for (int i = 0; i < 8; i++) {
@@ -611,27 +657,37 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const uint16_t
                     acc[2 * i + 1] += f.y * sc;
                 }
             };
-            if (S == 1) {
-                // all k rows' loads in flight at once
 #pragma unroll
-                for (int j = 0; j < 8; j++)
-                    if (slot[j] >= 0) add_row(static_cast<size_t>(slot[j]));
-            } else {
+            for (int r = 0; r < 8; r++) {
+                const int g = r / k, j = r - g * k;
+                if (g >= G || t0 + g >= T) continue;
+                if (j == 0) {
 #pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    if (slot[j] < 0) continue;
-                    for (int sp = 0; sp < S; sp++) add_row(static_cast<size_t>(sp) * copy + slot[j]);
+                    for (int i = 0; i < 16; i++) acc[i] = 0.0f;
+                }
+                if (slot[r] >= 0) {
+                    if (S == 1) {
+                        add(q[r][0], q[r][1], ex[r]);
+                    } else {
+                        for (int sp = 0; sp < S; sp++) {
+                            const size_t row = static_cast<size_t>(sp) * copy + slot[r];
+                            const uint4* src = reinterpret_cast<const uint4*>(o + row * H + c0);
+                            add(src[0], src[1], oe[row * HB + (c0 >> 5)]);
+                        }
+                    }
+                }
+                if (j == k - 1) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+                        w[i] = *reinterpret_cast<const uint32_t*>(&b2);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(y + static_cast<size_t>(t0 + g) * H + c0);
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                 }
             }
-            uint32_t r[8];
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-                r[q] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + c0);
-            dst[0] = make_uint4(r[0], r[1], r[2], r[3]);
-            dst[1] = make_uint4(r[4], r[5], r[6], r[7]);
         }
     }
 }

@@ -901,6 +901,27 @@ __global__ void __launch_bounds__(gemm_threads<16>(), 1)
                                                                                    smem_raw);
 }
 
+// FP8_ROW gate/up GEMM whose CTA mode is chosen on the device: launched as
+// 2-CTA clusters; the dispatch's scan writes pick_gu_pairs to *cfg, and both
+// CTAs of every cluster read it and run either the pair body (M = 256 over two
+// m-tiles of an expert) or, each on its own, the single-CTA body.  No host
+// round trip.
+constexpr int GU_POLY_SMEM = GemmSmem<256, 4, 16>::TOTAL > GemmSmem<256, GU_PAIR_STAGES, 16, true>::TOTAL
+                                 ? GemmSmem<256, 4, 16>::TOTAL
+                                 : GemmSmem<256, GU_PAIR_STAGES, 16, true>::TOTAL;
+template <int ACT>
+__global__ void __launch_bounds__(gemm_threads<16>(), 1)
+    grouped_gemm_gu_poly_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB256,
+                                const __grid_constant__ CUtensorMap tmB128, const GemmParams p, const int32_t* cfg) {
+    extern __shared__ uint8_t smem_raw[];
+    pdl_wait();   // the mode was picked by the dispatch scan
+    if (*cfg == 1)
+        gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 256, GU_PAIR_STAGES, 16, ACT, true>(tmA, tmB128, p, p.n_blocks,
+                                                                                       smem_raw);
+    else
+        gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, ACT>(tmA, tmB256, p, p.n_blocks, smem_raw);
+}
+
 // Down GEMM whose tile width is chosen on the device: the dispatch's scan
 // kernel evaluates the wave cost model on the expert histogram and writes the
 // choice (0: BN=256, 1: 128, 2: 64) to *cfg; every CTA reads it and runs that

@@ -192,7 +192,7 @@ static WsLayout make_ws_layout(const moe_config& c) {
     L.offsets = take((c.E + 1) * 4);
     L.num_tiles = take(4);
     L.tile_ptr = take((c.E + 1) * 4);
-    L.pick = take(8);
+    L.pick = take(16);
     L.gu_done = take(c.E * 4);
     L.chunk = take(nchunks * c.E * 4);
     L.tiles = take(tiles_cap * 8);
@@ -255,6 +255,16 @@ static WLayout make_w_layout(const moe_config& c) {
 }
 
 // ------------------------------------------------------------------ init
+// per-unit cost kb * a + b (ps) of a gate/up unit on a single CTA (a_s, b_s)
+// and on a CTA pair (a_p, b_p).  a_s is the per-K-block cost of a 128 x 256
+// unit from a least-squares fit of an interleaved B200 sweep of both modes
+// (the FP8_ROW SwiGLU workloads at every batch size, two more shapes);
+// a_p = a_s / 1.069 puts the boundary between the wave ratios at which pairs
+// measured faster (1.04) and slower (>= 1.07); b_p = 0.2 us, a pair unit's
+// fixed cost (cross-CTA arrivals), keeps batches that fill one wave either
+// way on single CTAs (a 16-token layer ran 39% slower on half-empty pairs).
+static const long long GU_PAIR_FIT[4] = {527000, 0, 493000, 200000};
+
 extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
     if (!cfg || !out) return fail(MOE_ERR_INVALID_ARG, "moe_init: null argument");
     const moe_config& c = *cfg;
@@ -303,6 +313,10 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
     h->picker.split_nb = c.fmt == MOE_FMT_FP8_ROW ? c.H / MX_BN : 0;
     h->picker.split_kb = c.I / 128;
     h->picker.o_rows = static_cast<int>(o_rows(c));
+    // gate/up CTA mode (FP8_ROW SwiGLU), per-unit costs fitted to a B200 sweep
+    h->picker.gu_nb = (c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU) ? 2 * c.I / 256 : 0;
+    h->picker.gu_kb = c.H / 128;
+    for (int i = 0; i < 4; i++) h->picker.gu_ps[i] = GU_PAIR_FIT[i];
     *out = h;
     return MOE_OK;
 }
@@ -791,9 +805,10 @@ static moe_status gate_up_impl(const moe_handle* h, const void* packed, int T, v
     if (r != MOE_OK) return r;
     const int n_gu = c.act == MOE_ACT_RELU2 ? c.I : 2 * c.I;   // rows of the packed gate/up weights
     // CTA pairs: each CTA loads half of a B tile's 256 rows
-    const bool pairs = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU &&
-                       (h->gemm_pairs == 2 || (h->gemm_pairs == 1 && static_cast<long long>(T) * c.k >= 4LL * TILE_M * c.E));
-    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, pairs ? 128 : 256);
+    // CTA pairs always (2), never (0), or picked on the device (1, the default)
+    const bool pair_kernel = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU && h->gemm_pairs == 2;
+    const bool poly = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU && h->gemm_pairs == 1;
+    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, pair_kernel ? 128 : 256);
     if (r != MOE_OK) return r;
     GemmParams p;
     memset(&p, 0, sizeof(p));
@@ -821,11 +836,25 @@ static moe_status gate_up_impl(const moe_handle* h, const void* packed, int T, v
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (pairs) {
-        // large batches (>= 4 m-tiles per expert on average): CTA pairs, so an odd
-        // m-tile count leaves at most one half-empty pair per expert
+    if (pair_kernel) {
         const int pairs = std::max(1, std::min(h->num_sms / 2, (max_m_tiles(c, T) + 1) / 2 * p.n_blocks));
         return launch_gemm_pairs<MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, 2 * pairs, st);
+    }
+    if (poly) {
+        // 2-CTA clusters; the dispatch's pick says whether they run as pairs or
+        // as single CTAs (an even grid large enough for either)
+        CUtensorMap tb128;
+        r = make_tmap(&tb128, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, 128);
+        if (r != MOE_OK) return r;
+        const int g2 = std::max(2, (std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks) + 1) / 2 * 2);
+        auto kern = grouped_gemm_gu_poly_kernel<MOE_ACT_SWIGLU>;
+        static_assert(GU_POLY_SMEM <= 232448, "shared memory of the GEMM exceeds 227 KB");
+        CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GU_POLY_SMEM));
+        const cudaError_t err = launch_k_pairs(h->pdl, kern, dim3(g2), dim3(gemm_threads<16>()), GU_POLY_SMEM, st, ta,
+                                               tb, tb128, p, static_cast<const int32_t*>(v.pick + 2));
+        if (err != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "launch of grouped_gemm_gu_poly_kernel failed: %s", cudaGetErrorString(err));
+        return MOE_OK;
     }
     if (c.fmt == MOE_FMT_FP8_ROW) {
         switch (c.act) {
@@ -1021,6 +1050,23 @@ extern "C" moe_status moe_get_picker_params(const moe_handle* h, long long* para
     return MOE_OK;
 }
 
+extern "C" moe_status moe_set_pair_params(moe_handle* h, const long long* params) {
+    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_set_pair_params: null argument");
+    for (int i = 0; i < 4; i++)
+        if (params[i] < 0) return fail(MOE_ERR_INVALID_ARG, "moe_set_pair_params: costs must be >= 0");
+    for (int i = 0; i < 4; i++) h->picker.gu_ps[i] = params[i];
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_get_pair_params(const moe_handle* h, long long* params) {
+    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_get_pair_params: null argument");
+    for (int i = 0; i < 4; i++) params[i] = h->picker.gu_ps[i];
+    params[4] = h->picker.gu_nb;
+    params[5] = h->picker.gu_kb;
+    params[6] = h->picker.num_sms;
+    return MOE_OK;
+}
+
 extern "C" moe_status moe_set_tile_config(moe_handle* h, int down_bn) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_tile_config: null handle");
     if (down_bn != 0 && down_bn != 64 && down_bn != 128 && down_bn != 256)
@@ -1061,13 +1107,14 @@ extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws,
     if (T == 0) return MOE_OK;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
-    // one CTA per (token group, 2048-column slice): small batches still spread.
+    // one CTA per (group of 8 / k tokens, 2048-column slice): small batches still spread.
     // Launched without the PDL attribute: launched early, its CTAs would be
     // placed on the few SMs the down GEMM leaves room on and run ~2x slower
     // (Qwen3.5 T=64: 5.4 vs 2.6 us) than when placed after the GEMM ends.
     constexpr int span = COMBINE_COLS * COMBINE_THREADS;
     const int ncb = (h->cfg.H + span - 1) / span;
-    const dim3 grid(std::max(1, std::min(T, 16 * h->num_sms / ncb)), ncb);
+    const int groups = (T + combine_group(h->cfg.k) - 1) / combine_group(h->cfg.k);
+    const dim3 grid(std::max(1, std::min(groups, 16 * h->num_sms / ncb)), ncb);
     LAUNCH(false, "combine_kernel", combine_kernel, grid, COMBINE_THREADS, 0, reinterpret_cast<cudaStream_t>(stream),
            static_cast<const uint16_t*>(v.o), static_cast<const int8_t*>(v.o_exp), static_cast<const int32_t*>(v.inv),
            T, h->cfg.H, h->cfg.k,

@@ -23,7 +23,7 @@ EXPORTED = (
     "moe_workspace_view_get", "moe_pack_weights", "moe_route", "moe_dispatch", "moe_gate_up",
     "moe_down", "moe_combine", "moe_forward", "moe_forward_routed", "moe_workspace_init",
     "moe_get_status", "moe_dispatch_noalloc", "moe_set_tile_config", "moe_set_launch_options", "moe_set_gemm_options", "moe_set_wait_limit", "moe_set_picker_params",
-    "moe_get_picker_params",
+    "moe_get_picker_params", "moe_set_pair_params", "moe_get_pair_params",
 )
 
 
@@ -89,6 +89,8 @@ def load(path=LIB_PATH):
             "moe_set_wait_limit": (I, [P, ctypes.c_longlong]),
             "moe_set_picker_params": (I, [P, P]),
             "moe_get_picker_params": (I, [P, P]),
+            "moe_set_pair_params": (I, [P, P]),
+            "moe_get_pair_params": (I, [P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -215,6 +217,18 @@ def moe_get_picker_params(h):
     """-> (alpha, beta, bw, gamma, num_sms)"""
     arr = (ctypes.c_longlong * 5)()
     _check(load().moe_get_picker_params(h, arr))
+    return tuple(arr)
+
+
+def moe_set_pair_params(h, a_s, b_s, a_p, b_p):
+    arr = (ctypes.c_longlong * 4)(a_s, b_s, a_p, b_p)
+    _check(load().moe_set_pair_params(h, arr))
+
+
+def moe_get_pair_params(h):
+    """(a_s, b_s, a_p, b_p, nb, kb, num_sms)"""
+    arr = (ctypes.c_longlong * 7)()
+    _check(load().moe_get_pair_params(h, arr))
     return tuple(arr)
 
 

@@ -76,6 +76,7 @@ def lib():
             "orc_num_threads": (I, []),
             "orc_pick_down_tile": (I, [P, I, I, I, I, I64, I64, I64, I64, P]),
             "orc_pick_split": (I, [P, I, I, I, I64, I]),
+            "orc_pick_gu_pairs": (I, [P, I, I, I, I, P]),
             "orc_glu": (ctypes.c_double, [I, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double]),
         }
         for name, (res, args) in sig.items():
@@ -201,6 +202,13 @@ def pick_split(counts, split_nb, split_kb, o_rows, num_sms):
 
 
 # ---------------------------------------------------------------- quantisers
+def pick_gu_pairs(counts, nb, kb, num_sms, ps):
+    """1: the FP8_ROW gate/up GEMM on CTA pairs, 0: single CTAs (moe_oracle.h)."""
+    c = _c(counts, np.int32)
+    p = _c(ps, np.int64)
+    return int(lib().orc_pick_gu_pairs(_p(c), c.size, nb, kb, num_sms, _p(p)))
+
+
 def code_bytes(fmt, K):
     return K // 2 if fmt == FMT_NVFP4 else K
 

@@ -270,6 +270,23 @@ int orc_pick_split(const int32_t* counts, int E, int split_nb, int split_kb, int
     return best;
 }
 
+int orc_pick_gu_pairs(const int32_t* counts, int E, int nb, int kb, int num_sms, const int64_t* ps)
+{
+    int64_t m_tiles = 0, n_odd = 0;
+    for (int e = 0; e < E; e++) {
+        int64_t mt = (counts[e] + ORC_TILE_M - 1) / ORC_TILE_M;
+        m_tiles += mt;
+        n_odd += mt & 1;
+    }
+    if (nb <= 0 || m_tiles == 0) return 0;
+    int64_t single_units = m_tiles * nb;
+    int64_t pair_units = (m_tiles + n_odd) / 2 * nb;
+    int64_t clusters = num_sms / 2;
+    int64_t single_cost = (single_units + num_sms - 1) / num_sms * (kb * ps[0] + ps[1]);
+    int64_t pair_cost = (pair_units + clusters - 1) / clusters * (kb * ps[2] + ps[3]);
+    return pair_cost < single_cost ? 1 : 0;
+}
+
 /* ------------------------------------------------ activation quantisation */
 
 float orc_nvfp4_global(const float* x, int64_t n)

@@ -22,7 +22,7 @@ CASES = {
     "fp8-row-deep-k": W.custom(H=512, I=2304, E=8, k=2),
     # both GEMMs on CTA pairs (the down GEMM's pairs wait on each other's copies too)
     "fp8-row-deep-k-pairs": W.custom(H=512, I=2304, E=8, k=2),
-    # T k >= 512 E: the gate/up GEMM on CTA pairs (waits on the other CTA's copies)
+    # the gate/up GEMM on CTA pairs (waits on the other CTA's copies)
     "fp8-row-pairs": W.custom(H=512, I=256, E=8, k=2),
     "fp8-block128": W.custom(H=512, I=256, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128),
     "nvfp4": W.custom(H=512, I=256, E=8, k=2, fmt=W.FMT_NVFP4),
@@ -42,8 +42,13 @@ def test_wait_timeout_is_reported_and_the_context_stays_usable(name):
     T = 2100 if name.endswith("pairs") else 200
     d = synth.layer(wl, seed=5)
     layer = native.Layer(wl, d, max_T=T)
+    if name.endswith("pairs"):
+        # the cost model's parameters chosen so that the gate/up kernel runs as pairs
+        native.moe_set_pair_params(layer.h, 10 ** 12, 10 ** 12, 0, 0)
     x, wr = synth.tokens(wl, T, seed=5).cuda(), d["wr"].cuda()
     y_ref = layer.forward(x, wr, None).clone()
+    if name.endswith("pairs"):
+        assert int(layer.region("pick", torch.int32, 3)[2]) == 1
     torch.cuda.synchronize()
     assert layer.status()[0] == 0
 

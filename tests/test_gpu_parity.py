@@ -303,9 +303,15 @@ def test_dispatch_bit_exact(name):
     assert (tile_ptr == np.searchsorted(te, np.arange(E + 1), side="left")).all()
     a, b, bw, g, sms = native.moe_get_picker_params(layer.h)
     want, _ = oracle.pick_down_tile(counts, wl.H, wl.I, sms, a, b, bw, g)
-    pick = layer.region("pick", torch.int32, 2).cpu().numpy()
+    pick = layer.region("pick", torch.int32, 3).cpu().numpy()
     assert int(pick[0]) == want
     assert int(pick[1]) == expected_split(wl, T, counts, sms)
+    a_s, b_s, a_p, b_p, nb, kb, sms = native.moe_get_pair_params(layer.h)
+    if wl.fmt == W.FMT_FP8_ROW and wl.act == W.ACT_SWIGLU:
+        assert (nb, kb) == (2 * wl.I // 256, wl.H // 128)
+        assert int(pick[2]) == oracle.pick_gu_pairs(counts, nb, kb, sms, [a_s, b_s, a_p, b_p])
+    else:
+        assert nb == 0 and int(pick[2]) == 0
     rows = gpu_slot_rows(layer, wl, ids, T)
     if nvfp4(wl):
         xq = gpu_rows(layer, wl, "xq", wl.H // 2)[rows]
@@ -559,18 +565,35 @@ def test_cta_pairs_match_single_ctas(name):
     wl, T, d, x = build_case(name)
     layer = native.Layer(wl, d, max_T=T)
     xc, wr = x.cuda(), d["wr"].cuda()
-    native.moe_set_gemm_options(layer.h, 1)
-    y_pair = layer.forward(xc, wr, None).clone()
-    hq_pair = layer.region("hq", torch.uint8, (T * wl.k + 128 * wl.E) * wl.I).clone()
-    native.moe_set_gemm_options(layer.h, 0)
-    y_single = layer.forward(xc, wr, None).clone()
-    hq_single = layer.region("hq", torch.uint8, (T * wl.k + 128 * wl.E) * wl.I).clone()
-    torch.cuda.synchronize()
-    assert layer.status()[0] == 0
+    n_hq = (T * wl.k + 128 * wl.E) * wl.I
+
+    def run(mode, params=None):
+        native.moe_set_gemm_options(layer.h, mode)
+        if params is not None:
+            native.moe_set_pair_params(layer.h, *params)
+        y = layer.forward(xc, wr, None).clone()
+        torch.cuda.synchronize()
+        assert layer.status()[0] == 0
+        return y, layer.region("hq", torch.uint8, n_hq).clone(), int(layer.region("pick", torch.int32, 3)[2])
+
+    big = 10 ** 12
+    default = native.moe_get_pair_params(layer.h)[:4]
+    y_pair, hq_pair, _ = run(2)
+    y_single, hq_single, _ = run(0)
+    # the kernel that picks its mode on the device, forced each way by the cost
+    # parameters: the same results as the dedicated kernel of that mode
+    y_p1, hq_p1, pk1 = run(1, (big, big, 0, 0))
+    y_p0, hq_p0, pk0 = run(1, (0, 0, big, big))
+    assert (pk1, pk0) == (1, 0)
+    assert torch.equal(hq_p1, hq_pair) and torch.equal(y_p1, y_pair)
+    assert torch.equal(hq_p0, hq_single) and torch.equal(y_p0, y_single)
+    native.moe_set_pair_params(layer.h, *default)
     assert (hq_pair != hq_single).float().mean().item() <= 1e-3
     assert tolerance_violations(y_pair.float().cpu().numpy(), y_single.float().cpu().numpy()) == 0
     with pytest.raises(native.MoeError):
         native.moe_set_gemm_options(layer.h, 3)
+    with pytest.raises(native.MoeError):
+        native.moe_set_pair_params(layer.h, -1, 0, 0, 0)
 
 
 def test_empty_batch():

@@ -360,3 +360,26 @@ def test_mx32_exponent_is_the_smallest_that_fits():
     deq = torch_e4m3_value(codes) * np.repeat(scale, 32, axis=1)
     bound = np.maximum(np.abs(x) * 2.0 ** -4, np.repeat(scale, 32, axis=1) * 2.0 ** -10)
     assert (np.abs(deq - x) <= bound).all()
+
+
+def test_gate_up_pair_rule_hand_cases():
+    """The gate/up CTA-mode rule on histograms worked out by hand (148 SMs,
+    nb n-blocks, kb K-blocks, per-unit costs kb a + b)."""
+    ps = [1000, 0, 1000, 0]             # equal per-unit cost: only the wave counts decide
+    # 8 experts x 8 m-tiles (1024 rows each), nb = 112: single 64 x 112 = 7168
+    # units -> 49 waves; pairs 32 x 112 = 3584 units -> ceil(3584 / 74) = 49 waves
+    # -> equal cost, single CTAs
+    assert oracle.pick_gu_pairs([1024] * 8, 112, 32, 148, ps) == 0
+    # a pair unit cheaper than a single one (a_p < a_s) breaks the tie for pairs
+    assert oracle.pick_gu_pairs([1024] * 8, 112, 32, 148, [1000, 0, 990, 0]) == 1
+    # one m-tile per expert: pairs are half empty -> as many pair units as single
+    # ones on half the slots: 160 experts, nb = 4 -> single ceil(640/148) = 5,
+    # pairs ceil(640/74) = 9 waves
+    assert oracle.pick_gu_pairs([100] * 160 + [0] * 96, 4, 16, 148, ps) == 0
+    # odd counts: 3 m-tiles -> pairs (3 + 1) / 2 = 2 units per expert
+    assert oracle.pick_gu_pairs([300] * 50, 8, 16, 148, [10, 0, 6, 0]) == 1   # 150 x 8 = 1200 -> 9 waves x 160 vs
+    #                                                  100 x 8 = 800 -> 11 waves x 96 = 1056 < 1440
+    assert oracle.pick_gu_pairs([300] * 50, 8, 16, 148, [10, 0, 9, 0]) == 0   # 11 x 144 = 1584 > 1440
+    # no n-blocks (not a SwiGLU FP8_ROW layer) or no rows: single CTAs
+    assert oracle.pick_gu_pairs([1024] * 8, 0, 32, 148, [10, 0, 1, 0]) == 0
+    assert oracle.pick_gu_pairs([0] * 8, 112, 32, 148, [10, 0, 1, 0]) == 0

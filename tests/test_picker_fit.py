@@ -1,9 +1,14 @@
 """The down-tile cost model's fit against the committed B200 sweep: the table
 parses, the installed parameters give the picks and regrets the table states,
-and refitting the table gives back the installed parameters."""
+and refitting the table gives back the installed parameters.  The gate/up
+CTA-mode sweep tool restates the dispatch's pair rule; it is checked against
+the oracle's rule."""
 import os
 
+import numpy as np
 import pytest
+
+import oracle
 
 from mixture_experts_topk_b200 import picker_fit
 
@@ -46,3 +51,31 @@ def test_refit_reproduces_the_installed_parameters(rows):
     p = picker_fit.fit(rows)
     for got, want in zip(p, INSTALLED):
         assert got == pytest.approx(want, rel=0.02)
+
+
+def test_pair_sweep_rule_is_the_oracle_rule():
+    """The sweep tool's restatement of the gate/up CTA-mode rule (on m-tile
+    counts) picks what the oracle's rule picks on the histograms themselves."""
+    from mixture_experts_topk_b200 import pair_sweep
+    rng = np.random.default_rng(3)
+    for trial in range(300):
+        E = int(rng.choice([8, 32, 64, 256]))
+        counts = rng.integers(0, int(rng.choice([3, 200, 1500])), size=E).astype(np.int32)
+        nb, kb = int(rng.choice([1, 4, 16, 112])), int(rng.choice([2, 16, 32]))
+        ps = [int(v) for v in rng.integers(1, 10 ** 6, size=4)]
+        mt = (counts + 127) // 128
+        want = oracle.pick_gu_pairs(counts, nb, kb, 148, ps)
+        assert pair_sweep.pick(int(mt.sum()), int((mt % 2).sum()), nb, kb, ps) == want, (trial, E, nb, kb, ps)
+
+
+def test_pair_sweep_table_reader(tmp_path):
+    from mixture_experts_topk_b200 import pair_sweep
+    f = tmp_path / "t.md"
+    f.write_text(pair_sweep.HEADER + "\n| tiny T=16 | 8 | 8 | 1 | 2 | 0.0086 | 0.0120 |\n"
+                 "| mixtral-8x7b T=4096 | 67 | 3 | 112 | 32 | 0.9292 | 0.9248 |\n")
+    rows = pair_sweep.read_table(str(f))
+    assert [r["workload"] for r in rows] == ["tiny T=16", "mixtral-8x7b T=4096"]
+    res = pair_sweep.evaluate(rows, (527000, 0, 493000, 200000))
+    # one wave either way: single CTAs; Mixtral-8x7B T = 4096: pairs (53 vs 51 waves)
+    assert [p for _, p, _ in res] == [0, 1]
+    assert all(rg == 0.0 for _, _, rg in res)
