@@ -420,7 +420,7 @@ __device__ __forceinline__ void canonical_logit2(const RouterParams& p, int t, i
     const __nv_bfloat16* xrow = p.x + static_cast<size_t>(t) * p.H + 8 * lane;
     float a0 = 0.0f, a1 = 0.0f;
     const int nI = p.H >> 8;
-#pragma unroll 4
+#pragma unroll 2
     for (int i = 0; i < nI; i++) {
         const float4 pa = __ldg(reinterpret_cast<const float4*>(w0 + 256 * i));
         const float4 pb = __ldg(reinterpret_cast<const float4*>(w0 + 256 * i + 4));
@@ -459,10 +459,34 @@ __device__ __forceinline__ bool rank_before(float v, int id, float v2, int id2) 
     return v > v2 || (v == v2 && id < id2);
 }
 
+// More candidates than lanes (8-9 per token on the workloads, so rare): k
+// rounds of a warp argmax over them, as router_topk_select; lane l reads back
+// the canonical logits it wrote (experts l + 32 m).  Out of line, so that its
+// registers do not weigh on the common path.
+__device__ __noinline__ void select_among_many(const float* lrow, uint32_t cand, int t, int E, int k, int score,
+                                               int32_t* ids, float* w, int lane) {
+    RouterParams q;
+    q.x = nullptr;
+    q.wr = nullptr;
+    q.bias = nullptr;
+    q.logits = nullptr;
+    q.ids = ids;
+    q.w = w;
+    q.T = 0;
+    q.H = 0;
+    q.E = E;
+    q.k = k;
+    q.score = score;
+    float cv[8];
+#pragma unroll
+    for (int m = 0; m < 8; m++) cv[m] = ((cand >> m) & 1u) ? lrow[32 * m + lane] : 0.0f;
+    router_topk_candidates(q, cv, cand, t, lane);
+}
+
 // One warp per token: bounds, the k-th largest lower bound, candidates, their
 // canonical logits (written over the approximations), then the top k of the
 // candidates and the weights, computed as router_topk_select computes them.
-__global__ void __launch_bounds__(256, 3) router_select_kernel(RouterParams p, RouterFix f) {
+__global__ void __launch_bounds__(256, 4) router_select_kernel(RouterParams p, RouterFix f) {
     __shared__ int s_list[8][256];
     pdl_wait();
     pdl_trigger();
@@ -477,26 +501,25 @@ __global__ void __launch_bounds__(256, 3) router_select_kernel(RouterParams p, R
         const double sx = f.x_sum[t];
         const float mx = f.x_max[t];
         // bounds of the canonical logits, rounded outward to fp32 (only looser)
-        float lb[8], ub[8];
+        float srt[8], ub[8];   // srt: the lower bounds, sorted below
 #pragma unroll
         for (int m = 0; m < 8; m++) {
             const int e = 32 * m + lane;
-            lb[m] = -INFINITY;
+            srt[m] = -INFINITY;
             ub[m] = -INFINITY;
             if (m < nm && e < p.E) {
                 const float l = lrow[e];
                 const double d = router_bound(eps_x, sx, mx, pow2d(f.w_exp[e] - 15), f.w_sum[e], f.w_sumq[e],
                                               f.w_max[e], p.bias ? fabsf(p.bias[e]) : 0.0f, l, gamma);
-                lb[m] = __double2float_rd(static_cast<double>(l) - d);
+                srt[m] = __double2float_rd(static_cast<double>(l) - d);
                 ub[m] = __double2float_ru(static_cast<double>(l) + d);
             }
+            // four experts' loads at a time in flight (fewer live registers)
+            if (m == 3) asm volatile("" ::: "memory");
         }
         // LB_k, the k-th largest lower bound: each lane sorts its eight lower
         // bounds (descending), then k rounds take the warp maximum of the
         // lanes' current heads and advance the winning lane's head
-        float srt[8];
-#pragma unroll
-        for (int m = 0; m < 8; m++) srt[m] = lb[m];
 #pragma unroll
         for (int i = 0; i < 8; i++)
 #pragma unroll
@@ -536,11 +559,9 @@ __global__ void __launch_bounds__(256, 3) router_select_kernel(RouterParams p, R
             ncand += __popc(bal);
         }
         __syncwarp();
-        // their canonical logits, two at a time; lane e % 32 keeps expert e's,
-        // and lane i < 32 also holds candidate i's (for the sort below)
-        float cv[8];
-#pragma unroll
-        for (int m = 0; m < 8; m++) cv[m] = 0.0f;
+        // their canonical logits, two at a time, written over the
+        // approximations in the logits row; lane i < 32 also holds candidate
+        // i's (for the sort below)
         float my_v = -INFINITY;
         int my_e = 0x7FFFFFFF;
         for (int i = 0; i < ncand; i += 2) {
@@ -553,12 +574,7 @@ __global__ void __launch_bounds__(256, 3) router_select_kernel(RouterParams p, R
                 if (h == 1 && !two) break;
                 const int e = h ? e1 : e0;
                 const float c = h ? c1 : c0;
-                if ((e & 31) == lane) {
-#pragma unroll
-                    for (int m = 0; m < 8; m++)
-                        if (m == (e >> 5)) cv[m] = c;
-                    lrow[e] = c;
-                }
+                if ((e & 31) == lane) lrow[e] = c;
                 if (lane == i + h) {
                     my_v = c;
                     my_e = e;
@@ -567,7 +583,7 @@ __global__ void __launch_bounds__(256, 3) router_select_kernel(RouterParams p, R
         }
         __syncwarp();   // the list is rewritten for the warp's next token
         if (ncand > 32) {
-            router_topk_candidates(p, cv, cand, t, lane);
+            select_among_many(lrow, cand, t, p.E, p.k, p.score, p.ids, p.w, lane);
             continue;
         }
         // at most 32 candidates: a bitonic sort over the lanes in selection order
