@@ -429,6 +429,8 @@ def run_ours(args, rank, world, local_rank):
         native.moe_set_tile_config(layer.h, args.down_bn)
     if args.cta_pairs is not None:
         native.moe_set_gemm_options(layer.h, args.cta_pairs)
+    if args.gate_up_bn:
+        native.moe_set_gate_up_tile(layer.h, args.gate_up_bn)
     wr = d["wr"]
     bias = d["bias"]
     del d                      # the packed copy is all the layer reads
@@ -568,6 +570,8 @@ def main():
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the sweep over every (workload, T) point (done at N = 1 only)")
     ap.add_argument("--down-bn", type=int, default=0, help="down GEMM tile width (0 = chosen per call)")
+    ap.add_argument("--gate-up-bn", type=int, default=0, choices=[0, 128, 256],
+                    help="gated FP8_ROW gate/up tile width (0 = by batch size)")
     ap.add_argument("--cta-pairs", type=int, default=None, choices=[0, 1, 2],
                     help="FP8_ROW GEMMs on CTA pairs: 0 never, 1 by the library's rule (default), 2 always")
     ap.add_argument("--act", default="swiglu", choices=sorted(ACTS),

@@ -146,7 +146,8 @@ typedef struct {
     int32_t* tile_ptr;   /* [E+1] index of each expert's first row tile */
     int32_t* pick;       /* [3] choices from the histogram: [0] down GEMM tile (0 -> 256, 1 -> 128, 2 -> 64
                           * columns, FP8_BLOCK128); [1] S, the K split of the FP8_ROW down GEMM (1 = none);
-                          * [2] the FP8_ROW SwiGLU gate/up GEMM on CTA pairs (1) or single CTAs (0) */
+                          * [2] the gated FP8_ROW gate/up GEMM's mode: 0 single CTAs, 256-wide
+                          * tiles; 1 CTA pairs; 2 single CTAs, 128-wide tiles */
     int32_t* tiles;      /* [A/128 + E + 1][2] (expert, first row) per row tile */
     int32_t* perm;       /* [A] slot -> t*k + j */
     int32_t* inv;        /* [A] t*k + j -> slot */
@@ -257,9 +258,9 @@ moe_status moe_set_tile_config(moe_handle* h, int down_bn);
  * plain stream order.  Host state only; MOE_ERR_INVALID_ARG for other values. */
 moe_status moe_set_launch_options(moe_handle* h, int pdl);
 
-/* GEMM options.  cta_pairs = 1 (the default): an FP8_ROW SwiGLU layer runs
- * the gate/up GEMM on CTA pairs where the dispatch's cost model picks them
- * from the expert histogram (moe_set_pair_params): 2-CTA clusters whose
+/* GEMM options.  cta_pairs = 1 (the default): a gated FP8_ROW layer runs the
+ * gate/up GEMM on CTA pairs where the dispatch's cost model picks them from
+ * the expert histogram (moe_set_gate_up_model): 2-CTA clusters whose
  * tcgen05.mma.cta_group::2 covers two row tiles of one expert (M = 256), each
  * CTA loading its own 128 rows of X and half of the 256 weight rows (no
  * multicast), so a 32 KB stage feeds what a 48 KB stage feeds alone.  With
@@ -273,8 +274,19 @@ moe_status moe_set_launch_options(moe_handle* h, int pdl);
  * inside the tensor core.  cta_pairs = 0 keeps single CTAs; cta_pairs = 2
  * runs these GEMMs on CTA pairs at every batch size (the down GEMM still only
  * where K > 2048 and no K split is chosen).  Errors: MOE_ERR_INVALID_ARG for a
- * null handle or another value. */
+ * null handle, another value, or 2 while moe_set_gate_up_tile forces 128. */
 moe_status moe_set_gemm_options(moe_handle* h, int cta_pairs);
+
+/* Gate/up tile width of a gated FP8_ROW layer.  bn = 0 (the default): picked
+ * on the device with the mode (moe_set_gate_up_model); 128 forces 128-wide
+ * tiles (64 gate + 64 up accumulator columns, 64 hidden columns, 8 of the 16
+ * epilogue warps working), 256 forbids them.  Narrow tiles double the units
+ * and halve each unit's weight bytes, so a small batch's weight stream can end
+ * in a shorter last wave.  Per element the same products and roundings as the
+ * 256-wide tile.  Host state only.  MOE_ERR_INVALID_ARG for another value or
+ * for 128 while CTA pairs are forced on; MOE_ERR_UNSUPPORTED_SHAPE for 128 on
+ * an NVFP4, FP8_BLOCK128 or ReLU^2 layer. */
+moe_status moe_set_gate_up_tile(moe_handle* h, int bn);
 
 /* Limit, in SM clock cycles, of every wait of the GEMM kernels on another
  * role or CTA (stage, accumulator and exchange barriers); default 2e9 (about
@@ -305,21 +317,27 @@ moe_status moe_set_wait_limit(moe_handle* h, long long cycles);
 moe_status moe_set_picker_params(moe_handle* h, const long long* params);
 moe_status moe_get_picker_params(const moe_handle* h, long long* params);
 
-/* Parameters of the model that picks, from the runtime expert histogram, whether
- * the FP8_ROW SwiGLU gate/up GEMM runs on single CTAs or on CTA pairs (RaMP
- * abstract: a cost model of CTA waves, fitted once to a profiling sweep).  The
- * dispatch evaluates, with mt_e = ceil(count_e / 128), m_tiles = sum_e mt_e,
- * n_odd = #{e : mt_e odd}, nb = 2I / 256 n-blocks and kb = H / 128 K-blocks:
- *   single = ceil(m_tiles nb / num_sms) (kb a_s + b_s)
- *   pair   = ceil((m_tiles + n_odd) / 2 nb / (num_sms / 2)) (kb a_p + b_p)
- * (integers, picoseconds) and writes view.pick[2] = 1 (pairs) when pair <
- * single, else 0; the gate/up kernel, launched as 2-CTA clusters, reads it.
- * params = {a_s, b_s, a_p, b_p}; get also returns nb, kb and num_sms in
- * params[4..6] (nb = 0: the layer has no choice, single CTAs).  Host state only;
- * MOE_ERR_INVALID_ARG for a negative cost.  moe_set_gemm_options overrides
- * the pick. */
-moe_status moe_set_pair_params(moe_handle* h, const long long* params);
-moe_status moe_get_pair_params(const moe_handle* h, long long* params);
+/* Parameters of the model that picks, from the runtime expert histogram, the
+ * mode of a gated FP8_ROW layer's gate/up GEMM (RaMP abstract: a cost model
+ * of CTA waves over the histogram, fitted once to a profiling sweep):
+ *   0  single CTAs on 256-wide tiles (128 gate + 128 up accumulator columns),
+ *   1  CTA pairs: tcgen05.mma.cta_group::2 with M = 256 over two row tiles of
+ *      one expert, each CTA loading half of the 256 weight rows,
+ *   2  single CTAs on 128-wide tiles (64 gate + 64 up columns).
+ * The dispatch evaluates, with mt_e = ceil(count_e / 128), m_tiles = sum_e mt_e,
+ * n_odd = #{e : mt_e odd}, nb = 2I / 256 and kb = H / 128 (integers, ps):
+ *   c0 = ceil(m_tiles nb / num_sms) (kb a_0 + b_0)
+ *   c1 = ceil((m_tiles + n_odd) / 2 nb / (num_sms / 2)) (kb a_1 + b_1)
+ *   c2 = ceil(2 m_tiles nb / num_sms) (kb a_2 + b_2)
+ * and writes view.pick[2] = the cheapest allowed mode (ties to the lower);
+ * the gate/up kernel, launched as 2-CTA clusters, reads it.  The allowed modes
+ * follow moe_set_gemm_options and moe_set_gate_up_tile.
+ * params = {a_0, b_0, a_1, b_1, a_2, b_2}; get also returns nb, kb, num_sms
+ * and the allowed-mode mask (bit m: mode m) in params[6..9] (nb = 0: the
+ * layer has no choice, mode 0).  Host state only; MOE_ERR_INVALID_ARG for a
+ * negative cost. */
+moe_status moe_set_gate_up_model(moe_handle* h, const long long* params);
+moe_status moe_get_gate_up_model(const moe_handle* h, long long* params);
 
 /* Deterministic combine (LightMoE README, "Highlights": deterministic
  * combine): y[t] = bf16( sum_{j=0..k-1} o[inv[t k + j]] ) in fixed j order,

@@ -38,29 +38,41 @@ struct PickerParams {
     int split_nb;              // n-blocks of a K-splittable down GEMM (0: no split)
     int split_kb;              // its K-blocks
     int o_rows;                // rows of the fp32 down-output buffer
-    // gate/up GEMM on single CTAs or on CTA pairs (pick_gu_pairs)
-    int gu_nb;                 // its n-blocks (0: no choice, single CTAs)
+    // gate/up GEMM mode (pick_gu_mode)
+    int gu_nb;                 // n-blocks of its 256-wide tiles (0: no choice, mode 0)
     int gu_kb;                 // its K-blocks
-    long long gu_ps[4];        // per-unit cost kb * a + b: single (a, b), pair (a, b), picoseconds
+    int gu_allow;              // allowed modes: bit 0 wide single, bit 1 pairs, bit 2 narrow
+    long long gu_ps[6];        // per-unit cost kb * a + b of each mode, (a, b) in that order, picoseconds
 };
 
-// Gate/up GEMM on single CTAs or on 2-CTA pairs (M = 256 over two m-tiles of
-// one expert), chosen from the expert histogram.  A single unit is an
-// (m-tile, n-block), num_sms run at once; a pair unit is an (m-pair, n-block)
-// whose m-tiles are an expert's 2j and 2j + 1 (the second absent for the last
-// of an odd count), num_sms / 2 run at once.  With m_tiles = sum_e mt_e and
-// n_odd = #{e : mt_e odd}:
-//   single = ceil(m_tiles nb / num_sms) (kb a_s + b_s)
-//   pair   = ceil((m_tiles + n_odd) / 2 nb / (num_sms / 2)) (kb a_p + b_p)
-// Pairs when strictly cheaper (1), else single CTAs (0).
-__host__ __device__ inline int pick_gu_pairs(const PickerParams& q, int m_tiles, int n_odd) {
+// Mode of the gated FP8_ROW gate/up GEMM, chosen from the expert histogram:
+// 0 single CTAs on 256-wide tiles (128 gate + 128 up columns), 1 CTA pairs
+// (M = 256 over two m-tiles of one expert, the second absent for the last of
+// an odd count; num_sms / 2 pairs run at once), 2 single CTAs on 128-wide
+// tiles (twice the units, half the weight rows each).  With
+// m_tiles = sum_e mt_e and n_odd = #{e : mt_e odd}:
+//   c0 = ceil(m_tiles nb / num_sms) (kb a_0 + b_0)
+//   c1 = ceil((m_tiles + n_odd) / 2 nb / (num_sms / 2)) (kb a_1 + b_1)
+//   c2 = ceil(m_tiles 2 nb / num_sms) (kb a_2 + b_2)
+// The cheapest allowed mode wins; ties go to the lower mode.
+__host__ __device__ inline int pick_gu_mode(const PickerParams& q, int m_tiles, int n_odd) {
     if (q.gu_nb <= 0 || m_tiles <= 0) return 0;
-    const long long su = static_cast<long long>(m_tiles) * q.gu_nb;
-    const long long pu = static_cast<long long>((m_tiles + n_odd) / 2) * q.gu_nb;
     const long long ns = q.num_sms, np = q.num_sms / 2;
-    const long long c_s = (su + ns - 1) / ns * (q.gu_kb * q.gu_ps[0] + q.gu_ps[1]);
-    const long long c_p = (pu + np - 1) / np * (q.gu_kb * q.gu_ps[2] + q.gu_ps[3]);
-    return c_p < c_s ? 1 : 0;
+    const long long u[3] = {static_cast<long long>(m_tiles) * q.gu_nb,
+                            static_cast<long long>((m_tiles + n_odd) / 2) * q.gu_nb,
+                            static_cast<long long>(m_tiles) * 2 * q.gu_nb};
+    const long long slots[3] = {ns, np, ns};
+    int best = -1;
+    long long best_c = 0;
+    for (int m = 0; m < 3; m++) {
+        if (!((q.gu_allow >> m) & 1)) continue;
+        const long long c = (u[m] + slots[m] - 1) / slots[m] * (q.gu_kb * q.gu_ps[2 * m] + q.gu_ps[2 * m + 1]);
+        if (best < 0 || c < best_c) {
+            best = m;
+            best_c = c;
+        }
+    }
+    return best < 0 ? 0 : best;
 }
 
 // Split of the down GEMM's K for small batches: when the (m-tile, n-block)
@@ -186,7 +198,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
         if (pick_out) {
             pick_out[0] = pick_down_tile(pq, trun, touched);
             pick_out[1] = pick_split(pq, trun, A);
-            pick_out[2] = pick_gu_pairs(pq, trun, n_odd);
+            pick_out[2] = pick_gu_mode(pq, trun, n_odd);
         }
     }
     if (e < E) {
@@ -305,7 +317,7 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK) dispatch_small_kernel(
             tile_ptr[E] = total >> 20;
             pick_out[0] = pick_down_tile(pq, total >> 20, touched);
             pick_out[1] = pick_split(pq, total >> 20, total & 0xFFFFF);
-            pick_out[2] = pick_gu_pairs(pq, total >> 20, n_odd);
+            pick_out[2] = pick_gu_mode(pq, total >> 20, n_odd);
         }
         if (tid < E) {
             counts[tid] = c;
@@ -557,7 +569,7 @@ __global__ void __launch_bounds__(256) dispatch_quant_small_kernel(
             tile_ptr[E] = total >> 20;
             pick_out[0] = pick_down_tile(pq, total >> 20, touched);
             pick_out[1] = pick_split(pq, total >> 20, total & 0xFFFFF);
-            pick_out[2] = pick_gu_pairs(pq, total >> 20, n_odd);
+            pick_out[2] = pick_gu_mode(pq, total >> 20, n_odd);
         }
         if (tid < E) {
             counts[tid] = c;

@@ -336,13 +336,26 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
 template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI = 8, int ACT = 0, bool PAIR = false>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                                           const int n_blocks, uint8_t* smem_raw) {
-    static_assert(EPI == 8 || (EPI == 16 && KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW && !PROMOTE && BN == 256),
+    static_assert(EPI == 8 || (EPI == 16 && KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW && !PROMOTE),
                   "16 epilogue warps are built for the FP8_ROW gate/up GEMM only");
     static_assert(!PAIR || (KIND == KIND_GATE_UP && BSCALE == BSCALE_ROW && !PROMOTE && BN == 256),
                   "CTA pairs are built for the FP8_ROW gate/up GEMM only");
+    static_assert(KIND != KIND_GATE_UP || BN == 256 || (BN == 128 && BSCALE == BSCALE_ROW && !PROMOTE && ACT != 5 &&
+                                                        !PAIR),
+                  "128-wide gate/up tiles are built for gated FP8_ROW activations on single CTAs");
     using S = GemmSmem<BN, STAGES, EPI, PAIR>;
-    constexpr int CG = EPI / 4;          // column groups
-    constexpr int GC = 128 / CG;         // gate/up: hidden columns per thread (64 or 32)
+    // column groups with work: a 128-wide gate/up tile launched with 16
+    // epilogue warps gives its 64 hidden columns to two groups (32 each, so a
+    // 32-column MX block stays in one thread); the other 8 warps idle
+    constexpr int CG = (KIND == KIND_GATE_UP && BN == 128 && EPI == 16) ? 2 : EPI / 4;
+    constexpr int EPA = 4 * CG;          // epilogue warps with work
+    // gate/up: a tile's gate half and up half (128 + 128 accumulator columns, or
+    // 64 + 64 in a 128-wide tile), and the hidden columns of each per thread
+    constexpr int GU_HALF = KIND == KIND_GATE_UP ? BN / 2 : 128;
+    constexpr int GC = GU_HALF / CG;     // 64 or 32
+    // first packed weight row of gate/up n-block nb: packed rows come in groups
+    // of 128 gate + 128 up rows; a 128-wide tile takes 64 of each, at 64 (nb & 1)
+    auto gu_row0 = [&](int nb) { return BN == 256 ? nb * 256 : 256 * (nb >> 1) + 64 * (nb & 1); };
     constexpr int NH = GC / 32;          // 32-column blocks per thread
     constexpr int SR = sparse_round<EPI>();
     constexpr int EWF = epi_warp_floats<EPI>();
@@ -371,7 +384,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
         }
         for (int b = 0; b < NBUF; b++) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], PAIR ? 2 * EPI : EPI);   // one arrival per epilogue warp
+            mbar_init(&tempty[b], PAIR ? 2 * EPA : EPA);   // one arrival per working epilogue warp
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -441,7 +454,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                 // a pair's rank 1 without an m-tile (odd count) loads rank 0's rows,
                 // so its A stays inside the tensor; its accumulator rows are not stored
                 const int row0 = s_off[e] + GEMM_BM * (mi - (has_rows ? 0 : 1) - s_tptr[e]);
-                const int brow = e * p.b_rows + nb * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
+                const int brow = e * p.b_rows + (KIND == KIND_GATE_UP ? gu_row0(nb) : nb * BN) +
+                                 (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
                 const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
                 for (int kb = 0; kb < p.num_kb; kb++, it++) {
                     const int s = it % STAGES;
@@ -460,7 +474,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     } else {
                         mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
                         tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
-                        tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                        if (KIND == KIND_GATE_UP && BN == 128) {
+                            // 64 gate rows, then the 64 matching up rows 128 further
+                            // (the tensor map's box is 64 rows)
+                            tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                            tma_load_2d_hint(sa + GEMM_A_BYTES + 64 * GEMM_BK, &tmB, &full[s], kb * GEMM_BK,
+                                             brow + 128, pol);
+                        } else {
+                            tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                        }
                     }
                     if (PROMOTE) KTRACE_BLK(it, 7);
                 }
@@ -532,7 +554,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
             else mma_commit(drain);
             mbar_wait(drain, 0, DRAIN_LIMIT);        // ... before TMEM can be released
         }
-    } else {
+    } else if (warp - 2 < EPA) {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;
         const int q = warp & 3;               // TMEM lane quadrant this warp may access
@@ -575,7 +597,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     // and lane c holds the weight scale of column c of each 32-column
                     // half (read back with a shuffle)
                     const float sa = valid ? p.a_scale[static_cast<size_t>(row) * p.a_ld] : 0.0f;
-                    const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + nb * BN;
+                    const float* bs = p.b_scale + static_cast<size_t>(e) * p.b_rows + gu_row0(nb);
                     float bsg[NH], bsu[NH];
 #pragma unroll
                     for (int half = 0; half < NH; half++) {
@@ -607,7 +629,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         for (int half = 0; half < NH; half++) {
                             float gv[32], uv[32];
                             const int c0 = GC * g + 32 * half;
-                            tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, gv, uv);
+                            tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + GU_HALF + c0, gv, uv);
                             if (half == NH - 1) {
                                 tc_fence_before();
                                 __syncwarp();
@@ -615,7 +637,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                             }
                             // first hidden column of this 32-block (ReLU^2: the gate-half
                             // columns are up rows 256 nb + c0, the up half 256 nb + 128 + c0)
-                            const int hcol = ACT == 5 ? nb * 256 + c0 : nb * 128 + c0;
+                            const int hcol = ACT == 5 ? nb * 256 + c0 : nb * GU_HALF + c0;
                             uint32_t m = vmask;
                             for (int r0 = 0; r0 < nv; r0 += SR) {
                                 if (valid && cidx >= r0 && cidx < r0 + SR) {
@@ -662,7 +684,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     for (int half = 0; half < NH; half++) {
                         float gv[32], uv[32];
                         const int c0 = GC * g + 32 * half;
-                        tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, gv, uv);
+                        tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + GU_HALF + c0, gv, uv);
 #pragma unroll
                         for (int c = 0; c < 32; c++) {
                             const float gg = gv[c] * (sa * __shfl_sync(0xffffffffu, bsg[half], c));
@@ -704,7 +726,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                             if (!any_valid) break;   // no stored row: skip the readback
                             float vg[32], vu[32];
                             const int c0 = 64 * g + 32 * half;
-                            tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + 128 + c0, vg, vu);
+                            tmem_ld32x2(lane_addr + acc * BN + c0, lane_addr + acc * BN + GU_HALF + c0, vg, vu);
 #pragma unroll
                             for (int c = 0; c < 32; c++) {
                                 ag[32 * half + c] = fmaf(vg[c], sg, ag[32 * half + c]);
@@ -738,14 +760,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     if (valid) {
                         const long long prow = static_cast<long long>(mi) * 128 + r;
                         // 32-column blocks of this thread: gated NH blocks at hidden
-                        // 128 nb + GC g + 32 b; ReLU^2 2 NH blocks, the gate-half
+                        // GU_HALF nb + GC g + 32 b; ReLU^2 2 NH blocks, the gate-half
                         // columns at 256 nb + GC g + 32 b, the up half 128 further
                         constexpr int NB = ACT == 5 ? 2 * NH : NH;
                         static_assert(BSCALE != BSCALE_ROW || 32 * NB <= 64, "hidden values held per thread");
 #pragma unroll
                         for (int b = 0; b < NB; b++) {
                             const int col = ACT == 5 ? nb * 256 + (b < NH ? GC * g + 32 * b : 128 + GC * g + 32 * (b - NH))
-                                                     : nb * 128 + GC * g + 32 * b;
+                                                     : nb * GU_HALF + GC * g + 32 * b;
                             float amax = 0.0f;
 #pragma unroll
                             for (int c = 0; c < 32; c++) amax = fmaxf(amax, fabsf(hv[32 * b + c]));
@@ -890,36 +912,42 @@ __global__ void __launch_bounds__(gemm_threads<EPI>(), 1)
     gemm_body<KIND, BSCALE, PROMOTE, BN, STAGES, EPI, ACT>(tmA, tmB, p, p.n_blocks, smem_raw);
 }
 
-// FP8_ROW gate/up on CTA pairs (launched as 2-CTA clusters)
+// The gated FP8_ROW gate/up GEMM, whose mode the dispatch picks from the
+// expert histogram (pick_gu_mode): launched as 2-CTA clusters of 16-epilogue-
+// warp CTAs; every CTA reads the mode and runs
+//   0: the single-CTA body on 256-wide tiles (128 gate + 128 up columns),
+//   1: the pair body (M = 256 over two m-tiles of one expert, each CTA loading
+//      half of the 256 weight rows),
+//   2: the single-CTA body on 128-wide tiles (64 gate + 64 up columns, twice
+//      the n-blocks; 8 of the 16 epilogue warps work).
+// No host round trip.  p.n_blocks counts the 256-wide n-blocks.
 constexpr int GU_PAIR_STAGES = 6;
-template <int ACT>
-__global__ void __launch_bounds__(gemm_threads<16>(), 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const GemmParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 256, GU_PAIR_STAGES, 16, ACT, true>(tmA, tmB, p, p.n_blocks,
-                                                                                   smem_raw);
+constexpr int GU_WIDE_STAGES = 4;
+constexpr int GU_NARROW_STAGES = 6;
+constexpr int gu_poly_smem() {
+    constexpr int a = GemmSmem<256, GU_WIDE_STAGES, 16>::TOTAL;
+    constexpr int b = GemmSmem<256, GU_PAIR_STAGES, 16, true>::TOTAL;
+    constexpr int c = GemmSmem<128, GU_NARROW_STAGES, 16>::TOTAL;
+    return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
-
-// FP8_ROW gate/up GEMM whose CTA mode is chosen on the device: launched as
-// 2-CTA clusters; the dispatch's scan writes pick_gu_pairs to *cfg, and both
-// CTAs of every cluster read it and run either the pair body (M = 256 over two
-// m-tiles of an expert) or, each on its own, the single-CTA body.  No host
-// round trip.
-constexpr int GU_POLY_SMEM = GemmSmem<256, 4, 16>::TOTAL > GemmSmem<256, GU_PAIR_STAGES, 16, true>::TOTAL
-                                 ? GemmSmem<256, 4, 16>::TOTAL
-                                 : GemmSmem<256, GU_PAIR_STAGES, 16, true>::TOTAL;
+constexpr int GU_POLY_SMEM = gu_poly_smem();
 template <int ACT>
 __global__ void __launch_bounds__(gemm_threads<16>(), 1)
     grouped_gemm_gu_poly_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB256,
-                                const __grid_constant__ CUtensorMap tmB128, const GemmParams p, const int32_t* cfg) {
+                                const __grid_constant__ CUtensorMap tmB128, const __grid_constant__ CUtensorMap tmB64,
+                                const GemmParams p, const int32_t* cfg) {
     extern __shared__ uint8_t smem_raw[];
-    pdl_wait();   // the mode was picked by the dispatch scan
-    if (*cfg == 1)
+    pdl_wait();   // the mode was picked by the dispatch
+    const int mode = *cfg;
+    if (mode == 1)
         gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 256, GU_PAIR_STAGES, 16, ACT, true>(tmA, tmB128, p, p.n_blocks,
                                                                                        smem_raw);
+    else if (mode == 2)
+        gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 128, GU_NARROW_STAGES, 16, ACT>(tmA, tmB64, p, 2 * p.n_blocks,
+                                                                                   smem_raw);
     else
-        gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, ACT>(tmA, tmB256, p, p.n_blocks, smem_raw);
+        gemm_body<KIND_GATE_UP, BSCALE_ROW, false, 256, GU_WIDE_STAGES, 16, ACT>(tmA, tmB256, p, p.n_blocks,
+                                                                                 smem_raw);
 }
 
 // Down GEMM whose tile width is chosen on the device: the dispatch's scan

@@ -119,6 +119,7 @@ struct moe_handle {
     long long spin_limit;
     int down_bn;          // 0 = picked per call, else 64 / 128 / 256
     int gemm_pairs;       // large FP8_ROW batches run the gate/up GEMM on CTA pairs
+    int gu_bn;            // gated FP8_ROW gate/up tile width: 0 = picked on the device, else 128 / 256
     PickerParams picker;
     int pdl;              // launch with programmatic dependent launch allowed
 };
@@ -255,15 +256,27 @@ static WLayout make_w_layout(const moe_config& c) {
 }
 
 // ------------------------------------------------------------------ init
-// per-unit cost kb * a + b (ps) of a gate/up unit on a single CTA (a_s, b_s)
-// and on a CTA pair (a_p, b_p).  a_s is the per-K-block cost of a 128 x 256
-// unit from a least-squares fit of an interleaved B200 sweep of both modes
-// (the FP8_ROW SwiGLU workloads at every batch size, two more shapes);
-// a_p = a_s / 1.069 puts the boundary between the wave ratios at which pairs
-// measured faster (1.04) and slower (>= 1.07); b_p = 0.2 us, a pair unit's
-// fixed cost (cross-CTA arrivals), keeps batches that fill one wave either
-// way on single CTAs (a 16-token layer ran 39% slower on half-empty pairs).
-static const long long GU_PAIR_FIT[4] = {527000, 0, 493000, 200000};
+// Gate/up mode model: per-unit cost kb * a + b (ps) on 256-wide single CTAs,
+// CTA pairs and 128-wide single CTAs.  a_0 is the per-K-block cost of a
+// 128 x 256 unit from a least-squares fit of an interleaved B200 sweep of the
+// modes; the others are set against it so that the rule reproduces the
+// fastest measured mode of each point of that sweep (gated FP8_ROW workloads
+// at every batch size and two more shapes): a_1 = a_0 / 1.069 and b_1 = 0.2 us
+// (a pair unit's fixed cost: one-wave batches stay on single CTAs); a_2 =
+// 0.634 a_0, the middle of the range (0.60-0.66 a_0) that separates the
+// points where 128-wide tiles measured faster from those where they did not.
+static const long long GU_MODE_FIT[6] = {527000, 0, 493000, 200000, 334000, 0};
+
+// allowed gate/up modes (bit 0 wide single, 1 pairs, 2 narrow) under the
+// host's options, 0 when they contradict each other
+static int gu_allow_of(int gemm_pairs, int gu_bn) {
+    int allow = 7;
+    if (gemm_pairs == 0) allow &= ~2;
+    if (gemm_pairs == 2) allow &= 2;
+    if (gu_bn == 128) allow &= 4;
+    if (gu_bn == 256) allow &= ~4;
+    return allow;
+}
 
 extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
     if (!cfg || !out) return fail(MOE_ERR_INVALID_ARG, "moe_init: null argument");
@@ -308,15 +321,17 @@ extern "C" moe_status moe_init(const moe_config* cfg, moe_handle** out) {
     h->picker.num_sms = h->num_sms;
     h->pdl = 1;
     h->gemm_pairs = 1;
+    h->gu_bn = 0;
     h->picker.H = c.H;
     h->picker.I = c.I;
     h->picker.split_nb = c.fmt == MOE_FMT_FP8_ROW ? c.H / MX_BN : 0;
     h->picker.split_kb = c.I / 128;
     h->picker.o_rows = static_cast<int>(o_rows(c));
     // gate/up CTA mode (FP8_ROW SwiGLU), per-unit costs fitted to a B200 sweep
-    h->picker.gu_nb = (c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU) ? 2 * c.I / 256 : 0;
+    h->picker.gu_nb = (c.fmt == MOE_FMT_FP8_ROW && c.act != MOE_ACT_RELU2) ? 2 * c.I / 256 : 0;
     h->picker.gu_kb = c.H / 128;
-    for (int i = 0; i < 4; i++) h->picker.gu_ps[i] = GU_PAIR_FIT[i];
+    h->picker.gu_allow = gu_allow_of(h->gemm_pairs, h->gu_bn);
+    for (int i = 0; i < 6; i++) h->picker.gu_ps[i] = GU_MODE_FIT[i];
     *out = h;
     return MOE_OK;
 }
@@ -757,18 +772,16 @@ static moe_status launch_gemm(bool pdl, const CUtensorMap& ta, const CUtensorMap
     return MOE_OK;
 }
 
-// FP8_ROW gate/up on CTA pairs: M = 256 MMAs over two m-tiles of one expert,
-// each CTA loading its 128 A rows and half of the B tile (32 KB stages, 6 deep)
+// The gated FP8_ROW gate/up GEMM as 2-CTA clusters running the picked mode
 template <int ACT>
-static moe_status launch_gemm_pairs(bool pdl, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                                    int grid, cudaStream_t st) {
-    using S = GemmSmem<256, GU_PAIR_STAGES, 16, true>;
-    static_assert(S::TOTAL <= 232448, "shared memory of the GEMM exceeds 227 KB");
-    auto kern = grouped_gemm_pair_kernel<ACT>;
-    CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL));
-    const cudaError_t err = launch_k_pairs(pdl, kern, dim3(grid), dim3(gemm_threads<16>()), S::TOTAL, st, ta, tb, p);
-    if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "launch of grouped_gemm_pair_kernel failed: %s", cudaGetErrorString(err));
-    return MOE_OK;
+static cudaError_t launch_gu_poly(bool pdl, int grid, cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb256,
+                                  const CUtensorMap& tb128, const CUtensorMap& tb64, const GemmParams& p,
+                                  const int32_t* mode) {
+    auto kern = grouped_gemm_gu_poly_kernel<ACT>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GU_POLY_SMEM);
+    if (e != cudaSuccess) return e;
+    return launch_k_pairs(pdl, kern, dim3(grid), dim3(gemm_threads<16>()), GU_POLY_SMEM, st, ta, tb256, tb128, tb64, p,
+                          mode);
 }
 
 // upper bound of the m-tiles the schedule can hold for T tokens
@@ -804,11 +817,7 @@ static moe_status gate_up_impl(const moe_handle* h, const void* packed, int T, v
     moe_status r = make_tmap(&ta, v.xq, c.H, padded_rows(c), c.H, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
     const int n_gu = c.act == MOE_ACT_RELU2 ? c.I : 2 * c.I;   // rows of the packed gate/up weights
-    // CTA pairs: each CTA loads half of a B tile's 256 rows
-    // CTA pairs always (2), never (0), or picked on the device (1, the default)
-    const bool pair_kernel = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU && h->gemm_pairs == 2;
-    const bool poly = c.fmt == MOE_FMT_FP8_ROW && c.act == MOE_ACT_SWIGLU && h->gemm_pairs == 1;
-    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, pair_kernel ? 128 : 256);
+    r = make_tmap(&tb, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, 256);
     if (r != MOE_OK) return r;
     GemmParams p;
     memset(&p, 0, sizeof(p));
@@ -836,42 +845,44 @@ static moe_status gate_up_impl(const moe_handle* h, const void* packed, int T, v
     p.spin_limit = h->spin_limit;
     const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (pair_kernel) {
-        const int pairs = std::max(1, std::min(h->num_sms / 2, (max_m_tiles(c, T) + 1) / 2 * p.n_blocks));
-        return launch_gemm_pairs<MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, 2 * pairs, st);
-    }
-    if (poly) {
-        // 2-CTA clusters; the dispatch's pick says whether they run as pairs or
-        // as single CTAs (an even grid large enough for either)
-        CUtensorMap tb128;
+    if (c.fmt == MOE_FMT_FP8_ROW && c.act != MOE_ACT_RELU2) {
+        // 2-CTA clusters that run the mode the dispatch picked (pick[2]): single
+        // CTAs on 256- or 128-wide tiles, or CTA pairs; weight maps with boxes of
+        // 256 rows (wide), 128 (half of a pair's tile) and 64 (narrow: 64 gate
+        // rows, then the 64 matching up rows); an even grid that covers the
+        // largest unit count of the three
+        CUtensorMap tb128, tb64;
         r = make_tmap(&tb128, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, 128);
         if (r != MOE_OK) return r;
-        const int g2 = std::max(2, (std::min(h->num_sms, max_m_tiles(c, T) * p.n_blocks) + 1) / 2 * 2);
-        auto kern = grouped_gemm_gu_poly_kernel<MOE_ACT_SWIGLU>;
+        r = make_tmap(&tb64, pw + h->wl.gu_q, c.H, static_cast<uint64_t>(c.E) * n_gu, c.H, GEMM_BK, 64);
+        if (r != MOE_OK) return r;
+        const int g2 = std::max(2, (std::min(h->num_sms, max_m_tiles(c, T) * 2 * p.n_blocks) + 1) / 2 * 2);
         static_assert(GU_POLY_SMEM <= 232448, "shared memory of the GEMM exceeds 227 KB");
-        CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GU_POLY_SMEM));
-        const cudaError_t err = launch_k_pairs(h->pdl, kern, dim3(g2), dim3(gemm_threads<16>()), GU_POLY_SMEM, st, ta,
-                                               tb, tb128, p, static_cast<const int32_t*>(v.pick + 2));
+        const int32_t* mode = static_cast<const int32_t*>(v.pick + 2);
+        cudaError_t err;
+        switch (c.act) {
+        case MOE_ACT_SWIGLU_BOUNDED:
+            err = launch_gu_poly<MOE_ACT_SWIGLU_BOUNDED>(h->pdl, g2, st, ta, tb, tb128, tb64, p, mode);
+            break;
+        case MOE_ACT_SWIGLU_OAI:
+            err = launch_gu_poly<MOE_ACT_SWIGLU_OAI>(h->pdl, g2, st, ta, tb, tb128, tb64, p, mode);
+            break;
+        case MOE_ACT_GEGLU:
+            err = launch_gu_poly<MOE_ACT_GEGLU>(h->pdl, g2, st, ta, tb, tb128, tb64, p, mode);
+            break;
+        case MOE_ACT_REGLU:
+            err = launch_gu_poly<MOE_ACT_REGLU>(h->pdl, g2, st, ta, tb, tb128, tb64, p, mode);
+            break;
+        default:
+            err = launch_gu_poly<MOE_ACT_SWIGLU>(h->pdl, g2, st, ta, tb, tb128, tb64, p, mode);
+            break;
+        }
         if (err != cudaSuccess)
             return fail(MOE_ERR_CUDA, "launch of grouped_gemm_gu_poly_kernel failed: %s", cudaGetErrorString(err));
         return MOE_OK;
     }
-    if (c.fmt == MOE_FMT_FP8_ROW) {
-        switch (c.act) {
-        case MOE_ACT_SWIGLU_BOUNDED:
-            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_SWIGLU_BOUNDED>(h->pdl, ta, tb, p, grid, st);
-        case MOE_ACT_SWIGLU_OAI:
-            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_SWIGLU_OAI>(h->pdl, ta, tb, p, grid, st);
-        case MOE_ACT_GEGLU:
-            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_GEGLU>(h->pdl, ta, tb, p, grid, st);
-        case MOE_ACT_REGLU:
-            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_REGLU>(h->pdl, ta, tb, p, grid, st);
-        case MOE_ACT_RELU2:
-            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_RELU2>(h->pdl, ta, tb, p, grid, st);
-        default:
-            return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_SWIGLU>(h->pdl, ta, tb, p, grid, st);
-        }
-    }
+    if (c.fmt == MOE_FMT_FP8_ROW)   // ReLU^2: the up projection alone, 256 rows per tile
+        return launch_gemm<KIND_GATE_UP, BSCALE_ROW, false, 256, 4, 16, MOE_ACT_RELU2>(h->pdl, ta, tb, p, grid, st);
     switch (c.act) {
     case MOE_ACT_SWIGLU_BOUNDED:
         return launch_gemm<KIND_GATE_UP, BSCALE_BLOCK128, true, 256, 4, 8, MOE_ACT_SWIGLU_BOUNDED>(h->pdl, ta, tb, p, grid, st);
@@ -1050,20 +1061,21 @@ extern "C" moe_status moe_get_picker_params(const moe_handle* h, long long* para
     return MOE_OK;
 }
 
-extern "C" moe_status moe_set_pair_params(moe_handle* h, const long long* params) {
-    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_set_pair_params: null argument");
-    for (int i = 0; i < 4; i++)
-        if (params[i] < 0) return fail(MOE_ERR_INVALID_ARG, "moe_set_pair_params: costs must be >= 0");
-    for (int i = 0; i < 4; i++) h->picker.gu_ps[i] = params[i];
+extern "C" moe_status moe_set_gate_up_model(moe_handle* h, const long long* params) {
+    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_set_gate_up_model: null argument");
+    for (int i = 0; i < 6; i++)
+        if (params[i] < 0) return fail(MOE_ERR_INVALID_ARG, "moe_set_gate_up_model: costs must be >= 0");
+    for (int i = 0; i < 6; i++) h->picker.gu_ps[i] = params[i];
     return MOE_OK;
 }
 
-extern "C" moe_status moe_get_pair_params(const moe_handle* h, long long* params) {
-    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_get_pair_params: null argument");
-    for (int i = 0; i < 4; i++) params[i] = h->picker.gu_ps[i];
-    params[4] = h->picker.gu_nb;
-    params[5] = h->picker.gu_kb;
-    params[6] = h->picker.num_sms;
+extern "C" moe_status moe_get_gate_up_model(const moe_handle* h, long long* params) {
+    if (!h || !params) return fail(MOE_ERR_INVALID_ARG, "moe_get_gate_up_model: null argument");
+    for (int i = 0; i < 6; i++) params[i] = h->picker.gu_ps[i];
+    params[6] = h->picker.gu_nb;
+    params[7] = h->picker.gu_kb;
+    params[8] = h->picker.num_sms;
+    params[9] = h->picker.gu_allow;
     return MOE_OK;
 }
 
@@ -1089,11 +1101,29 @@ extern "C" moe_status moe_set_launch_options(moe_handle* h, int pdl) {
     return MOE_OK;
 }
 
+extern "C" moe_status moe_set_gate_up_tile(moe_handle* h, int bn) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_gate_up_tile: null handle");
+    if (bn != 0 && bn != 128 && bn != 256)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_gate_up_tile: bn must be 0, 128 or 256 (got %d)", bn);
+    if (bn == 128 && (h->cfg.fmt != MOE_FMT_FP8_ROW || h->cfg.act == MOE_ACT_RELU2))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_set_gate_up_tile: 128-wide tiles need a gated FP8_ROW layer");
+    const int allow = gu_allow_of(h->gemm_pairs, bn);
+    if (allow == 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_gate_up_tile: 128-wide tiles contradict CTA pairs forced on");
+    h->gu_bn = bn;
+    h->picker.gu_allow = allow;
+    return MOE_OK;
+}
+
 extern "C" moe_status moe_set_gemm_options(moe_handle* h, int cta_pairs) {
     if (!h) return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: null handle");
     if (cta_pairs < 0 || cta_pairs > 2)
         return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: cta_pairs must be 0, 1 or 2 (got %d)", cta_pairs);
+    const int allow = gu_allow_of(cta_pairs, h->gu_bn);
+    if (allow == 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_options: CTA pairs contradict 128-wide gate/up tiles forced on");
     h->gemm_pairs = cta_pairs;
+    h->picker.gu_allow = allow;
     return MOE_OK;
 }
 

@@ -23,7 +23,7 @@ EXPORTED = (
     "moe_workspace_view_get", "moe_pack_weights", "moe_route", "moe_dispatch", "moe_gate_up",
     "moe_down", "moe_combine", "moe_forward", "moe_forward_routed", "moe_workspace_init",
     "moe_get_status", "moe_dispatch_noalloc", "moe_set_tile_config", "moe_set_launch_options", "moe_set_gemm_options", "moe_set_wait_limit", "moe_set_picker_params",
-    "moe_get_picker_params", "moe_set_pair_params", "moe_get_pair_params",
+    "moe_get_picker_params", "moe_set_gate_up_model", "moe_get_gate_up_model", "moe_set_gate_up_tile",
 )
 
 
@@ -89,8 +89,9 @@ def load(path=LIB_PATH):
             "moe_set_wait_limit": (I, [P, ctypes.c_longlong]),
             "moe_set_picker_params": (I, [P, P]),
             "moe_get_picker_params": (I, [P, P]),
-            "moe_set_pair_params": (I, [P, P]),
-            "moe_get_pair_params": (I, [P, P]),
+            "moe_set_gate_up_model": (I, [P, P]),
+            "moe_set_gate_up_tile": (I, [P, I]),
+            "moe_get_gate_up_model": (I, [P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -220,15 +221,20 @@ def moe_get_picker_params(h):
     return tuple(arr)
 
 
-def moe_set_pair_params(h, a_s, b_s, a_p, b_p):
-    arr = (ctypes.c_longlong * 4)(a_s, b_s, a_p, b_p)
-    _check(load().moe_set_pair_params(h, arr))
+def moe_set_gate_up_tile(h, bn):
+    _check(load().moe_set_gate_up_tile(h, bn))
 
 
-def moe_get_pair_params(h):
-    """(a_s, b_s, a_p, b_p, nb, kb, num_sms)"""
-    arr = (ctypes.c_longlong * 7)()
-    _check(load().moe_get_pair_params(h, arr))
+def moe_set_gate_up_model(h, *params):
+    """params: a_0, b_0, a_1, b_1, a_2, b_2 (ps per unit: kb a + b of each mode)"""
+    arr = (ctypes.c_longlong * 6)(*params)
+    _check(load().moe_set_gate_up_model(h, arr))
+
+
+def moe_get_gate_up_model(h):
+    """(a_0, b_0, a_1, b_1, a_2, b_2, nb, kb, num_sms, allowed-mode mask)"""
+    arr = (ctypes.c_longlong * 10)()
+    _check(load().moe_get_gate_up_model(h, arr))
     return tuple(arr)
 
 

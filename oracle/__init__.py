@@ -76,7 +76,7 @@ def lib():
             "orc_num_threads": (I, []),
             "orc_pick_down_tile": (I, [P, I, I, I, I, I64, I64, I64, I64, P]),
             "orc_pick_split": (I, [P, I, I, I, I64, I]),
-            "orc_pick_gu_pairs": (I, [P, I, I, I, I, P]),
+            "orc_pick_gu_mode": (I, [P, I, I, I, I, I, P]),
             "orc_glu": (ctypes.c_double, [I, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double]),
         }
         for name, (res, args) in sig.items():
@@ -202,11 +202,13 @@ def pick_split(counts, split_nb, split_kb, o_rows, num_sms):
 
 
 # ---------------------------------------------------------------- quantisers
-def pick_gu_pairs(counts, nb, kb, num_sms, ps):
-    """1: the FP8_ROW gate/up GEMM on CTA pairs, 0: single CTAs (moe_oracle.h)."""
+def pick_gu_mode(counts, nb, kb, num_sms, ps, allow=7):
+    """Gated FP8_ROW gate/up mode: 0 single CTAs on 256-wide tiles, 1 CTA
+    pairs, 2 single CTAs on 128-wide tiles (moe_oracle.h)."""
     c = _c(counts, np.int32)
     p = _c(ps, np.int64)
-    return int(lib().orc_pick_gu_pairs(_p(c), c.size, nb, kb, num_sms, _p(p)))
+    assert p.size == 6
+    return int(lib().orc_pick_gu_mode(_p(c), c.size, nb, kb, num_sms, allow, _p(p)))
 
 
 def code_bytes(fmt, K):

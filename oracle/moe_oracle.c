@@ -270,7 +270,7 @@ int orc_pick_split(const int32_t* counts, int E, int split_nb, int split_kb, int
     return best;
 }
 
-int orc_pick_gu_pairs(const int32_t* counts, int E, int nb, int kb, int num_sms, const int64_t* ps)
+int orc_pick_gu_mode(const int32_t* counts, int E, int nb, int kb, int num_sms, int allow, const int64_t* ps)
 {
     int64_t m_tiles = 0, n_odd = 0;
     for (int e = 0; e < E; e++) {
@@ -279,12 +279,26 @@ int orc_pick_gu_pairs(const int32_t* counts, int E, int nb, int kb, int num_sms,
         n_odd += mt & 1;
     }
     if (nb <= 0 || m_tiles == 0) return 0;
-    int64_t single_units = m_tiles * nb;
-    int64_t pair_units = (m_tiles + n_odd) / 2 * nb;
-    int64_t clusters = num_sms / 2;
-    int64_t single_cost = (single_units + num_sms - 1) / num_sms * (kb * ps[0] + ps[1]);
-    int64_t pair_cost = (pair_units + clusters - 1) / clusters * (kb * ps[2] + ps[3]);
-    return pair_cost < single_cost ? 1 : 0;
+    /* units and the CTAs (or pairs) that run at once, per mode */
+    int64_t units[3], slots[3];
+    units[0] = m_tiles * nb;                  /* 256-wide tiles on single CTAs */
+    slots[0] = num_sms;
+    units[1] = (m_tiles + n_odd) / 2 * nb;    /* pairs of an expert's m-tiles */
+    slots[1] = num_sms / 2;
+    units[2] = m_tiles * 2 * nb;              /* 128-wide tiles on single CTAs */
+    slots[2] = num_sms;
+    int best = -1;
+    int64_t best_cost = 0;
+    for (int m = 0; m < 3; m++) {
+        if (!((allow >> m) & 1)) continue;
+        int64_t waves = (units[m] + slots[m] - 1) / slots[m];
+        int64_t cost = waves * (kb * ps[2 * m] + ps[2 * m + 1]);
+        if (best < 0 || cost < best_cost) {
+            best = m;
+            best_cost = cost;
+        }
+    }
+    return best < 0 ? 0 : best;
 }
 
 /* ------------------------------------------------ activation quantisation */

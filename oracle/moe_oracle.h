@@ -85,16 +85,18 @@ int orc_pick_down_tile(const int32_t* counts, int E, int H, int I, int num_sms,
                        int64_t alpha, int64_t beta, int64_t bw, int64_t gamma, int64_t* costs);
 /* K split of the FP8_ROW down GEMM (1 = none) from the expert histogram. */
 int orc_pick_split(const int32_t* counts, int E, int split_nb, int split_kb, int64_t o_rows, int num_sms);
-/* FP8_ROW gate/up GEMM on CTA pairs (1) or single CTAs (0), from the expert
- * histogram.  mt_e = ceil(counts[e] / 128) m-tiles per expert, m_tiles their
- * sum, n_odd the number of experts with an odd mt_e.  A single unit is an
- * (m-tile, n-block), num_sms run at once; a pair unit an (m-tile pair,
- * n-block), num_sms / 2 run at once:
- *   single = ceil(m_tiles nb / num_sms) (kb ps[0] + ps[1])
- *   pair   = ceil((m_tiles + n_odd) / 2 nb / (num_sms / 2)) (kb ps[2] + ps[3])
- * (integers; / truncates).  1 when pair < single, else 0; 0 when nb <= 0 or
- * the histogram is empty. */
-int orc_pick_gu_pairs(const int32_t* counts, int E, int nb, int kb, int num_sms, const int64_t* ps);
+/* Mode of the gated FP8_ROW gate/up GEMM from the expert histogram (RaMP
+ * abstract: the configuration comes from the runtime histogram through a
+ * cost model of CTA waves): 0 single CTAs on 256-wide tiles, 1 CTA pairs, 2
+ * single CTAs on 128-wide tiles.  mt_e = ceil(counts[e] / 128) m-tiles per
+ * expert, m_tiles their sum, n_odd the number of experts with an odd mt_e.
+ * Mode 0 has m_tiles nb units, num_sms at once; mode 1 (m_tiles + n_odd) / 2 nb
+ * units (pairs of an expert's m-tiles), num_sms / 2 at once; mode 2
+ * 2 m_tiles nb units, num_sms at once.  cost_m = ceil(units_m / at_once_m)
+ * (kb ps[2m] + ps[2m+1]) in integers.  The cheapest mode whose bit is set in
+ * allow wins, ties to the lower mode; 0 when nb <= 0, the histogram is empty
+ * or no mode is allowed. */
+int orc_pick_gu_mode(const int32_t* counts, int E, int nb, int kb, int num_sms, int allow, const int64_t* ps);
 
 /* ---- activation quantisation of token rows (X or the hidden) ----
  * FP8_ROW:      one fp32 scale per row: s = fp32(amax/448), q = e4m3(fp32(x/s)),

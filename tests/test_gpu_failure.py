@@ -24,6 +24,8 @@ CASES = {
     "fp8-row-deep-k-pairs": W.custom(H=512, I=2304, E=8, k=2),
     # the gate/up GEMM on CTA pairs (waits on the other CTA's copies)
     "fp8-row-pairs": W.custom(H=512, I=256, E=8, k=2),
+    # the gate/up GEMM on 128-wide tiles (8 of 16 epilogue warps working)
+    "fp8-row-narrow": W.custom(H=512, I=256, E=8, k=2),
     "fp8-block128": W.custom(H=512, I=256, E=8, k=2, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128),
     "nvfp4": W.custom(H=512, I=256, E=8, k=2, fmt=W.FMT_NVFP4),
 }
@@ -44,11 +46,15 @@ def test_wait_timeout_is_reported_and_the_context_stays_usable(name):
     layer = native.Layer(wl, d, max_T=T)
     if name.endswith("pairs"):
         # the cost model's parameters chosen so that the gate/up kernel runs as pairs
-        native.moe_set_pair_params(layer.h, 10 ** 12, 10 ** 12, 0, 0)
+        native.moe_set_gate_up_model(layer.h, 10 ** 12, 10 ** 12, 0, 0, 10 ** 12, 10 ** 12)
+    if name.endswith("narrow"):
+        native.moe_set_gate_up_tile(layer.h, 128)
     x, wr = synth.tokens(wl, T, seed=5).cuda(), d["wr"].cuda()
     y_ref = layer.forward(x, wr, None).clone()
     if name.endswith("pairs"):
         assert int(layer.region("pick", torch.int32, 3)[2]) == 1
+    if name.endswith("narrow"):
+        assert int(layer.region("pick", torch.int32, 3)[2]) == 2
     torch.cuda.synchronize()
     assert layer.status()[0] == 0
 

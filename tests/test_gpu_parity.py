@@ -306,10 +306,11 @@ def test_dispatch_bit_exact(name):
     pick = layer.region("pick", torch.int32, 3).cpu().numpy()
     assert int(pick[0]) == want
     assert int(pick[1]) == expected_split(wl, T, counts, sms)
-    a_s, b_s, a_p, b_p, nb, kb, sms = native.moe_get_pair_params(layer.h)
-    if wl.fmt == W.FMT_FP8_ROW and wl.act == W.ACT_SWIGLU:
-        assert (nb, kb) == (2 * wl.I // 256, wl.H // 128)
-        assert int(pick[2]) == oracle.pick_gu_pairs(counts, nb, kb, sms, [a_s, b_s, a_p, b_p])
+    model = native.moe_get_gate_up_model(layer.h)
+    nb, kb, sms, allow = model[6:]
+    if wl.fmt == W.FMT_FP8_ROW and wl.act != W.ACT_RELU2:
+        assert (nb, kb, allow) == (2 * wl.I // 256, wl.H // 128, 7)
+        assert int(pick[2]) == oracle.pick_gu_mode(counts, nb, kb, sms, list(model[:6]), allow)
     else:
         assert nb == 0 and int(pick[2]) == 0
     rows = gpu_slot_rows(layer, wl, ids, T)
@@ -561,39 +562,86 @@ def test_cta_pairs_match_single_ctas(name):
     """The GEMMs on CTA pairs (M = 256 MMAs over two row tiles; the gate/up GEMM,
     and with K > 2048 the down GEMM too) give the hidden codes and the layer
     output of the single-CTA kernels, up to the fp32 summation order inside
-    the tensor core."""
+    the tensor core.  The gate/up modes are forced both through the options
+    and through the cost model's parameters; either way the dispatch writes
+    the mode the kernel then runs."""
     wl, T, d, x = build_case(name)
     layer = native.Layer(wl, d, max_T=T)
     xc, wr = x.cuda(), d["wr"].cuda()
     n_hq = (T * wl.k + 128 * wl.E) * wl.I
 
-    def run(mode, params=None):
-        native.moe_set_gemm_options(layer.h, mode)
+    def run(mode=None, params=None):
+        if mode is not None:
+            native.moe_set_gemm_options(layer.h, mode)
         if params is not None:
-            native.moe_set_pair_params(layer.h, *params)
+            native.moe_set_gate_up_model(layer.h, *params)
         y = layer.forward(xc, wr, None).clone()
         torch.cuda.synchronize()
         assert layer.status()[0] == 0
         return y, layer.region("hq", torch.uint8, n_hq).clone(), int(layer.region("pick", torch.int32, 3)[2])
 
     big = 10 ** 12
-    default = native.moe_get_pair_params(layer.h)[:4]
-    y_pair, hq_pair, _ = run(2)
-    y_single, hq_single, _ = run(0)
-    # the kernel that picks its mode on the device, forced each way by the cost
-    # parameters: the same results as the dedicated kernel of that mode
-    y_p1, hq_p1, pk1 = run(1, (big, big, 0, 0))
-    y_p0, hq_p0, pk0 = run(1, (0, 0, big, big))
+    default = native.moe_get_gate_up_model(layer.h)[:6]
+    y_pair, hq_pair, pk_pair = run(2)
+    y_single, hq_single, pk_single = run(0, (0, 0, big, big, big, big))
+    assert (pk_pair, pk_single) == (1, 0)
+    # the options back to the default; the model's parameters force each mode
+    y_p1, hq_p1, pk1 = run(1, (big, big, 0, 0, big, big))
+    y_p0, hq_p0, pk0 = run(None, (0, 0, big, big, big, big))
     assert (pk1, pk0) == (1, 0)
     assert torch.equal(hq_p1, hq_pair) and torch.equal(y_p1, y_pair)
     assert torch.equal(hq_p0, hq_single) and torch.equal(y_p0, y_single)
-    native.moe_set_pair_params(layer.h, *default)
+    native.moe_set_gate_up_model(layer.h, *default)
     assert (hq_pair != hq_single).float().mean().item() <= 1e-3
     assert tolerance_violations(y_pair.float().cpu().numpy(), y_single.float().cpu().numpy()) == 0
     with pytest.raises(native.MoeError):
         native.moe_set_gemm_options(layer.h, 3)
     with pytest.raises(native.MoeError):
-        native.moe_set_pair_params(layer.h, -1, 0, 0, 0)
+        native.moe_set_gate_up_model(layer.h, -1, 0, 0, 0, 0, 0)
+    # pairs forced on and 128-wide tiles forced on contradict each other
+    native.moe_set_gemm_options(layer.h, 2)
+    with pytest.raises(native.MoeError):
+        native.moe_set_gate_up_tile(layer.h, 128)
+    native.moe_set_gemm_options(layer.h, 1)
+
+
+@pytest.mark.parametrize("name", ["row-ragged", "row-t700", "row-split-boxes-t96", "row-skew-e64"])
+def test_gate_up_tile_widths_agree(name):
+    """The gated FP8_ROW gate/up GEMM on 128-wide tiles (64 gate + 64 up
+    columns) and on 256-wide tiles: the same hidden codes and scales up to the
+    fp32 summation order inside the tensor core, and outputs within the
+    tolerance of each other.  The oracle parity tests run whichever width the
+    dispatch picks."""
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    xc, wr = x.cuda(), d["wr"].cuda()
+    bias = None if d["bias"] is None else d["bias"].cuda()
+    n_hq = (T * wl.k + 128 * wl.E) * wl.I
+    n_hs = (T * wl.k + 128 * wl.E) * wl.I // 32
+    out = {}
+    for bn, mode in ((128, 2), (256, 0)):
+        native.moe_set_gemm_options(layer.h, 0)
+        native.moe_set_gate_up_tile(layer.h, bn)
+        y = layer.forward(xc, wr, bias).clone()
+        torch.cuda.synchronize()
+        assert layer.status()[0] == 0
+        assert int(layer.region("pick", torch.int32, 3)[2]) == mode
+        out[bn] = (y, layer.region("hq", torch.uint8, n_hq).clone(), layer.region("hs", torch.uint8, n_hs).clone())
+    (y1, hq1, hs1), (y2, hq2, hs2) = out[128], out[256]
+    assert (hq1 != hq2).float().mean().item() <= 1e-3
+    assert (hs1 != hs2).float().mean().item() <= 1e-3
+    assert tolerance_violations(y1.float().cpu().numpy(), y2.float().cpu().numpy()) == 0
+    native.moe_set_gate_up_tile(layer.h, 0)
+    with pytest.raises(native.MoeError):
+        native.moe_set_gate_up_tile(layer.h, 64)
+
+
+def test_gate_up_tile_width_needs_a_gated_fp8_row_layer():
+    wl, T, d, x = build_case("block128-ragged")
+    layer = native.Layer(wl, d, max_T=T)
+    with pytest.raises(native.MoeError):
+        native.moe_set_gate_up_tile(layer.h, 128)
+    native.moe_set_gate_up_tile(layer.h, 256)
 
 
 def test_empty_batch():

@@ -362,24 +362,43 @@ def test_mx32_exponent_is_the_smallest_that_fits():
     assert (np.abs(deq - x) <= bound).all()
 
 
-def test_gate_up_pair_rule_hand_cases():
-    """The gate/up CTA-mode rule on histograms worked out by hand (148 SMs,
-    nb n-blocks, kb K-blocks, per-unit costs kb a + b)."""
-    ps = [1000, 0, 1000, 0]             # equal per-unit cost: only the wave counts decide
+def test_gate_up_mode_rule_hand_cases():
+    """The gate/up mode rule on histograms worked out by hand (148 SMs, nb
+    256-wide n-blocks, kb K-blocks, per-unit costs kb a + b per mode)."""
+    P = 3   # narrow tiles not allowed: single CTAs or pairs
+    ps = [1000, 0, 1000, 0, 0, 0]      # equal per-unit cost: only the wave counts decide
     # 8 experts x 8 m-tiles (1024 rows each), nb = 112: single 64 x 112 = 7168
     # units -> 49 waves; pairs 32 x 112 = 3584 units -> ceil(3584 / 74) = 49 waves
-    # -> equal cost, single CTAs
-    assert oracle.pick_gu_pairs([1024] * 8, 112, 32, 148, ps) == 0
-    # a pair unit cheaper than a single one (a_p < a_s) breaks the tie for pairs
-    assert oracle.pick_gu_pairs([1024] * 8, 112, 32, 148, [1000, 0, 990, 0]) == 1
+    # -> equal cost, the lower mode (single CTAs)
+    assert oracle.pick_gu_mode([1024] * 8, 112, 32, 148, ps, P) == 0
+    # a pair unit cheaper than a single one (a_1 < a_0) breaks the tie for pairs
+    assert oracle.pick_gu_mode([1024] * 8, 112, 32, 148, [1000, 0, 990, 0, 0, 0], P) == 1
     # one m-tile per expert: pairs are half empty -> as many pair units as single
     # ones on half the slots: 160 experts, nb = 4 -> single ceil(640/148) = 5,
     # pairs ceil(640/74) = 9 waves
-    assert oracle.pick_gu_pairs([100] * 160 + [0] * 96, 4, 16, 148, ps) == 0
+    assert oracle.pick_gu_mode([100] * 160 + [0] * 96, 4, 16, 148, ps, P) == 0
     # odd counts: 3 m-tiles -> pairs (3 + 1) / 2 = 2 units per expert
-    assert oracle.pick_gu_pairs([300] * 50, 8, 16, 148, [10, 0, 6, 0]) == 1   # 150 x 8 = 1200 -> 9 waves x 160 vs
-    #                                                  100 x 8 = 800 -> 11 waves x 96 = 1056 < 1440
-    assert oracle.pick_gu_pairs([300] * 50, 8, 16, 148, [10, 0, 9, 0]) == 0   # 11 x 144 = 1584 > 1440
-    # no n-blocks (not a SwiGLU FP8_ROW layer) or no rows: single CTAs
-    assert oracle.pick_gu_pairs([1024] * 8, 0, 32, 148, [10, 0, 1, 0]) == 0
-    assert oracle.pick_gu_pairs([0] * 8, 112, 32, 148, [10, 0, 1, 0]) == 0
+    # single 150 x 8 = 1200 units -> 9 waves x 160; pairs 100 x 8 = 800 -> 11 waves
+    assert oracle.pick_gu_mode([300] * 50, 8, 16, 148, [10, 0, 6, 0, 0, 0], P) == 1    # 11 x 96 = 1056 < 1440
+    assert oracle.pick_gu_mode([300] * 50, 8, 16, 148, [10, 0, 9, 0, 0, 0], P) == 0    # 11 x 144 = 1584 > 1440
+    # narrow tiles: 47 experts with one m-tile, nb = 4, kb = 16: wide 188 units ->
+    # 2 waves x 16 a_0; narrow 376 units -> 3 waves x 16 a_2; pairs 188 units on
+    # 74 -> 3 waves x 16 a_1
+    q = [1000, 0, 990, 0, 600, 0]
+    h47 = [10] * 47 + [0] * 209
+    assert oracle.pick_gu_mode(h47, 4, 16, 148, q) == 2          # 3 x 9600 < 2 x 16000 < 3 x 15840
+    assert oracle.pick_gu_mode(h47, 4, 16, 148, [1000, 0, 990, 0, 700, 0]) == 0   # 3 x 11200 > 32000
+    # two experts with one m-tile, nb = 112, kb = 32: wide 224 units -> 2 waves,
+    # narrow 448 -> 4 waves (3 x 148 = 444 < 448)
+    assert oracle.pick_gu_mode([1, 1] + [0] * 6, 112, 32, 148, q) == 0   # 4 x 19200 > 2 x 32000
+    # one wave either way (nb = 1, kb = 2): equal per-unit cost ties to wide,
+    # a cheaper narrow unit wins
+    assert oracle.pick_gu_mode([10] * 8, 1, 2, 148, [5, 0, 9, 0, 5, 0]) == 0
+    assert oracle.pick_gu_mode([10] * 8, 1, 2, 148, [5, 0, 9, 0, 4, 0]) == 2
+    # the allowed-mode mask: only one mode allowed -> that mode; none -> 0
+    assert oracle.pick_gu_mode([1024] * 8, 112, 32, 148, q, 4) == 2
+    assert oracle.pick_gu_mode([1, 1] + [0] * 6, 112, 32, 148, q, 2) == 1
+    assert oracle.pick_gu_mode([1024] * 8, 112, 32, 148, q, 0) == 0
+    # no n-blocks (not a gated FP8_ROW layer) or no rows: mode 0
+    assert oracle.pick_gu_mode([1024] * 8, 0, 32, 148, [10, 0, 1, 0, 1, 0]) == 0
+    assert oracle.pick_gu_mode([0] * 8, 112, 32, 148, [10, 0, 1, 0, 1, 0]) == 0

@@ -53,29 +53,32 @@ def test_refit_reproduces_the_installed_parameters(rows):
         assert got == pytest.approx(want, rel=0.02)
 
 
-def test_pair_sweep_rule_is_the_oracle_rule():
-    """The sweep tool's restatement of the gate/up CTA-mode rule (on m-tile
+def test_mode_sweep_rule_is_the_oracle_rule():
+    """The sweep tool's restatement of the gate/up mode rule (on m-tile
     counts) picks what the oracle's rule picks on the histograms themselves."""
-    from mixture_experts_topk_b200 import pair_sweep
+    from mixture_experts_topk_b200 import gate_up_mode_sweep as gs
     rng = np.random.default_rng(3)
-    for trial in range(300):
+    for trial in range(400):
         E = int(rng.choice([8, 32, 64, 256]))
         counts = rng.integers(0, int(rng.choice([3, 200, 1500])), size=E).astype(np.int32)
         nb, kb = int(rng.choice([1, 4, 16, 112])), int(rng.choice([2, 16, 32]))
-        ps = [int(v) for v in rng.integers(1, 10 ** 6, size=4)]
+        ps = [int(v) for v in rng.integers(1, 10 ** 6, size=6)]
+        allow = int(rng.integers(0, 8))
         mt = (counts + 127) // 128
-        want = oracle.pick_gu_pairs(counts, nb, kb, 148, ps)
-        assert pair_sweep.pick(int(mt.sum()), int((mt % 2).sum()), nb, kb, ps) == want, (trial, E, nb, kb, ps)
+        want = oracle.pick_gu_mode(counts, nb, kb, 148, ps, allow)
+        assert gs.pick(int(mt.sum()), int((mt % 2).sum()), nb, kb, ps, allow) == want, (trial, E, nb, kb, ps)
 
 
-def test_pair_sweep_table_reader(tmp_path):
-    from mixture_experts_topk_b200 import pair_sweep
+def test_mode_sweep_table_reader(tmp_path):
+    from mixture_experts_topk_b200 import gate_up_mode_sweep as gs
     f = tmp_path / "t.md"
-    f.write_text(pair_sweep.HEADER + "\n| tiny T=16 | 8 | 8 | 1 | 2 | 0.0086 | 0.0120 |\n"
-                 "| mixtral-8x7b T=4096 | 67 | 3 | 112 | 32 | 0.9292 | 0.9248 |\n")
-    rows = pair_sweep.read_table(str(f))
+    f.write_text(gs.HEADER + "\n| tiny T=16 | 8 | 8 | 1 | 2 | 0.0086 | 0.0120 | 0.0070 |\n"
+                 "| mixtral-8x7b T=4096 | 67 | 3 | 112 | 32 | 0.9292 | 0.9248 | 1.1 |\n")
+    rows = gs.read_table(str(f))
     assert [r["workload"] for r in rows] == ["tiny T=16", "mixtral-8x7b T=4096"]
-    res = pair_sweep.evaluate(rows, (527000, 0, 493000, 200000))
-    # one wave either way: single CTAs; Mixtral-8x7B T = 4096: pairs (53 vs 51 waves)
-    assert [p for _, p, _ in res] == [0, 1]
+    # tiny: one wave in every mode -> the cheapest unit, narrow (2 x 334000);
+    # Mixtral-8x7B T = 4096: pairs (53 waves of 16.0 us against 51 of 16.9 and
+    # 102 of 10.7)
+    res = gs.evaluate(rows, gs.INSTALLED)
+    assert [p for _, p, _ in res] == [2, 1]
     assert all(rg == 0.0 for _, _, rg in res)
