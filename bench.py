@@ -565,7 +565,10 @@ def main():
     ap.add_argument("--workload", default="mixtral-8x7b")
     ap.add_argument("--tokens", type=int, default=4096)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-sample", type=int, default=2)
+    ap.add_argument("--ref-sample", type=int, default=2,
+                    help="tokens per step through the oracle's expert MLP in --impl reference")
+    ap.add_argument("--cpu-sample", type=int, default=40,
+                    help="tokens through the oracle's expert MLP for cpu_baseline (about 10 s of host work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the sweep over every (workload, T) point (done at N = 1 only)")
@@ -600,7 +603,7 @@ def main():
     out = run_ours(args, rank, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline and not args.profile:
-            cb = cpu_baseline(workload_of(args), args.tokens, args.ref_sample)
+            cb = cpu_baseline(workload_of(args), args.tokens, args.cpu_sample)
             cb.pop("seconds")
             out["cpu_baseline"] = cb
         print(json.dumps(out))

@@ -246,7 +246,10 @@ moe_status moe_down(const moe_handle* h, const void* packed, const float* w, int
 /* Explicit tile choice of the down GEMM (LightMoE README, "Grouped GEMM",
  * leaves the tile configuration to the caller, since the best one varies with
  * the matrix sizes and with how the assignments spread over experts).  down_bn: 0 = chosen per call, or 64,
- * 128, 256 output columns per tile.  Host state only. */
+ * 128, 256 output columns per tile.  FP8_BLOCK128 takes all three; FP8_ROW
+ * takes 128 (128-wide tiles with two accumulators in TMEM, so a tile's MMAs
+ * run while the previous tile's epilogue drains; single CTAs) and otherwise
+ * runs 256-wide tiles; NVFP4 ignores it.  Host state only. */
 moe_status moe_set_tile_config(moe_handle* h, int down_bn);
 
 /* Launch option of every kernel the layer calls (no counterpart in the pages:

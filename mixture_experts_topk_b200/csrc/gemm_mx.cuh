@@ -42,23 +42,29 @@ constexpr int MX_BN = 256;
 constexpr int MX_A_BYTES = 128 * 128;
 constexpr int MX_SFA_BYTES = 512;
 constexpr int MX_BOX_BYTES = 32 * 128;                           // 32 rows x 64 fp16
-constexpr int MX_SFA_TMEM = MX_BN;                               // 4 columns per stage
-constexpr int MX_SFB_TMEM = MX_BN + 32;                          // 8 columns (two 128-row chunks)
+// TMEM: the accumulators fill columns [0, 256) (one 256-wide or two 128-wide),
+// then the A-scale ring and the constant B-scale chunks
+constexpr int MX_SFA_TMEM = 256;                                 // 4 columns per stage
+constexpr int MX_SFB_TMEM = 256 + 32;                            // 8 columns (two 128-row chunks)
 // Deep K (many K stages per tile): 4 stages, rows stored from registers.
 // Shallow K, where a tile's stores outlast its MMAs: 3 stages and the box stores.
 constexpr int MX_BOX_MAX_KB = 16;
 // CTA pairs (deep K, large batches): 33 KB stages, 5 deep.
 constexpr int MX_PAIR_STAGES = 5;
+// 128-wide tiles: 33 KB stages, 4 deep beside the box stores, 6 without.
+constexpr int MX_NARROW_BOX_STAGES = 4;
+constexpr int MX_NARROW_STAGES = 6;
 
 // PAIR: a CTA pair (tcgen05 cta_group::2, M = 256) where each CTA loads its 128
 // A rows and 128 of the 256 B rows.
-template <int STAGES, bool BOXES, bool PAIR = false>
+template <int STAGES, bool BOXES, bool PAIR = false, int BN = MX_BN>
 struct MxSmem {
-    static constexpr int B_BYTES = (PAIR ? MX_BN / 2 : MX_BN) * 128;
+    static constexpr int NACC = 256 / BN;                             // accumulators in TMEM
+    static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * 128;
     static constexpr int STAGE_BYTES = MX_A_BYTES + B_BYTES + 1024;   // + 512 B A scales, padded to 1 KB
     static constexpr int SFB_OFF = STAGES * STAGE_BYTES;              // 2 constant chunks (1 KB)
     static constexpr int BAR_OFF = SFB_OFF + 1024;
-    static constexpr int NUM_BARS = 2 * STAGES + 3;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NACC + 1;
     static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int TMAP_OFF = TMEM_SLOT_OFF + 16;
     // per epilogue warp: two swizzled boxes, or the float4 row staging
@@ -133,20 +139,25 @@ struct MxDownParams {
     long long spin_limit;
 };
 
-template <int STAGES, bool BOXES, bool PAIR = false>
+// BN: 256-wide tiles with one accumulator, or 128-wide tiles with two, so that
+// a tile's MMAs run while the epilogue drains the previous tile's accumulator
+template <int STAGES, bool BOXES, bool PAIR = false, int BN = MX_BN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     grouped_gemm_mx_down_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                                 const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmS,
                                 const MxDownParams p) {
-    using L = MxSmem<STAGES, BOXES, PAIR>;
+    static_assert(BN == 256 || (BN == 128 && !PAIR), "128-wide down tiles run on single CTAs");
+    using L = MxSmem<STAGES, BOXES, PAIR, BN>;
+    constexpr int NACC = L::NACC;
+    constexpr int NC = BN / 2;                       // output columns per epilogue thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
-    uint64_t* tfull = bars + 2 * STAGES;
-    uint64_t* tempty = bars + 2 * STAGES + 1;
-    uint64_t* drain = bars + 2 * STAGES + 2;
+    uint64_t* tfull = bars + 2 * STAGES;             // [NACC]
+    uint64_t* tempty = bars + 2 * STAGES + NACC;     // [NACC]
+    uint64_t* drain = bars + 2 * STAGES + 2 * NACC;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // CTA pairs: rank 0 issues the MMAs; its full and tempty barriers take the
@@ -161,8 +172,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_init(&full[s], PAIR ? 2 : 1);   // pairs: one expect_tx arrival per CTA
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tfull, 1);
-        mbar_init(tempty, PAIR ? 16 : 8);       // one arrival per epilogue warp
+        for (int a = 0; a < NACC; a++) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], PAIR ? 16 : 8);   // one arrival per epilogue warp
+        }
         mbar_init(drain, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
@@ -242,7 +255,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 // a pair's rank 1 without an m-tile (odd count) loads rank 0's rows and
                 // scales, so its reads stay inside the buffers; its rows are not stored
                 const int mi_ld = has_rows ? mi : mi - 1;
-                const int brow = e * p.b_rows + nb * MX_BN + (PAIR ? static_cast<int>(rank) * (MX_BN / 2) : 0);
+                const int brow = e * p.b_rows + nb * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
                 const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
                 const uint8_t* sfa = p.sfa + static_cast<size_t>(mi_ld) * p.num_kb * 512;
                 // both CTAs of a pair complete their stage bytes on rank 0's barrier
@@ -347,7 +360,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int t = t_first; t < total && ok; t += t_step) {
                 const int sp = t % S;
                 const int kb0 = sp * p.num_kb / S, kb1 = (sp + 1) * p.num_kb / S;
-                if (!mbar_wait(tempty, (u & 1) ^ 1, limit)) { ok = false; break; }
+                const uint32_t acc = u % NACC;
+                if (!mbar_wait(&tempty[acc], ((u / NACC) & 1) ^ 1, limit)) { ok = false; break; }
                 tc_fence_after();
                 for (int kb = kb0; kb < kb1; kb++, it++) {
                     const int s = it % STAGES;
@@ -361,17 +375,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     for (int j = 0; j < 4; j++) {
                         if constexpr (PAIR)
                             mma_mxf8_pair(tmem_base, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
-                                          idesc_mxf8(256, MX_BN, j), sfa, sfb, (kb > kb0 || j > 0));
+                                          idesc_mxf8(256, BN, j), sfa, sfb, (kb > kb0 || j > 0));
                         else
-                            mma_mxf8(tmem_base, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
-                                     idesc_mxf8(128, MX_BN, j), sfa, sfb, (kb > kb0 || j > 0));
+                            mma_mxf8(tmem_base + acc * BN, sdesc_sw128(a_addr + 32 * j), sdesc_sw128(b_addr + 32 * j),
+                                     idesc_mxf8(128, BN, j), sfa, sfb, (kb > kb0 || j > 0));
                     }
                     if constexpr (PAIR) mma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
                     else mma_commit(&empty[s]);
                 }
                 if (!ok) break;
                 if constexpr (PAIR) mma_commit_pair_both(tfull);   // both CTAs' epilogues
-                else mma_commit(tfull);
+                else mma_commit(&tfull[acc]);
                 u++;
             }
             if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
@@ -382,7 +396,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
-        const int g = (warp - 2) >> 2;             // 128 columns per column group
+        const int g = (warp - 2) >> 2;             // NC columns per column group
         const int r = 32 * q + lane;
         const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
         uint8_t* ostg = smem + L::STG_OFF + (warp - 2) * L::STG_WARP_BYTES;
@@ -390,9 +404,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         bool ok = true;
         // the accumulator is free again: a pair's MMA thread (rank 0) counts both
         // CTAs' epilogue warps
-        auto release_acc = [&]() {
+        auto release_acc = [&](uint32_t acc) {
             if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(tempty, 0));
-            else mbar_arrive(tempty);
+            else mbar_arrive(&tempty[acc]);
         };
         for (int t = t_first; t < total && ok; t += t_step) {
             const int sp = t % S;
@@ -405,34 +419,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             // the row's routing weight is loaded while the tile's MMAs run
             const int slot = s_off[e] + local;
             const float rw = valid ? p.route_w[p.perm[slot]] : 0.0f;
-            const int n0 = nb * MX_BN + 128 * g;
+            const int n0 = nb * BN + NC * g;
             const float* cs = p.w_scale + static_cast<size_t>(e) * p.H + n0;
-            if (!warp_wait(tfull, u & 1, limit)) { ok = false; break; }
+            const uint32_t acc = u % NACC;
+            if (!warp_wait(&tfull[acc], (u / NACC) & 1, limit)) { ok = false; break; }
             tc_fence_after();
             if (!__any_sync(0xffffffffu, valid)) {
                 // none of this warp's rows is stored: release the accumulator only
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) release_acc();
+                if (lane == 0) release_acc(acc);
                 u++;
                 continue;
             }
-            float v[128];
+            float v[NC];
+            const uint32_t col0 = acc * BN + NC * g;
 #pragma unroll
-            for (int ch = 0; ch < 2; ch++)
-                tmem_ld32x2(lane_addr + 128 * g + 64 * ch, lane_addr + 128 * g + 64 * ch + 32, v + 64 * ch,
+            for (int ch = 0; ch < NC / 64; ch++)
+                tmem_ld32x2(lane_addr + col0 + 64 * ch, lane_addr + col0 + 64 * ch + 32, v + 64 * ch,
                             v + 64 * ch + 32);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) release_acc();   // the next tile's MMAs may start
+            if (lane == 0) release_acc(acc);   // the next tile's MMAs may start
             u++;
             const size_t orow = static_cast<size_t>(sp) * p.A + slot;
             if (BOXES && __all_sync(0xffffffffu, valid)) {
-                // rows sp A + slot(lane 0) + lane: two boxes of 64 fp16 columns
+                // rows sp A + slot(lane 0) + lane: NC / 64 boxes of 64 fp16 columns
                 const int y0 = __shfl_sync(0xffffffffu, static_cast<int>(orow), 0);
                 uint32_t ebytes = 0;
 #pragma unroll
-                for (int b = 0; b < 2; b++, nbox++) {
+                for (int b = 0; b < NC / 64; b++, nbox++) {
                     uint8_t* buf = ostg + (nbox & 1) * MX_BOX_BYTES;
                     uint32_t w0[16], w1[16];
                     const int e0 = o16_block<true>(v + 64 * b, cs + 64 * b, rw, w0);
@@ -456,14 +472,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         bulk_commit();
                     }
                 }
-                *reinterpret_cast<uint32_t*>(p.oe + orow * (p.H / 32) + n0 / 32) = ebytes;
+                if constexpr (NC == 128) *reinterpret_cast<uint32_t*>(p.oe + orow * (p.H / 32) + n0 / 32) = ebytes;
+                else *reinterpret_cast<uint16_t*>(p.oe + orow * (p.H / 32) + n0 / 32) = static_cast<uint16_t>(ebytes);
             } else {
                 if constexpr (BOXES) {
                     // the box buffers serve as the row staging once their stores have read them
                     if (lane == 0) bulk_wait_read0();
                     __syncwarp();
                 }
-                store_rows16<128, true>(v, reinterpret_cast<uint32_t*>(ostg), valid ? p.o + orow * p.H + n0 : nullptr,
+                store_rows16<NC, true>(v, reinterpret_cast<uint32_t*>(ostg), valid ? p.o + orow * p.H + n0 : nullptr,
                                         p.oe + orow * (p.H / 32) + n0 / 32, cs, rw, lane);
                 __syncwarp();
             }

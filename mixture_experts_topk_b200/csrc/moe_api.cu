@@ -915,11 +915,15 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     // the gate/up GEMM) and no K split can be chosen; shallow K keeps single
     // CTAs and the box stores.
     const bool pairs = c.I / 128 > MX_BOX_MAX_KB && split_limit(h->picker, T * c.k) == 1 &&
-                       (h->gemm_pairs == 2 || (h->gemm_pairs == 1 && T * c.k >= 4 * TILE_M * c.E));
+                       (h->gemm_pairs == 2 || (h->gemm_pairs == 1 && T * c.k >= 4 * TILE_M * c.E)) &&
+                       h->down_bn != 128;
+    // 128-wide tiles with two accumulators in TMEM (moe_set_tile_config(h, 128))
+    const bool narrow = !pairs && h->down_bn == 128;
+    const int bn = narrow ? 128 : MX_BN;
     CUtensorMap ta, tb, to, ts;
     moe_status r = make_tmap(&ta, v.hq, c.I, hidden_rows(c), c.I, GEMM_BK, GEMM_BM);
     if (r != MOE_OK) return r;
-    r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, pairs ? MX_BN / 2 : MX_BN);
+    r = make_tmap(&tb, pw + h->wl.d_q, c.I, static_cast<uint64_t>(c.E) * c.H, c.I, GEMM_BK, pairs ? MX_BN / 2 : bn);
     if (r != MOE_OK) return r;
     // hidden scales as rows of 256 bytes (a 512-byte chunk per row tile and K
     // stage is two rows), copied as they are: the pairs' scale loads
@@ -936,7 +940,7 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
     p.tile_ptr = v.tile_ptr;
     p.offsets = v.offsets;
     p.E = c.E;
-    p.n_blocks = c.H / MX_BN;
+    p.n_blocks = c.H / bn;
     p.num_kb = c.I / 128;
     p.b_rows = c.H;
     p.sfa = static_cast<const uint8_t*>(v.hs);
@@ -966,7 +970,17 @@ static moe_status mx_down(const moe_handle* h, const void* packed, const float* 
             return fail(MOE_ERR_CUDA, "launch of grouped_gemm_mx_down_kernel (pairs) failed: %s", cudaGetErrorString(err));
         return MOE_OK;
     }
-    if (p.num_kb <= MX_BOX_MAX_KB) {
+    if (narrow && p.num_kb <= MX_BOX_MAX_KB) {
+        using Ln = MxSmem<MX_NARROW_BOX_STAGES, true, false, 128>;
+        auto kern = grouped_gemm_mx_down_kernel<MX_NARROW_BOX_STAGES, true, false, 128>;
+        CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ln::TOTAL));
+        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Ln::TOTAL, st, ta, tb, to, ts, p);
+    } else if (narrow) {
+        using Ln = MxSmem<MX_NARROW_STAGES, false, false, 128>;
+        auto kern = grouped_gemm_mx_down_kernel<MX_NARROW_STAGES, false, false, 128>;
+        CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ln::TOTAL));
+        LAUNCH(h->pdl, "grouped_gemm_mx_down_kernel", kern, grid, GEMM_THREADS, Ln::TOTAL, st, ta, tb, to, ts, p);
+    } else if (p.num_kb <= MX_BOX_MAX_KB) {
         using Lb = MxSmem<3, true>;
         auto kern = grouped_gemm_mx_down_kernel<3, true>;
         CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lb::TOTAL));

@@ -370,8 +370,9 @@ def test_gate_up_hidden_matches_oracle(name):
 
 
 # the FP8_BLOCK128 down GEMM has three tile widths (0 = picked from the
-# histogram); the other formats' down GEMMs have one
-DOWN_CASES = [(n, bn) for n in CASES for bn in ((0, 64, 128, 256) if CASES[n][0].fmt == W.FMT_FP8_BLOCK128 else (0,))]
+# histogram), the FP8_ROW one two (128: two accumulators in TMEM), NVFP4 one
+DOWN_WIDTHS = {W.FMT_FP8_BLOCK128: (0, 64, 128, 256), W.FMT_FP8_ROW: (0, 128), W.FMT_NVFP4: (0,)}
+DOWN_CASES = [(n, bn) for n in CASES for bn in DOWN_WIDTHS[CASES[n][0].fmt]]
 
 
 @pytest.mark.parametrize("name,down_bn", DOWN_CASES, ids=[f"{n}-bn{b}" for n, b in DOWN_CASES])
@@ -634,6 +635,25 @@ def test_gate_up_tile_widths_agree(name):
     native.moe_set_gate_up_tile(layer.h, 0)
     with pytest.raises(native.MoeError):
         native.moe_set_gate_up_tile(layer.h, 64)
+
+
+@pytest.mark.parametrize("name", ["row-ragged", "row-t700", "row-split-boxes-t96", "row-pairs-deepk-t2100"])
+def test_down_tile_widths_agree(name):
+    """The FP8_ROW down GEMM on 128-wide tiles (two accumulators) and on its
+    default tiles, through the whole layer (chained behind the gate/up GEMM
+    for T k <= 4096, with a K split at T = 96, deep K at I = 2304): the same
+    fp16 rows up to the fp32 summation order inside the tensor core."""
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    xc, wr = x.cuda(), d["wr"].cuda()
+    ys = {}
+    for bn in (128, 0):
+        native.moe_set_tile_config(layer.h, bn)
+        ys[bn] = layer.forward(xc, wr, None).clone()
+        torch.cuda.synchronize()
+        assert layer.status()[0] == 0
+    assert tolerance_violations(ys[128].float().cpu().numpy(), ys[0].float().cpu().numpy()) == 0
+    assert (ys[128] != ys[0]).float().mean().item() <= 1e-3
 
 
 def test_gate_up_tile_width_needs_a_gated_fp8_row_layer():
