@@ -1151,6 +1151,7 @@ extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws,
     if (T == 0) return MOE_OK;
     moe_workspace_view v;
     moe_workspace_view_get(h, ws, &v);
+    const int s_max = split_limit(h->picker, T * h->cfg.k);
     // one CTA per (group of 8 / k tokens, 2048-column slice): small batches still spread.
     // Launched without the PDL attribute: launched early, its CTAs would be
     // placed on the few SMs the down GEMM leaves room on and run ~2x slower
@@ -1162,8 +1163,8 @@ extern "C" moe_status moe_combine(const moe_handle* h, int T, void* y, void* ws,
     LAUNCH(false, "combine_kernel", combine_kernel, grid, COMBINE_THREADS, 0, reinterpret_cast<cudaStream_t>(stream),
            static_cast<const uint16_t*>(v.o), static_cast<const int8_t*>(v.o_exp), static_cast<const int32_t*>(v.inv),
            T, h->cfg.H, h->cfg.k,
-           static_cast<const int32_t*>(h->cfg.fmt == MOE_FMT_FP8_ROW ? v.pick + 1 : nullptr),
-           split_limit(h->picker, T * h->cfg.k), static_cast<__nv_bfloat16*>(y));
+           static_cast<const int32_t*>(h->cfg.fmt == MOE_FMT_FP8_ROW ? v.pick + 1 : nullptr), s_max,
+           static_cast<__nv_bfloat16*>(y));
     return MOE_OK;
 }
 

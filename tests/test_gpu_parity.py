@@ -41,6 +41,8 @@ CASES = {
     # above 128 tokens with more than 8 experts the router runs on the tensor cores
     "row-skew-e64-t300": (W.custom(H=512, I=256, E=64, k=8, zipf_s=1.2), 300),
     "block128-e48-t260": (W.custom(H=512, I=256, E=48, k=6, score=W.SCORE_SIGMOID, fmt=W.FMT_FP8_BLOCK128), 260),
+    # H = 1024: two 512-column slices of the combine per token group
+    "row-h1024": (W.custom(H=1024, I=256, E=8, k=2), 300),
 }
 
 
@@ -662,6 +664,38 @@ def test_gate_up_tile_width_needs_a_gated_fp8_row_layer():
     with pytest.raises(native.MoeError):
         native.moe_set_gate_up_tile(layer.h, 128)
     native.moe_set_gate_up_tile(layer.h, 256)
+
+
+def bf16_bits_rne(a):
+    """float32 -> bfloat16 bits, round to nearest even (finite values)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = u + 0x7FFF + ((u >> 16) & 1)
+    return (u >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("name", ["row-h1024", "row-ragged", "row-split-boxes-t96", "block128-ragged", "nvfp4-ragged"])
+def test_combine_adds_rows_in_fixed_order(name):
+    """Y is, bit for bit, bf16 of the fp32 sum of each token's k weighted rows
+    (and their K-split copies) in (j, s) order, from the fp16 rows and block
+    exponents the down GEMM wrote."""
+    wl, T, d, x = build_case(name)
+    layer = native.Layer(wl, d, max_T=T)
+    bias = None if d["bias"] is None else d["bias"].cuda()
+    y = layer.forward(x.cuda(), d["wr"].cuda(), bias)
+    torch.cuda.synchronize()
+    assert layer.status()[0] == 0
+    A = T * wl.k
+    S = int(layer.region("pick", torch.int32, 3).cpu().numpy()[1]) if wl.fmt == W.FMT_FP8_ROW else 1
+    rows = decode_o(layer, wl, S, A).astype(np.float32)          # exact: fp16 x a power of two
+    inv = layer.region("inv", torch.int32, A).cpu().numpy().reshape(T, wl.k)
+    acc = np.zeros((T, wl.H), np.float32)
+    for j in range(wl.k):
+        for sp in range(S):
+            ok = inv[:, j] >= 0
+            acc[ok] = acc[ok] + rows[sp, inv[ok, j]]
+    want = bf16_bits_rne(acc).reshape(T, wl.H)
+    got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert (got == want).all(), f"{(got != want).sum()} of {got.size} differ"
 
 
 def test_empty_batch():
