@@ -150,21 +150,70 @@ __global__ void __launch_bounds__(DISPATCH_CHUNK)
 // chunk counts), the row-tile table (expert, first row) in expert order, and
 // tile_ptr[e] = index of expert e's first row tile (may be null), and the down
 // GEMM's tile choice and K split from the histogram (pick_out[0], pick_out[1];
+// Copy n 4-byte words with the whole CTA: 16-byte accesses when both ends and
+// n allow them, each thread's 8 loads issued before any of its stores, so a
+// chain of single-word round trips never forms.
+__device__ __forceinline__ void stage_words(int32_t* dst, const int32_t* src, int n) {
+    const bool vec = (n % 4 == 0) && ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) % 16 == 0);
+    if (vec) {
+        const int n4 = n / 4;
+        const int4* s4 = reinterpret_cast<const int4*>(src);
+        int4* d4 = reinterpret_cast<int4*>(dst);
+        for (int b = threadIdx.x; b < n4; b += 8 * blockDim.x) {
+            int4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int i = b + j * blockDim.x;
+                if (i < n4) v[j] = s4[i];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int i = b + j * blockDim.x;
+                if (i < n4) d4[i] = v[j];
+            }
+        }
+    } else {
+        for (int b = threadIdx.x; b < n; b += 8 * blockDim.x) {
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int i = b + j * blockDim.x;
+                if (i < n) v[j] = src[i];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int i = b + j * blockDim.x;
+                if (i < n) dst[i] = v[j];
+            }
+        }
+    }
+}
+
+// shared memory of scan_kernel: the chunk counts of the largest batch
+// (131072 assignments = 128 chunks of 1024, at most 256 experts)
+constexpr int SCAN_SMEM_MAX = 128 * 256 * 4;
+
 // may be null).  One exclusive block scan over experts of the packed pair
 // (count, row tiles): count < 2^20, so count + (tiles << 20) cannot carry.
+// The chunk counts ([nchunks][E], at most 128 KB) are staged in shared memory
+// with coalesced loads, summed and scanned there, and written back as bases,
+// so no thread walks a chain of dependent global loads.
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nchunks, int E, int32_t* counts,
                                                    int32_t* offsets, int32_t* tiles, int32_t* num_tiles,
                                                    int32_t* tile_ptr, int32_t* pick_out, PickerParams pq,
                                                    int32_t* gu_done) {
+    extern __shared__ int s_cc[];   // [nchunks][E]
     pdl_wait();
     pdl_trigger();
     KTRACE(TR_SCAN);
     __shared__ int warp_tot[8];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    const int ncc = nchunks * E;
+    stage_words(s_cc, chunk_counts, ncc);
+    __syncthreads();
     int c = 0;
     if (e < E) {
-#pragma unroll 8
-        for (int ch = 0; ch < nchunks; ch++) c += chunk_counts[ch * E + e];
+        for (int ch = 0; ch < nchunks; ch++) c += s_cc[ch * E + e];
     }
     const int nt_e = (c + TILE_M - 1) / TILE_M;
     const int packed = c + (nt_e << 20);
@@ -208,8 +257,8 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
         if (tile_ptr) tile_ptr[e] = tptr_e;
         int run = off_e;
         for (int ch = 0; ch < nchunks; ch++) {
-            const int v = chunk_counts[ch * E + e];
-            chunk_counts[ch * E + e] = run;
+            const int v = s_cc[ch * E + e];
+            s_cc[ch * E + e] = run;
             run += v;
         }
         for (int i = 0; i < nt_e; i++) {
@@ -217,6 +266,8 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* chunk_counts, int nc
             tiles[2 * (tptr_e + i) + 1] = off_e + TILE_M * i;
         }
     }
+    __syncthreads();
+    stage_words(chunk_counts, s_cc, ncc);
 }
 
 __global__ void __launch_bounds__(DISPATCH_CHUNK)

@@ -622,7 +622,9 @@ extern "C" moe_status moe_dispatch(const moe_handle* h, const void* x, const int
         if (A > 0) {
             LAUNCH(h->pdl, "hist_kernel", hist_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.status);
         }
-        LAUNCH(h->pdl, "scan_kernel", scan_kernel, 1, 256, 0, st, chunk, nchunks, c.E, v.counts, v.offsets, v.tiles,
+        const int scan_smem = nchunks * c.E * 4;   // at most 128 chunks x 256 experts
+        CUDA_TRY(cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM_MAX));
+        LAUNCH(h->pdl, "scan_kernel", scan_kernel, 1, 256, scan_smem, st, chunk, nchunks, c.E, v.counts, v.offsets, v.tiles,
                v.num_tiles, v.tile_ptr, v.pick, h->picker, gu_done_of(h, ws));
         if (A == 0) return MOE_OK;
         LAUNCH(h->pdl, "rank_kernel", rank_kernel, nchunks, DISPATCH_CHUNK, 0, st, ids, A, c.E, chunk, v.perm, v.inv);
@@ -1312,7 +1314,8 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_handle* h, const void* x, c
         hist_kernel<<<n, DISPATCH_CHUNK, 0, st>>>(ids, a, c.E, chunk, status);
         LAUNCH_CHECK("hist_kernel");
     }
-    scan_kernel<<<1, 256, 0, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles, nullptr, nullptr, h->picker,
+    CUDA_TRY(cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM_MAX));
+    scan_kernel<<<1, 256, n * c.E * 4, st>>>(chunk, n, c.E, counts, offsets, tiles, num_tiles, nullptr, nullptr, h->picker,
                                    nullptr);
     LAUNCH_CHECK("scan_kernel");
     if (a == 0) return MOE_OK;
