@@ -170,6 +170,8 @@ def job_throughput(tokens_per_rank, steps, world, ms_max):
 # setting the LightMoE README gives, alpha 1.702 / limit 7 the common SwiGLU-OAI one
 ACTS = {"swiglu": (0, 0.0, 0.0), "bounded": (1, 0.0, 10.0), "oai": (2, 1.702, 7.0), "geglu": (3, 0.0, 0.0),
         "reglu": (4, 0.0, 0.0), "relu2": (5, 0.0, 0.0)}
+ACT_LABEL = {"swiglu": "SwiGLU", "bounded": "bounded SwiGLU", "oai": "SwiGLU-OAI", "geglu": "GeGLU",
+             "reglu": "ReGLU", "relu2": "ReLU2, up only"}
 
 
 def workload_of(args):
@@ -491,7 +493,7 @@ def run_ours(args, rank, world, local_rank):
                            "model": "max(tensor FLOPs / P_tensor + router FLOPs / P_fp32, algorithmic bytes / HBM)",
                            "peaks": f"{pk_kind}: P_tensor = (2 fp8 | 4 fp4) x bf16_tflops (burst; frac_sustained: "
                                     "x bf16_tflops_sustained), hbm_gbs; P_fp32 = 148 SMs x 128 lanes x 2 x sm_max_mhz"},
-        "roofline": {"kernel": "grouped_gemm gate/up (SwiGLU + requant epilogue)", "bound": "tensor",
+        "roofline": {"kernel": f"grouped_gemm gate/up ({ACT_LABEL[args.act]} + requant epilogue)", "bound": "tensor",
                      "achieved": rf["gu_achieved"], "peak": rf["burst"], "unit": "TFLOP/s",
                      "frac": rf["gu_frac"], "frac_sustained": rf["gu_frac_sustained"],
                      "traffic": gemm_traffic(args.workload, T),
