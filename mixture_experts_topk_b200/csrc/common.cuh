@@ -189,6 +189,18 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
 }
 
 // ------------------------------------------------------------------ tcgen05
+// Per-warpgroup register limits (all four warps of a warpgroup execute the
+// same one); an increase waits until the block has that many registers free.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    static_assert(N >= 24 && N <= 256 && N % 8 == 0, "setmaxnreg count");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                  "r"(ncols)

@@ -250,8 +250,29 @@ __device__ __forceinline__ void store_rows16(const float (&v)[NC], uint32_t* stg
 constexpr int EPI_WARP_FLOATS = SPARSE_WARP_FLOATS > STG_WARP_FLOATS ? SPARSE_WARP_FLOATS : STG_WARP_FLOATS;
 
 // EPI epilogue warps (8 or 16): 4 TMEM lane quadrants x EPI/4 column groups.
-template <int EPI>
-__host__ __device__ constexpr int gemm_threads() { return 64 + 32 * EPI; }
+// The promoted (FP8_BLOCK128) GEMMs hold 128 fp32 partial sums per epilogue
+// thread across the K loop; they launch a whole warpgroup 0 (producer, MMA
+// issuer, two idle warps) so that registers can move from it to the epilogue
+// warpgroups (setmaxnreg), and their epilogue warps start at warp 4.
+template <int EPI, bool PROMOTE = false>
+__host__ __device__ constexpr int gemm_threads() { return (PROMOTE ? 128 : 64) + 32 * EPI; }
+template <bool PROMOTE>
+__host__ __device__ constexpr int first_epi_warp() { return PROMOTE ? 4 : 2; }
+// Register split of the promoted GEMMs: 384 threads launch with 168 registers
+// each (65536 / 384, rounded down to the allocation step of 8); warpgroup 0
+// drops to 40 and the two epilogue warpgroups rise to 232, which uses exactly
+// the launch's 64512 (128 x 40 + 256 x 232), and each sub-partition holds one
+// warp of each warpgroup: 32 x (40 + 2 x 232) = 16128 of its 16384.  At 232
+// the 128 partial sums, a 64-column TMEM load and the loop state fit without
+// spills (at 168 the K loop spilled to local memory, whose traffic competes
+// with the MMAs' shared-memory operand reads).
+constexpr int PROMOTE_LAUNCH_REGS = 168;
+constexpr int PROMOTE_CTRL_REGS = 40;
+constexpr int PROMOTE_EPI_REGS = 232;
+static_assert(gemm_threads<8, true>() * PROMOTE_LAUNCH_REGS >= 128 * PROMOTE_CTRL_REGS + 256 * PROMOTE_EPI_REGS,
+              "the promoted GEMM's register split exceeds its launch allocation");
+static_assert(32 * (PROMOTE_CTRL_REGS + 2 * PROMOTE_EPI_REGS) <= 16384,
+              "the promoted GEMM's register split exceeds a sub-partition's register file");
 // sparse gate/up staging rows per round: 8 with 8 epilogue warps, 4 with 16
 template <int EPI>
 __host__ __device__ constexpr int sparse_round() { return EPI == 8 ? 8 : 4; }
@@ -357,6 +378,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
     // of 128 gate + 128 up rows; a 128-wide tile takes 64 of each, at 64 (nb & 1)
     auto gu_row0 = [&](int nb) { return BN == 256 ? nb * 256 : 256 * (nb >> 1) + 64 * (nb & 1); };
     constexpr int NH = GC / 32;          // 32-column blocks per thread
+    constexpr int EPI0 = first_epi_warp<PROMOTE>();
     constexpr int SR = sparse_round<EPI>();
     constexpr int EWF = epi_warp_floats<EPI>();
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -442,121 +464,129 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
         }
     };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            for (int t = t_first; t < total && ok; t += t_step) {
-                int e, mi, nb;
-                bool has_rows;
-                unit_tile(t, e, mi, nb, has_rows);
-                // a pair's rank 1 without an m-tile (odd count) loads rank 0's rows,
-                // so its A stays inside the tensor; its accumulator rows are not stored
-                const int row0 = s_off[e] + GEMM_BM * (mi - (has_rows ? 0 : 1) - s_tptr[e]);
-                const int brow = e * p.b_rows + (KIND == KIND_GATE_UP ? gu_row0(nb) : nb * BN) +
-                                 (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
-                const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
-                for (int kb = 0; kb < p.num_kb; kb++, it++) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, limit)) {
-                        report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* sa = smem + s * S::STAGE_BYTES;
-                    if constexpr (PAIR) {
-                        // both CTAs' halves complete on rank 0's barrier
-                        const uint32_t fb = cluster_addr(&full[s], 0);
-                        mbar_arrive_expect_tx_cluster(fb, S::STAGE_BYTES);
-                        tma_load_2d_pair(sa, &tmA, fb, kb * GEMM_BK, row0, l2_policy(false));
-                        tma_load_2d_pair(sa + GEMM_A_BYTES, &tmB, fb, kb * GEMM_BK, brow, pol);
-                    } else {
-                        mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-                        tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
-                        if (KIND == KIND_GATE_UP && BN == 128) {
-                            // 64 gate rows, then the 64 matching up rows 128 further
-                            // (the tensor map's box is 64 rows)
-                            tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
-                            tma_load_2d_hint(sa + GEMM_A_BYTES + 64 * GEMM_BK, &tmB, &full[s], kb * GEMM_BK,
-                                             brow + 128, pol);
-                        } else {
-                            tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+    if (warp < EPI0) {
+        // control warps: the producer (warp 0), the MMA issuer (warp 1) and, in
+        // the promoted GEMMs, two idle warps that complete warpgroup 0, which
+        // needs few registers
+        if constexpr (PROMOTE) setmaxnreg_dec<PROMOTE_CTRL_REGS>();
+        if (warp == 0) {
+            // -------------------------------------------------------- producer
+            if (lane == 0) {
+                uint32_t it = 0;
+                bool ok = true;
+                for (int t = t_first; t < total && ok; t += t_step) {
+                    int e, mi, nb;
+                    bool has_rows;
+                    unit_tile(t, e, mi, nb, has_rows);
+                    // a pair's rank 1 without an m-tile (odd count) loads rank 0's rows,
+                    // so its A stays inside the tensor; its accumulator rows are not stored
+                    const int row0 = s_off[e] + GEMM_BM * (mi - (has_rows ? 0 : 1) - s_tptr[e]);
+                    const int brow = e * p.b_rows + (KIND == KIND_GATE_UP ? gu_row0(nb) : nb * BN) +
+                                     (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
+                    const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
+                    for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                        const int s = it % STAGES;
+                        if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, limit)) {
+                            report(p.status, ST_TIMEOUT, WHERE_GEMM_PRODUCER);
+                            ok = false;
+                            break;
                         }
+                        uint8_t* sa = smem + s * S::STAGE_BYTES;
+                        if constexpr (PAIR) {
+                            // both CTAs' halves complete on rank 0's barrier
+                            const uint32_t fb = cluster_addr(&full[s], 0);
+                            mbar_arrive_expect_tx_cluster(fb, S::STAGE_BYTES);
+                            tma_load_2d_pair(sa, &tmA, fb, kb * GEMM_BK, row0, l2_policy(false));
+                            tma_load_2d_pair(sa + GEMM_A_BYTES, &tmB, fb, kb * GEMM_BK, brow, pol);
+                        } else {
+                            mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+                            tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
+                            if (KIND == KIND_GATE_UP && BN == 128) {
+                                // 64 gate rows, then the 64 matching up rows 128 further
+                                // (the tensor map's box is 64 rows)
+                                tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                                tma_load_2d_hint(sa + GEMM_A_BYTES + 64 * GEMM_BK, &tmB, &full[s], kb * GEMM_BK,
+                                                 brow + 128, pol);
+                            } else {
+                                tma_load_2d_hint(sa + GEMM_A_BYTES, &tmB, &full[s], kb * GEMM_BK, brow, pol);
+                            }
+                        }
+                        if (PROMOTE) KTRACE_BLK(it, 7);
                     }
-                    if (PROMOTE) KTRACE_BLK(it, 7);
+                }
+                // loads still in flight land before the CTA may exit (for a pair, rank
+                // 0's barriers count both CTAs' loads, and the closing cluster barrier
+                // keeps rank 1 until rank 0 is past this)
+                if (!PAIR || rank == 0) {
+                    const uint32_t first = it > STAGES ? it - STAGES : 0;
+                    for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, DRAIN_LIMIT);
                 }
             }
-            // loads still in flight land before the CTA may exit (for a pair, rank
-            // 0's barriers count both CTAs' loads, and the closing cluster barrier
-            // keeps rank 1 until rank 0 is past this)
-            if (!PAIR || rank == 0) {
-                const uint32_t first = it > STAGES ? it - STAGES : 0;
-                for (uint32_t j = first; j < it; j++) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, DRAIN_LIMIT);
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && (!PAIR || rank == 0)) {
-            // a pair's MMA covers both CTAs' 128 rows (M = 256)
-            constexpr uint32_t idesc = idesc_e4m3(PAIR ? 2 * GEMM_BM : GEMM_BM, BN);
-            uint32_t it = 0, u = 0;
-            bool ok = true;
-            for (int t = t_first; t < total && ok; t += t_step) {
-                uint32_t acc = 0;
-                if (!PROMOTE) {
-                    acc = u % NBUF;
-                    if (!mbar_wait(&tempty[acc], ((u / NBUF) & 1) ^ 1, limit)) { ok = false; break; }
-                    tc_fence_after();
-                }
-                for (int kb = 0; kb < p.num_kb; kb++, it++) {
-                    if (PROMOTE) {
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0 && (!PAIR || rank == 0)) {
+                // a pair's MMA covers both CTAs' 128 rows (M = 256)
+                constexpr uint32_t idesc = idesc_e4m3(PAIR ? 2 * GEMM_BM : GEMM_BM, BN);
+                uint32_t it = 0, u = 0;
+                bool ok = true;
+                for (int t = t_first; t < total && ok; t += t_step) {
+                    uint32_t acc = 0;
+                    if (!PROMOTE) {
                         acc = u % NBUF;
                         if (!mbar_wait(&tempty[acc], ((u / NBUF) & 1) ^ 1, limit)) { ok = false; break; }
                         tc_fence_after();
-                        KTRACE_BLK(u, 0);
                     }
-                    const int s = it % STAGES;
-                    if (!mbar_wait(&full[s], (it / STAGES) & 1, limit)) { ok = false; break; }
-                    tc_fence_after();
-                    if (PROMOTE) KTRACE_BLK(u, 1);
-                    const uint32_t a_addr = smem_u32(smem + s * S::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + GEMM_A_BYTES;
-                    const uint32_t d = tmem_base + acc * BN;
-                    if constexpr (PAIR) {
-#pragma unroll
-                        for (int kk = 0; kk < GEMM_BK / 32; kk++)
-                            mma_f8_pair(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
-                                        kb > 0 || kk > 0);
-                        mma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
-                    } else {
-#pragma unroll
-                        for (int kk = 0; kk < GEMM_BK / 32; kk++)
-                            mma_f8(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
-                                   PROMOTE ? (kk > 0) : (kb > 0 || kk > 0));
-                        mma_commit(&empty[s]);
+                    for (int kb = 0; kb < p.num_kb; kb++, it++) {
+                        if (PROMOTE) {
+                            acc = u % NBUF;
+                            if (!mbar_wait(&tempty[acc], ((u / NBUF) & 1) ^ 1, limit)) { ok = false; break; }
+                            tc_fence_after();
+                            KTRACE_BLK(u, 0);
+                        }
+                        const int s = it % STAGES;
+                        if (!mbar_wait(&full[s], (it / STAGES) & 1, limit)) { ok = false; break; }
+                        tc_fence_after();
+                        if (PROMOTE) KTRACE_BLK(u, 1);
+                        const uint32_t a_addr = smem_u32(smem + s * S::STAGE_BYTES);
+                        const uint32_t b_addr = a_addr + GEMM_A_BYTES;
+                        const uint32_t d = tmem_base + acc * BN;
+                        if constexpr (PAIR) {
+    #pragma unroll
+                            for (int kk = 0; kk < GEMM_BK / 32; kk++)
+                                mma_f8_pair(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
+                                            kb > 0 || kk > 0);
+                            mma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
+                        } else {
+    #pragma unroll
+                            for (int kk = 0; kk < GEMM_BK / 32; kk++)
+                                mma_f8(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
+                                       PROMOTE ? (kk > 0) : (kb > 0 || kk > 0));
+                            mma_commit(&empty[s]);
+                        }
+                        if (PROMOTE) {
+                            mma_commit(&tfull[acc]);
+                            KTRACE_BLK(u, 2);
+                            u++;
+                        }
                     }
-                    if (PROMOTE) {
-                        mma_commit(&tfull[acc]);
-                        KTRACE_BLK(u, 2);
+                    if (!ok) break;
+                    if (!PROMOTE) {
+                        if constexpr (PAIR) mma_commit_pair_both(&tfull[acc]);   // both CTAs' epilogues
+                        else mma_commit(&tfull[acc]);
                         u++;
                     }
                 }
-                if (!ok) break;
-                if (!PROMOTE) {
-                    if constexpr (PAIR) mma_commit_pair_both(&tfull[acc]);   // both CTAs' epilogues
-                    else mma_commit(&tfull[acc]);
-                    u++;
-                }
+                if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
+                if constexpr (PAIR) mma_commit_pair(drain);   // every issued MMA has completed ...
+                else mma_commit(drain);
+                mbar_wait(drain, 0, DRAIN_LIMIT);        // ... before TMEM can be released
             }
-            if (!ok) report(p.status, ST_TIMEOUT, WHERE_GEMM_MMA);
-            if constexpr (PAIR) mma_commit_pair(drain);   // every issued MMA has completed ...
-            else mma_commit(drain);
-            mbar_wait(drain, 0, DRAIN_LIMIT);        // ... before TMEM can be released
         }
-    } else if (warp - 2 < EPA) {
+    } else if (warp - EPI0 < EPA) {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;
+        // (the promoted GEMMs' partial sums take the registers warpgroup 0 gave up)
+        if constexpr (PROMOTE) setmaxnreg_inc<PROMOTE_EPI_REGS>();
+        const int ew = warp - EPI0;
         const int q = warp & 3;               // TMEM lane quadrant this warp may access
         const int g = ew >> 2;                // column group
         const int r = 32 * q + lane;          // row within the tile
@@ -905,7 +935,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
 }
 
 template <int KIND, int BSCALE, bool PROMOTE, int BN, int STAGES, int EPI, int ACT>
-__global__ void __launch_bounds__(gemm_threads<EPI>(), 1)
+__global__ void __launch_bounds__(gemm_threads<EPI, PROMOTE>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -961,7 +991,7 @@ constexpr int POLY_SMEM = GemmSmem<256, 4>::TOTAL > GemmSmem<128, 6>::TOTAL
                                                                                  : GemmSmem<64, 8>::TOTAL);
 
 template <int BSCALE>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(gemm_threads<8, true>(), 1)
     down_gemm_poly_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB256,
                           const __grid_constant__ CUtensorMap tmB128, const __grid_constant__ CUtensorMap tmB64,
                           const GemmParams p, const int32_t* cfg) {

@@ -770,7 +770,7 @@ static moe_status launch_gemm(bool pdl, const CUtensorMap& ta, const CUtensorMap
     static_assert(S::TOTAL <= 232448, "shared memory of the GEMM exceeds 227 KB");
     auto kern = grouped_gemm_kernel<KIND, BSCALE, PROMOTE, BN, STAGES, EPI, ACT>;
     CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL));
-    LAUNCH(pdl, "grouped_gemm_kernel", kern, grid, gemm_threads<EPI>(), S::TOTAL, st, ta, tb, p);
+    LAUNCH(pdl, "grouped_gemm_kernel", kern, grid, (gemm_threads<EPI, PROMOTE>()), S::TOTAL, st, ta, tb, p);
     return MOE_OK;
 }
 
@@ -1046,7 +1046,7 @@ extern "C" moe_status moe_down(const moe_handle* h, const void* packed, const fl
         const int grid = std::max(1, std::min(h->num_sms, max_m_tiles(c, T) * (c.H / 64)));
         CUDA_TRY(cudaFuncSetAttribute(down_gemm_poly_kernel<BSCALE_BLOCK128>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, POLY_SMEM));
-        LAUNCH(h->pdl, "down_gemm_poly_kernel", down_gemm_poly_kernel<BSCALE_BLOCK128>, grid, GEMM_THREADS,
+        LAUNCH(h->pdl, "down_gemm_poly_kernel", down_gemm_poly_kernel<BSCALE_BLOCK128>, grid, (gemm_threads<8, true>()),
                POLY_SMEM, st, ta, tb, tb128, tb64, p, static_cast<const int32_t*>(v.pick));
         return MOE_OK;
     }
