@@ -483,7 +483,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                     const int row0 = s_off[e] + GEMM_BM * (mi - (has_rows ? 0 : 1) - s_tptr[e]);
                     const int brow = e * p.b_rows + (KIND == KIND_GATE_UP ? gu_row0(nb) : nb * BN) +
                                      (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
-                    const uint64_t pol = l2_policy(s_tptr[e + 1] - s_tptr[e] == 1);   // weight tile read once?
+                    // L2 policies: a weight tile read once goes first; in the promoted
+                    // GEMMs (slower per K block, so the CTAs sharing a tile drift further
+                    // apart) every weight tile goes first and the A tile, which all the
+                    // n-blocks of its m-tile read, is kept
+                    const uint64_t pol = l2_policy(PROMOTE || s_tptr[e + 1] - s_tptr[e] == 1);
                     for (int kb = 0; kb < p.num_kb; kb++, it++) {
                         const int s = it % STAGES;
                         if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, limit)) {
@@ -500,7 +504,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                             tma_load_2d_pair(sa + GEMM_A_BYTES, &tmB, fb, kb * GEMM_BK, brow, pol);
                         } else {
                             mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-                            tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
+                            if constexpr (PROMOTE)
+                                tma_load_2d_hint(sa, &tmA, &full[s], kb * GEMM_BK, row0, l2_policy_keep());
+                            else
+                                tma_load_2d(sa, &tmA, &full[s], kb * GEMM_BK, row0);
                             if (KIND == KIND_GATE_UP && BN == 128) {
                                 // 64 gate rows, then the 64 matching up rows 128 further
                                 // (the tensor map's box is 64 rows)
