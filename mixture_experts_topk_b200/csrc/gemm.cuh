@@ -8,14 +8,18 @@
 // activation, requantisation of the hidden, down projection and the routing
 // weight are part of the one layer call.
 //
-// Roles (320 threads, one CTA per SM, persistent over tiles):
+// Roles (one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: A tile [128 rows x 128 K] + B tile [BN rows x 128 K]
 //               per stage into a STAGES-deep shared-memory ring (128-byte swizzle)
 //   warp 1      allocates TMEM, one thread issues tcgen05.mma (M=128, N=BN, K=32)
 //               into a ring of NBUF fp32 accumulators in TMEM (2 for BN=256,
 //               4 for narrower tiles)
-//   warps 2..9  epilogue: tcgen05.ld of the accumulator, scales, SwiGLU and
-//               requantisation (gate/up) or routing weight + fp32 store (down)
+//   epilogue    warps 2..9 (320 threads), 2..17 (576 threads, the FP8_ROW gate/up
+//               GEMM) or 4..11 (384 threads, the promoted GEMMs, whose warps 2
+//               and 3 idle so that warpgroup 0 can hand registers to the two
+//               epilogue warpgroups): tcgen05.ld of the accumulator, scales,
+//               SwiGLU and requantisation (gate/up) or routing weight and the
+//               fp16 row store (down)
 // Tiles are visited expert by expert; inside an expert, n-block-major with the
 // expert's m-tiles fastest, so all readers of one weight tile run at the same
 // time and an expert's rows stay in L2 while its n-blocks go by.
