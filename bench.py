@@ -152,6 +152,15 @@ def algorithmic_work(wl, T, counts):
     return flops_tensor, flops_router, byts, touched
 
 
+def workload_config(wl, act, T, world, counts):
+    """The workload a bench line measures; both arms print the same dict (the
+    expert histogram is the routing's, identical on both arms)."""
+    byts = algorithmic_work(wl, T, counts)[2]
+    return {"workload": f"{wl.name} T={T}", "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "activation": act,
+            "T_per_gpu": T, "parallelism": f"replicas x{world} (token batches)",
+            "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (byts / 1e9)}
+
+
 def max_over_ranks(ms, world, device):
     """The largest of the ranks' times (every rank calls it, in the same order)."""
     if world == 1:
@@ -478,15 +487,13 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8-e4m3 (fp32 accumulate)" if wl.fmt != FMT_NVFP4 else "nvfp4-e2m1 (fp32 accumulate)",
         "data": "synthetic (seeded; X ~ N(0,1) bf16, weights ~ N(0,1/fan_in) quantised offline)",
-        "config": {"workload": f"{wl.name} T={T}", "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "activation": args.act,
-                   "T_per_gpu": T, "parallelism": f"replicas x{world} (token batches)",
-                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (rf["bytes"] / 1e9),
-                   "touched_experts": rf["touched"], "m_tiles": m["m_tiles"],
-                   "launch": "CUDA graph of one moe_forward call, replayed per step" if m["graph"]
-                             else "moe_forward per step",
-                   "down_tile": args.down_bn or {0: 256, 1: 128, 2: 64}[m["pick"][0]],
-                   "down_tile_source": "fixed" if args.down_bn else "picked from the histogram",
-                   "down_k_split": m["pick"][1]},
+        "config": workload_config(wl, args.act, T, world, m["counts"]),
+        "run": {"touched_experts": rf["touched"], "m_tiles": m["m_tiles"],
+                "launch": "CUDA graph of one moe_forward call, replayed per step" if m["graph"]
+                          else "moe_forward per step",
+                "down_tile": args.down_bn or {0: 256, 1: 128, 2: 64}[m["pick"][0]],
+                "down_tile_source": "fixed" if args.down_bn else "picked from the histogram",
+                "down_k_split": m["pick"][1]},
         "tflops": (rf["flops_tensor"] + rf["flops_router"]) * world * args.steps / (ms_max * 1e-3) / 1e12,
         "layer_roofline": {"t_roof_ms": rf["t_roof_ms"], "frac": rf["frac"], "frac_sustained": rf["frac_sustained"],
                            "bound": rf["bound"],
@@ -536,10 +543,10 @@ def cpu_baseline(wl, T, n_sel, seed=0):
     dt = time.perf_counter() - t0
     return {"value": n_sel / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{n_sel} of {T} tokens through the expert MLP and combine; router and top-k over all {T}",
-            "seconds": dt}
+            "seconds": dt, "counts": np.bincount(ids.reshape(-1), minlength=wl.E)}
 
 
-def run_reference(args):
+def run_reference(args, world):
     wl = workload_of(args)
     T = args.tokens
     for _ in range(args.warmup):
@@ -553,7 +560,7 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 router)",
-            "data": "synthetic (seeded)", "config": {"workload": f"{wl.name} T={T}", "T_per_gpu": T},
+            "data": "synthetic (seeded)", "config": workload_config(wl, args.act, T, world, r["counts"]),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
                              "sample": r["sample"]},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -594,7 +601,7 @@ def main():
 
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)))
+            print(json.dumps(run_reference(args, world)))
         return
 
     if world > 1:
@@ -607,6 +614,7 @@ def main():
         if world == 1 and not args.no_cpu_baseline and not args.profile:
             cb = cpu_baseline(workload_of(args), args.tokens, args.cpu_sample)
             cb.pop("seconds")
+            cb.pop("counts")
             out["cpu_baseline"] = cb
         print(json.dumps(out))
     if world > 1:
