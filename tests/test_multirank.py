@@ -68,6 +68,27 @@ def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
                                       "--warmup", "3"])
     called = []
-    monkeypatch.setattr(bench, "run_reference", lambda args: called.append(args) or {})
+    monkeypatch.setattr(bench, "run_reference", lambda args, world: called.append((args, world)) or {})
     bench.main()
     assert called == [] and capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_zero(capsys, monkeypatch):
+    """Rank 0 prints the reference line: the oracle on a token sample, with the
+    workload config the GPU arm prints for the same workload and world size."""
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("LOCAL_RANK", "0")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2", "--workload", "tiny",
+                                      "--tokens", "16", "--steps", "1", "--warmup", "3", "--ref-sample", "2"])
+    bench.main()
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    cfg = line["config"]
+    assert cfg["workload"] == "tiny T=16" and cfg["T_per_gpu"] == 16
+    assert cfg["parallelism"] == "replicas x2 (token batches)"
+    assert set(cfg) == {"workload", "H", "I", "E", "k", "activation", "T_per_gpu", "parallelism", "l2"}
