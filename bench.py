@@ -113,19 +113,30 @@ class Regions:
         return _Span()
 
 
+def kernel_sources_hash():
+    """First 16 hex digits of a sha256 over the GEMM sources with comments and
+    whitespace removed, so that an edit of comments or layout keeps a capture
+    valid and any change of the code itself invalidates it."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in ("gemm.cuh", "gemm_mx.cuh", "common.cuh"):
+        src = open(os.path.join(ROOT, "mixture_experts_topk_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", "", src).encode())
+    return h.hexdigest()[:16]
+
+
 def gemm_traffic(workload, T):
     """DRAM bytes per launch of the gate/up GEMM from the committed ncu capture,
     or None when the capture is of another workload or the kernel sources
     changed since it was taken."""
-    import hashlib
     p = os.path.join(ROOT, "profiles", "grouped_gemm_mixtral8x7b_t4096_traffic.json")
     if workload != "mixtral-8x7b" or T != 4096 or not os.path.exists(p):
         return None
     d = json.load(open(p))
-    h = hashlib.sha256()
-    for f in ("gemm.cuh", "gemm_mx.cuh", "common.cuh"):
-        h.update(open(os.path.join(ROOT, "mixture_experts_topk_b200", "csrc", f), "rb").read())
-    if h.hexdigest()[:16] != d["kernel_sources_sha256_16"]:
+    if kernel_sources_hash() != d["kernel_sources_sha256_16"]:
         return None
     return d["gate_up"]["dram_read_bytes"] + d["gate_up"]["dram_write_bytes"]
 

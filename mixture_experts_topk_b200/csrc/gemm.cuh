@@ -562,13 +562,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tmA, const CUtensor
                         const uint32_t b_addr = a_addr + GEMM_A_BYTES;
                         const uint32_t d = tmem_base + acc * BN;
                         if constexpr (PAIR) {
-    #pragma unroll
+#pragma unroll
                             for (int kk = 0; kk < GEMM_BK / 32; kk++)
                                 mma_f8_pair(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
                                             kb > 0 || kk > 0);
                             mma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
                         } else {
-    #pragma unroll
+#pragma unroll
                             for (int kk = 0; kk < GEMM_BK / 32; kk++)
                                 mma_f8(d, sdesc_sw128(a_addr + 32 * kk), sdesc_sw128(b_addr + 32 * kk), idesc,
                                        PROMOTE ? (kk > 0) : (kb > 0 || kk > 0));
