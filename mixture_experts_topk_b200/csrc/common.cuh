@@ -159,6 +159,8 @@ __device__ __forceinline__ uint64_t l2_policy(bool evict_first) {
         asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
+// evict_last: lines that several CTAs read at different times stay in L2
+// ahead of normal and evict_first lines
 __device__ __forceinline__ uint64_t l2_policy_keep() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
