@@ -58,3 +58,22 @@ def test_relu2_experts_have_two_matrices(bench):
     fl_t, _, byts, _ = bench.algorithmic_work(wl, 2, np.array([1, 1]))
     assert fl_t == 2 * 2 * 2 * 256 * 256
     assert byts == 2 * (2 * 65_536 + 4 * (256 + 256)) + 2 * 256 * 4 + 2 * 2 * 256 * 2
+
+
+def test_traffic_record_hash_ignores_comments_and_layout(bench, tmp_path, monkeypatch):
+    """The committed DRAM counters stay valid across comment or layout edits of
+    the GEMM sources and are dropped when the code itself changes."""
+    import shutil
+    src = os.path.join(bench.ROOT, "mixture_experts_topk_b200", "csrc")
+    root = tmp_path / "repo"
+    (root / "mixture_experts_topk_b200" / "csrc").mkdir(parents=True)
+    for f in ("gemm.cuh", "gemm_mx.cuh", "common.cuh"):
+        shutil.copy(os.path.join(src, f), root / "mixture_experts_topk_b200" / "csrc" / f)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h0 = bench.kernel_sources_hash()
+    g = root / "mixture_experts_topk_b200" / "csrc" / "gemm.cuh"
+    text = g.read_text()
+    g.write_text("// a new comment line\n/* and a block\n   comment */\n" + text.replace("\n", "\n  ", 5))
+    assert bench.kernel_sources_hash() == h0
+    g.write_text(text.replace("GEMM_BK = 128", "GEMM_BK = 64", 1))
+    assert bench.kernel_sources_hash() != h0
